@@ -1,0 +1,383 @@
+"""Throughput of the L³ forward pass (plan + forward per batch) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl l3|reference]
+
+One step = l3_plan + l3_forward over one batch of the workload (the whole
+hot path: sort by token ID, gather-attention, W_up + LayerNorm, W_mix), with
+inputs resident in HBM. Rank 0 prints one JSON line.
+
+Multi-GPU (torchrun): every rank runs its own batch of the workload (tokens
+are independent, so the batch shards with no collective on the data path);
+`value` is all ranks' tokens divided by the slowest rank's time.
+
+--impl reference times the CPU oracle (fp64, all host cores) on bounded
+samples of the same workload, on rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import ctypes
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import static_token_routed_b200 as l3  # noqa: E402
+from static_token_routed_b200 import workloads as wl  # noqa: E402
+
+METRIC = "L3 fwd tokens/sec (bf16, 1 B200) and % of roofline (HBM GB/s or tensor-pipe)"
+EPS = 1e-5
+L2_BYTES = 126 * 2 ** 20
+FP32_ALU_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12  # FFMA lanes x 2 flops x max SM clock
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": p["hbm_gbs"], "bf16_tflops": p["bf16_tflops"],
+                "bf16_tflops_sustained": p.get("bf16_tflops_sustained", p["bf16_tflops"]),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+# ----------------------------------------------------------------------------
+# algorithmic work (bytes that must move, flops that must be done)
+# ----------------------------------------------------------------------------
+
+def algorithmic_work(w: wl.Workload, info) -> dict:
+    el = 2 if w.dtype == "bf16" else 4
+    n = w.n_tokens
+    k_bytes = info.unique_rows_multi * w.d_in * el      # K_t rows read (d_t > 1 groups)
+    v_bytes = info.unique_rows * w.d_emb * el           # V_t rows read
+    x_bytes = n * w.d_in * el
+    y_bytes = n * w.d_out * el
+    w_bytes = (w.d_up * w.d_emb + 2 * w.d_up + w.d_out * (w.d_up + w.d_in)) * el
+    ids_bytes = n * 4
+    total_bytes = k_bytes + v_bytes + x_bytes + y_bytes + w_bytes + ids_bytes
+    return {"bytes": total_bytes, "k_bytes": k_bytes, "v_bytes": v_bytes,
+            "x_bytes": x_bytes, "y_bytes": y_bytes, "w_bytes": w_bytes,
+            "a_bytes": n * w.d_emb * el, "h_bytes": n * w.d_up * el,
+            "up_flops": 2 * n * w.d_emb * w.d_up,
+            "mix_flops": 2 * n * w.d_out * (w.d_up + w.d_in)}
+
+
+def attention_flops(ids: np.ndarray, offsets: np.ndarray, w: wl.Workload) -> int:
+    d = np.diff(offsets.astype(np.int64))[ids]
+    return int(2 * np.sum(d[d > 1]) * (w.d_in + w.d_emb))
+
+
+# per-kernel roofline: what each kernel must move or compute per launch
+def kernel_roofline(name: str, work: dict, attn_flops: int, peaks: dict):
+    if name.startswith("attn"):
+        bytes_ = work["k_bytes"] + work["v_bytes"] + work["x_bytes"] + work["a_bytes"]
+        return "hbm", bytes_, "GB/s", peaks["hbm_gbs"]
+    if name.startswith("up"):
+        f = work["up_flops"]
+    elif name.startswith("mix"):
+        f = work["mix_flops"]
+    else:
+        return None
+    if name.endswith("simt"):
+        return "alu", f, "TFLOP/s", FP32_ALU_PEAK_TFLOPS
+    return "tensor", f, "TFLOP/s", peaks["bf16_tflops_sustained"]
+
+
+# ----------------------------------------------------------------------------
+# clocks during the timed region
+# ----------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device: int):
+        self.proc = None
+        self.device = device
+
+    def __enter__(self):
+        try:
+            props = torch.cuda.get_device_properties(self.device)
+            uuid = str(getattr(props, "uuid", "") or "")
+            sel = ["-i", uuid if uuid.startswith("GPU-") else f"GPU-{uuid}"] if uuid else []
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200", *sel], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                text=True)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+                out = ""
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in getattr(self, "lines", []):
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------
+# CPU oracle timing (baseline / reference arm)
+# ----------------------------------------------------------------------------
+
+def time_oracle(w, tables, batch, n_sample: int, seed: int = 0):
+    import oracle  # test infrastructure: only the CPU-baseline and reference legs use it
+    rng = np.random.default_rng(seed)
+    sel = np.sort(rng.choice(w.n_tokens, size=min(n_sample, w.n_tokens), replace=False))
+    t0 = time.perf_counter()
+    oracle.forward(batch.ids, tables.offsets, batch.x, tables.W_K, tables.W_V, tables.W_up,
+                   tables.ln_gamma, tables.ln_beta, tables.W_mix, EPS, select=sel)
+    dt = time.perf_counter() - t0
+    return len(sel), dt, oracle.threads()
+
+
+def run_reference(args, w, rank):
+    if rank != 0:
+        return
+    tables, batch = wl.make_tables(w), wl.make_batch(w)
+    n_sample = args.ref_sample
+    for _ in range(args.warmup):
+        time_oracle(w, tables, batch, max(1, n_sample // 8), seed=1)
+    total_tok, total_s, cores = 0, 0.0, 1
+    for k in range(args.steps):
+        n, dt, cores = time_oracle(w, tables, batch, n_sample, seed=100 + k)
+        total_tok += n
+        total_s += dt
+    value = total_tok / total_s
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * total_s / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": config_of(w, args),
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                             "sample": f"{n_sample} random tokens of the {w.name} batch per step"},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def config_of(w, args):
+    return {"workload": w.name, "global_batch": w.n_tokens * args.gpus, "tokens_per_gpu": w.n_tokens,
+            "vocab": w.vocab, "v": w.v, "k": w.k, "d_in": w.d_in, "d_emb": w.d_emb,
+            "d_up": w.d_up, "d_out": w.d_out, "alloc": w.alloc, "ids": w.ids,
+            "parallelism": f"dp{args.gpus}",
+            "l2": "no flush: per-step working set (W_K/W_V rows, x, y, weights) >> 126 MB L2"}
+
+
+# ----------------------------------------------------------------------------
+# GPU arm
+# ----------------------------------------------------------------------------
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="paper_shaped", choices=sorted(wl.WORKLOADS))
+    ap.add_argument("--impl", default="l3", choices=["l3", "reference"])
+    ap.add_argument("--ref-sample", type=int, default=48, help="oracle tokens per reference step")
+    ap.add_argument("--cpu-sample", type=int, default=192, help="oracle tokens for cpu_baseline")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    base = wl.WORKLOADS[args.workload]
+
+    if args.impl == "reference":
+        run_reference(args, base, rank)
+        return
+
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    # each rank: same tables, its own batch
+    w = wl.with_tokens(base, base.n_tokens, base.batch_seed + 1000 * rank) if rank else base
+    tables, batch = wl.make_tables(w), wl.make_batch(w)
+    d = {k: getattr(tables, k).to(dev) for k in ("offsets", "W_K", "W_V", "W_up", "ln_gamma",
+                                                 "ln_beta", "W_mix")}
+    ids_d, x_d = batch.ids.to(dev), batch.x.to(dev)
+    y_d = torch.empty(w.n_tokens, w.d_out, dtype=w.torch_dtype, device=dev)
+    dims = l3.make_dims(w.vocab, w.v, w.k, w.d_in, w.d_emb, w.d_up, w.d_out, w.torch_dtype, EPS)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(ids_t, x_t, y_t):
+        plan = l3.l3_plan(ids_t, d["offsets"], dims, stream)
+        l3.l3_forward(x_t, plan, d["W_K"], d["W_V"], d["W_up"], d["ln_gamma"], d["ln_beta"],
+                      d["W_mix"], y_t, stream)
+        return plan
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    for _ in range(max(3, args.warmup)):
+        step(ids_d, x_d, y_d).destroy()
+    plan0 = step(ids_d, x_d, y_d)
+    l3.l3_forward_status(plan0)
+    info = plan0.info()
+    plan0.destroy()
+
+    # ---- timed region: K steps, plan + forward, device-timed ----
+    l3.l3_profile_enable(True)
+    barrier()
+    torch.cuda.synchronize(dev)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clocks:
+        ev0.record(stream)
+        for _ in range(args.steps):
+            step(ids_d, x_d, y_d).destroy()
+        ev1.record(stream)
+        torch.cuda.synchronize(dev)
+    barrier()
+    kernels = l3.l3_profile_read()
+    l3.l3_profile_enable(False)
+    ms = ev0.elapsed_time(ev1) / args.steps
+    ms_t = torch.tensor([ms], device=dev)
+    if dist is not None:
+        dist.all_reduce(ms_t, op=dist.ReduceOp.MAX)
+    ms_max = float(ms_t.item())
+    tokens_all = w.n_tokens * world
+    value = tokens_all / (ms_max * 1e-3)
+
+    # ---- end to end through the public API with host buffers ----
+    e2e = None
+    if not args.no_e2e:
+        ids_h = batch.ids.pin_memory()
+        x_h = batch.x.pin_memory()
+        y_h = torch.empty(w.n_tokens, w.d_out, dtype=w.torch_dtype).pin_memory()
+        ids_s = torch.empty_like(ids_d)
+        x_s = torch.empty_like(x_d)
+        y_s = torch.empty_like(y_d)
+
+        def e2e_step():
+            ids_s.copy_(ids_h, non_blocking=True)
+            x_s.copy_(x_h, non_blocking=True)
+            p = step(ids_s, x_s, y_s)
+            y_h.copy_(y_s, non_blocking=True)
+            return p
+
+        for _ in range(3):
+            e2e_step().destroy()
+        barrier()
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            e2e_step().destroy()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier()
+        ems = torch.tensor([e0.elapsed_time(e1) / args.steps], device=dev)
+        if dist is not None:
+            dist.all_reduce(ems, op=dist.ReduceOp.MAX)
+        e2e = {"value": tokens_all / (float(ems.item()) * 1e-3), "unit": "tokens/s",
+               "h2d_bytes_per_step": int(ids_h.numel() * 4 + x_h.numel() * x_h.element_size()),
+               "d2h_bytes_per_step": int(y_h.numel() * y_h.element_size())}
+
+    if rank != 0:
+        if dist is not None:
+            dist.destroy_process_group()
+        return
+
+    # ---- roofline ----
+    peaks = load_peaks()
+    work = algorithmic_work(w, info)
+    attn_flops = attention_flops(batch.ids.numpy(), tables.offsets.numpy(), w)
+    total_flops = attn_flops + work["up_flops"] + work["mix_flops"]
+    if w.dtype == "bf16":
+        t_flop = total_flops / (peaks["bf16_tflops_sustained"] * 1e12)
+    else:
+        t_flop = total_flops / (FP32_ALU_PEAK_TFLOPS * 1e12)
+    t_mem = work["bytes"] / (peaks["hbm_gbs"] * 1e9)
+    t_roof = max(t_mem, t_flop)
+    step_roof = {"t_mem_us": t_mem * 1e6, "t_flop_us": t_flop * 1e6,
+                 "bound": "hbm" if t_mem > t_flop else ("tensor" if w.dtype == "bf16" else "alu"),
+                 "frac": t_roof / (ms_max * 1e-3), "alg_bytes": work["bytes"],
+                 "alg_flops": total_flops,
+                 "peak_note": f"{peaks['source']}: HBM {peaks['hbm_gbs']} GB/s, bf16 "
+                              f"{peaks['bf16_tflops_sustained']} TFLOP/s sustained"}
+    kern = {k: {"launches": n, "total_ms": t, "per_step_ms": t / args.steps}
+            for k, (n, t) in kernels.items()}
+    top = max(kernels.items(), key=lambda kv: kv[1][1])[0] if kernels else None
+    roof = None
+    if top is not None:
+        kr = kernel_roofline(top, work, attn_flops, peaks)
+        n_launch, tot_ms = kernels[top]
+        if kr is not None:
+            bound, units, unit, peak = kr
+            per_launch_s = tot_ms * 1e-3 / n_launch
+            launches_per_step = n_launch / args.steps
+            per_launch_units = units / launches_per_step
+            achieved = per_launch_units / per_launch_s / (1e9 if unit == "GB/s" else 1e12)
+            roof = {"kernel": top, "bound": bound, "achieved": achieved, "peak": peak,
+                    "unit": unit, "frac": achieved / peak, "traffic": None,
+                    "peak_source": f"{peaks['source']} ({'sustained bf16' if bound == 'tensor' else 'HBM copy' if bound == 'hbm' else 'FFMA lanes x max clock'})"}
+
+    # ---- CPU baseline: the oracle on a bounded sample ----
+    cpu = None
+    if world == 1 and args.cpu_sample > 0:
+        n_s, dt, cores = time_oracle(w, tables, batch, args.cpu_sample)
+        cpu = {"value": n_s / dt, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+               "sample": f"{n_s} random tokens of the {w.name} batch (fp64 oracle, {dt:.1f} s)"}
+
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16" if w.dtype == "bf16" else "fp32", "data": "synthetic",
+            "config": config_of(w, args), "clocks": clocks.summary(), "e2e": e2e,
+            "gpu_launches": int(sum(n for n, _ in kernels.values())),
+            "roofline": roof, "step_roofline": step_roof, "kernels": kern,
+            "cpu_baseline": cpu,
+            "plan": {"groups": info.n_groups, "dense_groups": info.n_dense_groups,
+                     "dense_tiles": info.n_dense_tiles, "tail_items": info.n_tail_items,
+                     "unique_rows": info.unique_rows}}
+    print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,194 @@
+/*
+ * l3.h — C ABI of the B200 (sm_100a) L³ forward-pass library (libl3.so).
+ *
+ * The layer is the Large Lookup Layer of "L³: Large Lookup Layers" (Tseng &
+ * De Sa). For a token with hidden state x [d_in] and token ID t:
+ *
+ *     y = W_mix [ LayerNorm(W_up (V_t^T softmax(K_t x))) ; x ]      (kimjy99
+ *     review, Method, eq. L³; papernotes.org note, 整体框架)
+ *
+ * where K_t = W_K[offsets[t] .. offsets[t+1]-1] and V_t likewise of W_V: the
+ * per-token key/value sets are contiguous row slices of two concatenated
+ * tables (kimjy99 review, §2 Efficient Training and Inference). Routing
+ * depends on t alone (papernotes, 关键设计: static token routing).
+ *
+ * A batch is handled in two calls. l3_plan sorts the batch by token ID so
+ * that tokens sharing an ID form one group, the block-diagonal form of the
+ * sciencestack page's Fig. 3 caption. l3_forward then runs the layer over
+ * those groups and writes y back in the caller's token order (the inverse
+ * sort of the same caption).
+ *
+ * Conventions for every entry point:
+ *   - Tensors are dense, row-major, caller-owned DEVICE pointers on the
+ *     current CUDA device, 16-byte aligned. The library never frees them.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream). All device work is enqueued on it.
+ *   - Errors are returned as l3_status; l3_last_error() gives a message for
+ *     the calling thread. Nothing aborts the process and no exception
+ *     crosses the ABI. Invalid arguments are rejected before any launch.
+ *   - bf16 is IEEE bfloat16 (round to nearest even when the library rounds);
+ *     accumulation is fp32 on the GPU.
+ */
+#ifndef L3_H
+#define L3_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  L3_OK = 0,
+  L3_ERR_INVALID_ARG = 1,  /* null pointer, negative size, misaligned pointer */
+  L3_ERR_TOKEN_RANGE = 2,  /* a token ID outside [0, vocab) */
+  L3_ERR_BAD_OFFSETS = 3,  /* offsets[0] != 0, offsets[vocab] != v, or some d_t outside [1, k] */
+  L3_ERR_UNSUPPORTED = 4,  /* dims this build does not handle (see l3_dims_t) */
+  L3_ERR_CUDA = 5,         /* a CUDA runtime call failed; the message names it */
+  L3_ERR_TIMEOUT = 6,      /* a bounded device-side wait gave up (kernel returned early) */
+  L3_ERR_OOM = 7           /* device allocation failed */
+} l3_status;
+
+typedef enum { L3_BF16 = 0, L3_FP32 = 1 } l3_dtype;
+
+/*
+ * Layer dimensions (kimjy99 review, Method: W_mix in R^{d_out x (d_in+d_up)},
+ * K_t in R^{d_t x d_in}, V_t in R^{d_t x d_emb}; v = sum_t d_t with
+ * 1 <= d_t <= k, papernotes LZW 分配 / kimjy99 Embedding Allocation).
+ * W_up is read as d_up x d_emb: the shape printed on the review cannot map
+ * d_emb to d_up, and this is the only shape that makes the equation typecheck.
+ *
+ * Supported: vocab >= 1, v >= vocab, 1 <= k <= 1024; for L3_BF16 every one
+ * of d_in, d_emb, d_up, d_out a multiple of 16, d_in <= 8192, d_emb <= 512,
+ * d_up <= 4096; for L3_FP32 multiples of 4 with the same bounds.
+ * ln_eps is the LayerNorm epsilon (added to the biased variance).
+ */
+typedef struct {
+  int64_t vocab;   /* |tau|, number of token IDs */
+  int64_t v;       /* rows of W_K and W_V */
+  int64_t k;       /* cap on d_t */
+  int64_t d_in;
+  int64_t d_emb;
+  int64_t d_up;
+  int64_t d_out;
+  int32_t dtype;   /* l3_dtype of x, W_K, W_V, W_up, ln_gamma, ln_beta, W_mix, y */
+  float ln_eps;
+} l3_dims_t;
+
+/* Opaque plan: the sorted batch plus the library-owned device buffers that
+ * l3_forward uses. Owned by the library until l3_plan_destroy. */
+typedef struct l3_plan_s *l3_plan_t;
+
+/* Host-side summary of a plan. */
+typedef struct {
+  int64_t n_tokens;       /* N */
+  int64_t n_groups;       /* G, distinct IDs in the batch */
+  int64_t n_dense_groups; /* groups run on the tensor-core attention path */
+  int64_t n_dense_tiles;  /* 128-token tiles of those groups */
+  int64_t n_tail_items;   /* work items of the CUDA-core attention path */
+  int64_t unique_rows;    /* sum of d_t over the groups: rows of W_K/W_V touched */
+  int64_t unique_rows_multi; /* the same over groups with d_t > 1 (whose K_t is read) */
+} l3_plan_info_t;
+
+/*
+ * l3_plan — sort a batch by token ID and build the group structure
+ * (sciencestack page, Fig. 3 caption: sorting makes the attention mask
+ * block-diagonal; kimjy99 review §2: sort B by T).
+ *
+ *   token_ids  device int32 [n_tokens], each in [0, dims->vocab)
+ *   n_tokens   N >= 0 (N = 0 gives an empty plan; l3_forward then does nothing)
+ *   offsets    device int32 [vocab + 1]: K_t = W_K rows offsets[t] .. offsets[t+1]-1;
+ *              offsets[0] = 0, offsets[vocab] = v, 1 <= d_t <= k
+ *   dims       host pointer, copied
+ *   stream     cudaStream_t
+ *   out        host pointer; receives a new plan on L3_OK, NULL otherwise
+ *
+ * The sort is stable: tokens with equal IDs keep their order, and groups
+ * come in ascending ID order. token_ids and offsets are read during this
+ * call only. The call synchronizes `stream` once, to read the group counts
+ * and the validation flag; it is the only host-device round trip of the
+ * path. Errors: L3_ERR_INVALID_ARG, L3_ERR_UNSUPPORTED, L3_ERR_TOKEN_RANGE,
+ * L3_ERR_BAD_OFFSETS, L3_ERR_OOM, L3_ERR_CUDA.
+ */
+l3_status l3_plan(const int32_t *token_ids, int64_t n_tokens, const int32_t *offsets,
+                  const l3_dims_t *dims, void *stream, l3_plan_t *out);
+
+/* Host summary of a plan (no device work). */
+l3_status l3_plan_info(l3_plan_t plan, l3_plan_info_t *info);
+
+/*
+ * l3_plan_export — copy the plan's sort into caller-owned device buffers
+ * (for tests that compare it bit for bit with a CPU sort). Any pointer may
+ * be NULL to skip that array.
+ *   perm[i]            original index of the token at sorted position i      [N]
+ *   inv_perm[n]        sorted position of original token n                    [N]
+ *   sorted_ids[i]      token ID at sorted position i                          [N]
+ *   group_ids[g]       ID of group g, ascending                               [G]
+ *   group_tok_start[g] first sorted position of group g; [G] = N             [G+1]
+ *   seg_rows[g]        sum of d_t over groups before g; [G] = unique rows     [G+1]
+ *   G_out              host int64, number of groups
+ * Enqueued on `stream`; does not synchronize.
+ */
+l3_status l3_plan_export(l3_plan_t plan, int32_t *perm, int32_t *inv_perm, int32_t *sorted_ids,
+                         int32_t *group_ids, int32_t *group_tok_start, int32_t *seg_rows,
+                         int64_t *G_out, void *stream);
+
+/*
+ * l3_forward — y = L³(x, t) for every token of the plan's batch (kimjy99
+ * review, Method, eq. L³).
+ *
+ *   x         [N x d_in]              hidden states, caller's token order
+ *   W_K       [v x d_in]              concatenated key tables
+ *   W_V       [v x d_emb]             concatenated value tables
+ *   W_up      [d_up x d_emb]          up projection
+ *   ln_gamma  [d_up], ln_beta [d_up]  LayerNorm affine parameters
+ *   W_mix     [d_out x (d_up + d_in)] columns 0..d_up-1 multiply the LayerNorm
+ *                                     output, columns d_up.. multiply x
+ *   y         [N x d_out]             output, caller's token order
+ * All in dims->dtype. Softmax has no 1/sqrt(d) scale (none appears in the
+ * equation). The intermediates a = V_t^T p and h = LayerNorm(W_up a) are
+ * stored once each, as fp16 for a bf16 layer (fp16's 10-bit mantissa keeps
+ * the error that LayerNorm amplifies small) and as fp32 for an fp32 layer;
+ * y is rounded once to dtype. The call only enqueues work on `stream` and never
+ * synchronizes; a device-side wait that gives up is reported by
+ * l3_forward_status. Errors: L3_ERR_INVALID_ARG, L3_ERR_CUDA.
+ */
+l3_status l3_forward(const void *x, l3_plan_t plan, const void *W_K, const void *W_V,
+                     const void *W_up, const void *ln_gamma, const void *ln_beta,
+                     const void *W_mix, void *y, void *stream);
+
+/* Synchronizes the plan's last stream and returns L3_ERR_TIMEOUT if a
+ * bounded wait inside an l3_forward kernel gave up since the plan was made
+ * (the outputs of that call are then incomplete), L3_ERR_CUDA on a CUDA
+ * error, L3_OK otherwise. */
+l3_status l3_forward_status(l3_plan_t plan);
+
+/* Frees the plan's device buffers (stream-ordered on the plan's last
+ * stream). NULL is a no-op. */
+void l3_plan_destroy(l3_plan_t plan);
+
+/* Message for the last error on the calling thread ("" if none). */
+const char *l3_last_error(void);
+
+/*
+ * Per-kernel timing for profiling: while enabled, every kernel the library
+ * launches is bracketed by CUDA events recorded on the stream it is launched
+ * on. l3_profile_read synchronizes those streams and returns, per kernel
+ * name, the number of launches and the summed device time since the last
+ * l3_profile_enable(1). At most `max_entries` entries are written; the
+ * return value is the number of distinct kernels (or -1 on error).
+ */
+typedef struct {
+  char name[48];
+  int64_t launches;
+  double total_ms;
+} l3_kernel_time_t;
+
+void l3_profile_enable(int enable);
+int l3_profile_read(l3_kernel_time_t *out, int max_entries);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* L3_H */

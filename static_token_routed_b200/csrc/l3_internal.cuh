@@ -1,0 +1,114 @@
+// Internal declarations of the L³ library: the plan object, launch helpers
+// and the kernels' host-side entry points.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <string>
+
+#include "../../include/l3.h"
+
+namespace l3 {
+
+// ---------------------------------------------------------------------------
+// error plumbing
+// ---------------------------------------------------------------------------
+void set_error(const std::string &msg);
+l3_status cuda_fail(cudaError_t e, const char *what);
+
+#define L3_CUDA_TRY(expr)                                   \
+  do {                                                      \
+    cudaError_t _e = (expr);                                \
+    if (_e != cudaSuccess) return ::l3::cuda_fail(_e, #expr); \
+  } while (0)
+
+// Device-side error bits, OR-ed into a flag word by kernels.
+enum : int32_t {
+  DEV_ERR_TOKEN_RANGE = 1,
+  DEV_ERR_BAD_OFFSETS = 2,
+  DEV_ERR_TIMEOUT = 4,
+};
+
+// ---------------------------------------------------------------------------
+// profiling: optional CUDA-event bracketing of every launch
+// ---------------------------------------------------------------------------
+struct LaunchTimer {
+  const char *name;
+  cudaStream_t stream;
+  int slot;
+  LaunchTimer(const char *name, cudaStream_t s);
+  ~LaunchTimer();
+};
+
+// ---------------------------------------------------------------------------
+// work items built by the plan
+// ---------------------------------------------------------------------------
+// One 128-token tile of a group on the tensor-core attention path.
+struct DenseTile {
+  int32_t group;
+  int32_t tok0;  // first sorted position of the tile
+};
+// One item of the CUDA-core attention path: up to TAIL_TOKENS tokens of a group.
+struct TailItem {
+  int32_t group;
+  int32_t tok0;
+};
+
+constexpr int TAIL_TOKENS = 8;     // tokens per tail work item
+constexpr int DENSE_TILE_M = 128;  // tokens per dense tile
+
+}  // namespace l3
+
+// The plan object behind the opaque l3_plan_t.
+struct l3_plan_s {
+  int device = 0;
+  cudaStream_t stream = nullptr;  // last stream the plan's buffers were used on
+  l3_dims_t dims{};
+  int64_t n_tokens = 0;
+  int64_t n_groups = 0;
+  int64_t n_dense_groups = 0;
+  int64_t n_dense_tiles = 0;
+  int64_t n_tail_items = 0;
+  int64_t unique_rows = 0;
+  int64_t unique_rows_multi = 0;
+  int64_t max_group_tokens = 0;
+
+  void *block = nullptr;  // the one device allocation backing everything below
+  size_t block_bytes = 0;
+
+  int32_t *perm = nullptr;             // [N] sorted position -> original index
+  int32_t *inv_perm = nullptr;         // [N]
+  int32_t *sorted_ids = nullptr;       // [N]
+  int32_t *group_ids = nullptr;        // [N+1]
+  int32_t *group_tok_start = nullptr;  // [N+1]
+  int32_t *group_row_start = nullptr;  // [N+1] offsets[group_ids[g]]
+  int32_t *group_rows = nullptr;       // [N+1] d_t of group g
+  int32_t *seg_rows = nullptr;         // [N+1]
+  l3::DenseTile *dense_tiles = nullptr;
+  l3::TailItem *tail_items = nullptr;
+  int32_t *dev_flags = nullptr;        // [4]: plan error bits, forward error bits
+  void *a_buf = nullptr;               // [N x d_emb] dtype, original token order
+  void *h_buf = nullptr;               // [N x d_up] dtype
+  float *z_buf = nullptr;              // [N x d_up] fp32 (CUDA-core GEMM path only)
+};
+
+namespace l3 {
+
+// plan kernels (plan.cu)
+l3_status build_plan(l3_plan_s *p, const int32_t *token_ids, const int32_t *offsets,
+                     cudaStream_t s, void *scratch, size_t scratch_bytes);
+size_t plan_scratch_bytes(int64_t n_tokens);
+
+// attention, CUDA-core path (attn_tail.cu)
+l3_status launch_attn_tail(const l3_plan_s *p, const void *x, const void *W_K, const void *W_V,
+                           cudaStream_t s);
+
+// GEMMs + LayerNorm, CUDA-core path (gemm_simt.cu)
+l3_status launch_up_ln_simt(const l3_plan_s *p, const void *W_up, const void *gamma,
+                            const void *beta, cudaStream_t s);
+l3_status launch_mix_simt(const l3_plan_s *p, const void *x, const void *W_mix, void *y,
+                          cudaStream_t s);
+
+}  // namespace l3

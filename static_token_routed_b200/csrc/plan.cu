@@ -1,0 +1,424 @@
+// Batch plan: validate, stable LSD radix sort by token ID, group build and
+// work lists.
+//
+// "L³: Large Lookup Layers" — sciencestack page, Fig. 3 caption: since the
+// layer mixes channels only, sorting the batch by token ID turns its
+// attention mask block-diagonal, and the sort is cheap to invert; kimjy99
+// review §2 states the same (sort B by T). The sort here is stable, so equal
+// IDs keep their original order and the plan is unique.
+//
+// Kernels (all on the caller's stream, no host round trip until the end):
+//   validate offsets -> per pass { digit histogram per tile, one-CTA scan of
+//   the (digit, tile) counts, stable scatter } -> group heads + inverse
+//   permutation -> scan -> group fill -> scan of d_t -> work-item counts ->
+//   scans -> work-item fill.
+#include <algorithm>
+
+#include "l3_internal.cuh"
+
+namespace l3 {
+namespace {
+
+constexpr int RADIX_BITS = 8;
+constexpr int RADIX = 1 << RADIX_BITS;
+constexpr int SORT_THREADS = 256;
+constexpr int SORT_WARPS = SORT_THREADS / 32;
+constexpr int SORT_ITEMS = 8;                            // per thread
+constexpr int SORT_TILE = SORT_THREADS * SORT_ITEMS;     // elements per CTA
+constexpr int WARP_SPAN = SORT_TILE / SORT_WARPS;        // contiguous elements per warp
+constexpr int SCAN_THREADS = 1024;
+constexpr int SCAN_ITEMS = 4;
+constexpr int SCAN_CHUNK = SCAN_THREADS * SCAN_ITEMS;
+
+// slots of the device info block read back at the end of l3_plan
+enum {
+  INFO_ERR = 0,
+  INFO_G,
+  INFO_TILES,
+  INFO_TAILS,
+  INFO_ROWS,
+  INFO_ROWS_MULTI,
+  INFO_DENSE_GROUPS,
+  INFO_MAX_TOKENS,
+  INFO_SLOTS
+};
+
+__device__ __forceinline__ uint32_t lanemask_lt() {
+  uint32_t m;
+  asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+  return m;
+}
+
+__global__ void k_validate_offsets(const int32_t *__restrict__ offsets, int64_t vocab, int64_t v,
+                                   int64_t k, int32_t *info) {
+  int64_t t = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+  if (t >= vocab) return;
+  int64_t d = (int64_t)offsets[t + 1] - offsets[t];
+  bool bad = d < 1 || d > k;
+  if (t == 0 && offsets[0] != 0) bad = true;
+  if (t == vocab - 1 && offsets[vocab] != v) bad = true;
+  if (bad) atomicOr(&info[INFO_ERR], DEV_ERR_BAD_OFFSETS);
+}
+
+// Digit histogram of one tile; counts land digit-major: hist[d * n_tiles + tile].
+__global__ void __launch_bounds__(SORT_THREADS)
+    k_radix_hist(const int32_t *__restrict__ keys, int64_t n, int shift, int32_t *__restrict__ hist,
+                 int n_tiles, int64_t vocab, int32_t *info) {
+  __shared__ int32_t cnt[RADIX];
+  for (int i = threadIdx.x; i < RADIX; i += SORT_THREADS) cnt[i] = 0;
+  __syncthreads();
+  int64_t base = (int64_t)blockIdx.x * SORT_TILE;
+  bool bad = false;
+#pragma unroll
+  for (int j = 0; j < SORT_ITEMS; ++j) {
+    int64_t i = base + threadIdx.x + (int64_t)j * SORT_THREADS;
+    if (i < n) {
+      int32_t key = keys[i];
+      if (vocab > 0 && (key < 0 || key >= vocab)) bad = true;
+      atomicAdd(&cnt[((uint32_t)key >> shift) & (RADIX - 1)], 1);
+    }
+  }
+  if (bad) atomicOr(&info[INFO_ERR], DEV_ERR_TOKEN_RANGE);
+  __syncthreads();
+  for (int d = threadIdx.x; d < RADIX; d += SORT_THREADS) hist[(int64_t)d * n_tiles + blockIdx.x] = cnt[d];
+}
+
+// Stable scatter of one tile. offs[d * n_tiles + tile] is the first output
+// position of digit d for this tile (exclusive scan of the histogram in
+// digit-major order). Each warp owns a contiguous span of the tile and walks
+// it in order, ranking equal digits with __match_any_sync, so the output keeps
+// input order among equal digits.
+__global__ void __launch_bounds__(SORT_THREADS)
+    k_radix_scatter(const int32_t *__restrict__ keys_in, const int32_t *__restrict__ vals_in,
+                    int32_t *__restrict__ keys_out, int32_t *__restrict__ vals_out, int64_t n,
+                    int shift, const int32_t *__restrict__ offs, int n_tiles) {
+  __shared__ int32_t whist[SORT_WARPS][RADIX];
+  __shared__ int32_t dbase[RADIX];
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  for (int i = threadIdx.x; i < SORT_WARPS * RADIX; i += SORT_THREADS) (&whist[0][0])[i] = 0;
+  __syncthreads();
+
+  int64_t base = (int64_t)blockIdx.x * SORT_TILE + (int64_t)warp * WARP_SPAN;
+  int32_t key[SORT_ITEMS], rank[SORT_ITEMS];
+  int digit[SORT_ITEMS];
+  const uint32_t lt = lanemask_lt();
+#pragma unroll
+  for (int it = 0; it < SORT_ITEMS; ++it) {
+    int64_t i = base + it * 32 + lane;
+    bool valid = i < n;
+    key[it] = valid ? keys_in[i] : 0;
+    int d = valid ? (int)(((uint32_t)key[it] >> shift) & (RADIX - 1)) : RADIX;
+    digit[it] = d;
+    uint32_t peers = __match_any_sync(0xffffffffu, d);
+    int prior = valid ? whist[warp][d] : 0;
+    rank[it] = prior + __popc(peers & lt);
+    __syncwarp();
+    if (valid && lane == __ffs(peers) - 1) whist[warp][d] = prior + __popc(peers);
+    __syncwarp();
+  }
+  __syncthreads();
+  for (int d = threadIdx.x; d < RADIX; d += SORT_THREADS) {
+    int32_t run = 0;
+#pragma unroll
+    for (int w = 0; w < SORT_WARPS; ++w) {
+      int32_t c = whist[w][d];
+      whist[w][d] = run;
+      run += c;
+    }
+    dbase[d] = offs[(int64_t)d * n_tiles + blockIdx.x];
+  }
+  __syncthreads();
+#pragma unroll
+  for (int it = 0; it < SORT_ITEMS; ++it) {
+    int64_t i = base + it * 32 + lane;
+    if (i < n) {
+      int d = digit[it];
+      int32_t pos = dbase[d] + whist[warp][d] + rank[it];
+      keys_out[pos] = key[it];
+      vals_out[pos] = vals_in ? vals_in[i] : (int32_t)i;
+    }
+  }
+}
+
+// One-CTA exclusive scan: out[i] = sum in[0..i-1] for i <= n (out has n + 1
+// entries; in == out is allowed). The total also goes to *total if given.
+__global__ void __launch_bounds__(SCAN_THREADS)
+    k_scan_exclusive(const int32_t *in, int32_t *out, int64_t n, int32_t *total) {
+  __shared__ int32_t warp_sums[SCAN_THREADS / 32];
+  __shared__ int32_t chunk_total;
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  int32_t carry = 0;
+  for (int64_t base = 0; base < n; base += SCAN_CHUNK) {
+    int32_t v[SCAN_ITEMS];
+    int32_t local = 0;
+#pragma unroll
+    for (int j = 0; j < SCAN_ITEMS; ++j) {
+      int64_t i = base + (int64_t)threadIdx.x * SCAN_ITEMS + j;
+      v[j] = i < n ? in[i] : 0;
+      local += v[j];
+    }
+    // inclusive warp scan of the per-thread sums
+    int32_t incl = local;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      int32_t t = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += t;
+    }
+    if (lane == 31) warp_sums[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+      int32_t w = warp_sums[lane];
+      int32_t wi = w;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        int32_t t = __shfl_up_sync(0xffffffffu, wi, o);
+        if (lane >= o) wi += t;
+      }
+      warp_sums[lane] = wi - w;  // exclusive prefix of warp totals
+      if (lane == 31) chunk_total = wi;
+    }
+    __syncthreads();
+    int32_t run = carry + warp_sums[warp] + (incl - local);
+#pragma unroll
+    for (int j = 0; j < SCAN_ITEMS; ++j) {
+      int64_t i = base + (int64_t)threadIdx.x * SCAN_ITEMS + j;
+      if (i < n) out[i] = run;
+      run += v[j];
+    }
+    carry += chunk_total;
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    out[n] = carry;
+    if (total) *total = carry;
+  }
+}
+
+// head[i] = 1 where a new ID starts in sorted order; inv_perm[perm[i]] = i.
+__global__ void k_group_heads(const int32_t *__restrict__ sorted, const int32_t *__restrict__ perm,
+                              int64_t n, int32_t *__restrict__ head, int32_t *__restrict__ inv_perm) {
+  int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  head[i] = (i == 0 || sorted[i] != sorted[i - 1]) ? 1 : 0;
+  inv_perm[perm[i]] = (int32_t)i;
+}
+
+__global__ void k_group_fill(const int32_t *__restrict__ sorted, const int32_t *__restrict__ head,
+                             const int32_t *__restrict__ gpos, int64_t n,
+                             const int32_t *__restrict__ offsets, int64_t vocab,
+                             int32_t *__restrict__ group_ids, int32_t *__restrict__ group_tok_start,
+                             int32_t *__restrict__ group_row_start, int32_t *__restrict__ group_rows,
+                             const int32_t *info) {
+  int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+  if (i == 0) group_tok_start[info[INFO_G]] = (int32_t)n;
+  if (i >= n || !head[i]) return;
+  int32_t g = gpos[i];
+  int32_t id = sorted[i];
+  group_ids[g] = id;
+  group_tok_start[g] = (int32_t)i;
+  bool ok = id >= 0 && id < vocab;
+  int32_t r0 = ok ? offsets[id] : 0;
+  group_row_start[g] = r0;
+  group_rows[g] = ok ? offsets[id + 1] - r0 : 0;
+}
+
+__global__ void k_item_counts(const int32_t *__restrict__ group_tok_start,
+                              const int32_t *__restrict__ group_rows, int64_t cap,
+                              int dense_min_tokens, int dense_min_rows,
+                              int32_t *__restrict__ tiles, int32_t *__restrict__ tails,
+                              int32_t *info) {
+  int64_t g = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+  if (g >= cap) return;
+  int32_t G = info[INFO_G];
+  int32_t nt = 0, nl = 0;
+  if (g < G) {
+    int32_t c = group_tok_start[g + 1] - group_tok_start[g];
+    int32_t rows = group_rows[g];
+    bool dense = dense_min_tokens > 0 && c >= dense_min_tokens && rows >= dense_min_rows;
+    if (dense) {
+      nt = (c + DENSE_TILE_M - 1) / DENSE_TILE_M;
+      atomicAdd(&info[INFO_DENSE_GROUPS], 1);
+    } else {
+      nl = (c + TAIL_TOKENS - 1) / TAIL_TOKENS;
+    }
+    if (rows > 1) atomicAdd(&info[INFO_ROWS_MULTI], rows);
+    atomicMax(&info[INFO_MAX_TOKENS], c);
+  }
+  tiles[g] = nt;
+  tails[g] = nl;
+}
+
+__global__ void k_item_fill(const int32_t *__restrict__ group_tok_start,
+                            const int32_t *__restrict__ tiles, const int32_t *__restrict__ tile_off,
+                            const int32_t *__restrict__ tails, const int32_t *__restrict__ tail_off,
+                            int64_t cap, DenseTile *__restrict__ dense, TailItem *__restrict__ tail,
+                            const int32_t *info) {
+  int64_t g = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+  if (g >= cap || g >= info[INFO_G]) return;
+  int32_t start = group_tok_start[g];
+  for (int32_t j = 0; j < tiles[g]; ++j)
+    dense[tile_off[g] + j] = DenseTile{(int32_t)g, start + j * DENSE_TILE_M};
+  for (int32_t j = 0; j < tails[g]; ++j)
+    tail[tail_off[g] + j] = TailItem{(int32_t)g, start + j * TAIL_TOKENS};
+}
+
+inline int blocks_for(int64_t n, int threads) { return (int)std::max<int64_t>(1, (n + threads - 1) / threads); }
+
+}  // namespace
+
+// Scratch needed while building the plan, beyond the plan's own arrays.
+size_t plan_scratch_bytes(int64_t n) {
+  int64_t tiles = std::max<int64_t>(1, (n + SORT_TILE - 1) / SORT_TILE);
+  size_t ints = 0;
+  ints += 2 * (size_t)n;                 // ping-pong keys / vals
+  ints += (size_t)RADIX * tiles + 1;     // histogram / offsets
+  ints += 2 * ((size_t)n + 1);           // head flags, group positions
+  ints += 4 * ((size_t)n + 1);           // tiles, tile offsets, tails, tail offsets
+  ints += 64;                            // info block
+  return ints * sizeof(int32_t) + 256;
+}
+
+l3_status build_plan(l3_plan_s *p, const int32_t *ids, const int32_t *offsets, cudaStream_t s,
+                     void *scratch, size_t scratch_bytes) {
+  const int64_t n = p->n_tokens;
+  const int64_t vocab = p->dims.vocab;
+  const int64_t cap = n + 1;
+  int32_t *sp = reinterpret_cast<int32_t *>(scratch);
+  int32_t *keys_tmp = sp;
+  sp += n;
+  int32_t *vals_tmp = sp;
+  sp += n;
+  int64_t n_tiles = std::max<int64_t>(1, (n + SORT_TILE - 1) / SORT_TILE);
+  int32_t *hist = sp;
+  sp += RADIX * n_tiles + 1;
+  int32_t *head = sp;
+  sp += cap;
+  int32_t *gpos = sp;
+  sp += cap;
+  int32_t *tiles = sp;
+  sp += cap;
+  int32_t *tile_off = sp;
+  sp += cap;
+  int32_t *tails = sp;
+  sp += cap;
+  int32_t *tail_off = sp;
+  sp += cap;
+  int32_t *info = sp;
+  sp += 64;
+  if ((size_t)((char *)sp - (char *)scratch) > scratch_bytes) {
+    set_error("internal: plan scratch too small");
+    return L3_ERR_INVALID_ARG;
+  }
+
+  L3_CUDA_TRY(cudaMemsetAsync(info, 0, 64 * sizeof(int32_t), s));
+  {
+    LaunchTimer t("plan_validate", s);
+    k_validate_offsets<<<blocks_for(vocab, 256), 256, 0, s>>>(offsets, vocab, p->dims.v, p->dims.k,
+                                                              info);
+  }
+  if (n > 0) {
+    // number of 8-bit digits that cover IDs 0..vocab-1
+    int bits = 1;
+    while (bits < 31 && ((int64_t)1 << bits) < vocab) ++bits;
+    int passes = (bits + RADIX_BITS - 1) / RADIX_BITS;
+    // ping-pong so that the last pass lands in the plan's arrays
+    int32_t *kbuf[2], *vbuf[2];
+    if (passes % 2 == 1) {
+      kbuf[0] = keys_tmp; vbuf[0] = vals_tmp;      // (unused as input of pass 0)
+      kbuf[1] = p->sorted_ids; vbuf[1] = p->perm;
+    } else {
+      kbuf[0] = p->sorted_ids; vbuf[0] = p->perm;
+      kbuf[1] = keys_tmp; vbuf[1] = vals_tmp;
+    }
+    const int32_t *kin = ids;
+    const int32_t *vin = nullptr;
+    for (int pass = 0; pass < passes; ++pass) {
+      int shift = pass * RADIX_BITS;
+      int32_t *kout = kbuf[(pass + 1) % 2];
+      int32_t *vout = vbuf[(pass + 1) % 2];
+      {
+        LaunchTimer t("plan_radix_hist", s);
+        k_radix_hist<<<(int)n_tiles, SORT_THREADS, 0, s>>>(kin, n, shift, hist, (int)n_tiles,
+                                                          pass == 0 ? vocab : 0, info);
+      }
+      {
+        LaunchTimer t("plan_scan", s);
+        k_scan_exclusive<<<1, SCAN_THREADS, 0, s>>>(hist, hist, RADIX * n_tiles, nullptr);
+      }
+      {
+        LaunchTimer t("plan_radix_scatter", s);
+        k_radix_scatter<<<(int)n_tiles, SORT_THREADS, 0, s>>>(kin, vin, kout, vout, n, shift, hist,
+                                                             (int)n_tiles);
+      }
+      kin = kout;
+      vin = vout;
+    }
+    {
+      LaunchTimer t("plan_group_heads", s);
+      k_group_heads<<<blocks_for(n, 256), 256, 0, s>>>(p->sorted_ids, p->perm, n, head,
+                                                       p->inv_perm);
+    }
+    {
+      LaunchTimer t("plan_scan", s);
+      k_scan_exclusive<<<1, SCAN_THREADS, 0, s>>>(head, gpos, n, &info[INFO_G]);
+    }
+    L3_CUDA_TRY(cudaMemsetAsync(p->group_rows, 0, cap * sizeof(int32_t), s));
+    {
+      LaunchTimer t("plan_group_fill", s);
+      k_group_fill<<<blocks_for(n, 256), 256, 0, s>>>(p->sorted_ids, head, gpos, n, offsets, vocab,
+                                                      p->group_ids, p->group_tok_start,
+                                                      p->group_row_start, p->group_rows, info);
+    }
+    {
+      LaunchTimer t("plan_scan", s);
+      k_scan_exclusive<<<1, SCAN_THREADS, 0, s>>>(p->group_rows, p->seg_rows, n, &info[INFO_ROWS]);
+    }
+    int dense_min_tokens = 0, dense_min_rows = 0;  // tensor-core attention not wired yet
+    {
+      LaunchTimer t("plan_item_counts", s);
+      k_item_counts<<<blocks_for(cap, 256), 256, 0, s>>>(p->group_tok_start, p->group_rows, n,
+                                                         dense_min_tokens, dense_min_rows, tiles,
+                                                         tails, info);
+    }
+    {
+      LaunchTimer t("plan_scan", s);
+      k_scan_exclusive<<<1, SCAN_THREADS, 0, s>>>(tiles, tile_off, n, &info[INFO_TILES]);
+    }
+    {
+      LaunchTimer t("plan_scan", s);
+      k_scan_exclusive<<<1, SCAN_THREADS, 0, s>>>(tails, tail_off, n, &info[INFO_TAILS]);
+    }
+    {
+      LaunchTimer t("plan_item_fill", s);
+      k_item_fill<<<blocks_for(n, 256), 256, 0, s>>>(p->group_tok_start, tiles, tile_off, tails,
+                                                     tail_off, n, p->dense_tiles, p->tail_items,
+                                                     info);
+    }
+  } else {
+    L3_CUDA_TRY(cudaMemsetAsync(p->group_tok_start, 0, sizeof(int32_t), s));
+    L3_CUDA_TRY(cudaMemsetAsync(p->seg_rows, 0, sizeof(int32_t), s));
+  }
+  L3_CUDA_TRY(cudaGetLastError());
+
+  int32_t host_info[INFO_SLOTS];
+  L3_CUDA_TRY(cudaMemcpyAsync(host_info, info, sizeof host_info, cudaMemcpyDeviceToHost, s));
+  L3_CUDA_TRY(cudaStreamSynchronize(s));
+  if (host_info[INFO_ERR] & DEV_ERR_BAD_OFFSETS) {
+    set_error("offsets invalid: need offsets[0] = 0, offsets[vocab] = v and 1 <= d_t <= k");
+    return L3_ERR_BAD_OFFSETS;
+  }
+  if (host_info[INFO_ERR] & DEV_ERR_TOKEN_RANGE) {
+    set_error("a token id is outside [0, vocab)");
+    return L3_ERR_TOKEN_RANGE;
+  }
+  p->n_groups = host_info[INFO_G];
+  p->n_dense_tiles = host_info[INFO_TILES];
+  p->n_tail_items = host_info[INFO_TAILS];
+  p->unique_rows = host_info[INFO_ROWS];
+  p->unique_rows_multi = host_info[INFO_ROWS_MULTI];
+  p->n_dense_groups = host_info[INFO_DENSE_GROUPS];
+  p->max_group_tokens = host_info[INFO_MAX_TOKENS];
+  return L3_OK;
+}
+
+}  // namespace l3

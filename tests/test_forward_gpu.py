@@ -1,0 +1,102 @@
+"""l3_forward on the GPU against the fp64 oracle (kimjy99 review, Method,
+eq. L³), element by element on the same seeded inputs.
+
+Bar: max |y_gpu - y_oracle| / RMS(y_oracle) <= 2e-2 for bf16 and 1e-4 for
+fp32. Small workloads are compared on every token; the full-size workloads
+are run in the same launch configuration the bench times, and compared on
+a sample of tokens the oracle computes one by one.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import static_token_routed_b200 as l3
+from l3_cases import (EPS, TOL, dims_of, host_workload, rel_max_err, run_forward,
+                      sample_tokens, to_device)
+from static_token_routed_b200 import workloads as wl
+
+pytestmark = pytest.mark.gpu
+
+
+def oracle_y(t, b, select=None, eps=EPS):
+    return oracle.forward(b.ids, t.offsets, b.x, t.W_K, t.W_V, t.W_up, t.ln_gamma, t.ln_beta,
+                          t.W_mix, eps, select=select)
+
+
+def test_tiny_fp32_all_tokens():
+    w, t, b = host_workload("tiny_fp32")
+    y, plan = run_forward(w, to_device(t, b))
+    want = oracle_y(t, b)
+    err = rel_max_err(y.double().cpu().numpy(), want)
+    assert err <= TOL["fp32"], err
+
+
+@pytest.mark.parametrize("name,n_tokens", [("small_bf16", 2048), ("decode", None),
+                                           ("dense_stress", 4096), ("uniform", 4096),
+                                           ("paper_shaped", 1024)])
+def test_reduced_batch_all_tokens(name, n_tokens):
+    """Full tables, a batch small enough for the oracle on every token."""
+    w, t, b = host_workload(name, n_tokens)
+    y, plan = run_forward(w, to_device(t, b))
+    want = oracle_y(t, b)
+    err = rel_max_err(y.double().cpu().numpy(), want)
+    assert err <= TOL[w.dtype], err
+
+
+@pytest.mark.parametrize("name", ["small_bf16", "paper_shaped", "dense_stress", "uniform"])
+def test_full_size_sampled(name):
+    w, t, b = host_workload(name)
+    y, plan = run_forward(w, to_device(t, b))
+    sel = sample_tokens(b.ids.numpy(), t.offsets.numpy(), 384, seed=1)
+    want = oracle_y(t, b, select=sel)
+    got = y[torch.from_numpy(sel).cuda()].double().cpu().numpy()
+    err = rel_max_err(got, want)
+    assert err <= TOL[w.dtype], err
+    assert torch.isfinite(y.float()).all()
+
+
+def test_deterministic_and_permutation_consistent():
+    """Two runs are bitwise equal; permuting the batch permutes y (papernotes
+    整体框架: no cross-token mixing) to within the bf16 bar."""
+    w, t, b = host_workload("small_bf16", 3000)
+    dev = to_device(t, b)
+    y1, _ = run_forward(w, dev)
+    y2, _ = run_forward(w, dev)
+    assert torch.equal(y1, y2)
+    pi = torch.randperm(3000, generator=torch.Generator().manual_seed(0)).cuda()
+    dev2 = dict(dev, ids=dev["ids"][pi].contiguous(), x=dev["x"][pi].contiguous())
+    y3, _ = run_forward(w, dev2)
+    err = rel_max_err(y3.double().cpu().numpy(), y1[pi].double().cpu().numpy())
+    assert err <= TOL["bf16"], err
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp32"])
+def test_edge_cases_small(dtype):
+    """d_t = 1 everywhere, d_t = k everywhere, one token, ragged widths."""
+    tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    rng = np.random.default_rng(7)
+    for vocab, dt, n, d_in, d_emb, d_up, d_out in [(50, 1, 33, 32, 16, 48, 16),
+                                                    (20, 37, 300, 64, 32, 32, 80),
+                                                    (7, 5, 1, 16, 16, 16, 16),
+                                                    (300, 0, 1000, 144, 96, 176, 48)]:
+        d = rng.integers(1, 9, size=vocab) if dt == 0 else np.full(vocab, dt)
+        off = torch.from_numpy(np.concatenate([[0], np.cumsum(d)]).astype(np.int32))
+        v = int(off[-1])
+        g = torch.Generator().manual_seed(vocab)
+        ids = torch.randint(0, vocab, (n,), generator=g, dtype=torch.int32)
+        mk = lambda *s: (torch.randn(*s, generator=g) / s[-1] ** 0.5).to(tdt)
+        t = wl.Tables(off, mk(v, d_in), mk(v, d_emb), mk(d_up, d_emb),
+                      (1 + 0.1 * torch.randn(d_up, generator=g)).to(tdt),
+                      (0.1 * torch.randn(d_up, generator=g)).to(tdt), mk(d_out, d_up + d_in))
+        bt = wl.Batch(ids, mk(n, d_in))
+        dims = l3.make_dims(vocab, v, int(d.max()), d_in, d_emb, d_up, d_out, tdt, EPS)
+        dev = to_device(t, bt)
+        plan = l3.l3_plan(dev["ids"], dev["offsets"], dims)
+        y = torch.empty(n, d_out, dtype=tdt, device="cuda")
+        l3.l3_forward(dev["x"], plan, dev["W_K"], dev["W_V"], dev["W_up"], dev["ln_gamma"],
+                      dev["ln_beta"], dev["W_mix"], y)
+        l3.l3_forward_status(plan)
+        want = oracle_y(t, bt)
+        err = rel_max_err(y.double().cpu().numpy(), want)
+        assert err <= TOL[dtype], (vocab, dt, n, err)
