@@ -157,6 +157,45 @@ l3_status l3_forward(const void *x, l3_plan_t plan, const void *W_K, const void 
                      const void *W_up, const void *ln_gamma, const void *ln_beta,
                      const void *W_mix, void *y, void *stream);
 
+/*
+ * l3_sort_tokens_noalloc — the stable sort step of l3_plan, for callers that
+ * cannot allocate device memory. The pages have no counterpart: this entry
+ * point exists for integration, not for the method.
+ *
+ * Who needs it: a process whose device memory is already reserved by
+ * another allocator (a serving engine or framework caching allocator that
+ * takes nearly all of HBM at start-up, so a cudaMalloc would fail or compete
+ * with it), or a latency-critical loop that cannot accept the device-wide
+ * synchronisation cudaMalloc / cudaFree can imply. This call allocates
+ * nothing: no cudaMalloc, cudaFree or allocating library routine.
+ *
+ *   token_ids   device int32 [n_tokens], each in [0, vocab) (not checked:
+ *               an out-of-range ID gives an unspecified order, never an
+ *               out-of-bounds access)
+ *   n_tokens    0 <= N <= L3_SORT_NOALLOC_MAX_TOKENS (65536); larger N is
+ *               rejected with L3_ERR_INVALID_ARG
+ *   vocab       number of token IDs, >= 1
+ *   perm        device int32 [N], out: original index at sorted position i
+ *   inv_perm    device int32 [N], out: sorted position of original token n
+ *   sorted_ids  device int32 [N], out: token ID at sorted position i
+ * The outputs equal l3_plan's perm / inv_perm / sorted_ids for the same IDs.
+ *
+ * Scratch: a file-scope device array of 557,312 bytes (2 x 65536 keys and
+ * values plus the digit histogram) that every GPU which loads libl3.so holds
+ * until the process exits. The first call on a device looks up the array's
+ * device address (cudaGetSymbolAddress) with that device current; make that
+ * first call before any stream capture on the device. Every call shares the
+ * one array and overwrites it (each call writes every scratch word before it
+ * reads it, so stale contents do not matter): calls that overlap on the GPU,
+ * on different streams or from different host threads, race. Serialize them.
+ * Enqueued on `stream`; does not synchronize. Errors: L3_ERR_INVALID_ARG,
+ * L3_ERR_CUDA.
+ */
+#define L3_SORT_NOALLOC_MAX_TOKENS 65536
+l3_status l3_sort_tokens_noalloc(const int32_t *token_ids, int64_t n_tokens, int64_t vocab,
+                                 int32_t *perm, int32_t *inv_perm, int32_t *sorted_ids,
+                                 void *stream);
+
 /* Synchronizes the plan's last stream and returns L3_ERR_TIMEOUT if a
  * bounded wait inside an l3_forward kernel gave up since the plan was made
  * (the outputs of that call are then incomplete), L3_ERR_CUDA on a CUDA

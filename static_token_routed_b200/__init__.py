@@ -28,6 +28,8 @@ from ._binding import (  # noqa: F401
     l3_plan_info,
     l3_profile_enable,
     l3_profile_read,
+    l3_sort_tokens_noalloc,
+    L3_SORT_NOALLOC_MAX_TOKENS,
     library,
     make_dims,
 )

@@ -21,7 +21,9 @@ STATUS = {0: "L3_OK", 1: "L3_ERR_INVALID_ARG", 2: "L3_ERR_TOKEN_RANGE", 3: "L3_E
 
 # every symbol include/l3.h declares
 EXPORTED = ["l3_plan", "l3_plan_info", "l3_plan_export", "l3_forward", "l3_forward_status",
-            "l3_plan_destroy", "l3_last_error", "l3_profile_enable", "l3_profile_read"]
+            "l3_plan_destroy", "l3_last_error", "l3_profile_enable", "l3_profile_read",
+            "l3_sort_tokens_noalloc"]
+L3_SORT_NOALLOC_MAX_TOKENS = 65536
 
 
 class L3Error(RuntimeError):
@@ -78,6 +80,8 @@ def library() -> ctypes.CDLL:
     lib.l3_profile_enable.argtypes = [i32]
     lib.l3_profile_read.restype = i32
     lib.l3_profile_read.argtypes = [ctypes.POINTER(KernelTime), i32]
+    lib.l3_sort_tokens_noalloc.restype = i32
+    lib.l3_sort_tokens_noalloc.argtypes = [p, i64, i64, p, p, p, p]
     _lib = lib
     return lib
 
@@ -212,3 +216,18 @@ def l3_profile_read(max_entries: int = 64) -> dict:
         raise L3Error(5, "l3_profile_read failed")
     return {buf[i].name.decode(): (int(buf[i].launches), float(buf[i].total_ms))
             for i in range(min(n, max_entries))}
+
+
+def l3_sort_tokens_noalloc(token_ids: torch.Tensor, vocab: int, perm: torch.Tensor,
+                           inv_perm: torch.Tensor, sorted_ids: torch.Tensor, stream=None):
+    """Stable sort by token ID into caller-owned buffers, with no device
+    allocation inside the library (fixed scratch array; see include/l3.h)."""
+    for nm, t in (("token_ids", token_ids), ("perm", perm), ("inv_perm", inv_perm),
+                  ("sorted_ids", sorted_ids)):
+        if t.dtype != torch.int32:
+            raise TypeError(f"{nm} must be int32")
+    n = token_ids.numel()
+    _check(library().l3_sort_tokens_noalloc(
+        _ptr(token_ids, "token_ids") if n else None, n, vocab,
+        _ptr(perm, "perm") if n else None, _ptr(inv_perm, "inv_perm") if n else None,
+        _ptr(sorted_ids, "sorted_ids") if n else None, _stream(stream, token_ids.device)))

@@ -13,6 +13,7 @@
 //   permutation -> scan -> group fill -> scan of d_t -> work-item counts ->
 //   scans -> work-item fill.
 #include <algorithm>
+#include <mutex>
 
 #include "l3_internal.cuh"
 
@@ -422,3 +423,114 @@ l3_status build_plan(l3_plan_s *p, const int32_t *ids, const int32_t *offsets, c
 }
 
 }  // namespace l3
+
+// ---------------------------------------------------------------------------
+// Allocation-free stable sort by token ID
+//
+// Some callers cannot allocate device memory at the point where they sort a
+// batch: a serving engine or framework allocator that has reserved nearly
+// all of HBM up front (a cudaMalloc would fail or fight it), or a latency-
+// critical loop that cannot afford the device-wide synchronisation that
+// cudaMalloc / cudaFree may imply. l3_sort_tokens_noalloc gives them the
+// plan's stable sort with its temporaries in the fixed array below instead of
+// in memory it allocates. The array lives in every GPU that loads this
+// library, until the process exits.
+// ---------------------------------------------------------------------------
+namespace l3 {
+namespace {
+
+constexpr int64_t NOALLOC_MAX_TOKENS = 65536;
+constexpr int64_t NOALLOC_TILES = (NOALLOC_MAX_TOKENS + SORT_TILE - 1) / SORT_TILE;
+// ping-pong keys and values, then the (digit, tile) histogram plus its total
+constexpr int64_t NOALLOC_SCRATCH_INTS = 2 * NOALLOC_MAX_TOKENS + RADIX * NOALLOC_TILES + 64;
+
+static __device__ __align__(256) int32_t g_sort_scratch[NOALLOC_SCRATCH_INTS];
+
+__global__ void k_inverse_perm(const int32_t *__restrict__ perm, int64_t n,
+                               int32_t *__restrict__ inv_perm) {
+  int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+  if (i < n) inv_perm[perm[i]] = (int32_t)i;
+}
+
+std::mutex g_scratch_mu;
+int32_t *g_scratch_ptr[64] = {};  // device address of g_sort_scratch, per device
+
+}  // namespace
+}  // namespace l3
+
+extern "C" l3_status l3_sort_tokens_noalloc(const int32_t *token_ids, int64_t n_tokens,
+                                            int64_t vocab, int32_t *perm, int32_t *inv_perm,
+                                            int32_t *sorted_ids, void *stream) {
+  using namespace l3;
+  set_error("");
+  if (n_tokens < 0 || n_tokens > NOALLOC_MAX_TOKENS) {
+    set_error("l3_sort_tokens_noalloc: n_tokens must be in [0, 65536] (fixed scratch size)");
+    return L3_ERR_INVALID_ARG;
+  }
+  if (vocab < 1 || vocab > INT32_MAX - 1) {
+    set_error("l3_sort_tokens_noalloc: vocab must be in [1, 2^31 - 2]");
+    return L3_ERR_INVALID_ARG;
+  }
+  if (n_tokens == 0) return L3_OK;
+  if (!token_ids || !perm || !inv_perm || !sorted_ids) {
+    set_error("l3_sort_tokens_noalloc: a pointer is NULL");
+    return L3_ERR_INVALID_ARG;
+  }
+  int dev = -1;
+  L3_CUDA_TRY(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 64) {
+    set_error("l3_sort_tokens_noalloc: device ordinal out of range");
+    return L3_ERR_INVALID_ARG;
+  }
+  int32_t *scratch = nullptr;
+  {
+    // once per device, with that device current: the host-side name of the
+    // array is not a device address, so ask the runtime for the real one
+    std::lock_guard<std::mutex> lk(g_scratch_mu);
+    if (!g_scratch_ptr[dev]) {
+      void *ptr = nullptr;
+      L3_CUDA_TRY(cudaGetSymbolAddress(&ptr, g_sort_scratch));
+      g_scratch_ptr[dev] = reinterpret_cast<int32_t *>(ptr);
+    }
+    scratch = g_scratch_ptr[dev];
+  }
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int64_t n = n_tokens;
+  const int64_t n_tiles = (n + SORT_TILE - 1) / SORT_TILE;
+  int32_t *keys_tmp = scratch;
+  int32_t *vals_tmp = scratch + NOALLOC_MAX_TOKENS;
+  int32_t *hist = scratch + 2 * NOALLOC_MAX_TOKENS;  // RADIX * n_tiles + 1 entries
+
+  int bits = 1;
+  while (bits < 31 && ((int64_t)1 << bits) < vocab) ++bits;
+  const int passes = (bits + RADIX_BITS - 1) / RADIX_BITS;
+  int32_t *kbuf[2], *vbuf[2];
+  if (passes % 2 == 1) {
+    kbuf[0] = keys_tmp; vbuf[0] = vals_tmp;
+    kbuf[1] = sorted_ids; vbuf[1] = perm;
+  } else {
+    kbuf[0] = sorted_ids; vbuf[0] = perm;
+    kbuf[1] = keys_tmp; vbuf[1] = vals_tmp;
+  }
+  // Every scratch word that is read is written earlier in the same call (the
+  // histogram kernel writes each (digit, tile) count, the scan and the
+  // scatter write all they later read), so nothing needs clearing between
+  // calls.
+  const int32_t *kin = token_ids;
+  const int32_t *vin = nullptr;
+  for (int pass = 0; pass < passes; ++pass) {
+    int shift = pass * RADIX_BITS;
+    int32_t *kout = kbuf[(pass + 1) % 2];
+    int32_t *vout = vbuf[(pass + 1) % 2];
+    k_radix_hist<<<(int)n_tiles, SORT_THREADS, 0, s>>>(kin, n, shift, hist, (int)n_tiles, 0,
+                                                      nullptr);
+    k_scan_exclusive<<<1, SCAN_THREADS, 0, s>>>(hist, hist, RADIX * n_tiles, nullptr);
+    k_radix_scatter<<<(int)n_tiles, SORT_THREADS, 0, s>>>(kin, vin, kout, vout, n, shift, hist,
+                                                         (int)n_tiles);
+    kin = kout;
+    vin = vout;
+  }
+  k_inverse_perm<<<(int)((n + 255) / 256), 256, 0, s>>>(perm, n, inv_perm);
+  L3_CUDA_TRY(cudaGetLastError());
+  return L3_OK;
+}
