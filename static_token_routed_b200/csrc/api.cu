@@ -163,6 +163,7 @@ l3_status l3_plan(const int32_t *token_ids, int64_t n_tokens, const int32_t *off
 
   const int64_t n = n_tokens, cap = n + 1;
   const size_t el = dims->dtype == L3_BF16 ? 2 : 4;
+  p->tc_gemm = tc_gemm_supported(*dims);
   size_t sizes[] = {
       align256(n * 4),                                            // perm
       align256(n * 4),                                            // inv_perm
@@ -177,8 +178,10 @@ l3_status l3_plan(const int32_t *token_ids, int64_t n_tokens, const int32_t *off
       align256(64),                                               // device flags
       align256(n * dims->d_emb * el),                             // a
       align256(n * dims->d_up * el),                              // h
-      align256(n * dims->d_up * 4),                               // z (CUDA-core GEMM path)
+      align256(p->tc_gemm ? 0 : n * dims->d_up * 4),              // z (CUDA-core GEMM path)
       align256(plan_scratch_bytes(n)),                            // plan-build scratch
+      align256(p->tc_gemm ? dims->d_up * dims->d_emb * 2 : 0),    // fp16 W_up
+      align256(p->tc_gemm ? dims->d_out * dims->d_up * 2 : 0),    // fp16 W_mix[:, :d_up]
   };
   size_t total = 0;
   for (size_t b : sizes) total += b;
@@ -210,6 +213,8 @@ l3_status l3_plan(const int32_t *token_ids, int64_t n_tokens, const int32_t *off
   p->h_buf = next(i++);
   p->z_buf = reinterpret_cast<float *>(next(i++));
   void *scratch = next(i++);
+  p->w_up16 = next(i++);
+  p->w_mixh16 = next(i++);
 
   st = L3_OK;
   e = cudaMemsetAsync(p->dev_flags, 0, 64, s);
@@ -298,8 +303,14 @@ l3_status l3_forward(const void *x, l3_plan_t p, const void *W_K, const void *W_
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   p->stream = s;
   l3_status st = launch_attn_tail(p, x, W_K, W_V, s);
-  if (st == L3_OK) st = launch_up_ln_simt(p, W_up, ln_gamma, ln_beta, s);
-  if (st == L3_OK) st = launch_mix_simt(p, x, W_mix, y, s);
+  if (p->tc_gemm) {
+    if (st == L3_OK) st = launch_weights_f16(p, W_up, W_mix, s);
+    if (st == L3_OK) st = launch_up_ln_tc(p, ln_gamma, ln_beta, s);
+    if (st == L3_OK) st = launch_mix_tc(p, x, W_mix, y, s);
+  } else {
+    if (st == L3_OK) st = launch_up_ln_simt(p, W_up, ln_gamma, ln_beta, s);
+    if (st == L3_OK) st = launch_mix_simt(p, x, W_mix, y, s);
+  }
   return st;
 }
 
@@ -315,6 +326,11 @@ l3_status l3_forward_status(l3_plan_t p) {
   if (flags[1] & DEV_ERR_TIMEOUT) {
     set_error("a bounded device-side wait in l3_forward gave up; outputs are incomplete");
     return L3_ERR_TIMEOUT;
+  }
+  if (flags[1] & DEV_ERR_F16_RANGE) {
+    set_error("W_up or W_mix holds a value outside fp16's finite range (|w| > 65504), which "
+              "the bf16 layer's fp16 intermediate GEMMs cannot represent");
+    return L3_ERR_UNSUPPORTED;
   }
   return L3_OK;
 }

@@ -1,0 +1,658 @@
+// Tensor-core (tcgen05 + TMEM + TMA) GEMMs of the bf16 layer.
+//
+// kimjy99 review, Method, eq. L³:
+//   h = LayerNorm(W_up a)                      (W_up: d_up x d_emb)
+//   y = W_mix [h ; x] = W_mix[:, :d_up] h + W_mix[:, d_up:] x
+//
+// k_mix_gemm: persistent, warp-specialised. Warp 0 streams 128x64 A tiles and
+// 256x64 B tiles into a 4-stage shared-memory ring with TMA; warp 1 issues
+// tcgen05.mma (M=128, N=256, K=16) into one of two TMEM accumulators; warps
+// 2-5 drain the other accumulator (tcgen05.ld) and store y while the next
+// tile's MMAs run. The two K-ranges of W_mix (the LayerNorm output h, then x)
+// accumulate into the same TMEM tile, so the concat [h ; x] never exists.
+//
+// k_up_ln_gemm: W_up a with the LayerNorm fused into the epilogue. A cluster
+// of ceil(d_up / 256) CTAs covers one 128-token tile's whole d_up row: each
+// CTA holds a 128 x 256 fp32 slice in TMEM, computes per-row (mean, M2) of
+// its slice, the cluster exchanges them through distributed shared memory
+// and merges them (Chan et al.'s pairwise update), and every CTA normalises
+// its slice in place and stores h.
+//
+// Precision: h and a are fp16 and meet fp16 copies of W_mix[:, :d_up] and
+// W_up (converted in k_to_f16), since tcgen05 kind::f16 needs both operands of
+// one MMA in the same type; the x range stays bf16 x bf16.
+#include <cuda_fp16.h>
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "l3_internal.cuh"
+#include "sm100.cuh"
+
+namespace l3 {
+namespace {
+
+using namespace sm100;
+
+constexpr int BM = 128;  // tokens per tile (TMEM lanes)
+constexpr int BK = 64;   // 64 16-bit elements = one 128-byte swizzle row
+constexpr int BN = 256;  // output columns per tile (max N of one MMA)
+constexpr int A_BYTES = BM * BK * 2;
+constexpr int B_BYTES = BN * BK * 2;
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int MIX_STAGES = 4;
+constexpr int UP_STAGES = 4;
+constexpr int GEMM_THREADS = 192;  // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
+constexpr uint32_t IDESC_F16 = idesc_f16(0, 0, BM, BN);
+constexpr uint32_t IDESC_BF16 = idesc_f16(1, 0, BM, BN);
+
+struct MixParams {
+  int M, N;        // tokens, d_out
+  int kb0, kb1;    // 64-wide k-blocks of the h range and of the x range
+  int n_tiles_n, n_tiles;
+  __nv_bfloat16 *y;
+  int64_t ldy;
+  int *err;
+};
+
+struct UpParams {
+  int M, N;        // tokens, d_up
+  int kb;          // k-blocks of d_emb
+  const __nv_bfloat16 *gamma, *beta;
+  float eps;
+  __half *h;
+  int *err;
+};
+
+// shared-memory layout after the stage ring
+struct Bars {
+  uint64_t full[8], empty[8], tfull[2], tempty[2], drain;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+__device__ __forceinline__ uint8_t *align1024(uint8_t *p) {
+  return reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+
+// Make sure no TMA write or MMA is still in flight before the CTA frees TMEM
+// and exits after a give-up. Normal runs have already waited for all of them.
+__device__ void drain_after_abort(Bars *b, int stages, const uint32_t *armed_parity,
+                                  const bool *armed, bool is_producer, bool is_mma,
+                                  const Abort &ab) {
+  Abort quiet{ab.flag, ab.err};
+  if (is_producer) {
+    for (int s = 0; s < stages; ++s)
+      if (armed[s]) {
+        // wait for the last armed phase; ignore the abort flag, keep the time bound
+        const uint32_t a = smem_u32(&b->full[s]);
+        const uint64_t t0 = globaltimer_ns();
+        while (!mbar_try_wait(a, armed_parity[s]) && globaltimer_ns() - t0 < WAIT_LIMIT_NS) {
+        }
+      }
+  }
+  if (is_mma) {
+    umma_commit(&b->drain);
+    const uint32_t a = smem_u32(&b->drain);
+    const uint64_t t0 = globaltimer_ns();
+    while (!mbar_try_wait(a, 0) && globaltimer_ns() - t0 < WAIT_LIMIT_NS) {
+    }
+  }
+  (void)quiet;
+}
+
+// ---------------------------------------------------------------------------
+// y = W_mix[:, :d_up] h + W_mix[:, d_up:] x
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(GEMM_THREADS, 1)
+    k_mix_gemm(const __grid_constant__ CUtensorMap mA0, const __grid_constant__ CUtensorMap mB0,
+               const __grid_constant__ CUtensorMap mA1, const __grid_constant__ CUtensorMap mB1,
+               MixParams P) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = align1024(smem_raw);
+  uint8_t *ring = smem;
+  Bars *b = reinterpret_cast<Bars *>(smem + MIX_STAGES * STAGE_BYTES);
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < MIX_STAGES; ++s) {
+      mbar_init(&b->full[s], 1);
+      mbar_init(&b->empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&b->tfull[a], 1);
+      mbar_init(&b->tempty[a], 4);
+    }
+    mbar_init(&b->drain, 1);
+    b->abort_flag = 0;
+    fence_mbar_init();
+    prefetch_tensormap(&mA0);
+    prefetch_tensormap(&mB0);
+    prefetch_tensormap(&mA1);
+    prefetch_tensormap(&mB1);
+  }
+  if (warp == 1) {
+    tmem_alloc(&b->tmem_base, 2 * BN);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = b->tmem_base;
+  const Abort ab{&b->abort_flag, P.err};
+  const int n_kb = P.kb0 + P.kb1;
+
+  if (warp == 0) {
+    if (elect_one()) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t armed_parity[MIX_STAGES];
+      bool armed[MIX_STAGES];
+      for (int s = 0; s < MIX_STAGES; ++s) armed[s] = false;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < P.n_tiles; tile += gridDim.x) {
+        const int m0 = (tile / P.n_tiles_n) * BM;
+        const int n0 = (tile % P.n_tiles_n) * BN;
+        for (int kb = 0; kb < n_kb; ++kb) {
+          if (!mbar_wait(&b->empty[stage], phase ^ 1, ab)) {
+            ok = false;
+            break;
+          }
+          uint8_t *sa = ring + stage * STAGE_BYTES;
+          mbar_arrive_expect_tx(&b->full[stage], STAGE_BYTES);
+          armed[stage] = true;
+          armed_parity[stage] = phase;
+          if (kb < P.kb0) {
+            tma_load_2d(sa, &mA0, &b->full[stage], kb * BK, m0);
+            tma_load_2d(sa + A_BYTES, &mB0, &b->full[stage], kb * BK, n0);
+          } else {
+            tma_load_2d(sa, &mA1, &b->full[stage], (kb - P.kb0) * BK, m0);
+            tma_load_2d(sa + A_BYTES, &mB1, &b->full[stage], (kb - P.kb0) * BK, n0);
+          }
+          if (++stage == MIX_STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      if (!ok) drain_after_abort(b, MIX_STAGES, armed_parity, armed, true, false, ab);
+    }
+  } else if (warp == 1) {
+    if (elect_one()) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      int it = 0;
+      for (int tile = blockIdx.x; ok && tile < P.n_tiles; tile += gridDim.x, ++it) {
+        const int acc = it & 1;
+        if (!mbar_wait(&b->tempty[acc], ((it >> 1) & 1) ^ 1, ab)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d = tmem + acc * BN;
+        for (int kb = 0; kb < n_kb; ++kb) {
+          if (!mbar_wait(&b->full[stage], phase, ab)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(ring + stage * STAGE_BYTES);
+          const uint32_t sb = sa + A_BYTES;
+          const uint32_t idesc = kb < P.kb0 ? IDESC_F16 : IDESC_BF16;
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k)
+            umma_f16(d, sdesc_sw128(sa + k * 32, 16, 1024), sdesc_sw128(sb + k * 32, 16, 1024),
+                     idesc, (kb | k) != 0);
+          umma_commit(&b->empty[stage]);
+          if (++stage == MIX_STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (ok) umma_commit(&b->tfull[acc]);
+      }
+      if (!ok) drain_after_abort(b, MIX_STAGES, nullptr, nullptr, false, true, ab);
+    }
+  } else {
+    // epilogue: warp (2..5) % 4 selects the TMEM lane quarter it may read
+    const int q = warp & 3;
+    const int r = q * 32 + lane;
+    int it = 0;
+    for (int tile = blockIdx.x; tile < P.n_tiles; tile += gridDim.x, ++it) {
+      const int acc = it & 1;
+      const bool got = __all_sync(0xffffffffu, mbar_wait(&b->tfull[acc], (it >> 1) & 1, ab));
+      if (!got) break;
+      tc_fence_after();
+      const int m = (tile / P.n_tiles_n) * BM + r;
+      const int n0 = (tile % P.n_tiles_n) * BN;
+      __nv_bfloat16 *yrow = P.y + (int64_t)m * P.ldy + n0;
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + acc * BN + c * 32, v);
+        tmem_wait_ld();
+        if (m < P.M) {
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int col = n0 + c * 32 + j * 8;
+            if (col < P.N) {
+              uint4 o;
+              __nv_bfloat162 *o2 = reinterpret_cast<__nv_bfloat162 *>(&o);
+#pragma unroll
+              for (int e = 0; e < 4; ++e)
+                o2[e] = __floats2bfloat162_rn(__uint_as_float(v[j * 8 + 2 * e]),
+                                              __uint_as_float(v[j * 8 + 2 * e + 1]));
+              *reinterpret_cast<uint4 *>(yrow + c * 32 + j * 8) = o;
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&b->tempty[acc]);
+    }
+  }
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 2 * BN);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// h = LayerNorm(W_up a), one cluster of ceil(d_up / 256) CTAs per 128 tokens
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(GEMM_THREADS, 1)
+    k_up_ln_gemm(const __grid_constant__ CUtensorMap mA, const __grid_constant__ CUtensorMap mB,
+                 UpParams P) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = align1024(smem_raw);
+  uint8_t *ring = smem;
+  Bars *b = reinterpret_cast<Bars *>(smem + UP_STAGES * STAGE_BYTES);
+  float *g_s = reinterpret_cast<float *>(b + 1);  // gamma of this CTA's 256 columns
+  float *b_s = g_s + BN;                          // beta
+  float *st_mean = b_s + BN;                      // per-row mean of this CTA's slice
+  float *st_m2 = st_mean + BM;                    // per-row sum of squared deviations
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const uint32_t rank = cluster_ctarank();
+  const uint32_t n_ranks = gridDim.x;  // one cluster spans the grid's x dimension
+  const int m0 = blockIdx.y * BM;
+  const int n0 = (int)rank * BN;
+  const int n_valid = min(BN, P.N - n0);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < UP_STAGES; ++s) {
+      mbar_init(&b->full[s], 1);
+      mbar_init(&b->empty[s], 1);
+    }
+    mbar_init(&b->tfull[0], 1);
+    mbar_init(&b->drain, 1);
+    b->abort_flag = 0;
+    fence_mbar_init();
+    prefetch_tensormap(&mA);
+    prefetch_tensormap(&mB);
+  }
+  if (warp == 1) {
+    tmem_alloc(&b->tmem_base, BN);
+    tmem_relinquish();
+  }
+  for (int i = threadIdx.x; i < BN; i += GEMM_THREADS) {
+    const bool v = n0 + i < P.N;
+    g_s[i] = v ? __bfloat162float(P.gamma[n0 + i]) : 0.f;
+    b_s[i] = v ? __bfloat162float(P.beta[n0 + i]) : 0.f;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = b->tmem_base;
+  const Abort ab{&b->abort_flag, P.err};
+
+  if (warp == 0) {
+    if (elect_one()) {
+      uint32_t armed_parity[UP_STAGES];
+      bool armed[UP_STAGES];
+      for (int s = 0; s < UP_STAGES; ++s) armed[s] = false;
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int kb = 0; kb < P.kb; ++kb) {
+        if (!mbar_wait(&b->empty[stage], phase ^ 1, ab)) {
+          ok = false;
+          break;
+        }
+        uint8_t *sa = ring + stage * STAGE_BYTES;
+        mbar_arrive_expect_tx(&b->full[stage], STAGE_BYTES);
+        armed[stage] = true;
+        armed_parity[stage] = phase;
+        tma_load_2d(sa, &mA, &b->full[stage], kb * BK, m0);
+        tma_load_2d(sa + A_BYTES, &mB, &b->full[stage], kb * BK, n0);
+        if (++stage == UP_STAGES) {
+          stage = 0;
+          phase ^= 1;
+        }
+      }
+      if (!ok) drain_after_abort(b, UP_STAGES, armed_parity, armed, true, false, ab);
+    }
+  } else if (warp == 1) {
+    if (elect_one()) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int kb = 0; kb < P.kb; ++kb) {
+        if (!mbar_wait(&b->full[stage], phase, ab)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t sa = smem_u32(ring + stage * STAGE_BYTES);
+        const uint32_t sb = sa + A_BYTES;
+#pragma unroll
+        for (int k = 0; k < BK / 16; ++k)
+          umma_f16(tmem, sdesc_sw128(sa + k * 32, 16, 1024), sdesc_sw128(sb + k * 32, 16, 1024),
+                   IDESC_F16, (kb | k) != 0);
+        umma_commit(&b->empty[stage]);
+        if (++stage == UP_STAGES) {
+          stage = 0;
+          phase ^= 1;
+        }
+      }
+      if (ok) umma_commit(&b->tfull[0]);
+      else drain_after_abort(b, UP_STAGES, nullptr, nullptr, false, true, ab);
+    }
+  }
+
+  // epilogue part 1: per-row mean and M2 of this CTA's slice
+  const bool epi = warp >= 2;
+  const int q = warp & 3;
+  const int r = q * 32 + lane;
+  const uint32_t trow = tmem + ((uint32_t)(q * 32) << 16);
+  bool have = false;
+  __syncwarp();
+  if (epi) {
+    have = __all_sync(0xffffffffu, mbar_wait(&b->tfull[0], 0, ab));
+    tc_fence_after();
+    float sum = 0.f;
+    if (have) {
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld32(trow + c * 32, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          if (c * 32 + j < n_valid) sum += __uint_as_float(v[j]);
+      }
+    }
+    const float mean = sum / (float)n_valid;
+    float m2 = 0.f;
+    if (have) {
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld32(trow + c * 32, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          if (c * 32 + j < n_valid) {
+            const float dlt = __uint_as_float(v[j]) - mean;
+            m2 = fmaf(dlt, dlt, m2);
+          }
+      }
+    }
+    st_mean[r] = mean;
+    st_m2[r] = m2;
+  }
+  __syncwarp();
+  cluster_sync();  // every CTA's (mean, M2) is visible cluster-wide
+
+  float mu = 0.f, rstd = 0.f;
+  if (epi) {
+    // merge the slices in rank order: n_a, mean_a, M2_a  (+)  n_b, mean_b, M2_b
+    float n_acc = 0.f, mean_acc = 0.f, m2_acc = 0.f;
+    for (uint32_t j = 0; j < n_ranks; ++j) {
+      const float nb = (float)min(BN, P.N - (int)j * BN);
+      const float mb = ld_shared_cluster_f32(map_shared_rank(&st_mean[r], j));
+      const float qb = ld_shared_cluster_f32(map_shared_rank(&st_m2[r], j));
+      const float n_new = n_acc + nb;
+      const float delta = mb - mean_acc;
+      mean_acc += delta * (nb / n_new);
+      m2_acc += qb + delta * delta * (n_acc * nb / n_new);
+      n_acc = n_new;
+    }
+    mu = mean_acc;
+    rstd = 1.0f / sqrtf(m2_acc / n_acc + P.eps);
+  }
+  cluster_sync();  // peers are done reading this CTA's statistics
+
+  if (epi && have) {
+    const int m = m0 + r;
+    __half *hrow = P.h + (int64_t)m * P.N + n0;
+#pragma unroll 1
+    for (int c = 0; c < BN / 32; ++c) {
+      uint32_t v[32];
+      tmem_ld32(trow + c * 32, v);
+      tmem_wait_ld();
+      if (m < P.M) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int col = c * 32 + j * 8;
+          if (col < n_valid) {
+            uint4 o;
+            __half2 *o2 = reinterpret_cast<__half2 *>(&o);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int k0 = col + 2 * e;
+              const float h0 = g_s[k0] * ((__uint_as_float(v[j * 8 + 2 * e]) - mu) * rstd) + b_s[k0];
+              const float h1 =
+                  g_s[k0 + 1] * ((__uint_as_float(v[j * 8 + 2 * e + 1]) - mu) * rstd) + b_s[k0 + 1];
+              o2[e] = __floats2half2_rn(h0, h1);
+            }
+            *reinterpret_cast<uint4 *>(hrow + col) = o;
+          }
+        }
+      }
+    }
+  }
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, BN);
+  }
+}
+
+// bf16 -> fp16 copy of a row-strided matrix; flags values outside fp16's range
+__global__ void k_to_f16(const __nv_bfloat16 *__restrict__ src, int64_t ld_src, int64_t rows,
+                         int64_t cols, __half *__restrict__ dst, int *err) {
+  const int64_t vec_per_row = cols / 8;
+  const int64_t total = rows * vec_per_row;
+  bool bad = false;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t r = i / vec_per_row, c = (i - r * vec_per_row) * 8;
+    uint4 v = *reinterpret_cast<const uint4 *>(src + r * ld_src + c);
+    const __nv_bfloat162 *in = reinterpret_cast<const __nv_bfloat162 *>(&v);
+    uint4 o;
+    __half2 *out = reinterpret_cast<__half2 *>(&o);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      float2 f = __bfloat1622float2(in[e]);
+      bad |= fabsf(f.x) > 65504.f || fabsf(f.y) > 65504.f;
+      out[e] = __floats2half2_rn(f.x, f.y);
+    }
+    *reinterpret_cast<uint4 *>(dst + r * cols + c) = o;
+  }
+  if (bad) atomicOr(err, DEV_ERR_F16_RANGE);
+}
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+int g_num_sms[64] = {};
+
+l3_status encoder(PFN_cuTensorMapEncodeTiled_v12000 *out) {
+  std::call_once(g_encode_once, [] {
+    cudaDriverEntryPointQueryResult q;
+    void *fn = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  if (!g_encode) {
+    set_error("cuTensorMapEncodeTiled is not available from the driver");
+    return L3_ERR_CUDA;
+  }
+  *out = g_encode;
+  return L3_OK;
+}
+
+// 2-D row-major [rows x cols] tensor of 16-bit elements, row stride ld elements,
+// box = 64 columns x box_rows rows, 128-byte swizzle, zero fill out of bounds.
+l3_status make_map(CUtensorMap *m, const void *base, CUtensorMapDataType dt, uint64_t rows,
+                   uint64_t cols, uint64_t ld, uint32_t box_rows) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc;
+  l3_status st = encoder(&enc);
+  if (st != L3_OK) return st;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {ld * 2};
+  cuuint32_t box[2] = {(cuuint32_t)BK, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(m, dt, 2, const_cast<void *>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    set_error("cuTensorMapEncodeTiled failed (code " + std::to_string((int)r) + ")");
+    return L3_ERR_CUDA;
+  }
+  return L3_OK;
+}
+
+int num_sms() {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  dev &= 63;
+  if (g_num_sms[dev] == 0) cudaDeviceGetAttribute(&g_num_sms[dev], cudaDevAttrMultiProcessorCount, dev);
+  return g_num_sms[dev];
+}
+
+constexpr size_t MIX_SMEM = 1024 + MIX_STAGES * STAGE_BYTES + sizeof(Bars);
+constexpr size_t UP_SMEM =
+    1024 + UP_STAGES * STAGE_BYTES + sizeof(Bars) + (2 * BN + 2 * BM) * sizeof(float);
+
+}  // namespace
+
+bool tc_gemm_supported(const l3_dims_t &d) {
+  return d.dtype == L3_BF16 && d.d_in % BK == 0 && d.d_emb % BK == 0 && d.d_up % BK == 0 &&
+         d.d_up <= 8 * BN;
+}
+
+l3_status launch_weights_f16(const l3_plan_s *p, const void *W_up, const void *W_mix,
+                             cudaStream_t s) {
+  const l3_dims_t &d = p->dims;
+  int *err = p->dev_flags + 1;
+  {
+    LaunchTimer t("to_f16", s);
+    k_to_f16<<<num_sms() * 4, 256, 0, s>>>(reinterpret_cast<const __nv_bfloat16 *>(W_up), d.d_emb,
+                                           d.d_up, d.d_emb, reinterpret_cast<__half *>(p->w_up16),
+                                           err);
+    k_to_f16<<<num_sms() * 4, 256, 0, s>>>(reinterpret_cast<const __nv_bfloat16 *>(W_mix),
+                                           d.d_up + d.d_in, d.d_out, d.d_up,
+                                           reinterpret_cast<__half *>(p->w_mixh16), err);
+  }
+  L3_CUDA_TRY(cudaGetLastError());
+  return L3_OK;
+}
+
+l3_status launch_up_ln_tc(const l3_plan_s *p, const void *gamma, const void *beta,
+                          cudaStream_t s) {
+  const l3_dims_t &d = p->dims;
+  CUtensorMap mA, mB;
+  l3_status st;
+  if ((st = make_map(&mA, p->a_buf, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, p->n_tokens, d.d_emb, d.d_emb,
+                     BM)) != L3_OK)
+    return st;
+  if ((st = make_map(&mB, p->w_up16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, d.d_up, d.d_emb, d.d_emb,
+                     BN)) != L3_OK)
+    return st;
+  UpParams P;
+  P.M = (int)p->n_tokens;
+  P.N = (int)d.d_up;
+  P.kb = (int)(d.d_emb / BK);
+  P.gamma = reinterpret_cast<const __nv_bfloat16 *>(gamma);
+  P.beta = reinterpret_cast<const __nv_bfloat16 *>(beta);
+  P.eps = d.ln_eps;
+  P.h = reinterpret_cast<__half *>(p->h_buf);
+  P.err = p->dev_flags + 1;
+  static bool attr[64] = {};
+  if (!attr[p->device & 63]) {
+    L3_CUDA_TRY(cudaFuncSetAttribute(k_up_ln_gemm, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)UP_SMEM));
+    attr[p->device & 63] = true;
+  }
+  const int cn = (int)((d.d_up + BN - 1) / BN);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(cn, (unsigned)((p->n_tokens + BM - 1) / BM), 1);
+  cfg.blockDim = dim3(GEMM_THREADS, 1, 1);
+  cfg.dynamicSmemBytes = UP_SMEM;
+  cfg.stream = s;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = cn;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  LaunchTimer t("up_ln_gemm_tc", s);
+  L3_CUDA_TRY(cudaLaunchKernelEx(&cfg, k_up_ln_gemm, mA, mB, P));
+  return L3_OK;
+}
+
+l3_status launch_mix_tc(const l3_plan_s *p, const void *x, const void *W_mix, void *y,
+                        cudaStream_t s) {
+  const l3_dims_t &d = p->dims;
+  CUtensorMap mA0, mB0, mA1, mB1;
+  l3_status st;
+  const uint64_t M = p->n_tokens;
+  if ((st = make_map(&mA0, p->h_buf, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, M, d.d_up, d.d_up, BM)) !=
+      L3_OK)
+    return st;
+  if ((st = make_map(&mB0, p->w_mixh16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, d.d_out, d.d_up, d.d_up,
+                     BN)) != L3_OK)
+    return st;
+  if ((st = make_map(&mA1, x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, M, d.d_in, d.d_in, BM)) != L3_OK)
+    return st;
+  const __nv_bfloat16 *wx = reinterpret_cast<const __nv_bfloat16 *>(W_mix) + d.d_up;
+  if ((st = make_map(&mB1, wx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, d.d_out, d.d_in, d.d_up + d.d_in,
+                     BN)) != L3_OK)
+    return st;
+  MixParams P;
+  P.M = (int)M;
+  P.N = (int)d.d_out;
+  P.kb0 = (int)(d.d_up / BK);
+  P.kb1 = (int)(d.d_in / BK);
+  P.n_tiles_n = (int)((d.d_out + BN - 1) / BN);
+  P.n_tiles = (int)((M + BM - 1) / BM) * P.n_tiles_n;
+  P.y = reinterpret_cast<__nv_bfloat16 *>(y);
+  P.ldy = d.d_out;
+  P.err = p->dev_flags + 1;
+  static bool attr[64] = {};
+  if (!attr[p->device & 63]) {
+    L3_CUDA_TRY(cudaFuncSetAttribute(k_mix_gemm, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)MIX_SMEM));
+    attr[p->device & 63] = true;
+  }
+  const int grid = std::min(P.n_tiles, num_sms());
+  LaunchTimer t("mix_gemm_tc", s);
+  k_mix_gemm<<<grid, GEMM_THREADS, MIX_SMEM, s>>>(mA0, mB0, mA1, mB1, P);
+  L3_CUDA_TRY(cudaGetLastError());
+  return L3_OK;
+}
+
+}  // namespace l3

@@ -29,6 +29,7 @@ enum : int32_t {
   DEV_ERR_TOKEN_RANGE = 1,
   DEV_ERR_BAD_OFFSETS = 2,
   DEV_ERR_TIMEOUT = 4,
+  DEV_ERR_F16_RANGE = 8,  // a bf16 weight outside fp16's finite range
 };
 
 // ---------------------------------------------------------------------------
@@ -92,6 +93,9 @@ struct l3_plan_s {
   void *a_buf = nullptr;               // [N x d_emb] dtype, original token order
   void *h_buf = nullptr;               // [N x d_up] dtype
   float *z_buf = nullptr;              // [N x d_up] fp32 (CUDA-core GEMM path only)
+  void *w_up16 = nullptr;              // [d_up x d_emb] fp16 copy of W_up (tensor-core path)
+  void *w_mixh16 = nullptr;            // [d_out x d_up] fp16 copy of W_mix[:, :d_up]
+  bool tc_gemm = false;                // tensor-core GEMMs in use
 };
 
 namespace l3 {
@@ -104,6 +108,15 @@ size_t plan_scratch_bytes(int64_t n_tokens);
 // attention, CUDA-core path (attn_tail.cu)
 l3_status launch_attn_tail(const l3_plan_s *p, const void *x, const void *W_K, const void *W_V,
                            cudaStream_t s);
+
+// GEMMs + LayerNorm, tensor-core path (gemm_tc.cu)
+bool tc_gemm_supported(const l3_dims_t &d);
+l3_status launch_weights_f16(const l3_plan_s *p, const void *W_up, const void *W_mix,
+                             cudaStream_t s);
+l3_status launch_up_ln_tc(const l3_plan_s *p, const void *gamma, const void *beta,
+                          cudaStream_t s);
+l3_status launch_mix_tc(const l3_plan_s *p, const void *x, const void *W_mix, void *y,
+                        cudaStream_t s);
 
 // GEMMs + LayerNorm, CUDA-core path (gemm_simt.cu)
 l3_status launch_up_ln_simt(const l3_plan_s *p, const void *W_up, const void *gamma,

@@ -79,7 +79,12 @@ def test_edge_cases_small(dtype):
     for vocab, dt, n, d_in, d_emb, d_up, d_out in [(50, 1, 33, 32, 16, 48, 16),
                                                     (20, 37, 300, 64, 32, 32, 80),
                                                     (7, 5, 1, 16, 16, 16, 16),
-                                                    (300, 0, 1000, 144, 96, 176, 48)]:
+                                                    (300, 0, 1000, 144, 96, 176, 48),
+                                                    # tensor-core GEMM shapes with ragged
+                                                    # token count and partial N tiles
+                                                    (40, 0, 333, 128, 64, 192, 80),
+                                                    (90, 0, 1000, 64, 128, 576, 272),
+                                                    (9, 3, 129, 192, 64, 64, 16)]:
         d = rng.integers(1, 9, size=vocab) if dt == 0 else np.full(vocab, dt)
         off = torch.from_numpy(np.concatenate([[0], np.cumsum(d)]).astype(np.int32))
         v = int(off[-1])
@@ -100,3 +105,14 @@ def test_edge_cases_small(dtype):
         want = oracle_y(t, bt)
         err = rel_max_err(y.double().cpu().numpy(), want)
         assert err <= TOL[dtype], (vocab, dt, n, err)
+
+
+def test_tensor_core_kernels_run():
+    """The bf16 layer's GEMMs run on the tcgen05 kernels (not a fallback)."""
+    w, t, b = host_workload("small_bf16", 2048)
+    dev = to_device(t, b)
+    l3.l3_profile_enable(True)
+    run_forward(w, dev)
+    kernels = l3.l3_profile_read()
+    l3.l3_profile_enable(False)
+    assert "mix_gemm_tc" in kernels and "up_ln_gemm_tc" in kernels, kernels
