@@ -303,6 +303,7 @@ l3_status l3_forward(const void *x, l3_plan_t p, const void *W_K, const void *W_
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   p->stream = s;
   l3_status st = launch_attn_tail(p, x, W_K, W_V, s);
+  if (st == L3_OK) st = launch_attn_dense(p, x, W_K, W_V, s);
   if (p->tc_gemm) {
     if (st == L3_OK) st = launch_weights_f16(p, W_up, W_mix, s);
     if (st == L3_OK) st = launch_up_ln_tc(p, ln_gamma, ln_beta, s);

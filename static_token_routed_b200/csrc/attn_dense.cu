@@ -1,0 +1,447 @@
+// Gather-attention on tensor cores for groups with many tokens.
+//
+// After the batch sort, the tokens that share an ID t form a contiguous group
+// whose attention mask is one dense block (sciencestack page, Fig. 3 caption;
+// kimjy99 review §2): every token of the group attends to the same d_t rows
+// K_t, V_t. For such a group the per-token products become matrix products,
+//     S = X_g K_t^T   (tokens x d_t),   P = exp(S - rowmax),   O = P V_t,
+//     a = O / rowsum(P)
+// which is the layer's V_t^T softmax(K_t x) for every token of the group at
+// once (kimjy99 review, Method, eq. L³).
+//
+// One CTA takes one 128-token tile of one group:
+//   - warps 2-3 gather the tile's x rows (through the sort permutation) into
+//     128-byte-swizzled shared memory, 64 columns at a time;
+//   - warp 0 streams the matching 64-column slices of K_t with TMA;
+//   - warp 1 issues tcgen05.mma (M = 128 tokens, N = d_t up to 2 x 256) so that
+//     S accumulates in TMEM over d_in;
+//   - warps 4-7 (one token row per thread, the TMEM lane it owns) take an exact
+//     row max and the exponentials, and write P as fp16 into shared memory;
+//   - warp 0 then streams V_t in 32-row slices with TMA, warps 4-7 turn each
+//     slice into fp16 in place, and warp 1 accumulates O = P V_t in the TMEM
+//     columns S no longer needs;
+//   - warps 4-7 scale O by 1 / rowsum and store a[perm[i]] (fp16), i.e. already
+//     in the caller's token order.
+// K_t and V_t are read from HBM by the group's first tile; its other tiles run
+// at the same time and find them in L2.
+// P and V_t meet in fp16 (10-bit mantissa): tcgen05 kind::f16 needs one type
+// for both operands, and a bf16 P would cost as much accuracy as a bf16 a.
+#include <cuda_fp16.h>
+#include <cudaTypedefs.h>
+
+#include "l3_internal.cuh"
+#include "sm100.cuh"
+
+namespace l3 {
+
+l3_status make_map_2d16(CUtensorMap *m, const void *base, bool bf16, uint64_t rows, uint64_t cols,
+                        uint64_t ld, uint32_t box_cols, uint32_t box_rows);
+
+namespace {
+
+using namespace sm100;
+
+constexpr int TM = 128;                 // tokens per tile
+constexpr int CK = 64;                  // d_in columns per S-phase slice
+constexpr int MAX_D = 512;              // d_t handled here (TMEM columns)
+constexpr int MAX_EMB = 512;
+constexpr int X_BYTES = TM * CK * 2;    // 16 KB
+constexpr int K_BYTES = MAX_D * CK * 2; // 64 KB
+constexpr int S_STAGE = X_BYTES + K_BYTES;
+constexpr int S_STAGES = 2;
+constexpr int P_BYTES = TM * MAX_D * 2;                 // 128 KB, 8 slices of 64 columns
+constexpr int V_ROWS = 32;                              // d_t rows per V slice
+constexpr int V_BLOCK = V_ROWS * 128;                   // one 64-column block of a V slice
+constexpr int V_BYTES = V_ROWS * MAX_EMB * 2;           // 32 KB
+constexpr int V_BUFS = 2;
+constexpr int REGION = (S_STAGES * S_STAGE > P_BYTES + V_BUFS * V_BYTES)
+                           ? S_STAGES * S_STAGE
+                           : P_BYTES + V_BUFS * V_BYTES;  // 192 KB
+constexpr int DENSE_THREADS = 256;
+constexpr float LOG2E = 1.4426950408889634f;
+
+struct DenseBars {
+  uint64_t xfull[S_STAGES], kfull[S_STAGES], sempty[S_STAGES];
+  uint64_t sfull, pready, ofull;
+  uint64_t vfull[V_BUFS], vconv[V_BUFS], vempty[V_BUFS];
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+struct DenseParams {
+  const __nv_bfloat16 *x;
+  __half *a;
+  const int32_t *perm;
+  const int32_t *group_tok_start;
+  const int32_t *group_row_start;
+  const int32_t *group_rows;
+  const DenseTile *tiles;
+  int d_in, d_emb;
+  int *err;
+};
+
+__device__ __forceinline__ uint8_t *align1024(uint8_t *p) {
+  return reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+
+__device__ __forceinline__ void spin_bounded(uint64_t *bar, uint32_t parity) {
+  const uint32_t a = smem_u32(bar);
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(a, parity) && globaltimer_ns() - t0 < WAIT_LIMIT_NS) {
+  }
+}
+
+__global__ void __launch_bounds__(DENSE_THREADS, 1)
+    k_attn_dense(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUtensorMap mV,
+                 DenseParams P) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = align1024(smem_raw);
+  DenseBars *b = reinterpret_cast<DenseBars *>(smem + REGION);
+  uint8_t *pbuf = smem;                 // P slices (PV phase)
+  uint8_t *vbuf = smem + P_BYTES;       // V slices (PV phase)
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+
+  const DenseTile tile = P.tiles[blockIdx.x];
+  const int g = tile.group;
+  const int tok0 = tile.tok0;
+  const int n_valid = min(TM, P.group_tok_start[g + 1] - tok0);
+  const int r0 = P.group_row_start[g];
+  const int d = P.group_rows[g];
+  const int d16 = (d + 15) & ~15;       // N of the S product
+  const int d32 = (d + 31) & ~31;       // K extent of the PV product
+  const int n_kc = P.d_in / CK;
+  const int n_vc = d32 / V_ROWS;
+  const int k_boxes = (d + 63) / 64;    // 64-row TMA boxes per K_t slice
+  const int v_boxes = P.d_emb / 64;     // 64-column TMA boxes per V slice
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S_STAGES; ++s) {
+      mbar_init(&b->xfull[s], 2);
+      mbar_init(&b->kfull[s], 1);
+      mbar_init(&b->sempty[s], 1);
+    }
+    mbar_init(&b->sfull, 1);
+    mbar_init(&b->pready, 4);
+    mbar_init(&b->ofull, 1);
+    for (int i = 0; i < V_BUFS; ++i) {
+      mbar_init(&b->vfull[i], 1);
+      mbar_init(&b->vconv[i], 4);
+      mbar_init(&b->vempty[i], 1);
+    }
+    mbar_init(&b->drain, 1);
+    b->abort_flag = 0;
+    fence_mbar_init();
+    prefetch_tensormap(&mK);
+    prefetch_tensormap(&mV);
+  }
+  if (warp == 1) {
+    tmem_alloc(&b->tmem_base, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = b->tmem_base;
+  const Abort ab{&b->abort_flag, P.err};
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (elect_one()) {
+      bool ok = true;
+      bool armed[S_STAGES] = {false, false};
+      uint32_t armed_par[S_STAGES] = {0, 0};
+      for (int kc = 0; kc < n_kc; ++kc) {
+        const int s = kc % S_STAGES;
+        const uint32_t ph = (kc / S_STAGES) & 1;
+        if (!mbar_wait(&b->sempty[s], ph ^ 1, ab)) {
+          ok = false;
+          break;
+        }
+        uint8_t *kdst = smem + s * S_STAGE + X_BYTES;
+        mbar_arrive_expect_tx(&b->kfull[s], k_boxes * 64 * 128);
+        armed[s] = true;
+        armed_par[s] = ph;
+        for (int bx = 0; bx < k_boxes; ++bx)
+          tma_load_2d(kdst + bx * 64 * 128, &mK, &b->kfull[s], kc * CK, r0 + bx * 64);
+      }
+      // V slices go where the S ring was: wait until every S-phase MMA is done
+      if (ok) ok = mbar_wait(&b->sfull, 0, ab);
+      bool varmed[V_BUFS] = {false, false};
+      uint32_t varmed_par[V_BUFS] = {0, 0};
+      for (int vc = 0; ok && vc < n_vc; ++vc) {
+        const int i = vc % V_BUFS;
+        const uint32_t ph = (vc / V_BUFS) & 1;
+        if (!mbar_wait(&b->vempty[i], ph ^ 1, ab)) {
+          ok = false;
+          break;
+        }
+        uint8_t *vdst = vbuf + i * V_BYTES;
+        mbar_arrive_expect_tx(&b->vfull[i], v_boxes * V_BLOCK);
+        varmed[i] = true;
+        varmed_par[i] = ph;
+        for (int bx = 0; bx < v_boxes; ++bx)
+          tma_load_2d(vdst + bx * V_BLOCK, &mV, &b->vfull[i], bx * 64, r0 + vc * V_ROWS);
+      }
+      if (!ok) {
+        for (int s = 0; s < S_STAGES; ++s)
+          if (armed[s]) spin_bounded(&b->kfull[s], armed_par[s]);
+        for (int i = 0; i < V_BUFS; ++i)
+          if (varmed[i]) spin_bounded(&b->vfull[i], varmed_par[i]);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (elect_one()) {
+      bool ok = true;
+      const int n_half = d16 > 256 ? 2 : 1;
+      const uint32_t id_s0 = idesc_f16(1, 0, TM, d16 > 256 ? 256 : d16);
+      const uint32_t id_s1 = idesc_f16(1, 0, TM, d16 > 256 ? d16 - 256 : 16);
+      for (int kc = 0; ok && kc < n_kc; ++kc) {
+        const int s = kc % S_STAGES;
+        const uint32_t ph = (kc / S_STAGES) & 1;
+        if (!mbar_wait(&b->xfull[s], ph, ab) || !mbar_wait(&b->kfull[s], ph, ab)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t xa = smem_u32(smem + s * S_STAGE);
+        const uint32_t ka = xa + X_BYTES;
+#pragma unroll
+        for (int k = 0; k < CK / 16; ++k) {
+          const uint64_t adesc = sdesc_sw128(xa + k * 32, 16, 1024);
+          umma_f16(tmem, adesc, sdesc_sw128(ka + k * 32, 16, 1024), id_s0, (kc | k) != 0);
+          if (n_half == 2)
+            umma_f16(tmem + 256, adesc, sdesc_sw128(ka + 256 * 128 + k * 32, 16, 1024), id_s1,
+                     (kc | k) != 0);
+        }
+        umma_commit(&b->sempty[s]);
+      }
+      if (ok) umma_commit(&b->sfull);
+      // P V_t into the TMEM columns S used, once the softmax warps have read S
+      if (ok) ok = mbar_wait(&b->pready, 0, ab);
+      if (ok) {
+        tc_fence_after();
+        const int o_half = P.d_emb > 256 ? 2 : 1;
+        const uint32_t id_o0 = idesc_f16(0, 1, TM, P.d_emb > 256 ? 256 : P.d_emb);
+        const uint32_t id_o1 = idesc_f16(0, 1, TM, P.d_emb > 256 ? P.d_emb - 256 : 16);
+        const uint32_t pa = smem_u32(pbuf);
+        for (int vc = 0; ok && vc < n_vc; ++vc) {
+          const int i = vc % V_BUFS;
+          const uint32_t ph = (vc / V_BUFS) & 1;
+          if (!mbar_wait(&b->vconv[i], ph, ab)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t va = smem_u32(vbuf + i * V_BYTES);
+#pragma unroll
+          for (int s2 = 0; s2 < V_ROWS / 16; ++s2) {
+            const int kk = vc * V_ROWS + s2 * 16;  // column of P / row of V_t
+            const uint64_t adesc =
+                sdesc_sw128(pa + (kk / 64) * (TM * 128) + (kk % 64) * 2, 16, 1024);
+            const uint32_t vrow = va + s2 * 16 * 128;
+            umma_f16(tmem, adesc, sdesc_sw128(vrow, V_BLOCK, 1024), id_o0, (vc | s2) != 0);
+            if (o_half == 2)
+              umma_f16(tmem + 256, adesc, sdesc_sw128(vrow + 4 * V_BLOCK, V_BLOCK, 1024), id_o1,
+                       (vc | s2) != 0);
+          }
+          umma_commit(&b->vempty[i]);
+        }
+        if (ok) umma_commit(&b->ofull);
+      }
+      if (!ok) {
+        umma_commit(&b->drain);
+        spin_bounded(&b->drain, 0);
+      }
+    }
+  } else if (warp < 4) {
+    // ------------------------------------------------------------ x-row gather
+    const int t = (warp - 2) * 32 + lane;  // 0..63, rows t and t + 64
+    int64_t src_row[2];
+    bool valid[2];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int r = t + u * 64;
+      valid[u] = r < n_valid;
+      src_row[u] = valid[u] ? (int64_t)P.perm[tok0 + r] * P.d_in : 0;
+    }
+    for (int kc = 0; kc < n_kc; ++kc) {
+      const int s = kc % S_STAGES;
+      const uint32_t ph = (kc / S_STAGES) & 1;
+      if (!__all_sync(0xffffffffu, mbar_wait(&b->sempty[s], ph ^ 1, ab))) break;
+      uint8_t *xdst = smem + s * S_STAGE;
+      uint4 v[2][8];
+#pragma unroll
+      for (int u = 0; u < 2; ++u)
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          v[u][j] = valid[u] ? *reinterpret_cast<const uint4 *>(P.x + src_row[u] + kc * CK + j * 8)
+                             : make_uint4(0, 0, 0, 0);
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const int r = t + u * 64;
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          *reinterpret_cast<uint4 *>(xdst + r * 128 + ((j ^ (r & 7)) << 4)) = v[u][j];
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&b->xfull[s]);
+    }
+  } else {
+    // ------------------------------------------------------------ softmax, V convert, epilogue
+    const int q = warp & 3;
+    const int r = q * 32 + lane;
+    const uint32_t trow = tmem + ((uint32_t)(q * 32) << 16);
+    float inv_sum = 0.f;
+    bool ok = __all_sync(0xffffffffu, mbar_wait(&b->sfull, 0, ab));
+    if (ok) {
+      tc_fence_after();
+      float m = -INFINITY;
+      for (int c = 0; c < d32; c += 32) {
+        uint32_t v[32];
+        tmem_ld32(trow + c, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          if (c + j < d) m = fmaxf(m, __uint_as_float(v[j]));
+      }
+      const float mb = m * LOG2E;
+      float sum = 0.f;
+      for (int c = 0; c < d32; c += 32) {
+        uint32_t v[32];
+        tmem_ld32(trow + c, v);
+        tmem_wait_ld();
+        // 32 columns -> four 16-byte chunks of the 128-byte swizzled P row
+        uint8_t *prow = pbuf + (c / 64) * (TM * 128) + r * 128;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          uint4 o;
+          __half2 *o2 = reinterpret_cast<__half2 *>(&o);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int col = c + j * 8 + 2 * e;
+            const float p0 = col < d ? exp2f(fmaf(__uint_as_float(v[j * 8 + 2 * e]), LOG2E, -mb)) : 0.f;
+            const float p1 =
+                col + 1 < d ? exp2f(fmaf(__uint_as_float(v[j * 8 + 2 * e + 1]), LOG2E, -mb)) : 0.f;
+            const __half2 hp = __floats2half2_rn(p0, p1);
+            // the sum uses the rounded values the MMA will see
+            const float2 hf = __half22float2(hp);
+            sum += hf.x + hf.y;
+            o2[e] = hp;
+          }
+          const int chunk = ((c % 64) / 8) + j;  // 16-byte chunk index within the row
+          *reinterpret_cast<uint4 *>(prow + ((chunk ^ (r & 7)) << 4)) = o;
+        }
+      }
+      inv_sum = 1.0f / sum;
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0 && ok) mbar_arrive(&b->pready);
+
+    // V slices: bf16 -> fp16 in place, then hand them to the MMA warp
+    const int eth = (warp - 4) * 32 + lane;  // 0..127
+    const int v_vecs = V_ROWS * P.d_emb / 8;
+    for (int vc = 0; ok && vc < n_vc; ++vc) {
+      const int i = vc % V_BUFS;
+      const uint32_t ph = (vc / V_BUFS) & 1;
+      ok = __all_sync(0xffffffffu, mbar_wait(&b->vfull[i], ph, ab));
+      if (!ok) break;
+      uint4 *vb = reinterpret_cast<uint4 *>(vbuf + i * V_BYTES);
+      bool bad = false;
+      for (int e = eth; e < v_vecs; e += 128) {
+        uint4 w = vb[e];
+        const __nv_bfloat162 *in = reinterpret_cast<const __nv_bfloat162 *>(&w);
+        uint4 o;
+        __half2 *out = reinterpret_cast<__half2 *>(&o);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float2 f = __bfloat1622float2(in[k]);
+          bad |= fabsf(f.x) > 65504.f || fabsf(f.y) > 65504.f;
+          out[k] = __floats2half2_rn(f.x, f.y);
+        }
+        vb[e] = o;
+      }
+      if (bad) atomicOr(P.err, DEV_ERR_F16_RANGE);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&b->vconv[i]);
+    }
+
+    // epilogue: a = O / rowsum, fp16, to the token's original position
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&b->ofull, 0, ab));
+    if (ok) {
+      tc_fence_after();
+      __half *arow = P.a + (r < n_valid ? (int64_t)P.perm[tok0 + r] * P.d_emb : 0);
+      for (int c = 0; c < P.d_emb; c += 32) {
+        uint32_t v[32];
+        tmem_ld32(trow + c, v);
+        tmem_wait_ld();
+        if (r < n_valid) {
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            uint4 o;
+            __half2 *o2 = reinterpret_cast<__half2 *>(&o);
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              o2[e] = __floats2half2_rn(__uint_as_float(v[j * 8 + 2 * e]) * inv_sum,
+                                        __uint_as_float(v[j * 8 + 2 * e + 1]) * inv_sum);
+            *reinterpret_cast<uint4 *>(arow + c + j * 8) = o;
+          }
+        }
+      }
+    }
+  }
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+constexpr size_t DENSE_SMEM = 1024 + REGION + sizeof(DenseBars);
+
+}  // namespace
+
+bool dense_attention_supported(const l3_dims_t &d) {
+  return d.dtype == L3_BF16 && d.d_in % CK == 0 && d.d_emb % 64 == 0 && d.d_emb <= MAX_EMB;
+}
+int dense_attention_max_rows() { return MAX_D; }
+
+l3_status launch_attn_dense(const l3_plan_s *p, const void *x, const void *W_K, const void *W_V,
+                            cudaStream_t s) {
+  if (p->n_dense_tiles == 0) return L3_OK;
+  const l3_dims_t &d = p->dims;
+  CUtensorMap mK, mV;
+  l3_status st;
+  if ((st = make_map_2d16(&mK, W_K, true, d.v, d.d_in, d.d_in, 64, 64)) != L3_OK) return st;
+  if ((st = make_map_2d16(&mV, W_V, true, d.v, d.d_emb, d.d_emb, 64, V_ROWS)) != L3_OK) return st;
+  DenseParams P;
+  P.x = reinterpret_cast<const __nv_bfloat16 *>(x);
+  P.a = reinterpret_cast<__half *>(p->a_buf);
+  P.perm = p->perm;
+  P.group_tok_start = p->group_tok_start;
+  P.group_row_start = p->group_row_start;
+  P.group_rows = p->group_rows;
+  P.tiles = p->dense_tiles;
+  P.d_in = (int)d.d_in;
+  P.d_emb = (int)d.d_emb;
+  P.err = p->dev_flags + 1;
+  static bool attr[64] = {};
+  if (!attr[p->device & 63]) {
+    L3_CUDA_TRY(cudaFuncSetAttribute(k_attn_dense, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)DENSE_SMEM));
+    attr[p->device & 63] = true;
+  }
+  LaunchTimer t("attn_dense", s);
+  k_attn_dense<<<(unsigned)p->n_dense_tiles, DENSE_THREADS, DENSE_SMEM, s>>>(mK, mV, P);
+  L3_CUDA_TRY(cudaGetLastError());
+  return L3_OK;
+}
+
+}  // namespace l3

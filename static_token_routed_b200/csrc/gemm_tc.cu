@@ -548,6 +548,26 @@ constexpr size_t UP_SMEM =
 
 }  // namespace
 
+l3_status make_map_2d16(CUtensorMap *m, const void *base, bool bf16, uint64_t rows, uint64_t cols,
+                        uint64_t ld, uint32_t box_cols, uint32_t box_rows) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc;
+  l3_status st = encoder(&enc);
+  if (st != L3_OK) return st;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {ld * 2};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
+                   const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    set_error("cuTensorMapEncodeTiled failed (code " + std::to_string((int)r) + ")");
+    return L3_ERR_CUDA;
+  }
+  return L3_OK;
+}
+
 bool tc_gemm_supported(const l3_dims_t &d) {
   return d.dtype == L3_BF16 && d.d_in % BK == 0 && d.d_emb % BK == 0 && d.d_up % BK == 0 &&
          d.d_up <= 8 * BN;

@@ -59,6 +59,10 @@ struct TailItem {
 
 constexpr int TAIL_TOKENS = 8;     // tokens per tail work item
 constexpr int DENSE_TILE_M = 128;  // tokens per dense tile
+// a group runs on the tensor-core attention kernel when it has at least this
+// many tokens and rows (and d_t fits the kernel); otherwise on CUDA cores
+constexpr int DENSE_MIN_TOKENS = 16;
+constexpr int DENSE_MIN_ROWS = 16;
 
 }  // namespace l3
 
@@ -108,6 +112,12 @@ size_t plan_scratch_bytes(int64_t n_tokens);
 // attention, CUDA-core path (attn_tail.cu)
 l3_status launch_attn_tail(const l3_plan_s *p, const void *x, const void *W_K, const void *W_V,
                            cudaStream_t s);
+
+// attention, tensor-core path (attn_dense.cu)
+bool dense_attention_supported(const l3_dims_t &d);
+int dense_attention_max_rows();
+l3_status launch_attn_dense(const l3_plan_s *p, const void *x, const void *W_K, const void *W_V,
+                            cudaStream_t s);
 
 // GEMMs + LayerNorm, tensor-core path (gemm_tc.cu)
 bool tc_gemm_supported(const l3_dims_t &d);

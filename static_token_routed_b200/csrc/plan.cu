@@ -225,7 +225,7 @@ __global__ void k_group_fill(const int32_t *__restrict__ sorted, const int32_t *
 
 __global__ void k_item_counts(const int32_t *__restrict__ group_tok_start,
                               const int32_t *__restrict__ group_rows, int64_t cap,
-                              int dense_min_tokens, int dense_min_rows,
+                              int dense_min_tokens, int dense_min_rows, int dense_max_rows,
                               int32_t *__restrict__ tiles, int32_t *__restrict__ tails,
                               int32_t *info) {
   int64_t g = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
@@ -235,7 +235,8 @@ __global__ void k_item_counts(const int32_t *__restrict__ group_tok_start,
   if (g < G) {
     int32_t c = group_tok_start[g + 1] - group_tok_start[g];
     int32_t rows = group_rows[g];
-    bool dense = dense_min_tokens > 0 && c >= dense_min_tokens && rows >= dense_min_rows;
+    bool dense = dense_min_tokens > 0 && c >= dense_min_tokens && rows >= dense_min_rows &&
+                 rows <= dense_max_rows;
     if (dense) {
       nt = (c + DENSE_TILE_M - 1) / DENSE_TILE_M;
       atomicAdd(&info[INFO_DENSE_GROUPS], 1);
@@ -374,12 +375,18 @@ l3_status build_plan(l3_plan_s *p, const int32_t *ids, const int32_t *offsets, c
       LaunchTimer t("plan_scan", s);
       k_scan_exclusive<<<1, SCAN_THREADS, 0, s>>>(p->group_rows, p->seg_rows, n, &info[INFO_ROWS]);
     }
-    int dense_min_tokens = 0, dense_min_rows = 0;  // tensor-core attention not wired yet
+    // groups with enough tokens and rows go to the tensor-core attention kernel
+    int dense_min_tokens = 0, dense_min_rows = 0, dense_max_rows = 0;
+    if (dense_attention_supported(p->dims)) {
+      dense_min_tokens = DENSE_MIN_TOKENS;
+      dense_min_rows = DENSE_MIN_ROWS;
+      dense_max_rows = dense_attention_max_rows();
+    }
     {
       LaunchTimer t("plan_item_counts", s);
       k_item_counts<<<blocks_for(cap, 256), 256, 0, s>>>(p->group_tok_start, p->group_rows, n,
-                                                         dense_min_tokens, dense_min_rows, tiles,
-                                                         tails, info);
+                                                         dense_min_tokens, dense_min_rows,
+                                                         dense_max_rows, tiles, tails, info);
     }
     {
       LaunchTimer t("plan_scan", s);

@@ -116,3 +116,38 @@ def test_tensor_core_kernels_run():
     kernels = l3.l3_profile_read()
     l3.l3_profile_enable(False)
     assert "mix_gemm_tc" in kernels and "up_ln_gemm_tc" in kernels, kernels
+
+
+@pytest.mark.parametrize("vocab,d_t,n,d_in,d_emb,d_up,d_out", [
+    (5, 37, 300, 128, 64, 64, 64),      # d_t not a multiple of 16, partial token tiles
+    (3, 300, 400, 64, 192, 128, 48),    # two N halves for S, PV N = 192
+    (4, 512, 700, 128, 512, 256, 64),   # d_t = 512 fills TMEM, two PV halves
+    (6, 16, 140, 64, 128, 64, 16),      # smallest dense group
+])
+def test_dense_attention_shapes(vocab, d_t, n, d_in, d_emb, d_up, d_out):
+    """Groups on the tensor-core attention kernel, ragged in tokens and d_t."""
+    g = torch.Generator().manual_seed(d_t)
+    off = torch.arange(0, vocab + 1, dtype=torch.int32) * d_t
+    v = vocab * d_t
+    ids = torch.randint(0, vocab, (n,), generator=g, dtype=torch.int32)
+    mk = lambda *s: (torch.randn(*s, generator=g) / s[-1] ** 0.5).to(torch.bfloat16)
+    # larger logits than the workloads' so the softmax is far from uniform
+    t = wl.Tables(off, mk(v, d_in) * 4, mk(v, d_emb), mk(d_up, d_emb),
+                  (1 + 0.1 * torch.randn(d_up, generator=g)).to(torch.bfloat16),
+                  (0.1 * torch.randn(d_up, generator=g)).to(torch.bfloat16), mk(d_out, d_up + d_in))
+    bt = wl.Batch(ids, mk(n, d_in) * 4)
+    dims = l3.make_dims(vocab, v, d_t, d_in, d_emb, d_up, d_out, torch.bfloat16, EPS)
+    dev = to_device(t, bt)
+    plan = l3.l3_plan(dev["ids"], dev["offsets"], dims)
+    assert plan.info().n_dense_tiles > 0
+    y = torch.empty(n, d_out, dtype=torch.bfloat16, device="cuda")
+    l3.l3_profile_enable(True)
+    l3.l3_forward(dev["x"], plan, dev["W_K"], dev["W_V"], dev["W_up"], dev["ln_gamma"],
+                  dev["ln_beta"], dev["W_mix"], y)
+    l3.l3_forward_status(plan)
+    kernels = l3.l3_profile_read()
+    l3.l3_profile_enable(False)
+    assert "attn_dense" in kernels
+    want = oracle_y(t, bt)
+    err = rel_max_err(y.double().cpu().numpy(), want)
+    assert err <= TOL["bf16"], err
