@@ -43,6 +43,27 @@ cudaEvent_t take_event() {
 
 std::once_flag g_pool_once[64];
 
+// Per-device helper stream and events that let the two attention kernels
+// (CUDA-core tail, tensor-core dense) run side by side: they write disjoint
+// rows of a, and the tail's small CTAs fit next to a dense CTA on an SM.
+struct Aux {
+  std::mutex mu;
+  cudaStream_t stream = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+};
+Aux g_aux[64];
+
+l3_status aux_for(int device, Aux **out) {
+  Aux &a = g_aux[device & 63];
+  if (!a.stream) {
+    L3_CUDA_TRY(cudaStreamCreateWithFlags(&a.stream, cudaStreamNonBlocking));
+    L3_CUDA_TRY(cudaEventCreateWithFlags(&a.fork, cudaEventDisableTiming));
+    L3_CUDA_TRY(cudaEventCreateWithFlags(&a.join, cudaEventDisableTiming));
+  }
+  *out = &a;
+  return L3_OK;
+}
+
 // Keep freed plan memory in the device's stream-ordered pool, so a plan per
 // batch costs no driver allocation after the first.
 void keep_pool_warm(int device) {
@@ -302,10 +323,29 @@ l3_status l3_forward(const void *x, l3_plan_t p, const void *W_K, const void *W_
   }
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   p->stream = s;
-  l3_status st = launch_attn_tail(p, x, W_K, W_V, s);
-  if (st == L3_OK) st = launch_attn_dense(p, x, W_K, W_V, s);
+  l3_status st = L3_OK;
+  if (p->n_dense_tiles > 0 && p->n_tail_items > 0) {
+    // fork: tail attention and the fp16 weight copies on the helper stream,
+    // dense attention on the caller's stream; join before W_up
+    Aux *aux = nullptr;
+    if ((st = aux_for(p->device, &aux)) != L3_OK) return st;
+    std::lock_guard<std::mutex> lk(aux->mu);
+    L3_CUDA_TRY(cudaEventRecord(aux->fork, s));
+    L3_CUDA_TRY(cudaStreamWaitEvent(aux->stream, aux->fork, 0));
+    if (p->tc_gemm) st = launch_weights_f16(p, W_up, W_mix, aux->stream);
+    if (st == L3_OK)
+      st = tail_cls_supported(p->dims) ? launch_attn_tail_cls(p, x, W_K, W_V, aux->stream)
+                                       : launch_attn_tail(p, x, W_K, W_V, aux->stream);
+    if (st == L3_OK) st = launch_attn_dense(p, x, W_K, W_V, s);
+    L3_CUDA_TRY(cudaEventRecord(aux->join, aux->stream));
+    L3_CUDA_TRY(cudaStreamWaitEvent(s, aux->join, 0));
+  } else {
+    st = tail_cls_supported(p->dims) ? launch_attn_tail_cls(p, x, W_K, W_V, s)
+                                     : launch_attn_tail(p, x, W_K, W_V, s);
+    if (st == L3_OK) st = launch_attn_dense(p, x, W_K, W_V, s);
+    if (st == L3_OK && p->tc_gemm) st = launch_weights_f16(p, W_up, W_mix, s);
+  }
   if (p->tc_gemm) {
-    if (st == L3_OK) st = launch_weights_f16(p, W_up, W_mix, s);
     if (st == L3_OK) st = launch_up_ln_tc(p, ln_gamma, ln_beta, s);
     if (st == L3_OK) st = launch_mix_tc(p, x, W_mix, y, s);
   } else {

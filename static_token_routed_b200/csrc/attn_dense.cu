@@ -11,16 +11,19 @@
 //
 // One CTA takes one 128-token tile of one group:
 //   - warps 2-3 gather the tile's x rows (through the sort permutation) into
-//     128-byte-swizzled shared memory, 64 columns at a time;
-//   - warp 0 streams the matching 64-column slices of K_t with TMA;
+//     64-byte-swizzled shared memory with cp.async, 32 columns at a time and
+//     several slices ahead;
+//   - warp 0 streams the matching 32-column slices of K_t with TMA, as many
+//     slices in flight as the shared-memory ring holds for this d_t;
 //   - warp 1 issues tcgen05.mma (M = 128 tokens, N = d_t up to 2 x 256) so that
 //     S accumulates in TMEM over d_in;
-//   - warps 4-7 (one token row per thread, the TMEM lane it owns) take an exact
-//     row max and the exponentials, and write P as fp16 into shared memory;
-//   - warp 0 then streams V_t in 32-row slices with TMA, warps 4-7 turn each
+//   - warps 4-11 (two per TMEM lane quarter, so two threads per token row,
+//     each with half of the row's columns) take an exact row max and the
+//     exponentials, and write P as fp16 into shared memory;
+//   - warp 0 then streams V_t in 16-row slices with TMA, warps 4-11 turn each
 //     slice into fp16 in place, and warp 1 accumulates O = P V_t in the TMEM
 //     columns S no longer needs;
-//   - warps 4-7 scale O by 1 / rowsum and store a[perm[i]] (fp16), i.e. already
+//   - warps 4-11 scale O by 1 / rowsum and store a[perm[i]] (fp16), i.e. already
 //     in the caller's token order.
 // K_t and V_t are read from HBM by the group's first tile; its other tiles run
 // at the same time and find them in L2.
@@ -35,38 +38,34 @@
 namespace l3 {
 
 l3_status make_map_2d16(CUtensorMap *m, const void *base, bool bf16, uint64_t rows, uint64_t cols,
-                        uint64_t ld, uint32_t box_cols, uint32_t box_rows);
+                        uint64_t ld, uint32_t box_cols, uint32_t box_rows, int swizzle_bytes);
 
 namespace {
 
 using namespace sm100;
 
 constexpr int TM = 128;                 // tokens per tile
-constexpr int CK = 64;                  // d_in columns per S-phase slice
+constexpr int CK = 32;                  // d_in columns per S-phase slice (64-byte rows)
 constexpr int MAX_D = 512;              // d_t handled here (TMEM columns)
 constexpr int MAX_EMB = 512;
-constexpr int X_BYTES = TM * CK * 2;    // 16 KB
-constexpr int K_BYTES = MAX_D * CK * 2; // 64 KB
-constexpr int S_STAGE = X_BYTES + K_BYTES;
-constexpr int S_STAGES = 2;
-constexpr int P_BYTES = TM * MAX_D * 2;                 // 128 KB, 8 slices of 64 columns
-constexpr int V_ROWS = 32;                              // d_t rows per V slice
-constexpr int V_BLOCK = V_ROWS * 128;                   // one 64-column block of a V slice
-constexpr int V_BYTES = V_ROWS * MAX_EMB * 2;           // 32 KB
-constexpr int V_BUFS = 2;
-constexpr int REGION = (S_STAGES * S_STAGE > P_BYTES + V_BUFS * V_BYTES)
-                           ? S_STAGES * S_STAGE
-                           : P_BYTES + V_BUFS * V_BYTES;  // 192 KB
-constexpr int DENSE_THREADS = 256;
+constexpr int X_BYTES = TM * CK * 2;    // 8 KB
+constexpr int REGION = 192 * 1024;      // S-phase ring, later P + V slices
+constexpr int MAX_STAGES = 8;
+constexpr int V_ROWS = 16;              // d_t rows per V slice (one MMA k-step)
+constexpr int V_BLOCK = V_ROWS * 128;   // one 64-column block of a V slice
+constexpr int DENSE_THREADS = 384;  // 0 TMA, 1 MMA, 2-3 x gather, 4-11 softmax / epilogue
+constexpr int SOFTMAX_THREADS = 256;
 constexpr float LOG2E = 1.4426950408889634f;
 
 struct DenseBars {
-  uint64_t xfull[S_STAGES], kfull[S_STAGES], sempty[S_STAGES];
+  uint64_t xfull[MAX_STAGES], kfull[MAX_STAGES], sempty[MAX_STAGES];
   uint64_t sfull, pready, ofull;
-  uint64_t vfull[V_BUFS], vconv[V_BUFS], vempty[V_BUFS];
+  uint64_t vfull[MAX_STAGES], vconv[MAX_STAGES], vempty[MAX_STAGES];
   uint64_t drain;
   uint32_t tmem_base;
   int abort_flag;
+  float red_max[2][128];  // per row: max of each half of the columns
+  float red_sum[2][128];
 };
 
 struct DenseParams {
@@ -85,6 +84,52 @@ __device__ __forceinline__ uint8_t *align1024(uint8_t *p) {
   return reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
 }
 
+// K-major operand with 64-byte rows (32 16-bit elements), 64-byte swizzle:
+// 8-row groups 512 bytes apart.
+__device__ __forceinline__ uint64_t sdesc_sw64(uint32_t smem_addr) {
+  return (uint64_t)((smem_addr >> 4) & 0x3FFFu) | (1ull << 16) | ((uint64_t)(512 >> 4) << 32) |
+         (1ull << 46) | (4ull << 61);
+}
+
+__device__ __forceinline__ void cp_async16_zfill(void *dst, const void *src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src),
+               "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.wait_group 0;" ::: "memory");
+}
+// wait until at most `lag` committed groups of this thread are still in flight
+__device__ __forceinline__ void cp_async_wait_group_lag(int lag) {
+  switch (lag) {
+    case 0: asm volatile("cp.async.wait_group 0;" ::: "memory"); break;
+    case 1: asm volatile("cp.async.wait_group 1;" ::: "memory"); break;
+    case 2: asm volatile("cp.async.wait_group 2;" ::: "memory"); break;
+    case 3: asm volatile("cp.async.wait_group 3;" ::: "memory"); break;
+    case 4: asm volatile("cp.async.wait_group 4;" ::: "memory"); break;
+    case 5: asm volatile("cp.async.wait_group 5;" ::: "memory"); break;
+    case 6: asm volatile("cp.async.wait_group 6;" ::: "memory"); break;
+    default: asm volatile("cp.async.wait_group 7;" ::: "memory"); break;
+  }
+}
+
+// barrier of the 256 softmax / epilogue threads that ANDs a flag across them
+__device__ __forceinline__ bool softmax_sync_and(bool ok) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 q, %1, 0;\n\t"
+      "bar.red.and.pred p, 1, %2, q;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(r)
+      : "r"((uint32_t)ok), "n"(SOFTMAX_THREADS)
+      : "memory");
+  return r != 0;
+}
+
 __device__ __forceinline__ void spin_bounded(uint64_t *bar, uint32_t parity) {
   const uint32_t a = smem_u32(bar);
   const uint64_t t0 = globaltimer_ns();
@@ -98,8 +143,6 @@ __global__ void __launch_bounds__(DENSE_THREADS, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = align1024(smem_raw);
   DenseBars *b = reinterpret_cast<DenseBars *>(smem + REGION);
-  uint8_t *pbuf = smem;                 // P slices (PV phase)
-  uint8_t *vbuf = smem + P_BYTES;       // V slices (PV phase)
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
 
   const DenseTile tile = P.tiles[blockIdx.x];
@@ -108,25 +151,35 @@ __global__ void __launch_bounds__(DENSE_THREADS, 1)
   const int n_valid = min(TM, P.group_tok_start[g + 1] - tok0);
   const int r0 = P.group_row_start[g];
   const int d = P.group_rows[g];
-  const int d16 = (d + 15) & ~15;       // N of the S product
-  const int d32 = (d + 31) & ~31;       // K extent of the PV product
+  const int d16 = (d + 15) & ~15;       // N of the S product, K extent of the PV product
+  const int d32 = (d + 31) & ~31;       // softmax works in 32-column TMEM loads
+  const int d64 = (d + 63) & ~63;
   const int n_kc = P.d_in / CK;
-  const int n_vc = d32 / V_ROWS;
-  const int k_boxes = (d + 63) / 64;    // 64-row TMA boxes per K_t slice
+  const int n_vc = d16 / V_ROWS;
+  const int k_boxes = d64 / 64;         // 64-row TMA boxes per K_t slice
   const int v_boxes = P.d_emb / 64;     // 64-column TMA boxes per V slice
+  // pipeline depth follows from d_t: the S ring holds as many slices as fit,
+  // and so do the V buffers after P
+  const int s_stage = X_BYTES + d64 * CK * 2;
+  const int n_s = min(MAX_STAGES, REGION / s_stage);
+  const int p_bytes = (d64 / 64) * (TM * 128);
+  const int v_bytes = V_ROWS * P.d_emb * 2;
+  const int n_v = min(MAX_STAGES, (REGION - p_bytes) / v_bytes);
+  uint8_t *pbuf = smem;                 // P slices (PV phase)
+  uint8_t *vbuf = smem + p_bytes;       // V slices (PV phase)
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < S_STAGES; ++s) {
+    for (int s = 0; s < MAX_STAGES; ++s) {
       mbar_init(&b->xfull[s], 2);
       mbar_init(&b->kfull[s], 1);
       mbar_init(&b->sempty[s], 1);
     }
     mbar_init(&b->sfull, 1);
-    mbar_init(&b->pready, 4);
+    mbar_init(&b->pready, 8);
     mbar_init(&b->ofull, 1);
-    for (int i = 0; i < V_BUFS; ++i) {
+    for (int i = 0; i < MAX_STAGES; ++i) {
       mbar_init(&b->vfull[i], 1);
-      mbar_init(&b->vconv[i], 4);
+      mbar_init(&b->vconv[i], 8);
       mbar_init(&b->vempty[i], 1);
     }
     mbar_init(&b->drain, 1);
@@ -149,34 +202,36 @@ __global__ void __launch_bounds__(DENSE_THREADS, 1)
     // ------------------------------------------------------------ TMA producer
     if (elect_one()) {
       bool ok = true;
-      bool armed[S_STAGES] = {false, false};
-      uint32_t armed_par[S_STAGES] = {0, 0};
+      bool armed[MAX_STAGES];
+      uint32_t armed_par[MAX_STAGES];
+      for (int i = 0; i < MAX_STAGES; ++i) armed[i] = false;
       for (int kc = 0; kc < n_kc; ++kc) {
-        const int s = kc % S_STAGES;
-        const uint32_t ph = (kc / S_STAGES) & 1;
+        const int s = kc % n_s;
+        const uint32_t ph = (kc / n_s) & 1;
         if (!mbar_wait(&b->sempty[s], ph ^ 1, ab)) {
           ok = false;
           break;
         }
-        uint8_t *kdst = smem + s * S_STAGE + X_BYTES;
-        mbar_arrive_expect_tx(&b->kfull[s], k_boxes * 64 * 128);
+        uint8_t *kdst = smem + s * s_stage + X_BYTES;
+        mbar_arrive_expect_tx(&b->kfull[s], k_boxes * 64 * CK * 2);
         armed[s] = true;
         armed_par[s] = ph;
         for (int bx = 0; bx < k_boxes; ++bx)
-          tma_load_2d(kdst + bx * 64 * 128, &mK, &b->kfull[s], kc * CK, r0 + bx * 64);
+          tma_load_2d(kdst + bx * 64 * CK * 2, &mK, &b->kfull[s], kc * CK, r0 + bx * 64);
       }
       // V slices go where the S ring was: wait until every S-phase MMA is done
       if (ok) ok = mbar_wait(&b->sfull, 0, ab);
-      bool varmed[V_BUFS] = {false, false};
-      uint32_t varmed_par[V_BUFS] = {0, 0};
+      bool varmed[MAX_STAGES];
+      uint32_t varmed_par[MAX_STAGES];
+      for (int i = 0; i < MAX_STAGES; ++i) varmed[i] = false;
       for (int vc = 0; ok && vc < n_vc; ++vc) {
-        const int i = vc % V_BUFS;
-        const uint32_t ph = (vc / V_BUFS) & 1;
+        const int i = vc % n_v;
+        const uint32_t ph = (vc / n_v) & 1;
         if (!mbar_wait(&b->vempty[i], ph ^ 1, ab)) {
           ok = false;
           break;
         }
-        uint8_t *vdst = vbuf + i * V_BYTES;
+        uint8_t *vdst = vbuf + i * v_bytes;
         mbar_arrive_expect_tx(&b->vfull[i], v_boxes * V_BLOCK);
         varmed[i] = true;
         varmed_par[i] = ph;
@@ -184,9 +239,9 @@ __global__ void __launch_bounds__(DENSE_THREADS, 1)
           tma_load_2d(vdst + bx * V_BLOCK, &mV, &b->vfull[i], bx * 64, r0 + vc * V_ROWS);
       }
       if (!ok) {
-        for (int s = 0; s < S_STAGES; ++s)
+        for (int s = 0; s < MAX_STAGES; ++s)
           if (armed[s]) spin_bounded(&b->kfull[s], armed_par[s]);
-        for (int i = 0; i < V_BUFS; ++i)
+        for (int i = 0; i < MAX_STAGES; ++i)
           if (varmed[i]) spin_bounded(&b->vfull[i], varmed_par[i]);
       }
     }
@@ -198,21 +253,21 @@ __global__ void __launch_bounds__(DENSE_THREADS, 1)
       const uint32_t id_s0 = idesc_f16(1, 0, TM, d16 > 256 ? 256 : d16);
       const uint32_t id_s1 = idesc_f16(1, 0, TM, d16 > 256 ? d16 - 256 : 16);
       for (int kc = 0; ok && kc < n_kc; ++kc) {
-        const int s = kc % S_STAGES;
-        const uint32_t ph = (kc / S_STAGES) & 1;
+        const int s = kc % n_s;
+        const uint32_t ph = (kc / n_s) & 1;
         if (!mbar_wait(&b->xfull[s], ph, ab) || !mbar_wait(&b->kfull[s], ph, ab)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint32_t xa = smem_u32(smem + s * S_STAGE);
+        const uint32_t xa = smem_u32(smem + s * s_stage);
         const uint32_t ka = xa + X_BYTES;
 #pragma unroll
         for (int k = 0; k < CK / 16; ++k) {
-          const uint64_t adesc = sdesc_sw128(xa + k * 32, 16, 1024);
-          umma_f16(tmem, adesc, sdesc_sw128(ka + k * 32, 16, 1024), id_s0, (kc | k) != 0);
+          const uint64_t adesc = sdesc_sw64(xa + k * 32);
+          umma_f16(tmem, adesc, sdesc_sw64(ka + k * 32), id_s0, (kc | k) != 0);
           if (n_half == 2)
-            umma_f16(tmem + 256, adesc, sdesc_sw128(ka + 256 * 128 + k * 32, 16, 1024), id_s1,
+            umma_f16(tmem + 256, adesc, sdesc_sw64(ka + 256 * CK * 2 + k * 32), id_s1,
                      (kc | k) != 0);
         }
         umma_commit(&b->sempty[s]);
@@ -227,25 +282,20 @@ __global__ void __launch_bounds__(DENSE_THREADS, 1)
         const uint32_t id_o1 = idesc_f16(0, 1, TM, P.d_emb > 256 ? P.d_emb - 256 : 16);
         const uint32_t pa = smem_u32(pbuf);
         for (int vc = 0; ok && vc < n_vc; ++vc) {
-          const int i = vc % V_BUFS;
-          const uint32_t ph = (vc / V_BUFS) & 1;
+          const int i = vc % n_v;
+          const uint32_t ph = (vc / n_v) & 1;
           if (!mbar_wait(&b->vconv[i], ph, ab)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t va = smem_u32(vbuf + i * V_BYTES);
-#pragma unroll
-          for (int s2 = 0; s2 < V_ROWS / 16; ++s2) {
-            const int kk = vc * V_ROWS + s2 * 16;  // column of P / row of V_t
-            const uint64_t adesc =
-                sdesc_sw128(pa + (kk / 64) * (TM * 128) + (kk % 64) * 2, 16, 1024);
-            const uint32_t vrow = va + s2 * 16 * 128;
-            umma_f16(tmem, adesc, sdesc_sw128(vrow, V_BLOCK, 1024), id_o0, (vc | s2) != 0);
-            if (o_half == 2)
-              umma_f16(tmem + 256, adesc, sdesc_sw128(vrow + 4 * V_BLOCK, V_BLOCK, 1024), id_o1,
-                       (vc | s2) != 0);
-          }
+          const uint32_t va = smem_u32(vbuf + i * v_bytes);
+          const int kk = vc * V_ROWS;  // column of P / row of V_t
+          const uint64_t adesc = sdesc_sw128(pa + (kk / 64) * (TM * 128) + (kk % 64) * 2, 16, 1024);
+          umma_f16(tmem, adesc, sdesc_sw128(va, V_BLOCK, 1024), id_o0, vc != 0);
+          if (o_half == 2)
+            umma_f16(tmem + 256, adesc, sdesc_sw128(va + 4 * V_BLOCK, V_BLOCK, 1024), id_o1,
+                     vc != 0);
           umma_commit(&b->vempty[i]);
         }
         if (ok) umma_commit(&b->ofull);
@@ -257,49 +307,71 @@ __global__ void __launch_bounds__(DENSE_THREADS, 1)
     }
   } else if (warp < 4) {
     // ------------------------------------------------------------ x-row gather
+    // cp.async copies (16 bytes each, zero-filled past the group's tokens),
+    // up to n_s - 1 slices ahead; a slice is handed to the MMA warp once this
+    // thread's copies for it have landed and been made visible to the async proxy.
     const int t = (warp - 2) * 32 + lane;  // 0..63, rows t and t + 64
-    int64_t src_row[2];
-    bool valid[2];
+    const __nv_bfloat16 *src_row[2];
+    uint32_t src_bytes[2];
 #pragma unroll
     for (int u = 0; u < 2; ++u) {
       const int r = t + u * 64;
-      valid[u] = r < n_valid;
-      src_row[u] = valid[u] ? (int64_t)P.perm[tok0 + r] * P.d_in : 0;
+      const bool valid = r < n_valid;
+      src_row[u] = P.x + (valid ? (int64_t)P.perm[tok0 + r] * P.d_in : 0);
+      src_bytes[u] = valid ? 16u : 0u;
     }
+    const int lag = n_s - 1;
+    bool ok = true;
+    int issued = 0, done = 0;
     for (int kc = 0; kc < n_kc; ++kc) {
-      const int s = kc % S_STAGES;
-      const uint32_t ph = (kc / S_STAGES) & 1;
-      if (!__all_sync(0xffffffffu, mbar_wait(&b->sempty[s], ph ^ 1, ab))) break;
-      uint8_t *xdst = smem + s * S_STAGE;
-      uint4 v[2][8];
-#pragma unroll
-      for (int u = 0; u < 2; ++u)
-#pragma unroll
-        for (int j = 0; j < 8; ++j)
-          v[u][j] = valid[u] ? *reinterpret_cast<const uint4 *>(P.x + src_row[u] + kc * CK + j * 8)
-                             : make_uint4(0, 0, 0, 0);
+      const int s = kc % n_s;
+      const uint32_t ph = (kc / n_s) & 1;
+      ok = __all_sync(0xffffffffu, mbar_wait(&b->sempty[s], ph ^ 1, ab));
+      if (!ok) break;
+      uint8_t *xdst = smem + s * s_stage;
+      // 64-byte rows; the 64-byte swizzle XORs the 16-byte chunk index with
+      // bits 1-2 of the row
 #pragma unroll
       for (int u = 0; u < 2; ++u) {
         const int r = t + u * 64;
 #pragma unroll
-        for (int j = 0; j < 8; ++j)
-          *reinterpret_cast<uint4 *>(xdst + r * 128 + ((j ^ (r & 7)) << 4)) = v[u][j];
+        for (int j = 0; j < 4; ++j)
+          cp_async16_zfill(xdst + r * 64 + ((j ^ ((r >> 1) & 3)) << 4), src_row[u] + kc * CK + j * 8,
+                           src_bytes[u]);
       }
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&b->xfull[s]);
+      cp_async_commit();
+      ++issued;
+      if (issued - done > lag) {
+        cp_async_wait_group_lag(lag);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&b->xfull[done % n_s]);
+        ++done;
+      }
     }
+    // the last slices, and on a give-up every copy still in flight
+    cp_async_wait_all();
+    fence_proxy_async_smem();
+    __syncwarp();
+    for (; ok && done < issued; ++done)
+      if (lane == 0) mbar_arrive(&b->xfull[done % n_s]);
   } else {
     // ------------------------------------------------------------ softmax, V convert, epilogue
+    // warps 4-11: two warps per TMEM lane quarter, each taking every other
+    // 32-column slice of the row; row max and row sum combine through shared
+    // memory at barriers of these 256 threads
+    const int sw = warp - 4;  // 0..7
     const int q = warp & 3;
+    const int half = sw / 4;
     const int r = q * 32 + lane;
     const uint32_t trow = tmem + ((uint32_t)(q * 32) << 16);
     float inv_sum = 0.f;
     bool ok = __all_sync(0xffffffffu, mbar_wait(&b->sfull, 0, ab));
+    ok = softmax_sync_and(ok);
     if (ok) {
       tc_fence_after();
       float m = -INFINITY;
-      for (int c = 0; c < d32; c += 32) {
+      for (int c = half * 32; c < d32; c += 64) {
         uint32_t v[32];
         tmem_ld32(trow + c, v);
         tmem_wait_ld();
@@ -307,9 +379,13 @@ __global__ void __launch_bounds__(DENSE_THREADS, 1)
         for (int j = 0; j < 32; ++j)
           if (c + j < d) m = fmaxf(m, __uint_as_float(v[j]));
       }
-      const float mb = m * LOG2E;
+      b->red_max[half][r] = m;
+    }
+    ok = softmax_sync_and(ok);
+    if (ok) {
+      const float m = fmaxf(b->red_max[0][r], b->red_max[1][r]);
       float sum = 0.f;
-      for (int c = 0; c < d32; c += 32) {
+      for (int c = half * 32; c < d32; c += 64) {
         uint32_t v[32];
         tmem_ld32(trow + c, v);
         tmem_wait_ld();
@@ -322,9 +398,8 @@ __global__ void __launch_bounds__(DENSE_THREADS, 1)
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const int col = c + j * 8 + 2 * e;
-            const float p0 = col < d ? exp2f(fmaf(__uint_as_float(v[j * 8 + 2 * e]), LOG2E, -mb)) : 0.f;
-            const float p1 =
-                col + 1 < d ? exp2f(fmaf(__uint_as_float(v[j * 8 + 2 * e + 1]), LOG2E, -mb)) : 0.f;
+            const float p0 = col < d ? __expf(__uint_as_float(v[j * 8 + 2 * e]) - m) : 0.f;
+            const float p1 = col + 1 < d ? __expf(__uint_as_float(v[j * 8 + 2 * e + 1]) - m) : 0.f;
             const __half2 hp = __floats2half2_rn(p0, p1);
             // the sum uses the rounded values the MMA will see
             const float2 hf = __half22float2(hp);
@@ -335,24 +410,26 @@ __global__ void __launch_bounds__(DENSE_THREADS, 1)
           *reinterpret_cast<uint4 *>(prow + ((chunk ^ (r & 7)) << 4)) = o;
         }
       }
-      inv_sum = 1.0f / sum;
+      b->red_sum[half][r] = sum;
     }
     fence_proxy_async_smem();
     tc_fence_before();
     __syncwarp();
     if (lane == 0 && ok) mbar_arrive(&b->pready);
+    ok = softmax_sync_and(ok);
+    if (ok) inv_sum = 1.0f / (b->red_sum[0][r] + b->red_sum[1][r]);
 
     // V slices: bf16 -> fp16 in place, then hand them to the MMA warp
-    const int eth = (warp - 4) * 32 + lane;  // 0..127
+    const int eth = sw * 32 + lane;  // 0..255
     const int v_vecs = V_ROWS * P.d_emb / 8;
     for (int vc = 0; ok && vc < n_vc; ++vc) {
-      const int i = vc % V_BUFS;
-      const uint32_t ph = (vc / V_BUFS) & 1;
+      const int i = vc % n_v;
+      const uint32_t ph = (vc / n_v) & 1;
       ok = __all_sync(0xffffffffu, mbar_wait(&b->vfull[i], ph, ab));
       if (!ok) break;
-      uint4 *vb = reinterpret_cast<uint4 *>(vbuf + i * V_BYTES);
+      uint4 *vb = reinterpret_cast<uint4 *>(vbuf + i * v_bytes);
       bool bad = false;
-      for (int e = eth; e < v_vecs; e += 128) {
+      for (int e = eth; e < v_vecs; e += 256) {
         uint4 w = vb[e];
         const __nv_bfloat162 *in = reinterpret_cast<const __nv_bfloat162 *>(&w);
         uint4 o;
@@ -376,7 +453,7 @@ __global__ void __launch_bounds__(DENSE_THREADS, 1)
     if (ok) {
       tc_fence_after();
       __half *arow = P.a + (r < n_valid ? (int64_t)P.perm[tok0 + r] * P.d_emb : 0);
-      for (int c = 0; c < P.d_emb; c += 32) {
+      for (int c = half * 32; c < P.d_emb; c += 64) {
         uint32_t v[32];
         tmem_ld32(trow + c, v);
         tmem_wait_ld();
@@ -419,8 +496,9 @@ l3_status launch_attn_dense(const l3_plan_s *p, const void *x, const void *W_K, 
   const l3_dims_t &d = p->dims;
   CUtensorMap mK, mV;
   l3_status st;
-  if ((st = make_map_2d16(&mK, W_K, true, d.v, d.d_in, d.d_in, 64, 64)) != L3_OK) return st;
-  if ((st = make_map_2d16(&mV, W_V, true, d.v, d.d_emb, d.d_emb, 64, V_ROWS)) != L3_OK) return st;
+  if ((st = make_map_2d16(&mK, W_K, true, d.v, d.d_in, d.d_in, CK, 64, 64)) != L3_OK) return st;
+  if ((st = make_map_2d16(&mV, W_V, true, d.v, d.d_emb, d.d_emb, 64, V_ROWS, 128)) != L3_OK)
+    return st;
   DenseParams P;
   P.x = reinterpret_cast<const __nv_bfloat16 *>(x);
   P.a = reinterpret_cast<__half *>(p->a_buf);

@@ -82,10 +82,6 @@ struct TailParams {
   const uint4 *W_K;    // [v][d_in / VEC]
   const uint4 *W_V;    // [v][d_emb / VEC]
   uint4 *a;            // [N][d_emb / VEC]
-  const int32_t *perm;
-  const int32_t *group_tok_start;
-  const int32_t *group_row_start;
-  const int32_t *group_rows;
   const TailItem *items;
   int nv_in;   // 16-byte vectors per x / K row
   int nv_emb;  // 16-byte vectors per V / a row
@@ -114,11 +110,9 @@ __global__ void __launch_bounds__(TAIL_THREADS) k_attn_tail(TailParams P) {
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
 
   const TailItem item = P.items[blockIdx.x];
-  const int g = item.group;
-  const int tok0 = item.tok0;
-  const int nt = min(TB, P.group_tok_start[g + 1] - tok0);
-  const int64_t r0 = P.group_row_start[g];
-  const int d = P.group_rows[g];
+  const int nt = item.nt;
+  const int64_t r0 = item.r0;
+  const int d = item.d;
 
   const size_t xs_bytes = (size_t)TB * P.nv_in * 16;
   const size_t red_bytes = (size_t)P.red_rows * TB * P.nv_emb * VEC * sizeof(float);
@@ -128,7 +122,7 @@ __global__ void __launch_bounds__(TAIL_THREADS) k_attn_tail(TailParams P) {
   float *inv_sum = logit + (size_t)TB * P.k_cap;
 
   __shared__ int32_t tok_index[TB];
-  if (tid < TB) tok_index[tid] = tid < nt ? P.perm[tok0 + tid] : 0;
+  if (tid < TB) tok_index[tid] = tid < nt ? item.tok[tid] : 0;
   __syncthreads();
 
   if (d > 1) {
@@ -306,10 +300,6 @@ l3_status launch_attn_tail(const l3_plan_s *p, const void *x, const void *W_K, c
   P.W_K = reinterpret_cast<const uint4 *>(W_K);
   P.W_V = reinterpret_cast<const uint4 *>(W_V);
   P.a = reinterpret_cast<uint4 *>(p->a_buf);
-  P.perm = p->perm;
-  P.group_tok_start = p->group_tok_start;
-  P.group_row_start = p->group_row_start;
-  P.group_rows = p->group_rows;
   P.items = p->tail_items;
   P.nv_in = (int)(p->dims.d_in / vec);
   P.nv_emb = (int)(p->dims.d_emb / vec);

@@ -41,7 +41,7 @@ constexpr int A_BYTES = BM * BK * 2;
 constexpr int B_BYTES = BN * BK * 2;
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int MIX_STAGES = 4;
-constexpr int UP_STAGES = 4;
+constexpr int UP_STAGES = 2;  // two CTAs per SM: one drains its epilogue while the other computes
 constexpr int GEMM_THREADS = 192;  // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
 constexpr uint32_t IDESC_F16 = idesc_f16(0, 0, BM, BN);
 constexpr uint32_t IDESC_BF16 = idesc_f16(1, 0, BM, BN);
@@ -265,7 +265,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 // ---------------------------------------------------------------------------
 // h = LayerNorm(W_up a), one cluster of ceil(d_up / 256) CTAs per 128 tokens
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(GEMM_THREADS, 1)
+__global__ void __launch_bounds__(GEMM_THREADS, 2)
     k_up_ln_gemm(const __grid_constant__ CUtensorMap mA, const __grid_constant__ CUtensorMap mB,
                  UpParams P) {
   extern __shared__ uint8_t smem_raw[];
@@ -549,7 +549,7 @@ constexpr size_t UP_SMEM =
 }  // namespace
 
 l3_status make_map_2d16(CUtensorMap *m, const void *base, bool bf16, uint64_t rows, uint64_t cols,
-                        uint64_t ld, uint32_t box_cols, uint32_t box_rows) {
+                        uint64_t ld, uint32_t box_cols, uint32_t box_rows, int swizzle_bytes) {
   PFN_cuTensorMapEncodeTiled_v12000 enc;
   l3_status st = encoder(&enc);
   if (st != L3_OK) return st;
@@ -559,8 +559,8 @@ l3_status make_map_2d16(CUtensorMap *m, const void *base, bool bf16, uint64_t ro
   cuuint32_t estr[2] = {1, 1};
   CUresult r = enc(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
                    const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                   swizzle_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) {
     set_error("cuTensorMapEncodeTiled failed (code " + std::to_string((int)r) + ")");
     return L3_ERR_CUDA;

@@ -51,18 +51,24 @@ struct DenseTile {
   int32_t group;
   int32_t tok0;  // first sorted position of the tile
 };
-// One item of the CUDA-core attention path: up to TAIL_TOKENS tokens of a group.
-struct TailItem {
-  int32_t group;
-  int32_t tok0;
+// One item of the CUDA-core attention path: up to TAIL_TOKENS tokens of one
+// group, with everything a kernel needs to run it (no further lookups).
+struct alignas(16) TailItem {
+  int32_t r0;         // first row of K_t / V_t
+  int16_t d;          // d_t
+  int16_t nt;         // tokens in the item (1..TAIL_TOKENS)
+  int32_t tok[8];     // original indices of the tokens
+  int32_t pad[2];
 };
 
-constexpr int TAIL_TOKENS = 8;     // tokens per tail work item
+constexpr int TAIL_TOKENS = 8;     // tokens per tail work item (size of TailItem::tok)
 constexpr int DENSE_TILE_M = 128;  // tokens per dense tile
 // a group runs on the tensor-core attention kernel when it has at least this
 // many tokens and rows (and d_t fits the kernel); otherwise on CUDA cores
-constexpr int DENSE_MIN_TOKENS = 16;
-constexpr int DENSE_MIN_ROWS = 16;
+constexpr int DENSE_MIN_TOKENS = 5;
+constexpr int DENSE_MIN_ROWS = 32;
+// tail items with at most this many rows are "small" (latency-bound)
+constexpr int TAIL_SMALL_ROWS = 16;
 
 }  // namespace l3
 
@@ -79,6 +85,8 @@ struct l3_plan_s {
   int64_t unique_rows = 0;
   int64_t unique_rows_multi = 0;
   int64_t max_group_tokens = 0;
+  int64_t tail_class_start[5] = {};  // tail items of token class c are [start[c], start[c+1])
+  int64_t tail_class_split[4] = {};  // ... of which [split[c], start[c+1]) have d_t <= TAIL_SMALL_ROWS
 
   void *block = nullptr;  // the one device allocation backing everything below
   size_t block_bytes = 0;
@@ -93,7 +101,7 @@ struct l3_plan_s {
   int32_t *seg_rows = nullptr;         // [N+1]
   l3::DenseTile *dense_tiles = nullptr;
   l3::TailItem *tail_items = nullptr;
-  int32_t *dev_flags = nullptr;        // [4]: plan error bits, forward error bits
+  int32_t *dev_flags = nullptr;        // [0] plan errors, [1] forward errors, [2] work counter
   void *a_buf = nullptr;               // [N x d_emb] dtype, original token order
   void *h_buf = nullptr;               // [N x d_up] dtype
   float *z_buf = nullptr;              // [N x d_up] fp32 (CUDA-core GEMM path only)
@@ -112,6 +120,11 @@ size_t plan_scratch_bytes(int64_t n_tokens);
 // attention, CUDA-core path (attn_tail.cu)
 l3_status launch_attn_tail(const l3_plan_s *p, const void *x, const void *W_K, const void *W_V,
                            cudaStream_t s);
+
+// attention, CUDA-core path specialised by token count (attn_tail_cls.cu)
+bool tail_cls_supported(const l3_dims_t &d);
+l3_status launch_attn_tail_cls(const l3_plan_s *p, const void *x, const void *W_K,
+                               const void *W_V, cudaStream_t s);
 
 // attention, tensor-core path (attn_dense.cu)
 bool dense_attention_supported(const l3_dims_t &d);

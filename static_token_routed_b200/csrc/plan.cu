@@ -13,6 +13,7 @@
 //   permutation -> scan -> group fill -> scan of d_t -> work-item counts ->
 //   scans -> work-item fill.
 #include <algorithm>
+#include <initializer_list>
 #include <mutex>
 
 #include "l3_internal.cuh"
@@ -28,8 +29,14 @@ constexpr int SORT_ITEMS = 8;                            // per thread
 constexpr int SORT_TILE = SORT_THREADS * SORT_ITEMS;     // elements per CTA
 constexpr int WARP_SPAN = SORT_TILE / SORT_WARPS;        // contiguous elements per warp
 constexpr int SCAN_THREADS = 1024;
-constexpr int SCAN_ITEMS = 4;
+constexpr int SCAN_ITEMS = 16;
 constexpr int SCAN_CHUNK = SCAN_THREADS * SCAN_ITEMS;
+constexpr int MAX_DT_BUCKETS = 1025;  // d_t <= k <= 1024
+constexpr int N_CLASSES = 4;          // tail items with 1, 2, 3-4 and 5-8 tokens
+
+__host__ __device__ __forceinline__ int token_class(int nt) {
+  return nt <= 1 ? 0 : nt == 2 ? 1 : nt <= 4 ? 2 : 3;
+}
 
 // slots of the device info block read back at the end of l3_plan
 enum {
@@ -41,7 +48,9 @@ enum {
   INFO_ROWS_MULTI,
   INFO_DENSE_GROUPS,
   INFO_MAX_TOKENS,
-  INFO_SLOTS
+  INFO_CLS,              // 5 slots: first tail item of each token-count class, then the total
+  INFO_SPLIT = INFO_CLS + 5,  // 4 slots: first item of each class with d_t <= TAIL_SMALL_ROWS
+  INFO_SLOTS = INFO_SPLIT + 4
 };
 
 __device__ __forceinline__ uint32_t lanemask_lt() {
@@ -141,58 +150,91 @@ __global__ void __launch_bounds__(SORT_THREADS)
   }
 }
 
-// One-CTA exclusive scan: out[i] = sum in[0..i-1] for i <= n (out has n + 1
-// entries; in == out is allowed). The total also goes to *total if given.
-__global__ void __launch_bounds__(SCAN_THREADS)
-    k_scan_exclusive(const int32_t *in, int32_t *out, int64_t n, int32_t *total) {
+// Exclusive scans, one array per CTA: out[i] = sum in[0..i-1] for i <= n (out
+// has n + 1 entries; in == out is allowed: every value is read before the
+// chunk's first store); the total also goes to *total if given.
+struct ScanJob {
+  const int32_t *in;
+  int32_t *out;
+  int64_t n;
+  int32_t *total;
+};
+struct ScanJobs {
+  ScanJob job[4];
+};
+
+__global__ void __launch_bounds__(SCAN_THREADS) k_scan_multi(ScanJobs jobs) {
   __shared__ int32_t warp_sums[SCAN_THREADS / 32];
   __shared__ int32_t chunk_total;
+  // select the job without indexing the parameter array dynamically
+  ScanJob J = jobs.job[0];
+  if (blockIdx.x == 1) J = jobs.job[1];
+  if (blockIdx.x == 2) J = jobs.job[2];
+  if (blockIdx.x == 3) J = jobs.job[3];
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  // Each warp owns a contiguous segment of SCAN_ITEMS * 32 values of the chunk
+  // and walks it in rounds of 32 consecutive values (coalesced loads and
+  // stores); a round's inclusive warp scan plus the carry of earlier rounds
+  // gives the prefix inside the segment, and segment totals are scanned
+  // across warps through shared memory.
   int32_t carry = 0;
-  for (int64_t base = 0; base < n; base += SCAN_CHUNK) {
-    int32_t v[SCAN_ITEMS];
-    int32_t local = 0;
+  for (int64_t base = 0; base < J.n; base += SCAN_CHUNK) {
+    const int64_t seg = base + (int64_t)warp * (SCAN_ITEMS * 32);
+    int32_t v[SCAN_ITEMS], incl[SCAN_ITEMS];
 #pragma unroll
-    for (int j = 0; j < SCAN_ITEMS; ++j) {
-      int64_t i = base + (int64_t)threadIdx.x * SCAN_ITEMS + j;
-      v[j] = i < n ? in[i] : 0;
-      local += v[j];
+    for (int r = 0; r < SCAN_ITEMS; ++r) {
+      const int64_t i = seg + r * 32 + lane;
+      v[r] = i < J.n ? J.in[i] : 0;
     }
-    // inclusive warp scan of the per-thread sums
-    int32_t incl = local;
+    int32_t run = 0;  // sum of earlier rounds in this warp's segment
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      int32_t t = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += t;
+    for (int r = 0; r < SCAN_ITEMS; ++r) {
+      int32_t x = v[r];
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int32_t t = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += t;
+      }
+      incl[r] = x + run;
+      run += __shfl_sync(0xffffffffu, x, 31);
     }
-    if (lane == 31) warp_sums[warp] = incl;
+    if (lane == 0) warp_sums[warp] = run;
     __syncthreads();
     if (warp == 0) {
-      int32_t w = warp_sums[lane];
+      const int32_t w = warp_sums[lane];
       int32_t wi = w;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
-        int32_t t = __shfl_up_sync(0xffffffffu, wi, o);
+        const int32_t t = __shfl_up_sync(0xffffffffu, wi, o);
         if (lane >= o) wi += t;
       }
-      warp_sums[lane] = wi - w;  // exclusive prefix of warp totals
+      warp_sums[lane] = wi - w;  // exclusive prefix of segment totals
       if (lane == 31) chunk_total = wi;
     }
     __syncthreads();
-    int32_t run = carry + warp_sums[warp] + (incl - local);
+    const int32_t off = carry + warp_sums[warp];
 #pragma unroll
-    for (int j = 0; j < SCAN_ITEMS; ++j) {
-      int64_t i = base + (int64_t)threadIdx.x * SCAN_ITEMS + j;
-      if (i < n) out[i] = run;
-      run += v[j];
+    for (int r = 0; r < SCAN_ITEMS; ++r) {
+      const int64_t i = seg + r * 32 + lane;
+      if (i < J.n) J.out[i] = off + incl[r] - v[r];
     }
     carry += chunk_total;
     __syncthreads();
   }
   if (threadIdx.x == 0) {
-    out[n] = carry;
-    if (total) *total = carry;
+    J.out[J.n] = carry;
+    if (J.total) *J.total = carry;
   }
+}
+
+// launch up to four independent scans as one grid
+l3_status scan_multi(std::initializer_list<ScanJob> js, cudaStream_t s) {
+  ScanJobs jobs{};
+  int k = 0;
+  for (const ScanJob &j : js) jobs.job[k++] = j;
+  LaunchTimer t("plan_scan", s);
+  k_scan_multi<<<k, SCAN_THREADS, 0, s>>>(jobs);
+  return L3_OK;
 }
 
 // head[i] = 1 where a new ID starts in sorted order; inv_perm[perm[i]] = i.
@@ -227,7 +269,7 @@ __global__ void k_item_counts(const int32_t *__restrict__ group_tok_start,
                               const int32_t *__restrict__ group_rows, int64_t cap,
                               int dense_min_tokens, int dense_min_rows, int dense_max_rows,
                               int32_t *__restrict__ tiles, int32_t *__restrict__ tails,
-                              int32_t *info) {
+                              int32_t *__restrict__ dcount, int k_cap, int32_t *info) {
   int64_t g = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
   if (g >= cap) return;
   int32_t G = info[INFO_G];
@@ -245,23 +287,58 @@ __global__ void k_item_counts(const int32_t *__restrict__ group_tok_start,
     }
     if (rows > 1) atomicAdd(&info[INFO_ROWS_MULTI], rows);
     atomicMax(&info[INFO_MAX_TOKENS], c);
+    // tail items are listed by token-count class, then largest d_t first:
+    // bucket class * (k_cap + 1) + (k_cap - d_t), so an ascending scan gives
+    // the order
+    if (nl > 0) {
+      const int db = k_cap - min(rows, k_cap);
+      const int full = c / TAIL_TOKENS, rest = c % TAIL_TOKENS;
+      if (full > 0) atomicAdd(&dcount[token_class(TAIL_TOKENS) * (k_cap + 1) + db], full);
+      if (rest > 0) atomicAdd(&dcount[token_class(rest) * (k_cap + 1) + db], 1);
+    }
   }
   tiles[g] = nt;
   tails[g] = nl;
 }
 
 __global__ void k_item_fill(const int32_t *__restrict__ group_tok_start,
+                            const int32_t *__restrict__ group_row_start,
+                            const int32_t *__restrict__ group_rows,
+                            const int32_t *__restrict__ perm,
                             const int32_t *__restrict__ tiles, const int32_t *__restrict__ tile_off,
-                            const int32_t *__restrict__ tails, const int32_t *__restrict__ tail_off,
-                            int64_t cap, DenseTile *__restrict__ dense, TailItem *__restrict__ tail,
-                            const int32_t *info) {
+                            const int32_t *__restrict__ tails, int32_t *__restrict__ dcursor,
+                            int k_cap, int64_t cap, DenseTile *__restrict__ dense,
+                            TailItem *__restrict__ tail, const int32_t *info) {
   int64_t g = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
   if (g >= cap || g >= info[INFO_G]) return;
-  int32_t start = group_tok_start[g];
+  const int32_t start = group_tok_start[g];
+  const int32_t c = group_tok_start[g + 1] - start;
   for (int32_t j = 0; j < tiles[g]; ++j)
     dense[tile_off[g] + j] = DenseTile{(int32_t)g, start + j * DENSE_TILE_M};
-  for (int32_t j = 0; j < tails[g]; ++j)
-    tail[tail_off[g] + j] = TailItem{(int32_t)g, start + j * TAIL_TOKENS};
+  const int32_t rows = group_rows[g];
+  for (int32_t j = 0; j < tails[g]; ++j) {
+    TailItem it;
+    it.r0 = group_row_start[g];
+    it.d = (int16_t)rows;
+    it.nt = (int16_t)min(TAIL_TOKENS, c - j * TAIL_TOKENS);
+#pragma unroll
+    for (int t = 0; t < TAIL_TOKENS; ++t)
+      it.tok[t] = t < it.nt ? perm[start + j * TAIL_TOKENS + t] : 0;
+    it.pad[0] = it.pad[1] = 0;
+    // position within its bucket: any order inside a bucket gives the same results
+    const int bucket = token_class(it.nt) * (k_cap + 1) + (k_cap - min(rows, k_cap));
+    const int32_t pos = atomicAdd(&dcursor[bucket], 1);
+    tail[pos] = it;
+  }
+}
+
+// first tail item of each class (read before the fill kernel moves the cursors)
+__global__ void k_class_starts(const int32_t *__restrict__ scanned, int k_cap, int32_t *info) {
+  const int c = threadIdx.x;
+  if (c <= N_CLASSES) info[INFO_CLS + c] = scanned[c * (k_cap + 1)];
+  // buckets run from d_t = k_cap down to 1 inside a class
+  const int small = min(TAIL_SMALL_ROWS, k_cap);
+  if (c < N_CLASSES) info[INFO_SPLIT + c] = scanned[c * (k_cap + 1) + (k_cap - small)];
 }
 
 inline int blocks_for(int64_t n, int threads) { return (int)std::max<int64_t>(1, (n + threads - 1) / threads); }
@@ -277,6 +354,7 @@ size_t plan_scratch_bytes(int64_t n) {
   ints += 2 * ((size_t)n + 1);           // head flags, group positions
   ints += 4 * ((size_t)n + 1);           // tiles, tile offsets, tails, tail offsets
   ints += 64;                            // info block
+  ints += 2 * (N_CLASSES * MAX_DT_BUCKETS + 1);  // tail items per bucket, and their cursors
   return ints * sizeof(int32_t) + 256;
 }
 
@@ -307,6 +385,11 @@ l3_status build_plan(l3_plan_s *p, const int32_t *ids, const int32_t *offsets, c
   sp += cap;
   int32_t *info = sp;
   sp += 64;
+  int32_t *dcount = sp;
+  sp += N_CLASSES * MAX_DT_BUCKETS + 1;
+  int32_t *dcursor = sp;
+  sp += N_CLASSES * MAX_DT_BUCKETS + 1;
+  const int k_cap = (int)std::min<int64_t>(p->dims.k, MAX_DT_BUCKETS - 1);
   if ((size_t)((char *)sp - (char *)scratch) > scratch_bytes) {
     set_error("internal: plan scratch too small");
     return L3_ERR_INVALID_ARG;
@@ -343,10 +426,7 @@ l3_status build_plan(l3_plan_s *p, const int32_t *ids, const int32_t *offsets, c
         k_radix_hist<<<(int)n_tiles, SORT_THREADS, 0, s>>>(kin, n, shift, hist, (int)n_tiles,
                                                           pass == 0 ? vocab : 0, info);
       }
-      {
-        LaunchTimer t("plan_scan", s);
-        k_scan_exclusive<<<1, SCAN_THREADS, 0, s>>>(hist, hist, RADIX * n_tiles, nullptr);
-      }
+      scan_multi({{hist, hist, RADIX * n_tiles, nullptr}}, s);
       {
         LaunchTimer t("plan_radix_scatter", s);
         k_radix_scatter<<<(int)n_tiles, SORT_THREADS, 0, s>>>(kin, vin, kout, vout, n, shift, hist,
@@ -360,20 +440,13 @@ l3_status build_plan(l3_plan_s *p, const int32_t *ids, const int32_t *offsets, c
       k_group_heads<<<blocks_for(n, 256), 256, 0, s>>>(p->sorted_ids, p->perm, n, head,
                                                        p->inv_perm);
     }
-    {
-      LaunchTimer t("plan_scan", s);
-      k_scan_exclusive<<<1, SCAN_THREADS, 0, s>>>(head, gpos, n, &info[INFO_G]);
-    }
+    scan_multi({{head, gpos, n, &info[INFO_G]}}, s);
     L3_CUDA_TRY(cudaMemsetAsync(p->group_rows, 0, cap * sizeof(int32_t), s));
     {
       LaunchTimer t("plan_group_fill", s);
       k_group_fill<<<blocks_for(n, 256), 256, 0, s>>>(p->sorted_ids, head, gpos, n, offsets, vocab,
                                                       p->group_ids, p->group_tok_start,
                                                       p->group_row_start, p->group_rows, info);
-    }
-    {
-      LaunchTimer t("plan_scan", s);
-      k_scan_exclusive<<<1, SCAN_THREADS, 0, s>>>(p->group_rows, p->seg_rows, n, &info[INFO_ROWS]);
     }
     // groups with enough tokens and rows go to the tensor-core attention kernel
     int dense_min_tokens = 0, dense_min_rows = 0, dense_max_rows = 0;
@@ -382,25 +455,28 @@ l3_status build_plan(l3_plan_s *p, const int32_t *ids, const int32_t *offsets, c
       dense_min_rows = DENSE_MIN_ROWS;
       dense_max_rows = dense_attention_max_rows();
     }
+    const int n_buckets = N_CLASSES * (k_cap + 1);
+    L3_CUDA_TRY(cudaMemsetAsync(dcount, 0, n_buckets * sizeof(int32_t), s));
     {
       LaunchTimer t("plan_item_counts", s);
       k_item_counts<<<blocks_for(cap, 256), 256, 0, s>>>(p->group_tok_start, p->group_rows, n,
                                                          dense_min_tokens, dense_min_rows,
-                                                         dense_max_rows, tiles, tails, info);
+                                                         dense_max_rows, tiles, tails, dcount,
+                                                         k_cap, info);
     }
-    {
-      LaunchTimer t("plan_scan", s);
-      k_scan_exclusive<<<1, SCAN_THREADS, 0, s>>>(tiles, tile_off, n, &info[INFO_TILES]);
-    }
-    {
-      LaunchTimer t("plan_scan", s);
-      k_scan_exclusive<<<1, SCAN_THREADS, 0, s>>>(tails, tail_off, n, &info[INFO_TAILS]);
-    }
+    // three independent scans in one launch: d_t over groups (segment row
+    // offsets), dense tiles over groups, tail items over (class, d_t) buckets
+    scan_multi({{p->group_rows, p->seg_rows, n, &info[INFO_ROWS]},
+                {tiles, tile_off, n, &info[INFO_TILES]},
+                {dcount, dcursor, n_buckets, &info[INFO_TAILS]}},
+               s);
+    k_class_starts<<<1, 32, 0, s>>>(dcursor, k_cap, info);
     {
       LaunchTimer t("plan_item_fill", s);
-      k_item_fill<<<blocks_for(n, 256), 256, 0, s>>>(p->group_tok_start, tiles, tile_off, tails,
-                                                     tail_off, n, p->dense_tiles, p->tail_items,
-                                                     info);
+      k_item_fill<<<blocks_for(n, 256), 256, 0, s>>>(p->group_tok_start, p->group_row_start,
+                                                     p->group_rows, p->perm, tiles, tile_off,
+                                                     tails, dcursor, k_cap, n, p->dense_tiles,
+                                                     p->tail_items, info);
     }
   } else {
     L3_CUDA_TRY(cudaMemsetAsync(p->group_tok_start, 0, sizeof(int32_t), s));
@@ -426,6 +502,10 @@ l3_status build_plan(l3_plan_s *p, const int32_t *ids, const int32_t *offsets, c
   p->unique_rows_multi = host_info[INFO_ROWS_MULTI];
   p->n_dense_groups = host_info[INFO_DENSE_GROUPS];
   p->max_group_tokens = host_info[INFO_MAX_TOKENS];
+  for (int c = 0; c <= N_CLASSES; ++c)
+    p->tail_class_start[c] = n > 0 ? host_info[INFO_CLS + c] : 0;
+  for (int c = 0; c < N_CLASSES; ++c)
+    p->tail_class_split[c] = n > 0 ? host_info[INFO_SPLIT + c] : 0;
   return L3_OK;
 }
 
@@ -531,7 +611,11 @@ extern "C" l3_status l3_sort_tokens_noalloc(const int32_t *token_ids, int64_t n_
     int32_t *vout = vbuf[(pass + 1) % 2];
     k_radix_hist<<<(int)n_tiles, SORT_THREADS, 0, s>>>(kin, n, shift, hist, (int)n_tiles, 0,
                                                       nullptr);
-    k_scan_exclusive<<<1, SCAN_THREADS, 0, s>>>(hist, hist, RADIX * n_tiles, nullptr);
+    {
+      ScanJobs jobs{};
+      jobs.job[0] = ScanJob{hist, hist, RADIX * n_tiles, nullptr};
+      k_scan_multi<<<1, SCAN_THREADS, 0, s>>>(jobs);
+    }
     k_radix_scatter<<<(int)n_tiles, SORT_THREADS, 0, s>>>(kin, vin, kout, vout, n, shift, hist,
                                                          (int)n_tiles);
     kin = kout;

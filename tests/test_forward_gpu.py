@@ -122,7 +122,8 @@ def test_tensor_core_kernels_run():
     (5, 37, 300, 128, 64, 64, 64),      # d_t not a multiple of 16, partial token tiles
     (3, 300, 400, 64, 192, 128, 48),    # two N halves for S, PV N = 192
     (4, 512, 700, 128, 512, 256, 64),   # d_t = 512 fills TMEM, two PV halves
-    (6, 16, 140, 64, 128, 64, 16),      # smallest dense group
+    (6, 32, 140, 64, 128, 64, 16),      # smallest dense d_t
+    (9, 40, 45, 128, 64, 64, 32),       # groups of ~5 tokens: the fewest that go dense
 ])
 def test_dense_attention_shapes(vocab, d_t, n, d_in, d_emb, d_up, d_out):
     """Groups on the tensor-core attention kernel, ragged in tokens and d_t."""
