@@ -202,8 +202,9 @@ l3_status l3_sort_tokens_noalloc(const int32_t *token_ids, int64_t n_tokens, int
  * error, L3_OK otherwise. */
 l3_status l3_forward_status(l3_plan_t plan);
 
-/* Frees the plan's device buffers (stream-ordered on the plan's last
- * stream). NULL is a no-op. */
+/* Releases the plan. Its device memory returns to a small per-process cache
+ * (at most four blocks, reused by later plans once the work last enqueued on
+ * the plan's stream has finished; older blocks are freed). NULL is a no-op. */
 void l3_plan_destroy(l3_plan_t plan);
 
 /* Message for the last error on the calling thread ("" if none). */

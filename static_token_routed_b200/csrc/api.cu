@@ -41,7 +41,6 @@ cudaEvent_t take_event() {
   return e;
 }
 
-std::once_flag g_pool_once[64];
 
 // Per-device helper stream and events that let the two attention kernels
 // (CUDA-core tail, tensor-core dense) run side by side: they write disjoint
@@ -64,17 +63,63 @@ l3_status aux_for(int device, Aux **out) {
   return L3_OK;
 }
 
-// Keep freed plan memory in the device's stream-ordered pool, so a plan per
-// batch costs no driver allocation after the first.
-void keep_pool_warm(int device) {
-  if (device < 0 || device >= 64) return;
-  std::call_once(g_pool_once[device], [device] {
-    cudaMemPool_t pool;
-    if (cudaDeviceGetDefaultMemPool(&pool, device) == cudaSuccess) {
-      uint64_t threshold = UINT64_MAX;
-      cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &threshold);
-    }
-  });
+// Plan memory cache. A destroyed plan's block goes back to a per-process list
+// with an event recorded on the stream that last used it; a new plan takes a
+// cached block on its device that is large enough and whose event has
+// completed, so a plan per batch costs no allocator call after warm-up, and a
+// plan built on one stream while an earlier forward still runs on another
+// never waits for it or grows the pool.
+struct CachedBlock {
+  void *ptr;
+  size_t bytes;
+  int device;
+  cudaEvent_t ready;
+};
+std::mutex g_cache_mu;
+std::vector<CachedBlock> g_cache;
+constexpr size_t CACHE_MAX_BLOCKS = 4;
+
+// returns a cached block of at least `bytes` on `device` (and its size), or nullptr
+void *cache_take(int device, size_t bytes, size_t *got) {
+  std::lock_guard<std::mutex> lk(g_cache_mu);
+  int best = -1;
+  for (int i = 0; i < (int)g_cache.size(); ++i) {
+    const CachedBlock &c = g_cache[i];
+    if (c.device != device || c.bytes < bytes) continue;
+    if (cudaEventQuery(c.ready) != cudaSuccess) continue;  // still in use on the GPU
+    if (best < 0 || c.bytes < g_cache[best].bytes) best = i;
+  }
+  if (best < 0) return nullptr;
+  void *p = g_cache[best].ptr;
+  *got = g_cache[best].bytes;
+  cudaEventDestroy(g_cache[best].ready);
+  g_cache.erase(g_cache.begin() + best);
+  return p;
+}
+
+void cache_give(void *ptr, size_t bytes, int device, cudaStream_t s) {
+  cudaEvent_t ev = nullptr;
+  if (cudaEventCreateWithFlags(&ev, cudaEventDisableTiming) != cudaSuccess ||
+      cudaEventRecord(ev, s) != cudaSuccess) {
+    if (ev) cudaEventDestroy(ev);
+    cudaStreamSynchronize(s);
+    cudaFree(ptr);
+    return;
+  }
+  std::lock_guard<std::mutex> lk(g_cache_mu);
+  g_cache.push_back(CachedBlock{ptr, bytes, device, ev});
+  while (g_cache.size() > CACHE_MAX_BLOCKS) {
+    // drop the oldest block once its last user has finished
+    CachedBlock old = g_cache.front();
+    g_cache.erase(g_cache.begin());
+    cudaEventSynchronize(old.ready);
+    cudaEventDestroy(old.ready);
+    int cur = -1;
+    cudaGetDevice(&cur);
+    if (cur != old.device) cudaSetDevice(old.device);
+    cudaFree(old.ptr);
+    if (cur != old.device) cudaSetDevice(cur);
+  }
 }
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -180,7 +225,6 @@ l3_status l3_plan(const int32_t *token_ids, int64_t n_tokens, const int32_t *off
   p->n_tokens = n_tokens;
   p->stream = s;
   L3_CUDA_TRY(cudaGetDevice(&p->device));
-  keep_pool_warm(p->device);
 
   const int64_t n = n_tokens, cap = n + 1;
   const size_t el = dims->dtype == L3_BF16 ? 2 : 4;
@@ -206,12 +250,19 @@ l3_status l3_plan(const int32_t *token_ids, int64_t n_tokens, const int32_t *off
   };
   size_t total = 0;
   for (size_t b : sizes) total += b;
-  cudaError_t e = cudaMallocAsync(&p->block, total, s);
-  if (e != cudaSuccess) {
-    delete p;
-    return cuda_fail(e, "cudaMallocAsync(plan)");
+  size_t got = 0;
+  p->block = cache_take(p->device, total, &got);
+  cudaError_t e = cudaSuccess;
+  if (p->block) {
+    p->block_bytes = got;  // a cached block keeps its size for its next owner
+  } else {
+    e = cudaMalloc(&p->block, total);
+    if (e != cudaSuccess) {
+      delete p;
+      return cuda_fail(e, "cudaMalloc(plan)");
+    }
+    p->block_bytes = total;
   }
-  p->block_bytes = total;
   char *c = reinterpret_cast<char *>(p->block);
   size_t i = 0;
   auto next = [&](size_t k) {
@@ -243,7 +294,7 @@ l3_status l3_plan(const int32_t *token_ids, int64_t n_tokens, const int32_t *off
   if (st == L3_OK) st = build_plan(p, token_ids, offsets, s, scratch, sizes[14]);
   if (st != L3_OK) {
     std::string msg = g_error;
-    cudaFreeAsync(p->block, s);
+    cache_give(p->block, p->block_bytes, p->device, s);
     delete p;
     g_error = msg;
     return st;
@@ -378,7 +429,7 @@ l3_status l3_forward_status(l3_plan_t p) {
 
 void l3_plan_destroy(l3_plan_t p) {
   if (!p) return;
-  if (p->block) cudaFreeAsync(p->block, p->stream);
+  if (p->block) cache_give(p->block, p->block_bytes, p->device, p->stream);
   delete p;
 }
 
