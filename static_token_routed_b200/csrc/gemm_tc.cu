@@ -265,7 +265,23 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 // ---------------------------------------------------------------------------
 // h = LayerNorm(W_up a), one cluster of ceil(d_up / 256) CTAs per 128 tokens
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(GEMM_THREADS, 2)
+constexpr int UP_THREADS = 320;  // warp 0 TMA, warp 1 MMA, warps 2-9 epilogue
+
+// barrier of the 256 epilogue threads of k_up_ln_gemm that ANDs a flag across them
+__device__ __forceinline__ bool epi_sync_and(bool ok) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 q, %1, 0;\n\t"
+      "bar.red.and.pred p, 1, 256, q;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(r)
+      : "r"((uint32_t)ok)
+      : "memory");
+  return r != 0;
+}
+
+__global__ void __launch_bounds__(UP_THREADS, 2)
     k_up_ln_gemm(const __grid_constant__ CUtensorMap mA, const __grid_constant__ CUtensorMap mB,
                  UpParams P) {
   extern __shared__ uint8_t smem_raw[];
@@ -276,6 +292,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2)
   float *b_s = g_s + BN;                          // beta
   float *st_mean = b_s + BN;                      // per-row mean of this CTA's slice
   float *st_m2 = st_mean + BM;                    // per-row sum of squared deviations
+  float(*red)[BM] = reinterpret_cast<float(*)[BM]>(st_m2 + BM);  // [2][BM] halves of a row
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const uint32_t rank = cluster_ctarank();
   const uint32_t n_ranks = gridDim.x;  // one cluster spans the grid's x dimension
@@ -299,7 +316,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2)
     tmem_alloc(&b->tmem_base, BN);
     tmem_relinquish();
   }
-  for (int i = threadIdx.x; i < BN; i += GEMM_THREADS) {
+  for (int i = threadIdx.x; i < BN; i += UP_THREADS) {
     const bool v = n0 + i < P.N;
     g_s[i] = v ? __bfloat162float(P.gamma[n0 + i]) : 0.f;
     b_s[i] = v ? __bfloat162float(P.beta[n0 + i]) : 0.f;
@@ -364,20 +381,24 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2)
     }
   }
 
-  // epilogue part 1: per-row mean and M2 of this CTA's slice
+  // epilogue part 1: per-row mean and M2 of this CTA's slice. Warps 2-9, two
+  // per TMEM lane quarter; each takes every other 32-column chunk, and the two
+  // halves of a row combine through shared memory.
   const bool epi = warp >= 2;
   const int q = warp & 3;
+  const int half = (warp - 2) / 4;
   const int r = q * 32 + lane;
   const uint32_t trow = tmem + ((uint32_t)(q * 32) << 16);
   bool have = false;
   __syncwarp();
   if (epi) {
     have = __all_sync(0xffffffffu, mbar_wait(&b->tfull[0], 0, ab));
+    have = epi_sync_and(have);
     tc_fence_after();
     float sum = 0.f;
     if (have) {
 #pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
+      for (int c = half; c < BN / 32; c += 2) {
         uint32_t v[32];
         tmem_ld32(trow + c * 32, v);
         tmem_wait_ld();
@@ -386,11 +407,13 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2)
           if (c * 32 + j < n_valid) sum += __uint_as_float(v[j]);
       }
     }
-    const float mean = sum / (float)n_valid;
+    red[half][r] = sum;
+    epi_sync_and(true);
+    const float mean = (red[0][r] + red[1][r]) / (float)n_valid;
     float m2 = 0.f;
     if (have) {
 #pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
+      for (int c = half; c < BN / 32; c += 2) {
         uint32_t v[32];
         tmem_ld32(trow + c * 32, v);
         tmem_wait_ld();
@@ -402,20 +425,35 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2)
           }
       }
     }
-    st_mean[r] = mean;
-    st_m2[r] = m2;
+    epi_sync_and(true);  // both halves have read red[.][r] (the sums)
+    red[half][r] = m2;
+    epi_sync_and(true);
+    if (half == 0) {
+      st_mean[r] = mean;
+      st_m2[r] = red[0][r] + red[1][r];
+    }
   }
   __syncwarp();
   cluster_sync();  // every CTA's (mean, M2) is visible cluster-wide
 
   float mu = 0.f, rstd = 0.f;
   if (epi) {
-    // merge the slices in rank order: n_a, mean_a, M2_a  (+)  n_b, mean_b, M2_b
+    // all slices' statistics first (independent remote loads in flight
+    // together), then merge in rank order: n_a, mean_a, M2_a (+) n_b, mean_b, M2_b
+    float mbv[8], qbv[8];
+#pragma unroll
+    for (uint32_t j = 0; j < 8; ++j)
+      if (j < n_ranks) {
+        mbv[j] = ld_shared_cluster_f32(map_shared_rank(&st_mean[r], j));
+        qbv[j] = ld_shared_cluster_f32(map_shared_rank(&st_m2[r], j));
+      }
     float n_acc = 0.f, mean_acc = 0.f, m2_acc = 0.f;
-    for (uint32_t j = 0; j < n_ranks; ++j) {
+#pragma unroll
+    for (uint32_t j = 0; j < 8; ++j) {
+      if (j >= n_ranks) break;
       const float nb = (float)min(BN, P.N - (int)j * BN);
-      const float mb = ld_shared_cluster_f32(map_shared_rank(&st_mean[r], j));
-      const float qb = ld_shared_cluster_f32(map_shared_rank(&st_m2[r], j));
+      const float mb = mbv[j];
+      const float qb = qbv[j];
       const float n_new = n_acc + nb;
       const float delta = mb - mean_acc;
       mean_acc += delta * (nb / n_new);
@@ -431,7 +469,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2)
     const int m = m0 + r;
     __half *hrow = P.h + (int64_t)m * P.N + n0;
 #pragma unroll 1
-    for (int c = 0; c < BN / 32; ++c) {
+    for (int c = half; c < BN / 32; c += 2) {
       uint32_t v[32];
       tmem_ld32(trow + c * 32, v);
       tmem_wait_ld();
@@ -544,7 +582,7 @@ int num_sms() {
 
 constexpr size_t MIX_SMEM = 1024 + MIX_STAGES * STAGE_BYTES + sizeof(Bars);
 constexpr size_t UP_SMEM =
-    1024 + UP_STAGES * STAGE_BYTES + sizeof(Bars) + (2 * BN + 2 * BM) * sizeof(float);
+    1024 + UP_STAGES * STAGE_BYTES + sizeof(Bars) + (2 * BN + 4 * BM) * sizeof(float);
 
 }  // namespace
 
@@ -619,7 +657,7 @@ l3_status launch_up_ln_tc(const l3_plan_s *p, const void *gamma, const void *bet
   const int cn = (int)((d.d_up + BN - 1) / BN);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(cn, (unsigned)((p->n_tokens + BM - 1) / BM), 1);
-  cfg.blockDim = dim3(GEMM_THREADS, 1, 1);
+  cfg.blockDim = dim3(UP_THREADS, 1, 1);
   cfg.dynamicSmemBytes = UP_SMEM;
   cfg.stream = s;
   cudaLaunchAttribute at[1];
