@@ -27,6 +27,8 @@
 //     in the caller's token order.
 // K_t and V_t are read from HBM by the group's first tile; its other tiles run
 // at the same time and find them in L2.
+// Groups with d_t <= 256 run in a second launch with half the shared memory
+// and TMEM per CTA (two CTAs per SM), O then computed in 256-column passes.
 // P and V_t meet in fp16 (10-bit mantissa): tcgen05 kind::f16 needs one type
 // for both operands, and a bf16 P would cost as much accuracy as a bf16 a.
 #include <cuda_fp16.h>
@@ -49,8 +51,21 @@ constexpr int CK = 32;                  // d_in columns per S-phase slice (64-by
 constexpr int MAX_D = 512;              // d_t handled here (TMEM columns)
 constexpr int MAX_EMB = 512;
 constexpr int X_BYTES = TM * CK * 2;    // 8 KB
-constexpr int REGION = 192 * 1024;      // S-phase ring, later P + V slices
 constexpr int MAX_STAGES = 8;
+
+// Two launch configurations. The big one holds S for d_t up to 512 (all 512
+// TMEM columns, 192 KB of shared memory: one CTA per SM). The small one takes
+// groups with d_t <= 256 in half of both, so two CTAs share an SM and twice as
+// many K_t / x bytes are in flight; with d_emb > 256 it computes O in
+// 256-column passes through the same TMEM columns.
+template <bool SMALL>
+struct DenseCfg {
+  static constexpr int REGION = SMALL ? 96 * 1024 : 192 * 1024;  // S ring, later P + V slices
+  static constexpr int TMEM_COLS = SMALL ? 256 : 512;
+  static constexpr int MAX_ROWS = SMALL ? 256 : MAX_D;
+  static constexpr int MIN_BLOCKS = SMALL ? 2 : 1;
+};
+static_assert(DenseCfg<true>::MAX_ROWS == DENSE_SMALL_ROWS, "plan and kernel disagree on small d_t");
 constexpr int V_ROWS = 16;              // d_t rows per V slice (one MMA k-step)
 constexpr int V_BLOCK = V_ROWS * 128;   // one 64-column block of a V slice
 constexpr int DENSE_THREADS = 384;  // 0 TMA, 1 MMA, 2-3 x gather, 4-11 softmax / epilogue
@@ -61,6 +76,7 @@ struct DenseBars {
   uint64_t xfull[MAX_STAGES], kfull[MAX_STAGES], sempty[MAX_STAGES];
   uint64_t sfull, pready, ofull;
   uint64_t vfull[MAX_STAGES], vconv[MAX_STAGES], vempty[MAX_STAGES];
+  uint64_t odrained;  // the epilogue has read this O pass out of TMEM
   uint64_t drain;
   uint32_t tmem_base;
   int abort_flag;
@@ -137,9 +153,12 @@ __device__ __forceinline__ void spin_bounded(uint64_t *bar, uint32_t parity) {
   }
 }
 
-__global__ void __launch_bounds__(DENSE_THREADS, 1)
+template <bool SMALL>
+__global__ void __launch_bounds__(DENSE_THREADS, DenseCfg<SMALL>::MIN_BLOCKS)
     k_attn_dense(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUtensorMap mV,
                  DenseParams P) {
+  using Cfg = DenseCfg<SMALL>;
+  constexpr int REGION = Cfg::REGION;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = align1024(smem_raw);
   DenseBars *b = reinterpret_cast<DenseBars *>(smem + REGION);
@@ -157,13 +176,16 @@ __global__ void __launch_bounds__(DENSE_THREADS, 1)
   const int n_kc = P.d_in / CK;
   const int n_vc = d16 / V_ROWS;
   const int k_boxes = d64 / 64;         // 64-row TMA boxes per K_t slice
-  const int v_boxes = P.d_emb / 64;     // 64-column TMA boxes per V slice
+  // O = P V_t in passes of at most TMEM_COLS columns of d_emb
+  const int o_max = min(P.d_emb, Cfg::TMEM_COLS);
+  const int n_op = (P.d_emb + o_max - 1) / o_max;
+  const int n_vs = n_op * n_vc;         // V slices over all passes
   // pipeline depth follows from d_t: the S ring holds as many slices as fit,
   // and so do the V buffers after P
   const int s_stage = X_BYTES + d64 * CK * 2;
   const int n_s = min(MAX_STAGES, REGION / s_stage);
   const int p_bytes = (d64 / 64) * (TM * 128);
-  const int v_bytes = V_ROWS * P.d_emb * 2;
+  const int v_bytes = V_ROWS * o_max * 2;
   const int n_v = min(MAX_STAGES, (REGION - p_bytes) / v_bytes);
   uint8_t *pbuf = smem;                 // P slices (PV phase)
   uint8_t *vbuf = smem + p_bytes;       // V slices (PV phase)
@@ -182,6 +204,7 @@ __global__ void __launch_bounds__(DENSE_THREADS, 1)
       mbar_init(&b->vconv[i], 8);
       mbar_init(&b->vempty[i], 1);
     }
+    mbar_init(&b->odrained, 8);
     mbar_init(&b->drain, 1);
     b->abort_flag = 0;
     fence_mbar_init();
@@ -189,7 +212,7 @@ __global__ void __launch_bounds__(DENSE_THREADS, 1)
     prefetch_tensormap(&mV);
   }
   if (warp == 1) {
-    tmem_alloc(&b->tmem_base, 512);
+    tmem_alloc(&b->tmem_base, Cfg::TMEM_COLS);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -224,9 +247,11 @@ __global__ void __launch_bounds__(DENSE_THREADS, 1)
       bool varmed[MAX_STAGES];
       uint32_t varmed_par[MAX_STAGES];
       for (int i = 0; i < MAX_STAGES; ++i) varmed[i] = false;
-      for (int vc = 0; ok && vc < n_vc; ++vc) {
-        const int i = vc % n_v;
-        const uint32_t ph = (vc / n_v) & 1;
+      for (int gv = 0; ok && gv < n_vs; ++gv) {
+        const int h = gv / n_vc, vc = gv % n_vc;
+        const int v_boxes = min(o_max, P.d_emb - h * o_max) / 64;
+        const int i = gv % n_v;
+        const uint32_t ph = (gv / n_v) & 1;
         if (!mbar_wait(&b->vempty[i], ph ^ 1, ab)) {
           ok = false;
           break;
@@ -236,7 +261,8 @@ __global__ void __launch_bounds__(DENSE_THREADS, 1)
         varmed[i] = true;
         varmed_par[i] = ph;
         for (int bx = 0; bx < v_boxes; ++bx)
-          tma_load_2d(vdst + bx * V_BLOCK, &mV, &b->vfull[i], bx * 64, r0 + vc * V_ROWS);
+          tma_load_2d(vdst + bx * V_BLOCK, &mV, &b->vfull[i], h * o_max + bx * 64,
+                      r0 + vc * V_ROWS);
       }
       if (!ok) {
         for (int s = 0; s < MAX_STAGES; ++s)
@@ -275,15 +301,22 @@ __global__ void __launch_bounds__(DENSE_THREADS, 1)
       if (ok) umma_commit(&b->sfull);
       // P V_t into the TMEM columns S used, once the softmax warps have read S
       if (ok) ok = mbar_wait(&b->pready, 0, ab);
-      if (ok) {
+      const uint32_t pa = smem_u32(pbuf);
+      for (int h = 0; ok && h < n_op; ++h) {
+        // a later pass reuses the TMEM columns once the epilogue has read them
+        if (h > 0 && !mbar_wait(&b->odrained, (h - 1) & 1, ab)) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
-        const int o_half = P.d_emb > 256 ? 2 : 1;
-        const uint32_t id_o0 = idesc_f16(0, 1, TM, P.d_emb > 256 ? 256 : P.d_emb);
-        const uint32_t id_o1 = idesc_f16(0, 1, TM, P.d_emb > 256 ? P.d_emb - 256 : 16);
-        const uint32_t pa = smem_u32(pbuf);
-        for (int vc = 0; ok && vc < n_vc; ++vc) {
-          const int i = vc % n_v;
-          const uint32_t ph = (vc / n_v) & 1;
+        const int o_w = min(o_max, P.d_emb - h * o_max);
+        const int o_half = o_w > 256 ? 2 : 1;
+        const uint32_t id_o0 = idesc_f16(0, 1, TM, o_w > 256 ? 256 : o_w);
+        const uint32_t id_o1 = idesc_f16(0, 1, TM, o_w > 256 ? o_w - 256 : 16);
+        for (int vc = 0; vc < n_vc; ++vc) {
+          const int gv = h * n_vc + vc;
+          const int i = gv % n_v;
+          const uint32_t ph = (gv / n_v) & 1;
           if (!mbar_wait(&b->vconv[i], ph, ab)) {
             ok = false;
             break;
@@ -419,41 +452,44 @@ __global__ void __launch_bounds__(DENSE_THREADS, 1)
     ok = softmax_sync_and(ok);
     if (ok) inv_sum = 1.0f / (b->red_sum[0][r] + b->red_sum[1][r]);
 
-    // V slices: bf16 -> fp16 in place, then hand them to the MMA warp
     const int eth = sw * 32 + lane;  // 0..255
-    const int v_vecs = V_ROWS * P.d_emb / 8;
-    for (int vc = 0; ok && vc < n_vc; ++vc) {
-      const int i = vc % n_v;
-      const uint32_t ph = (vc / n_v) & 1;
-      ok = __all_sync(0xffffffffu, mbar_wait(&b->vfull[i], ph, ab));
-      if (!ok) break;
-      uint4 *vb = reinterpret_cast<uint4 *>(vbuf + i * v_bytes);
-      bool bad = false;
-      for (int e = eth; e < v_vecs; e += 256) {
-        uint4 w = vb[e];
-        const __nv_bfloat162 *in = reinterpret_cast<const __nv_bfloat162 *>(&w);
-        uint4 o;
-        __half2 *out = reinterpret_cast<__half2 *>(&o);
+    __half *arow = P.a + (r < n_valid ? (int64_t)P.perm[tok0 + r] * P.d_emb : 0);
+    for (int h = 0; ok && h < n_op; ++h) {
+      const int o_w = min(o_max, P.d_emb - h * o_max);
+      // this pass's V slices: bf16 -> fp16 in place, then hand them to the MMA warp
+      const int v_vecs = V_ROWS * o_w / 8;
+      for (int vc = 0; vc < n_vc; ++vc) {
+        const int gv = h * n_vc + vc;
+        const int i = gv % n_v;
+        const uint32_t ph = (gv / n_v) & 1;
+        ok = __all_sync(0xffffffffu, mbar_wait(&b->vfull[i], ph, ab));
+        if (!ok) break;
+        uint4 *vb = reinterpret_cast<uint4 *>(vbuf + i * v_bytes);
+        bool bad = false;
+        for (int e = eth; e < v_vecs; e += 256) {
+          uint4 w = vb[e];
+          const __nv_bfloat162 *in = reinterpret_cast<const __nv_bfloat162 *>(&w);
+          uint4 o;
+          __half2 *out = reinterpret_cast<__half2 *>(&o);
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const float2 f = __bfloat1622float2(in[k]);
-          bad |= fabsf(f.x) > 65504.f || fabsf(f.y) > 65504.f;
-          out[k] = __floats2half2_rn(f.x, f.y);
+          for (int k = 0; k < 4; ++k) {
+            const float2 f = __bfloat1622float2(in[k]);
+            bad |= fabsf(f.x) > 65504.f || fabsf(f.y) > 65504.f;
+            out[k] = __floats2half2_rn(f.x, f.y);
+          }
+          vb[e] = o;
         }
-        vb[e] = o;
+        if (bad) atomicOr(P.err, DEV_ERR_F16_RANGE);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&b->vconv[i]);
       }
-      if (bad) atomicOr(P.err, DEV_ERR_F16_RANGE);
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&b->vconv[i]);
-    }
 
-    // epilogue: a = O / rowsum, fp16, to the token's original position
-    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&b->ofull, 0, ab));
-    if (ok) {
+      // epilogue: a = O / rowsum, fp16, to the token's original position
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&b->ofull, h & 1, ab));
+      if (!ok) break;
       tc_fence_after();
-      __half *arow = P.a + (r < n_valid ? (int64_t)P.perm[tok0 + r] * P.d_emb : 0);
-      for (int c = half * 32; c < P.d_emb; c += 64) {
+      for (int c = half * 32; c < o_w; c += 64) {
         uint32_t v[32];
         tmem_ld32(trow + c, v);
         tmem_wait_ld();
@@ -466,9 +502,14 @@ __global__ void __launch_bounds__(DENSE_THREADS, 1)
             for (int e = 0; e < 4; ++e)
               o2[e] = __floats2half2_rn(__uint_as_float(v[j * 8 + 2 * e]) * inv_sum,
                                         __uint_as_float(v[j * 8 + 2 * e + 1]) * inv_sum);
-            *reinterpret_cast<uint4 *>(arow + c + j * 8) = o;
+            *reinterpret_cast<uint4 *>(arow + h * o_max + c + j * 8) = o;
           }
         }
+      }
+      if (h + 1 < n_op) {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&b->odrained);
       }
     }
   }
@@ -477,11 +518,31 @@ __global__ void __launch_bounds__(DENSE_THREADS, 1)
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, 512);
+    tmem_dealloc(tmem, Cfg::TMEM_COLS);
   }
 }
 
-constexpr size_t DENSE_SMEM = 1024 + REGION + sizeof(DenseBars);
+template <bool SMALL>
+constexpr size_t dense_smem() {
+  return 1024 + DenseCfg<SMALL>::REGION + sizeof(DenseBars);
+}
+
+template <bool SMALL>
+l3_status launch_cfg(const CUtensorMap &mK, const CUtensorMap &mV, const DenseParams &P,
+                     int64_t n_tiles, int device, const char *name, cudaStream_t s) {
+  if (n_tiles == 0) return L3_OK;
+  static bool attr[64] = {};
+  if (!attr[device & 63]) {
+    L3_CUDA_TRY(cudaFuncSetAttribute(k_attn_dense<SMALL>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)dense_smem<SMALL>()));
+    attr[device & 63] = true;
+  }
+  LaunchTimer t(name, s);
+  k_attn_dense<SMALL><<<(unsigned)n_tiles, DENSE_THREADS, dense_smem<SMALL>(), s>>>(mK, mV, P);
+  L3_CUDA_TRY(cudaGetLastError());
+  return L3_OK;
+}
 
 }  // namespace
 
@@ -510,16 +571,11 @@ l3_status launch_attn_dense(const l3_plan_s *p, const void *x, const void *W_K, 
   P.d_in = (int)d.d_in;
   P.d_emb = (int)d.d_emb;
   P.err = p->dev_flags + 1;
-  static bool attr[64] = {};
-  if (!attr[p->device & 63]) {
-    L3_CUDA_TRY(cudaFuncSetAttribute(k_attn_dense, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     (int)DENSE_SMEM));
-    attr[p->device & 63] = true;
-  }
-  LaunchTimer t("attn_dense", s);
-  k_attn_dense<<<(unsigned)p->n_dense_tiles, DENSE_THREADS, DENSE_SMEM, s>>>(mK, mV, P);
-  L3_CUDA_TRY(cudaGetLastError());
-  return L3_OK;
+  // the plan lists the tiles of groups with d_t > DENSE_SMALL_ROWS first
+  const int64_t n_big = p->n_dense_tiles - p->n_dense_small;
+  if ((st = launch_cfg<false>(mK, mV, P, n_big, p->device, "attn_dense", s)) != L3_OK) return st;
+  P.tiles = p->dense_tiles + n_big;
+  return launch_cfg<true>(mK, mV, P, p->n_dense_small, p->device, "attn_dense_small", s);
 }
 
 }  // namespace l3

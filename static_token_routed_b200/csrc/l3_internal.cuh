@@ -67,6 +67,9 @@ constexpr int DENSE_TILE_M = 128;  // tokens per dense tile
 // many tokens and rows (and d_t fits the kernel); otherwise on CUDA cores
 constexpr int DENSE_MIN_TOKENS = 5;
 constexpr int DENSE_MIN_ROWS = 32;
+// dense groups with at most this many rows run in a configuration that fits
+// two CTAs per SM (256 TMEM columns, O computed in 256-column passes)
+constexpr int DENSE_SMALL_ROWS = 256;
 // tail items with at most this many rows are "small" (latency-bound)
 constexpr int TAIL_SMALL_ROWS = 16;
 
@@ -81,6 +84,7 @@ struct l3_plan_s {
   int64_t n_groups = 0;
   int64_t n_dense_groups = 0;
   int64_t n_dense_tiles = 0;
+  int64_t n_dense_small = 0;  // the last n_dense_small tiles have d_t <= DENSE_SMALL_ROWS
   int64_t n_tail_items = 0;
   int64_t unique_rows = 0;
   int64_t unique_rows_multi = 0;

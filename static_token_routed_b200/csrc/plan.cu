@@ -50,7 +50,10 @@ enum {
   INFO_MAX_TOKENS,
   INFO_CLS,              // 5 slots: first tail item of each token-count class, then the total
   INFO_SPLIT = INFO_CLS + 5,  // 4 slots: first item of each class with d_t <= TAIL_SMALL_ROWS
-  INFO_SLOTS = INFO_SPLIT + 4
+  INFO_DENSE_SMALL = INFO_SPLIT + 4,  // dense tiles of groups with d_t <= DENSE_SMALL_ROWS
+  INFO_CUR_BIG,                       // fill cursors of the two dense tile classes
+  INFO_CUR_SMALL,
+  INFO_SLOTS
 };
 
 __device__ __forceinline__ uint32_t lanemask_lt() {
@@ -282,6 +285,7 @@ __global__ void k_item_counts(const int32_t *__restrict__ group_tok_start,
     if (dense) {
       nt = (c + DENSE_TILE_M - 1) / DENSE_TILE_M;
       atomicAdd(&info[INFO_DENSE_GROUPS], 1);
+      if (rows <= DENSE_SMALL_ROWS) atomicAdd(&info[INFO_DENSE_SMALL], nt);
     } else {
       nl = (c + TAIL_TOKENS - 1) / TAIL_TOKENS;
     }
@@ -308,13 +312,21 @@ __global__ void k_item_fill(const int32_t *__restrict__ group_tok_start,
                             const int32_t *__restrict__ tiles, const int32_t *__restrict__ tile_off,
                             const int32_t *__restrict__ tails, int32_t *__restrict__ dcursor,
                             int k_cap, int64_t cap, DenseTile *__restrict__ dense,
-                            TailItem *__restrict__ tail, const int32_t *info) {
+                            TailItem *__restrict__ tail, int32_t *info) {
   int64_t g = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
   if (g >= cap || g >= info[INFO_G]) return;
   const int32_t start = group_tok_start[g];
   const int32_t c = group_tok_start[g + 1] - start;
-  for (int32_t j = 0; j < tiles[g]; ++j)
-    dense[tile_off[g] + j] = DenseTile{(int32_t)g, start + j * DENSE_TILE_M};
+  // dense tiles: groups with d_t > DENSE_SMALL_ROWS first, then the others
+  // (two launch configurations); any order inside a class gives the same results
+  const int32_t n_big = info[INFO_TILES] - info[INFO_DENSE_SMALL];
+  const bool small_rows = group_rows[g] <= DENSE_SMALL_ROWS;
+  for (int32_t j = 0; j < tiles[g]; ++j) {
+    const int32_t pos = small_rows ? n_big + atomicAdd((int32_t *)&info[INFO_CUR_SMALL], 1)
+                                   : atomicAdd((int32_t *)&info[INFO_CUR_BIG], 1);
+    dense[pos] = DenseTile{(int32_t)g, start + j * DENSE_TILE_M};
+  }
+  (void)tile_off;
   const int32_t rows = group_rows[g];
   for (int32_t j = 0; j < tails[g]; ++j) {
     TailItem it;
@@ -497,6 +509,7 @@ l3_status build_plan(l3_plan_s *p, const int32_t *ids, const int32_t *offsets, c
   }
   p->n_groups = host_info[INFO_G];
   p->n_dense_tiles = host_info[INFO_TILES];
+  p->n_dense_small = host_info[INFO_DENSE_SMALL];
   p->n_tail_items = host_info[INFO_TAILS];
   p->unique_rows = host_info[INFO_ROWS];
   p->unique_rows_multi = host_info[INFO_ROWS_MULTI];

@@ -124,12 +124,17 @@ def test_tensor_core_kernels_run():
     (4, 512, 700, 128, 512, 256, 64),   # d_t = 512 fills TMEM, two PV halves
     (6, 32, 140, 64, 128, 64, 16),      # smallest dense d_t
     (9, 40, 45, 128, 64, 64, 32),       # groups of ~5 tokens: the fewest that go dense
+    (4, 256, 600, 128, 512, 128, 64),   # largest d_t of the two-CTA configuration, two O passes
+    (5, 200, 500, 64, 320, 64, 32),     # O passes of 256 and 64 columns
+    (6, (300, 96, 512, 256, 257, 33), 900, 64, 512, 64, 32),  # both configurations in one batch
 ])
 def test_dense_attention_shapes(vocab, d_t, n, d_in, d_emb, d_up, d_out):
     """Groups on the tensor-core attention kernel, ragged in tokens and d_t."""
-    g = torch.Generator().manual_seed(d_t)
-    off = torch.arange(0, vocab + 1, dtype=torch.int32) * d_t
-    v = vocab * d_t
+    rows = [d_t] * vocab if isinstance(d_t, int) else list(d_t)
+    g = torch.Generator().manual_seed(sum(rows))
+    off = torch.tensor([0] + rows, dtype=torch.int64).cumsum(0).to(torch.int32)
+    v = int(off[-1])
+    d_t = max(rows)
     ids = torch.randint(0, vocab, (n,), generator=g, dtype=torch.int32)
     mk = lambda *s: (torch.randn(*s, generator=g) / s[-1] ** 0.5).to(torch.bfloat16)
     # larger logits than the workloads' so the softmax is far from uniform
@@ -148,7 +153,8 @@ def test_dense_attention_shapes(vocab, d_t, n, d_in, d_emb, d_up, d_out):
     l3.l3_forward_status(plan)
     kernels = l3.l3_profile_read()
     l3.l3_profile_enable(False)
-    assert "attn_dense" in kernels
+    want_cfg = {"attn_dense" if r > 256 else "attn_dense_small" for r in rows}
+    assert want_cfg <= set(kernels), kernels
     want = oracle_y(t, bt)
     err = rel_max_err(y.double().cpu().numpy(), want)
     assert err <= TOL["bf16"], err
