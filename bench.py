@@ -20,7 +20,6 @@ import ctypes
 import json
 import os
 import statistics
-import subprocess
 import sys
 import time
 
@@ -97,63 +96,82 @@ def kernel_roofline(name: str, work: dict, attn_flops: int, peaks: dict):
 # clocks during the timed region
 # ----------------------------------------------------------------------------
 
-class ClockSampler:
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+REASON_BITS = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+               "sw_power_cap": 0x4}
 
-    def __init__(self, device: int):
-        self.proc = None
-        self.device = device
+
+def summarize_clocks(samples):
+    """samples: (sm_mhz, sm_max_mhz, reasons bitmask) tuples taken under load."""
+    if not samples:
+        return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+    reasons = sorted(nm for nm, bit in REASON_BITS.items() if any(r & bit for _, _, r in samples))
+    return {"sm_mhz": statistics.median(s for s, _, _ in samples),
+            "sm_max_mhz": max(m for _, m, _ in samples), "reasons": reasons,
+            "samples": len(samples)}
+
+
+class ClockSampler:
+    """SM clock and clock-event reasons sampled every few ms by NVML (read-only
+    queries) on a host thread while the timed region runs."""
+
+    def __init__(self, device: int, period_s: float = 0.005):
+        self.device, self.period = device, period_s
+        self.samples, self.thread, self.nvml = [], None, None
 
     def __enter__(self):
+        import threading
         try:
-            props = torch.cuda.get_device_properties(self.device)
-            uuid = str(getattr(props, "uuid", "") or "")
-            sel = ["-i", uuid if uuid.startswith("GPU-") else f"GPU-{uuid}"] if uuid else []
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "200", *sel], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
-                text=True)
+            import pynvml as nv
+            nv.nvmlInit()
+            uuid = str(getattr(torch.cuda.get_device_properties(self.device), "uuid", "") or "")
+            uuid = uuid if uuid.startswith("GPU-") else f"GPU-{uuid}"
+            h = nv.nvmlDeviceGetHandleByUUID(uuid)
+            mx = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+            self.nvml = nv
         except Exception:
-            self.proc = None
+            return self
+        self.stop = threading.Event()
+
+        def run():
+            while True:
+                try:
+                    self.samples.append((nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM), mx,
+                                         nv.nvmlDeviceGetCurrentClocksEventReasons(h)))
+                except Exception:
+                    pass
+                if self.stop.wait(self.period):
+                    return
+
+        self.thread = threading.Thread(target=run, daemon=True)
+        self.thread.start()
         return self
 
     def __exit__(self, *exc):
-        self.lines = []
-        if self.proc is not None:
-            self.proc.terminate()
+        if self.thread is not None:
+            self.stop.set()
+            self.thread.join()
+        if self.nvml is not None:
             try:
-                out, _ = self.proc.communicate(timeout=5)
+                self.nvml.nvmlShutdown()
             except Exception:
-                self.proc.kill()
-                out = ""
-            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+                pass
 
     def summary(self):
-        sm, mx, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in getattr(self, "lines", []):
-            parts = [p.strip() for p in ln.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                sm.append(float(parts[1]))
-                mx.append(float(parts[2]))
-            except ValueError:
-                continue
-            for nm, val in zip(names, parts[5:9]):
-                if val.lower() == "active":
-                    reasons.add(nm)
-        if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx),
-                "reasons": sorted(reasons), "samples": len(sm)}
+        return summarize_clocks(self.samples)
 
 
 # ----------------------------------------------------------------------------
 # CPU oracle timing (baseline / reference arm)
 # ----------------------------------------------------------------------------
+
+def time_oracle_bounded(w, tables, batch, min_seconds: float, chunk: int = 256, seed: int = 0):
+    """The oracle on random chunks of the batch until min_seconds of work."""
+    n_tok, total, cores, k = 0, 0.0, 1, 0
+    while total < min_seconds and n_tok < w.n_tokens:
+        n, dt, cores = time_oracle(w, tables, batch, chunk, seed=seed + k)
+        n_tok, total, k = n_tok + n, total + dt, k + 1
+    return n_tok, total, cores
+
 
 def time_oracle(w, tables, batch, n_sample: int, seed: int = 0):
     import oracle  # test infrastructure: only the CPU-baseline and reference legs use it
@@ -191,6 +209,27 @@ def run_reference(args, w, rank):
     print(json.dumps(line), flush=True)
 
 
+# ----------------------------------------------------------------------------
+# ranks: each rank plans and runs its own batch; only the timing is reduced
+# ----------------------------------------------------------------------------
+
+def rank_workload(base: wl.Workload, rank: int) -> wl.Workload:
+    """Same tables on every rank, a different batch per rank (weak scaling)."""
+    return wl.with_tokens(base, base.n_tokens, base.batch_seed + 1000 * rank) if rank else base
+
+
+def max_over_ranks(value: float, dist, device) -> float:
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    if dist is not None:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(tokens_per_rank: int, world: int, ms_max: float) -> float:
+    """Tokens of all ranks over the slowest rank's time."""
+    return tokens_per_rank * world / (ms_max * 1e-3)
+
+
 def config_of(w, args):
     return {"workload": w.name, "global_batch": w.n_tokens * args.gpus, "tokens_per_gpu": w.n_tokens,
             "vocab": w.vocab, "v": w.v, "k": w.k, "d_in": w.d_in, "d_emb": w.d_emb,
@@ -210,8 +249,11 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="paper_shaped", choices=sorted(wl.WORKLOADS))
     ap.add_argument("--impl", default="l3", choices=["l3", "reference"])
-    ap.add_argument("--ref-sample", type=int, default=48, help="oracle tokens per reference step")
-    ap.add_argument("--cpu-sample", type=int, default=192, help="oracle tokens for cpu_baseline")
+    ap.add_argument("--ref-sample", type=int, default=256, help="oracle tokens per reference step")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0,
+                    help="seconds of oracle work for cpu_baseline (0: skip)")
+    ap.add_argument("--tokens", type=int, default=0,
+                    help="tokens per rank (default: the workload's batch size)")
     ap.add_argument("--no-e2e", action="store_true")
     args = ap.parse_args()
 
@@ -219,6 +261,8 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     base = wl.WORKLOADS[args.workload]
+    if args.tokens > 0:
+        base = wl.with_tokens(base, args.tokens)
 
     if args.impl == "reference":
         run_reference(args, base, rank)
@@ -234,7 +278,7 @@ def main():
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     # each rank: same tables, its own batch
-    w = wl.with_tokens(base, base.n_tokens, base.batch_seed + 1000 * rank) if rank else base
+    w = rank_workload(base, rank)
     tables, batch = wl.make_tables(w), wl.make_batch(w)
     d = {k: getattr(tables, k).to(dev) for k in ("offsets", "W_K", "W_V", "W_up", "ln_gamma",
                                                  "ln_beta", "W_mix")}
@@ -288,30 +332,48 @@ def main():
     barrier()
     kernels = l3.l3_profile_read()
     l3.l3_profile_enable(False)
-    ms = ev0.elapsed_time(ev1) / args.steps
-    ms_t = torch.tensor([ms], device=dev)
-    if dist is not None:
-        dist.all_reduce(ms_t, op=dist.ReduceOp.MAX)
-    ms_max = float(ms_t.item())
-    tokens_all = w.n_tokens * world
-    value = tokens_all / (ms_max * 1e-3)
+    ms_max = max_over_ranks(ev0.elapsed_time(ev1) / args.steps, dist, dev)
+    value = job_throughput(w.n_tokens, world, ms_max)
 
     # ---- end to end through the public API with host buffers ----
+    # Each step copies its batch (ids, x) from pinned host memory and reads y
+    # back. The copies run on their own streams into two sets of device
+    # buffers, so batch i+1 moves over PCIe while batch i computes and batch
+    # i-1's y comes back, as in a serving pipeline.
     e2e = None
     if not args.no_e2e:
         ids_h = batch.ids.pin_memory()
         x_h = batch.x.pin_memory()
-        y_h = torch.empty(w.n_tokens, w.d_out, dtype=w.torch_dtype).pin_memory()
-        ids_s = torch.empty_like(ids_d)
-        x_s = torch.empty_like(x_d)
-        y_s = torch.empty_like(y_d)
+        y_h = [torch.empty(w.n_tokens, w.d_out, dtype=w.torch_dtype).pin_memory()
+               for _ in range(2)]
+        ids_s = [torch.empty_like(ids_d) for _ in range(2)]
+        x_s = [torch.empty_like(x_d) for _ in range(2)]
+        y_s = [torch.empty_like(y_d) for _ in range(2)]
+        h2d, d2h = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        ev = lambda: [torch.cuda.Event(), torch.cuda.Event()]  # noqa: E731
+        in_ready, fwd_done, out_done = ev(), ev(), ev()
+        n_e2e = [0]
 
         def e2e_step():
-            with torch.cuda.stream(plan_stream):
-                ids_s.copy_(ids_h, non_blocking=True)
-            x_s.copy_(x_h, non_blocking=True)
-            p = step(ids_s, x_s, y_s)
-            y_h.copy_(y_s, non_blocking=True)
+            k = n_e2e[0]
+            j = k % 2
+            if k >= 2:
+                h2d.wait_event(fwd_done[j])       # forward k-2 no longer reads slot j
+            with torch.cuda.stream(h2d):
+                ids_s[j].copy_(ids_h, non_blocking=True)
+                x_s[j].copy_(x_h, non_blocking=True)
+            in_ready[j].record(h2d)
+            plan_stream.wait_event(in_ready[j])
+            stream.wait_event(in_ready[j])
+            if k >= 2:
+                stream.wait_event(out_done[j])    # y of step k-2 has left slot j
+            p = step(ids_s[j], x_s[j], y_s[j])
+            fwd_done[j].record(stream)
+            d2h.wait_event(fwd_done[j])
+            with torch.cuda.stream(d2h):
+                y_h[j].copy_(y_s[j], non_blocking=True)
+            out_done[j].record(d2h)
+            n_e2e[0] = k + 1
             return p
 
         for _ in range(3):
@@ -320,18 +382,21 @@ def main():
         torch.cuda.synchronize(dev)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
-        plan_stream.wait_event(e0)
+        for st in (plan_stream, h2d, d2h):
+            st.wait_event(e0)
         for _ in range(args.steps):
             e2e_step().destroy()
+        last = torch.cuda.Event()
+        last.record(d2h)
+        stream.wait_event(last)
         e1.record(stream)
         torch.cuda.synchronize(dev)
         barrier()
-        ems = torch.tensor([e0.elapsed_time(e1) / args.steps], device=dev)
-        if dist is not None:
-            dist.all_reduce(ems, op=dist.ReduceOp.MAX)
-        e2e = {"value": tokens_all / (float(ems.item()) * 1e-3), "unit": "tokens/s",
+        ems = max_over_ranks(e0.elapsed_time(e1) / args.steps, dist, dev)
+        e2e = {"value": job_throughput(w.n_tokens, world, ems), "unit": "tokens/s",
                "h2d_bytes_per_step": int(ids_h.numel() * 4 + x_h.numel() * x_h.element_size()),
-               "d2h_bytes_per_step": int(y_h.numel() * y_h.element_size())}
+               "d2h_bytes_per_step": int(y_h[0].numel() * y_h[0].element_size()),
+               "copies": "own streams, double-buffered: overlap the previous and next steps"}
 
     if rank != 0:
         if dist is not None:
@@ -374,10 +439,11 @@ def main():
 
     # ---- CPU baseline: the oracle on a bounded sample ----
     cpu = None
-    if world == 1 and args.cpu_sample > 0:
-        n_s, dt, cores = time_oracle(w, tables, batch, args.cpu_sample)
+    if world == 1 and args.cpu_seconds > 0:
+        n_s, dt, cores = time_oracle_bounded(w, tables, batch, args.cpu_seconds)
         cpu = {"value": n_s / dt, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-               "sample": f"{n_s} random tokens of the {w.name} batch (fp64 oracle, {dt:.1f} s)"}
+               "sample": f"{n_s} random tokens of the {w.name} batch in chunks of 256 "
+                         f"(fp64 oracle, {dt:.1f} s)"}
 
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max,
