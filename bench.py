@@ -76,6 +76,16 @@ def attention_flops(ids: np.ndarray, offsets: np.ndarray, w: wl.Workload) -> int
     return int(2 * np.sum(d[d > 1]) * (w.d_in + w.d_emb))
 
 
+# DRAM bytes (read + write) per launch of a kernel, from one ncu capture of
+#   ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum,gpu__time_duration.sum
+#       --clock-control none -k regex:<kernel> -s 3 -c 1
+#       python bench.py --workload <w> --steps 1 --warmup 3 --no-e2e --cpu-seconds 0
+# keyed by (kernel, workload, tokens); remove an entry when its kernel changes
+TRAFFIC = {
+    ("mix_gemm_tc", "paper_shaped", 65536): 556745472 + 245015296,
+}
+
+
 # per-kernel roofline: what each kernel must move or compute per launch
 def kernel_roofline(name: str, work: dict, attn_flops: int, peaks: dict):
     if name.startswith("attn"):
@@ -434,7 +444,8 @@ def main():
             per_launch_units = units / launches_per_step
             achieved = per_launch_units / per_launch_s / (1e9 if unit == "GB/s" else 1e12)
             roof = {"kernel": top, "bound": bound, "achieved": achieved, "peak": peak,
-                    "unit": unit, "frac": achieved / peak, "traffic": None,
+                    "unit": unit, "frac": achieved / peak,
+                    "traffic": TRAFFIC.get((top, w.name, w.n_tokens)),
                     "peak_source": f"{peaks['source']} ({'sustained bf16' if bound == 'tensor' else 'HBM copy' if bound == 'hbm' else 'FFMA lanes x max clock'})"}
 
     # ---- CPU baseline: the oracle on a bounded sample ----

@@ -375,25 +375,33 @@ l3_status l3_forward(const void *x, l3_plan_t p, const void *W_K, const void *W_
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   p->stream = s;
   l3_status st = L3_OK;
-  if (p->n_dense_tiles > 0 && p->n_tail_items > 0) {
-    // fork: tail attention and the fp16 weight copies on the helper stream,
-    // dense attention on the caller's stream; join before W_up
+  const bool has_big = p->n_dense_tiles > p->n_dense_small;
+  const bool has_small = p->n_dense_small > 0;
+  const bool has_tail = p->n_tail_items > 0;
+  auto tail = [&](cudaStream_t q) {
+    return tail_cls_supported(p->dims) ? launch_attn_tail_cls(p, x, W_K, W_V, q)
+                                       : launch_attn_tail(p, x, W_K, W_V, q);
+  };
+  if ((has_big || has_small) && has_tail) {
+    // fork: dense attention (both configurations, in turn) on the caller's
+    // stream; the fp16 weight copies and the tail attention on the helper
+    // stream, whose short CTAs fill the SMs the long dense CTAs leave; join
+    // before W_up. The launches write disjoint rows of a.
     Aux *aux = nullptr;
     if ((st = aux_for(p->device, &aux)) != L3_OK) return st;
     std::lock_guard<std::mutex> lk(aux->mu);
     L3_CUDA_TRY(cudaEventRecord(aux->fork, s));
     L3_CUDA_TRY(cudaStreamWaitEvent(aux->stream, aux->fork, 0));
     if (p->tc_gemm) st = launch_weights_f16(p, W_up, W_mix, aux->stream);
-    if (st == L3_OK)
-      st = tail_cls_supported(p->dims) ? launch_attn_tail_cls(p, x, W_K, W_V, aux->stream)
-                                       : launch_attn_tail(p, x, W_K, W_V, aux->stream);
-    if (st == L3_OK) st = launch_attn_dense(p, x, W_K, W_V, s);
+    if (st == L3_OK) st = launch_attn_dense(p, x, W_K, W_V, false, s);
+    if (st == L3_OK) st = launch_attn_dense(p, x, W_K, W_V, true, s);
+    if (st == L3_OK) st = tail(aux->stream);
     L3_CUDA_TRY(cudaEventRecord(aux->join, aux->stream));
     L3_CUDA_TRY(cudaStreamWaitEvent(s, aux->join, 0));
   } else {
-    st = tail_cls_supported(p->dims) ? launch_attn_tail_cls(p, x, W_K, W_V, s)
-                                     : launch_attn_tail(p, x, W_K, W_V, s);
-    if (st == L3_OK) st = launch_attn_dense(p, x, W_K, W_V, s);
+    st = tail(s);
+    if (st == L3_OK) st = launch_attn_dense(p, x, W_K, W_V, false, s);
+    if (st == L3_OK) st = launch_attn_dense(p, x, W_K, W_V, true, s);
     if (st == L3_OK && p->tc_gemm) st = launch_weights_f16(p, W_up, W_mix, s);
   }
   if (p->tc_gemm) {

@@ -552,8 +552,10 @@ bool dense_attention_supported(const l3_dims_t &d) {
 int dense_attention_max_rows() { return MAX_D; }
 
 l3_status launch_attn_dense(const l3_plan_s *p, const void *x, const void *W_K, const void *W_V,
-                            cudaStream_t s) {
-  if (p->n_dense_tiles == 0) return L3_OK;
+                            bool small, cudaStream_t s) {
+  // the plan lists the tiles of groups with d_t > DENSE_SMALL_ROWS first
+  const int64_t n_big = p->n_dense_tiles - p->n_dense_small;
+  if ((small ? p->n_dense_small : n_big) == 0) return L3_OK;
   const l3_dims_t &d = p->dims;
   CUtensorMap mK, mV;
   l3_status st;
@@ -571,9 +573,7 @@ l3_status launch_attn_dense(const l3_plan_s *p, const void *x, const void *W_K, 
   P.d_in = (int)d.d_in;
   P.d_emb = (int)d.d_emb;
   P.err = p->dev_flags + 1;
-  // the plan lists the tiles of groups with d_t > DENSE_SMALL_ROWS first
-  const int64_t n_big = p->n_dense_tiles - p->n_dense_small;
-  if ((st = launch_cfg<false>(mK, mV, P, n_big, p->device, "attn_dense", s)) != L3_OK) return st;
+  if (!small) return launch_cfg<false>(mK, mV, P, n_big, p->device, "attn_dense", s);
   P.tiles = p->dense_tiles + n_big;
   return launch_cfg<true>(mK, mV, P, p->n_dense_small, p->device, "attn_dense_small", s);
 }

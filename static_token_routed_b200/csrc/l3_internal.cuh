@@ -133,8 +133,10 @@ l3_status launch_attn_tail_cls(const l3_plan_s *p, const void *x, const void *W_
 // attention, tensor-core path (attn_dense.cu)
 bool dense_attention_supported(const l3_dims_t &d);
 int dense_attention_max_rows();
+// one of the two launch configurations: tiles with d_t > DENSE_SMALL_ROWS
+// (small = false) or the others
 l3_status launch_attn_dense(const l3_plan_s *p, const void *x, const void *W_K, const void *W_V,
-                            cudaStream_t s);
+                            bool small, cudaStream_t s);
 
 // GEMMs + LayerNorm, tensor-core path (gemm_tc.cu)
 bool tc_gemm_supported(const l3_dims_t &d);

@@ -51,8 +51,6 @@ enum {
   INFO_CLS,              // 5 slots: first tail item of each token-count class, then the total
   INFO_SPLIT = INFO_CLS + 5,  // 4 slots: first item of each class with d_t <= TAIL_SMALL_ROWS
   INFO_DENSE_SMALL = INFO_SPLIT + 4,  // dense tiles of groups with d_t <= DENSE_SMALL_ROWS
-  INFO_CUR_BIG,                       // fill cursors of the two dense tile classes
-  INFO_CUR_SMALL,
   INFO_SLOTS
 };
 
@@ -272,7 +270,8 @@ __global__ void k_item_counts(const int32_t *__restrict__ group_tok_start,
                               const int32_t *__restrict__ group_rows, int64_t cap,
                               int dense_min_tokens, int dense_min_rows, int dense_max_rows,
                               int32_t *__restrict__ tiles, int32_t *__restrict__ tails,
-                              int32_t *__restrict__ dcount, int k_cap, int32_t *info) {
+                              int32_t *__restrict__ dcount, int32_t *__restrict__ tcount,
+                              int k_cap, int32_t *info) {
   int64_t g = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
   if (g >= cap) return;
   int32_t G = info[INFO_G];
@@ -286,6 +285,10 @@ __global__ void k_item_counts(const int32_t *__restrict__ group_tok_start,
       nt = (c + DENSE_TILE_M - 1) / DENSE_TILE_M;
       atomicAdd(&info[INFO_DENSE_GROUPS], 1);
       if (rows <= DENSE_SMALL_ROWS) atomicAdd(&info[INFO_DENSE_SMALL], nt);
+      // dense tiles are listed largest d_t first (bucket k_cap - d_t): the
+      // longest CTAs start first, and the d_t > DENSE_SMALL_ROWS tiles come
+      // before the others
+      atomicAdd(&tcount[k_cap - min(rows, k_cap)], nt);
     } else {
       nl = (c + TAIL_TOKENS - 1) / TAIL_TOKENS;
     }
@@ -309,7 +312,7 @@ __global__ void k_item_fill(const int32_t *__restrict__ group_tok_start,
                             const int32_t *__restrict__ group_row_start,
                             const int32_t *__restrict__ group_rows,
                             const int32_t *__restrict__ perm,
-                            const int32_t *__restrict__ tiles, const int32_t *__restrict__ tile_off,
+                            const int32_t *__restrict__ tiles, int32_t *__restrict__ tcursor,
                             const int32_t *__restrict__ tails, int32_t *__restrict__ dcursor,
                             int k_cap, int64_t cap, DenseTile *__restrict__ dense,
                             TailItem *__restrict__ tail, int32_t *info) {
@@ -317,17 +320,14 @@ __global__ void k_item_fill(const int32_t *__restrict__ group_tok_start,
   if (g >= cap || g >= info[INFO_G]) return;
   const int32_t start = group_tok_start[g];
   const int32_t c = group_tok_start[g + 1] - start;
-  // dense tiles: groups with d_t > DENSE_SMALL_ROWS first, then the others
-  // (two launch configurations); any order inside a class gives the same results
-  const int32_t n_big = info[INFO_TILES] - info[INFO_DENSE_SMALL];
-  const bool small_rows = group_rows[g] <= DENSE_SMALL_ROWS;
-  for (int32_t j = 0; j < tiles[g]; ++j) {
-    const int32_t pos = small_rows ? n_big + atomicAdd((int32_t *)&info[INFO_CUR_SMALL], 1)
-                                   : atomicAdd((int32_t *)&info[INFO_CUR_BIG], 1);
-    dense[pos] = DenseTile{(int32_t)g, start + j * DENSE_TILE_M};
-  }
-  (void)tile_off;
   const int32_t rows = group_rows[g];
+  // a group's dense tiles sit side by side (they share K_t, V_t through L2);
+  // any order of the groups inside a d_t bucket gives the same results
+  if (tiles[g] > 0) {
+    const int32_t pos = atomicAdd(&tcursor[k_cap - min(rows, k_cap)], tiles[g]);
+    for (int32_t j = 0; j < tiles[g]; ++j)
+      dense[pos + j] = DenseTile{(int32_t)g, start + j * DENSE_TILE_M};
+  }
   for (int32_t j = 0; j < tails[g]; ++j) {
     TailItem it;
     it.r0 = group_row_start[g];
@@ -364,9 +364,10 @@ size_t plan_scratch_bytes(int64_t n) {
   ints += 2 * (size_t)n;                 // ping-pong keys / vals
   ints += (size_t)RADIX * tiles + 1;     // histogram / offsets
   ints += 2 * ((size_t)n + 1);           // head flags, group positions
-  ints += 4 * ((size_t)n + 1);           // tiles, tile offsets, tails, tail offsets
+  ints += 2 * ((size_t)n + 1);           // dense tiles and tail items per group
   ints += 64;                            // info block
   ints += 2 * (N_CLASSES * MAX_DT_BUCKETS + 1);  // tail items per bucket, and their cursors
+  ints += 2 * (MAX_DT_BUCKETS + 1);      // dense tiles per d_t bucket, and their cursors
   return ints * sizeof(int32_t) + 256;
 }
 
@@ -389,11 +390,7 @@ l3_status build_plan(l3_plan_s *p, const int32_t *ids, const int32_t *offsets, c
   sp += cap;
   int32_t *tiles = sp;
   sp += cap;
-  int32_t *tile_off = sp;
-  sp += cap;
   int32_t *tails = sp;
-  sp += cap;
-  int32_t *tail_off = sp;
   sp += cap;
   int32_t *info = sp;
   sp += 64;
@@ -401,6 +398,10 @@ l3_status build_plan(l3_plan_s *p, const int32_t *ids, const int32_t *offsets, c
   sp += N_CLASSES * MAX_DT_BUCKETS + 1;
   int32_t *dcursor = sp;
   sp += N_CLASSES * MAX_DT_BUCKETS + 1;
+  int32_t *tcount = sp;
+  sp += MAX_DT_BUCKETS + 1;
+  int32_t *tcursor = sp;
+  sp += MAX_DT_BUCKETS + 1;
   const int k_cap = (int)std::min<int64_t>(p->dims.k, MAX_DT_BUCKETS - 1);
   if ((size_t)((char *)sp - (char *)scratch) > scratch_bytes) {
     set_error("internal: plan scratch too small");
@@ -469,24 +470,25 @@ l3_status build_plan(l3_plan_s *p, const int32_t *ids, const int32_t *offsets, c
     }
     const int n_buckets = N_CLASSES * (k_cap + 1);
     L3_CUDA_TRY(cudaMemsetAsync(dcount, 0, n_buckets * sizeof(int32_t), s));
+    L3_CUDA_TRY(cudaMemsetAsync(tcount, 0, (k_cap + 1) * sizeof(int32_t), s));
     {
       LaunchTimer t("plan_item_counts", s);
       k_item_counts<<<blocks_for(cap, 256), 256, 0, s>>>(p->group_tok_start, p->group_rows, n,
                                                          dense_min_tokens, dense_min_rows,
                                                          dense_max_rows, tiles, tails, dcount,
-                                                         k_cap, info);
+                                                         tcount, k_cap, info);
     }
     // three independent scans in one launch: d_t over groups (segment row
-    // offsets), dense tiles over groups, tail items over (class, d_t) buckets
+    // offsets), dense tiles over d_t buckets, tail items over (class, d_t) buckets
     scan_multi({{p->group_rows, p->seg_rows, n, &info[INFO_ROWS]},
-                {tiles, tile_off, n, &info[INFO_TILES]},
+                {tcount, tcursor, k_cap + 1, &info[INFO_TILES]},
                 {dcount, dcursor, n_buckets, &info[INFO_TAILS]}},
                s);
     k_class_starts<<<1, 32, 0, s>>>(dcursor, k_cap, info);
     {
       LaunchTimer t("plan_item_fill", s);
       k_item_fill<<<blocks_for(n, 256), 256, 0, s>>>(p->group_tok_start, p->group_row_start,
-                                                     p->group_rows, p->perm, tiles, tile_off,
+                                                     p->group_rows, p->perm, tiles, tcursor,
                                                      tails, dcursor, k_cap, n, p->dense_tiles,
                                                      p->tail_items, info);
     }
