@@ -281,18 +281,53 @@ __device__ __forceinline__ bool epi_sync_and(bool ok) {
   return r != 0;
 }
 
+// (n_a, mean_a, M2_a) <- (n_a, mean_a, M2_a) (+) (n_b, mean_b, M2_b): Chan,
+// Golub and LeVeque's pairwise update of a mean and a sum of squared deviations
+__device__ __forceinline__ void chan_merge(float &n_a, float &mean_a, float &m2_a, float n_b,
+                                           float mean_b, float m2_b) {
+  const float n = n_a + n_b;
+  if (n_b == 0.f) return;
+  const float delta = mean_b - mean_a;
+  mean_a += delta * (n_b / n);
+  m2_a += m2_b + delta * delta * (n_a * n_b / n);
+  n_a = n;
+}
+
+__device__ __forceinline__ void st_shared_cluster_f32(uint32_t addr, float v) {
+  asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
+}
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_arrive_release() {
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait_acquire() {
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, const void *src, int x,
+                                             int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(map),
+      "r"(smem_u32(src)), "r"(x), "r"(y)
+      : "memory");
+}
+__device__ __forceinline__ void bulk_commit_and_wait_all() {
+  asm volatile("cp.async.bulk.commit_group;\n\tcp.async.bulk.wait_group 0;" ::: "memory");
+}
+
 __global__ void __launch_bounds__(UP_THREADS, 2)
     k_up_ln_gemm(const __grid_constant__ CUtensorMap mA, const __grid_constant__ CUtensorMap mB,
-                 UpParams P) {
+                 const __grid_constant__ CUtensorMap mH, UpParams P) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = align1024(smem_raw);
   uint8_t *ring = smem;
   Bars *b = reinterpret_cast<Bars *>(smem + UP_STAGES * STAGE_BYTES);
   float *g_s = reinterpret_cast<float *>(b + 1);  // gamma of this CTA's 256 columns
   float *b_s = g_s + BN;                          // beta
-  float *st_mean = b_s + BN;                      // per-row mean of this CTA's slice
-  float *st_m2 = st_mean + BM;                    // per-row sum of squared deviations
-  float(*red)[BM] = reinterpret_cast<float(*)[BM]>(st_m2 + BM);  // [2][BM] halves of a row
+  float(*red)[BM] = reinterpret_cast<float(*)[BM]>(b_s + BN);  // [4][BM]: mean, M2 of two halves
+  // [2][8][BM]: every slice's (mean, M2) per row, written by the cluster's CTAs
+  float(*st_all)[8][BM] = reinterpret_cast<float(*)[8][BM]>(red[4]);
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const uint32_t rank = cluster_ctarank();
   const uint32_t n_ranks = gridDim.x;  // one cluster spans the grid's x dimension
@@ -324,6 +359,9 @@ __global__ void __launch_bounds__(UP_THREADS, 2)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  // first phase of the cluster barrier: every CTA of the cluster has started
+  // before any writes into another's shared memory (waited on before that)
+  cluster_arrive_relaxed();
   const uint32_t tmem = b->tmem_base;
   const Abort ab{&b->abort_flag, P.err};
 
@@ -381,9 +419,10 @@ __global__ void __launch_bounds__(UP_THREADS, 2)
     }
   }
 
-  // epilogue part 1: per-row mean and M2 of this CTA's slice. Warps 2-9, two
-  // per TMEM lane quarter; each takes every other 32-column chunk, and the two
-  // halves of a row combine through shared memory.
+  // epilogue part 1: per-row (mean, M2) of this CTA's slice in one pass over
+  // TMEM. Warps 2-9, two per TMEM lane quarter; each takes every other
+  // 32-column chunk, takes each chunk's exact mean and M2 in registers and
+  // merges chunks, then the two halves of a row merge through shared memory.
   const bool epi = warp >= 2;
   const int q = warp & 3;
   const int half = (warp - 2) / 4;
@@ -395,103 +434,99 @@ __global__ void __launch_bounds__(UP_THREADS, 2)
     have = __all_sync(0xffffffffu, mbar_wait(&b->tfull[0], 0, ab));
     have = epi_sync_and(have);
     tc_fence_after();
-    float sum = 0.f;
+    float n_acc = 0.f, mean_acc = 0.f, m2_acc = 0.f;
     if (have) {
 #pragma unroll 1
       for (int c = half; c < BN / 32; c += 2) {
+        const int nv = min(32, n_valid - c * 32);
+        if (nv <= 0) break;
         uint32_t v[32];
         tmem_ld32(trow + c * 32, v);
         tmem_wait_ld();
+        float sum = 0.f;
 #pragma unroll
         for (int j = 0; j < 32; ++j)
-          if (c * 32 + j < n_valid) sum += __uint_as_float(v[j]);
-      }
-    }
-    red[half][r] = sum;
-    epi_sync_and(true);
-    const float mean = (red[0][r] + red[1][r]) / (float)n_valid;
-    float m2 = 0.f;
-    if (have) {
-#pragma unroll 1
-      for (int c = half; c < BN / 32; c += 2) {
-        uint32_t v[32];
-        tmem_ld32(trow + c * 32, v);
-        tmem_wait_ld();
+          if (j < nv) sum += __uint_as_float(v[j]);
+        const float mc = sum / (float)nv;
+        float qc = 0.f;
 #pragma unroll
         for (int j = 0; j < 32; ++j)
-          if (c * 32 + j < n_valid) {
-            const float dlt = __uint_as_float(v[j]) - mean;
-            m2 = fmaf(dlt, dlt, m2);
+          if (j < nv) {
+            const float dlt = __uint_as_float(v[j]) - mc;
+            qc = fmaf(dlt, dlt, qc);
           }
+        chan_merge(n_acc, mean_acc, m2_acc, (float)nv, mc, qc);
       }
     }
-    epi_sync_and(true);  // both halves have read red[.][r] (the sums)
-    red[half][r] = m2;
+    red[2 * half][r] = mean_acc;
+    red[2 * half + 1][r] = m2_acc;
     epi_sync_and(true);
     if (half == 0) {
-      st_mean[r] = mean;
-      st_m2[r] = red[0][r] + red[1][r];
+      // this slice's statistics go to every CTA of the cluster (this one
+      // included); the other half's column count follows from n_valid
+      float n1 = 0.f;
+      for (int c = 1; c < BN / 32; c += 2) n1 += (float)max(0, min(32, n_valid - c * 32));
+      chan_merge(n_acc, mean_acc, m2_acc, n1, red[2][r], red[3][r]);
+      // wait for the start-up phase (every CTA of the cluster is running)
+      asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
+      for (uint32_t j = 0; j < n_ranks; ++j) {
+        st_shared_cluster_f32(map_shared_rank(&st_all[0][rank][r], j), mean_acc);
+        st_shared_cluster_f32(map_shared_rank(&st_all[1][rank][r], j), m2_acc);
+      }
+    } else {
+      asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
     }
+  } else {
+    asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
   }
   __syncwarp();
-  cluster_sync();  // every CTA's (mean, M2) is visible cluster-wide
+  // second phase: every CTA's statistics have landed in every CTA; nothing is
+  // read from or written to another CTA's shared memory after this
+  cluster_arrive_release();
+  cluster_wait_acquire();
 
-  float mu = 0.f, rstd = 0.f;
   if (epi) {
-    // all slices' statistics first (independent remote loads in flight
-    // together), then merge in rank order: n_a, mean_a, M2_a (+) n_b, mean_b, M2_b
-    float mbv[8], qbv[8];
-#pragma unroll
-    for (uint32_t j = 0; j < 8; ++j)
-      if (j < n_ranks) {
-        mbv[j] = ld_shared_cluster_f32(map_shared_rank(&st_mean[r], j));
-        qbv[j] = ld_shared_cluster_f32(map_shared_rank(&st_m2[r], j));
-      }
+    // merge the slices in rank order
     float n_acc = 0.f, mean_acc = 0.f, m2_acc = 0.f;
-#pragma unroll
-    for (uint32_t j = 0; j < 8; ++j) {
-      if (j >= n_ranks) break;
-      const float nb = (float)min(BN, P.N - (int)j * BN);
-      const float mb = mbv[j];
-      const float qb = qbv[j];
-      const float n_new = n_acc + nb;
-      const float delta = mb - mean_acc;
-      mean_acc += delta * (nb / n_new);
-      m2_acc += qb + delta * delta * (n_acc * nb / n_new);
-      n_acc = n_new;
-    }
-    mu = mean_acc;
-    rstd = 1.0f / sqrtf(m2_acc / n_acc + P.eps);
-  }
-  cluster_sync();  // peers are done reading this CTA's statistics
-
-  if (epi && have) {
-    const int m = m0 + r;
-    __half *hrow = P.h + (int64_t)m * P.N + n0;
 #pragma unroll 1
-    for (int c = half; c < BN / 32; c += 2) {
-      uint32_t v[32];
-      tmem_ld32(trow + c * 32, v);
-      tmem_wait_ld();
-      if (m < P.M) {
+    for (uint32_t j = 0; j < n_ranks; ++j)
+      chan_merge(n_acc, mean_acc, m2_acc, (float)min(BN, P.N - (int)j * BN), st_all[0][j][r],
+                 st_all[1][j][r]);
+    const float mu = mean_acc;
+    const float rstd = 1.0f / sqrtf(m2_acc / n_acc + P.eps);
+    // normalise into the (now idle) stage ring in the 128-byte-swizzled layout
+    // of 64-column TMA boxes, then one thread stores the boxes with TMA
+    if (have) {
+#pragma unroll 1
+      for (int c = half; c < BN / 32; c += 2) {
+        if (c * 32 >= n_valid) break;
+        uint32_t v[32];
+        tmem_ld32(trow + c * 32, v);
+        tmem_wait_ld();
+        uint8_t *box = ring + (c / 2) * (BM * 128);
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          const int col = c * 32 + j * 8;
-          if (col < n_valid) {
-            uint4 o;
-            __half2 *o2 = reinterpret_cast<__half2 *>(&o);
+          uint4 o;
+          __half2 *o2 = reinterpret_cast<__half2 *>(&o);
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int k0 = col + 2 * e;
-              const float h0 = g_s[k0] * ((__uint_as_float(v[j * 8 + 2 * e]) - mu) * rstd) + b_s[k0];
-              const float h1 =
-                  g_s[k0 + 1] * ((__uint_as_float(v[j * 8 + 2 * e + 1]) - mu) * rstd) + b_s[k0 + 1];
-              o2[e] = __floats2half2_rn(h0, h1);
-            }
-            *reinterpret_cast<uint4 *>(hrow + col) = o;
+          for (int e = 0; e < 4; ++e) {
+            const int k0 = c * 32 + j * 8 + 2 * e;
+            const float h0 = g_s[k0] * ((__uint_as_float(v[j * 8 + 2 * e]) - mu) * rstd) + b_s[k0];
+            const float h1 =
+                g_s[k0 + 1] * ((__uint_as_float(v[j * 8 + 2 * e + 1]) - mu) * rstd) + b_s[k0 + 1];
+            o2[e] = __floats2half2_rn(h0, h1);
           }
+          const int chunk = (c % 2) * 4 + j;  // 16-byte chunk within the box's 128-byte row
+          *reinterpret_cast<uint4 *>(box + r * 128 + ((chunk ^ (r & 7)) << 4)) = o;
         }
       }
+    }
+    fence_proxy_async_smem();
+    have = epi_sync_and(have);
+    if (have && warp == 2 && lane == 0) {
+      for (int bx = 0; bx * 64 < n_valid; ++bx)
+        tma_store_2d(&mH, ring + bx * (BM * 128), n0 + bx * 64, m0);
+      bulk_commit_and_wait_all();
     }
   }
   __syncwarp();
@@ -582,7 +617,8 @@ int num_sms() {
 
 constexpr size_t MIX_SMEM = 1024 + MIX_STAGES * STAGE_BYTES + sizeof(Bars);
 constexpr size_t UP_SMEM =
-    1024 + UP_STAGES * STAGE_BYTES + sizeof(Bars) + (2 * BN + 4 * BM) * sizeof(float);
+    1024 + UP_STAGES * STAGE_BYTES + sizeof(Bars) + (2 * BN + 4 * BM + 2 * 8 * BM) * sizeof(float);
+static_assert(UP_STAGES * STAGE_BYTES >= (BN / 64) * BM * 128, "h staging fits the stage ring");
 
 }  // namespace
 
@@ -639,6 +675,10 @@ l3_status launch_up_ln_tc(const l3_plan_s *p, const void *gamma, const void *bet
   if ((st = make_map(&mB, p->w_up16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, d.d_up, d.d_emb, d.d_emb,
                      BN)) != L3_OK)
     return st;
+  CUtensorMap mH;  // h is written with TMA from 64-column, 128-row boxes
+  if ((st = make_map(&mH, p->h_buf, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, p->n_tokens, d.d_up, d.d_up,
+                     BM)) != L3_OK)
+    return st;
   UpParams P;
   P.M = (int)p->n_tokens;
   P.N = (int)d.d_up;
@@ -668,7 +708,7 @@ l3_status launch_up_ln_tc(const l3_plan_s *p, const void *gamma, const void *bet
   cfg.attrs = at;
   cfg.numAttrs = 1;
   LaunchTimer t("up_ln_gemm_tc", s);
-  L3_CUDA_TRY(cudaLaunchKernelEx(&cfg, k_up_ln_gemm, mA, mB, P));
+  L3_CUDA_TRY(cudaLaunchKernelEx(&cfg, k_up_ln_gemm, mA, mB, mH, P));
   return L3_OK;
 }
 
