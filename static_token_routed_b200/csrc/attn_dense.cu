@@ -11,10 +11,12 @@
 //
 // One CTA takes one 128-token tile of one group:
 //   - warps 2-3 gather the tile's x rows (through the sort permutation) into
-//     64-byte-swizzled shared memory with cp.async, 32 columns at a time and
-//     several slices ahead;
-//   - warp 0 streams the matching 32-column slices of K_t with TMA, as many
-//     slices in flight as the shared-memory ring holds for this d_t;
+//     128-byte-swizzled shared memory with cp.async, 64 columns at a time and
+//     up to a ring's depth of slices ahead;
+//   - warp 0 streams the matching 64-column slices of K_t with TMA (128 bytes
+//     of each row per request: half as many, twice as long DRAM reads as
+//     32-column slices, which streamed K_t markedly slower), as many slices in
+//     flight as the shared-memory ring holds for this d_t;
 //   - warp 1 issues tcgen05.mma (M = 128 tokens, N = d_t up to 2 x 256) so that
 //     S accumulates in TMEM over d_in;
 //   - warps 4-11 (two per TMEM lane quarter, so two threads per token row,
@@ -47,10 +49,10 @@ namespace {
 using namespace sm100;
 
 constexpr int TM = 128;                 // tokens per tile
-constexpr int CK = 32;                  // d_in columns per S-phase slice (64-byte rows)
+constexpr int CK = 64;                  // d_in columns per S-phase slice (128-byte rows)
 constexpr int MAX_D = 512;              // d_t handled here (TMEM columns)
 constexpr int MAX_EMB = 512;
-constexpr int X_BYTES = TM * CK * 2;    // 8 KB
+constexpr int X_BYTES = TM * CK * 2;    // 16 KB
 constexpr int MAX_STAGES = 8;
 
 // Two launch configurations. The big one holds S for d_t up to 512 (all 512
@@ -98,13 +100,6 @@ struct DenseParams {
 
 __device__ __forceinline__ uint8_t *align1024(uint8_t *p) {
   return reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
-}
-
-// K-major operand with 64-byte rows (32 16-bit elements), 64-byte swizzle:
-// 8-row groups 512 bytes apart.
-__device__ __forceinline__ uint64_t sdesc_sw64(uint32_t smem_addr) {
-  return (uint64_t)((smem_addr >> 4) & 0x3FFFu) | (1ull << 16) | ((uint64_t)(512 >> 4) << 32) |
-         (1ull << 46) | (4ull << 61);
 }
 
 __device__ __forceinline__ void cp_async16_zfill(void *dst, const void *src, uint32_t src_bytes) {
@@ -290,10 +285,10 @@ __global__ void __launch_bounds__(DENSE_THREADS, DenseCfg<SMALL>::MIN_BLOCKS)
         const uint32_t ka = xa + X_BYTES;
 #pragma unroll
         for (int k = 0; k < CK / 16; ++k) {
-          const uint64_t adesc = sdesc_sw64(xa + k * 32);
-          umma_f16(tmem, adesc, sdesc_sw64(ka + k * 32), id_s0, (kc | k) != 0);
+          const uint64_t adesc = sdesc_sw128(xa + k * 32, 16, 1024);
+          umma_f16(tmem, adesc, sdesc_sw128(ka + k * 32, 16, 1024), id_s0, (kc | k) != 0);
           if (n_half == 2)
-            umma_f16(tmem + 256, adesc, sdesc_sw64(ka + 256 * CK * 2 + k * 32), id_s1,
+            umma_f16(tmem + 256, adesc, sdesc_sw128(ka + 256 * CK * 2 + k * 32, 16, 1024), id_s1,
                      (kc | k) != 0);
         }
         umma_commit(&b->sempty[s]);
@@ -362,14 +357,14 @@ __global__ void __launch_bounds__(DENSE_THREADS, DenseCfg<SMALL>::MIN_BLOCKS)
       ok = __all_sync(0xffffffffu, mbar_wait(&b->sempty[s], ph ^ 1, ab));
       if (!ok) break;
       uint8_t *xdst = smem + s * s_stage;
-      // 64-byte rows; the 64-byte swizzle XORs the 16-byte chunk index with
-      // bits 1-2 of the row
+      // 128-byte rows; the 128-byte swizzle XORs the 16-byte chunk index with
+      // bits 0-2 of the row
 #pragma unroll
       for (int u = 0; u < 2; ++u) {
         const int r = t + u * 64;
 #pragma unroll
-        for (int j = 0; j < 4; ++j)
-          cp_async16_zfill(xdst + r * 64 + ((j ^ ((r >> 1) & 3)) << 4), src_row[u] + kc * CK + j * 8,
+        for (int j = 0; j < 8; ++j)
+          cp_async16_zfill(xdst + r * 128 + ((j ^ (r & 7)) << 4), src_row[u] + kc * CK + j * 8,
                            src_bytes[u]);
       }
       cp_async_commit();
@@ -559,7 +554,7 @@ l3_status launch_attn_dense(const l3_plan_s *p, const void *x, const void *W_K, 
   const l3_dims_t &d = p->dims;
   CUtensorMap mK, mV;
   l3_status st;
-  if ((st = make_map_2d16(&mK, W_K, true, d.v, d.d_in, d.d_in, CK, 64, 64)) != L3_OK) return st;
+  if ((st = make_map_2d16(&mK, W_K, true, d.v, d.d_in, d.d_in, CK, 64, 128)) != L3_OK) return st;
   if ((st = make_map_2d16(&mV, W_V, true, d.v, d.d_emb, d.d_emb, 64, V_ROWS, 128)) != L3_OK)
     return st;
   DenseParams P;
