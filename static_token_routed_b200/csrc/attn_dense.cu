@@ -196,7 +196,7 @@ __global__ void __launch_bounds__(DENSE_THREADS, DenseCfg<SMALL>::MIN_BLOCKS)
     mbar_init(&b->ofull, 1);
     for (int i = 0; i < MAX_STAGES; ++i) {
       mbar_init(&b->vfull[i], 1);
-      mbar_init(&b->vconv[i], 8);
+      mbar_init(&b->vconv[i], 1);
       mbar_init(&b->vempty[i], 1);
     }
     mbar_init(&b->odrained, 8);
@@ -447,21 +447,25 @@ __global__ void __launch_bounds__(DENSE_THREADS, DenseCfg<SMALL>::MIN_BLOCKS)
     ok = softmax_sync_and(ok);
     if (ok) inv_sum = 1.0f / (b->red_sum[0][r] + b->red_sum[1][r]);
 
-    const int eth = sw * 32 + lane;  // 0..255
     __half *arow = P.a + (r < n_valid ? (int64_t)P.perm[tok0 + r] * P.d_emb : 0);
     for (int h = 0; ok && h < n_op; ++h) {
       const int o_w = min(o_max, P.d_emb - h * o_max);
-      // this pass's V slices: bf16 -> fp16 in place, then hand them to the MMA warp
+      // this pass's V slices: bf16 -> fp16 in place, then hand them to the MMA
+      // warp. Warp sw owns ring slot sw (n_v <= 8) and converts every slice
+      // that lands there, in order, so the slices in the ring are converted
+      // side by side, each by one warp, instead of one after another by all
+      // eight (a chain of waits and proxy fences per slice); a warp never
+      // waits on a slot phase more than one ahead of the one it last saw.
       const int v_vecs = V_ROWS * o_w / 8;
-      for (int vc = 0; vc < n_vc; ++vc) {
-        const int gv = h * n_vc + vc;
+      for (int gv = h * n_vc; gv < (h + 1) * n_vc; ++gv) {
         const int i = gv % n_v;
+        if (i != sw) continue;
         const uint32_t ph = (gv / n_v) & 1;
         ok = __all_sync(0xffffffffu, mbar_wait(&b->vfull[i], ph, ab));
         if (!ok) break;
         uint4 *vb = reinterpret_cast<uint4 *>(vbuf + i * v_bytes);
         bool bad = false;
-        for (int e = eth; e < v_vecs; e += 256) {
+        for (int e = lane; e < v_vecs; e += 32) {
           uint4 w = vb[e];
           const __nv_bfloat162 *in = reinterpret_cast<const __nv_bfloat162 *>(&w);
           uint4 o;
