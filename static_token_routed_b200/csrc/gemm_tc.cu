@@ -4,12 +4,15 @@
 //   h = LayerNorm(W_up a)                      (W_up: d_up x d_emb)
 //   y = W_mix [h ; x] = W_mix[:, :d_up] h + W_mix[:, d_up:] x
 //
-// k_mix_gemm: persistent, warp-specialised. Warp 0 streams 128x64 A tiles and
-// 256x64 B tiles into a 4-stage shared-memory ring with TMA; warp 1 issues
-// tcgen05.mma (M=128, N=256, K=16) into one of two TMEM accumulators; warps
-// 2-5 drain the other accumulator (tcgen05.ld) and store y while the next
-// tile's MMAs run. The two K-ranges of W_mix (the LayerNorm output h, then x)
-// accumulate into the same TMEM tile, so the concat [h ; x] never exists.
+// k_mix_gemm_pair: persistent, warp-specialised, on CTA pairs (cta_group::2).
+// A pair computes a 256 x 256 tile of y: warp 0 of each CTA streams its own
+// 128x64 A tiles and 128x64 half of the pair's B tiles into a 6-stage ring
+// with TMA; warp 1 of the pair's first CTA issues tcgen05.mma (M=256, N=256,
+// K=16) into one of two TMEM accumulators (each CTA's TMEM holds its 128
+// rows); warps 2-5 of each CTA drain the other accumulator and store y while
+// the next tile's MMAs run. The two K-ranges of W_mix (the LayerNorm output h,
+// then x) accumulate into the same TMEM tile, so the concat [h ; x] never
+// exists.
 //
 // k_up_ln_gemm: W_up a with the LayerNorm fused into the epilogue. A cluster
 // of ceil(d_up / 256) CTAs covers one 128-token tile's whole d_up row: each
@@ -40,11 +43,9 @@ constexpr int BN = 256;  // output columns per tile (max N of one MMA)
 constexpr int A_BYTES = BM * BK * 2;
 constexpr int B_BYTES = BN * BK * 2;
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-constexpr int MIX_STAGES = 4;
 constexpr int UP_STAGES = 2;  // two CTAs per SM: one drains its epilogue while the other computes
 constexpr int GEMM_THREADS = 192;  // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
 constexpr uint32_t IDESC_F16 = idesc_f16(0, 0, BM, BN);
-constexpr uint32_t IDESC_BF16 = idesc_f16(1, 0, BM, BN);
 
 struct MixParams {
   int M, N;        // tokens, d_out
@@ -102,26 +103,84 @@ __device__ void drain_after_abort(Bars *b, int stages, const uint32_t *armed_par
 }
 
 // ---------------------------------------------------------------------------
-// y = W_mix[:, :d_up] h + W_mix[:, d_up:] x
+// y = W_mix[:, :d_up] h + W_mix[:, d_up:] x on CTA pairs (tcgen05 cta_group::2)
+//
+// Two CTAs on neighbouring SMs compute one 256 x 256 tile of y: each loads its
+// own 128 rows of the A operand (h or x) and its own 128 of the 256 rows of
+// W_mix, and the pair's first CTA issues M = 256 MMAs that read both CTAs'
+// shared memory and accumulate each CTA's 128 rows in its own TMEM. Per SM
+// this moves 32 KB per 64-wide k-block instead of 48 KB (B is split between
+// the two SMs instead of loaded by each), and a 32 KB stage lets six stages
+// fit instead of four.
 // ---------------------------------------------------------------------------
+constexpr int MIX2_STAGES = 6;
+constexpr int B2_ROWS = 128;                    // W_mix rows per CTA of a pair
+constexpr int STAGE2_BYTES = A_BYTES + B2_ROWS * BK * 2;
+constexpr uint32_t IDESC2_F16 = idesc_f16(0, 0, 2 * BM, BN);
+constexpr uint32_t IDESC2_BF16 = idesc_f16(1, 0, 2 * BM, BN);
+
+__device__ __forceinline__ void mbar_arrive_expect_tx_cluster(uint32_t cluster_addr,
+                                                              uint32_t bytes) {
+  // default (CTA-scope release) semantics: a cluster-scope release here is a
+  // full memory fence per stage, which starved the pipeline
+  asm volatile("mbarrier.arrive.expect_tx.shared::cluster.b64 _, [%0], %1;" ::"r"(
+                   cluster_addr),
+               "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
+               : "memory");
+}
+// TMA load into this CTA's shared memory whose completion is counted on an
+// mbarrier of either CTA of the pair (no multicast)
+__device__ __forceinline__ void tma_load_2d_pair(void *dst, const CUtensorMap *map,
+                                                 uint32_t bar_cluster_addr, int x, int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(map), "r"(bar_cluster_addr), "r"(x), "r"(y)
+      : "memory");
+}
+__device__ __forceinline__ void umma_f16_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                              uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// arrive on `bar` (same offset) in both CTAs of the pair once every MMA issued
+// so far by this thread has completed
+__device__ __forceinline__ void umma_commit_pair(uint64_t *bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+      " [%0], %1;" ::"r"(smem_u32(bar)),
+      "h"((uint16_t)3)
+      : "memory");
+}
+
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
-    k_mix_gemm(const __grid_constant__ CUtensorMap mA0, const __grid_constant__ CUtensorMap mB0,
-               const __grid_constant__ CUtensorMap mA1, const __grid_constant__ CUtensorMap mB1,
-               MixParams P) {
+    k_mix_gemm_pair(const __grid_constant__ CUtensorMap mA0, const __grid_constant__ CUtensorMap mB0,
+                    const __grid_constant__ CUtensorMap mA1, const __grid_constant__ CUtensorMap mB1,
+                    MixParams P) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = align1024(smem_raw);
   uint8_t *ring = smem;
-  Bars *b = reinterpret_cast<Bars *>(smem + MIX_STAGES * STAGE_BYTES);
+  Bars *b = reinterpret_cast<Bars *>(smem + MIX2_STAGES * STAGE2_BYTES);
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const uint32_t rank = cluster_ctarank();  // 0 issues the MMAs
+  const int pair_id = blockIdx.x / 2, n_pairs = gridDim.x / 2;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < MIX_STAGES; ++s) {
-      mbar_init(&b->full[s], 1);
-      mbar_init(&b->empty[s], 1);
+    for (int s = 0; s < MIX2_STAGES; ++s) {
+      mbar_init(&b->full[s], 2);   // used in CTA 0: one arrival per CTA, plus both CTAs' bytes
+      mbar_init(&b->empty[s], 1);  // MMA completion, signalled in both CTAs
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&b->tfull[a], 1);
-      mbar_init(&b->tempty[a], 4);
+      mbar_init(&b->tempty[a], 8);  // used in CTA 0: four epilogue warps of each CTA
     }
     mbar_init(&b->drain, 1);
     b->abort_flag = 0;
@@ -132,11 +191,15 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     prefetch_tensormap(&mB1);
   }
   if (warp == 1) {
-    tmem_alloc(&b->tmem_base, 2 * BN);
-    tmem_relinquish();
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(&b->tmem_base)),
+                 "r"(2 * BN)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
   }
   tc_fence_before();
   __syncthreads();
+  cluster_sync();  // both CTAs' barriers initialised before any cross-CTA signal
   tc_fence_after();
   const uint32_t tmem = b->tmem_base;
   const Abort ab{&b->abort_flag, P.err};
@@ -146,44 +209,47 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     if (elect_one()) {
       int stage = 0;
       uint32_t phase = 0;
-      uint32_t armed_parity[MIX_STAGES];
-      bool armed[MIX_STAGES];
-      for (int s = 0; s < MIX_STAGES; ++s) armed[s] = false;
+      uint32_t armed_parity[MIX2_STAGES];
+      bool armed[MIX2_STAGES];
+      for (int s = 0; s < MIX2_STAGES; ++s) armed[s] = false;
       bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < P.n_tiles; tile += gridDim.x) {
-        const int m0 = (tile / P.n_tiles_n) * BM;
-        const int n0 = (tile % P.n_tiles_n) * BN;
+      for (int tile = pair_id; ok && tile < P.n_tiles; tile += n_pairs) {
+        const int m0 = (tile / P.n_tiles_n) * (2 * BM) + (int)rank * BM;
+        const int n0 = (tile % P.n_tiles_n) * BN + (int)rank * B2_ROWS;
         for (int kb = 0; kb < n_kb; ++kb) {
           if (!mbar_wait(&b->empty[stage], phase ^ 1, ab)) {
             ok = false;
             break;
           }
-          uint8_t *sa = ring + stage * STAGE_BYTES;
-          mbar_arrive_expect_tx(&b->full[stage], STAGE_BYTES);
+          uint8_t *sa = ring + stage * STAGE2_BYTES;
+          const uint32_t full0 = map_shared_rank(&b->full[stage], 0);
+          mbar_arrive_expect_tx_cluster(full0, STAGE2_BYTES);
           armed[stage] = true;
           armed_parity[stage] = phase;
           if (kb < P.kb0) {
-            tma_load_2d(sa, &mA0, &b->full[stage], kb * BK, m0);
-            tma_load_2d(sa + A_BYTES, &mB0, &b->full[stage], kb * BK, n0);
+            tma_load_2d_pair(sa, &mA0, full0, kb * BK, m0);
+            tma_load_2d_pair(sa + A_BYTES, &mB0, full0, kb * BK, n0);
           } else {
-            tma_load_2d(sa, &mA1, &b->full[stage], (kb - P.kb0) * BK, m0);
-            tma_load_2d(sa + A_BYTES, &mB1, &b->full[stage], (kb - P.kb0) * BK, n0);
+            tma_load_2d_pair(sa, &mA1, full0, (kb - P.kb0) * BK, m0);
+            tma_load_2d_pair(sa + A_BYTES, &mB1, full0, (kb - P.kb0) * BK, n0);
           }
-          if (++stage == MIX_STAGES) {
+          if (++stage == MIX2_STAGES) {
             stage = 0;
             phase ^= 1;
           }
         }
       }
-      if (!ok) drain_after_abort(b, MIX_STAGES, armed_parity, armed, true, false, ab);
+      // after a give-up CTA 0 waits for the phases it armed, which complete
+      // only once both CTAs' copies have landed
+      if (!ok && rank == 0) drain_after_abort(b, MIX2_STAGES, armed_parity, armed, true, false, ab);
     }
   } else if (warp == 1) {
-    if (elect_one()) {
+    if (rank == 0 && elect_one()) {
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
       int it = 0;
-      for (int tile = blockIdx.x; ok && tile < P.n_tiles; tile += gridDim.x, ++it) {
+      for (int tile = pair_id; ok && tile < P.n_tiles; tile += n_pairs, ++it) {
         const int acc = it & 1;
         if (!mbar_wait(&b->tempty[acc], ((it >> 1) & 1) ^ 1, ab)) {
           ok = false;
@@ -197,34 +263,43 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             break;
           }
           tc_fence_after();
-          const uint32_t sa = smem_u32(ring + stage * STAGE_BYTES);
+          const uint32_t sa = smem_u32(ring + stage * STAGE2_BYTES);
           const uint32_t sb = sa + A_BYTES;
-          const uint32_t idesc = kb < P.kb0 ? IDESC_F16 : IDESC_BF16;
+          const uint32_t idesc = kb < P.kb0 ? IDESC2_F16 : IDESC2_BF16;
 #pragma unroll
           for (int k = 0; k < BK / 16; ++k)
-            umma_f16(d, sdesc_sw128(sa + k * 32, 16, 1024), sdesc_sw128(sb + k * 32, 16, 1024),
-                     idesc, (kb | k) != 0);
-          umma_commit(&b->empty[stage]);
-          if (++stage == MIX_STAGES) {
+            umma_f16_pair(d, sdesc_sw128(sa + k * 32, 16, 1024), sdesc_sw128(sb + k * 32, 16, 1024),
+                          idesc, (kb | k) != 0);
+          umma_commit_pair(&b->empty[stage]);
+          if (++stage == MIX2_STAGES) {
             stage = 0;
             phase ^= 1;
           }
         }
-        if (ok) umma_commit(&b->tfull[acc]);
+        if (ok) umma_commit_pair(&b->tfull[acc]);
       }
-      if (!ok) drain_after_abort(b, MIX_STAGES, nullptr, nullptr, false, true, ab);
+      if (!ok) {
+        umma_commit_pair(&b->drain);
+        const uint32_t a = smem_u32(&b->drain);
+        const uint64_t t0 = globaltimer_ns();
+        while (!mbar_try_wait(a, 0) && globaltimer_ns() - t0 < WAIT_LIMIT_NS) {
+        }
+      }
     }
   } else {
-    // epilogue: warp (2..5) % 4 selects the TMEM lane quarter it may read
+    // epilogue: warp (2..5) % 4 selects the TMEM lane quarter it may read;
+    // each CTA drains its own 128 rows of the pair's tile
     const int q = warp & 3;
     const int r = q * 32 + lane;
+    const uint32_t tempty0[2] = {map_shared_rank(&b->tempty[0], 0),
+                                 map_shared_rank(&b->tempty[1], 0)};
     int it = 0;
-    for (int tile = blockIdx.x; tile < P.n_tiles; tile += gridDim.x, ++it) {
+    for (int tile = pair_id; tile < P.n_tiles; tile += n_pairs, ++it) {
       const int acc = it & 1;
       const bool got = __all_sync(0xffffffffu, mbar_wait(&b->tfull[acc], (it >> 1) & 1, ab));
       if (!got) break;
       tc_fence_after();
-      const int m = (tile / P.n_tiles_n) * BM + r;
+      const int m = (tile / P.n_tiles_n) * (2 * BM) + (int)rank * BM + r;
       const int n0 = (tile % P.n_tiles_n) * BN;
       __nv_bfloat16 *yrow = P.y + (int64_t)m * P.ldy + n0;
 #pragma unroll 1
@@ -250,15 +325,17 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&b->tempty[acc]);
+      if (lane == 0) mbar_arrive_cluster(tempty0[acc]);
     }
   }
   __syncwarp();
   tc_fence_before();
   __syncthreads();
+  cluster_sync();  // no signal crosses between the CTAs after this
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, 2 * BN);
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(2 * BN)
+                 : "memory");
   }
 }
 
@@ -615,7 +692,7 @@ int num_sms() {
   return g_num_sms[dev];
 }
 
-constexpr size_t MIX_SMEM = 1024 + MIX_STAGES * STAGE_BYTES + sizeof(Bars);
+constexpr size_t MIX2_SMEM = 1024 + MIX2_STAGES * STAGE2_BYTES + sizeof(Bars);
 constexpr size_t UP_SMEM =
     1024 + UP_STAGES * STAGE_BYTES + sizeof(Bars) + (2 * BN + 4 * BM + 2 * 8 * BM) * sizeof(float);
 static_assert(UP_STAGES * STAGE_BYTES >= (BN / 64) * BM * 128, "h staging fits the stage ring");
@@ -718,17 +795,19 @@ l3_status launch_mix_tc(const l3_plan_s *p, const void *x, const void *W_mix, vo
   CUtensorMap mA0, mB0, mA1, mB1;
   l3_status st;
   const uint64_t M = p->n_tokens;
+  // A: 128-row boxes of h and x (each CTA of a pair loads its own rows);
+  // B: 128-row halves of the pair's 256 W_mix rows
   if ((st = make_map(&mA0, p->h_buf, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, M, d.d_up, d.d_up, BM)) !=
       L3_OK)
     return st;
   if ((st = make_map(&mB0, p->w_mixh16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, d.d_out, d.d_up, d.d_up,
-                     BN)) != L3_OK)
+                     B2_ROWS)) != L3_OK)
     return st;
   if ((st = make_map(&mA1, x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, M, d.d_in, d.d_in, BM)) != L3_OK)
     return st;
   const __nv_bfloat16 *wx = reinterpret_cast<const __nv_bfloat16 *>(W_mix) + d.d_up;
   if ((st = make_map(&mB1, wx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, d.d_out, d.d_in, d.d_up + d.d_in,
-                     BN)) != L3_OK)
+                     B2_ROWS)) != L3_OK)
     return st;
   MixParams P;
   P.M = (int)M;
@@ -736,20 +815,32 @@ l3_status launch_mix_tc(const l3_plan_s *p, const void *x, const void *W_mix, vo
   P.kb0 = (int)(d.d_up / BK);
   P.kb1 = (int)(d.d_in / BK);
   P.n_tiles_n = (int)((d.d_out + BN - 1) / BN);
-  P.n_tiles = (int)((M + BM - 1) / BM) * P.n_tiles_n;
+  P.n_tiles = (int)((M + 2 * BM - 1) / (2 * BM)) * P.n_tiles_n;
   P.y = reinterpret_cast<__nv_bfloat16 *>(y);
   P.ldy = d.d_out;
   P.err = p->dev_flags + 1;
   static bool attr[64] = {};
   if (!attr[p->device & 63]) {
-    L3_CUDA_TRY(cudaFuncSetAttribute(k_mix_gemm, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     (int)MIX_SMEM));
+    L3_CUDA_TRY(cudaFuncSetAttribute(k_mix_gemm_pair, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)MIX2_SMEM));
     attr[p->device & 63] = true;
   }
-  const int grid = std::min(P.n_tiles, num_sms());
+  // persistent: one CTA pair per two SMs, 256 x 256 tiles
+  const int pairs = std::min(P.n_tiles, num_sms() / 2);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * pairs, 1, 1);
+  cfg.blockDim = dim3(GEMM_THREADS, 1, 1);
+  cfg.dynamicSmemBytes = MIX2_SMEM;
+  cfg.stream = s;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = 2;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
   LaunchTimer t("mix_gemm_tc", s);
-  k_mix_gemm<<<grid, GEMM_THREADS, MIX_SMEM, s>>>(mA0, mB0, mA1, mB1, P);
-  L3_CUDA_TRY(cudaGetLastError());
+  L3_CUDA_TRY(cudaLaunchKernelEx(&cfg, k_mix_gemm_pair, mA0, mB0, mA1, mB1, P));
   return L3_OK;
 }
 
