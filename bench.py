@@ -81,7 +81,9 @@ def attention_flops(ids: np.ndarray, offsets: np.ndarray, w: wl.Workload) -> int
 #       --clock-control none -k regex:<kernel> -s 3 -c 1
 #       python bench.py --workload <w> --steps 1 --warmup 3 --no-e2e --cpu-seconds 0
 # keyed by (kernel, workload, tokens); remove an entry when its kernel changes
-TRAFFIC = {}
+TRAFFIC = {
+    ("mix_gemm_tc", "paper_shaped", 65536): 572293888 + 249231360,
+}
 
 
 # per-kernel roofline: what each kernel must move or compute per launch
