@@ -59,6 +59,9 @@ def algorithmic_work(w: wl.Workload, info) -> dict:
     n = w.n_tokens
     k_bytes = info.unique_rows_multi * w.d_in * el      # K_t rows read (d_t > 1 groups)
     v_bytes = info.unique_rows * w.d_emb * el           # V_t rows read
+    if w.tied:
+        # one table: every unique row is read once and serves as key and value
+        k_bytes, v_bytes = info.unique_rows * w.d_in * el, 0
     x_bytes = n * w.d_in * el
     y_bytes = n * w.d_out * el
     w_bytes = (w.d_up * w.d_emb + 2 * w.d_up + w.d_out * (w.d_up + w.d_in)) * el
@@ -243,7 +246,7 @@ def job_throughput(tokens_per_rank: int, world: int, ms_max: float) -> float:
 def config_of(w, args):
     return {"workload": w.name, "global_batch": w.n_tokens * args.gpus, "tokens_per_gpu": w.n_tokens,
             "vocab": w.vocab, "v": w.v, "k": w.k, "d_in": w.d_in, "d_emb": w.d_emb,
-            "d_up": w.d_up, "d_out": w.d_out, "alloc": w.alloc, "ids": w.ids,
+            "d_up": w.d_up, "d_out": w.d_out, "alloc": w.alloc, "ids": w.ids, "tied": w.tied,
             "parallelism": f"dp{args.gpus}",
             "l2": "no flush: per-step working set (W_K/W_V rows, x, y, weights) >> 126 MB L2"}
 
@@ -290,8 +293,10 @@ def main():
     # each rank: same tables, its own batch
     w = rank_workload(base, rank)
     tables, batch = wl.make_tables(w), wl.make_batch(w)
-    d = {k: getattr(tables, k).to(dev) for k in ("offsets", "W_K", "W_V", "W_up", "ln_gamma",
+    d = {k: getattr(tables, k).to(dev) for k in ("offsets", "W_K", "W_up", "ln_gamma",
                                                  "ln_beta", "W_mix")}
+    # a tied workload passes one device table as keys and values
+    d["W_V"] = d["W_K"] if tables.W_V is tables.W_K else tables.W_V.to(dev)
     ids_d, x_d = batch.ids.to(dev), batch.x.to(dev)
     y_d = torch.empty(w.n_tokens, w.d_out, dtype=w.torch_dtype, device=dev)
     dims = l3.make_dims(w.vocab, w.v, w.k, w.d_in, w.d_emb, w.d_up, w.d_out, w.torch_dtype, EPS)
@@ -408,6 +413,27 @@ def main():
                "d2h_bytes_per_step": int(y_h[0].numel() * y_h[0].element_size()),
                "copies": "own streams, double-buffered: overlap the previous and next steps"}
 
+    # ---- forward alone: one plan, K forwards (the sort done ahead of time) ----
+    plan_f = l3.l3_plan(ids_d, d["offsets"], dims, stream)
+    for _ in range(3):
+        l3.l3_forward(x_d, plan_f, d["W_K"], d["W_V"], d["W_up"], d["ln_gamma"], d["ln_beta"],
+                      d["W_mix"], y_d, stream)
+    barrier()
+    torch.cuda.synchronize(dev)
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    f0.record(stream)
+    for _ in range(args.steps):
+        l3.l3_forward(x_d, plan_f, d["W_K"], d["W_V"], d["W_up"], d["ln_gamma"], d["ln_beta"],
+                      d["W_mix"], y_d, stream)
+    f1.record(stream)
+    torch.cuda.synchronize(dev)
+    l3.l3_forward_status(plan_f)
+    plan_f.destroy()
+    barrier()
+    fwd_ms = max_over_ranks(f0.elapsed_time(f1) / args.steps, dist, dev)
+    fwd_only = {"value": job_throughput(w.n_tokens, world, fwd_ms), "unit": "tokens/s",
+                "ms_per_step": fwd_ms, "note": "l3_forward alone on a plan built ahead of time"}
+
     if rank != 0:
         if dist is not None:
             dist.destroy_process_group()
@@ -455,6 +481,14 @@ def main():
         cpu = {"value": n_s / dt, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                "sample": f"{n_s} random tokens of the {w.name} batch in chunks of 256 "
                          f"(fp64 oracle, {dt:.1f} s)"}
+        if w.n_tokens <= 4096:
+            # small batches: the whole batch on one host thread as well
+            import oracle  # test infrastructure: CPU-baseline leg only
+            t0 = time.perf_counter()
+            oracle.forward(batch.ids, tables.offsets, batch.x, tables.W_K, tables.W_V, tables.W_up,
+                           tables.ln_gamma, tables.ln_beta, tables.W_mix, EPS, n_threads=1)
+            cpu["single_thread"] = {"value": w.n_tokens / (time.perf_counter() - t0),
+                                    "unit": "tokens/s", "sample": "the whole batch"}
 
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max,
@@ -463,7 +497,7 @@ def main():
             "config": config_of(w, args), "clocks": clocks.summary(), "e2e": e2e,
             "gpu_launches": int(sum(n for n, _ in kernels.values())),
             "roofline": roof, "step_roofline": step_roof, "kernels": kern,
-            "cpu_baseline": cpu,
+            "cpu_baseline": cpu, "forward_only": fwd_only,
             "pipelining": "batch i+1's l3_plan on its own stream overlaps batch i's l3_forward",
             "plan": {"groups": info.n_groups, "dense_groups": info.n_dense_groups,
                      "dense_tiles": info.n_dense_tiles, "tail_items": info.n_tail_items,

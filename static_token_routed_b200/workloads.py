@@ -54,6 +54,7 @@ class Workload:
     table_seed: int     # seed of the allocation and of the weight tables
     batch_seed: int     # seed of token IDs and x
     zipf_s: float = 1.1
+    tied: bool = False  # W_V is W_K (one table serves as keys and values; d_in = d_emb)
 
     @property
     def torch_dtype(self) -> torch.dtype:
@@ -86,6 +87,11 @@ WORKLOADS = {
         # d_t = 4 for every ID, uniform IDs: every group is short
         Workload("uniform", n_tokens=131072, table_seed=4, batch_seed=4,
                  **_cfg2(alloc="uniform", ids="uniform")),
+        # paper-shaped allocation and batch with one table for keys and values
+        # (d_in = d_emb = 512)
+        Workload("paper_tied", vocab=180000, v=710000, k=512, d_in=512, d_emb=512,
+                 d_up=2048, d_out=2048, n_tokens=65536, dtype="bf16", alloc="zipf",
+                 ids="zipf", table_seed=5, batch_seed=5, tied=True),
     ]
 }
 
@@ -241,10 +247,13 @@ def make_tables(w: Workload) -> Tables:
     dt = w.torch_dtype
     s = w.table_seed
     off = torch.from_numpy(offsets_from_allocation(allocation(w)))
+    W_K = normal_tensor(s, "W_K", (w.v, w.d_in), w.d_in ** -0.5, dt)
+    if w.tied and w.d_in != w.d_emb:
+        raise ValueError("a tied workload needs d_in == d_emb")
     return Tables(
         offsets=off,
-        W_K=normal_tensor(s, "W_K", (w.v, w.d_in), w.d_in ** -0.5, dt),
-        W_V=normal_tensor(s, "W_V", (w.v, w.d_emb), w.d_emb ** -0.5, dt),
+        W_K=W_K,
+        W_V=W_K if w.tied else normal_tensor(s, "W_V", (w.v, w.d_emb), w.d_emb ** -0.5, dt),
         W_up=normal_tensor(s, "W_up", (w.d_up, w.d_emb), w.d_emb ** -0.5, dt),
         ln_gamma=torch.ones(w.d_up, dtype=dt),
         ln_beta=torch.zeros(w.d_up, dtype=dt),

@@ -26,7 +26,9 @@ def host_workload(name: str, n_tokens: int | None = None, batch_seed: int | None
 
 def to_device(tables: wl.Tables, batch: wl.Batch, device="cuda"):
     dev = {k: getattr(tables, k).to(device) for k in
-           ("offsets", "W_K", "W_V", "W_up", "ln_gamma", "ln_beta", "W_mix")}
+           ("offsets", "W_K", "W_up", "ln_gamma", "ln_beta", "W_mix")}
+    # a tied workload passes one device table as keys and values
+    dev["W_V"] = dev["W_K"] if tables.W_V is tables.W_K else tables.W_V.to(device)
     dev["ids"] = batch.ids.to(device)
     dev["x"] = batch.x.to(device)
     return dev
@@ -69,3 +71,26 @@ def sample_tokens(ids: np.ndarray, offsets: np.ndarray, n_sample: int, seed: int
 def rel_max_err(got: np.ndarray, want: np.ndarray) -> float:
     rms = float(np.sqrt(np.mean(want ** 2)))
     return float(np.max(np.abs(got - want))) / rms
+
+
+def bf16_half_ulp(v: np.ndarray) -> np.ndarray:
+    """Half the bf16 spacing at |v| (8 significant bits): the largest error of
+    rounding v itself to bf16."""
+    e = np.floor(np.log2(np.maximum(np.abs(v), np.finfo(np.float64).tiny)))
+    return 0.5 * np.exp2(e - 7)
+
+
+def rounding_floor(want: np.ndarray) -> float:
+    """max |bf16(want) - want| / RMS(want): the error of the exact result
+    rounded once to bf16, which no bf16 output can beat."""
+    rms = float(np.sqrt(np.mean(want ** 2)))
+    rounded = torch.from_numpy(want).to(torch.bfloat16).double().numpy()
+    return float(np.max(np.abs(rounded - want))) / rms
+
+
+def within_bf16_bar(got: np.ndarray, want: np.ndarray, tol: float) -> bool:
+    """Per element |got - want| <= tol * RMS(want) + bf16_half_ulp(want): the
+    bar with the output's own final bf16 rounding excepted. Used where the
+    exactly rounded result itself exceeds tol * RMS."""
+    rms = float(np.sqrt(np.mean(want ** 2)))
+    return bool(np.all(np.abs(got - want) <= tol * rms + bf16_half_ulp(want)))

@@ -12,8 +12,8 @@ import torch
 
 import oracle
 import static_token_routed_b200 as l3
-from l3_cases import (EPS, TOL, dims_of, host_workload, rel_max_err, run_forward,
-                      sample_tokens, to_device)
+from l3_cases import (EPS, TOL, dims_of, host_workload, rel_max_err, rounding_floor,
+                      run_forward, sample_tokens, to_device, within_bf16_bar)
 from static_token_routed_b200 import workloads as wl
 
 pytestmark = pytest.mark.gpu
@@ -34,17 +34,25 @@ def test_tiny_fp32_all_tokens():
 
 @pytest.mark.parametrize("name,n_tokens", [("small_bf16", 2048), ("decode", None),
                                            ("dense_stress", 4096), ("uniform", 4096),
-                                           ("paper_shaped", 1024)])
+                                           ("paper_shaped", 1024), ("paper_tied", 2048)])
 def test_reduced_batch_all_tokens(name, n_tokens):
     """Full tables, a batch small enough for the oracle on every token."""
     w, t, b = host_workload(name, n_tokens)
     y, plan = run_forward(w, to_device(t, b))
     want = oracle_y(t, b)
-    err = rel_max_err(y.double().cpu().numpy(), want)
-    assert err <= TOL[w.dtype], err
+    got = y.double().cpu().numpy()
+    err = rel_max_err(got, want)
+    if w.dtype == "bf16" and rounding_floor(want) > TOL["bf16"]:
+        # the exact result rounded to bf16 is itself over the bar on this
+        # batch (its largest outputs sit far above the RMS); hold the GPU to
+        # the bar plus the unavoidable half-ulp of that final rounding
+        assert within_bf16_bar(got, want, TOL["bf16"]), (err, rounding_floor(want))
+    else:
+        assert err <= TOL[w.dtype], err
 
 
-@pytest.mark.parametrize("name", ["small_bf16", "paper_shaped", "dense_stress", "uniform"])
+@pytest.mark.parametrize("name", ["small_bf16", "paper_shaped", "dense_stress", "uniform",
+                                  "paper_tied"])
 def test_full_size_sampled(name):
     w, t, b = host_workload(name)
     y, plan = run_forward(w, to_device(t, b))
@@ -52,7 +60,10 @@ def test_full_size_sampled(name):
     want = oracle_y(t, b, select=sel)
     got = y[torch.from_numpy(sel).cuda()].double().cpu().numpy()
     err = rel_max_err(got, want)
-    assert err <= TOL[w.dtype], err
+    if w.dtype == "bf16" and rounding_floor(want) > TOL["bf16"]:
+        assert within_bf16_bar(got, want, TOL["bf16"]), (err, rounding_floor(want))
+    else:
+        assert err <= TOL[w.dtype], err
     assert torch.isfinite(y.float()).all()
 
 

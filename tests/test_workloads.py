@@ -54,3 +54,15 @@ def test_normal_tensor_independent_of_threads():
     b = wl.normal_tensor(3, "W_K", (3 * (1 << 24) // 1000 + 5, 1000), 0.5, torch.bfloat16, threads=8)
     assert torch.equal(a, b)
     assert abs(float(a.float().std()) - 0.5) < 0.01
+
+
+def test_tied_tables_share_one_tensor():
+    """A tied workload (one table as keys and values: the W_K / W_V tying
+    row of the papernotes page's ablation table, 消融实验) hands out the same
+    tensor twice."""
+    import dataclasses
+    w = dataclasses.replace(wl.WORKLOADS["paper_tied"], vocab=300, v=1200, k=16, n_tokens=64)
+    t = wl.make_tables(w)
+    assert t.W_V is t.W_K and t.W_K.shape == (1200, 512)
+    with pytest.raises(ValueError):
+        wl.make_tables(dataclasses.replace(w, d_emb=256))
