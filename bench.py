@@ -243,6 +243,78 @@ def job_throughput(tokens_per_rank: int, world: int, ms_max: float) -> float:
     return tokens_per_rank * world / (ms_max * 1e-3)
 
 
+def run_offload(args, w, tables, batch, dev, dist, world, rank):
+    """Tables in pinned host memory: each step plans the batch (l3_plan_staged),
+    copies its rows across PCIe into device staging tables (l3_stage_rows) and
+    runs l3_forward on them. Staging of batch i+1 overlaps the forward of i."""
+    d = {k: getattr(tables, k).to(dev) for k in ("offsets", "W_up", "ln_gamma", "ln_beta",
+                                                 "W_mix")}
+    WK = tables.W_K.pin_memory()
+    WV = WK if tables.W_V is tables.W_K else tables.W_V.pin_memory()
+    ids_d, x_d = batch.ids.to(dev), batch.x.to(dev)
+    y_d = torch.empty(w.n_tokens, w.d_out, dtype=w.torch_dtype, device=dev)
+    dims = l3.make_dims(w.vocab, w.v, w.k, w.d_in, w.d_emb, w.d_up, w.d_out, w.torch_dtype, EPS)
+    stream, side = torch.cuda.current_stream(dev), torch.cuda.Stream(dev)
+    staged_ev = [torch.cuda.Event(), torch.cuda.Event()]
+    done = [torch.cuda.Event(), torch.cuda.Event()]
+    n = [0]
+
+    def step():
+        k = n[0]
+        if k >= 2:
+            done[k % 2].synchronize()
+        plan = l3.l3_plan(ids_d, d["offsets"], dims, side, staged=True)
+        rows = plan.info().unique_rows
+        with torch.cuda.stream(side):
+            Ks = torch.empty(rows, w.d_in, dtype=w.torch_dtype, device=dev)
+            Vs = torch.empty(rows, w.d_emb, dtype=w.torch_dtype, device=dev)
+        l3.l3_stage_rows(plan, WK, WV, Ks, Vs, side)
+        staged_ev[k % 2].record(side)
+        stream.wait_event(staged_ev[k % 2])
+        l3.l3_forward(x_d, plan, Ks, Vs, d["W_up"], d["ln_gamma"], d["ln_beta"], d["W_mix"], y_d,
+                      stream)
+        Ks.record_stream(stream)
+        Vs.record_stream(stream)
+        done[k % 2].record(stream)
+        n[0] = k + 1
+        return plan
+
+    for _ in range(max(3, args.warmup)):
+        step().destroy()
+    p0 = step()
+    l3.l3_forward_status(p0)
+    rows = p0.info().unique_rows
+    p0.destroy()
+    l3.l3_profile_enable(True)
+    torch.cuda.synchronize(dev)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(dev.index or 0) as clocks:
+        ev0.record(stream)
+        side.wait_event(ev0)
+        for _ in range(args.steps):
+            step().destroy()
+        ev1.record(stream)
+        torch.cuda.synchronize(dev)
+    kernels = l3.l3_profile_read()
+    l3.l3_profile_enable(False)
+    ms = max_over_ranks(ev0.elapsed_time(ev1) / args.steps, dist, dev)
+    if rank != 0:
+        return
+    el = 2 if w.dtype == "bf16" else 4
+    staged_bytes = rows * (w.d_in + w.d_emb) * el
+    line = {"metric": METRIC, "mode": "offload", "value": job_throughput(w.n_tokens, world, ms),
+            "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "dtype": "bf16" if w.dtype == "bf16" else "fp32", "data": "synthetic",
+            "config": dict(config_of(w, args), tables="pinned host memory"),
+            "clocks": clocks.summary(),
+            "staged_rows_per_step": rows, "staged_bytes_per_step_max": staged_bytes,
+            "host_link_GBps": staged_bytes / (ms * 1e-3) / 1e9,
+            "kernels": {k: {"launches": nl, "per_step_ms": t / args.steps}
+                        for k, (nl, t) in kernels.items()}}
+    print(json.dumps(line), flush=True)
+
+
 def config_of(w, args):
     return {"workload": w.name, "global_batch": w.n_tokens * args.gpus, "tokens_per_gpu": w.n_tokens,
             "vocab": w.vocab, "v": w.v, "k": w.k, "d_in": w.d_in, "d_emb": w.d_emb,
@@ -268,6 +340,8 @@ def main():
     ap.add_argument("--tokens", type=int, default=0,
                     help="tokens per rank (default: the workload's batch size)")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--offload", action="store_true",
+                    help="W_K / W_V in pinned host memory; each step stages the batch's rows")
     args = ap.parse_args()
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -293,6 +367,9 @@ def main():
     # each rank: same tables, its own batch
     w = rank_workload(base, rank)
     tables, batch = wl.make_tables(w), wl.make_batch(w)
+    if args.offload:
+        run_offload(args, w, tables, batch, dev, dist, world, rank)
+        return
     d = {k: getattr(tables, k).to(dev) for k in ("offsets", "W_K", "W_up", "ln_gamma",
                                                  "ln_beta", "W_mix")}
     # a tied workload passes one device table as keys and values

@@ -113,6 +113,41 @@ typedef struct {
 l3_status l3_plan(const int32_t *token_ids, int64_t n_tokens, const int32_t *offsets,
                   const l3_dims_t *dims, void *stream, l3_plan_t *out);
 
+/*
+ * l3_plan_staged — l3_plan for tables kept outside device memory (CPU
+ * offload: the papernotes note, 关键设计 / CPU offload, and the sciencestack
+ * page's inference section: the rows a token needs follow from its ID alone,
+ * so they can be fetched before the layer runs).
+ *
+ * Same arguments, sort, synchronization and errors as l3_plan. The plan
+ * addresses K_t / V_t in STAGED tables holding only this batch's rows:
+ * group g's d_t rows at rows seg_rows[g] .. seg_rows[g+1]-1 (see
+ * l3_plan_export), info.unique_rows rows in all. Fill them with
+ * l3_stage_rows, then pass the staged tables to l3_forward as W_K / W_V.
+ */
+l3_status l3_plan_staged(const int32_t *token_ids, int64_t n_tokens, const int32_t *offsets,
+                         const l3_dims_t *dims, void *stream, l3_plan_t *out);
+
+/*
+ * l3_stage_rows — copy the rows of a staged plan's batch from the full
+ * tables into staged tables.
+ *
+ *   plan        from l3_plan_staged
+ *   W_K, W_V    full tables [v x d_in], [v x d_emb] (dims->dtype): device
+ *               memory, or page-locked host memory mapped into the device's
+ *               address space (cudaHostAlloc / cudaHostRegister with
+ *               mapping; the kernel reads it across PCIe)
+ *   W_K_staged  device [info.unique_rows x d_in], caller-allocated
+ *   W_V_staged  device [info.unique_rows x d_emb], caller-allocated
+ * Rows of W_K are copied only for groups with d_t > 1 (a single row's
+ * logit is never used); those staged rows are left as they were. All
+ * pointers 16-byte aligned. Enqueued on `stream`; does not synchronize.
+ * Errors: L3_ERR_INVALID_ARG (not a staged plan, NULL or misaligned
+ * pointer, wrong device), L3_ERR_CUDA.
+ */
+l3_status l3_stage_rows(l3_plan_t plan, const void *W_K, const void *W_V, void *W_K_staged,
+                        void *W_V_staged, void *stream);
+
 /* Host summary of a plan (no device work). */
 l3_status l3_plan_info(l3_plan_t plan, l3_plan_info_t *info);
 

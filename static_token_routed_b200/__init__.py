@@ -26,6 +26,8 @@ from ._binding import (  # noqa: F401
     l3_plan_destroy,
     l3_plan_export,
     l3_plan_info,
+    l3_plan_staged,
+    l3_stage_rows,
     l3_profile_enable,
     l3_profile_read,
     l3_sort_tokens_noalloc,

@@ -22,7 +22,7 @@ STATUS = {0: "L3_OK", 1: "L3_ERR_INVALID_ARG", 2: "L3_ERR_TOKEN_RANGE", 3: "L3_E
 # every symbol include/l3.h declares
 EXPORTED = ["l3_plan", "l3_plan_info", "l3_plan_export", "l3_forward", "l3_forward_status",
             "l3_plan_destroy", "l3_last_error", "l3_profile_enable", "l3_profile_read",
-            "l3_sort_tokens_noalloc"]
+            "l3_sort_tokens_noalloc", "l3_plan_staged", "l3_stage_rows"]
 L3_SORT_NOALLOC_MAX_TOKENS = 65536
 
 
@@ -64,6 +64,10 @@ def library() -> ctypes.CDLL:
     p, i64, i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
     lib.l3_plan.restype = i32
     lib.l3_plan.argtypes = [p, i64, p, ctypes.POINTER(Dims), p, ctypes.POINTER(p)]
+    lib.l3_plan_staged.restype = i32
+    lib.l3_plan_staged.argtypes = [p, i64, p, ctypes.POINTER(Dims), p, ctypes.POINTER(p)]
+    lib.l3_stage_rows.restype = i32
+    lib.l3_stage_rows.argtypes = [p, p, p, p, p, p]
     lib.l3_plan_info.restype = i32
     lib.l3_plan_info.argtypes = [p, ctypes.POINTER(PlanInfo)]
     lib.l3_plan_export.restype = i32
@@ -121,10 +125,12 @@ def make_dims(vocab, v, k, d_in, d_emb, d_up, d_out, dtype=torch.bfloat16, ln_ep
 class Plan:
     """Owns an l3_plan_t; destroyed explicitly or when garbage collected."""
 
-    def __init__(self, handle: int, dims: Dims, n_tokens: int):
+    def __init__(self, handle: int, dims: Dims, n_tokens: int, staged: bool = False):
         self.handle = handle
         self.dims = dims
         self.n_tokens = n_tokens
+        self.staged = staged  # the forward reads staged tables of the batch's rows
+        self.table_rows = l3_plan_info(self).unique_rows if staged else dims.v
 
     def info(self) -> PlanInfo:
         return l3_plan_info(self)
@@ -147,16 +153,46 @@ class Plan:
             pass
 
 
-def l3_plan(token_ids: torch.Tensor, offsets: torch.Tensor, dims: Dims, stream=None) -> Plan:
+def l3_plan(token_ids: torch.Tensor, offsets: torch.Tensor, dims: Dims, stream=None,
+            staged: bool = False) -> Plan:
+    """l3_plan, or l3_plan_staged when staged=True."""
     if token_ids.dtype != torch.int32 or offsets.dtype != torch.int32:
         raise TypeError("token_ids and offsets must be int32")
     out = ctypes.c_void_p()
     n = token_ids.numel()
-    st = library().l3_plan(_ptr(token_ids, "token_ids") if n else None, n,
-                           _ptr(offsets, "offsets"), ctypes.byref(dims),
-                           _stream(stream, offsets.device), ctypes.byref(out))
+    fn = library().l3_plan_staged if staged else library().l3_plan
+    st = fn(_ptr(token_ids, "token_ids") if n else None, n, _ptr(offsets, "offsets"),
+            ctypes.byref(dims), _stream(stream, offsets.device), ctypes.byref(out))
     _check(st)
-    return Plan(out.value, dims, n)
+    return Plan(out.value, dims, n, staged)
+
+
+def l3_plan_staged(token_ids: torch.Tensor, offsets: torch.Tensor, dims: Dims,
+                   stream=None) -> Plan:
+    return l3_plan(token_ids, offsets, dims, stream, staged=True)
+
+
+def _table_ptr(t: torch.Tensor, name: str) -> int:
+    """A device tensor, or a pinned host tensor (read by the kernel through
+    the device's mapping of it)."""
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if not (t.is_cuda or t.is_pinned()):
+        raise ValueError(f"{name} must be a CUDA tensor or pinned host memory")
+    return t.data_ptr()
+
+
+def l3_stage_rows(plan: Plan, W_K: torch.Tensor, W_V: torch.Tensor, W_K_staged: torch.Tensor,
+                  W_V_staged: torch.Tensor, stream=None) -> None:
+    d = plan.dims
+    for nm, t, shape in (("W_K", W_K, (d.v, d.d_in)), ("W_V", W_V, (d.v, d.d_emb)),
+                         ("W_K_staged", W_K_staged, (plan.table_rows, d.d_in)),
+                         ("W_V_staged", W_V_staged, (plan.table_rows, d.d_emb))):
+        if tuple(t.shape) != shape:
+            raise ValueError(f"{nm} has shape {tuple(t.shape)}, want {shape}")
+    _check(library().l3_stage_rows(plan.handle, _table_ptr(W_K, "W_K"), _table_ptr(W_V, "W_V"),
+                                   _ptr(W_K_staged, "W_K_staged"), _ptr(W_V_staged, "W_V_staged"),
+                                   _stream(stream, W_K_staged.device)))
 
 
 def l3_plan_info(plan: Plan) -> PlanInfo:
@@ -186,7 +222,8 @@ def l3_forward(x: torch.Tensor, plan: Plan, W_K, W_V, W_up, ln_gamma, ln_beta, W
         if t.dtype != want:
             raise TypeError(f"{nm} must be {want}")
     d = plan.dims
-    shapes = {"x": (plan.n_tokens, d.d_in), "W_K": (d.v, d.d_in), "W_V": (d.v, d.d_emb),
+    rows = plan.table_rows
+    shapes = {"x": (plan.n_tokens, d.d_in), "W_K": (rows, d.d_in), "W_V": (rows, d.d_emb),
               "W_up": (d.d_up, d.d_emb), "ln_gamma": (d.d_up,), "ln_beta": (d.d_up,),
               "W_mix": (d.d_out, d.d_up + d.d_in), "y": (plan.n_tokens, d.d_out)}
     for nm, t in zip(names, tensors):

@@ -199,8 +199,49 @@ extern "C" {
 
 const char *l3_last_error(void) { return g_error.c_str(); }
 
+static l3_status plan_impl(const int32_t *token_ids, int64_t n_tokens, const int32_t *offsets,
+                           const l3_dims_t *dims, void *stream, l3_plan_t *out, bool staged);
+
 l3_status l3_plan(const int32_t *token_ids, int64_t n_tokens, const int32_t *offsets,
                   const l3_dims_t *dims, void *stream, l3_plan_t *out) {
+  return plan_impl(token_ids, n_tokens, offsets, dims, stream, out, false);
+}
+
+l3_status l3_plan_staged(const int32_t *token_ids, int64_t n_tokens, const int32_t *offsets,
+                         const l3_dims_t *dims, void *stream, l3_plan_t *out) {
+  return plan_impl(token_ids, n_tokens, offsets, dims, stream, out, true);
+}
+
+l3_status l3_stage_rows(l3_plan_t p, const void *W_K, const void *W_V, void *W_K_staged,
+                        void *W_V_staged, void *stream) {
+  g_error.clear();
+  if (!p || !p->staged) {
+    set_error(p ? "l3_stage_rows needs a plan from l3_plan_staged" : "plan is NULL");
+    return L3_ERR_INVALID_ARG;
+  }
+  if (p->n_groups == 0) return L3_OK;
+  for (const void *q : {W_K, W_V, (const void *)W_K_staged, (const void *)W_V_staged}) {
+    if (!q) {
+      set_error("a table pointer is NULL");
+      return L3_ERR_INVALID_ARG;
+    }
+    if (reinterpret_cast<uintptr_t>(q) & 15u) {
+      set_error("table pointers must be 16-byte aligned");
+      return L3_ERR_INVALID_ARG;
+    }
+  }
+  int dev = -1;
+  L3_CUDA_TRY(cudaGetDevice(&dev));
+  if (dev != p->device) {
+    set_error("l3_stage_rows called on a different device than l3_plan_staged");
+    return L3_ERR_INVALID_ARG;
+  }
+  return launch_stage_rows(p, W_K, W_V, W_K_staged, W_V_staged,
+                           reinterpret_cast<cudaStream_t>(stream));
+}
+
+static l3_status plan_impl(const int32_t *token_ids, int64_t n_tokens, const int32_t *offsets,
+                           const l3_dims_t *dims, void *stream, l3_plan_t *out, bool staged) {
   g_error.clear();
   if (!out) {
     set_error("out is NULL");
@@ -227,6 +268,7 @@ l3_status l3_plan(const int32_t *token_ids, int64_t n_tokens, const int32_t *off
   }
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   auto *p = new l3_plan_s();
+  p->staged = staged;
   p->dims = *dims;
   p->n_tokens = n_tokens;
   p->stream = s;
@@ -242,6 +284,7 @@ l3_status l3_plan(const int32_t *token_ids, int64_t n_tokens, const int32_t *off
       align256(cap * 4),                                          // group_ids
       align256(cap * 4),                                          // group_tok_start
       align256(cap * 4),                                          // group_row_start
+      align256(cap * 4),                                          // group_row_src
       align256(cap * 4),                                          // group_rows
       align256(cap * 4),                                          // seg_rows
       align256((n / DENSE_TILE_M + cap) * sizeof(DenseTile)),     // dense tiles
@@ -282,6 +325,7 @@ l3_status l3_plan(const int32_t *token_ids, int64_t n_tokens, const int32_t *off
   p->group_ids = reinterpret_cast<int32_t *>(next(i++));
   p->group_tok_start = reinterpret_cast<int32_t *>(next(i++));
   p->group_row_start = reinterpret_cast<int32_t *>(next(i++));
+  p->group_row_src = reinterpret_cast<int32_t *>(next(i++));
   p->group_rows = reinterpret_cast<int32_t *>(next(i++));
   p->seg_rows = reinterpret_cast<int32_t *>(next(i++));
   p->dense_tiles = reinterpret_cast<DenseTile *>(next(i++));
@@ -290,6 +334,7 @@ l3_status l3_plan(const int32_t *token_ids, int64_t n_tokens, const int32_t *off
   p->a_buf = next(i++);
   p->h_buf = next(i++);
   p->z_buf = reinterpret_cast<float *>(next(i++));
+  const size_t scratch_idx = i;
   void *scratch = next(i++);
   p->w_up16 = next(i++);
   p->w_mixh16 = next(i++);
@@ -297,7 +342,7 @@ l3_status l3_plan(const int32_t *token_ids, int64_t n_tokens, const int32_t *off
   st = L3_OK;
   e = cudaMemsetAsync(p->dev_flags, 0, 64, s);
   if (e != cudaSuccess) st = cuda_fail(e, "cudaMemsetAsync(flags)");
-  if (st == L3_OK) st = build_plan(p, token_ids, offsets, s, scratch, sizes[14]);
+  if (st == L3_OK) st = build_plan(p, token_ids, offsets, s, scratch, sizes[scratch_idx]);
   if (st != L3_OK) {
     std::string msg = g_error;
     cache_give(p->block, p->block_bytes, p->device, s);

@@ -558,8 +558,11 @@ l3_status launch_attn_dense(const l3_plan_s *p, const void *x, const void *W_K, 
   const l3_dims_t &d = p->dims;
   CUtensorMap mK, mV;
   l3_status st;
-  if ((st = make_map_2d16(&mK, W_K, true, d.v, d.d_in, d.d_in, CK, 64, 128)) != L3_OK) return st;
-  if ((st = make_map_2d16(&mV, W_V, true, d.v, d.d_emb, d.d_emb, 64, V_ROWS, 128)) != L3_OK)
+  // rows of the tables the kernel reads: all v, or the batch's rows when staged
+  // (TMA fills rows past the end with zeros, so padding never reads past it)
+  const uint64_t rows = p->staged ? (uint64_t)p->unique_rows : (uint64_t)d.v;
+  if ((st = make_map_2d16(&mK, W_K, true, rows, d.d_in, d.d_in, CK, 64, 128)) != L3_OK) return st;
+  if ((st = make_map_2d16(&mV, W_V, true, rows, d.d_emb, d.d_emb, 64, V_ROWS, 128)) != L3_OK)
     return st;
   DenseParams P;
   P.x = reinterpret_cast<const __nv_bfloat16 *>(x);

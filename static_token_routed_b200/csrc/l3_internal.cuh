@@ -100,7 +100,9 @@ struct l3_plan_s {
   int32_t *sorted_ids = nullptr;       // [N]
   int32_t *group_ids = nullptr;        // [N+1]
   int32_t *group_tok_start = nullptr;  // [N+1]
-  int32_t *group_row_start = nullptr;  // [N+1] offsets[group_ids[g]]
+  int32_t *group_row_start = nullptr;  // [N+1] first row of group g in the table the forward reads
+  int32_t *group_row_src = nullptr;    // [N+1] offsets[group_ids[g]]: first row in the full table
+  bool staged = false;  // the forward reads a staged table (rows of group g at seg_rows[g])
   int32_t *group_rows = nullptr;       // [N+1] d_t of group g
   int32_t *seg_rows = nullptr;         // [N+1]
   l3::DenseTile *dense_tiles = nullptr;
@@ -117,6 +119,10 @@ struct l3_plan_s {
 namespace l3 {
 
 // plan kernels (plan.cu)
+// copy each group's rows of the full tables into staged tables (rows of
+// group g at seg_rows[g]); the full tables may be in mapped host memory
+l3_status launch_stage_rows(const l3_plan_s *p, const void *W_K, const void *W_V, void *K_staged,
+                            void *V_staged, cudaStream_t s);
 l3_status build_plan(l3_plan_s *p, const int32_t *token_ids, const int32_t *offsets,
                      cudaStream_t s, void *scratch, size_t scratch_bytes);
 size_t plan_scratch_bytes(int64_t n_tokens);

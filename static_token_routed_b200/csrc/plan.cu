@@ -357,6 +357,41 @@ inline int blocks_for(int64_t n, int threads) { return (int)std::max<int64_t>(1,
 
 }  // namespace
 
+// Staging copy: CTA g copies group g's rows of W_V (and of W_K when d_t > 1;
+// a single row's logit is never needed) from the full tables to rows
+// seg_rows[g].. of the staged tables, 16 bytes per thread per load, four
+// loads in flight per thread (the source may sit across PCIe).
+__global__ void k_stage_rows(const int32_t *__restrict__ group_row_src,
+                             const int32_t *__restrict__ seg_rows,
+                             const int32_t *__restrict__ group_rows,
+                             const uint4 *__restrict__ W_K, const uint4 *__restrict__ W_V,
+                             uint4 *__restrict__ K_st, uint4 *__restrict__ V_st, int k_vecs,
+                             int v_vecs) {
+  const int64_t g = blockIdx.x;  // one CTA per group of the plan
+  const int64_t src = group_row_src[g], dst = seg_rows[g];
+  const int32_t d = group_rows[g];
+  for (int pass = 0; pass < 2; ++pass) {
+    const int vecs = pass == 0 ? v_vecs : k_vecs;
+    if (pass == 1 && d == 1) break;
+    const uint4 *from = (pass == 0 ? W_V : W_K) + src * vecs;
+    uint4 *to = (pass == 0 ? V_st : K_st) + dst * vecs;
+    const int64_t total = (int64_t)d * vecs;
+    for (int64_t i = threadIdx.x; i < total; i += 4 * (int64_t)blockDim.x) {
+      uint4 r[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int64_t j = i + u * (int64_t)blockDim.x;
+        if (j < total) r[u] = from[j];
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int64_t j = i + u * (int64_t)blockDim.x;
+        if (j < total) to[j] = r[u];
+      }
+    }
+  }
+}
+
 // Scratch needed while building the plan, beyond the plan's own arrays.
 size_t plan_scratch_bytes(int64_t n) {
   int64_t tiles = std::max<int64_t>(1, (n + SORT_TILE - 1) / SORT_TILE);
@@ -485,6 +520,13 @@ l3_status build_plan(l3_plan_s *p, const int32_t *ids, const int32_t *offsets, c
                 {dcount, dcursor, n_buckets, &info[INFO_TAILS]}},
                s);
     k_class_starts<<<1, 32, 0, s>>>(dcursor, k_cap, info);
+    // keep each group's row in the full table; a staged plan addresses the
+    // group's rows where the staging copy puts them, at seg_rows[g]
+    L3_CUDA_TRY(cudaMemcpyAsync(p->group_row_src, p->group_row_start, cap * sizeof(int32_t),
+                                cudaMemcpyDeviceToDevice, s));
+    if (p->staged)
+      L3_CUDA_TRY(cudaMemcpyAsync(p->group_row_start, p->seg_rows, cap * sizeof(int32_t),
+                                  cudaMemcpyDeviceToDevice, s));
     {
       LaunchTimer t("plan_item_fill", s);
       k_item_fill<<<blocks_for(n, 256), 256, 0, s>>>(p->group_tok_start, p->group_row_start,
@@ -521,6 +563,20 @@ l3_status build_plan(l3_plan_s *p, const int32_t *ids, const int32_t *offsets, c
     p->tail_class_start[c] = n > 0 ? host_info[INFO_CLS + c] : 0;
   for (int c = 0; c < N_CLASSES; ++c)
     p->tail_class_split[c] = n > 0 ? host_info[INFO_SPLIT + c] : 0;
+  return L3_OK;
+}
+
+l3_status launch_stage_rows(const l3_plan_s *p, const void *W_K, const void *W_V, void *K_staged,
+                            void *V_staged, cudaStream_t s) {
+  if (p->n_groups == 0) return L3_OK;
+  const size_t el = p->dims.dtype == L3_BF16 ? 2 : 4;
+  const int k_vecs = (int)(p->dims.d_in * el / 16), v_vecs = (int)(p->dims.d_emb * el / 16);
+  LaunchTimer t("stage_rows", s);
+  k_stage_rows<<<(unsigned)p->n_groups, 256, 0, s>>>(
+      p->group_row_src, p->seg_rows, p->group_rows, reinterpret_cast<const uint4 *>(W_K),
+      reinterpret_cast<const uint4 *>(W_V), reinterpret_cast<uint4 *>(K_staged),
+      reinterpret_cast<uint4 *>(V_staged), k_vecs, v_vecs);
+  L3_CUDA_TRY(cudaGetLastError());
   return L3_OK;
 }
 
