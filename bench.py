@@ -243,6 +243,34 @@ def job_throughput(tokens_per_rank: int, world: int, ms_max: float) -> float:
     return tokens_per_rank * world / (ms_max * 1e-3)
 
 
+def run_lzw(args, w):
+    """Host-side LZW allocation (l3_lzw_allocate) of the workload's vocab / v /
+    k on a synthetic phrase-structured Zipf corpus; the plain-Python oracle
+    on a prefix of it is the CPU baseline."""
+    corpus = wl.zipf_corpus(w.vocab, args.lzw, seed=w.table_seed)
+    times = []
+    for _ in range(max(1, args.steps)):
+        t0 = time.perf_counter()
+        d, n_words = l3.l3_lzw_allocate(corpus, w.vocab, w.v, w.k)
+        times.append(time.perf_counter() - t0)
+    sec = statistics.median(times)
+    from oracle import lzw_allocation  # test infrastructure: CPU-baseline leg only
+    n_ref = min(len(corpus), 100_000)
+    t0 = time.perf_counter()
+    lzw_allocation.allocate(corpus[:n_ref], w.vocab, w.v, w.k)
+    ref = time.perf_counter() - t0
+    line = {"mode": "lzw_allocation", "metric": "corpus tokens/s through the allocation",
+            "value": len(corpus) / sec, "unit": "tokens/s", "higher_is_better": True,
+            "seconds": sec, "steps": max(1, args.steps),
+            "config": {"workload": w.name, "vocab": w.vocab, "v": w.v, "k": w.k,
+                       "corpus_tokens": len(corpus), "corpus": "synthetic phrase-structured Zipf"},
+            "codewords": n_words, "tokens_at_k": int((d == w.k).sum()),
+            "tokens_at_1": int((d == 1).sum()), "max_d": int(d.max()),
+            "cpu_baseline": {"value": n_ref / ref, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                             "sample": f"first {n_ref} corpus tokens, plain-Python oracle"}}
+    print(json.dumps(line), flush=True)
+
+
 def run_offload(args, w, tables, batch, dev, dist, world, rank):
     """Tables in pinned host memory: each step plans the batch (l3_plan_staged),
     copies its rows across PCIe into device staging tables (l3_stage_rows) and
@@ -340,6 +368,8 @@ def main():
     ap.add_argument("--tokens", type=int, default=0,
                     help="tokens per rank (default: the workload's batch size)")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--lzw", type=int, default=0, metavar="TOKENS",
+                    help="time the LZW allocation on a synthetic corpus of this many tokens")
     ap.add_argument("--offload", action="store_true",
                     help="W_K / W_V in pinned host memory; each step stages the batch's rows")
     args = ap.parse_args()
@@ -353,6 +383,10 @@ def main():
 
     if args.impl == "reference":
         run_reference(args, base, rank)
+        return
+    if args.lzw:
+        if rank == 0:
+            run_lzw(args, base)
         return
 
     dist = None

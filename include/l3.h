@@ -231,6 +231,36 @@ l3_status l3_sort_tokens_noalloc(const int32_t *token_ids, int64_t n_tokens, int
                                  int32_t *perm, int32_t *inv_perm, int32_t *sorted_ids,
                                  void *stream);
 
+/*
+ * l3_lzw_allocate — how many rows of W_K / W_V each token ID gets: the
+ * LZW-based allocation (kimjy99 review, 1. Embedding Allocation; papernotes
+ * note, LZW 分配). Host code, no device work; run once, its output turned
+ * into `offsets` (prefix sums) for l3_plan.
+ *
+ *   corpus       host int32 [n], token IDs in [0, vocab)
+ *   n            corpus length >= 0 (< 2^31 - 2)
+ *   vocab        number of token IDs >= 1
+ *   v            row budget, vocab <= v <= vocab * k
+ *   k            cap on rows per token >= 1
+ *   d_out        host int32 [vocab], out: d_t, 1 <= d_t <= k, sum = v
+ *   n_codewords  host int64, out: codewords the scan made (may be NULL)
+ *
+ * The scan makes one codeword per corpus position: the longest suffix of
+ * the text ending there that is already a codeword, extended one token
+ * further back, with frequency 1, and the suffix it extends gains 1 (a
+ * suffix never reaches before position 0). Codewords are then walked from
+ * most to least frequent, equal frequencies in creation order; each gives
+ * its last token one row unless that token holds k. Every token starts
+ * with one row; walks repeat until the rows sum to v. Time grows with the
+ * corpus length times the length of the matched suffixes (short on natural
+ * or Zipf-like text, up to quadratic on a text that repeats itself).
+ * Errors: L3_ERR_INVALID_ARG (NULL pointer, a token out of range, v outside
+ * [vocab, vocab * k], or v out of reach because every token that ends a
+ * codeword already holds k), L3_ERR_OOM (host memory).
+ */
+l3_status l3_lzw_allocate(const int32_t *corpus, int64_t n, int64_t vocab, int64_t v, int64_t k,
+                          int32_t *d_out, int64_t *n_codewords);
+
 /* Synchronizes the plan's last stream and returns L3_ERR_TIMEOUT if a
  * bounded wait inside an l3_forward kernel gave up since the plan was made
  * (the outputs of that call are then incomplete), L3_ERR_CUDA on a CUDA

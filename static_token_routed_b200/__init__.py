@@ -22,6 +22,7 @@ from ._binding import (  # noqa: F401
     l3_forward,
     l3_forward_status,
     l3_last_error,
+    l3_lzw_allocate,
     l3_plan,
     l3_plan_destroy,
     l3_plan_export,

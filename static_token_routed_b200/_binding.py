@@ -10,6 +10,8 @@ from __future__ import annotations
 import ctypes
 import os
 
+import numpy as np
+
 import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -22,7 +24,7 @@ STATUS = {0: "L3_OK", 1: "L3_ERR_INVALID_ARG", 2: "L3_ERR_TOKEN_RANGE", 3: "L3_E
 # every symbol include/l3.h declares
 EXPORTED = ["l3_plan", "l3_plan_info", "l3_plan_export", "l3_forward", "l3_forward_status",
             "l3_plan_destroy", "l3_last_error", "l3_profile_enable", "l3_profile_read",
-            "l3_sort_tokens_noalloc", "l3_plan_staged", "l3_stage_rows"]
+            "l3_sort_tokens_noalloc", "l3_plan_staged", "l3_stage_rows", "l3_lzw_allocate"]
 L3_SORT_NOALLOC_MAX_TOKENS = 65536
 
 
@@ -68,6 +70,8 @@ def library() -> ctypes.CDLL:
     lib.l3_plan_staged.argtypes = [p, i64, p, ctypes.POINTER(Dims), p, ctypes.POINTER(p)]
     lib.l3_stage_rows.restype = i32
     lib.l3_stage_rows.argtypes = [p, p, p, p, p, p]
+    lib.l3_lzw_allocate.restype = i32
+    lib.l3_lzw_allocate.argtypes = [p, i64, i64, i64, i64, p, ctypes.POINTER(i64)]
     lib.l3_plan_info.restype = i32
     lib.l3_plan_info.argtypes = [p, ctypes.POINTER(PlanInfo)]
     lib.l3_plan_export.restype = i32
@@ -193,6 +197,16 @@ def l3_stage_rows(plan: Plan, W_K: torch.Tensor, W_V: torch.Tensor, W_K_staged: 
     _check(library().l3_stage_rows(plan.handle, _table_ptr(W_K, "W_K"), _table_ptr(W_V, "W_V"),
                                    _ptr(W_K_staged, "W_K_staged"), _ptr(W_V_staged, "W_V_staged"),
                                    _stream(stream, W_K_staged.device)))
+
+
+def l3_lzw_allocate(corpus, vocab: int, v: int, k: int) -> tuple[np.ndarray, int]:
+    """d_t for every token ID (int32 [vocab]) and the number of codewords."""
+    c = np.ascontiguousarray(np.asarray(corpus, dtype=np.int32))
+    d = np.empty(int(vocab), dtype=np.int32)
+    nw = ctypes.c_int64(0)
+    _check(library().l3_lzw_allocate(c.ctypes.data if c.size else None, int(c.size), int(vocab),
+                                     int(v), int(k), d.ctypes.data, ctypes.byref(nw)))
+    return d, int(nw.value)
 
 
 def l3_plan_info(plan: Plan) -> PlanInfo:

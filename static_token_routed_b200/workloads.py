@@ -32,7 +32,7 @@ import torch
 
 _CHUNK = 1 << 24  # elements per independent random stream of a large tensor
 
-_TAGS = {"x": 1, "W_K": 2, "W_V": 3, "W_up": 4, "W_mix": 5, "ids": 6}
+_TAGS = {"x": 1, "W_K": 2, "W_V": 3, "W_up": 4, "W_mix": 5, "ids": 6, "corpus": 7}
 
 
 @dataclasses.dataclass(frozen=True)
@@ -200,6 +200,38 @@ def token_ids(w: Workload) -> np.ndarray:
     else:
         raise ValueError(w.ids)
     return ids.astype(np.int32)
+
+
+def zipf_corpus(vocab: int, n: int, seed: int, s: float = 1.1, n_phrases: int = 50000,
+                phrase_share: float = 0.5) -> np.ndarray:
+    """A synthetic token stream standing in for a tokenised corpus (the pages'
+    FineWeb-Edu text is not here): half of its items are single tokens drawn
+    Zipf(s) over the vocabulary, half are phrases of 2-6 such tokens drawn
+    Zipf(s) from a fixed phrase list, so frequent multi-token sequences recur
+    as in text. int32 [n]."""
+    rng = _rng(seed, "corpus")
+    p_tok = zipf_weights(vocab, s)
+    p_tok /= p_tok.sum()
+    plen = rng.integers(2, 7, size=n_phrases)
+    pstart = np.concatenate([[0], np.cumsum(plen)])
+    ptoks = rng.choice(vocab, size=int(pstart[-1]), p=p_tok)
+    p_phr = zipf_weights(n_phrases, s)
+    p_phr /= p_phr.sum()
+    out, have = [], 0
+    while have < n:
+        m = max(1024, (n - have) // 2)
+        is_phr = rng.random(m) < phrase_share
+        which = rng.choice(n_phrases, size=m, p=p_phr)
+        single = rng.choice(vocab, size=m, p=p_tok)
+        lens = np.where(is_phr, plen[which], 1)
+        starts = np.where(is_phr, pstart[which], 0)
+        item = np.repeat(np.arange(m), lens)
+        offs = np.arange(int(lens.sum())) - np.repeat(np.cumsum(lens) - lens, lens)
+        toks = np.where(is_phr[item], ptoks[np.minimum(starts[item] + offs, len(ptoks) - 1)],
+                        single[item])
+        out.append(toks)
+        have += len(toks)
+    return np.concatenate(out)[:n].astype(np.int32)
 
 
 def normal_tensor(seed: int, tag: str, shape, std: float, dtype: torch.dtype,

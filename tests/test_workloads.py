@@ -66,3 +66,14 @@ def test_tied_tables_share_one_tensor():
     assert t.W_V is t.W_K and t.W_K.shape == (1200, 512)
     with pytest.raises(ValueError):
         wl.make_tables(dataclasses.replace(w, d_emb=256))
+
+
+def test_zipf_corpus_is_seeded_and_in_range():
+    a = wl.zipf_corpus(500, 20000, seed=3)
+    b = wl.zipf_corpus(500, 20000, seed=3)
+    assert a.dtype == np.int32 and len(a) == 20000 and np.array_equal(a, b)
+    assert a.min() >= 0 and a.max() < 500
+    assert not np.array_equal(a, wl.zipf_corpus(500, 20000, seed=4))
+    # frequent IDs come first (Zipf ranks)
+    counts = np.bincount(a, minlength=500)
+    assert counts[:5].sum() > counts[-100:].sum()
