@@ -261,6 +261,21 @@ l3_status l3_sort_tokens_noalloc(const int32_t *token_ids, int64_t n_tokens, int
 l3_status l3_lzw_allocate(const int32_t *corpus, int64_t n, int64_t vocab, int64_t v, int64_t k,
                           int32_t *d_out, int64_t *n_codewords);
 
+/*
+ * l3_check_bounded_wait — exercise the give-up path that every kernel's
+ * waits share, on the device. The pages have no counterpart: this entry
+ * point exists for failure detection, not for the method.
+ *
+ * Launches one small kernel that waits on an mbarrier nothing completes,
+ * with the kernels' own bounded wait (2 s by %globaltimer). The wait gives
+ * up, raises its CTA's abort flag, reports the timeout in device memory and
+ * returns; the launch ends normally and the context stays usable.
+ * Synchronizes `stream` and takes about 2 s.
+ * Returns L3_ERR_TIMEOUT when the give-up was reported (the expected
+ * result), L3_ERR_CUDA otherwise.
+ */
+l3_status l3_check_bounded_wait(void *stream);
+
 /* Synchronizes the plan's last stream and returns L3_ERR_TIMEOUT if a
  * bounded wait inside an l3_forward kernel gave up since the plan was made
  * (the outputs of that call are then incomplete), L3_ERR_CUDA on a CUDA

@@ -24,7 +24,8 @@ STATUS = {0: "L3_OK", 1: "L3_ERR_INVALID_ARG", 2: "L3_ERR_TOKEN_RANGE", 3: "L3_E
 # every symbol include/l3.h declares
 EXPORTED = ["l3_plan", "l3_plan_info", "l3_plan_export", "l3_forward", "l3_forward_status",
             "l3_plan_destroy", "l3_last_error", "l3_profile_enable", "l3_profile_read",
-            "l3_sort_tokens_noalloc", "l3_plan_staged", "l3_stage_rows", "l3_lzw_allocate"]
+            "l3_sort_tokens_noalloc", "l3_plan_staged", "l3_stage_rows", "l3_lzw_allocate",
+            "l3_check_bounded_wait"]
 L3_SORT_NOALLOC_MAX_TOKENS = 65536
 
 
@@ -70,6 +71,8 @@ def library() -> ctypes.CDLL:
     lib.l3_plan_staged.argtypes = [p, i64, p, ctypes.POINTER(Dims), p, ctypes.POINTER(p)]
     lib.l3_stage_rows.restype = i32
     lib.l3_stage_rows.argtypes = [p, p, p, p, p, p]
+    lib.l3_check_bounded_wait.restype = i32
+    lib.l3_check_bounded_wait.argtypes = [p]
     lib.l3_lzw_allocate.restype = i32
     lib.l3_lzw_allocate.argtypes = [p, i64, i64, i64, i64, p, ctypes.POINTER(i64)]
     lib.l3_plan_info.restype = i32
@@ -207,6 +210,12 @@ def l3_lzw_allocate(corpus, vocab: int, v: int, k: int) -> tuple[np.ndarray, int
     _check(library().l3_lzw_allocate(c.ctypes.data if c.size else None, int(c.size), int(vocab),
                                      int(v), int(k), d.ctypes.data, ctypes.byref(nw)))
     return d, int(nw.value)
+
+
+def l3_check_bounded_wait(stream=None, device=None) -> int:
+    """Status of the device-side give-up check (L3_ERR_TIMEOUT = 6 expected)."""
+    dev = device if device is not None else torch.cuda.current_device()
+    return int(library().l3_check_bounded_wait(_stream(stream, torch.device("cuda", dev))))
 
 
 def l3_plan_info(plan: Plan) -> PlanInfo:
