@@ -150,8 +150,8 @@ __device__ __forceinline__ void spin_bounded(uint64_t *bar, uint32_t parity) {
 
 template <bool SMALL>
 __global__ void __launch_bounds__(DENSE_THREADS, DenseCfg<SMALL>::MIN_BLOCKS)
-    k_attn_dense(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUtensorMap mV,
-                 DenseParams P) {
+    k_attn_dense(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUtensorMap mK16,
+                 const __grid_constant__ CUtensorMap mV, DenseParams P) {
   using Cfg = DenseCfg<SMALL>;
   constexpr int REGION = Cfg::REGION;
   extern __shared__ uint8_t smem_raw[];
@@ -170,7 +170,10 @@ __global__ void __launch_bounds__(DENSE_THREADS, DenseCfg<SMALL>::MIN_BLOCKS)
   const int d64 = (d + 63) & ~63;
   const int n_kc = P.d_in / CK;
   const int n_vc = d16 / V_ROWS;
-  const int k_boxes = d64 / 64;         // 64-row TMA boxes per K_t slice
+  // K_t rows per slice: whole 64-row TMA boxes, then 16-row boxes up to d16
+  // (the rows the MMA reads), so no slice fetches more than 15 rows past d_t
+  const int k_full = d16 / 64, k_rest = (d16 % 64) / 16;
+  const uint32_t k_slice_bytes = (uint32_t)(k_full * 64 + k_rest * 16) * CK * 2;
   // O = P V_t in passes of at most TMEM_COLS columns of d_emb
   const int o_max = min(P.d_emb, Cfg::TMEM_COLS);
   const int n_op = (P.d_emb + o_max - 1) / o_max;
@@ -204,6 +207,7 @@ __global__ void __launch_bounds__(DENSE_THREADS, DenseCfg<SMALL>::MIN_BLOCKS)
     b->abort_flag = 0;
     fence_mbar_init();
     prefetch_tensormap(&mK);
+    prefetch_tensormap(&mK16);
     prefetch_tensormap(&mV);
   }
   if (warp == 1) {
@@ -231,11 +235,14 @@ __global__ void __launch_bounds__(DENSE_THREADS, DenseCfg<SMALL>::MIN_BLOCKS)
           break;
         }
         uint8_t *kdst = smem + s * s_stage + X_BYTES;
-        mbar_arrive_expect_tx(&b->kfull[s], k_boxes * 64 * CK * 2);
+        mbar_arrive_expect_tx(&b->kfull[s], k_slice_bytes);
         armed[s] = true;
         armed_par[s] = ph;
-        for (int bx = 0; bx < k_boxes; ++bx)
+        for (int bx = 0; bx < k_full; ++bx)
           tma_load_2d(kdst + bx * 64 * CK * 2, &mK, &b->kfull[s], kc * CK, r0 + bx * 64);
+        for (int bx = 0; bx < k_rest; ++bx)
+          tma_load_2d(kdst + (k_full * 64 + bx * 16) * CK * 2, &mK16, &b->kfull[s], kc * CK,
+                      r0 + k_full * 64 + bx * 16);
       }
       // V slices go where the S ring was: wait until every S-phase MMA is done
       if (ok) ok = mbar_wait(&b->sfull, 0, ab);
@@ -527,7 +534,8 @@ constexpr size_t dense_smem() {
 }
 
 template <bool SMALL>
-l3_status launch_cfg(const CUtensorMap &mK, const CUtensorMap &mV, const DenseParams &P,
+l3_status launch_cfg(const CUtensorMap &mK, const CUtensorMap &mK16, const CUtensorMap &mV,
+                     const DenseParams &P,
                      int64_t n_tiles, int device, const char *name, cudaStream_t s) {
   if (n_tiles == 0) return L3_OK;
   static bool attr[64] = {};
@@ -538,7 +546,7 @@ l3_status launch_cfg(const CUtensorMap &mK, const CUtensorMap &mV, const DensePa
     attr[device & 63] = true;
   }
   LaunchTimer t(name, s);
-  k_attn_dense<SMALL><<<(unsigned)n_tiles, DENSE_THREADS, dense_smem<SMALL>(), s>>>(mK, mV, P);
+  k_attn_dense<SMALL><<<(unsigned)n_tiles, DENSE_THREADS, dense_smem<SMALL>(), s>>>(mK, mK16, mV, P);
   L3_CUDA_TRY(cudaGetLastError());
   return L3_OK;
 }
@@ -556,12 +564,14 @@ l3_status launch_attn_dense(const l3_plan_s *p, const void *x, const void *W_K, 
   const int64_t n_big = p->n_dense_tiles - p->n_dense_small;
   if ((small ? p->n_dense_small : n_big) == 0) return L3_OK;
   const l3_dims_t &d = p->dims;
-  CUtensorMap mK, mV;
+  CUtensorMap mK, mK16, mV;
   l3_status st;
   // rows of the tables the kernel reads: all v, or the batch's rows when staged
   // (TMA fills rows past the end with zeros, so padding never reads past it)
   const uint64_t rows = p->staged ? (uint64_t)p->unique_rows : (uint64_t)d.v;
   if ((st = make_map_2d16(&mK, W_K, true, rows, d.d_in, d.d_in, CK, 64, 128)) != L3_OK) return st;
+  if ((st = make_map_2d16(&mK16, W_K, true, rows, d.d_in, d.d_in, CK, 16, 128)) != L3_OK)
+    return st;
   if ((st = make_map_2d16(&mV, W_V, true, rows, d.d_emb, d.d_emb, 64, V_ROWS, 128)) != L3_OK)
     return st;
   DenseParams P;
@@ -575,9 +585,9 @@ l3_status launch_attn_dense(const l3_plan_s *p, const void *x, const void *W_K, 
   P.d_in = (int)d.d_in;
   P.d_emb = (int)d.d_emb;
   P.err = p->dev_flags + 1;
-  if (!small) return launch_cfg<false>(mK, mV, P, n_big, p->device, "attn_dense", s);
+  if (!small) return launch_cfg<false>(mK, mK16, mV, P, n_big, p->device, "attn_dense", s);
   P.tiles = p->dense_tiles + n_big;
-  return launch_cfg<true>(mK, mV, P, p->n_dense_small, p->device, "attn_dense_small", s);
+  return launch_cfg<true>(mK, mK16, mV, P, p->n_dense_small, p->device, "attn_dense_small", s);
 }
 
 }  // namespace l3
