@@ -271,6 +271,55 @@ def run_lzw(args, w):
     print(json.dumps(line), flush=True)
 
 
+def run_backward(args, w, tables, batch, dev, dist, world, rank):
+    """Plan, forward and backward (fp32 gradients for a random dL/dy) per
+    batch; the backward is the CUDA-core implementation."""
+    d = {k: getattr(tables, k).to(dev) for k in ("offsets", "W_K", "W_up", "ln_gamma", "ln_beta",
+                                                 "W_mix")}
+    d["W_V"] = d["W_K"] if tables.W_V is tables.W_K else tables.W_V.to(dev)
+    ids_d, x_d = batch.ids.to(dev), batch.x.to(dev)
+    y_d = torch.empty(w.n_tokens, w.d_out, dtype=w.torch_dtype, device=dev)
+    g = torch.Generator(device=dev).manual_seed(0)
+    dy = torch.randn(w.n_tokens, w.d_out, generator=g, device=dev).to(w.torch_dtype)
+    dims = l3.make_dims(w.vocab, w.v, w.k, w.d_in, w.d_emb, w.d_up, w.d_out, w.torch_dtype, EPS)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        plan = l3.l3_plan(ids_d, d["offsets"], dims, stream)
+        l3.l3_forward(x_d, plan, d["W_K"], d["W_V"], d["W_up"], d["ln_gamma"], d["ln_beta"],
+                      d["W_mix"], y_d, stream)
+        grads = l3.l3_backward(x_d, plan, d["W_K"], d["W_V"], d["W_up"], d["ln_gamma"],
+                               d["ln_beta"], d["W_mix"], dy, stream)
+        return plan, grads
+
+    for _ in range(max(3, args.warmup)):
+        p, _ = step()
+        p.destroy()
+    l3.l3_profile_enable(True)
+    torch.cuda.synchronize(dev)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for _ in range(args.steps):
+        p, _ = step()
+        p.destroy()
+    ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    kernels = l3.l3_profile_read()
+    l3.l3_profile_enable(False)
+    ms = max_over_ranks(ev0.elapsed_time(ev1) / args.steps, dist, dev)
+    if rank != 0:
+        return
+    bwd_ms = sum(t for k, (_, t) in kernels.items() if k.startswith("bwd")) / args.steps
+    line = {"metric": METRIC, "mode": "forward+backward", "value": job_throughput(w.n_tokens, world, ms),
+            "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms, "backward_ms_per_step": bwd_ms, "higher_is_better": True,
+            "scaling": "weak", "dtype": "bf16" if w.dtype == "bf16" else "fp32",
+            "data": "synthetic", "config": config_of(w, args),
+            "kernels": {k: {"launches": nl, "per_step_ms": t / args.steps}
+                        for k, (nl, t) in kernels.items()}}
+    print(json.dumps(line), flush=True)
+
+
 def run_offload(args, w, tables, batch, dev, dist, world, rank):
     """Tables in pinned host memory: each step plans the batch (l3_plan_staged),
     copies its rows across PCIe into device staging tables (l3_stage_rows) and
@@ -370,6 +419,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--lzw", type=int, default=0, metavar="TOKENS",
                     help="time the LZW allocation on a synthetic corpus of this many tokens")
+    ap.add_argument("--backward", action="store_true",
+                    help="time l3_forward + l3_backward per batch (CUDA-core backward)")
     ap.add_argument("--offload", action="store_true",
                     help="W_K / W_V in pinned host memory; each step stages the batch's rows")
     args = ap.parse_args()
@@ -403,6 +454,9 @@ def main():
     tables, batch = wl.make_tables(w), wl.make_batch(w)
     if args.offload:
         run_offload(args, w, tables, batch, dev, dist, world, rank)
+        return
+    if args.backward:
+        run_backward(args, w, tables, batch, dev, dist, world, rank)
         return
     d = {k: getattr(tables, k).to(dev) for k in ("offsets", "W_K", "W_up", "ln_gamma",
                                                  "ln_beta", "W_mix")}

@@ -193,6 +193,32 @@ l3_status l3_forward(const void *x, l3_plan_t plan, const void *W_K, const void 
                      const void *W_mix, void *y, void *stream);
 
 /*
+ * l3_backward — gradients of the layer (kimjy99 review, Method, eq. L³, by
+ * the chain rule) for dL/dy, on CUDA cores in fp32 arithmetic.
+ *
+ * Call after l3_forward on the same plan and the same inputs: it reuses the
+ * a = V_t^T softmax(K_t x) and h = LayerNorm(W_up a) that forward stored
+ * in the plan (and recomputes W_up a).
+ *   x .. W_mix   as for l3_forward (dims->dtype); ln_beta is not read
+ *   dy           [N x d_out] dims->dtype, caller's token order
+ *   dx           fp32 [N x d_in], out
+ *   dW_K, dW_V   fp32 [v x d_in], [v x d_emb], out: the rows of every ID in
+ *                the batch are written; other rows are left as they were
+ *   dW_up        fp32 [d_up x d_emb], out
+ *   dgamma, dbeta fp32 [d_up], out
+ *   dW_mix       fp32 [d_out x (d_up + d_in)], out
+ * Deterministic (no atomics). Scratch (3 N d_up + N d_emb floats) is taken
+ * from and returned to the stream-ordered pool on `stream`. Enqueued on
+ * `stream`; does not synchronize. Errors: L3_ERR_INVALID_ARG (NULL pointer,
+ * a staged plan), L3_ERR_UNSUPPORTED (k > 1024, or d_in / d_emb / d_up too
+ * wide for its shared-memory layout), L3_ERR_OOM, L3_ERR_CUDA.
+ */
+l3_status l3_backward(const void *x, l3_plan_t plan, const void *W_K, const void *W_V,
+                      const void *W_up, const void *ln_gamma, const void *ln_beta,
+                      const void *W_mix, const void *dy, float *dx, float *dW_K, float *dW_V,
+                      float *dW_up, float *dgamma, float *dbeta, float *dW_mix, void *stream);
+
+/*
  * l3_sort_tokens_noalloc — the stable sort step of l3_plan, for callers that
  * cannot allocate device memory. The pages have no counterpart: this entry
  * point exists for integration, not for the method.

@@ -21,6 +21,7 @@ from ._binding import (  # noqa: F401
     PlanInfo,
     l3_forward,
     l3_forward_status,
+    l3_backward,
     l3_check_bounded_wait,
     l3_last_error,
     l3_lzw_allocate,

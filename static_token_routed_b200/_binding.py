@@ -25,7 +25,7 @@ STATUS = {0: "L3_OK", 1: "L3_ERR_INVALID_ARG", 2: "L3_ERR_TOKEN_RANGE", 3: "L3_E
 EXPORTED = ["l3_plan", "l3_plan_info", "l3_plan_export", "l3_forward", "l3_forward_status",
             "l3_plan_destroy", "l3_last_error", "l3_profile_enable", "l3_profile_read",
             "l3_sort_tokens_noalloc", "l3_plan_staged", "l3_stage_rows", "l3_lzw_allocate",
-            "l3_check_bounded_wait"]
+            "l3_check_bounded_wait", "l3_backward"]
 L3_SORT_NOALLOC_MAX_TOKENS = 65536
 
 
@@ -71,6 +71,8 @@ def library() -> ctypes.CDLL:
     lib.l3_plan_staged.argtypes = [p, i64, p, ctypes.POINTER(Dims), p, ctypes.POINTER(p)]
     lib.l3_stage_rows.restype = i32
     lib.l3_stage_rows.argtypes = [p, p, p, p, p, p]
+    lib.l3_backward.restype = i32
+    lib.l3_backward.argtypes = [p] * 17
     lib.l3_check_bounded_wait.restype = i32
     lib.l3_check_bounded_wait.argtypes = [p]
     lib.l3_lzw_allocate.restype = i32
@@ -210,6 +212,29 @@ def l3_lzw_allocate(corpus, vocab: int, v: int, k: int) -> tuple[np.ndarray, int
     _check(library().l3_lzw_allocate(c.ctypes.data if c.size else None, int(c.size), int(vocab),
                                      int(v), int(k), d.ctypes.data, ctypes.byref(nw)))
     return d, int(nw.value)
+
+
+def l3_backward(x, plan: Plan, W_K, W_V, W_up, ln_gamma, ln_beta, W_mix, dy,
+                stream=None) -> dict:
+    """Gradients for dL/dy = dy after l3_forward on the same plan and inputs.
+    Returns fp32 tensors: x, W_K, W_V (rows of IDs outside the batch zero),
+    W_up, ln_gamma, ln_beta, W_mix."""
+    d = plan.dims
+    dev = x.device
+    f32 = dict(dtype=torch.float32, device=dev)
+    out = {"x": torch.empty(plan.n_tokens, d.d_in, **f32),
+           "W_K": torch.zeros(d.v, d.d_in, **f32), "W_V": torch.zeros(d.v, d.d_emb, **f32),
+           "W_up": torch.empty(d.d_up, d.d_emb, **f32), "ln_gamma": torch.empty(d.d_up, **f32),
+           "ln_beta": torch.empty(d.d_up, **f32),
+           "W_mix": torch.empty(d.d_out, d.d_up + d.d_in, **f32)}
+    ins = [_ptr(t, nm) for t, nm in ((x, "x"), (None, "plan"), (W_K, "W_K"), (W_V, "W_V"),
+                                     (W_up, "W_up"), (ln_gamma, "ln_gamma"),
+                                     (ln_beta, "ln_beta"), (W_mix, "W_mix"), (dy, "dy"))]
+    ins[1] = plan.handle
+    outs = [out[k].data_ptr() for k in ("x", "W_K", "W_V", "W_up", "ln_gamma", "ln_beta",
+                                        "W_mix")]
+    _check(library().l3_backward(*ins, *outs, _stream(stream, dev)))
+    return out
 
 
 def l3_check_bounded_wait(stream=None, device=None) -> int:

@@ -1,0 +1,419 @@
+// Backward pass of the layer on CUDA cores (fp32 arithmetic), after an
+// l3_forward on the same plan: it reuses the a and h that forward stored.
+//
+// kimjy99 review, Method, eq. L³, per token with rows K_t, V_t:
+//   s = K_t x, p = softmax(s), a = V_t^T p, z = W_up a,
+//   h = gamma (z - mean z) / sqrt(var z + eps) + beta, y = W_mix [h ; x].
+// Given g_y = dL/dy (chain rule, step by step):
+//   dW_mix = g_y^T [h ; x]              g_h = g_y W_mix[:, :d_up]
+//   dx     = g_y W_mix[:, d_up:]  (+ K_t^T g_s below)
+//   dgamma = sum g_h hhat, dbeta = sum g_h, g_hhat = g_h gamma
+//   g_z    = (g_hhat - mean g_hhat - hhat mean(g_hhat hhat)) / sqrt(var z + eps)
+//   dW_up  = g_z^T a                    g_a = g_z W_up
+//   g_p    = V_t g_a, g_s = p (g_p - p.g_p)
+//   dV_t  += p g_a^T, dK_t += g_s x^T, dx += K_t^T g_s
+// The GEMMs run as one strided tiled FFMA kernel (operands read through
+// element strides, so transposed operands need no copies). The attention
+// part runs one CTA per token group: the group's rows belong to that CTA
+// alone, so dW_K / dW_V rows are written without atomics, and eight tokens
+// at a time share every row it reads. The dgamma / dbeta column sums are
+// per-CTA partials reduced by a second kernel (no atomics: deterministic).
+#include <cuda_fp16.h>
+
+#include <algorithm>
+
+#include "l3_internal.cuh"
+
+namespace l3 {
+namespace {
+
+enum { T_F32 = 0, T_BF16 = 1, T_F16 = 2 };
+
+__device__ __forceinline__ float ldx(const void *p, int type, int64_t i) {
+  if (type == T_F32) return reinterpret_cast<const float *>(p)[i];
+  if (type == T_BF16) return __bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(p)[i]);
+  return __half2float(reinterpret_cast<const __half *>(p)[i]);
+}
+
+// ---------------------------------------------------------------- GEMM
+// C[m][n] (+)= sum_k A(m, k) B(n, k), A(m, k) = A[m * a_sm + k * a_sk],
+// B(n, k) = B[n * b_sn + k * b_sk]; fp32 accumulate and output.
+struct Operand {
+  const void *p;
+  int64_t s_row, s_k;  // element strides along the output dimension and along k
+  int type;
+};
+
+constexpr int GB_M = 64, GB_N = 64, GB_K = 16, G_THREADS = 256;
+
+__global__ void __launch_bounds__(G_THREADS)
+    k_gemm_strided(Operand A, Operand B, int M, int N, int K, float *__restrict__ C, int64_t ldc,
+                   int accumulate) {
+  __shared__ float As[GB_K][GB_M + 4];
+  __shared__ float Bs[GB_K][GB_N + 4];
+  const int tid = threadIdx.x, tx = tid % 16, ty = tid / 16;
+  const int m0 = blockIdx.y * GB_M, n0 = blockIdx.x * GB_N;
+  float acc[4][4] = {};
+  for (int k0 = 0; k0 < K; k0 += GB_K) {
+#pragma unroll
+    for (int i = 0; i < (GB_M * GB_K) / G_THREADS; ++i) {
+      const int e = tid + i * G_THREADS;
+      // consecutive threads walk the operand's unit-stride dimension
+      int row = A.s_k == 1 ? e / GB_K : e % GB_M, kk = A.s_k == 1 ? e % GB_K : e / GB_M;
+      int gm = m0 + row, gk = k0 + kk;
+      As[kk][row] = (gm < M && gk < K) ? ldx(A.p, A.type, gm * A.s_row + gk * A.s_k) : 0.f;
+      row = B.s_k == 1 ? e / GB_K : e % GB_N;
+      kk = B.s_k == 1 ? e % GB_K : e / GB_N;
+      const int gn = n0 + row;
+      gk = k0 + kk;
+      Bs[kk][row] = (gn < N && gk < K) ? ldx(B.p, B.type, gn * B.s_row + gk * B.s_k) : 0.f;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int kk = 0; kk < GB_K; ++kk) {
+      float a[4], b[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) a[i] = As[kk][ty * 4 + i];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) b[j] = Bs[kk][tx * 4 + j];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int gm = m0 + ty * 4 + i;
+    if (gm >= M) continue;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int gn = n0 + tx * 4 + j;
+      if (gn >= N) continue;
+      float *c = C + (int64_t)gm * ldc + gn;
+      *c = accumulate ? *c + acc[i][j] : acc[i][j];
+    }
+  }
+}
+
+l3_status gemm(Operand A, Operand B, int M, int N, int K, float *C, int64_t ldc, bool accumulate,
+               cudaStream_t s) {
+  if (M == 0 || N == 0) return L3_OK;
+  dim3 grid((N + GB_N - 1) / GB_N, (M + GB_M - 1) / GB_M);
+  k_gemm_strided<<<grid, G_THREADS, 0, s>>>(A, B, M, N, K, C, ldc, accumulate ? 1 : 0);
+  L3_CUDA_TRY(cudaGetLastError());
+  return L3_OK;
+}
+
+// ---------------------------------------------------------------- LayerNorm
+constexpr int LN_ROWS = 16;  // token rows per CTA (one warp per row at a time)
+
+// g_z from g_h and z for LN_ROWS rows per CTA; column partials of
+// dgamma = sum g_h hhat and dbeta = sum g_h into part[cta][2][d_up]
+__global__ void __launch_bounds__(256)
+    k_ln_backward(const float *__restrict__ z, const float *__restrict__ g_h, const void *gamma,
+                  int gtype, int d_up, float eps, int64_t M, float *__restrict__ g_z,
+                  float *__restrict__ part) {
+  extern __shared__ float sm[];  // [8 warps][2][d_up]
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  float *pg = sm + warp * 2 * d_up, *pb = pg + d_up;
+  for (int u = lane; u < d_up; u += 32) pg[u] = pb[u] = 0.f;
+  for (int rr = warp; rr < LN_ROWS; rr += 8) {
+    const int64_t row = blockIdx.x * (int64_t)LN_ROWS + rr;
+    if (row >= M) break;
+    const float *zr = z + row * d_up, *gr = g_h + row * d_up;
+    float s = 0.f;
+    for (int u = lane; u < d_up; u += 32) s += zr[u];
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    const float mu = s / d_up;
+    float q = 0.f;
+    for (int u = lane; u < d_up; u += 32) q = fmaf(zr[u] - mu, zr[u] - mu, q);
+    for (int o = 16; o > 0; o >>= 1) q += __shfl_xor_sync(0xffffffffu, q, o);
+    const float rstd = 1.0f / sqrtf(q / d_up + eps);
+    float m1 = 0.f, m2 = 0.f;  // sums of g_hhat and g_hhat * hhat
+    for (int u = lane; u < d_up; u += 32) {
+      const float hh = (zr[u] - mu) * rstd, gh = gr[u] * ldx(gamma, gtype, u);
+      m1 += gh;
+      m2 = fmaf(gh, hh, m2);
+      pg[u] = fmaf(gr[u], hh, pg[u]);
+      pb[u] += gr[u];
+    }
+    for (int o = 16; o > 0; o >>= 1) {
+      m1 += __shfl_xor_sync(0xffffffffu, m1, o);
+      m2 += __shfl_xor_sync(0xffffffffu, m2, o);
+    }
+    m1 /= d_up;
+    m2 /= d_up;
+    float *gzr = g_z + row * d_up;
+    for (int u = lane; u < d_up; u += 32) {
+      const float hh = (zr[u] - mu) * rstd, gh = gr[u] * ldx(gamma, gtype, u);
+      gzr[u] = (gh - m1 - hh * m2) * rstd;
+    }
+  }
+  __syncthreads();
+  for (int u = threadIdx.x; u < d_up; u += blockDim.x) {
+    float g = 0.f, bsum = 0.f;
+    for (int w = 0; w < 8; ++w) {
+      g += sm[w * 2 * d_up + u];
+      bsum += sm[w * 2 * d_up + d_up + u];
+    }
+    part[(int64_t)blockIdx.x * 2 * d_up + u] = g;
+    part[(int64_t)blockIdx.x * 2 * d_up + d_up + u] = bsum;
+  }
+}
+
+// column sums of the per-CTA partials, in CTA order
+__global__ void k_sum_partials(const float *__restrict__ part, int n_parts, int d_up,
+                               float *__restrict__ dgamma, float *__restrict__ dbeta) {
+  const int u = blockIdx.x * blockDim.x + threadIdx.x;
+  if (u >= d_up) return;
+  float g = 0.f, b = 0.f;
+  for (int i = 0; i < n_parts; ++i) {
+    g += part[(int64_t)i * 2 * d_up + u];
+    b += part[(int64_t)i * 2 * d_up + d_up + u];
+  }
+  dgamma[u] = g;
+  dbeta[u] = b;
+}
+
+// ---------------------------------------------------------------- attention
+constexpr int AT = 8;        // tokens per chunk
+constexpr int A_MAX_K = 1024;
+
+// One CTA per group; its tokens in chunks of AT.
+__global__ void __launch_bounds__(256)
+    k_attn_backward(const void *x, const void *W_K, const void *W_V, int wtype,
+                    const float *__restrict__ g_a, const int32_t *__restrict__ perm,
+                    const int32_t *__restrict__ group_tok_start,
+                    const int32_t *__restrict__ group_row_start,
+                    const int32_t *__restrict__ group_rows, int d_in, int d_emb,
+                    float *__restrict__ dx, float *__restrict__ dW_K, float *__restrict__ dW_V) {
+  extern __shared__ float sm[];
+  float *xs = sm;                  // [AT][d_in]
+  float *gas = xs + AT * d_in;     // [AT][d_emb]
+  float *ps = gas + AT * d_emb;    // [AT][A_MAX_K] logits, then p
+  float *gs = ps + AT * A_MAX_K;   // [AT][A_MAX_K] g_p, then g_s
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int g = blockIdx.x;
+  const int t0 = group_tok_start[g], c = group_tok_start[g + 1] - t0;
+  const int64_t r0 = group_row_start[g];
+  const int d = group_rows[g];
+  for (int c0 = 0; c0 < c; c0 += AT) {
+    const int nt = min(AT, c - c0);
+    for (int i = threadIdx.x; i < AT * d_in; i += blockDim.x) {
+      const int t = i / d_in, col = i % d_in;
+      xs[i] = t < nt ? ldx(x, wtype, (int64_t)perm[t0 + c0 + t] * d_in + col) : 0.f;
+    }
+    for (int i = threadIdx.x; i < AT * d_emb; i += blockDim.x) {
+      const int t = i / d_emb, col = i % d_emb;
+      gas[i] = t < nt ? g_a[(int64_t)perm[t0 + c0 + t] * d_emb + col] : 0.f;
+    }
+    __syncthreads();
+    // logits s = K_j . x_t and g_p = V_j . g_a_t, one warp per row
+    for (int j = warp; j < d; j += 8) {
+      float sv[AT], gv[AT];
+#pragma unroll
+      for (int t = 0; t < AT; ++t) sv[t] = gv[t] = 0.f;
+      if (d > 1)
+        for (int col = lane; col < d_in; col += 32) {
+          const float kv = ldx(W_K, wtype, (r0 + j) * d_in + col);
+#pragma unroll
+          for (int t = 0; t < AT; ++t) sv[t] = fmaf(kv, xs[t * d_in + col], sv[t]);
+        }
+      for (int col = lane; col < d_emb; col += 32) {
+        const float vv = ldx(W_V, wtype, (r0 + j) * d_emb + col);
+#pragma unroll
+        for (int t = 0; t < AT; ++t) gv[t] = fmaf(vv, gas[t * d_emb + col], gv[t]);
+      }
+#pragma unroll
+      for (int t = 0; t < AT; ++t) {
+        for (int o = 16; o > 0; o >>= 1) {
+          sv[t] += __shfl_xor_sync(0xffffffffu, sv[t], o);
+          gv[t] += __shfl_xor_sync(0xffffffffu, gv[t], o);
+        }
+        if (lane == 0) {
+          ps[t * A_MAX_K + j] = sv[t];
+          gs[t * A_MAX_K + j] = gv[t];
+        }
+      }
+    }
+    __syncthreads();
+    // softmax and g_s = p (g_p - p . g_p), one warp per token
+    if (warp < nt) {
+      float *pr = ps + warp * A_MAX_K, *gr = gs + warp * A_MAX_K;
+      float mx = -INFINITY;
+      for (int j = lane; j < d; j += 32) mx = fmaxf(mx, pr[j]);
+      for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      float sum = 0.f;
+      for (int j = lane; j < d; j += 32) {
+        const float e = d > 1 ? expf(pr[j] - mx) : 1.f;
+        pr[j] = e;
+        sum += e;
+      }
+      for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+      float dot = 0.f;
+      for (int j = lane; j < d; j += 32) {
+        pr[j] /= sum;
+        dot = fmaf(pr[j], gr[j], dot);
+      }
+      for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+      for (int j = lane; j < d; j += 32) gr[j] = pr[j] * (gr[j] - dot);
+    }
+    __syncthreads();
+    // dx_t += K_t^T g_s_t and dK_j (+)= sum_t g_s[t][j] x_t: thread per column
+    if (d > 1) {
+      for (int col = threadIdx.x; col < d_in; col += blockDim.x) {
+        float acc[AT];
+#pragma unroll
+        for (int t = 0; t < AT; ++t) acc[t] = 0.f;
+        for (int j = 0; j < d; ++j) {
+          const int64_t kidx = (r0 + j) * d_in + col;
+          const float kv = ldx(W_K, wtype, kidx);
+          float gk = 0.f;
+#pragma unroll
+          for (int t = 0; t < AT; ++t) {
+            const float gst = gs[t * A_MAX_K + j];
+            acc[t] = fmaf(gst, kv, acc[t]);
+            gk = fmaf(gst, xs[t * d_in + col], gk);
+          }
+          dW_K[kidx] = c0 == 0 ? gk : dW_K[kidx] + gk;
+        }
+        for (int t = 0; t < nt; ++t) dx[(int64_t)perm[t0 + c0 + t] * d_in + col] += acc[t];
+      }
+    } else {
+      for (int col = threadIdx.x; col < d_in; col += blockDim.x)
+        dW_K[r0 * d_in + col] = 0.f;  // one row: p = 1, no gradient reaches K
+    }
+    // dV_j (+)= sum_t p[t][j] g_a_t
+    for (int col = threadIdx.x; col < d_emb; col += blockDim.x) {
+      for (int j = 0; j < d; ++j) {
+        float gv = 0.f;
+#pragma unroll
+        for (int t = 0; t < AT; ++t) gv = fmaf(ps[t * A_MAX_K + j], gas[t * d_emb + col], gv);
+        const int64_t vidx = (r0 + j) * d_emb + col;
+        dW_V[vidx] = c0 == 0 ? gv : dW_V[vidx] + gv;
+      }
+    }
+    __syncthreads();
+  }
+}
+
+}  // namespace
+}  // namespace l3
+
+using namespace l3;
+
+extern "C" l3_status l3_backward(const void *x, l3_plan_t p, const void *W_K, const void *W_V,
+                                 const void *W_up, const void *ln_gamma, const void *ln_beta,
+                                 const void *W_mix, const void *dy, float *dx, float *dW_K,
+                                 float *dW_V, float *dW_up, float *dgamma, float *dbeta,
+                                 float *dW_mix, void *stream) {
+  set_error("");
+  if (!p) {
+    set_error("plan is NULL");
+    return L3_ERR_INVALID_ARG;
+  }
+  (void)ln_beta;  // beta shifts h, which the forward stored; no step below reads it
+  const l3_dims_t &d = p->dims;
+  const int64_t N = p->n_tokens;
+  for (const void *q : {x, W_K, W_V, W_up, ln_gamma, W_mix, dy, (const void *)dx,
+                        (const void *)dW_K, (const void *)dW_V, (const void *)dW_up,
+                        (const void *)dgamma, (const void *)dbeta, (const void *)dW_mix})
+    if (!q) {
+      set_error("a tensor pointer is NULL");
+      return L3_ERR_INVALID_ARG;
+    }
+  if (p->staged) {
+    set_error("l3_backward takes a plan over the full tables (l3_plan)");
+    return L3_ERR_INVALID_ARG;
+  }
+  const size_t attn_smem = (AT * d.d_in + AT * d.d_emb + 2 * AT * A_MAX_K) * sizeof(float);
+  if (d.k > A_MAX_K || attn_smem > 220 * 1024 || 16 * d.d_up * sizeof(float) > 220 * 1024) {
+    set_error("l3_backward: k, d_in, d_emb or d_up beyond this kernel's shared-memory layout");
+    return L3_ERR_UNSUPPORTED;
+  }
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (N == 0) {
+    L3_CUDA_TRY(cudaMemsetAsync(dW_up, 0, d.d_up * d.d_emb * sizeof(float), s));
+    L3_CUDA_TRY(cudaMemsetAsync(dgamma, 0, d.d_up * sizeof(float), s));
+    L3_CUDA_TRY(cudaMemsetAsync(dbeta, 0, d.d_up * sizeof(float), s));
+    L3_CUDA_TRY(cudaMemsetAsync(dW_mix, 0, d.d_out * (d.d_up + d.d_in) * sizeof(float), s));
+    return L3_OK;
+  }
+  const int wt = d.dtype == L3_BF16 ? T_BF16 : T_F32;
+  const int it = d.dtype == L3_BF16 ? T_F16 : T_F32;  // a and h as the forward stored them
+  const int64_t n_ln = (N + LN_ROWS - 1) / LN_ROWS;
+  // scratch: g_h, z, g_z [N x d_up], g_a [N x d_emb], LayerNorm partials
+  const size_t f = sizeof(float);
+  const size_t bytes = (3 * N * d.d_up + N * d.d_emb + n_ln * 2 * d.d_up) * f;
+  float *scratch = nullptr;
+  cudaError_t e = cudaMallocAsync(reinterpret_cast<void **>(&scratch), bytes, s);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMallocAsync(backward scratch)");
+  float *g_h = scratch, *z = g_h + N * d.d_up, *g_z = z + N * d.d_up, *g_a = g_z + N * d.d_up;
+  float *part = g_a + N * d.d_emb;
+  const int64_t ldm = d.d_up + d.d_in;
+  const char *wmx = reinterpret_cast<const char *>(W_mix) + d.d_up * (wt == T_F32 ? 4 : 2);
+  l3_status st = L3_OK;
+  {
+    LaunchTimer t("bwd_gemms_mix", s);
+    // g_h = g_y W_mix[:, :d_up];  dx = g_y W_mix[:, d_up:]
+    if (st == L3_OK)
+      st = gemm({dy, d.d_out, 1, wt}, {W_mix, 1, ldm, wt}, (int)N, (int)d.d_up, (int)d.d_out, g_h,
+                d.d_up, false, s);
+    if (st == L3_OK)
+      st = gemm({dy, d.d_out, 1, wt}, {wmx, 1, ldm, wt}, (int)N, (int)d.d_in, (int)d.d_out, dx,
+                d.d_in, false, s);
+    // dW_mix = g_y^T [h ; x]
+    if (st == L3_OK)
+      st = gemm({dy, 1, d.d_out, wt}, {p->h_buf, 1, d.d_up, it}, (int)d.d_out, (int)d.d_up, (int)N,
+                dW_mix, ldm, false, s);
+    if (st == L3_OK)
+      st = gemm({dy, 1, d.d_out, wt}, {x, 1, d.d_in, wt}, (int)d.d_out, (int)d.d_in, (int)N,
+                dW_mix + d.d_up, ldm, false, s);
+  }
+  {
+    LaunchTimer t("bwd_layernorm", s);
+    // z = a W_up^T again, then the LayerNorm backward
+    if (st == L3_OK)
+      st = gemm({p->a_buf, d.d_emb, 1, it}, {W_up, d.d_emb, 1, wt}, (int)N, (int)d.d_up,
+                (int)d.d_emb, z, d.d_up, false, s);
+    if (st == L3_OK) {
+      const size_t smem = 8 * 2 * d.d_up * f;
+      if (smem > 48 * 1024)
+        L3_CUDA_TRY(cudaFuncSetAttribute(k_ln_backward, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem));
+      k_ln_backward<<<(unsigned)n_ln, 256, smem, s>>>(z, g_h, ln_gamma, wt, (int)d.d_up,
+                                                      d.ln_eps, N, g_z, part);
+      k_sum_partials<<<(unsigned)((d.d_up + 255) / 256), 256, 0, s>>>(part, (int)n_ln,
+                                                                       (int)d.d_up, dgamma, dbeta);
+      e = cudaGetLastError();
+      if (e != cudaSuccess) st = cuda_fail(e, "LayerNorm backward");
+    }
+  }
+  {
+    LaunchTimer t("bwd_gemms_up", s);
+    // dW_up = g_z^T a;  g_a = g_z W_up
+    if (st == L3_OK)
+      st = gemm({g_z, 1, d.d_up, T_F32}, {p->a_buf, 1, d.d_emb, it}, (int)d.d_up, (int)d.d_emb,
+                (int)N, dW_up, d.d_emb, false, s);
+    if (st == L3_OK)
+      st = gemm({g_z, d.d_up, 1, T_F32}, {W_up, 1, d.d_emb, wt}, (int)N, (int)d.d_emb,
+                (int)d.d_up, g_a, d.d_emb, false, s);
+  }
+  if (st == L3_OK && p->n_groups > 0) {
+    LaunchTimer t("bwd_attention", s);
+    e = cudaFuncSetAttribute(k_attn_backward, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)attn_smem);
+    if (e == cudaSuccess) {
+      k_attn_backward<<<(unsigned)p->n_groups, 256, attn_smem, s>>>(
+          x, W_K, W_V, wt, g_a, p->perm, p->group_tok_start, p->group_row_start, p->group_rows,
+          (int)d.d_in, (int)d.d_emb, dx, dW_K, dW_V);
+      e = cudaGetLastError();
+    }
+    if (e != cudaSuccess) st = cuda_fail(e, "attention backward");
+  }
+  e = cudaFreeAsync(scratch, s);
+  if (st == L3_OK && e != cudaSuccess) st = cuda_fail(e, "cudaFreeAsync(backward scratch)");
+  return st;
+}

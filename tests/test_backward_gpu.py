@@ -1,0 +1,72 @@
+"""l3_backward on the GPU against the fp64 backward oracle (chain rule of
+kimjy99 review, Method, eq. L³), gradient by gradient, on the same seeded
+inputs: max |err| <= 1e-4 x RMS for the fp32 layer and 2e-2 x RMS for bf16
+(the same bars as the forward)."""
+import numpy as np
+import pytest
+import torch
+
+import static_token_routed_b200 as l3
+from l3_cases import EPS, TOL, dims_of, host_workload, rel_max_err, run_forward, to_device
+from oracle import backward as bwd
+from static_token_routed_b200 import workloads as wl
+
+pytestmark = pytest.mark.gpu
+
+NAMES = ("x", "W_K", "W_V", "W_up", "ln_gamma", "ln_beta", "W_mix")
+
+
+def check(w, t, b, dims, tol, seed=0):
+    dev = to_device(t, b)
+    plan = l3.l3_plan(dev["ids"], dev["offsets"], dims)
+    y = torch.empty(b.ids.numel(), w.d_out, dtype=w.torch_dtype, device="cuda")
+    l3.l3_forward(dev["x"], plan, dev["W_K"], dev["W_V"], dev["W_up"], dev["ln_gamma"],
+                  dev["ln_beta"], dev["W_mix"], y)
+    g = torch.Generator().manual_seed(seed)
+    dy = torch.randn(b.ids.numel(), w.d_out, generator=g).to(w.torch_dtype)
+    got = l3.l3_backward(dev["x"], plan, dev["W_K"], dev["W_V"], dev["W_up"], dev["ln_gamma"],
+                         dev["ln_beta"], dev["W_mix"], dy.cuda())
+    l3.l3_forward_status(plan)
+    want = bwd.backward(b.ids, t.offsets, b.x, t.W_K, t.W_V, t.W_up, t.ln_gamma, t.ln_beta,
+                        t.W_mix, EPS, dy)
+    for k in NAMES:
+        err = rel_max_err(got[k].double().cpu().numpy(), want[k])
+        assert err <= tol, (k, err)
+    # deterministic: a second call gives the same bits
+    again = l3.l3_backward(dev["x"], plan, dev["W_K"], dev["W_V"], dev["W_up"], dev["ln_gamma"],
+                           dev["ln_beta"], dev["W_mix"], dy.cuda())
+    for k in NAMES:
+        assert torch.equal(got[k], again[k]), k
+
+
+def small_layer(vocab, rows, n, d_in, d_emb, d_up, d_out, dtype, seed):
+    g = torch.Generator().manual_seed(seed)
+    off = torch.tensor([0] + list(rows), dtype=torch.int64).cumsum(0).to(torch.int32)
+    v = int(off[-1])
+    ids = torch.randint(0, vocab, (n,), generator=g, dtype=torch.int32)
+    mk = lambda *s: (torch.randn(*s, generator=g) / s[-1] ** 0.5).to(dtype)
+    t = wl.Tables(off, mk(v, d_in) * 4, mk(v, d_emb), mk(d_up, d_emb),
+                  (1 + 0.1 * torch.randn(d_up, generator=g)).to(dtype),
+                  (0.1 * torch.randn(d_up, generator=g)).to(dtype), mk(d_out, d_up + d_in))
+    b = wl.Batch(ids, mk(n, d_in) * 4)
+    dims = l3.make_dims(vocab, v, max(rows), d_in, d_emb, d_up, d_out, dtype, EPS)
+    return t, b, dims
+
+
+def test_backward_tiny_fp32():
+    w, t, b = host_workload("tiny_fp32")
+    check(w, t, b, dims_of(w), TOL["fp32"])
+
+
+@pytest.mark.parametrize("vocab,rows,n,d_in,d_emb,d_up,d_out", [
+    # dense groups of both sizes and short ones in one batch
+    (6, (300, 96, 512, 256, 257, 33), 900, 64, 512, 64, 32),
+    # many short groups, single rows among them
+    (50, tuple(int(r) for r in np.random.default_rng(5).integers(1, 9, size=50)), 300, 128, 64,
+     192, 80),
+])
+def test_backward_bf16(vocab, rows, n, d_in, d_emb, d_up, d_out):
+    t, b, dims = small_layer(vocab, rows, n, d_in, d_emb, d_up, d_out, torch.bfloat16, vocab)
+    w = wl.Workload("case", vocab, int(sum(rows)), max(rows), d_in, d_emb, d_up, d_out, n, "bf16",
+                    "zipf", "zipf", 0, 0)
+    check(w, t, b, dims, TOL["bf16"])
