@@ -202,12 +202,14 @@ l3_status l3_forward(const void *x, l3_plan_t plan, const void *W_K, const void 
  *   x .. W_mix   as for l3_forward (dims->dtype); ln_beta is not read
  *   dy           [N x d_out] dims->dtype, caller's token order
  *   dx           fp32 [N x d_in], out
- *   dW_K, dW_V   fp32 [v x d_in], [v x d_emb], out: the rows of every ID in
- *                the batch are written; other rows are left as they were
+ *   dW_K, dW_V   fp32 [v x d_in], [v x d_emb], in/out: the batch's
+ *                gradient is ADDED to the rows of every ID in the batch
+ *                (zero them first for a fresh gradient); other rows untouched
  *   dW_up        fp32 [d_up x d_emb], out
  *   dgamma, dbeta fp32 [d_up], out
  *   dW_mix       fp32 [d_out x (d_up + d_in)], out
- * Deterministic (no atomics). Scratch (3 N d_up + N d_emb floats) is taken
+ * dW_K / dW_V take atomic adds (the order of a group's partial sums may
+ * differ between calls); every other output is deterministic. Scratch (3 N d_up + N d_emb floats) is taken
  * from and returned to the stream-ordered pool on `stream`. Enqueued on
  * `stream`; does not synchronize. Errors: L3_ERR_INVALID_ARG (NULL pointer,
  * a staged plan), L3_ERR_UNSUPPORTED (k > 1024, or d_in / d_emb / d_up too

@@ -217,8 +217,9 @@ def l3_lzw_allocate(corpus, vocab: int, v: int, k: int) -> tuple[np.ndarray, int
 def l3_backward(x, plan: Plan, W_K, W_V, W_up, ln_gamma, ln_beta, W_mix, dy,
                 stream=None) -> dict:
     """Gradients for dL/dy = dy after l3_forward on the same plan and inputs.
-    Returns fp32 tensors: x, W_K, W_V (rows of IDs outside the batch zero),
-    W_up, ln_gamma, ln_beta, W_mix."""
+    Returns fp32 tensors: x, W_K, W_V (fresh zero buffers the library adds
+    the batch's rows into; rows of IDs outside the batch stay zero), W_up,
+    ln_gamma, ln_beta, W_mix."""
     d = plan.dims
     dev = x.device
     f32 = dict(dtype=torch.float32, device=dev)

@@ -14,10 +14,11 @@
 //   dV_t  += p g_a^T, dK_t += g_s x^T, dx += K_t^T g_s
 // The GEMMs run as one strided tiled FFMA kernel (operands read through
 // element strides, so transposed operands need no copies). The attention
-// part runs one CTA per token group: the group's rows belong to that CTA
-// alone, so dW_K / dW_V rows are written without atomics, and eight tokens
-// at a time share every row it reads. The dgamma / dbeta column sums are
-// per-CTA partials reduced by a second kernel (no atomics: deterministic).
+// part runs one CTA per work unit of the plan (a dense tile of up to 128
+// tokens or a tail item of up to 8), eight tokens at a time sharing every row
+// it reads; units of one group add into the group's dW_K / dW_V rows with
+// atomic adds. The dgamma / dbeta column sums are per-CTA partials reduced
+// by a second kernel (deterministic).
 #include <cuda_fp16.h>
 
 #include <algorithm>
@@ -187,7 +188,8 @@ __global__ void __launch_bounds__(256)
                     const float *__restrict__ g_a, const int32_t *__restrict__ perm,
                     const int32_t *__restrict__ group_tok_start,
                     const int32_t *__restrict__ group_row_start,
-                    const int32_t *__restrict__ group_rows, int d_in, int d_emb,
+                    const int32_t *__restrict__ group_rows, const DenseTile *__restrict__ tiles,
+                    int64_t n_tiles, const TailItem *__restrict__ items, int d_in, int d_emb,
                     float *__restrict__ dx, float *__restrict__ dW_K, float *__restrict__ dW_V) {
   extern __shared__ float sm[];
   float *xs = sm;                  // [AT][d_in]
@@ -195,19 +197,38 @@ __global__ void __launch_bounds__(256)
   float *ps = gas + AT * d_emb;    // [AT][A_MAX_K] logits, then p
   float *gs = ps + AT * A_MAX_K;   // [AT][A_MAX_K] g_p, then g_s
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const int g = blockIdx.x;
-  const int t0 = group_tok_start[g], c = group_tok_start[g + 1] - t0;
-  const int64_t r0 = group_row_start[g];
-  const int d = group_rows[g];
+  __shared__ int32_t tok[AT];  // original indices of the chunk's tokens
+  // work unit: a dense tile (up to 128 tokens of one group) or a tail item
+  // (up to 8), the same units as the forward's attention
+  int64_t r0;
+  int d, c, t0 = 0;
+  const TailItem *item = nullptr;
+  if (blockIdx.x < n_tiles) {
+    const DenseTile tl = tiles[blockIdx.x];
+    r0 = group_row_start[tl.group];
+    d = group_rows[tl.group];
+    t0 = tl.tok0;
+    c = min(128, group_tok_start[tl.group + 1] - tl.tok0);
+  } else {
+    item = items + (blockIdx.x - n_tiles);
+    r0 = item->r0;
+    d = item->d;
+    c = item->nt;
+  }
   for (int c0 = 0; c0 < c; c0 += AT) {
     const int nt = min(AT, c - c0);
+    if (threadIdx.x < AT)
+      tok[threadIdx.x] = threadIdx.x < nt
+                             ? (item ? item->tok[c0 + threadIdx.x] : perm[t0 + c0 + threadIdx.x])
+                             : 0;
+    __syncthreads();
     for (int i = threadIdx.x; i < AT * d_in; i += blockDim.x) {
       const int t = i / d_in, col = i % d_in;
-      xs[i] = t < nt ? ldx(x, wtype, (int64_t)perm[t0 + c0 + t] * d_in + col) : 0.f;
+      xs[i] = t < nt ? ldx(x, wtype, (int64_t)tok[t] * d_in + col) : 0.f;
     }
     for (int i = threadIdx.x; i < AT * d_emb; i += blockDim.x) {
       const int t = i / d_emb, col = i % d_emb;
-      gas[i] = t < nt ? g_a[(int64_t)perm[t0 + c0 + t] * d_emb + col] : 0.f;
+      gas[i] = t < nt ? g_a[(int64_t)tok[t] * d_emb + col] : 0.f;
     }
     __syncthreads();
     // logits s = K_j . x_t and g_p = V_j . g_a_t, one warp per row
@@ -277,22 +298,18 @@ __global__ void __launch_bounds__(256)
             acc[t] = fmaf(gst, kv, acc[t]);
             gk = fmaf(gst, xs[t * d_in + col], gk);
           }
-          dW_K[kidx] = c0 == 0 ? gk : dW_K[kidx] + gk;
+          atomicAdd(dW_K + kidx, gk);  // several units may share a group's rows
         }
-        for (int t = 0; t < nt; ++t) dx[(int64_t)perm[t0 + c0 + t] * d_in + col] += acc[t];
+        for (int t = 0; t < nt; ++t) dx[(int64_t)tok[t] * d_in + col] += acc[t];
       }
-    } else {
-      for (int col = threadIdx.x; col < d_in; col += blockDim.x)
-        dW_K[r0 * d_in + col] = 0.f;  // one row: p = 1, no gradient reaches K
-    }
+    }  // one row: p = 1, no gradient reaches K
     // dV_j (+)= sum_t p[t][j] g_a_t
     for (int col = threadIdx.x; col < d_emb; col += blockDim.x) {
       for (int j = 0; j < d; ++j) {
         float gv = 0.f;
 #pragma unroll
         for (int t = 0; t < AT; ++t) gv = fmaf(ps[t * A_MAX_K + j], gas[t * d_emb + col], gv);
-        const int64_t vidx = (r0 + j) * d_emb + col;
-        dW_V[vidx] = c0 == 0 ? gv : dW_V[vidx] + gv;
+        atomicAdd(dW_V + (r0 + j) * d_emb + col, gv);
       }
     }
     __syncthreads();
@@ -401,14 +418,16 @@ extern "C" l3_status l3_backward(const void *x, l3_plan_t p, const void *W_K, co
       st = gemm({g_z, d.d_up, 1, T_F32}, {W_up, 1, d.d_emb, wt}, (int)N, (int)d.d_emb,
                 (int)d.d_up, g_a, d.d_emb, false, s);
   }
-  if (st == L3_OK && p->n_groups > 0) {
+  const int64_t n_units = p->n_dense_tiles + p->n_tail_items;
+  if (st == L3_OK && n_units > 0) {
     LaunchTimer t("bwd_attention", s);
     e = cudaFuncSetAttribute(k_attn_backward, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)attn_smem);
     if (e == cudaSuccess) {
-      k_attn_backward<<<(unsigned)p->n_groups, 256, attn_smem, s>>>(
+      k_attn_backward<<<(unsigned)n_units, 256, attn_smem, s>>>(
           x, W_K, W_V, wt, g_a, p->perm, p->group_tok_start, p->group_row_start, p->group_rows,
-          (int)d.d_in, (int)d.d_emb, dx, dW_K, dW_V);
+          p->dense_tiles, p->n_dense_tiles, p->tail_items, (int)d.d_in, (int)d.d_emb, dx, dW_K,
+          dW_V);
       e = cudaGetLastError();
     }
     if (e != cudaSuccess) st = cuda_fail(e, "attention backward");

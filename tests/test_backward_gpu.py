@@ -32,11 +32,15 @@ def check(w, t, b, dims, tol, seed=0):
     for k in NAMES:
         err = rel_max_err(got[k].double().cpu().numpy(), want[k])
         assert err <= tol, (k, err)
-    # deterministic: a second call gives the same bits
+    # a second call gives the same bits, except dW_K / dW_V whose rows take
+    # atomic adds from several units of a group
     again = l3.l3_backward(dev["x"], plan, dev["W_K"], dev["W_V"], dev["W_up"], dev["ln_gamma"],
                            dev["ln_beta"], dev["W_mix"], dy.cuda())
     for k in NAMES:
-        assert torch.equal(got[k], again[k]), k
+        if k in ("W_K", "W_V"):
+            assert rel_max_err(again[k].double().cpu().numpy(), want[k]) <= tol, k
+        else:
+            assert torch.equal(got[k], again[k]), k
 
 
 def small_layer(vocab, rows, n, d_in, d_emb, d_up, d_out, dtype, seed):
@@ -61,6 +65,8 @@ def test_backward_tiny_fp32():
 @pytest.mark.parametrize("vocab,rows,n,d_in,d_emb,d_up,d_out", [
     # dense groups of both sizes and short ones in one batch
     (6, (300, 96, 512, 256, 257, 33), 900, 64, 512, 64, 32),
+    # groups of several 128-token tiles (units of one group share its rows)
+    (3, (511, 260, 96), 1200, 128, 256, 64, 32),
     # many short groups, single rows among them
     (50, tuple(int(r) for r in np.random.default_rng(5).integers(1, 9, size=50)), 300, 128, 64,
      192, 80),
