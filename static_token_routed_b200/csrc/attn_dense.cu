@@ -64,15 +64,13 @@ template <bool SMALL>
 struct DenseCfg {
   static constexpr int REGION = SMALL ? 96 * 1024 : 192 * 1024;  // S ring, later P + V slices
   static constexpr int TMEM_COLS = SMALL ? 256 : 512;
-  static constexpr int MAX_ROWS = SMALL ? 256 : MAX_D;
   static constexpr int MIN_BLOCKS = SMALL ? 2 : 1;
 };
-static_assert(DenseCfg<true>::MAX_ROWS == DENSE_SMALL_ROWS, "plan and kernel disagree on small d_t");
+static_assert(DenseCfg<true>::TMEM_COLS == DENSE_SMALL_ROWS, "plan and kernel disagree on small d_t");
 constexpr int V_ROWS = 16;              // d_t rows per V slice (one MMA k-step)
 constexpr int V_BLOCK = V_ROWS * 128;   // one 64-column block of a V slice
 constexpr int DENSE_THREADS = 384;  // 0 TMA, 1 MMA, 2-3 x gather, 4-11 softmax / epilogue
 constexpr int SOFTMAX_THREADS = 256;
-constexpr float LOG2E = 1.4426950408889634f;
 
 struct DenseBars {
   uint64_t xfull[MAX_STAGES], kfull[MAX_STAGES], sempty[MAX_STAGES];

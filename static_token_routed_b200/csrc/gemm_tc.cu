@@ -81,7 +81,7 @@ __device__ __forceinline__ uint8_t *align1024(uint8_t *p) {
 __device__ void drain_after_abort(Bars *b, int stages, const uint32_t *armed_parity,
                                   const bool *armed, bool is_producer, bool is_mma,
                                   const Abort &ab) {
-  Abort quiet{ab.flag, ab.err};
+  (void)ab;  // the drain ignores the abort flag and keeps only the time bound
   if (is_producer) {
     for (int s = 0; s < stages; ++s)
       if (armed[s]) {
@@ -99,7 +99,6 @@ __device__ void drain_after_abort(Bars *b, int stages, const uint32_t *armed_par
     while (!mbar_try_wait(a, 0) && globaltimer_ns() - t0 < WAIT_LIMIT_NS) {
     }
   }
-  (void)quiet;
 }
 
 // ---------------------------------------------------------------------------
