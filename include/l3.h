@@ -194,7 +194,10 @@ l3_status l3_forward(const void *x, l3_plan_t plan, const void *W_K, const void 
 
 /*
  * l3_backward — gradients of the layer (kimjy99 review, Method, eq. L³, by
- * the chain rule) for dL/dy, on CUDA cores in fp32 arithmetic.
+ * the chain rule) for dL/dy. bf16 layers run the dense GEMMs on the tensor
+ * cores (bf16 operands, fp32 accumulate; g_z enters g_a as the sum of two
+ * bf16 parts) and the rest on CUDA cores in fp32; fp32 layers run all of it
+ * on CUDA cores in fp32.
  *
  * Call after l3_forward on the same plan and the same inputs: it reuses the
  * a = V_t^T softmax(K_t x) and h = LayerNorm(W_up a) that forward stored
@@ -209,9 +212,11 @@ l3_status l3_forward(const void *x, l3_plan_t plan, const void *W_K, const void 
  *   dgamma, dbeta fp32 [d_up], out
  *   dW_mix       fp32 [d_out x (d_up + d_in)], out
  * dW_K / dW_V take atomic adds (the order of a group's partial sums may
- * differ between calls); every other output is deterministic. Scratch (3 N d_up + N d_emb floats) is taken
- * from and returned to the stream-ordered pool on `stream`. Enqueued on
- * `stream`; does not synchronize. Errors: L3_ERR_INVALID_ARG (NULL pointer,
+ * differ between calls); every other output is deterministic. Scratch (about
+ * 3 N d_up + N d_emb floats, plus bf16 transposes of g_y, [h ; x], g_z and a
+ * on the tensor-core path) comes from the library's device block cache
+ * (cudaMalloc on a miss) and goes back to it, ordered after the work on
+ * `stream`. Enqueued on `stream`; does not synchronize. Errors: L3_ERR_INVALID_ARG (NULL pointer,
  * a staged plan), L3_ERR_UNSUPPORTED (k > 1024, or d_in / d_emb / d_up too
  * wide for its shared-memory layout), L3_ERR_OOM, L3_ERR_CUDA.
  */

@@ -69,12 +69,16 @@ l3_status aux_for(int device, Aux **out) {
   return L3_OK;
 }
 
+}  // namespace
+
 // Plan memory cache. A destroyed plan's block goes back to a per-process list
 // with an event recorded on the stream that last used it; a new plan takes a
 // cached block on its device that is large enough and whose event has
 // completed, so a plan per batch costs no allocator call after warm-up, and a
 // plan built on one stream while an earlier forward still runs on another
-// never waits for it or grows the pool.
+// never waits for it or grows the pool. The backward pass takes its scratch
+// from the same cache.
+namespace {
 struct CachedBlock {
   void *ptr;
   size_t bytes;
@@ -84,6 +88,7 @@ struct CachedBlock {
 std::mutex g_cache_mu;
 std::vector<CachedBlock> g_cache;
 constexpr size_t CACHE_MAX_BLOCKS = 4;
+}  // namespace
 
 // returns a cached block of at least `bytes` on `device` (and its size), or nullptr
 void *cache_take(int device, size_t bytes, size_t *got) {
@@ -127,6 +132,8 @@ void cache_give(void *ptr, size_t bytes, int device, cudaStream_t s) {
     if (cur != old.device) cudaSetDevice(cur);
   }
 }
+
+namespace {
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 

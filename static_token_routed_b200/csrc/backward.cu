@@ -12,7 +12,12 @@
 //   dW_up  = g_z^T a                    g_a = g_z W_up
 //   g_p    = V_t g_a, g_s = p (g_p - p.g_p)
 //   dV_t  += p g_a^T, dK_t += g_s x^T, dx += K_t^T g_s
-// The GEMMs run as one strided tiled FFMA kernel (operands read through
+// bf16 layers run the GEMMs on the tensor cores (the pair kernel of the
+// forward, fp32 output): that kernel reads both operands K-major, so the
+// operands whose K is the token axis or whose rows are the wrong way round
+// are first transposed into bf16 copies (fp16 a and h become bf16 there,
+// since one MMA takes one operand type), and g_z is kept in bf16. fp32
+// layers run them as one strided tiled FFMA kernel (operands read through
 // element strides, so transposed operands need no copies). The attention
 // part runs one CTA per work unit of the plan (a dense tile of up to 128
 // tokens or a tail item of up to 8), eight tokens at a time sharing every row
@@ -107,14 +112,79 @@ l3_status gemm(Operand A, Operand B, int M, int N, int K, float *C, int64_t ldc,
   return L3_OK;
 }
 
+// out[c][r] = in[r][c] as bf16: in is [R x C] 16-bit (fp16 or bf16) with row
+// stride ld_in, out [C x ld_out]. 64 x 64 tiles, a grid-stride loop over them;
+// 16-byte loads and stores, so C, ld_in and ld_out are multiples of 8 (the
+// last store of a row may run into out's padding up to ld_out).
+constexpr int TT = 64;
+
+template <typename Tin>
+__global__ void __launch_bounds__(256)
+    k_transpose_bf16(const Tin *__restrict__ in, int64_t ld_in, int64_t R, int64_t C,
+                     __nv_bfloat16 *__restrict__ out, int64_t ld_out) {
+  __shared__ float tile[TT][TT + 1];
+  const int64_t tiles_c = (C + TT - 1) / TT, n_tiles = tiles_c * ((R + TT - 1) / TT);
+  const int tid = threadIdx.x;
+  for (int64_t t = blockIdx.x; t < n_tiles; t += gridDim.x) {
+    const int64_t r0 = (t / tiles_c) * TT, c0 = (t % tiles_c) * TT;
+    // load: 8 threads per 64-element row, 32 rows per pass
+    for (int rr = tid / 8; rr < TT; rr += 32) {
+      const int cc = (tid % 8) * 8;
+      const int64_t r = r0 + rr, c = c0 + cc;
+      float f[8];
+      if (r < R && c < C) {
+        const uint4 u = *reinterpret_cast<const uint4 *>(in + r * ld_in + c);
+        const Tin *e = reinterpret_cast<const Tin *>(&u);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) f[i] = static_cast<float>(e[i]);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) f[i] = 0.f;
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) tile[rr][cc + i] = f[i];
+    }
+    __syncthreads();
+    // store: 8 threads per 64-element output row
+    for (int cc = tid / 8; cc < TT; cc += 32) {
+      const int rr = (tid % 8) * 8;
+      const int64_t c = c0 + cc, r = r0 + rr;
+      if (c < C && r < R) {
+        uint4 u;
+        __nv_bfloat162 *o = reinterpret_cast<__nv_bfloat162 *>(&u);
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          o[i] = __floats2bfloat162_rn(tile[rr + 2 * i][cc], tile[rr + 2 * i + 1][cc]);
+        *reinterpret_cast<uint4 *>(out + c * ld_out + r) = u;
+      }
+    }
+    __syncthreads();
+  }
+}
+
+template <typename Tin>
+l3_status transpose_bf16(const void *in, int64_t ld_in, int64_t R, int64_t C, void *out,
+                         int64_t ld_out, int n_sms, cudaStream_t s) {
+  if (R == 0 || C == 0) return L3_OK;
+  const int64_t n_tiles = ((R + TT - 1) / TT) * ((C + TT - 1) / TT);
+  const unsigned grid = (unsigned)std::min<int64_t>(n_tiles, (int64_t)n_sms * 8);
+  k_transpose_bf16<Tin><<<grid, 256, 0, s>>>(reinterpret_cast<const Tin *>(in), ld_in, R, C,
+                                             reinterpret_cast<__nv_bfloat16 *>(out), ld_out);
+  L3_CUDA_TRY(cudaGetLastError());
+  return L3_OK;
+}
+
 // ---------------------------------------------------------------- LayerNorm
 constexpr int LN_ROWS = 16;  // token rows per CTA (one warp per row at a time)
 
-// g_z from g_h and z for LN_ROWS rows per CTA; column partials of
+// g_z from g_h and z for LN_ROWS rows per CTA (into g_z16 + g_z16_lo, its
+// bf16 rounding and the bf16 rounding of the rest, when they are given, else
+// into g_z as fp32); column partials of
 // dgamma = sum g_h hhat and dbeta = sum g_h into part[cta][2][d_up]
 __global__ void __launch_bounds__(256)
     k_ln_backward(const float *__restrict__ z, const float *__restrict__ g_h, const void *gamma,
                   int gtype, int d_up, float eps, int64_t M, float *__restrict__ g_z,
+                  __nv_bfloat16 *__restrict__ g_z16, __nv_bfloat16 *__restrict__ g_z16_lo,
                   float *__restrict__ part) {
   extern __shared__ float sm[];  // [8 warps][2][d_up]
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -146,10 +216,15 @@ __global__ void __launch_bounds__(256)
     }
     m1 /= d_up;
     m2 /= d_up;
-    float *gzr = g_z + row * d_up;
     for (int u = lane; u < d_up; u += 32) {
       const float hh = (zr[u] - mu) * rstd, gh = gr[u] * ldx(gamma, gtype, u);
-      gzr[u] = (gh - m1 - hh * m2) * rstd;
+      const float gz = (gh - m1 - hh * m2) * rstd;
+      if (g_z16) {
+        const __nv_bfloat16 hi = __float2bfloat16_rn(gz);
+        g_z16[row * d_up + u] = hi;
+        g_z16_lo[row * d_up + u] = __float2bfloat16_rn(gz - __bfloat162float(hi));
+      } else
+        g_z[row * d_up + u] = gz;
     }
   }
   __syncthreads();
@@ -361,62 +436,146 @@ extern "C" l3_status l3_backward(const void *x, l3_plan_t p, const void *W_K, co
   const int wt = d.dtype == L3_BF16 ? T_BF16 : T_F32;
   const int it = d.dtype == L3_BF16 ? T_F16 : T_F32;  // a and h as the forward stored them
   const int64_t n_ln = (N + LN_ROWS - 1) / LN_ROWS;
-  // scratch: g_h, z, g_z [N x d_up], g_a [N x d_emb], LayerNorm partials
+  const int64_t D = d.d_up + d.d_in;  // columns of W_mix
+  auto a16 = [](const void *q) { return (reinterpret_cast<uintptr_t>(q) & 15u) == 0; };
+  // tensor cores for bf16 layers whose forward ran on them (it left the fp16
+  // W_up copy in the plan) and whose operands meet the TMA alignment
+  const bool tc = p->tc_gemm && a16(x) && a16(W_up) && a16(W_mix) && a16(dy) && a16(dx) &&
+                  a16(dW_up) && a16(dW_mix);
+  const int64_t ldn = (N + 7) / 8 * 8;  // row stride of the copies whose rows run over tokens
+  // scratch: g_h, z [N x d_up] fp32, g_a [N x d_emb] fp32, LayerNorm partials,
+  // g_z [N x d_up] (bf16 on the tensor-core path, else fp32) and the
+  // tensor-core path's bf16 transposes
   const size_t f = sizeof(float);
-  const size_t bytes = (3 * N * d.d_up + N * d.d_emb + n_ln * 2 * d.d_up) * f;
-  float *scratch = nullptr;
-  cudaError_t e = cudaMallocAsync(reinterpret_cast<void **>(&scratch), bytes, s);
-  if (e != cudaSuccess) return cuda_fail(e, "cudaMallocAsync(backward scratch)");
-  float *g_h = scratch, *z = g_h + N * d.d_up, *g_z = z + N * d.d_up, *g_a = g_z + N * d.d_up;
-  float *part = g_a + N * d.d_emb;
-  const int64_t ldm = d.d_up + d.d_in;
+  size_t bytes = 0;
+  auto take = [&](size_t b) {
+    const size_t o = bytes;
+    bytes += (b + 255) / 256 * 256;
+    return o;
+  };
+  const size_t o_gh = take(N * d.d_up * f), o_z = take(N * d.d_up * f),
+               o_ga = take(N * d.d_emb * f), o_part = take(n_ln * 2 * d.d_up * f),
+               o_gz = take(N * d.d_up * (tc ? 2 : f)), o_gzlo = take(tc ? N * d.d_up * 2 : 0);
+  size_t o_wmt = 0, o_gyt = 0, o_hxt = 0, o_gzt = 0, o_at = 0, o_wut = 0;
+  if (tc) {
+    o_wmt = take(D * d.d_out * 2);      // W_mix^T   [D x d_out]
+    o_gyt = take(d.d_out * ldn * 2);    // g_y^T     [d_out x N]
+    o_hxt = take(D * ldn * 2);          // [h ; x]^T [D x N]
+    o_gzt = take(d.d_up * ldn * 2);     // g_z^T     [d_up x N]
+    o_at = take(d.d_emb * ldn * 2);     // a^T       [d_emb x N]
+    o_wut = take(d.d_emb * d.d_up * 2); // W_up^T    [d_emb x d_up]
+  }
+  // from the device block cache, so a backward per batch maps no memory
+  // after warm-up
+  size_t got = 0;
+  char *scratch = reinterpret_cast<char *>(cache_take(p->device, bytes, &got));
+  cudaError_t e = cudaSuccess;
+  if (!scratch) {
+    e = cudaMalloc(reinterpret_cast<void **>(&scratch), bytes);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMalloc(backward scratch)");
+    got = bytes;
+  }
+  float *g_h = reinterpret_cast<float *>(scratch + o_gh);
+  float *z = reinterpret_cast<float *>(scratch + o_z);
+  float *g_a = reinterpret_cast<float *>(scratch + o_ga);
+  float *part = reinterpret_cast<float *>(scratch + o_part);
+  float *g_z = tc ? nullptr : reinterpret_cast<float *>(scratch + o_gz);
+  __nv_bfloat16 *g_z16 = tc ? reinterpret_cast<__nv_bfloat16 *>(scratch + o_gz) : nullptr;
+  __nv_bfloat16 *g_z16_lo = tc ? reinterpret_cast<__nv_bfloat16 *>(scratch + o_gzlo) : nullptr;
+  auto bf = [&](size_t o) { return reinterpret_cast<__nv_bfloat16 *>(scratch + o); };
+  __nv_bfloat16 *wmt = bf(o_wmt), *gyt = bf(o_gyt), *hxt = bf(o_hxt), *gzt = bf(o_gzt),
+                *at = bf(o_at), *wut = bf(o_wut);
+  int *err = p->dev_flags + 1;  // a tensor-core wait that gives up reports here
+  const int dev = p->device;
+  int n_sms = 148;
+  cudaDeviceGetAttribute(&n_sms, cudaDevAttrMultiProcessorCount, dev);
+  using BF = __nv_bfloat16;
+  const int64_t ldm = D;
   const char *wmx = reinterpret_cast<const char *>(W_mix) + d.d_up * (wt == T_F32 ? 4 : 2);
   l3_status st = L3_OK;
+  if (tc) {
+    LaunchTimer t("bwd_transpose", s);
+    if (st == L3_OK) st = transpose_bf16<BF>(W_mix, D, d.d_out, D, wmt, d.d_out, n_sms, s);
+    if (st == L3_OK) st = transpose_bf16<BF>(dy, d.d_out, N, d.d_out, gyt, ldn, n_sms, s);
+    if (st == L3_OK) st = transpose_bf16<__half>(p->h_buf, d.d_up, N, d.d_up, hxt, ldn, n_sms, s);
+    if (st == L3_OK)
+      st = transpose_bf16<BF>(x, d.d_in, N, d.d_in, hxt + d.d_up * ldn, ldn, n_sms, s);
+    if (st == L3_OK) st = transpose_bf16<BF>(W_up, d.d_emb, d.d_up, d.d_emb, wut, d.d_up, n_sms, s);
+    if (st == L3_OK) st = transpose_bf16<__half>(p->a_buf, d.d_emb, N, d.d_emb, at, ldn, n_sms, s);
+  }
   {
     LaunchTimer t("bwd_gemms_mix", s);
-    // g_h = g_y W_mix[:, :d_up];  dx = g_y W_mix[:, d_up:]
-    if (st == L3_OK)
-      st = gemm({dy, d.d_out, 1, wt}, {W_mix, 1, ldm, wt}, (int)N, (int)d.d_up, (int)d.d_out, g_h,
-                d.d_up, false, s);
-    if (st == L3_OK)
-      st = gemm({dy, d.d_out, 1, wt}, {wmx, 1, ldm, wt}, (int)N, (int)d.d_in, (int)d.d_out, dx,
-                d.d_in, false, s);
-    // dW_mix = g_y^T [h ; x]
-    if (st == L3_OK)
-      st = gemm({dy, 1, d.d_out, wt}, {p->h_buf, 1, d.d_up, it}, (int)d.d_out, (int)d.d_up, (int)N,
-                dW_mix, ldm, false, s);
-    if (st == L3_OK)
-      st = gemm({dy, 1, d.d_out, wt}, {x, 1, d.d_in, wt}, (int)d.d_out, (int)d.d_in, (int)N,
-                dW_mix + d.d_up, ldm, false, s);
+    // g_h = g_y W_mix[:, :d_up];  dx = g_y W_mix[:, d_up:];  dW_mix = g_y^T [h ; x]
+    if (tc) {
+      if (st == L3_OK)
+        st = launch_gemm_nt_tc(dy, wmt, nullptr, nullptr, false, N, d.d_up, d.d_out, d.d_out,
+                               d.d_out, g_h, d.d_up, err, dev, s);
+      if (st == L3_OK)
+        st = launch_gemm_nt_tc(dy, wmt + d.d_up * d.d_out, nullptr, nullptr, false, N, d.d_in,
+                               d.d_out, d.d_out, d.d_out, dx, d.d_in, err, dev, s);
+      if (st == L3_OK)
+        st = launch_gemm_nt_tc(gyt, hxt, nullptr, nullptr, false, d.d_out, D, N, ldn, ldn, dW_mix,
+                               D, err, dev, s);
+    } else {
+      if (st == L3_OK)
+        st = gemm({dy, d.d_out, 1, wt}, {W_mix, 1, ldm, wt}, (int)N, (int)d.d_up, (int)d.d_out,
+                  g_h, d.d_up, false, s);
+      if (st == L3_OK)
+        st = gemm({dy, d.d_out, 1, wt}, {wmx, 1, ldm, wt}, (int)N, (int)d.d_in, (int)d.d_out, dx,
+                  d.d_in, false, s);
+      if (st == L3_OK)
+        st = gemm({dy, 1, d.d_out, wt}, {p->h_buf, 1, d.d_up, it}, (int)d.d_out, (int)d.d_up,
+                  (int)N, dW_mix, ldm, false, s);
+      if (st == L3_OK)
+        st = gemm({dy, 1, d.d_out, wt}, {x, 1, d.d_in, wt}, (int)d.d_out, (int)d.d_in, (int)N,
+                  dW_mix + d.d_up, ldm, false, s);
+    }
   }
   {
     LaunchTimer t("bwd_layernorm", s);
-    // z = a W_up^T again, then the LayerNorm backward
+    // z = a W_up^T again (the tensor-core path with the forward's fp16
+    // operands, so z is the forward's), then the LayerNorm backward
     if (st == L3_OK)
-      st = gemm({p->a_buf, d.d_emb, 1, it}, {W_up, d.d_emb, 1, wt}, (int)N, (int)d.d_up,
-                (int)d.d_emb, z, d.d_up, false, s);
+      st = tc ? launch_gemm_nt_tc(p->a_buf, p->w_up16, nullptr, nullptr, true, N, d.d_up, d.d_emb,
+                                  d.d_emb, d.d_emb, z, d.d_up, err, dev, s)
+              : gemm({p->a_buf, d.d_emb, 1, it}, {W_up, d.d_emb, 1, wt}, (int)N, (int)d.d_up,
+                     (int)d.d_emb, z, d.d_up, false, s);
     if (st == L3_OK) {
       const size_t smem = 8 * 2 * d.d_up * f;
       if (smem > 48 * 1024)
-        L3_CUDA_TRY(cudaFuncSetAttribute(k_ln_backward, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem));
-      k_ln_backward<<<(unsigned)n_ln, 256, smem, s>>>(z, g_h, ln_gamma, wt, (int)d.d_up,
-                                                      d.ln_eps, N, g_z, part);
-      k_sum_partials<<<(unsigned)((d.d_up + 255) / 256), 256, 0, s>>>(part, (int)n_ln,
-                                                                       (int)d.d_up, dgamma, dbeta);
-      e = cudaGetLastError();
+        e = cudaFuncSetAttribute(k_ln_backward, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)smem);
+      if (e == cudaSuccess) {
+        k_ln_backward<<<(unsigned)n_ln, 256, smem, s>>>(z, g_h, ln_gamma, wt, (int)d.d_up,
+                                                        d.ln_eps, N, g_z, g_z16, g_z16_lo, part);
+        k_sum_partials<<<(unsigned)((d.d_up + 255) / 256), 256, 0, s>>>(
+            part, (int)n_ln, (int)d.d_up, dgamma, dbeta);
+        e = cudaGetLastError();
+      }
       if (e != cudaSuccess) st = cuda_fail(e, "LayerNorm backward");
     }
   }
   {
     LaunchTimer t("bwd_gemms_up", s);
-    // dW_up = g_z^T a;  g_a = g_z W_up
-    if (st == L3_OK)
-      st = gemm({g_z, 1, d.d_up, T_F32}, {p->a_buf, 1, d.d_emb, it}, (int)d.d_up, (int)d.d_emb,
-                (int)N, dW_up, d.d_emb, false, s);
-    if (st == L3_OK)
-      st = gemm({g_z, d.d_up, 1, T_F32}, {W_up, 1, d.d_emb, wt}, (int)N, (int)d.d_emb,
-                (int)d.d_up, g_a, d.d_emb, false, s);
+    // dW_up = g_z^T a;  g_a = g_z W_up, with g_z as the sum of its two bf16
+    // parts: the attention backward's g_s = p (g_p - p . g_p) cancels, and
+    // bf16 rounding of g_z alone shows in dW_K beyond the bf16 bar
+    if (tc) {
+      if (st == L3_OK) st = transpose_bf16<BF>(g_z16, d.d_up, N, d.d_up, gzt, ldn, n_sms, s);
+      if (st == L3_OK)
+        st = launch_gemm_nt_tc(gzt, at, nullptr, nullptr, false, d.d_up, d.d_emb, N, ldn, ldn,
+                               dW_up, d.d_emb, err, dev, s);
+      if (st == L3_OK)
+        st = launch_gemm_nt_tc(g_z16, wut, g_z16_lo, wut, false, N, d.d_emb, d.d_up, d.d_up,
+                               d.d_up, g_a, d.d_emb, err, dev, s);
+    } else {
+      if (st == L3_OK)
+        st = gemm({g_z, 1, d.d_up, T_F32}, {p->a_buf, 1, d.d_emb, it}, (int)d.d_up, (int)d.d_emb,
+                  (int)N, dW_up, d.d_emb, false, s);
+      if (st == L3_OK)
+        st = gemm({g_z, d.d_up, 1, T_F32}, {W_up, 1, d.d_emb, wt}, (int)N, (int)d.d_emb,
+                  (int)d.d_up, g_a, d.d_emb, false, s);
+    }
   }
   const int64_t n_units = p->n_dense_tiles + p->n_tail_items;
   if (st == L3_OK && n_units > 0) {
@@ -432,7 +591,6 @@ extern "C" l3_status l3_backward(const void *x, l3_plan_t p, const void *W_K, co
     }
     if (e != cudaSuccess) st = cuda_fail(e, "attention backward");
   }
-  e = cudaFreeAsync(scratch, s);
-  if (st == L3_OK && e != cudaSuccess) st = cuda_fail(e, "cudaFreeAsync(backward scratch)");
+  cache_give(scratch, got, p->device, s);
   return st;
 }

@@ -51,8 +51,9 @@ struct MixParams {
   int M, N;        // tokens, d_out
   int kb0, kb1;    // 64-wide k-blocks of the h range and of the x range
   int n_tiles_n, n_tiles;
-  __nv_bfloat16 *y;
+  void *y;         // bf16 (the layer's y) or fp32 (the backward pass's GEMMs)
   int64_t ldy;
+  uint32_t idesc0, idesc1;  // instruction descriptors of the two ranges (fp32-output form)
   int *err;
 };
 
@@ -103,6 +104,9 @@ __device__ void drain_after_abort(Bars *b, int stages, const uint32_t *armed_par
 
 // ---------------------------------------------------------------------------
 // y = W_mix[:, :d_up] h + W_mix[:, d_up:] x on CTA pairs (tcgen05 cta_group::2)
+//
+// The same kernel, instantiated with F32OUT, is the backward pass's NT GEMM
+// C = A B^T with fp32 output (one K-range, operand types from the params).
 //
 // Two CTAs on neighbouring SMs compute one 256 x 256 tile of y: each loads its
 // own 128 rows of the A operand (h or x) and its own 128 of the 256 rows of
@@ -160,6 +164,7 @@ __device__ __forceinline__ void umma_commit_pair(uint64_t *bar) {
       : "memory");
 }
 
+template <bool F32OUT>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
     k_mix_gemm_pair(const __grid_constant__ CUtensorMap mA0, const __grid_constant__ CUtensorMap mB0,
                     const __grid_constant__ CUtensorMap mA1, const __grid_constant__ CUtensorMap mB1,
@@ -264,7 +269,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           tc_fence_after();
           const uint32_t sa = smem_u32(ring + stage * STAGE2_BYTES);
           const uint32_t sb = sa + A_BYTES;
-          const uint32_t idesc = kb < P.kb0 ? IDESC2_F16 : IDESC2_BF16;
+          const uint32_t idesc = F32OUT ? (kb < P.kb0 ? P.idesc0 : P.idesc1)
+                                        : (kb < P.kb0 ? IDESC2_F16 : IDESC2_BF16);
 #pragma unroll
           for (int k = 0; k < BK / 16; ++k)
             umma_f16_pair(d, sdesc_sw128(sa + k * 32, 16, 1024), sdesc_sw128(sb + k * 32, 16, 1024),
@@ -300,13 +306,22 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       tc_fence_after();
       const int m = (tile / P.n_tiles_n) * (2 * BM) + (int)rank * BM + r;
       const int n0 = (tile % P.n_tiles_n) * BN;
-      __nv_bfloat16 *yrow = P.y + (int64_t)m * P.ldy + n0;
+      __nv_bfloat16 *yrow = reinterpret_cast<__nv_bfloat16 *>(P.y) + (int64_t)m * P.ldy + n0;
+      float *crow = reinterpret_cast<float *>(P.y) + (int64_t)m * P.ldy + n0;
 #pragma unroll 1
       for (int c = 0; c < BN / 32; ++c) {
         uint32_t v[32];
         tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + acc * BN + c * 32, v);
         tmem_wait_ld();
-        if (m < P.M) {
+        if (F32OUT) {
+          if (m < P.M) {
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+              if (n0 + c * 32 + j * 4 < P.N)
+                *reinterpret_cast<uint4 *>(crow + c * 32 + j * 4) =
+                    make_uint4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+          }
+        } else if (m < P.M) {
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
             const int col = n0 + c * 32 + j * 8;
@@ -815,13 +830,15 @@ l3_status launch_mix_tc(const l3_plan_s *p, const void *x, const void *W_mix, vo
   P.kb1 = (int)(d.d_in / BK);
   P.n_tiles_n = (int)((d.d_out + BN - 1) / BN);
   P.n_tiles = (int)((M + 2 * BM - 1) / (2 * BM)) * P.n_tiles_n;
-  P.y = reinterpret_cast<__nv_bfloat16 *>(y);
+  P.y = y;
   P.ldy = d.d_out;
+  P.idesc0 = IDESC2_F16;
+  P.idesc1 = IDESC2_BF16;
   P.err = p->dev_flags + 1;
   static bool attr[64] = {};
   if (!attr[p->device & 63]) {
-    L3_CUDA_TRY(cudaFuncSetAttribute(k_mix_gemm_pair, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     (int)MIX2_SMEM));
+    L3_CUDA_TRY(cudaFuncSetAttribute(k_mix_gemm_pair<false>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, (int)MIX2_SMEM));
     attr[p->device & 63] = true;
   }
   // persistent: one CTA pair per two SMs, 256 x 256 tiles
@@ -839,7 +856,70 @@ l3_status launch_mix_tc(const l3_plan_s *p, const void *x, const void *W_mix, vo
   cfg.attrs = at;
   cfg.numAttrs = 1;
   LaunchTimer t("mix_gemm_tc", s);
-  L3_CUDA_TRY(cudaLaunchKernelEx(&cfg, k_mix_gemm_pair, mA0, mB0, mA1, mB1, P));
+  L3_CUDA_TRY(cudaLaunchKernelEx(&cfg, k_mix_gemm_pair<false>, mA0, mB0, mA1, mB1, P));
+  return L3_OK;
+}
+
+l3_status launch_gemm_nt_tc(const void *A, const void *B, const void *A1, const void *B1, bool f16,
+                            int64_t M, int64_t N, int64_t K, int64_t lda, int64_t ldb, float *C,
+                            int64_t ldc, int *err, int device, cudaStream_t s) {
+  if (M == 0 || N == 0) return L3_OK;
+  if (!A1 != !B1) {
+    set_error("launch_gemm_nt_tc: the second range needs both operands");
+    return L3_ERR_INVALID_ARG;
+  }
+  const uintptr_t mis = reinterpret_cast<uintptr_t>(A) | reinterpret_cast<uintptr_t>(B) |
+                        reinterpret_cast<uintptr_t>(A1) | reinterpret_cast<uintptr_t>(B1) |
+                        reinterpret_cast<uintptr_t>(C);
+  if (K < 1 || M > INT32_MAX || N > INT32_MAX || (mis & 15) || lda % 8 || ldb % 8 || ldc % 4 ||
+      N % 4 || lda < K || ldb < K || ldc < N) {
+    set_error("launch_gemm_nt_tc: shape, stride or alignment outside the kernel's layout");
+    return L3_ERR_UNSUPPORTED;
+  }
+  const CUtensorMapDataType dt =
+      f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  CUtensorMap mA, mB, mA1, mB1;
+  l3_status st;
+  if ((st = make_map(&mA, A, dt, M, K, lda, BM)) != L3_OK) return st;
+  if ((st = make_map(&mB, B, dt, N, K, ldb, B2_ROWS)) != L3_OK) return st;
+  if (A1) {
+    if ((st = make_map(&mA1, A1, dt, M, K, lda, BM)) != L3_OK) return st;
+    if ((st = make_map(&mB1, B1, dt, N, K, ldb, B2_ROWS)) != L3_OK) return st;
+  } else {
+    mA1 = mA;  // never read (kb1 = 0)
+    mB1 = mB;
+  }
+  MixParams P;
+  P.M = (int)M;
+  P.N = (int)N;
+  P.kb0 = (int)((K + BK - 1) / BK);  // the K tail is zero-filled by TMA in both operands
+  P.kb1 = A1 ? P.kb0 : 0;
+  P.n_tiles_n = (int)((N + BN - 1) / BN);
+  P.n_tiles = (int)((M + 2 * BM - 1) / (2 * BM)) * P.n_tiles_n;
+  P.y = C;
+  P.ldy = ldc;
+  P.idesc0 = P.idesc1 = f16 ? IDESC2_F16 : IDESC2_BF16;
+  P.err = err;
+  static bool attr[64] = {};
+  if (!attr[device & 63]) {
+    L3_CUDA_TRY(cudaFuncSetAttribute(k_mix_gemm_pair<true>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, (int)MIX2_SMEM));
+    attr[device & 63] = true;
+  }
+  const int pairs = std::min(P.n_tiles, num_sms() / 2);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * pairs, 1, 1);
+  cfg.blockDim = dim3(GEMM_THREADS, 1, 1);
+  cfg.dynamicSmemBytes = MIX2_SMEM;
+  cfg.stream = s;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = 2;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  L3_CUDA_TRY(cudaLaunchKernelEx(&cfg, k_mix_gemm_pair<true>, mA, mB, mA1, mB1, P));
   return L3_OK;
 }
 

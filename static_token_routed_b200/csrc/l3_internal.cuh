@@ -118,6 +118,13 @@ struct l3_plan_s {
 
 namespace l3 {
 
+// device block cache (api.cu): cache_take returns a cached block of at
+// least `bytes` on `device` whose last user has finished (its size in *got),
+// or nullptr; cache_give returns a block once the work enqueued on `s` so far
+// is done with it
+void *cache_take(int device, size_t bytes, size_t *got);
+void cache_give(void *ptr, size_t bytes, int device, cudaStream_t s);
+
 // plan kernels (plan.cu)
 // copy each group's rows of the full tables into staged tables (rows of
 // group g at seg_rows[g]); the full tables may be in mapped host memory
@@ -152,6 +159,15 @@ l3_status launch_up_ln_tc(const l3_plan_s *p, const void *gamma, const void *bet
                           cudaStream_t s);
 l3_status launch_mix_tc(const l3_plan_s *p, const void *x, const void *W_mix, void *y,
                         cudaStream_t s);
+// C[M x N] (fp32, row stride ldc) = A[M x K] B[N x K]^T (+ A1 B1^T when A1
+// and B1 are given, same shapes and strides) on the pair kernel: operands
+// row-major 16-bit, all fp16 (f16) or all bf16, row strides lda / ldb
+// elements (multiples of 8), all pointers 16-byte aligned, N and ldc
+// multiples of 4, K >= 1; anything else returns L3_ERR_UNSUPPORTED. A wait
+// that gives up sets *err.
+l3_status launch_gemm_nt_tc(const void *A, const void *B, const void *A1, const void *B1, bool f16,
+                            int64_t M, int64_t N, int64_t K, int64_t lda, int64_t ldb, float *C,
+                            int64_t ldc, int *err, int device, cudaStream_t s);
 
 // GEMMs + LayerNorm, CUDA-core path (gemm_simt.cu)
 l3_status launch_up_ln_simt(const l3_plan_s *p, const void *W_up, const void *gamma,
