@@ -175,127 +175,168 @@ l3_status transpose_bf16(const void *in, int64_t ld_in, int64_t R, int64_t C, vo
 }
 
 // ---------------------------------------------------------------- LayerNorm
-constexpr int LN_ROWS = 16;  // token rows per CTA (one warp per row at a time)
+// Sum of K values over the CTA's 256 threads, the same in every thread and
+// in a fixed order (deterministic); red holds 8 x 4 floats.
+template <int K>
+__device__ __forceinline__ void block_sum(float (&v)[K], float (*red)[4]) {
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+#pragma unroll
+  for (int k = 0; k < K; ++k)
+    for (int o = 16; o > 0; o >>= 1) v[k] += __shfl_xor_sync(0xffffffffu, v[k], o);
+  if (lane == 0)
+#pragma unroll
+    for (int k = 0; k < K; ++k) red[warp][k] = v[k];
+  __syncthreads();
+#pragma unroll
+  for (int k = 0; k < K; ++k) {
+    float t = 0.f;
+    for (int w = 0; w < 8; ++w) t += red[w][k];
+    v[k] = t;
+  }
+  __syncthreads();
+}
 
-// g_z from g_h and z for LN_ROWS rows per CTA (into g_z16 + g_z16_lo, its
-// bf16 rounding and the bf16 rounding of the rest, when they are given, else
-// into g_z as fp32); column partials of
-// dgamma = sum g_h hhat and dbeta = sum g_h into part[cta][2][d_up]
+// g_z from g_h and z, rows [blockIdx.x * rows, +rows) of M, one row at a
+// time over the whole CTA: thread i holds columns i, i + 256, ... (NC of
+// them, d_up <= 256 NC) in registers, the row's mean, variance and the two
+// means of the LayerNorm gradient are CTA sums. g_z goes to g_z16 + g_z16_lo
+// (its bf16 rounding and the bf16 rounding of the rest) when they are given,
+// else to g_z as fp32. The CTA's column sums of g_h hhat (dgamma) and g_h
+// (dbeta) go to part[cta][2][d_up].
+template <int NC>
 __global__ void __launch_bounds__(256)
     k_ln_backward(const float *__restrict__ z, const float *__restrict__ g_h, const void *gamma,
-                  int gtype, int d_up, float eps, int64_t M, float *__restrict__ g_z,
-                  __nv_bfloat16 *__restrict__ g_z16, __nv_bfloat16 *__restrict__ g_z16_lo,
-                  float *__restrict__ part) {
-  extern __shared__ float sm[];  // [8 warps][2][d_up]
-  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  float *pg = sm + warp * 2 * d_up, *pb = pg + d_up;
-  for (int u = lane; u < d_up; u += 32) pg[u] = pb[u] = 0.f;
-  for (int rr = warp; rr < LN_ROWS; rr += 8) {
-    const int64_t row = blockIdx.x * (int64_t)LN_ROWS + rr;
-    if (row >= M) break;
+                  int gtype, int d_up, float eps, int64_t M, int64_t rows,
+                  float *__restrict__ g_z, __nv_bfloat16 *__restrict__ g_z16,
+                  __nv_bfloat16 *__restrict__ g_z16_lo, float *__restrict__ part) {
+  __shared__ float red[8][4];
+  const int tid = threadIdx.x;
+  float gam[NC], pg[NC], pb[NC];
+#pragma unroll
+  for (int i = 0; i < NC; ++i) {
+    const int u = tid + i * 256;
+    gam[i] = u < d_up ? ldx(gamma, gtype, u) : 0.f;
+    pg[i] = pb[i] = 0.f;
+  }
+  const int64_t r_end = min(M, (int64_t)(blockIdx.x + 1) * rows);
+  for (int64_t row = (int64_t)blockIdx.x * rows; row < r_end; ++row) {
     const float *zr = z + row * d_up, *gr = g_h + row * d_up;
-    float s = 0.f;
-    for (int u = lane; u < d_up; u += 32) s += zr[u];
-    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-    const float mu = s / d_up;
-    float q = 0.f;
-    for (int u = lane; u < d_up; u += 32) q = fmaf(zr[u] - mu, zr[u] - mu, q);
-    for (int o = 16; o > 0; o >>= 1) q += __shfl_xor_sync(0xffffffffu, q, o);
-    const float rstd = 1.0f / sqrtf(q / d_up + eps);
-    float m1 = 0.f, m2 = 0.f;  // sums of g_hhat and g_hhat * hhat
-    for (int u = lane; u < d_up; u += 32) {
-      const float hh = (zr[u] - mu) * rstd, gh = gr[u] * ldx(gamma, gtype, u);
-      m1 += gh;
-      m2 = fmaf(gh, hh, m2);
-      pg[u] = fmaf(gr[u], hh, pg[u]);
-      pb[u] += gr[u];
+    float zv[NC], gv[NC];
+    float sum[1] = {0.f};
+#pragma unroll
+    for (int i = 0; i < NC; ++i) {
+      const int u = tid + i * 256;
+      zv[i] = u < d_up ? zr[u] : 0.f;
+      gv[i] = u < d_up ? gr[u] : 0.f;
+      sum[0] += zv[i];
     }
-    for (int o = 16; o > 0; o >>= 1) {
-      m1 += __shfl_xor_sync(0xffffffffu, m1, o);
-      m2 += __shfl_xor_sync(0xffffffffu, m2, o);
+    block_sum<1>(sum, red);
+    const float mu = sum[0] / d_up;
+    float q[1] = {0.f};
+#pragma unroll
+    for (int i = 0; i < NC; ++i)
+      if (tid + i * 256 < d_up) q[0] = fmaf(zv[i] - mu, zv[i] - mu, q[0]);
+    block_sum<1>(q, red);
+    const float rstd = 1.0f / sqrtf(q[0] / d_up + eps);
+    float m[2] = {0.f, 0.f};  // sums of g_hhat and g_hhat * hhat
+#pragma unroll
+    for (int i = 0; i < NC; ++i) {
+      const float hh = (zv[i] - mu) * rstd, gh = gv[i] * gam[i];
+      zv[i] = hh;  // zv holds hhat from here on
+      m[0] += gh;
+      m[1] = fmaf(gh, hh, m[1]);
+      pg[i] = fmaf(gv[i], hh, pg[i]);
+      pb[i] += gv[i];
     }
-    m1 /= d_up;
-    m2 /= d_up;
-    for (int u = lane; u < d_up; u += 32) {
-      const float hh = (zr[u] - mu) * rstd, gh = gr[u] * ldx(gamma, gtype, u);
-      const float gz = (gh - m1 - hh * m2) * rstd;
+    block_sum<2>(m, red);
+    const float m1 = m[0] / d_up, m2 = m[1] / d_up;
+#pragma unroll
+    for (int i = 0; i < NC; ++i) {
+      const int u = tid + i * 256;
+      if (u >= d_up) continue;
+      const float gz = (gv[i] * gam[i] - m1 - zv[i] * m2) * rstd;
       if (g_z16) {
         const __nv_bfloat16 hi = __float2bfloat16_rn(gz);
         g_z16[row * d_up + u] = hi;
         g_z16_lo[row * d_up + u] = __float2bfloat16_rn(gz - __bfloat162float(hi));
-      } else
+      } else {
         g_z[row * d_up + u] = gz;
+      }
     }
   }
-  __syncthreads();
-  for (int u = threadIdx.x; u < d_up; u += blockDim.x) {
-    float g = 0.f, bsum = 0.f;
-    for (int w = 0; w < 8; ++w) {
-      g += sm[w * 2 * d_up + u];
-      bsum += sm[w * 2 * d_up + d_up + u];
+#pragma unroll
+  for (int i = 0; i < NC; ++i) {
+    const int u = tid + i * 256;
+    if (u < d_up) {
+      part[(int64_t)blockIdx.x * 2 * d_up + u] = pg[i];
+      part[(int64_t)blockIdx.x * 2 * d_up + d_up + u] = pb[i];
     }
-    part[(int64_t)blockIdx.x * 2 * d_up + u] = g;
-    part[(int64_t)blockIdx.x * 2 * d_up + d_up + u] = bsum;
   }
 }
 
-// column sums of the per-CTA partials, in CTA order
-__global__ void k_sum_partials(const float *__restrict__ part, int n_parts, int d_up,
-                               float *__restrict__ dgamma, float *__restrict__ dbeta) {
-  const int u = blockIdx.x * blockDim.x + threadIdx.x;
-  if (u >= d_up) return;
+// column sums of the per-CTA partials in a fixed order: a CTA per 32
+// columns, warp w adds partials w, w + 8, ..., then warp order
+__global__ void __launch_bounds__(256)
+    k_sum_partials(const float *__restrict__ part, int n_parts, int d_up,
+                   float *__restrict__ dgamma, float *__restrict__ dbeta) {
+  __shared__ float red[2][8][32];
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int u = blockIdx.x * 32 + lane;
   float g = 0.f, b = 0.f;
-  for (int i = 0; i < n_parts; ++i) {
-    g += part[(int64_t)i * 2 * d_up + u];
-    b += part[(int64_t)i * 2 * d_up + d_up + u];
+  if (u < d_up)
+    for (int i = warp; i < n_parts; i += 8) {
+      g += part[(int64_t)i * 2 * d_up + u];
+      b += part[(int64_t)i * 2 * d_up + d_up + u];
+    }
+  red[0][warp][lane] = g;
+  red[1][warp][lane] = b;
+  __syncthreads();
+  if (warp == 0 && u < d_up) {
+    g = b = 0.f;
+    for (int w = 0; w < 8; ++w) {
+      g += red[0][w][lane];
+      b += red[1][w][lane];
+    }
+    dgamma[u] = g;
+    dbeta[u] = b;
   }
-  dgamma[u] = g;
-  dbeta[u] = b;
+}
+
+template <int NC>
+void launch_ln_backward(unsigned grid, int64_t rows, cudaStream_t s, const float *z,
+                        const float *g_h, const void *gamma, int gtype, int d_up, float eps,
+                        int64_t M, float *g_z, __nv_bfloat16 *g_z16, __nv_bfloat16 *g_z16_lo,
+                        float *part) {
+  k_ln_backward<NC><<<grid, 256, 0, s>>>(z, g_h, gamma, gtype, d_up, eps, M, rows, g_z, g_z16,
+                                         g_z16_lo, part);
 }
 
 // ---------------------------------------------------------------- attention
 constexpr int AT = 8;        // tokens per chunk
 constexpr int A_MAX_K = 1024;
 
-// One CTA per group; its tokens in chunks of AT.
+// Tail items (up to TAIL_TOKENS tokens of one group): one CTA per item,
+// every row it reads shared by the item's tokens; dK / dV rows take atomic
+// adds (several items of a group share its rows).
+static_assert(AT == TAIL_TOKENS, "one chunk per tail item");
 __global__ void __launch_bounds__(256)
-    k_attn_backward(const void *x, const void *W_K, const void *W_V, int wtype,
-                    const float *__restrict__ g_a, const int32_t *__restrict__ perm,
-                    const int32_t *__restrict__ group_tok_start,
-                    const int32_t *__restrict__ group_row_start,
-                    const int32_t *__restrict__ group_rows, const DenseTile *__restrict__ tiles,
-                    int64_t n_tiles, const TailItem *__restrict__ items, int d_in, int d_emb,
-                    float *__restrict__ dx, float *__restrict__ dW_K, float *__restrict__ dW_V) {
+    k_attn_backward_tail(const void *x, const void *W_K, const void *W_V, int wtype,
+                         const float *__restrict__ g_a, const TailItem *__restrict__ items,
+                         int d_in, int d_emb, float *__restrict__ dx, float *__restrict__ dW_K,
+                         float *__restrict__ dW_V) {
   extern __shared__ float sm[];
   float *xs = sm;                  // [AT][d_in]
   float *gas = xs + AT * d_in;     // [AT][d_emb]
   float *ps = gas + AT * d_emb;    // [AT][A_MAX_K] logits, then p
   float *gs = ps + AT * A_MAX_K;   // [AT][A_MAX_K] g_p, then g_s
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  __shared__ int32_t tok[AT];  // original indices of the chunk's tokens
-  // work unit: a dense tile (up to 128 tokens of one group) or a tail item
-  // (up to 8), the same units as the forward's attention
-  int64_t r0;
-  int d, c, t0 = 0;
-  const TailItem *item = nullptr;
-  if (blockIdx.x < n_tiles) {
-    const DenseTile tl = tiles[blockIdx.x];
-    r0 = group_row_start[tl.group];
-    d = group_rows[tl.group];
-    t0 = tl.tok0;
-    c = min(128, group_tok_start[tl.group + 1] - tl.tok0);
-  } else {
-    item = items + (blockIdx.x - n_tiles);
-    r0 = item->r0;
-    d = item->d;
-    c = item->nt;
-  }
+  __shared__ int32_t tok[AT];  // original indices of the item's tokens
+  const TailItem *item = items + blockIdx.x;
+  const int64_t r0 = item->r0;
+  const int d = item->d, c = item->nt;
   for (int c0 = 0; c0 < c; c0 += AT) {
     const int nt = min(AT, c - c0);
-    if (threadIdx.x < AT)
-      tok[threadIdx.x] = threadIdx.x < nt
-                             ? (item ? item->tok[c0 + threadIdx.x] : perm[t0 + c0 + threadIdx.x])
-                             : 0;
+    if (threadIdx.x < AT) tok[threadIdx.x] = threadIdx.x < nt ? item->tok[c0 + threadIdx.x] : 0;
     __syncthreads();
     for (int i = threadIdx.x; i < AT * d_in; i += blockDim.x) {
       const int t = i / d_in, col = i % d_in;
@@ -373,7 +414,7 @@ __global__ void __launch_bounds__(256)
             acc[t] = fmaf(gst, kv, acc[t]);
             gk = fmaf(gst, xs[t * d_in + col], gk);
           }
-          atomicAdd(dW_K + kidx, gk);  // several units may share a group's rows
+          atomicAdd(dW_K + kidx, gk);
         }
         for (int t = 0; t < nt; ++t) dx[(int64_t)tok[t] * d_in + col] += acc[t];
       }
@@ -388,6 +429,234 @@ __global__ void __launch_bounds__(256)
       }
     }
     __syncthreads();
+  }
+}
+
+// ---------------------------------------------------------------- dense tiles
+// A dense tile (up to 128 tokens of one group, 32..512 rows) runs the
+// attention backward as four register-tiled kernels over its slot in
+// scratch, two [slot_rows][DENSE_TILE_M] fp32 planes (row j, token t):
+//   k_bwd_dense_scores   plane 0 = S = K_t X^T, plane 1 = G_p = V_t G_a^T
+//   k_bwd_dense_softmax  plane 0 = P = softmax_j(S), plane 1 = G_s = P (G_p - sum_j P G_p)
+//   k_bwd_dense_dx       dx_t += K_t^T g_s_t
+//   k_attn_backward_dw   dK_t += G_s X, dV_t += P G_a
+// Each thread holds a 4 x 8 (or 8 x 4) block of outputs; operands pass
+// through shared memory 32 k-steps at a time.
+constexpr int DB_K = 32;  // k-steps per shared-memory stage
+constexpr int DB_J = 64;  // rows of a scores block
+
+__device__ __forceinline__ float *slot_plane(float *slots, int64_t b, int slot_rows, int plane) {
+  return slots + (b * 2 + plane) * (int64_t)slot_rows * DENSE_TILE_M;
+}
+
+// CTA per (tile, 64-row block): S and G_p for 64 rows x 128 tokens.
+__global__ void __launch_bounds__(256)
+    k_bwd_dense_scores(const void *x, const void *W_K, const void *W_V, int wtype,
+                       const float *__restrict__ g_a, const int32_t *__restrict__ perm,
+                       const int32_t *__restrict__ group_tok_start,
+                       const int32_t *__restrict__ group_row_start,
+                       const int32_t *__restrict__ group_rows, const DenseTile *__restrict__ tiles,
+                       float *__restrict__ slots, int slot_rows, int d_in, int d_emb) {
+  __shared__ float as[DB_K][DB_J + 1];          // rows of K_t or V_t, k-major
+  __shared__ float bs[DB_K][DENSE_TILE_M + 1];  // x or g_a of the tokens, k-major
+  __shared__ int64_t tok[DENSE_TILE_M];
+  const int n_jb = slot_rows / DB_J;
+  const int64_t b = blockIdx.x / n_jb;
+  const int jb = (blockIdx.x % n_jb) * DB_J;
+  const DenseTile tl = tiles[b];
+  const int d = group_rows[tl.group];
+  if (jb >= d) return;  // the whole CTA leaves
+  const int64_t r0 = group_row_start[tl.group];
+  const int c = min(DENSE_TILE_M, group_tok_start[tl.group + 1] - tl.tok0);
+  const int tid = threadIdx.x, tx = tid % 16, ty = tid / 16;
+  if (tid < DENSE_TILE_M) tok[tid] = tid < c ? perm[tl.tok0 + tid] : -1;
+  for (int plane = 0; plane < 2; ++plane) {
+    const int K = plane == 0 ? d_in : d_emb;
+    float acc[4][8] = {};
+    for (int k0 = 0; k0 < K; k0 += DB_K) {
+      __syncthreads();  // tok written / the previous stage read
+      for (int i = tid; i < DB_J * DB_K; i += 256) {
+        const int jj = i / DB_K, kk = i % DB_K;
+        const int64_t idx = (r0 + jb + jj) * K + k0 + kk;
+        as[kk][jj] = jb + jj < d ? ldx(plane == 0 ? W_K : W_V, wtype, idx) : 0.f;
+      }
+      for (int i = tid; i < DENSE_TILE_M * DB_K; i += 256) {
+        const int t = i / DB_K, kk = i % DB_K;
+        const int64_t tk = tok[t];
+        bs[kk][t] = tk < 0 ? 0.f
+                    : plane == 0 ? ldx(x, wtype, tk * d_in + k0 + kk)
+                                 : g_a[tk * d_emb + k0 + kk];
+      }
+      __syncthreads();
+#pragma unroll 4
+      for (int kk = 0; kk < DB_K; ++kk) {
+        float a[4], bv[8];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) a[i] = as[kk][ty + 16 * i];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) bv[e] = bs[kk][tx + 16 * e];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+          for (int e = 0; e < 8; ++e) acc[i][e] = fmaf(a[i], bv[e], acc[i][e]);
+      }
+    }
+    float *out = slot_plane(slots, b, slot_rows, plane);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int j = jb + ty + 16 * i;
+      if (j < d)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) out[(int64_t)j * DENSE_TILE_M + tx + 16 * e] = acc[i][e];
+    }
+  }
+}
+
+// CTA per tile, thread per token: P = softmax over the d rows of S, and
+// G_s = P (G_p - sum_j P G_p), in place.
+__global__ void __launch_bounds__(DENSE_TILE_M)
+    k_bwd_dense_softmax(const int32_t *__restrict__ group_rows, const DenseTile *__restrict__ tiles,
+                        float *__restrict__ slots, int slot_rows) {
+  const int64_t b = blockIdx.x;
+  const int d = group_rows[tiles[b].group];
+  const int t = threadIdx.x;
+  float *S = slot_plane(slots, b, slot_rows, 0) + t, *G = slot_plane(slots, b, slot_rows, 1) + t;
+  float mx = -INFINITY;
+  for (int j = 0; j < d; ++j) mx = fmaxf(mx, S[j * DENSE_TILE_M]);
+  float sum = 0.f;
+  for (int j = 0; j < d; ++j) sum += expf(S[j * DENSE_TILE_M] - mx);
+  const float inv = 1.f / sum;
+  float dot = 0.f;
+  for (int j = 0; j < d; ++j) {
+    const float pj = expf(S[j * DENSE_TILE_M] - mx) * inv;
+    S[j * DENSE_TILE_M] = pj;
+    dot = fmaf(pj, G[j * DENSE_TILE_M], dot);
+  }
+  for (int j = 0; j < d; ++j) G[j * DENSE_TILE_M] = S[j * DENSE_TILE_M] * (G[j * DENSE_TILE_M] - dot);
+}
+
+// CTA per (tile, 64-column block of d_in): dx[t][col] += sum_j G_s[j][t] K_t[j][col]
+// for the tile's 128 tokens (each token's dx belongs to this CTA alone).
+__global__ void __launch_bounds__(256)
+    k_bwd_dense_dx(const void *W_K, int wtype, const int32_t *__restrict__ perm,
+                   const int32_t *__restrict__ group_tok_start,
+                   const int32_t *__restrict__ group_row_start,
+                   const int32_t *__restrict__ group_rows, const DenseTile *__restrict__ tiles,
+                   const float *__restrict__ slots, int slot_rows, int d_in,
+                   float *__restrict__ dx) {
+  __shared__ float as[DB_K][DENSE_TILE_M + 1];  // g_s, j-major
+  __shared__ float bs[DB_K][64 + 1];            // K_t rows, j-major
+  const int n_cb = d_in / 64;
+  const int64_t b = blockIdx.x / n_cb;
+  const int col0 = (blockIdx.x % n_cb) * 64;
+  const DenseTile tl = tiles[b];
+  const int d = group_rows[tl.group];
+  const int64_t r0 = group_row_start[tl.group];
+  const int c = min(DENSE_TILE_M, group_tok_start[tl.group + 1] - tl.tok0);
+  const float *G = slot_plane(const_cast<float *>(slots), b, slot_rows, 1);
+  const int tid = threadIdx.x, tx = tid % 16, ty = tid / 16;
+  float acc[8][4] = {};
+  for (int j0 = 0; j0 < d; j0 += DB_K) {
+    __syncthreads();
+    for (int i = tid; i < DB_K * DENSE_TILE_M; i += 256) {
+      const int jj = i / DENSE_TILE_M, t = i % DENSE_TILE_M;
+      as[jj][t] = j0 + jj < d ? G[(int64_t)(j0 + jj) * DENSE_TILE_M + t] : 0.f;
+    }
+    for (int i = tid; i < DB_K * 64; i += 256) {
+      const int jj = i / 64, cc = i % 64;
+      bs[jj][cc] = j0 + jj < d ? ldx(W_K, wtype, (r0 + j0 + jj) * d_in + col0 + cc) : 0.f;
+    }
+    __syncthreads();
+#pragma unroll 4
+    for (int jj = 0; jj < DB_K; ++jj) {
+      float a[8], bv[4];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) a[i] = as[jj][ty + 16 * i];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) bv[e] = bs[jj][tx + 16 * e];
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[i][e] = fmaf(a[i], bv[e], acc[i][e]);
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int t = ty + 16 * i;
+    if (t >= c) continue;
+    float *o = dx + (int64_t)perm[tl.tok0 + t] * d_in + col0;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) o[tx + 16 * e] += acc[i][e];
+  }
+}
+
+// dK_t (+)= G_s^T X and dV_t (+)= P^T G_a over one dense tile's tokens, from
+// the planes k_bwd_dense_softmax left: CTA per (tile, 64-column
+// block of d_in for dK or of d_emb for dV), 64 rows x 64 columns at a time,
+// 4 x 4 outputs per thread, the sum over the tile's (up to 128) tokens in
+// registers, then one atomic add per element (the tiles of one group share
+// its rows).
+constexpr int DW_J = 64, DW_C = 64, DW_LD = DENSE_TILE_M + 4;
+
+__global__ void __launch_bounds__(256)
+    k_attn_backward_dw(const void *x, int wtype, const float *__restrict__ g_a,
+                       const int32_t *__restrict__ perm, const int32_t *__restrict__ group_tok_start,
+                       const int32_t *__restrict__ group_row_start,
+                       const int32_t *__restrict__ group_rows, const DenseTile *__restrict__ tiles,
+                       const float *__restrict__ slots, int slot_rows, int d_in, int d_emb,
+                       float *__restrict__ dW_K, float *__restrict__ dW_V) {
+  extern __shared__ float sm[];
+  float *xs = sm;                        // [DENSE_TILE_M][DW_C]: x or g_a of the tile's tokens
+  float *ms = xs + DENSE_TILE_M * DW_C;  // [DW_J][DW_LD]: g_s or p of 64 rows
+  const int n_cbk = d_in / DW_C, n_cb = n_cbk + d_emb / DW_C;
+  const int64_t b = blockIdx.x / n_cb;
+  const int cb = blockIdx.x % n_cb;
+  const bool is_k = cb < n_cbk;
+  const int width = is_k ? d_in : d_emb, col0 = (is_k ? cb : cb - n_cbk) * DW_C;
+  const DenseTile tl = tiles[b];
+  const int64_t r0 = group_row_start[tl.group];
+  const int d = group_rows[tl.group];
+  const int c = min(DENSE_TILE_M, group_tok_start[tl.group + 1] - tl.tok0);
+  const float *src = slots + (b * 2 + (is_k ? 1 : 0)) * (int64_t)slot_rows * DENSE_TILE_M;
+  float *out = is_k ? dW_K : dW_V;
+  const int tid = threadIdx.x, tx = tid % 16, ty = tid / 16;
+  for (int i = tid; i < DENSE_TILE_M * DW_C; i += blockDim.x) {
+    const int t = i / DW_C, cc = i % DW_C;
+    float v = 0.f;
+    if (t < c) {
+      const int64_t tok = perm[tl.tok0 + t];
+      v = is_k ? ldx(x, wtype, tok * d_in + col0 + cc) : g_a[tok * d_emb + col0 + cc];
+    }
+    xs[i] = v;
+  }
+  for (int jb = 0; jb < d; jb += DW_J) {
+    __syncthreads();  // xs written / the previous block's ms read
+    for (int i = tid; i < DW_J * DENSE_TILE_M; i += blockDim.x) {
+      const int jj = i / DENSE_TILE_M, t = i % DENSE_TILE_M;
+      ms[jj * DW_LD + t] =
+          (t < c && jb + jj < d) ? src[(int64_t)(jb + jj) * DENSE_TILE_M + t] : 0.f;
+    }
+    __syncthreads();
+    float acc[4][4] = {};
+    for (int t = 0; t < c; ++t) {
+      const float4 xv = *reinterpret_cast<const float4 *>(xs + t * DW_C + tx * 4);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float m = ms[(ty * 4 + i) * DW_LD + t];
+        acc[i][0] = fmaf(m, xv.x, acc[i][0]);
+        acc[i][1] = fmaf(m, xv.y, acc[i][1]);
+        acc[i][2] = fmaf(m, xv.z, acc[i][2]);
+        acc[i][3] = fmaf(m, xv.w, acc[i][3]);
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int j = jb + ty * 4 + i;
+      if (j >= d) continue;
+      float *o = out + (r0 + j) * width + col0 + tx * 4;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) atomicAdd(o + e, acc[i][e]);
+    }
   }
 }
 
@@ -421,7 +690,7 @@ extern "C" l3_status l3_backward(const void *x, l3_plan_t p, const void *W_K, co
     return L3_ERR_INVALID_ARG;
   }
   const size_t attn_smem = (AT * d.d_in + AT * d.d_emb + 2 * AT * A_MAX_K) * sizeof(float);
-  if (d.k > A_MAX_K || attn_smem > 220 * 1024 || 16 * d.d_up * sizeof(float) > 220 * 1024) {
+  if (d.k > A_MAX_K || attn_smem > 220 * 1024 || d.d_up > 16 * 256) {
     set_error("l3_backward: k, d_in, d_emb or d_up beyond this kernel's shared-memory layout");
     return L3_ERR_UNSUPPORTED;
   }
@@ -435,7 +704,11 @@ extern "C" l3_status l3_backward(const void *x, l3_plan_t p, const void *W_K, co
   }
   const int wt = d.dtype == L3_BF16 ? T_BF16 : T_F32;
   const int it = d.dtype == L3_BF16 ? T_F16 : T_F32;  // a and h as the forward stored them
-  const int64_t n_ln = (N + LN_ROWS - 1) / LN_ROWS;
+  int n_sms = 148;
+  cudaDeviceGetAttribute(&n_sms, cudaDevAttrMultiProcessorCount, p->device);
+  // LayerNorm backward: about four CTAs per SM, each over a run of rows
+  const int64_t ln_rows = (N + 4 * n_sms - 1) / (4 * n_sms);
+  const int64_t n_ln = (N + ln_rows - 1) / ln_rows;
   const int64_t D = d.d_up + d.d_in;  // columns of W_mix
   auto a16 = [](const void *q) { return (reinterpret_cast<uintptr_t>(q) & 15u) == 0; };
   // tensor cores for bf16 layers whose forward ran on them (it left the fp16
@@ -465,6 +738,10 @@ extern "C" l3_status l3_backward(const void *x, l3_plan_t p, const void *W_K, co
     o_at = take(d.d_emb * ldn * 2);     // a^T       [d_emb x N]
     o_wut = take(d.d_emb * d.d_up * 2); // W_up^T    [d_emb x d_up]
   }
+  // p and g_s of every dense tile for k_attn_backward_dw
+  const int64_t n_dt = p->n_dense_tiles;
+  const int slot_rows = n_dt > 0 ? dense_attention_max_rows() : 0;
+  const size_t o_slots = take(n_dt * 2 * slot_rows * DENSE_TILE_M * f);
   // from the device block cache, so a backward per batch maps no memory
   // after warm-up
   size_t got = 0;
@@ -479,6 +756,7 @@ extern "C" l3_status l3_backward(const void *x, l3_plan_t p, const void *W_K, co
   float *z = reinterpret_cast<float *>(scratch + o_z);
   float *g_a = reinterpret_cast<float *>(scratch + o_ga);
   float *part = reinterpret_cast<float *>(scratch + o_part);
+  float *slots = reinterpret_cast<float *>(scratch + o_slots);
   float *g_z = tc ? nullptr : reinterpret_cast<float *>(scratch + o_gz);
   __nv_bfloat16 *g_z16 = tc ? reinterpret_cast<__nv_bfloat16 *>(scratch + o_gz) : nullptr;
   __nv_bfloat16 *g_z16_lo = tc ? reinterpret_cast<__nv_bfloat16 *>(scratch + o_gzlo) : nullptr;
@@ -487,8 +765,6 @@ extern "C" l3_status l3_backward(const void *x, l3_plan_t p, const void *W_K, co
                 *at = bf(o_at), *wut = bf(o_wut);
   int *err = p->dev_flags + 1;  // a tensor-core wait that gives up reports here
   const int dev = p->device;
-  int n_sms = 148;
-  cudaDeviceGetAttribute(&n_sms, cudaDevAttrMultiProcessorCount, dev);
   using BF = __nv_bfloat16;
   const int64_t ldm = D;
   const char *wmx = reinterpret_cast<const char *>(W_mix) + d.d_up * (wt == T_F32 ? 4 : 2);
@@ -541,17 +817,14 @@ extern "C" l3_status l3_backward(const void *x, l3_plan_t p, const void *W_K, co
               : gemm({p->a_buf, d.d_emb, 1, it}, {W_up, d.d_emb, 1, wt}, (int)N, (int)d.d_up,
                      (int)d.d_emb, z, d.d_up, false, s);
     if (st == L3_OK) {
-      const size_t smem = 8 * 2 * d.d_up * f;
-      if (smem > 48 * 1024)
-        e = cudaFuncSetAttribute(k_ln_backward, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)smem);
-      if (e == cudaSuccess) {
-        k_ln_backward<<<(unsigned)n_ln, 256, smem, s>>>(z, g_h, ln_gamma, wt, (int)d.d_up,
-                                                        d.ln_eps, N, g_z, g_z16, g_z16_lo, part);
-        k_sum_partials<<<(unsigned)((d.d_up + 255) / 256), 256, 0, s>>>(
-            part, (int)n_ln, (int)d.d_up, dgamma, dbeta);
-        e = cudaGetLastError();
-      }
+      auto ln = d.d_up <= 4 * 256   ? launch_ln_backward<4>
+                : d.d_up <= 8 * 256 ? launch_ln_backward<8>
+                                    : launch_ln_backward<16>;
+      ln((unsigned)n_ln, ln_rows, s, z, g_h, ln_gamma, wt, (int)d.d_up, d.ln_eps, N, g_z, g_z16,
+         g_z16_lo, part);
+      k_sum_partials<<<(unsigned)((d.d_up + 31) / 32), 256, 0, s>>>(part, (int)n_ln, (int)d.d_up,
+                                                                     dgamma, dbeta);
+      e = cudaGetLastError();
       if (e != cudaSuccess) st = cuda_fail(e, "LayerNorm backward");
     }
   }
@@ -577,19 +850,41 @@ extern "C" l3_status l3_backward(const void *x, l3_plan_t p, const void *W_K, co
                   (int)d.d_up, g_a, d.d_emb, false, s);
     }
   }
-  const int64_t n_units = p->n_dense_tiles + p->n_tail_items;
-  if (st == L3_OK && n_units > 0) {
-    LaunchTimer t("bwd_attention", s);
-    e = cudaFuncSetAttribute(k_attn_backward, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  const int64_t n_tail = p->n_tail_items;
+  if (st == L3_OK && n_tail > 0) {
+    LaunchTimer t("bwd_attention_tail", s);
+    e = cudaFuncSetAttribute(k_attn_backward_tail, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)attn_smem);
     if (e == cudaSuccess) {
-      k_attn_backward<<<(unsigned)n_units, 256, attn_smem, s>>>(
-          x, W_K, W_V, wt, g_a, p->perm, p->group_tok_start, p->group_row_start, p->group_rows,
-          p->dense_tiles, p->n_dense_tiles, p->tail_items, (int)d.d_in, (int)d.d_emb, dx, dW_K,
-          dW_V);
+      k_attn_backward_tail<<<(unsigned)n_tail, 256, attn_smem, s>>>(
+          x, W_K, W_V, wt, g_a, p->tail_items, (int)d.d_in, (int)d.d_emb, dx, dW_K, dW_V);
       e = cudaGetLastError();
     }
-    if (e != cudaSuccess) st = cuda_fail(e, "attention backward");
+    if (e != cudaSuccess) st = cuda_fail(e, "attention backward (tail items)");
+  }
+  if (st == L3_OK && n_dt > 0) {
+    LaunchTimer t("bwd_attention_dense", s);
+    k_bwd_dense_scores<<<(unsigned)(n_dt * (slot_rows / DB_J)), 256, 0, s>>>(
+        x, W_K, W_V, wt, g_a, p->perm, p->group_tok_start, p->group_row_start, p->group_rows,
+        p->dense_tiles, slots, slot_rows, (int)d.d_in, (int)d.d_emb);
+    k_bwd_dense_softmax<<<(unsigned)n_dt, DENSE_TILE_M, 0, s>>>(p->group_rows, p->dense_tiles,
+                                                                 slots, slot_rows);
+    k_bwd_dense_dx<<<(unsigned)(n_dt * (d.d_in / 64)), 256, 0, s>>>(
+        W_K, wt, p->perm, p->group_tok_start, p->group_row_start, p->group_rows, p->dense_tiles,
+        slots, slot_rows, (int)d.d_in, dx);
+    e = cudaGetLastError();
+    const size_t dw_smem = (DENSE_TILE_M * DW_C + DW_J * DW_LD) * f;
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(k_attn_backward_dw, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)dw_smem);
+    if (e == cudaSuccess) {
+      const int64_t n_cb = d.d_in / DW_C + d.d_emb / DW_C;
+      k_attn_backward_dw<<<(unsigned)(n_dt * n_cb), 256, dw_smem, s>>>(
+          x, wt, g_a, p->perm, p->group_tok_start, p->group_row_start, p->group_rows,
+          p->dense_tiles, slots, slot_rows, (int)d.d_in, (int)d.d_emb, dW_K, dW_V);
+      e = cudaGetLastError();
+    }
+    if (e != cudaSuccess) st = cuda_fail(e, "attention backward (dense tiles)");
   }
   cache_give(scratch, got, p->device, s);
   return st;
