@@ -317,54 +317,56 @@ constexpr int A_MAX_K = 1024;
 
 // Tail items (up to TAIL_TOKENS tokens of one group): one CTA per item,
 // every row it reads shared by the item's tokens; dK / dV rows take atomic
-// adds (several items of a group share its rows).
+// adds (several items of a group share its rows). NT = the item class's
+// token bound (1, 2, 4 or 8): the plan lists items by class.
 static_assert(AT == TAIL_TOKENS, "one chunk per tail item");
+template <int NT>
 __global__ void __launch_bounds__(256)
     k_attn_backward_tail(const void *x, const void *W_K, const void *W_V, int wtype,
                          const float *__restrict__ g_a, const TailItem *__restrict__ items,
                          int d_in, int d_emb, float *__restrict__ dx, float *__restrict__ dW_K,
                          float *__restrict__ dW_V) {
   extern __shared__ float sm[];
-  float *xs = sm;                  // [AT][d_in]
-  float *gas = xs + AT * d_in;     // [AT][d_emb]
-  float *ps = gas + AT * d_emb;    // [AT][A_MAX_K] logits, then p
-  float *gs = ps + AT * A_MAX_K;   // [AT][A_MAX_K] g_p, then g_s
+  float *xs = sm;                  // [NT][d_in]
+  float *gas = xs + NT * d_in;     // [NT][d_emb]
+  float *ps = gas + NT * d_emb;    // [NT][A_MAX_K] logits, then p
+  float *gs = ps + NT * A_MAX_K;   // [NT][A_MAX_K] g_p, then g_s
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   __shared__ int32_t tok[AT];  // original indices of the item's tokens
   const TailItem *item = items + blockIdx.x;
   const int64_t r0 = item->r0;
   const int d = item->d, c = item->nt;
-  for (int c0 = 0; c0 < c; c0 += AT) {
-    const int nt = min(AT, c - c0);
-    if (threadIdx.x < AT) tok[threadIdx.x] = threadIdx.x < nt ? item->tok[c0 + threadIdx.x] : 0;
+  for (int c0 = 0; c0 < c; c0 += NT) {
+    const int nt = min(NT, c - c0);
+    if (threadIdx.x < NT) tok[threadIdx.x] = threadIdx.x < nt ? item->tok[c0 + threadIdx.x] : 0;
     __syncthreads();
-    for (int i = threadIdx.x; i < AT * d_in; i += blockDim.x) {
+    for (int i = threadIdx.x; i < NT * d_in; i += blockDim.x) {
       const int t = i / d_in, col = i % d_in;
       xs[i] = t < nt ? ldx(x, wtype, (int64_t)tok[t] * d_in + col) : 0.f;
     }
-    for (int i = threadIdx.x; i < AT * d_emb; i += blockDim.x) {
+    for (int i = threadIdx.x; i < NT * d_emb; i += blockDim.x) {
       const int t = i / d_emb, col = i % d_emb;
       gas[i] = t < nt ? g_a[(int64_t)tok[t] * d_emb + col] : 0.f;
     }
     __syncthreads();
     // logits s = K_j . x_t and g_p = V_j . g_a_t, one warp per row
     for (int j = warp; j < d; j += 8) {
-      float sv[AT], gv[AT];
+      float sv[NT], gv[NT];
 #pragma unroll
-      for (int t = 0; t < AT; ++t) sv[t] = gv[t] = 0.f;
+      for (int t = 0; t < NT; ++t) sv[t] = gv[t] = 0.f;
       if (d > 1)
         for (int col = lane; col < d_in; col += 32) {
           const float kv = ldx(W_K, wtype, (r0 + j) * d_in + col);
 #pragma unroll
-          for (int t = 0; t < AT; ++t) sv[t] = fmaf(kv, xs[t * d_in + col], sv[t]);
+          for (int t = 0; t < NT; ++t) sv[t] = fmaf(kv, xs[t * d_in + col], sv[t]);
         }
       for (int col = lane; col < d_emb; col += 32) {
         const float vv = ldx(W_V, wtype, (r0 + j) * d_emb + col);
 #pragma unroll
-        for (int t = 0; t < AT; ++t) gv[t] = fmaf(vv, gas[t * d_emb + col], gv[t]);
+        for (int t = 0; t < NT; ++t) gv[t] = fmaf(vv, gas[t * d_emb + col], gv[t]);
       }
 #pragma unroll
-      for (int t = 0; t < AT; ++t) {
+      for (int t = 0; t < NT; ++t) {
         for (int o = 16; o > 0; o >>= 1) {
           sv[t] += __shfl_xor_sync(0xffffffffu, sv[t], o);
           gv[t] += __shfl_xor_sync(0xffffffffu, gv[t], o);
@@ -401,15 +403,15 @@ __global__ void __launch_bounds__(256)
     // dx_t += K_t^T g_s_t and dK_j (+)= sum_t g_s[t][j] x_t: thread per column
     if (d > 1) {
       for (int col = threadIdx.x; col < d_in; col += blockDim.x) {
-        float acc[AT];
+        float acc[NT];
 #pragma unroll
-        for (int t = 0; t < AT; ++t) acc[t] = 0.f;
+        for (int t = 0; t < NT; ++t) acc[t] = 0.f;
         for (int j = 0; j < d; ++j) {
           const int64_t kidx = (r0 + j) * d_in + col;
           const float kv = ldx(W_K, wtype, kidx);
           float gk = 0.f;
 #pragma unroll
-          for (int t = 0; t < AT; ++t) {
+          for (int t = 0; t < NT; ++t) {
             const float gst = gs[t * A_MAX_K + j];
             acc[t] = fmaf(gst, kv, acc[t]);
             gk = fmaf(gst, xs[t * d_in + col], gk);
@@ -424,7 +426,7 @@ __global__ void __launch_bounds__(256)
       for (int j = 0; j < d; ++j) {
         float gv = 0.f;
 #pragma unroll
-        for (int t = 0; t < AT; ++t) gv = fmaf(ps[t * A_MAX_K + j], gas[t * d_emb + col], gv);
+        for (int t = 0; t < NT; ++t) gv = fmaf(ps[t * A_MAX_K + j], gas[t * d_emb + col], gv);
         atomicAdd(dW_V + (r0 + j) * d_emb + col, gv);
       }
     }
@@ -449,7 +451,59 @@ __device__ __forceinline__ float *slot_plane(float *slots, int64_t b, int slot_r
   return slots + (b * 2 + plane) * (int64_t)slot_rows * DENSE_TILE_M;
 }
 
-// CTA per (tile, 64-row block): S and G_p for 64 rows x 128 tokens.
+// S and G_p of 64 rows x 16 NE tokens (NE = ceil(c / 16) column groups of
+// the tile; columns c..16 NE - 1 come out zero, later columns are left alone).
+template <int NE>
+__device__ __forceinline__ void dense_scores(const void *x, const void *W_K, const void *W_V,
+                                             int wtype, const float *__restrict__ g_a,
+                                             const int64_t *tok, int64_t r0, int d, int jb,
+                                             int d_in, int d_emb, float *plane0, float *plane1,
+                                             float (*as)[DB_J + 1],
+                                             float (*bs)[DENSE_TILE_M + 1]) {
+  const int tid = threadIdx.x, tx = tid % 16, ty = tid / 16;
+  for (int plane = 0; plane < 2; ++plane) {
+    const int K = plane == 0 ? d_in : d_emb;
+    float acc[4][NE] = {};
+    for (int k0 = 0; k0 < K; k0 += DB_K) {
+      __syncthreads();  // tok written / the previous stage read
+      for (int i = tid; i < DB_J * DB_K; i += 256) {
+        const int jj = i / DB_K, kk = i % DB_K;
+        const int64_t idx = (r0 + jb + jj) * K + k0 + kk;
+        as[kk][jj] = jb + jj < d ? ldx(plane == 0 ? W_K : W_V, wtype, idx) : 0.f;
+      }
+      for (int i = tid; i < 16 * NE * DB_K; i += 256) {
+        const int t = i / DB_K, kk = i % DB_K;
+        const int64_t tk = tok[t];
+        bs[kk][t] = tk < 0 ? 0.f
+                    : plane == 0 ? ldx(x, wtype, tk * d_in + k0 + kk)
+                                 : g_a[tk * d_emb + k0 + kk];
+      }
+      __syncthreads();
+#pragma unroll 4
+      for (int kk = 0; kk < DB_K; ++kk) {
+        float a[4], bv[NE];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) a[i] = as[kk][ty + 16 * i];
+#pragma unroll
+        for (int e = 0; e < NE; ++e) bv[e] = bs[kk][tx + 16 * e];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+          for (int e = 0; e < NE; ++e) acc[i][e] = fmaf(a[i], bv[e], acc[i][e]);
+      }
+    }
+    float *out = plane == 0 ? plane0 : plane1;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int j = jb + ty + 16 * i;
+      if (j < d)
+#pragma unroll
+        for (int e = 0; e < NE; ++e) out[(int64_t)j * DENSE_TILE_M + tx + 16 * e] = acc[i][e];
+    }
+  }
+}
+
+// CTA per (tile, 64-row block): S and G_p for 64 rows x the tile's tokens.
 __global__ void __launch_bounds__(256)
     k_bwd_dense_scores(const void *x, const void *W_K, const void *W_V, int wtype,
                        const float *__restrict__ g_a, const int32_t *__restrict__ perm,
@@ -468,58 +522,35 @@ __global__ void __launch_bounds__(256)
   if (jb >= d) return;  // the whole CTA leaves
   const int64_t r0 = group_row_start[tl.group];
   const int c = min(DENSE_TILE_M, group_tok_start[tl.group + 1] - tl.tok0);
-  const int tid = threadIdx.x, tx = tid % 16, ty = tid / 16;
-  if (tid < DENSE_TILE_M) tok[tid] = tid < c ? perm[tl.tok0 + tid] : -1;
-  for (int plane = 0; plane < 2; ++plane) {
-    const int K = plane == 0 ? d_in : d_emb;
-    float acc[4][8] = {};
-    for (int k0 = 0; k0 < K; k0 += DB_K) {
-      __syncthreads();  // tok written / the previous stage read
-      for (int i = tid; i < DB_J * DB_K; i += 256) {
-        const int jj = i / DB_K, kk = i % DB_K;
-        const int64_t idx = (r0 + jb + jj) * K + k0 + kk;
-        as[kk][jj] = jb + jj < d ? ldx(plane == 0 ? W_K : W_V, wtype, idx) : 0.f;
-      }
-      for (int i = tid; i < DENSE_TILE_M * DB_K; i += 256) {
-        const int t = i / DB_K, kk = i % DB_K;
-        const int64_t tk = tok[t];
-        bs[kk][t] = tk < 0 ? 0.f
-                    : plane == 0 ? ldx(x, wtype, tk * d_in + k0 + kk)
-                                 : g_a[tk * d_emb + k0 + kk];
-      }
-      __syncthreads();
-#pragma unroll 4
-      for (int kk = 0; kk < DB_K; ++kk) {
-        float a[4], bv[8];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) a[i] = as[kk][ty + 16 * i];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) bv[e] = bs[kk][tx + 16 * e];
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-          for (int e = 0; e < 8; ++e) acc[i][e] = fmaf(a[i], bv[e], acc[i][e]);
-      }
-    }
-    float *out = slot_plane(slots, b, slot_rows, plane);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int j = jb + ty + 16 * i;
-      if (j < d)
-#pragma unroll
-        for (int e = 0; e < 8; ++e) out[(int64_t)j * DENSE_TILE_M + tx + 16 * e] = acc[i][e];
-    }
+  if (threadIdx.x < DENSE_TILE_M) tok[threadIdx.x] = threadIdx.x < c ? perm[tl.tok0 + threadIdx.x] : -1;
+  float *p0 = slot_plane(slots, b, slot_rows, 0), *p1 = slot_plane(slots, b, slot_rows, 1);
+#define L3_SCORES(NE)                                                                           \
+  dense_scores<NE>(x, W_K, W_V, wtype, g_a, tok, r0, d, jb, d_in, d_emb, p0, p1, as, bs); \
+  break;
+  switch ((c + 15) / 16) {
+    case 1: L3_SCORES(1)
+    case 2: L3_SCORES(2)
+    case 3: L3_SCORES(3)
+    case 4: L3_SCORES(4)
+    case 5: L3_SCORES(5)
+    case 6: L3_SCORES(6)
+    case 7: L3_SCORES(7)
+    default: L3_SCORES(8)
   }
+#undef L3_SCORES
 }
 
 // CTA per tile, thread per token: P = softmax over the d rows of S, and
 // G_s = P (G_p - sum_j P G_p), in place.
 __global__ void __launch_bounds__(DENSE_TILE_M)
-    k_bwd_dense_softmax(const int32_t *__restrict__ group_rows, const DenseTile *__restrict__ tiles,
+    k_bwd_dense_softmax(const int32_t *__restrict__ group_tok_start,
+                        const int32_t *__restrict__ group_rows, const DenseTile *__restrict__ tiles,
                         float *__restrict__ slots, int slot_rows) {
   const int64_t b = blockIdx.x;
-  const int d = group_rows[tiles[b].group];
+  const DenseTile tl = tiles[b];
+  const int d = group_rows[tl.group];
   const int t = threadIdx.x;
+  if (t >= group_tok_start[tl.group + 1] - tl.tok0) return;
   float *S = slot_plane(slots, b, slot_rows, 0) + t, *G = slot_plane(slots, b, slot_rows, 1) + t;
   float mx = -INFINITY;
   for (int j = 0; j < d; ++j) mx = fmaxf(mx, S[j * DENSE_TILE_M]);
@@ -535,8 +566,51 @@ __global__ void __launch_bounds__(DENSE_TILE_M)
   for (int j = 0; j < d; ++j) G[j * DENSE_TILE_M] = S[j * DENSE_TILE_M] * (G[j * DENSE_TILE_M] - dot);
 }
 
-// CTA per (tile, 64-column block of d_in): dx[t][col] += sum_j G_s[j][t] K_t[j][col]
-// for the tile's 128 tokens (each token's dx belongs to this CTA alone).
+// dx[t][col] += sum_j G_s[j][t] K_t[j][col] for tokens t < c of 16 NE
+template <int NE>
+__device__ __forceinline__ void dense_dx(const void *W_K, int wtype, const float *G,
+                                         const int32_t *__restrict__ perm, int tok0, int64_t r0,
+                                         int d, int c, int col0, int d_in, float *__restrict__ dx,
+                                         float (*as)[DENSE_TILE_M + 1], float (*bs)[64 + 1]) {
+  const int tid = threadIdx.x, tx = tid % 16, ty = tid / 16;
+  constexpr int T = 16 * NE;
+  float acc[NE][4] = {};
+  for (int j0 = 0; j0 < d; j0 += DB_K) {
+    __syncthreads();
+    for (int i = tid; i < DB_K * T; i += 256) {
+      const int jj = i / T, t = i % T;
+      as[jj][t] = j0 + jj < d ? G[(int64_t)(j0 + jj) * DENSE_TILE_M + t] : 0.f;
+    }
+    for (int i = tid; i < DB_K * 64; i += 256) {
+      const int jj = i / 64, cc = i % 64;
+      bs[jj][cc] = j0 + jj < d ? ldx(W_K, wtype, (r0 + j0 + jj) * d_in + col0 + cc) : 0.f;
+    }
+    __syncthreads();
+#pragma unroll 4
+    for (int jj = 0; jj < DB_K; ++jj) {
+      float a[NE], bv[4];
+#pragma unroll
+      for (int i = 0; i < NE; ++i) a[i] = as[jj][ty + 16 * i];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) bv[e] = bs[jj][tx + 16 * e];
+#pragma unroll
+      for (int i = 0; i < NE; ++i)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[i][e] = fmaf(a[i], bv[e], acc[i][e]);
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < NE; ++i) {
+    const int t = ty + 16 * i;
+    if (t >= c) continue;
+    float *o = dx + (int64_t)perm[tok0 + t] * d_in + col0;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) o[tx + 16 * e] += acc[i][e];
+  }
+}
+
+// CTA per (tile, 64-column block of d_in): dx of the tile's tokens (each
+// token's dx belongs to this CTA alone).
 __global__ void __launch_bounds__(256)
     k_bwd_dense_dx(const void *W_K, int wtype, const int32_t *__restrict__ perm,
                    const int32_t *__restrict__ group_tok_start,
@@ -554,40 +628,20 @@ __global__ void __launch_bounds__(256)
   const int64_t r0 = group_row_start[tl.group];
   const int c = min(DENSE_TILE_M, group_tok_start[tl.group + 1] - tl.tok0);
   const float *G = slot_plane(const_cast<float *>(slots), b, slot_rows, 1);
-  const int tid = threadIdx.x, tx = tid % 16, ty = tid / 16;
-  float acc[8][4] = {};
-  for (int j0 = 0; j0 < d; j0 += DB_K) {
-    __syncthreads();
-    for (int i = tid; i < DB_K * DENSE_TILE_M; i += 256) {
-      const int jj = i / DENSE_TILE_M, t = i % DENSE_TILE_M;
-      as[jj][t] = j0 + jj < d ? G[(int64_t)(j0 + jj) * DENSE_TILE_M + t] : 0.f;
-    }
-    for (int i = tid; i < DB_K * 64; i += 256) {
-      const int jj = i / 64, cc = i % 64;
-      bs[jj][cc] = j0 + jj < d ? ldx(W_K, wtype, (r0 + j0 + jj) * d_in + col0 + cc) : 0.f;
-    }
-    __syncthreads();
-#pragma unroll 4
-    for (int jj = 0; jj < DB_K; ++jj) {
-      float a[8], bv[4];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) a[i] = as[jj][ty + 16 * i];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) bv[e] = bs[jj][tx + 16 * e];
-#pragma unroll
-      for (int i = 0; i < 8; ++i)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) acc[i][e] = fmaf(a[i], bv[e], acc[i][e]);
-    }
+#define L3_DX(NE)                                                                    \
+  dense_dx<NE>(W_K, wtype, G, perm, tl.tok0, r0, d, c, col0, d_in, dx, as, bs); \
+  break;
+  switch ((c + 15) / 16) {
+    case 1: L3_DX(1)
+    case 2: L3_DX(2)
+    case 3: L3_DX(3)
+    case 4: L3_DX(4)
+    case 5: L3_DX(5)
+    case 6: L3_DX(6)
+    case 7: L3_DX(7)
+    default: L3_DX(8)
   }
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int t = ty + 16 * i;
-    if (t >= c) continue;
-    float *o = dx + (int64_t)perm[tl.tok0 + t] * d_in + col0;
-#pragma unroll
-    for (int e = 0; e < 4; ++e) o[tx + 16 * e] += acc[i][e];
-  }
+#undef L3_DX
 }
 
 // dK_t (+)= G_s^T X and dV_t (+)= P^T G_a over one dense tile's tokens, from
@@ -853,31 +907,47 @@ extern "C" l3_status l3_backward(const void *x, l3_plan_t p, const void *W_K, co
   const int64_t n_tail = p->n_tail_items;
   if (st == L3_OK && n_tail > 0) {
     LaunchTimer t("bwd_attention_tail", s);
-    e = cudaFuncSetAttribute(k_attn_backward_tail, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)attn_smem);
-    if (e == cudaSuccess) {
-      k_attn_backward_tail<<<(unsigned)n_tail, 256, attn_smem, s>>>(
-          x, W_K, W_V, wt, g_a, p->tail_items, (int)d.d_in, (int)d.d_emb, dx, dW_K, dW_V);
+    auto launch_tail = [&](auto kernel, int nt, int cls) {
+      const int64_t i0 = p->tail_class_start[cls], n = p->tail_class_start[cls + 1] - i0;
+      if (n <= 0 || e != cudaSuccess) return;
+      const size_t smem = (nt * d.d_in + nt * d.d_emb + 2 * nt * A_MAX_K) * f;
+      e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if (e != cudaSuccess) return;
+      kernel<<<(unsigned)n, 256, smem, s>>>(x, W_K, W_V, wt, g_a, p->tail_items + i0, (int)d.d_in,
+                                            (int)d.d_emb, dx, dW_K, dW_V);
       e = cudaGetLastError();
-    }
+    };
+    launch_tail(k_attn_backward_tail<1>, 1, 0);
+    launch_tail(k_attn_backward_tail<2>, 2, 1);
+    launch_tail(k_attn_backward_tail<4>, 4, 2);
+    launch_tail(k_attn_backward_tail<8>, 8, 3);
     if (e != cudaSuccess) st = cuda_fail(e, "attention backward (tail items)");
   }
   if (st == L3_OK && n_dt > 0) {
-    LaunchTimer t("bwd_attention_dense", s);
-    k_bwd_dense_scores<<<(unsigned)(n_dt * (slot_rows / DB_J)), 256, 0, s>>>(
-        x, W_K, W_V, wt, g_a, p->perm, p->group_tok_start, p->group_row_start, p->group_rows,
-        p->dense_tiles, slots, slot_rows, (int)d.d_in, (int)d.d_emb);
-    k_bwd_dense_softmax<<<(unsigned)n_dt, DENSE_TILE_M, 0, s>>>(p->group_rows, p->dense_tiles,
-                                                                 slots, slot_rows);
-    k_bwd_dense_dx<<<(unsigned)(n_dt * (d.d_in / 64)), 256, 0, s>>>(
-        W_K, wt, p->perm, p->group_tok_start, p->group_row_start, p->group_rows, p->dense_tiles,
-        slots, slot_rows, (int)d.d_in, dx);
+    {
+      LaunchTimer t("bwd_dense_scores", s);
+      k_bwd_dense_scores<<<(unsigned)(n_dt * (slot_rows / DB_J)), 256, 0, s>>>(
+          x, W_K, W_V, wt, g_a, p->perm, p->group_tok_start, p->group_row_start, p->group_rows,
+          p->dense_tiles, slots, slot_rows, (int)d.d_in, (int)d.d_emb);
+    }
+    {
+      LaunchTimer t("bwd_dense_softmax", s);
+      k_bwd_dense_softmax<<<(unsigned)n_dt, DENSE_TILE_M, 0, s>>>(
+          p->group_tok_start, p->group_rows, p->dense_tiles, slots, slot_rows);
+    }
+    {
+      LaunchTimer t("bwd_dense_dx", s);
+      k_bwd_dense_dx<<<(unsigned)(n_dt * (d.d_in / 64)), 256, 0, s>>>(
+          W_K, wt, p->perm, p->group_tok_start, p->group_row_start, p->group_rows, p->dense_tiles,
+          slots, slot_rows, (int)d.d_in, dx);
+    }
     e = cudaGetLastError();
     const size_t dw_smem = (DENSE_TILE_M * DW_C + DW_J * DW_LD) * f;
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(k_attn_backward_dw, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                (int)dw_smem);
     if (e == cudaSuccess) {
+      LaunchTimer t("bwd_dense_dw", s);
       const int64_t n_cb = d.d_in / DW_C + d.d_emb / DW_C;
       k_attn_backward_dw<<<(unsigned)(n_dt * n_cb), 256, dw_smem, s>>>(
           x, wt, g_a, p->perm, p->group_tok_start, p->group_row_start, p->group_rows,
