@@ -273,7 +273,7 @@ def run_lzw(args, w):
 
 def run_backward(args, w, tables, batch, dev, dist, world, rank):
     """Plan, forward and backward (fp32 gradients for a random dL/dy) per
-    batch; the backward is the CUDA-core implementation."""
+    batch."""
     d = {k: getattr(tables, k).to(dev) for k in ("offsets", "W_K", "W_up", "ln_gamma", "ln_beta",
                                                  "W_mix")}
     d["W_V"] = d["W_K"] if tables.W_V is tables.W_K else tables.W_V.to(dev)
@@ -420,7 +420,7 @@ def main():
     ap.add_argument("--lzw", type=int, default=0, metavar="TOKENS",
                     help="time the LZW allocation on a synthetic corpus of this many tokens")
     ap.add_argument("--backward", action="store_true",
-                    help="time l3_forward + l3_backward per batch (CUDA-core backward)")
+                    help="time l3_forward + l3_backward per batch")
     ap.add_argument("--offload", action="store_true",
                     help="W_K / W_V in pinned host memory; each step stages the batch's rows")
     args = ap.parse_args()
