@@ -451,54 +451,114 @@ __device__ __forceinline__ float *slot_plane(float *slots, int64_t b, int slot_r
   return slots + (b * 2 + plane) * (int64_t)slot_rows * DENSE_TILE_M;
 }
 
+// D += A B^T on the warp's tensor cores: A 16 x 16 bf16 (row-major
+// fragment), B 8 x 16 bf16 (one token per column), D 16 x 8 fp32.
+__device__ __forceinline__ void mma_bf16(float (&dacc)[4], const uint32_t (&a)[4], uint32_t b0,
+                                         uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+      "{%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(dacc[0]), "+f"(dacc[1]), "+f"(dacc[2]), "+f"(dacc[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// bf16 pair (lo element first) from two floats, and the hi / lo split of a float
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t *>(&v);
+}
+
+constexpr int DS_LD = DB_K + 8;  // bf16 row stride of the staged tiles (conflict-free fragments)
+
 // S and G_p of 64 rows x 16 NE tokens (NE = ceil(c / 16) column groups of
-// the tile; columns c..16 NE - 1 come out zero, later columns are left alone).
+// the tile; columns c..16 NE - 1 come out zero, later columns are left
+// alone), on mma.sync: warp w owns rows 16 (w % 4) .. + 15 and the 8-token
+// column blocks w / 4, w / 4 + 2, ... S takes K_t and x as they are (bf16);
+// G_p takes V_t against g_a split into two bf16 parts (hi + lo), so it keeps
+// about 16 bits of g_a.
 template <int NE>
 __device__ __forceinline__ void dense_scores(const void *x, const void *W_K, const void *W_V,
-                                             int wtype, const float *__restrict__ g_a,
-                                             const int64_t *tok, int64_t r0, int d, int jb,
-                                             int d_in, int d_emb, float *plane0, float *plane1,
-                                             float (*as)[DB_J + 1],
-                                             float (*bs)[DENSE_TILE_M + 1]) {
-  const int tid = threadIdx.x, tx = tid % 16, ty = tid / 16;
+                                             const float *__restrict__ g_a, const int64_t *tok,
+                                             int64_t r0, int d, int jb, int d_in, int d_emb,
+                                             float *plane0, float *plane1,
+                                             __nv_bfloat16 (*as)[DS_LD],
+                                             __nv_bfloat16 (*bs)[DS_LD],
+                                             __nv_bfloat16 (*bl)[DS_LD]) {
+  const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+  const int g = lane >> 2, tg = lane & 3;
+  const int jr = (warp & 3) * 16, nb0 = warp >> 2;
+  constexpr int T = 16 * NE;
   for (int plane = 0; plane < 2; ++plane) {
     const int K = plane == 0 ? d_in : d_emb;
-    float acc[4][NE] = {};
+    const __nv_bfloat16 *W = reinterpret_cast<const __nv_bfloat16 *>(plane == 0 ? W_K : W_V);
+    float acc[NE][4] = {};
     for (int k0 = 0; k0 < K; k0 += DB_K) {
       __syncthreads();  // tok written / the previous stage read
-      for (int i = tid; i < DB_J * DB_K; i += 256) {
-        const int jj = i / DB_K, kk = i % DB_K;
-        const int64_t idx = (r0 + jb + jj) * K + k0 + kk;
-        as[kk][jj] = jb + jj < d ? ldx(plane == 0 ? W_K : W_V, wtype, idx) : 0.f;
+      {  // 64 rows x 32 k of K_t or V_t: 16 bytes per thread
+        const int row = tid / 4, seg = (tid % 4) * 8;
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (jb + row < d) v = *reinterpret_cast<const uint4 *>(W + (r0 + jb + row) * K + k0 + seg);
+        *reinterpret_cast<uint4 *>(&as[row][seg]) = v;
       }
-      for (int i = tid; i < 16 * NE * DB_K; i += 256) {
-        const int t = i / DB_K, kk = i % DB_K;
+      for (int i = tid; i < T * 4; i += 256) {  // T tokens x 32 k
+        const int t = i / 4, seg = (i % 4) * 8;
         const int64_t tk = tok[t];
-        bs[kk][t] = tk < 0 ? 0.f
-                    : plane == 0 ? ldx(x, wtype, tk * d_in + k0 + kk)
-                                 : g_a[tk * d_emb + k0 + kk];
+        if (plane == 0) {
+          uint4 v = make_uint4(0, 0, 0, 0);
+          if (tk >= 0)
+            v = *reinterpret_cast<const uint4 *>(reinterpret_cast<const __nv_bfloat16 *>(x) +
+                                                 tk * d_in + k0 + seg);
+          *reinterpret_cast<uint4 *>(&bs[t][seg]) = v;
+        } else {
+          float f[8] = {};
+          if (tk >= 0) {
+            const float4 u0 = *reinterpret_cast<const float4 *>(g_a + tk * d_emb + k0 + seg);
+            const float4 u1 = *reinterpret_cast<const float4 *>(g_a + tk * d_emb + k0 + seg + 4);
+            f[0] = u0.x; f[1] = u0.y; f[2] = u0.z; f[3] = u0.w;
+            f[4] = u1.x; f[5] = u1.y; f[6] = u1.z; f[7] = u1.w;
+          }
+          uint32_t hi[4], lo[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const __nv_bfloat16 h0 = __float2bfloat16_rn(f[2 * e]);
+            const __nv_bfloat16 h1 = __float2bfloat16_rn(f[2 * e + 1]);
+            hi[e] = pack_bf16(__bfloat162float(h0), __bfloat162float(h1));
+            lo[e] = pack_bf16(f[2 * e] - __bfloat162float(h0), f[2 * e + 1] - __bfloat162float(h1));
+          }
+          *reinterpret_cast<uint4 *>(&bs[t][seg]) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+          *reinterpret_cast<uint4 *>(&bl[t][seg]) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+        }
       }
       __syncthreads();
-#pragma unroll 4
-      for (int kk = 0; kk < DB_K; ++kk) {
-        float a[4], bv[NE];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) a[i] = as[kk][ty + 16 * i];
+      for (int kk = 0; kk < DB_K; kk += 16) {
+        uint32_t a[4];
+        a[0] = *reinterpret_cast<const uint32_t *>(&as[jr + g][kk + 2 * tg]);
+        a[1] = *reinterpret_cast<const uint32_t *>(&as[jr + g + 8][kk + 2 * tg]);
+        a[2] = *reinterpret_cast<const uint32_t *>(&as[jr + g][kk + 8 + 2 * tg]);
+        a[3] = *reinterpret_cast<const uint32_t *>(&as[jr + g + 8][kk + 8 + 2 * tg]);
 #pragma unroll
-        for (int e = 0; e < NE; ++e) bv[e] = bs[kk][tx + 16 * e];
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-          for (int e = 0; e < NE; ++e) acc[i][e] = fmaf(a[i], bv[e], acc[i][e]);
+        for (int i = 0; i < NE; ++i) {
+          const int n = (nb0 + 2 * i) * 8 + g;  // this lane's token in the block
+          mma_bf16(acc[i], a, *reinterpret_cast<const uint32_t *>(&bs[n][kk + 2 * tg]),
+                   *reinterpret_cast<const uint32_t *>(&bs[n][kk + 8 + 2 * tg]));
+          if (plane == 1)
+            mma_bf16(acc[i], a, *reinterpret_cast<const uint32_t *>(&bl[n][kk + 2 * tg]),
+                     *reinterpret_cast<const uint32_t *>(&bl[n][kk + 8 + 2 * tg]));
+        }
       }
     }
     float *out = plane == 0 ? plane0 : plane1;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int j = jb + ty + 16 * i;
-      if (j < d)
-#pragma unroll
-        for (int e = 0; e < NE; ++e) out[(int64_t)j * DENSE_TILE_M + tx + 16 * e] = acc[i][e];
+    for (int i = 0; i < NE; ++i) {
+      const int col = (nb0 + 2 * i) * 8 + 2 * tg;
+      const int j0 = jb + jr + g, j1 = j0 + 8;
+      if (j0 < d)
+        *reinterpret_cast<float2 *>(out + (int64_t)j0 * DENSE_TILE_M + col) =
+            make_float2(acc[i][0], acc[i][1]);
+      if (j1 < d)
+        *reinterpret_cast<float2 *>(out + (int64_t)j1 * DENSE_TILE_M + col) =
+            make_float2(acc[i][2], acc[i][3]);
     }
   }
 }
@@ -511,9 +571,11 @@ __global__ void __launch_bounds__(256)
                        const int32_t *__restrict__ group_row_start,
                        const int32_t *__restrict__ group_rows, const DenseTile *__restrict__ tiles,
                        float *__restrict__ slots, int slot_rows, int d_in, int d_emb) {
-  __shared__ float as[DB_K][DB_J + 1];          // rows of K_t or V_t, k-major
-  __shared__ float bs[DB_K][DENSE_TILE_M + 1];  // x or g_a of the tokens, k-major
+  __shared__ __align__(16) __nv_bfloat16 as[DB_J][DS_LD];          // rows of K_t or V_t
+  __shared__ __align__(16) __nv_bfloat16 bs[DENSE_TILE_M][DS_LD];  // x, or g_a's hi part
+  __shared__ __align__(16) __nv_bfloat16 bl[DENSE_TILE_M][DS_LD];  // g_a's lo part
   __shared__ int64_t tok[DENSE_TILE_M];
+  (void)wtype;  // dense tiles exist for bf16 layers only
   const int n_jb = slot_rows / DB_J;
   const int64_t b = blockIdx.x / n_jb;
   const int jb = (blockIdx.x % n_jb) * DB_J;
@@ -525,7 +587,7 @@ __global__ void __launch_bounds__(256)
   if (threadIdx.x < DENSE_TILE_M) tok[threadIdx.x] = threadIdx.x < c ? perm[tl.tok0 + threadIdx.x] : -1;
   float *p0 = slot_plane(slots, b, slot_rows, 0), *p1 = slot_plane(slots, b, slot_rows, 1);
 #define L3_SCORES(NE)                                                                           \
-  dense_scores<NE>(x, W_K, W_V, wtype, g_a, tok, r0, d, jb, d_in, d_emb, p0, p1, as, bs); \
+  dense_scores<NE>(x, W_K, W_V, g_a, tok, r0, d, jb, d_in, d_emb, p0, p1, as, bs, bl);  \
   break;
   switch ((c + 15) / 16) {
     case 1: L3_SCORES(1)
@@ -922,6 +984,10 @@ extern "C" l3_status l3_backward(const void *x, l3_plan_t p, const void *W_K, co
     launch_tail(k_attn_backward_tail<4>, 4, 2);
     launch_tail(k_attn_backward_tail<8>, 8, 3);
     if (e != cudaSuccess) st = cuda_fail(e, "attention backward (tail items)");
+  }
+  if (st == L3_OK && n_dt > 0 && !(a16(x) && a16(W_K) && a16(W_V))) {
+    set_error("l3_backward: x, W_K and W_V must be 16-byte aligned");
+    st = L3_ERR_INVALID_ARG;
   }
   if (st == L3_OK && n_dt > 0) {
     {
