@@ -628,46 +628,82 @@ __global__ void __launch_bounds__(DENSE_TILE_M)
   for (int j = 0; j < d; ++j) G[j * DENSE_TILE_M] = S[j * DENSE_TILE_M] * (G[j * DENSE_TILE_M] - dot);
 }
 
-// dx[t][col] += sum_j G_s[j][t] K_t[j][col] for tokens t < c of 16 NE
+// A fragment (16 x 16, row-major, row stride DS_LD or wider) at row r0, k0
+template <int LD>
+__device__ __forceinline__ void load_a(uint32_t (&a)[4], const __nv_bfloat16 (*m)[LD], int r0,
+                                       int k0, int g, int tg) {
+  a[0] = *reinterpret_cast<const uint32_t *>(&m[r0 + g][k0 + 2 * tg]);
+  a[1] = *reinterpret_cast<const uint32_t *>(&m[r0 + g + 8][k0 + 2 * tg]);
+  a[2] = *reinterpret_cast<const uint32_t *>(&m[r0 + g][k0 + 8 + 2 * tg]);
+  a[3] = *reinterpret_cast<const uint32_t *>(&m[r0 + g + 8][k0 + 8 + 2 * tg]);
+}
+
+// dx[t][col] += sum_j G_s[j][t] K_t[j][col] for the tile's tokens t < c of
+// 16 NE, on mma.sync: M = tokens, N = 64 columns (warp w: columns 8w..8w+7,
+// all NE 16-token blocks), K = rows j, 32 per stage. G_s enters as a hi / lo
+// bf16 pair, K_t as it is.
 template <int NE>
-__device__ __forceinline__ void dense_dx(const void *W_K, int wtype, const float *G,
+__device__ __forceinline__ void dense_dx(const __nv_bfloat16 *__restrict__ Wk,
+                                         const float *__restrict__ G,
                                          const int32_t *__restrict__ perm, int tok0, int64_t r0,
                                          int d, int c, int col0, int d_in, float *__restrict__ dx,
-                                         float (*as)[DENSE_TILE_M + 1], float (*bs)[64 + 1]) {
-  const int tid = threadIdx.x, tx = tid % 16, ty = tid / 16;
+                                         __nv_bfloat16 (*ah)[DS_LD], __nv_bfloat16 (*al)[DS_LD],
+                                         __nv_bfloat16 (*bt)[DS_LD]) {
+  const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+  const int g = lane >> 2, tg = lane & 3;
   constexpr int T = 16 * NE;
   float acc[NE][4] = {};
   for (int j0 = 0; j0 < d; j0 += DB_K) {
-    __syncthreads();
-    for (int i = tid; i < DB_K * T; i += 256) {
-      const int jj = i / T, t = i % T;
-      as[jj][t] = j0 + jj < d ? G[(int64_t)(j0 + jj) * DENSE_TILE_M + t] : 0.f;
+    __syncthreads();  // the previous stage read
+    // G_s rows j0..j0+31 x tokens 0..T-1 -> ah / al [token][j]
+    for (int i = tid; i < DB_K * T / 4; i += 256) {
+      const int jj = i % DB_K, t4 = (i / DB_K) * 4;
+      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (j0 + jj < d) v = *reinterpret_cast<const float4 *>(G + (int64_t)(j0 + jj) * DENSE_TILE_M + t4);
+      const float f[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const __nv_bfloat16 h = __float2bfloat16_rn(f[e]);
+        ah[t4 + e][jj] = h;
+        al[t4 + e][jj] = __float2bfloat16_rn(f[e] - __bfloat162float(h));
+      }
     }
-    for (int i = tid; i < DB_K * 64; i += 256) {
-      const int jj = i / 64, cc = i % 64;
-      bs[jj][cc] = j0 + jj < d ? ldx(W_K, wtype, (r0 + j0 + jj) * d_in + col0 + cc) : 0.f;
+    {  // K_t rows j0..j0+31, columns col0..col0+63 -> bt [column][j]
+      const int jj = tid % DB_K, seg = (tid / DB_K) * 8;
+      uint4 v = make_uint4(0, 0, 0, 0);
+      if (j0 + jj < d) v = *reinterpret_cast<const uint4 *>(Wk + (r0 + j0 + jj) * d_in + col0 + seg);
+      const __nv_bfloat16 *e8 = reinterpret_cast<const __nv_bfloat16 *>(&v);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) bt[seg + q][jj] = e8[q];
     }
     __syncthreads();
-#pragma unroll 4
-    for (int jj = 0; jj < DB_K; ++jj) {
-      float a[NE], bv[4];
 #pragma unroll
-      for (int i = 0; i < NE; ++i) a[i] = as[jj][ty + 16 * i];
+    for (int kk = 0; kk < DB_K; kk += 16) {
+      const uint32_t b0 = *reinterpret_cast<const uint32_t *>(&bt[warp * 8 + g][kk + 2 * tg]);
+      const uint32_t b1 = *reinterpret_cast<const uint32_t *>(&bt[warp * 8 + g][kk + 8 + 2 * tg]);
 #pragma unroll
-      for (int e = 0; e < 4; ++e) bv[e] = bs[jj][tx + 16 * e];
-#pragma unroll
-      for (int i = 0; i < NE; ++i)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) acc[i][e] = fmaf(a[i], bv[e], acc[i][e]);
+      for (int i = 0; i < NE; ++i) {
+        uint32_t a[4];
+        load_a<DS_LD>(a, ah, 16 * i, kk, g, tg);
+        mma_bf16(acc[i], a, b0, b1);
+        load_a<DS_LD>(a, al, 16 * i, kk, g, tg);
+        mma_bf16(acc[i], a, b0, b1);
+      }
     }
   }
+  const int col = col0 + warp * 8 + 2 * tg;
 #pragma unroll
   for (int i = 0; i < NE; ++i) {
-    const int t = ty + 16 * i;
-    if (t >= c) continue;
-    float *o = dx + (int64_t)perm[tok0 + t] * d_in + col0;
 #pragma unroll
-    for (int e = 0; e < 4; ++e) o[tx + 16 * e] += acc[i][e];
+    for (int h = 0; h < 2; ++h) {
+      const int t = 16 * i + g + 8 * h;
+      if (t >= c) continue;
+      float2 *o = reinterpret_cast<float2 *>(dx + (int64_t)perm[tok0 + t] * d_in + col);
+      float2 v = *o;
+      v.x += acc[i][2 * h];
+      v.y += acc[i][2 * h + 1];
+      *o = v;
+    }
   }
 }
 
@@ -680,8 +716,10 @@ __global__ void __launch_bounds__(256)
                    const int32_t *__restrict__ group_rows, const DenseTile *__restrict__ tiles,
                    const float *__restrict__ slots, int slot_rows, int d_in,
                    float *__restrict__ dx) {
-  __shared__ float as[DB_K][DENSE_TILE_M + 1];  // g_s, j-major
-  __shared__ float bs[DB_K][64 + 1];            // K_t rows, j-major
+  __shared__ __align__(16) __nv_bfloat16 ah[DENSE_TILE_M][DS_LD];  // g_s hi, [token][j]
+  __shared__ __align__(16) __nv_bfloat16 al[DENSE_TILE_M][DS_LD];  // g_s lo
+  __shared__ __align__(16) __nv_bfloat16 bt[64][DS_LD];            // K_t, [column][j]
+  (void)wtype;  // dense tiles exist for bf16 layers only
   const int n_cb = d_in / 64;
   const int64_t b = blockIdx.x / n_cb;
   const int col0 = (blockIdx.x % n_cb) * 64;
@@ -690,8 +728,9 @@ __global__ void __launch_bounds__(256)
   const int64_t r0 = group_row_start[tl.group];
   const int c = min(DENSE_TILE_M, group_tok_start[tl.group + 1] - tl.tok0);
   const float *G = slot_plane(const_cast<float *>(slots), b, slot_rows, 1);
-#define L3_DX(NE)                                                                    \
-  dense_dx<NE>(W_K, wtype, G, perm, tl.tok0, r0, d, c, col0, d_in, dx, as, bs); \
+  const __nv_bfloat16 *Wk = reinterpret_cast<const __nv_bfloat16 *>(W_K);
+#define L3_DX(NE)                                                                 \
+  dense_dx<NE>(Wk, G, perm, tl.tok0, r0, d, c, col0, d_in, dx, ah, al, bt); \
   break;
   switch ((c + 15) / 16) {
     case 1: L3_DX(1)
@@ -706,13 +745,103 @@ __global__ void __launch_bounds__(256)
 #undef L3_DX
 }
 
-// dK_t (+)= G_s^T X and dV_t (+)= P^T G_a over one dense tile's tokens, from
-// the planes k_bwd_dense_softmax left: CTA per (tile, 64-column
-// block of d_in for dK or of d_emb for dV), 64 rows x 64 columns at a time,
-// 4 x 4 outputs per thread, the sum over the tile's (up to 128) tokens in
-// registers, then one atomic add per element (the tiles of one group share
-// its rows).
-constexpr int DW_J = 64, DW_C = 64, DW_LD = DENSE_TILE_M + 4;
+// dK_t (+)= G_s X and dV_t (+)= P G_a over one dense tile's tokens, from the
+// planes k_bwd_dense_softmax left, on mma.sync: CTA per (tile, 64-column
+// block of d_in for dK or of d_emb for dV); M = 64 rows at a time (warp w:
+// rows 16 (w % 4).., columns 32 (w / 4)..), N = 64 columns, K = the tile's
+// 16 NE tokens. G_s / P enter as hi / lo bf16 pairs, x as it is, g_a as a
+// pair (dV adds hi x hi, lo x hi, hi x lo). One atomic add per element: the
+// tiles of one group share its rows.
+constexpr int DW_C = 64, DW_LD = DENSE_TILE_M + 8;
+
+template <int NE>
+__device__ __forceinline__ void dense_dw(const __nv_bfloat16 *__restrict__ x,
+                                         const float *__restrict__ g_a, const float *__restrict__ A,
+                                         const int32_t *__restrict__ perm, int tok0, int64_t r0,
+                                         int d, int c, bool is_k, int col0, int width, int d_in,
+                                         int d_emb, float *__restrict__ out,
+                                         __nv_bfloat16 (*bh)[DW_LD], __nv_bfloat16 (*bl)[DW_LD],
+                                         __nv_bfloat16 (*ahi)[DW_LD],
+                                         __nv_bfloat16 (*alo)[DW_LD]) {
+  const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+  const int g = lane >> 2, tg = lane & 3;
+  constexpr int T = 16 * NE;
+  // B: x or g_a of tokens 0..T-1, columns col0..col0+63 -> bh / bl [column][token]
+  for (int i = tid; i < T * (DW_C / 8); i += 256) {
+    const int t = i % T, seg = (i / T) * 8;
+    float f[8] = {};
+    if (t < c) {
+      const int64_t tk = perm[tok0 + t];
+      if (is_k) {
+        const uint4 v = *reinterpret_cast<const uint4 *>(x + tk * d_in + col0 + seg);
+        const __nv_bfloat16 *e8 = reinterpret_cast<const __nv_bfloat16 *>(&v);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) f[q] = __bfloat162float(e8[q]);
+      } else {
+        const float4 u0 = *reinterpret_cast<const float4 *>(g_a + tk * d_emb + col0 + seg);
+        const float4 u1 = *reinterpret_cast<const float4 *>(g_a + tk * d_emb + col0 + seg + 4);
+        f[0] = u0.x; f[1] = u0.y; f[2] = u0.z; f[3] = u0.w;
+        f[4] = u1.x; f[5] = u1.y; f[6] = u1.z; f[7] = u1.w;
+      }
+    }
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const __nv_bfloat16 h = __float2bfloat16_rn(f[q]);
+      bh[seg + q][t] = h;
+      bl[seg + q][t] = __float2bfloat16_rn(f[q] - __bfloat162float(h));
+    }
+  }
+  const int mr = (warp & 3) * 16, nb = (warp >> 2) * 32;
+  for (int jb = 0; jb < d; jb += 64) {
+    __syncthreads();  // B written / the previous block's A read
+    // A: rows jb..jb+63 of G_s or P, tokens 0..T-1 -> ahi / alo [row][token]
+    for (int i = tid; i < 64 * T / 4; i += 256) {
+      const int jj = i / (T / 4), t4 = (i % (T / 4)) * 4;
+      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (jb + jj < d && t4 < c)
+        v = *reinterpret_cast<const float4 *>(A + (int64_t)(jb + jj) * DENSE_TILE_M + t4);
+      const float fv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float fe = t4 + e < c ? fv[e] : 0.f;
+        const __nv_bfloat16 h = __float2bfloat16_rn(fe);
+        ahi[jj][t4 + e] = h;
+        alo[jj][t4 + e] = __float2bfloat16_rn(fe - __bfloat162float(h));
+      }
+    }
+    __syncthreads();
+    float acc[4][4] = {};
+#pragma unroll
+    for (int kk = 0; kk < T; kk += 16) {
+      uint32_t ah4[4], al4[4];
+      load_a<DW_LD>(ah4, ahi, mr, kk, g, tg);
+      load_a<DW_LD>(al4, alo, mr, kk, g, tg);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int n = nb + q * 8 + g;
+        const uint32_t b0 = *reinterpret_cast<const uint32_t *>(&bh[n][kk + 2 * tg]);
+        const uint32_t b1 = *reinterpret_cast<const uint32_t *>(&bh[n][kk + 8 + 2 * tg]);
+        mma_bf16(acc[q], ah4, b0, b1);
+        mma_bf16(acc[q], al4, b0, b1);
+        if (!is_k)
+          mma_bf16(acc[q], ah4, *reinterpret_cast<const uint32_t *>(&bl[n][kk + 2 * tg]),
+                   *reinterpret_cast<const uint32_t *>(&bl[n][kk + 8 + 2 * tg]));
+      }
+    }
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int col = col0 + nb + q * 8 + 2 * tg;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int j = jb + mr + g + 8 * h;
+        if (j >= d) continue;
+        float *o = out + (r0 + j) * width + col;
+        atomicAdd(o, acc[q][2 * h]);
+        atomicAdd(o + 1, acc[q][2 * h + 1]);
+      }
+    }
+  }
+}
 
 __global__ void __launch_bounds__(256)
     k_attn_backward_dw(const void *x, int wtype, const float *__restrict__ g_a,
@@ -721,9 +850,12 @@ __global__ void __launch_bounds__(256)
                        const int32_t *__restrict__ group_rows, const DenseTile *__restrict__ tiles,
                        const float *__restrict__ slots, int slot_rows, int d_in, int d_emb,
                        float *__restrict__ dW_K, float *__restrict__ dW_V) {
-  extern __shared__ float sm[];
-  float *xs = sm;                        // [DENSE_TILE_M][DW_C]: x or g_a of the tile's tokens
-  float *ms = xs + DENSE_TILE_M * DW_C;  // [DW_J][DW_LD]: g_s or p of 64 rows
+  extern __shared__ __align__(16) uint8_t dw_raw[];
+  auto bh = reinterpret_cast<__nv_bfloat16 (*)[DW_LD]>(dw_raw);  // [64 columns][DW_LD]
+  auto bl = bh + DW_C;
+  auto ahi = bl + DW_C;  // [64 rows][DW_LD]
+  auto alo = ahi + 64;
+  (void)wtype;  // dense tiles exist for bf16 layers only
   const int n_cbk = d_in / DW_C, n_cb = n_cbk + d_emb / DW_C;
   const int64_t b = blockIdx.x / n_cb;
   const int cb = blockIdx.x % n_cb;
@@ -733,47 +865,24 @@ __global__ void __launch_bounds__(256)
   const int64_t r0 = group_row_start[tl.group];
   const int d = group_rows[tl.group];
   const int c = min(DENSE_TILE_M, group_tok_start[tl.group + 1] - tl.tok0);
-  const float *src = slots + (b * 2 + (is_k ? 1 : 0)) * (int64_t)slot_rows * DENSE_TILE_M;
+  const float *A = slots + (b * 2 + (is_k ? 1 : 0)) * (int64_t)slot_rows * DENSE_TILE_M;
   float *out = is_k ? dW_K : dW_V;
-  const int tid = threadIdx.x, tx = tid % 16, ty = tid / 16;
-  for (int i = tid; i < DENSE_TILE_M * DW_C; i += blockDim.x) {
-    const int t = i / DW_C, cc = i % DW_C;
-    float v = 0.f;
-    if (t < c) {
-      const int64_t tok = perm[tl.tok0 + t];
-      v = is_k ? ldx(x, wtype, tok * d_in + col0 + cc) : g_a[tok * d_emb + col0 + cc];
-    }
-    xs[i] = v;
+  const __nv_bfloat16 *xb = reinterpret_cast<const __nv_bfloat16 *>(x);
+#define L3_DW(NE)                                                                               \
+  dense_dw<NE>(xb, g_a, A, perm, tl.tok0, r0, d, c, is_k, col0, width, d_in, d_emb, out, bh, bl, \
+               ahi, alo);                                                                        \
+  break;
+  switch ((c + 15) / 16) {
+    case 1: L3_DW(1)
+    case 2: L3_DW(2)
+    case 3: L3_DW(3)
+    case 4: L3_DW(4)
+    case 5: L3_DW(5)
+    case 6: L3_DW(6)
+    case 7: L3_DW(7)
+    default: L3_DW(8)
   }
-  for (int jb = 0; jb < d; jb += DW_J) {
-    __syncthreads();  // xs written / the previous block's ms read
-    for (int i = tid; i < DW_J * DENSE_TILE_M; i += blockDim.x) {
-      const int jj = i / DENSE_TILE_M, t = i % DENSE_TILE_M;
-      ms[jj * DW_LD + t] =
-          (t < c && jb + jj < d) ? src[(int64_t)(jb + jj) * DENSE_TILE_M + t] : 0.f;
-    }
-    __syncthreads();
-    float acc[4][4] = {};
-    for (int t = 0; t < c; ++t) {
-      const float4 xv = *reinterpret_cast<const float4 *>(xs + t * DW_C + tx * 4);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float m = ms[(ty * 4 + i) * DW_LD + t];
-        acc[i][0] = fmaf(m, xv.x, acc[i][0]);
-        acc[i][1] = fmaf(m, xv.y, acc[i][1]);
-        acc[i][2] = fmaf(m, xv.z, acc[i][2]);
-        acc[i][3] = fmaf(m, xv.w, acc[i][3]);
-      }
-    }
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int j = jb + ty * 4 + i;
-      if (j >= d) continue;
-      float *o = out + (r0 + j) * width + col0 + tx * 4;
-#pragma unroll
-      for (int e = 0; e < 4; ++e) atomicAdd(o + e, acc[i][e]);
-    }
-  }
+#undef L3_DW
 }
 
 }  // namespace
@@ -985,8 +1094,8 @@ extern "C" l3_status l3_backward(const void *x, l3_plan_t p, const void *W_K, co
     launch_tail(k_attn_backward_tail<8>, 8, 3);
     if (e != cudaSuccess) st = cuda_fail(e, "attention backward (tail items)");
   }
-  if (st == L3_OK && n_dt > 0 && !(a16(x) && a16(W_K) && a16(W_V))) {
-    set_error("l3_backward: x, W_K and W_V must be 16-byte aligned");
+  if (st == L3_OK && n_dt > 0 && !(a16(x) && a16(W_K) && a16(W_V) && a16(dx))) {
+    set_error("l3_backward: x, W_K, W_V and dx must be 16-byte aligned");
     st = L3_ERR_INVALID_ARG;
   }
   if (st == L3_OK && n_dt > 0) {
@@ -1008,7 +1117,7 @@ extern "C" l3_status l3_backward(const void *x, l3_plan_t p, const void *W_K, co
           slots, slot_rows, (int)d.d_in, dx);
     }
     e = cudaGetLastError();
-    const size_t dw_smem = (DENSE_TILE_M * DW_C + DW_J * DW_LD) * f;
+    const size_t dw_smem = 4 * 64 * DW_LD * sizeof(__nv_bfloat16);
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(k_attn_backward_dw, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                (int)dw_smem);
