@@ -320,9 +320,15 @@ constexpr int A_MAX_K = 1024;
 // adds (several items of a group share its rows). NT = the item class's
 // token bound (1, 2, 4 or 8): the plan lists items by class.
 static_assert(AT == TAIL_TOKENS, "one chunk per tail item");
-template <int NT>
+template <int WT>
+__device__ __forceinline__ float ldt(const void *p, int64_t i) {
+  if (WT == T_F32) return reinterpret_cast<const float *>(p)[i];
+  return __bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(p)[i]);
+}
+
+template <int NT, int WT>
 __global__ void __launch_bounds__(256)
-    k_attn_backward_tail(const void *x, const void *W_K, const void *W_V, int wtype,
+    k_attn_backward_tail(const void *x, const void *W_K, const void *W_V,
                          const float *__restrict__ g_a, const TailItem *__restrict__ items,
                          int d_in, int d_emb, float *__restrict__ dx, float *__restrict__ dW_K,
                          float *__restrict__ dW_V) {
@@ -342,7 +348,7 @@ __global__ void __launch_bounds__(256)
     __syncthreads();
     for (int i = threadIdx.x; i < NT * d_in; i += blockDim.x) {
       const int t = i / d_in, col = i % d_in;
-      xs[i] = t < nt ? ldx(x, wtype, (int64_t)tok[t] * d_in + col) : 0.f;
+      xs[i] = t < nt ? ldt<WT>(x, (int64_t)tok[t] * d_in + col) : 0.f;
     }
     for (int i = threadIdx.x; i < NT * d_emb; i += blockDim.x) {
       const int t = i / d_emb, col = i % d_emb;
@@ -355,13 +361,15 @@ __global__ void __launch_bounds__(256)
 #pragma unroll
       for (int t = 0; t < NT; ++t) sv[t] = gv[t] = 0.f;
       if (d > 1)
+#pragma unroll 4
         for (int col = lane; col < d_in; col += 32) {
-          const float kv = ldx(W_K, wtype, (r0 + j) * d_in + col);
+          const float kv = ldt<WT>(W_K, (r0 + j) * d_in + col);
 #pragma unroll
           for (int t = 0; t < NT; ++t) sv[t] = fmaf(kv, xs[t * d_in + col], sv[t]);
         }
+#pragma unroll 4
       for (int col = lane; col < d_emb; col += 32) {
-        const float vv = ldx(W_V, wtype, (r0 + j) * d_emb + col);
+        const float vv = ldt<WT>(W_V, (r0 + j) * d_emb + col);
 #pragma unroll
         for (int t = 0; t < NT; ++t) gv[t] = fmaf(vv, gas[t * d_emb + col], gv[t]);
       }
@@ -406,9 +414,10 @@ __global__ void __launch_bounds__(256)
         float acc[NT];
 #pragma unroll
         for (int t = 0; t < NT; ++t) acc[t] = 0.f;
+#pragma unroll 4
         for (int j = 0; j < d; ++j) {
           const int64_t kidx = (r0 + j) * d_in + col;
-          const float kv = ldx(W_K, wtype, kidx);
+          const float kv = ldt<WT>(W_K, kidx);
           float gk = 0.f;
 #pragma unroll
           for (int t = 0; t < NT; ++t) {
@@ -423,6 +432,7 @@ __global__ void __launch_bounds__(256)
     }  // one row: p = 1, no gradient reaches K
     // dV_j (+)= sum_t p[t][j] g_a_t
     for (int col = threadIdx.x; col < d_emb; col += blockDim.x) {
+#pragma unroll 4
       for (int j = 0; j < d; ++j) {
         float gv = 0.f;
 #pragma unroll
@@ -1084,14 +1094,21 @@ extern "C" l3_status l3_backward(const void *x, l3_plan_t p, const void *W_K, co
       const size_t smem = (nt * d.d_in + nt * d.d_emb + 2 * nt * A_MAX_K) * f;
       e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
       if (e != cudaSuccess) return;
-      kernel<<<(unsigned)n, 256, smem, s>>>(x, W_K, W_V, wt, g_a, p->tail_items + i0, (int)d.d_in,
+      kernel<<<(unsigned)n, 256, smem, s>>>(x, W_K, W_V, g_a, p->tail_items + i0, (int)d.d_in,
                                             (int)d.d_emb, dx, dW_K, dW_V);
       e = cudaGetLastError();
     };
-    launch_tail(k_attn_backward_tail<1>, 1, 0);
-    launch_tail(k_attn_backward_tail<2>, 2, 1);
-    launch_tail(k_attn_backward_tail<4>, 4, 2);
-    launch_tail(k_attn_backward_tail<8>, 8, 3);
+    if (wt == T_BF16) {
+      launch_tail(k_attn_backward_tail<1, T_BF16>, 1, 0);
+      launch_tail(k_attn_backward_tail<2, T_BF16>, 2, 1);
+      launch_tail(k_attn_backward_tail<4, T_BF16>, 4, 2);
+      launch_tail(k_attn_backward_tail<8, T_BF16>, 8, 3);
+    } else {
+      launch_tail(k_attn_backward_tail<1, T_F32>, 1, 0);
+      launch_tail(k_attn_backward_tail<2, T_F32>, 2, 1);
+      launch_tail(k_attn_backward_tail<4, T_F32>, 4, 2);
+      launch_tail(k_attn_backward_tail<8, T_F32>, 8, 3);
+    }
     if (e != cudaSuccess) st = cuda_fail(e, "attention backward (tail items)");
   }
   if (st == L3_OK && n_dt > 0 && !(a16(x) && a16(W_K) && a16(W_V) && a16(dx))) {
