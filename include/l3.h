@@ -194,10 +194,11 @@ l3_status l3_forward(const void *x, l3_plan_t plan, const void *W_K, const void 
 
 /*
  * l3_backward — gradients of the layer (kimjy99 review, Method, eq. L³, by
- * the chain rule) for dL/dy. bf16 layers run the dense GEMMs on the tensor
- * cores (bf16 operands, fp32 accumulate; g_z enters g_a as the sum of two
- * bf16 parts) and the rest on CUDA cores in fp32; fp32 layers run all of it
- * on CUDA cores in fp32.
+ * the chain rule) for dL/dy. bf16 layers run the dense GEMMs and the dense
+ * tiles' attention GEMMs on the tensor cores (bf16 operands, fp32 accumulate;
+ * fp32 intermediates such as g_z, g_a, g_s and p enter as the sum of two bf16
+ * parts) and the rest on CUDA cores in fp32; fp32 layers run all of it on
+ * CUDA cores in fp32.
  *
  * Call after l3_forward on the same plan and the same inputs: it reuses the
  * a = V_t^T softmax(K_t x) and h = LayerNorm(W_up a) that forward stored
@@ -217,7 +218,8 @@ l3_status l3_forward(const void *x, l3_plan_t plan, const void *W_K, const void 
  * on the tensor-core path) comes from the library's device block cache
  * (cudaMalloc on a miss) and goes back to it, ordered after the work on
  * `stream`. Enqueued on `stream`; does not synchronize. Errors: L3_ERR_INVALID_ARG (NULL pointer,
- * a staged plan), L3_ERR_UNSUPPORTED (k > 1024, or d_in / d_emb / d_up too
+ * a staged plan, x / W_K / W_V / dx not 16-byte aligned when the plan has
+ * dense tiles), L3_ERR_UNSUPPORTED (k > 1024, or d_in / d_emb / d_up too
  * wide for its shared-memory layout), L3_ERR_OOM, L3_ERR_CUDA.
  */
 l3_status l3_backward(const void *x, l3_plan_t plan, const void *W_K, const void *W_V,

@@ -1,5 +1,5 @@
-// Backward pass of the layer on CUDA cores (fp32 arithmetic), after an
-// l3_forward on the same plan: it reuses the a and h that forward stored.
+// Backward pass of the layer, after an l3_forward on the same plan: it reuses
+// the a and h that forward stored.
 //
 // kimjy99 review, Method, eq. L³, per token with rows K_t, V_t:
 //   s = K_t x, p = softmax(s), a = V_t^T p, z = W_up a,
@@ -12,18 +12,18 @@
 //   dW_up  = g_z^T a                    g_a = g_z W_up
 //   g_p    = V_t g_a, g_s = p (g_p - p.g_p)
 //   dV_t  += p g_a^T, dK_t += g_s x^T, dx += K_t^T g_s
-// bf16 layers run the GEMMs on the tensor cores (the pair kernel of the
-// forward, fp32 output): that kernel reads both operands K-major, so the
-// operands whose K is the token axis or whose rows are the wrong way round
-// are first transposed into bf16 copies (fp16 a and h become bf16 there,
-// since one MMA takes one operand type), and g_z is kept in bf16. fp32
-// layers run them as one strided tiled FFMA kernel (operands read through
-// element strides, so transposed operands need no copies). The attention
-// part runs one CTA per work unit of the plan (a dense tile of up to 128
-// tokens or a tail item of up to 8), eight tokens at a time sharing every row
-// it reads; units of one group add into the group's dW_K / dW_V rows with
-// atomic adds. The dgamma / dbeta column sums are per-CTA partials reduced
-// by a second kernel (deterministic).
+// bf16 layers run the six dense GEMMs on the tcgen05 pair kernel of the
+// forward (fp32 output): it reads both operands K-major, so the operands
+// whose K is the token axis or whose rows are the wrong way round are first
+// transposed into bf16 copies (fp16 a and h become bf16 there, since one MMA
+// takes one operand type); g_z is kept as a hi / lo pair of bf16 numbers.
+// fp32 layers run them as one strided tiled FFMA kernel. The LayerNorm
+// backward walks rows with a thread per column; its dgamma / dbeta column
+// sums are per-CTA partials reduced in a fixed order (deterministic). The
+// attention part runs dense tiles (up to 128 tokens of one group) as
+// register-tiled warp-level MMA kernels over per-tile scratch planes, and
+// tail items (up to 8 tokens) one CTA each on CUDA cores; dW_K / dW_V rows
+// take atomic adds (several units of a group share them).
 #include <cuda_fp16.h>
 
 #include <algorithm>
