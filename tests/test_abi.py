@@ -57,3 +57,8 @@ def test_bad_dims_are_rejected_before_any_launch(lib, field, value, status):
 
 def test_forward_rejects_null_plan(lib):
     assert lib.l3_forward(None, None, None, None, None, None, None, None, None, None) == 1
+
+
+def test_backward_rejects_null_plan(lib):
+    assert lib.l3_backward(*([None] * 17)) == 1
+    assert "plan" in l3.l3_last_error()
