@@ -82,18 +82,34 @@ def attention_flops(ids: np.ndarray, offsets: np.ndarray, w: wl.Workload) -> int
 # DRAM bytes (read + write) per launch of a kernel, from one ncu capture of
 #   ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum,gpu__time_duration.sum
 #       --clock-control none -k regex:<kernel> -s 3 -c 1
-#       python bench.py --workload <w> --steps 1 --warmup 3 --no-e2e --cpu-seconds 0
-# keyed by (kernel, workload, tokens); remove an entry when its kernel changes
+#       python bench.py --workload <w> --only --steps 1 --warmup 3 --no-e2e --cpu-seconds 0
+# keyed by (kernel, workload, tokens), with the digest of the kernel's source
+# files at capture time: a figure is reported only while those sources are
+# unchanged (source_digest), else traffic is null
 TRAFFIC = {
-    ("mix_gemm_tc", "paper_shaped", 65536): 572293888 + 249231360,
+    ("mix_gemm_tc", "paper_shaped", 65536): {"bytes": 572293888 + 249231360,
+                                             "sources": ("gemm_tc.cu", "sm100.cuh"),
+                                             "digest": None, "captured": "2026-11"},
 }
 
 
+def traffic_for(kernel: str, w) -> dict:
+    t = TRAFFIC.get((kernel, w.name, w.n_tokens))
+    if t is None:
+        return {"traffic": None, "traffic_note": "no ncu capture for this kernel and workload"}
+    if t["digest"] is None or source_digest(*t["sources"]) != t["digest"]:
+        return {"traffic": None,
+                "traffic_note": f"ncu capture of {t['captured']} predates the current "
+                                f"{', '.join(t['sources'])}"}
+    return {"traffic": t["bytes"], "traffic_note": f"ncu dram read+write per launch, "
+                                                   f"captured {t['captured']}"}
+
+
 # per-kernel roofline: what each kernel must move or compute per launch
-def kernel_roofline(name: str, work: dict, attn_flops: int, peaks: dict):
+def kernel_roofline(name: str, work: dict, attn_flops: int, peaks: dict, tensor_peak: float):
     if name.startswith("attn"):
         bytes_ = work["k_bytes"] + work["v_bytes"] + work["x_bytes"] + work["a_bytes"]
-        return "hbm", bytes_, "GB/s", peaks["hbm_gbs"]
+        return "hbm", bytes_, "GB/s", peaks["hbm_gbs"], "HBM copy"
     if name.startswith("up"):
         f = work["up_flops"]
     elif name.startswith("mix"):
@@ -101,8 +117,8 @@ def kernel_roofline(name: str, work: dict, attn_flops: int, peaks: dict):
     else:
         return None
     if name.endswith("simt"):
-        return "alu", f, "TFLOP/s", FP32_ALU_PEAK_TFLOPS
-    return "tensor", f, "TFLOP/s", peaks["bf16_tflops_sustained"]
+        return "alu", f, "TFLOP/s", FP32_ALU_PEAK_TFLOPS, "FFMA lanes x max clock"
+    return "tensor", f, "TFLOP/s", tensor_peak, "bf16 tensor"
 
 
 # ----------------------------------------------------------------------------
@@ -404,60 +420,32 @@ def config_of(w, args):
 # GPU arm
 # ----------------------------------------------------------------------------
 
-def main():
-    ap = argparse.ArgumentParser()
-    ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
-    ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="paper_shaped", choices=sorted(wl.WORKLOADS))
-    ap.add_argument("--impl", default="l3", choices=["l3", "reference"])
-    ap.add_argument("--ref-sample", type=int, default=256, help="oracle tokens per reference step")
-    ap.add_argument("--cpu-seconds", type=float, default=10.0,
-                    help="seconds of oracle work for cpu_baseline (0: skip)")
-    ap.add_argument("--tokens", type=int, default=0,
-                    help="tokens per rank (default: the workload's batch size)")
-    ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--lzw", type=int, default=0, metavar="TOKENS",
-                    help="time the LZW allocation on a synthetic corpus of this many tokens")
-    ap.add_argument("--backward", action="store_true",
-                    help="time l3_forward + l3_backward per batch")
-    ap.add_argument("--offload", action="store_true",
-                    help="W_K / W_V in pinned host memory; each step stages the batch's rows")
-    args = ap.parse_args()
+def tensor_peak(peaks: dict, timed_s: float, clocks: dict):
+    """The bf16 tensor peak that applies to this timed region: the burst
+    figure (a kernel timed on its own at full clock) unless the region ran
+    for seconds with the SM clock well below its maximum, as in the
+    sustained measurement."""
+    mhz, mx = clocks.get("sm_mhz"), clocks.get("sm_max_mhz")
+    slowed = mhz is not None and mx and mhz < 0.9 * mx
+    if timed_s >= 2.0 and slowed:
+        return peaks["bf16_tflops_sustained"], "sustained"
+    return peaks["bf16_tflops"], "burst"
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    base = wl.WORKLOADS[args.workload]
-    if args.tokens > 0:
-        base = wl.with_tokens(base, args.tokens)
 
-    if args.impl == "reference":
-        run_reference(args, base, rank)
-        return
-    if args.lzw:
-        if rank == 0:
-            run_lzw(args, base)
-        return
+def source_digest(*names: str) -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for nm in names:
+        with open(os.path.join(ROOT, "static_token_routed_b200", "csrc", nm), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
 
-    dist = None
-    if world > 1:
-        import datetime
-        import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    # each rank: same tables, its own batch
-    w = rank_workload(base, rank)
+
+def measure(w, args, dev, dist, world, rank, steps, warmup, with_e2e=True, with_fwd_only=True,
+            cpu_seconds=0.0):
+    """Time plan + forward of workload `w` (every rank its own batch); returns
+    the fields of the JSON line for it (rank 0) or None."""
     tables, batch = wl.make_tables(w), wl.make_batch(w)
-    if args.offload:
-        run_offload(args, w, tables, batch, dev, dist, world, rank)
-        return
-    if args.backward:
-        run_backward(args, w, tables, batch, dev, dist, world, rank)
-        return
     d = {k: getattr(tables, k).to(dev) for k in ("offsets", "W_K", "W_up", "ln_gamma",
                                                  "ln_beta", "W_mix")}
     # a tied workload passes one device table as keys and values
@@ -490,7 +478,7 @@ def main():
         if dist is not None:
             dist.barrier()
 
-    for _ in range(max(3, args.warmup)):
+    for _ in range(max(3, warmup)):
         step(ids_d, x_d, y_d).destroy()
     plan0 = step(ids_d, x_d, y_d)
     l3.l3_forward_status(plan0)
@@ -502,18 +490,19 @@ def main():
     barrier()
     torch.cuda.synchronize(dev)
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with ClockSampler(local) as clocks:
+    with ClockSampler(dev.index or 0) as clocks:
         ev0.record(stream)
         plan_stream.wait_event(ev0)
-        for _ in range(args.steps):
+        for _ in range(steps):
             step(ids_d, x_d, y_d).destroy()
         ev1.record(stream)
         torch.cuda.synchronize(dev)
     barrier()
     kernels = l3.l3_profile_read()
     l3.l3_profile_enable(False)
-    ms_max = max_over_ranks(ev0.elapsed_time(ev1) / args.steps, dist, dev)
+    ms_max = max_over_ranks(ev0.elapsed_time(ev1) / steps, dist, dev)
     value = job_throughput(w.n_tokens, world, ms_max)
+    clock_summary = clocks.summary()
 
     # ---- end to end through the public API with host buffers ----
     # Each step copies its batch (ids, x) from pinned host memory and reads y
@@ -521,7 +510,7 @@ def main():
     # buffers, so batch i+1 moves over PCIe while batch i computes and batch
     # i-1's y comes back, as in a serving pipeline.
     e2e = None
-    if not args.no_e2e:
+    if with_e2e:
         ids_h = batch.ids.pin_memory()
         x_h = batch.x.pin_memory()
         y_h = [torch.empty(w.n_tokens, w.d_out, dtype=w.torch_dtype).pin_memory()
@@ -564,7 +553,7 @@ def main():
         e0.record(stream)
         for st in (plan_stream, h2d, d2h):
             st.wait_event(e0)
-        for _ in range(args.steps):
+        for _ in range(steps):
             e2e_step().destroy()
         last = torch.cuda.Event()
         last.record(d2h)
@@ -572,80 +561,83 @@ def main():
         e1.record(stream)
         torch.cuda.synchronize(dev)
         barrier()
-        ems = max_over_ranks(e0.elapsed_time(e1) / args.steps, dist, dev)
+        ems = max_over_ranks(e0.elapsed_time(e1) / steps, dist, dev)
         e2e = {"value": job_throughput(w.n_tokens, world, ems), "unit": "tokens/s",
                "h2d_bytes_per_step": int(ids_h.numel() * 4 + x_h.numel() * x_h.element_size()),
                "d2h_bytes_per_step": int(y_h[0].numel() * y_h[0].element_size()),
                "copies": "own streams, double-buffered: overlap the previous and next steps"}
 
     # ---- forward alone: one plan, K forwards (the sort done ahead of time) ----
-    plan_f = l3.l3_plan(ids_d, d["offsets"], dims, stream)
-    for _ in range(3):
-        l3.l3_forward(x_d, plan_f, d["W_K"], d["W_V"], d["W_up"], d["ln_gamma"], d["ln_beta"],
-                      d["W_mix"], y_d, stream)
-    barrier()
-    torch.cuda.synchronize(dev)
-    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    f0.record(stream)
-    for _ in range(args.steps):
-        l3.l3_forward(x_d, plan_f, d["W_K"], d["W_V"], d["W_up"], d["ln_gamma"], d["ln_beta"],
-                      d["W_mix"], y_d, stream)
-    f1.record(stream)
-    torch.cuda.synchronize(dev)
-    l3.l3_forward_status(plan_f)
-    plan_f.destroy()
-    barrier()
-    fwd_ms = max_over_ranks(f0.elapsed_time(f1) / args.steps, dist, dev)
-    fwd_only = {"value": job_throughput(w.n_tokens, world, fwd_ms), "unit": "tokens/s",
-                "ms_per_step": fwd_ms, "note": "l3_forward alone on a plan built ahead of time"}
+    fwd_only = None
+    if with_fwd_only:
+        plan_f = l3.l3_plan(ids_d, d["offsets"], dims, stream)
+        for _ in range(3):
+            l3.l3_forward(x_d, plan_f, d["W_K"], d["W_V"], d["W_up"], d["ln_gamma"],
+                          d["ln_beta"], d["W_mix"], y_d, stream)
+        barrier()
+        torch.cuda.synchronize(dev)
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        for _ in range(steps):
+            l3.l3_forward(x_d, plan_f, d["W_K"], d["W_V"], d["W_up"], d["ln_gamma"],
+                          d["ln_beta"], d["W_mix"], y_d, stream)
+        f1.record(stream)
+        torch.cuda.synchronize(dev)
+        l3.l3_forward_status(plan_f)
+        plan_f.destroy()
+        barrier()
+        fwd_ms = max_over_ranks(f0.elapsed_time(f1) / steps, dist, dev)
+        fwd_only = {"value": job_throughput(w.n_tokens, world, fwd_ms), "unit": "tokens/s",
+                    "ms_per_step": fwd_ms, "note": "l3_forward alone on a plan built ahead of time"}
 
     if rank != 0:
-        if dist is not None:
-            dist.destroy_process_group()
-        return
+        return None
 
     # ---- roofline ----
     peaks = load_peaks()
+    tpeak, regime = tensor_peak(peaks, ms_max * 1e-3 * steps, clock_summary)
     work = algorithmic_work(w, info)
     attn_flops = attention_flops(batch.ids.numpy(), tables.offsets.numpy(), w)
     total_flops = attn_flops + work["up_flops"] + work["mix_flops"]
     if w.dtype == "bf16":
-        t_flop = total_flops / (peaks["bf16_tflops_sustained"] * 1e12)
+        t_flop = total_flops / (tpeak * 1e12)
+        flop_note = f"bf16 {tpeak} TFLOP/s ({regime})"
     else:
         t_flop = total_flops / (FP32_ALU_PEAK_TFLOPS * 1e12)
+        flop_note = f"fp32 FFMA {FP32_ALU_PEAK_TFLOPS:.1f} TFLOP/s (148 SMs x 128 lanes x 2 x 1965 MHz)"
     t_mem = work["bytes"] / (peaks["hbm_gbs"] * 1e9)
     t_roof = max(t_mem, t_flop)
     step_roof = {"t_mem_us": t_mem * 1e6, "t_flop_us": t_flop * 1e6,
                  "bound": "hbm" if t_mem > t_flop else ("tensor" if w.dtype == "bf16" else "alu"),
                  "frac": t_roof / (ms_max * 1e-3), "alg_bytes": work["bytes"],
                  "alg_flops": total_flops,
-                 "peak_note": f"{peaks['source']}: HBM {peaks['hbm_gbs']} GB/s, bf16 "
-                              f"{peaks['bf16_tflops_sustained']} TFLOP/s sustained"}
-    kern = {k: {"launches": n, "total_ms": t, "per_step_ms": t / args.steps}
+                 "peak_note": f"{peaks['source']}: HBM {peaks['hbm_gbs']} GB/s, {flop_note}"}
+    kern = {k: {"launches": n, "total_ms": t, "per_step_ms": t / steps}
             for k, (n, t) in kernels.items()}
     top = max(kernels.items(), key=lambda kv: kv[1][1])[0] if kernels else None
     roof = None
     if top is not None:
-        kr = kernel_roofline(top, work, attn_flops, peaks)
+        kr = kernel_roofline(top, work, attn_flops, peaks, tpeak)
         n_launch, tot_ms = kernels[top]
         if kr is not None:
-            bound, units, unit, peak = kr
+            bound, units, unit, peak, peak_src = kr
             per_launch_s = tot_ms * 1e-3 / n_launch
-            launches_per_step = n_launch / args.steps
+            launches_per_step = n_launch / steps
             per_launch_units = units / launches_per_step
             achieved = per_launch_units / per_launch_s / (1e9 if unit == "GB/s" else 1e12)
             roof = {"kernel": top, "bound": bound, "achieved": achieved, "peak": peak,
                     "unit": unit, "frac": achieved / peak,
-                    "traffic": TRAFFIC.get((top, w.name, w.n_tokens)),
-                    "peak_source": f"{peaks['source']} ({'sustained bf16' if bound == 'tensor' else 'HBM copy' if bound == 'hbm' else 'FFMA lanes x max clock'})"}
+                    "peak_source": f"{peaks['source']} ({peak_src})"}
+            roof.update(traffic_for(top, w))
 
     # ---- CPU baseline: the oracle on a bounded sample ----
     cpu = None
-    if world == 1 and args.cpu_seconds > 0:
-        n_s, dt, cores = time_oracle_bounded(w, tables, batch, args.cpu_seconds)
+    if world == 1 and cpu_seconds > 0:
+        n_s, dt, cores = time_oracle_bounded(w, tables, batch, cpu_seconds,
+                                             chunk=min(256, w.n_tokens))
         cpu = {"value": n_s / dt, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-               "sample": f"{n_s} random tokens of the {w.name} batch in chunks of 256 "
-                         f"(fp64 oracle, {dt:.1f} s)"}
+               "sample": f"{n_s} random tokens of the {w.name} batch in chunks of "
+                         f"{min(256, w.n_tokens)} (fp64 oracle, {dt:.1f} s)"}
         if w.n_tokens <= 4096:
             # small batches: the whole batch on one host thread as well
             import oracle  # test infrastructure: CPU-baseline leg only
@@ -655,18 +647,109 @@ def main():
             cpu["single_thread"] = {"value": w.n_tokens / (time.perf_counter() - t0),
                                     "unit": "tokens/s", "sample": "the whole batch"}
 
-    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "bf16" if w.dtype == "bf16" else "fp32", "data": "synthetic",
-            "config": config_of(w, args), "clocks": clocks.summary(), "e2e": e2e,
+    return {"value": value, "ms_per_step": ms_max, "steps": steps, "warmup": warmup,
+            "dtype": "bf16" if w.dtype == "bf16" else "fp32", "config": config_of(w, args),
+            "clocks": clock_summary, "e2e": e2e,
             "gpu_launches": int(sum(n for n, _ in kernels.values())),
             "roofline": roof, "step_roofline": step_roof, "kernels": kern,
             "cpu_baseline": cpu, "forward_only": fwd_only,
-            "pipelining": "batch i+1's l3_plan on its own stream overlaps batch i's l3_forward",
             "plan": {"groups": info.n_groups, "dense_groups": info.n_dense_groups,
                      "dense_tiles": info.n_dense_tiles, "tail_items": info.n_tail_items,
                      "unique_rows": info.unique_rows}}
+
+
+# the BASELINE workloads besides the headline, each measured in the same run
+OTHER_WORKLOADS = ("tiny_fp32", "small_bf16", "decode", "dense_stress", "uniform")
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="paper_shaped", choices=sorted(wl.WORKLOADS))
+    ap.add_argument("--impl", default="l3", choices=["l3", "reference"])
+    ap.add_argument("--ref-sample", type=int, default=256, help="oracle tokens per reference step")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0,
+                    help="seconds of oracle work for cpu_baseline (0: skip)")
+    ap.add_argument("--tokens", type=int, default=0,
+                    help="tokens per rank (default: the workload's batch size)")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--only", action="store_true",
+                    help="measure the named workload alone (no per_workload lines)")
+    ap.add_argument("--lzw", type=int, default=0, metavar="TOKENS",
+                    help="time the LZW allocation on a synthetic corpus of this many tokens")
+    ap.add_argument("--backward", action="store_true",
+                    help="time l3_forward + l3_backward per batch")
+    ap.add_argument("--offload", action="store_true",
+                    help="W_K / W_V in pinned host memory; each step stages the batch's rows")
+    args = ap.parse_args()
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    base = wl.WORKLOADS[args.workload]
+    if args.tokens > 0:
+        base = wl.with_tokens(base, args.tokens)
+
+    if args.impl == "reference":
+        run_reference(args, base, rank)
+        return
+    if args.lzw:
+        if rank == 0:
+            run_lzw(args, base)
+        return
+
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    # each rank: same tables, its own batch
+    w = rank_workload(base, rank)
+    if args.offload or args.backward:
+        tables, batch = wl.make_tables(w), wl.make_batch(w)
+        (run_offload if args.offload else run_backward)(args, w, tables, batch, dev, dist, world,
+                                                        rank)
+        return
+
+    head = measure(w, args, dev, dist, world, rank, args.steps, args.warmup,
+                   with_e2e=not args.no_e2e, with_fwd_only=True, cpu_seconds=args.cpu_seconds)
+    per_workload = None
+    if world == 1 and not args.only and args.tokens == 0 and args.workload == "paper_shaped":
+        # the other BASELINE workloads at one GPU: shorter CPU samples, the
+        # same steps (each step is shorter than the headline's)
+        torch.cuda.empty_cache()
+        per_workload = {}
+        for name in OTHER_WORKLOADS:
+            r = measure(wl.WORKLOADS[name], args, dev, dist, world, rank, args.steps,
+                        args.warmup, with_e2e=False, with_fwd_only=True,
+                        cpu_seconds=min(3.0, args.cpu_seconds))
+            torch.cuda.empty_cache()
+            per_workload[name] = {k: r[k] for k in ("value", "ms_per_step", "dtype", "config",
+                                                    "clocks", "roofline", "step_roofline",
+                                                    "cpu_baseline", "forward_only", "plan",
+                                                    "gpu_launches", "kernels")}
+    if rank != 0:
+        if dist is not None:
+            dist.destroy_process_group()
+        return
+    line = {"metric": METRIC, "value": head["value"], "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": head["ms_per_step"],
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": head["dtype"], "data": "synthetic", "config": head["config"],
+            "clocks": head["clocks"], "e2e": head["e2e"], "gpu_launches": head["gpu_launches"],
+            "roofline": head["roofline"], "step_roofline": head["step_roofline"],
+            "kernels": head["kernels"], "cpu_baseline": head["cpu_baseline"],
+            "forward_only": head["forward_only"],
+            "pipelining": "batch i+1's l3_plan on its own stream overlaps batch i's l3_forward",
+            "plan": head["plan"]}
+    if per_workload is not None:
+        line["per_workload"] = per_workload
     print(json.dumps(line), flush=True)
     if dist is not None:
         dist.destroy_process_group()

@@ -249,6 +249,8 @@ l3_status l3_backward(const void *x, l3_plan_t plan, const void *W_K, const void
  *   inv_perm    device int32 [N], out: sorted position of original token n
  *   sorted_ids  device int32 [N], out: token ID at sorted position i
  * The outputs equal l3_plan's perm / inv_perm / sorted_ids for the same IDs.
+ * The four buffers must not overlap one another (an overlap is rejected with
+ * L3_ERR_INVALID_ARG: the sort reads its input while other blocks write).
  *
  * Scratch: a file-scope device array of 557,312 bytes (2 x 65536 keys and
  * values plus the digit histogram) that every GPU which loads libl3.so holds

@@ -469,17 +469,27 @@ __global__ void __launch_bounds__(DENSE_THREADS, DenseCfg<SMALL>::MIN_BLOCKS)
         ok = __all_sync(0xffffffffu, mbar_wait(&b->vfull[i], ph, ab));
         if (!ok) break;
         uint4 *vb = reinterpret_cast<uint4 *>(vbuf + i * v_bytes);
+        // slice rows at or past d_t belong to the next token IDs: they are
+        // written as zeros, not converted, so that nothing in another ID's
+        // rows (an Inf, a NaN, a value past fp16's range) reaches this
+        // group's P V_t through a zero of P (static routing: a token's output
+        // depends on its own rows only)
+        const int live_rows = d - (gv % n_vc) * V_ROWS;  // >= 1
         bool bad = false;
         for (int e = lane; e < v_vecs; e += 32) {
+          // 16-byte vector e: 64-column block e / 128, row (e % 128) / 8 of it
+          const bool live = ((e & 127) >> 3) < live_rows;
           uint4 w = vb[e];
           const __nv_bfloat162 *in = reinterpret_cast<const __nv_bfloat162 *>(&w);
-          uint4 o;
-          __half2 *out = reinterpret_cast<__half2 *>(&o);
+          uint4 o = make_uint4(0u, 0u, 0u, 0u);
+          if (live) {
+            __half2 *out = reinterpret_cast<__half2 *>(&o);
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const float2 f = __bfloat1622float2(in[k]);
-            bad |= fabsf(f.x) > 65504.f || fabsf(f.y) > 65504.f;
-            out[k] = __floats2half2_rn(f.x, f.y);
+            for (int k = 0; k < 4; ++k) {
+              const float2 f = __bfloat1622float2(in[k]);
+              bad |= fabsf(f.x) > 65504.f || fabsf(f.y) > 65504.f;
+              out[k] = __floats2half2_rn(f.x, f.y);
+            }
           }
           vb[e] = o;
         }

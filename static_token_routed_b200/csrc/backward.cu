@@ -929,7 +929,23 @@ extern "C" l3_status l3_backward(const void *x, l3_plan_t p, const void *W_K, co
     set_error("l3_backward: k, d_in, d_emb or d_up beyond this kernel's shared-memory layout");
     return L3_ERR_UNSUPPORTED;
   }
+  int cur_dev = -1;
+  L3_CUDA_TRY(cudaGetDevice(&cur_dev));
+  if (cur_dev != p->device) {
+    set_error("l3_backward called on a different device than l3_plan");
+    return L3_ERR_INVALID_ARG;
+  }
+  auto a16 = [](const void *q) { return (reinterpret_cast<uintptr_t>(q) & 15u) == 0; };
+  // checked before anything is enqueued: the tail kernels add into dW_K / dW_V,
+  // so a rejection after them would leave a partial gradient behind
+  if (p->n_dense_tiles > 0 && !(a16(x) && a16(W_K) && a16(W_V) && a16(dx))) {
+    set_error("l3_backward: x, W_K, W_V and dx must be 16-byte aligned");
+    return L3_ERR_INVALID_ARG;
+  }
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  // the plan's a / h buffers and flags are read on this stream from here on:
+  // l3_plan_destroy and l3_forward_status order themselves after it
+  p->stream = s;
   if (N == 0) {
     L3_CUDA_TRY(cudaMemsetAsync(dW_up, 0, d.d_up * d.d_emb * sizeof(float), s));
     L3_CUDA_TRY(cudaMemsetAsync(dgamma, 0, d.d_up * sizeof(float), s));
@@ -945,7 +961,6 @@ extern "C" l3_status l3_backward(const void *x, l3_plan_t p, const void *W_K, co
   const int64_t ln_rows = (N + 4 * n_sms - 1) / (4 * n_sms);
   const int64_t n_ln = (N + ln_rows - 1) / ln_rows;
   const int64_t D = d.d_up + d.d_in;  // columns of W_mix
-  auto a16 = [](const void *q) { return (reinterpret_cast<uintptr_t>(q) & 15u) == 0; };
   // tensor cores for bf16 layers whose forward ran on them (it left the fp16
   // W_up copy in the plan) and whose operands meet the TMA alignment
   const bool tc = p->tc_gemm && a16(x) && a16(W_up) && a16(W_mix) && a16(dy) && a16(dx) &&
@@ -1110,10 +1125,6 @@ extern "C" l3_status l3_backward(const void *x, l3_plan_t p, const void *W_K, co
       launch_tail(k_attn_backward_tail<8, T_F32>, 8, 3);
     }
     if (e != cudaSuccess) st = cuda_fail(e, "attention backward (tail items)");
-  }
-  if (st == L3_OK && n_dt > 0 && !(a16(x) && a16(W_K) && a16(W_V) && a16(dx))) {
-    set_error("l3_backward: x, W_K, W_V and dx must be 16-byte aligned");
-    st = L3_ERR_INVALID_ARG;
   }
   if (st == L3_OK && n_dt > 0) {
     {

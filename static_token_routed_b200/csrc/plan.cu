@@ -634,6 +634,23 @@ extern "C" l3_status l3_sort_tokens_noalloc(const int32_t *token_ids, int64_t n_
     set_error("l3_sort_tokens_noalloc: a pointer is NULL");
     return L3_ERR_INVALID_ARG;
   }
+  {
+    // the scatter of one pass reads token_ids (or the previous pass's keys)
+    // while other CTAs write the outputs, so no two of the four buffers may
+    // share a byte
+    const uintptr_t bytes = (uintptr_t)n_tokens * sizeof(int32_t);
+    const uintptr_t lo[4] = {reinterpret_cast<uintptr_t>(token_ids),
+                             reinterpret_cast<uintptr_t>(perm),
+                             reinterpret_cast<uintptr_t>(inv_perm),
+                             reinterpret_cast<uintptr_t>(sorted_ids)};
+    for (int i = 0; i < 4; ++i)
+      for (int j = i + 1; j < 4; ++j)
+        if (lo[i] < lo[j] + bytes && lo[j] < lo[i] + bytes) {
+          set_error("l3_sort_tokens_noalloc: token_ids, perm, inv_perm and sorted_ids must not "
+                    "overlap");
+          return L3_ERR_INVALID_ARG;
+        }
+  }
   int dev = -1;
   L3_CUDA_TRY(cudaGetDevice(&dev));
   if (dev < 0 || dev >= 64) {

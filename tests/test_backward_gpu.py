@@ -75,3 +75,44 @@ def test_backward_bf16(vocab, rows, n, d_in, d_emb, d_up, d_out):
     w = wl.Workload("case", vocab, int(sum(rows)), max(rows), d_in, d_emb, d_up, d_out, n, "bf16",
                     "zipf", "zipf", 0, 0)
     check(w, t, b, dims, TOL["bf16"])
+
+
+def test_backward_on_its_own_stream_then_replan():
+    """Forward on one stream, backward on another, the plan destroyed right
+    after and a new plan of the same size built and run at once on a third:
+    the new plan may reuse the old one's device block only after the backward
+    that reads it (a, h, the work lists) has finished, so the gradients still
+    match the oracle."""
+    vocab, rows, n, d_in, d_emb, d_up, d_out = 6, (300, 96, 512, 256, 257, 33), 900, 64, 512, 64, 32
+    t, b, dims = small_layer(vocab, rows, n, d_in, d_emb, d_up, d_out, torch.bfloat16, 7)
+    dev = to_device(t, b)
+    g = torch.Generator().manual_seed(3)
+    dy = torch.randn(n, d_out, generator=g).to(torch.bfloat16)
+    dy_d = dy.cuda()
+    s_fwd, s_bwd, s_next = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+    for s in (s_fwd, s_bwd, s_next):
+        s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s_fwd):
+        plan = l3.l3_plan(dev["ids"], dev["offsets"], dims, s_fwd)
+        y = torch.empty(n, d_out, dtype=torch.bfloat16, device="cuda")
+        l3.l3_forward(dev["x"], plan, dev["W_K"], dev["W_V"], dev["W_up"], dev["ln_gamma"],
+                      dev["ln_beta"], dev["W_mix"], y, s_fwd)
+    s_bwd.wait_stream(s_fwd)
+    with torch.cuda.stream(s_bwd):
+        got = l3.l3_backward(dev["x"], plan, dev["W_K"], dev["W_V"], dev["W_up"],
+                             dev["ln_gamma"], dev["ln_beta"], dev["W_mix"], dy_d, s_bwd)
+    plan.destroy()  # no host wait before it: the backward may still be running
+    # other IDs of the same count: same plan size, different sort and groups
+    ids2 = torch.flip(dev["ids"], [0]).contiguous()
+    with torch.cuda.stream(s_next):
+        plan2 = l3.l3_plan(ids2, dev["offsets"], dims, s_next)
+        y2 = torch.empty(n, d_out, dtype=torch.bfloat16, device="cuda")
+        l3.l3_forward(dev["x"], plan2, dev["W_K"], dev["W_V"], dev["W_up"], dev["ln_gamma"],
+                      dev["ln_beta"], dev["W_mix"], y2, s_next)
+    l3.l3_forward_status(plan2)
+    torch.cuda.synchronize()
+    plan2.destroy()
+    want = bwd.backward(b.ids, t.offsets, b.x, t.W_K, t.W_V, t.W_up, t.ln_gamma, t.ln_beta,
+                        t.W_mix, EPS, dy)
+    errs = {k: rel_max_err(got[k].double().cpu().numpy(), want[k]) for k in NAMES}
+    assert all(e <= TOL["bf16"] for e in errs.values()), errs

@@ -169,3 +169,60 @@ def test_dense_attention_shapes(vocab, d_t, n, d_in, d_emb, d_up, d_out):
     want = oracle_y(t, bt)
     err = rel_max_err(y.double().cpu().numpy(), want)
     assert err <= TOL["bf16"], err
+
+
+def test_neighbour_rows_never_reach_a_group():
+    """Static routing (papernotes, 关键设计; kimjy99 review, Method): a token's
+    output depends on its own ID's rows only. The dense attention kernel
+    loads K_t / V_t in 16-row slices, so for d_t not a multiple of 16 a slice
+    also covers the first rows of the next IDs. Here those IDs, absent from
+    the batch, hold NaN, +-Inf and values past fp16's range in both tables:
+    every output must stay finite and within the bar, and the status OK."""
+    vocab = 5
+    rows = (300, 5, 200, 7, 40)   # IDs 1 and 3 are never in the batch
+    off = torch.tensor([0] + list(rows), dtype=torch.int64).cumsum(0).to(torch.int32)
+    v, d_in, d_emb, d_up, d_out = int(off[-1]), 128, 512, 64, 64
+    g = torch.Generator().manual_seed(11)
+    mk = lambda *s: (torch.randn(*s, generator=g) / s[-1] ** 0.5).to(torch.bfloat16)  # noqa: E731
+    W_K, W_V = mk(v, d_in), mk(v, d_emb)
+    poison = torch.tensor([float("nan"), float("inf"), float("-inf"), 1e6, -3e5],
+                          dtype=torch.bfloat16)
+    for t_id in (1, 3):
+        r0, r1 = int(off[t_id]), int(off[t_id + 1])
+        for j, r in enumerate(range(r0, r1)):
+            W_K[r] = poison[j % 5]
+            W_V[r] = poison[(j + 2) % 5]
+    n = 700
+    ids = torch.tensor([(0, 2, 4)[i % 3] for i in range(n)], dtype=torch.int32)
+    ids = ids[torch.randperm(n, generator=g)].contiguous()
+    t = wl.Tables(off, W_K, W_V, mk(d_up, d_emb), torch.ones(d_up, dtype=torch.bfloat16),
+                  torch.zeros(d_up, dtype=torch.bfloat16), mk(d_out, d_up + d_in))
+    b = wl.Batch(ids, mk(n, d_in))
+    dims = l3.make_dims(vocab, v, max(rows), d_in, d_emb, d_up, d_out, torch.bfloat16, EPS)
+    dev = to_device(t, b)
+    plan = l3.l3_plan(dev["ids"], dev["offsets"], dims)
+    assert plan.info().n_dense_tiles > 0   # IDs 0 and 2 run on the dense kernel
+    y = torch.empty(n, d_out, dtype=torch.bfloat16, device="cuda")
+    l3.l3_forward(dev["x"], plan, dev["W_K"], dev["W_V"], dev["W_up"], dev["ln_gamma"],
+                  dev["ln_beta"], dev["W_mix"], y)
+    l3.l3_forward_status(plan)   # raises on L3_ERR_UNSUPPORTED from a range check
+    assert torch.isfinite(y.float()).all()
+    want = oracle_y(t, b)
+    assert rel_max_err(y.double().cpu().numpy(), want) <= TOL["bf16"]
+
+
+def test_paper_shaped_every_token():
+    """The full paper-shaped batch (65536 tokens) in the bench's launch
+    configuration, every output against the oracle: every dense tile and tail
+    class at full size. Where the exactly rounded result itself misses the
+    bar (largest outputs far above the RMS), each output is held to the bar
+    plus half a bf16 ulp of the exact value."""
+    w, t, b = host_workload("paper_shaped")
+    y, plan = run_forward(w, to_device(t, b))
+    want = oracle_y(t, b)
+    got = y.double().cpu().numpy()
+    err = rel_max_err(got, want)
+    if rounding_floor(want) > TOL["bf16"]:
+        assert within_bf16_bar(got, want, TOL["bf16"]), (err, rounding_floor(want))
+    else:
+        assert err <= TOL["bf16"], err
