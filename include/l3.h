@@ -299,6 +299,31 @@ l3_status l3_lzw_allocate(const int32_t *corpus, int64_t n, int64_t vocab, int64
                           int32_t *d_out, int64_t *n_codewords);
 
 /*
+ * l3_lzw_allocate_device — the same allocation as l3_lzw_allocate, with its
+ * walk over the codewords (kimjy99 review, 1. Embedding Allocation: walk
+ * the codewords by decreasing frequency, one row to each one's last token,
+ * repeat until the budget) on the GPU. The corpus scan that builds the
+ * codewords stays on the host: each position extends a suffix found among
+ * the codewords made before it, a sequential dependence.
+ *
+ *   corpus, n, vocab, v, k, n_codewords   as for l3_lzw_allocate; in
+ *                addition vocab < 2^31 - 1 and k < 2^31
+ *   d_out        DEVICE int32 [vocab], out: d_t (4-byte aligned)
+ *   stream       cudaStream_t the device work is enqueued on
+ *
+ * The result equals l3_lzw_allocate's bit for bit. On the device: a stable
+ * radix sort of the codewords by frequency (the walk order), the number P of
+ * complete walks found by binary search over P on T(P) = sum_t min(k, 1 + P
+ * c_t) (c_t: codewords ending with t), then the last, partial walk from each
+ * position's rank among the codewords ending with its token and one prefix
+ * sum. Device scratch (about 9 ints per codeword plus 2 per token) is
+ * cudaMalloc'ed and freed by the call; the call synchronizes `stream` once
+ * at the end. Errors as l3_lzw_allocate, plus L3_ERR_CUDA.
+ */
+l3_status l3_lzw_allocate_device(const int32_t *corpus, int64_t n, int64_t vocab, int64_t v,
+                                 int64_t k, int32_t *d_out, int64_t *n_codewords, void *stream);
+
+/*
  * l3_check_bounded_wait — exercise the give-up path that every kernel's
  * waits share, on the device. The pages have no counterpart: this entry
  * point exists for failure detection, not for the method.

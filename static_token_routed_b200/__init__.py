@@ -25,6 +25,7 @@ from ._binding import (  # noqa: F401
     l3_check_bounded_wait,
     l3_last_error,
     l3_lzw_allocate,
+    l3_lzw_allocate_device,
     l3_plan,
     l3_plan_destroy,
     l3_plan_export,

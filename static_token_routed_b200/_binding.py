@@ -25,7 +25,7 @@ STATUS = {0: "L3_OK", 1: "L3_ERR_INVALID_ARG", 2: "L3_ERR_TOKEN_RANGE", 3: "L3_E
 EXPORTED = ["l3_plan", "l3_plan_info", "l3_plan_export", "l3_forward", "l3_forward_status",
             "l3_plan_destroy", "l3_last_error", "l3_profile_enable", "l3_profile_read",
             "l3_sort_tokens_noalloc", "l3_plan_staged", "l3_stage_rows", "l3_lzw_allocate",
-            "l3_check_bounded_wait", "l3_backward"]
+            "l3_lzw_allocate_device", "l3_check_bounded_wait", "l3_backward"]
 L3_SORT_NOALLOC_MAX_TOKENS = 65536
 
 
@@ -77,6 +77,8 @@ def library() -> ctypes.CDLL:
     lib.l3_check_bounded_wait.argtypes = [p]
     lib.l3_lzw_allocate.restype = i32
     lib.l3_lzw_allocate.argtypes = [p, i64, i64, i64, i64, p, ctypes.POINTER(i64)]
+    lib.l3_lzw_allocate_device.restype = i32
+    lib.l3_lzw_allocate_device.argtypes = [p, i64, i64, i64, i64, p, ctypes.POINTER(i64), p]
     lib.l3_plan_info.restype = i32
     lib.l3_plan_info.argtypes = [p, ctypes.POINTER(PlanInfo)]
     lib.l3_plan_export.restype = i32
@@ -212,6 +214,23 @@ def l3_lzw_allocate(corpus, vocab: int, v: int, k: int) -> tuple[np.ndarray, int
     _check(library().l3_lzw_allocate(c.ctypes.data if c.size else None, int(c.size), int(vocab),
                                      int(v), int(k), d.ctypes.data, ctypes.byref(nw)))
     return d, int(nw.value)
+
+
+def l3_lzw_allocate_device(corpus, vocab: int, v: int, k: int, d_out: torch.Tensor | None = None,
+                           stream=None) -> tuple[torch.Tensor, int]:
+    """The LZW allocation with its codeword walk on the GPU: d_t as a device
+    int32 tensor [vocab] (d_out, or a new one on the current device), and the
+    number of codewords. The corpus is a host array."""
+    c = np.ascontiguousarray(np.asarray(corpus, dtype=np.int32))
+    if d_out is None:
+        d_out = torch.empty(int(vocab), dtype=torch.int32, device="cuda")
+    if d_out.dtype != torch.int32 or not d_out.is_cuda or d_out.numel() != int(vocab):
+        raise ValueError("d_out must be a CUDA int32 tensor of vocab entries")
+    nw = ctypes.c_int64(0)
+    _check(library().l3_lzw_allocate_device(c.ctypes.data if c.size else None, int(c.size),
+                                            int(vocab), int(v), int(k), d_out.data_ptr(),
+                                            ctypes.byref(nw), _stream(stream, d_out.device)))
+    return d_out, int(nw.value)
 
 
 def l3_backward(x, plan: Plan, W_K, W_V, W_up, ln_gamma, ln_beta, W_mix, dy,

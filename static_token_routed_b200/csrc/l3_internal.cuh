@@ -133,6 +133,16 @@ l3_status launch_stage_rows(const l3_plan_s *p, const void *W_K, const void *W_V
 l3_status build_plan(l3_plan_s *p, const int32_t *token_ids, const int32_t *offsets,
                      cudaStream_t s, void *scratch, size_t scratch_bytes);
 size_t plan_scratch_bytes(int64_t n_tokens);
+// stable LSD radix sort of int32 keys in [0, 2^bits) with int32 values (the
+// input index when vals_in is NULL); scratch of radix_sort_scratch_ints(n)
+// ints; outputs must not alias inputs
+size_t radix_sort_scratch_ints(int64_t n);
+l3_status radix_sort_pairs(const int32_t *keys_in, const int32_t *vals_in, int64_t n, int bits,
+                           int32_t *keys_out, int32_t *vals_out, int32_t *scratch,
+                           cudaStream_t s);
+// in-place exclusive scan of data[0..n) by one CTA; data[n] (and *total when
+// given) receives the sum
+l3_status exclusive_scan(int32_t *data, int64_t n, int32_t *total, cudaStream_t s);
 
 // attention, CUDA-core path (attn_tail.cu)
 l3_status launch_attn_tail(const l3_plan_s *p, const void *x, const void *W_K, const void *W_V,

@@ -33,9 +33,17 @@ constexpr int SCAN_ITEMS = 16;
 constexpr int SCAN_CHUNK = SCAN_THREADS * SCAN_ITEMS;
 constexpr int MAX_DT_BUCKETS = 1025;  // d_t <= k <= 1024
 constexpr int N_CLASSES = 4;          // tail items with 1, 2, 3-4 and 5-8 tokens
+constexpr int SMALL_PLAN_MAX_TOKENS = 4096;  // batches planned by one CTA
 
 __host__ __device__ __forceinline__ int token_class(int nt) {
   return nt <= 1 ? 0 : nt == 2 ? 1 : nt <= 4 ? 2 : 3;
+}
+
+// d_t bucket, largest d_t first: d_t = k_cap -> 0 ... d_t = 1 -> k_cap - 1.
+// Clamped so that rows from invalid offsets (reported by the plan, never
+// run) still index inside the bucket arrays.
+__host__ __device__ __forceinline__ int bucket_of(int rows, int k_cap) {
+  return k_cap - max(0, min(rows, k_cap));
 }
 
 // slots of the device info block read back at the end of l3_plan
@@ -288,7 +296,7 @@ __global__ void k_item_counts(const int32_t *__restrict__ group_tok_start,
       // dense tiles are listed largest d_t first (bucket k_cap - d_t): the
       // longest CTAs start first, and the d_t > DENSE_SMALL_ROWS tiles come
       // before the others
-      atomicAdd(&tcount[k_cap - min(rows, k_cap)], nt);
+      atomicAdd(&tcount[bucket_of(rows, k_cap)], nt);
     } else {
       nl = (c + TAIL_TOKENS - 1) / TAIL_TOKENS;
     }
@@ -298,7 +306,7 @@ __global__ void k_item_counts(const int32_t *__restrict__ group_tok_start,
     // bucket class * (k_cap + 1) + (k_cap - d_t), so an ascending scan gives
     // the order
     if (nl > 0) {
-      const int db = k_cap - min(rows, k_cap);
+      const int db = bucket_of(rows, k_cap);
       const int full = c / TAIL_TOKENS, rest = c % TAIL_TOKENS;
       if (full > 0) atomicAdd(&dcount[token_class(TAIL_TOKENS) * (k_cap + 1) + db], full);
       if (rest > 0) atomicAdd(&dcount[token_class(rest) * (k_cap + 1) + db], 1);
@@ -324,7 +332,7 @@ __global__ void k_item_fill(const int32_t *__restrict__ group_tok_start,
   // a group's dense tiles sit side by side (they share K_t, V_t through L2);
   // any order of the groups inside a d_t bucket gives the same results
   if (tiles[g] > 0) {
-    const int32_t pos = atomicAdd(&tcursor[k_cap - min(rows, k_cap)], tiles[g]);
+    const int32_t pos = atomicAdd(&tcursor[bucket_of(rows, k_cap)], tiles[g]);
     for (int32_t j = 0; j < tiles[g]; ++j)
       dense[pos + j] = DenseTile{(int32_t)g, start + j * DENSE_TILE_M};
   }
@@ -338,7 +346,7 @@ __global__ void k_item_fill(const int32_t *__restrict__ group_tok_start,
       it.tok[t] = t < it.nt ? perm[start + j * TAIL_TOKENS + t] : 0;
     it.pad[0] = it.pad[1] = 0;
     // position within its bucket: any order inside a bucket gives the same results
-    const int bucket = token_class(it.nt) * (k_cap + 1) + (k_cap - min(rows, k_cap));
+    const int bucket = token_class(it.nt) * (k_cap + 1) + bucket_of(rows, k_cap);
     const int32_t pos = atomicAdd(&dcursor[bucket], 1);
     tail[pos] = it;
   }
@@ -351,6 +359,240 @@ __global__ void k_class_starts(const int32_t *__restrict__ scanned, int k_cap, i
   // buckets run from d_t = k_cap down to 1 inside a class
   const int small = min(TAIL_SMALL_ROWS, k_cap);
   if (c < N_CLASSES) info[INFO_SPLIT + c] = scanned[c * (k_cap + 1) + (k_cap - small)];
+}
+
+// ---------------------------------------------------------------------------
+// Whole plan in one CTA for small batches (N <= SMALL_PLAN_MAX_TOKENS): the
+// same outputs as the multi-kernel path, built in shared memory by 1024
+// threads, so a decode-sized batch costs one launch instead of a dozen.
+//   1. keys (id << 32 | original index) are bitonic-sorted: unique keys, so
+//      the order is the stable sort by ID;
+//   2. group heads, their exclusive scan (group positions), the group arrays;
+//   3. the exclusive scan of d_t over groups (segment row offsets);
+//   4. dense tiles and tail items counted per bucket, bucket starts scanned,
+//      items written at their bucket's cursor (any order inside a bucket).
+// Info slots are all written here (the offsets check, launched after this
+// kernel, ORs its error bit into the same word).
+// ---------------------------------------------------------------------------
+constexpr int SMALL_THREADS = 1024;
+
+// in-place exclusive scan of data[0..n) by the whole CTA; returns the total
+// (every thread gets it). `tmp` holds SMALL_THREADS / 32 + 1 ints.
+__device__ int block_exclusive_scan(int32_t *data, int n, int32_t *tmp) {
+  const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+  const int per = (n + SMALL_THREADS - 1) / SMALL_THREADS;
+  const int b0 = min(n, tid * per), b1 = min(n, b0 + per);
+  int32_t local = 0;
+  for (int i = b0; i < b1; ++i) local += data[i];
+  int32_t incl = local;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int32_t t = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += t;
+  }
+  if (lane == 31) tmp[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    const int32_t w = lane < SMALL_THREADS / 32 ? tmp[lane] : 0;
+    int32_t wi = w;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int32_t t = __shfl_up_sync(0xffffffffu, wi, o);
+      if (lane >= o) wi += t;
+    }
+    if (lane < SMALL_THREADS / 32) tmp[lane] = wi - w;
+    if (lane == 31) tmp[SMALL_THREADS / 32] = wi;
+  }
+  __syncthreads();
+  int32_t run = tmp[warp] + incl - local;
+  for (int i = b0; i < b1; ++i) {
+    const int32_t v = data[i];
+    data[i] = run;
+    run += v;
+  }
+  const int32_t total = tmp[SMALL_THREADS / 32];
+  __syncthreads();
+  return total;
+}
+
+struct SmallPlanArgs {
+  const int32_t *ids;
+  const int32_t *offsets;
+  int64_t vocab;
+  int n;            // tokens, <= SMALL_PLAN_MAX_TOKENS
+  int np;           // n rounded up to a power of two (>= 2)
+  int k_cap;        // buckets per class: d_t in [1, k_cap]
+  int dense_min_tokens, dense_min_rows, dense_max_rows;
+  bool staged;
+  int32_t *perm, *inv_perm, *sorted_ids;
+  int32_t *group_ids, *group_tok_start, *group_row_start, *group_row_src, *group_rows, *seg_rows;
+  DenseTile *dense;
+  TailItem *tail;
+  int32_t *info;
+};
+
+__global__ void __launch_bounds__(SMALL_THREADS, 1) k_plan_small(SmallPlanArgs A) {
+  extern __shared__ __align__(16) uint8_t smem[];
+  const int tid = threadIdx.x;
+  const int n = A.n, np = A.np, k_cap = A.k_cap;
+  const int n_buckets = N_CLASSES * (k_cap + 1);
+  uint64_t *key = reinterpret_cast<uint64_t *>(smem);                  // [np]
+  int32_t *gpos = reinterpret_cast<int32_t *>(key + np);               // [n + 1]
+  int32_t *gstart = gpos + (n + 1);                                    // [n + 1]
+  int32_t *grows = gstart + (n + 1);                                   // [n + 1]
+  int32_t *dcount = grows + (n + 1);                                   // [n_buckets + 1]
+  int32_t *tcount = dcount + (n_buckets + 1);                          // [k_cap + 2]
+  int32_t *tmp = tcount + (k_cap + 2);                                 // [33]
+  __shared__ int32_t s_err, s_rows_multi, s_max_tokens, s_dense_groups, s_dense_small;
+
+  if (tid == 0) {
+    s_err = 0;
+    s_rows_multi = 0;
+    s_max_tokens = 0;
+    s_dense_groups = 0;
+    s_dense_small = 0;
+  }
+  for (int i = tid; i < n_buckets + 1; i += SMALL_THREADS) dcount[i] = 0;
+  for (int i = tid; i < k_cap + 2; i += SMALL_THREADS) tcount[i] = 0;
+  bool bad = false;
+  for (int i = tid; i < np; i += SMALL_THREADS) {
+    uint64_t k = ~0ull;  // padding sorts last
+    if (i < n) {
+      const int32_t id = A.ids[i];
+      if (id < 0 || id >= A.vocab) bad = true;
+      k = ((uint64_t)(uint32_t)id << 32) | (uint32_t)i;
+    }
+    key[i] = k;
+  }
+  if (bad) atomicOr(&s_err, DEV_ERR_TOKEN_RANGE);
+  __syncthreads();
+
+  // 1. bitonic sort, ascending
+  for (int size = 2; size <= np; size <<= 1) {
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      for (int t = tid; t < np / 2; t += SMALL_THREADS) {
+        const int lo = 2 * t - (t & (stride - 1));  // index whose partner is lo + stride
+        const int hi = lo + stride;
+        const bool up = (lo & size) == 0;
+        const uint64_t a = key[lo], b = key[hi];
+        if ((a > b) == up) {
+          key[lo] = b;
+          key[hi] = a;
+        }
+      }
+      __syncthreads();
+    }
+  }
+
+  // 2. sorted IDs, permutation, group heads
+  for (int i = tid; i < n; i += SMALL_THREADS) {
+    const int32_t id = (int32_t)(key[i] >> 32), src = (int32_t)(uint32_t)key[i];
+    A.sorted_ids[i] = id;
+    A.perm[i] = src;
+    A.inv_perm[src] = i;
+    gpos[i] = (i == 0 || (int32_t)(key[i - 1] >> 32) != id) ? 1 : 0;
+  }
+  __syncthreads();
+  const int G = block_exclusive_scan(gpos, n, tmp);
+  for (int i = tid; i < n; i += SMALL_THREADS) {
+    const int32_t id = (int32_t)(key[i] >> 32);
+    if (i == 0 || (int32_t)(key[i - 1] >> 32) != id) {
+      const int g = gpos[i];
+      const bool ok = id >= 0 && id < A.vocab;
+      const int32_t r0 = ok ? A.offsets[id] : 0;
+      const int32_t rows = ok ? A.offsets[id + 1] - r0 : 0;
+      A.group_ids[g] = id;
+      A.group_tok_start[g] = i;
+      A.group_row_src[g] = r0;
+      A.group_rows[g] = rows;
+      gstart[g] = i;
+      grows[g] = rows;
+    }
+  }
+  if (tid == 0) {
+    A.group_tok_start[G] = n;
+    gstart[G] = n;
+  }
+  __syncthreads();
+
+  // 3. bucket counts of dense tiles and tail items (grows is still d_t here)
+  for (int g = tid; g < G; g += SMALL_THREADS) {
+    const int c = gstart[g + 1] - gstart[g];
+    const int rows = grows[g];
+    const bool dense = A.dense_min_tokens > 0 && c >= A.dense_min_tokens &&
+                       rows >= A.dense_min_rows && rows <= A.dense_max_rows;
+    if (rows > 1) atomicAdd(&s_rows_multi, rows);
+    atomicMax(&s_max_tokens, c);
+    const int db = bucket_of(rows, k_cap);
+    if (dense) {
+      const int nt = (c + DENSE_TILE_M - 1) / DENSE_TILE_M;
+      atomicAdd(&s_dense_groups, 1);
+      if (rows <= DENSE_SMALL_ROWS) atomicAdd(&s_dense_small, nt);
+      atomicAdd(&tcount[db], nt);
+    } else {
+      const int full = c / TAIL_TOKENS, rest = c % TAIL_TOKENS;
+      if (full > 0) atomicAdd(&dcount[token_class(TAIL_TOKENS) * (k_cap + 1) + db], full);
+      if (rest > 0) atomicAdd(&dcount[token_class(rest) * (k_cap + 1) + db], 1);
+    }
+  }
+  __syncthreads();
+  // segment row offsets: exclusive prefix of d_t over groups
+  const int rows_total = block_exclusive_scan(grows, G, tmp);
+  for (int g = tid; g < G; g += SMALL_THREADS) A.seg_rows[g] = grows[g];
+  if (tid == 0) A.seg_rows[G] = rows_total;
+  const int n_tiles = block_exclusive_scan(tcount, k_cap + 1, tmp);
+  const int n_tails = block_exclusive_scan(dcount, n_buckets, tmp);
+  if (tid == 0) {
+    int32_t *info = A.info;
+    info[INFO_ERR] = s_err;
+    info[INFO_G] = G;
+    info[INFO_TILES] = n_tiles;
+    info[INFO_TAILS] = n_tails;
+    info[INFO_ROWS] = rows_total;
+    info[INFO_ROWS_MULTI] = s_rows_multi;
+    info[INFO_DENSE_GROUPS] = s_dense_groups;
+    info[INFO_MAX_TOKENS] = s_max_tokens;
+    const int small = min(TAIL_SMALL_ROWS, k_cap);
+    for (int c = 0; c <= N_CLASSES; ++c)
+      info[INFO_CLS + c] = c < N_CLASSES ? dcount[c * (k_cap + 1)] : n_tails;
+    for (int c = 0; c < N_CLASSES; ++c) info[INFO_SPLIT + c] = dcount[c * (k_cap + 1) + (k_cap - small)];
+    info[INFO_DENSE_SMALL] = s_dense_small;
+  }
+  __syncthreads();
+
+  // 4. the work items at their buckets' cursors
+  for (int g = tid; g < G; g += SMALL_THREADS) {
+    const int start = gstart[g];
+    const int c = gstart[g + 1] - start;
+    const int32_t id = (int32_t)(key[start] >> 32);
+    const bool ok = id >= 0 && id < A.vocab;
+    const int32_t rows = ok ? A.offsets[id + 1] - A.offsets[id] : 0;
+    // a staged plan addresses the group's rows where the staging copy puts them
+    const int32_t r0 = A.staged ? grows[g] : (ok ? A.offsets[id] : 0);
+    A.group_row_start[g] = r0;
+    const bool dense = A.dense_min_tokens > 0 && c >= A.dense_min_tokens &&
+                       rows >= A.dense_min_rows && rows <= A.dense_max_rows;
+    const int db = bucket_of(rows, k_cap);
+    if (dense) {
+      const int nt = (c + DENSE_TILE_M - 1) / DENSE_TILE_M;
+      const int pos = atomicAdd(&tcount[db], nt);
+      for (int j = 0; j < nt; ++j) A.dense[pos + j] = DenseTile{g, start + j * DENSE_TILE_M};
+    } else {
+      const int n_items = (c + TAIL_TOKENS - 1) / TAIL_TOKENS;
+      for (int j = 0; j < n_items; ++j) {
+        TailItem it;
+        it.r0 = r0;
+        it.d = (int16_t)rows;
+        it.nt = (int16_t)min(TAIL_TOKENS, c - j * TAIL_TOKENS);
+#pragma unroll
+        for (int t = 0; t < TAIL_TOKENS; ++t)
+          it.tok[t] = t < it.nt ? (int32_t)(uint32_t)key[start + j * TAIL_TOKENS + t] : 0;
+        it.pad[0] = it.pad[1] = 0;
+        const int pos = atomicAdd(&dcount[token_class(it.nt) * (k_cap + 1) + db], 1);
+        A.tail[pos] = it;
+      }
+    }
+  }
 }
 
 inline int blocks_for(int64_t n, int threads) { return (int)std::max<int64_t>(1, (n + threads - 1) / threads); }
@@ -406,6 +648,18 @@ size_t plan_scratch_bytes(int64_t n) {
   return ints * sizeof(int32_t) + 256;
 }
 
+namespace {
+std::mutex g_small_attr_mu;
+bool g_small_attr[64] = {};
+
+size_t small_plan_smem(int np, int n, int k_cap) {
+  return (size_t)np * 8 + 3 * (size_t)(n + 1) * 4 + (size_t)(N_CLASSES * (k_cap + 1) + 1) * 4 +
+         (size_t)(k_cap + 2) * 4 + 33 * 4 + 16;
+}
+}  // namespace
+
+l3_status finish_plan(l3_plan_s *p, const int32_t *info, int64_t n, cudaStream_t s);
+
 l3_status build_plan(l3_plan_s *p, const int32_t *ids, const int32_t *offsets, cudaStream_t s,
                      void *scratch, size_t scratch_bytes) {
   const int64_t n = p->n_tokens;
@@ -441,6 +695,64 @@ l3_status build_plan(l3_plan_s *p, const int32_t *ids, const int32_t *offsets, c
   if ((size_t)((char *)sp - (char *)scratch) > scratch_bytes) {
     set_error("internal: plan scratch too small");
     return L3_ERR_INVALID_ARG;
+  }
+
+  // groups with enough tokens and rows go to the tensor-core attention kernel
+  int dense_min_tokens = 0, dense_min_rows = 0, dense_max_rows = 0;
+  if (dense_attention_supported(p->dims)) {
+    dense_min_tokens = DENSE_MIN_TOKENS;
+    dense_min_rows = DENSE_MIN_ROWS;
+    dense_max_rows = dense_attention_max_rows();
+  }
+  if (n > 0 && n <= SMALL_PLAN_MAX_TOKENS) {
+    // one CTA builds the whole plan; the offsets check runs after it and ORs
+    // its error bit into the info word the plan kernel wrote
+    SmallPlanArgs A;
+    A.ids = ids;
+    A.offsets = offsets;
+    A.vocab = vocab;
+    A.n = (int)n;
+    A.np = 2;
+    while (A.np < n) A.np <<= 1;
+    A.k_cap = k_cap;
+    A.dense_min_tokens = dense_min_tokens;
+    A.dense_min_rows = dense_min_rows;
+    A.dense_max_rows = dense_max_rows;
+    A.staged = p->staged;
+    A.perm = p->perm;
+    A.inv_perm = p->inv_perm;
+    A.sorted_ids = p->sorted_ids;
+    A.group_ids = p->group_ids;
+    A.group_tok_start = p->group_tok_start;
+    A.group_row_start = p->group_row_start;
+    A.group_row_src = p->group_row_src;
+    A.group_rows = p->group_rows;
+    A.seg_rows = p->seg_rows;
+    A.dense = p->dense_tiles;
+    A.tail = p->tail_items;
+    A.info = info;
+    const size_t smem = small_plan_smem(A.np, (int)n, k_cap);
+    {
+      std::lock_guard<std::mutex> lk(g_small_attr_mu);
+      int dev = p->device & 63;
+      if (!g_small_attr[dev]) {
+        L3_CUDA_TRY(cudaFuncSetAttribute(k_plan_small, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)small_plan_smem(SMALL_PLAN_MAX_TOKENS,
+                                                              SMALL_PLAN_MAX_TOKENS,
+                                                              MAX_DT_BUCKETS - 1)));
+        g_small_attr[dev] = true;
+      }
+    }
+    {
+      LaunchTimer t("plan_small", s);
+      k_plan_small<<<1, SMALL_THREADS, smem, s>>>(A);
+    }
+    {
+      LaunchTimer t("plan_validate", s);
+      k_validate_offsets<<<blocks_for(vocab, 256), 256, 0, s>>>(offsets, vocab, p->dims.v,
+                                                                p->dims.k, info);
+    }
+    return finish_plan(p, info, n, s);
   }
 
   L3_CUDA_TRY(cudaMemsetAsync(info, 0, 64 * sizeof(int32_t), s));
@@ -496,13 +808,6 @@ l3_status build_plan(l3_plan_s *p, const int32_t *ids, const int32_t *offsets, c
                                                       p->group_ids, p->group_tok_start,
                                                       p->group_row_start, p->group_rows, info);
     }
-    // groups with enough tokens and rows go to the tensor-core attention kernel
-    int dense_min_tokens = 0, dense_min_rows = 0, dense_max_rows = 0;
-    if (dense_attention_supported(p->dims)) {
-      dense_min_tokens = DENSE_MIN_TOKENS;
-      dense_min_rows = DENSE_MIN_ROWS;
-      dense_max_rows = dense_attention_max_rows();
-    }
     const int n_buckets = N_CLASSES * (k_cap + 1);
     L3_CUDA_TRY(cudaMemsetAsync(dcount, 0, n_buckets * sizeof(int32_t), s));
     L3_CUDA_TRY(cudaMemsetAsync(tcount, 0, (k_cap + 1) * sizeof(int32_t), s));
@@ -538,6 +843,12 @@ l3_status build_plan(l3_plan_s *p, const int32_t *ids, const int32_t *offsets, c
     L3_CUDA_TRY(cudaMemsetAsync(p->group_tok_start, 0, sizeof(int32_t), s));
     L3_CUDA_TRY(cudaMemsetAsync(p->seg_rows, 0, sizeof(int32_t), s));
   }
+  return finish_plan(p, info, n, s);
+}
+
+// read the info block back (the path's one host round trip) and fill the
+// plan's host-side counts
+l3_status finish_plan(l3_plan_s *p, const int32_t *info, int64_t n, cudaStream_t s) {
   L3_CUDA_TRY(cudaGetLastError());
 
   int32_t host_info[INFO_SLOTS];
@@ -576,6 +887,58 @@ l3_status launch_stage_rows(const l3_plan_s *p, const void *W_K, const void *W_V
       p->group_row_src, p->seg_rows, p->group_rows, reinterpret_cast<const uint4 *>(W_K),
       reinterpret_cast<const uint4 *>(W_V), reinterpret_cast<uint4 *>(K_staged),
       reinterpret_cast<uint4 *>(V_staged), k_vecs, v_vecs);
+  L3_CUDA_TRY(cudaGetLastError());
+  return L3_OK;
+}
+
+// Stable LSD radix sort of int32 keys in [0, 2^bits) (pairs: vals_in, or the
+// input index when NULL), for other parts of the library. Scratch: see
+// radix_sort_scratch_ints. The result lands in keys_out / vals_out; neither
+// may alias the inputs.
+size_t radix_sort_scratch_ints(int64_t n) {
+  const int64_t tiles = std::max<int64_t>(1, (n + SORT_TILE - 1) / SORT_TILE);
+  return 2 * (size_t)n + (size_t)RADIX * tiles + 1;
+}
+
+l3_status radix_sort_pairs(const int32_t *keys_in, const int32_t *vals_in, int64_t n, int bits,
+                           int32_t *keys_out, int32_t *vals_out, int32_t *scratch,
+                           cudaStream_t s) {
+  if (n == 0) return L3_OK;
+  const int64_t n_tiles = std::max<int64_t>(1, (n + SORT_TILE - 1) / SORT_TILE);
+  int32_t *keys_tmp = scratch, *vals_tmp = scratch + n, *hist = scratch + 2 * n;
+  const int passes = std::max(1, (bits + RADIX_BITS - 1) / RADIX_BITS);
+  int32_t *kbuf[2], *vbuf[2];
+  if (passes % 2 == 1) {
+    kbuf[0] = keys_tmp; vbuf[0] = vals_tmp;
+    kbuf[1] = keys_out; vbuf[1] = vals_out;
+  } else {
+    kbuf[0] = keys_out; vbuf[0] = vals_out;
+    kbuf[1] = keys_tmp; vbuf[1] = vals_tmp;
+  }
+  const int32_t *kin = keys_in, *vin = vals_in;
+  for (int pass = 0; pass < passes; ++pass) {
+    const int shift = pass * RADIX_BITS;
+    int32_t *kout = kbuf[(pass + 1) % 2], *vout = vbuf[(pass + 1) % 2];
+    k_radix_hist<<<(int)n_tiles, SORT_THREADS, 0, s>>>(kin, n, shift, hist, (int)n_tiles, 0,
+                                                      nullptr);
+    ScanJobs jobs{};
+    jobs.job[0] = ScanJob{hist, hist, RADIX * n_tiles, nullptr};
+    k_scan_multi<<<1, SCAN_THREADS, 0, s>>>(jobs);
+    k_radix_scatter<<<(int)n_tiles, SORT_THREADS, 0, s>>>(kin, vin, kout, vout, n, shift, hist,
+                                                         (int)n_tiles);
+    kin = kout;
+    vin = vout;
+  }
+  L3_CUDA_TRY(cudaGetLastError());
+  return L3_OK;
+}
+
+// in-place exclusive scan of data[0..n) (data has n + 1 entries; data[n]
+// receives the total, and *total too when given), one CTA
+l3_status exclusive_scan(int32_t *data, int64_t n, int32_t *total, cudaStream_t s) {
+  ScanJobs jobs{};
+  jobs.job[0] = ScanJob{data, data, n, total};
+  k_scan_multi<<<1, SCAN_THREADS, 0, s>>>(jobs);
   L3_CUDA_TRY(cudaGetLastError());
   return L3_OK;
 }
