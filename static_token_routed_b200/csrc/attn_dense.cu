@@ -21,18 +21,20 @@
 //     S accumulates in TMEM over d_in;
 //   - warps 4-11 (two per TMEM lane quarter, so two threads per token row,
 //     each with half of the row's columns) take an exact row max and the
-//     exponentials, and write P as fp16 into shared memory;
-//   - warp 0 then streams V_t in 16-row slices with TMA, warps 4-11 turn each
-//     slice into fp16 in place, and warp 1 accumulates O = P V_t in the TMEM
-//     columns S no longer needs;
+//     exponentials, and write P as bf16 into shared memory;
+//   - warp 0 then streams V_t in 16-row slices with TMA and warp 1
+//     accumulates O = P V_t (bf16 x bf16, the slices as they land) in the
+//     TMEM columns S no longer needs, after zeroing the rows of the last
+//     slice that lie past d_t;
 //   - warps 4-11 scale O by 1 / rowsum and store a[perm[i]] (fp16), i.e. already
 //     in the caller's token order.
 // K_t and V_t are read from HBM by the group's first tile; its other tiles run
 // at the same time and find them in L2.
 // Groups with d_t <= 256 run in a second launch with half the shared memory
 // and TMEM per CTA (two CTAs per SM), O then computed in 256-column passes.
-// P and V_t meet in fp16 (10-bit mantissa): tcgen05 kind::f16 needs one type
-// for both operands, and a bf16 P would cost as much accuracy as a bf16 a.
+// P and V_t meet in bf16 (tcgen05 kind::f16 takes one type for both
+// operands): V_t needs no conversion, and P's largest entry, exp(0) = 1, is
+// exact, so P's rounding weighs only on the smaller weights.
 #include <cuda_fp16.h>
 #include <cudaTypedefs.h>
 
@@ -75,7 +77,7 @@ constexpr int SOFTMAX_THREADS = 256;
 struct DenseBars {
   uint64_t xfull[MAX_STAGES], kfull[MAX_STAGES], sempty[MAX_STAGES];
   uint64_t sfull, pready, ofull;
-  uint64_t vfull[MAX_STAGES], vconv[MAX_STAGES], vempty[MAX_STAGES];
+  uint64_t vfull[MAX_STAGES], vempty[MAX_STAGES];
   uint64_t odrained;  // the epilogue has read this O pass out of TMEM
   uint64_t drain;
   uint32_t tmem_base;
@@ -197,7 +199,6 @@ __global__ void __launch_bounds__(DENSE_THREADS, DenseCfg<SMALL>::MIN_BLOCKS)
     mbar_init(&b->ofull, 1);
     for (int i = 0; i < MAX_STAGES; ++i) {
       mbar_init(&b->vfull[i], 1);
-      mbar_init(&b->vconv[i], 1);
       mbar_init(&b->vempty[i], 1);
     }
     mbar_init(&b->odrained, 8);
@@ -273,8 +274,10 @@ __global__ void __launch_bounds__(DENSE_THREADS, DenseCfg<SMALL>::MIN_BLOCKS)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (elect_one()) {
-      bool ok = true;
+    // lane 0 issues; the whole warp waits for the V slices and zeroes the
+    // padding rows of the last slice of each pass
+    bool ok = true;
+    if (lane == 0) {
       const int n_half = d16 > 256 ? 2 : 1;
       const uint32_t id_s0 = idesc_f16(1, 0, TM, d16 > 256 ? 256 : d16);
       const uint32_t id_s1 = idesc_f16(1, 0, TM, d16 > 256 ? d16 - 256 : 16);
@@ -299,44 +302,64 @@ __global__ void __launch_bounds__(DENSE_THREADS, DenseCfg<SMALL>::MIN_BLOCKS)
         umma_commit(&b->sempty[s]);
       }
       if (ok) umma_commit(&b->sfull);
-      // P V_t into the TMEM columns S used, once the softmax warps have read S
-      if (ok) ok = mbar_wait(&b->pready, 0, ab);
-      const uint32_t pa = smem_u32(pbuf);
-      for (int h = 0; ok && h < n_op; ++h) {
-        // a later pass reuses the TMEM columns once the epilogue has read them
-        if (h > 0 && !mbar_wait(&b->odrained, (h - 1) & 1, ab)) {
+    }
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    // P V_t into the TMEM columns S used, once the softmax warps have read S
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&b->pready, 0, ab));
+    const uint32_t pa = smem_u32(pbuf);
+    for (int h = 0; ok && h < n_op; ++h) {
+      // a later pass reuses the TMEM columns once the epilogue has read them
+      if (h > 0 && !__all_sync(0xffffffffu, mbar_wait(&b->odrained, (h - 1) & 1, ab))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const int o_w = min(o_max, P.d_emb - h * o_max);
+      const int o_half = o_w > 256 ? 2 : 1;
+      const uint32_t id_o0 = idesc_f16(1, 1, TM, o_w > 256 ? 256 : o_w);
+      const uint32_t id_o1 = idesc_f16(1, 1, TM, o_w > 256 ? o_w - 256 : 16);
+      for (int vc = 0; vc < n_vc; ++vc) {
+        const int gv = h * n_vc + vc;
+        const int i = gv % n_v;
+        const uint32_t ph = (gv / n_v) & 1;
+        if (!__all_sync(0xffffffffu, mbar_wait(&b->vfull[i], ph, ab))) {
           ok = false;
           break;
         }
-        tc_fence_after();
-        const int o_w = min(o_max, P.d_emb - h * o_max);
-        const int o_half = o_w > 256 ? 2 : 1;
-        const uint32_t id_o0 = idesc_f16(0, 1, TM, o_w > 256 ? 256 : o_w);
-        const uint32_t id_o1 = idesc_f16(0, 1, TM, o_w > 256 ? o_w - 256 : 16);
-        for (int vc = 0; vc < n_vc; ++vc) {
-          const int gv = h * n_vc + vc;
-          const int i = gv % n_v;
-          const uint32_t ph = (gv / n_v) & 1;
-          if (!mbar_wait(&b->vconv[i], ph, ab)) {
-            ok = false;
-            break;
+        const int live = d - vc * V_ROWS;  // rows of this slice that belong to the group
+        if (live < V_ROWS) {
+          // rows at or past d_t belong to the next token IDs: zero them, so that
+          // nothing in another ID's rows (an Inf, a NaN) reaches this group's
+          // P V_t through a zero of P (static routing: a token's output
+          // depends on its own rows only)
+          const int blocks = o_w / 64, per_block = (V_ROWS - live) * 8;
+          uint4 *vb = reinterpret_cast<uint4 *>(vbuf + i * v_bytes);
+          for (int e = lane; e < blocks * per_block; e += 32) {
+            const int bk = e / per_block, w = e - bk * per_block;
+            vb[bk * (V_BLOCK / 16) + live * 8 + w] = make_uint4(0u, 0u, 0u, 0u);
           }
-          tc_fence_after();
+          fence_proxy_async_smem();
+          __syncwarp();
+        }
+        tc_fence_after();
+        if (lane == 0) {
           const uint32_t va = smem_u32(vbuf + i * v_bytes);
           const int kk = vc * V_ROWS;  // column of P / row of V_t
-          const uint64_t adesc = sdesc_sw128(pa + (kk / 64) * (TM * 128) + (kk % 64) * 2, 16, 1024);
+          const uint64_t adesc =
+              sdesc_sw128(pa + (kk / 64) * (TM * 128) + (kk % 64) * 2, 16, 1024);
           umma_f16(tmem, adesc, sdesc_sw128(va, V_BLOCK, 1024), id_o0, vc != 0);
           if (o_half == 2)
             umma_f16(tmem + 256, adesc, sdesc_sw128(va + 4 * V_BLOCK, V_BLOCK, 1024), id_o1,
                      vc != 0);
           umma_commit(&b->vempty[i]);
         }
-        if (ok) umma_commit(&b->ofull);
+        __syncwarp();
       }
-      if (!ok) {
-        umma_commit(&b->drain);
-        spin_bounded(&b->drain, 0);
-      }
+      if (ok && lane == 0) umma_commit(&b->ofull);
+    }
+    if (!ok && lane == 0) {
+      umma_commit(&b->drain);
+      spin_bounded(&b->drain, 0);
     }
   } else if (warp < 4) {
     // ------------------------------------------------------------ x-row gather
@@ -427,15 +450,15 @@ __global__ void __launch_bounds__(DENSE_THREADS, DenseCfg<SMALL>::MIN_BLOCKS)
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           uint4 o;
-          __half2 *o2 = reinterpret_cast<__half2 *>(&o);
+          __nv_bfloat162 *o2 = reinterpret_cast<__nv_bfloat162 *>(&o);
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const int col = c + j * 8 + 2 * e;
             const float p0 = col < d ? __expf(__uint_as_float(v[j * 8 + 2 * e]) - m) : 0.f;
             const float p1 = col + 1 < d ? __expf(__uint_as_float(v[j * 8 + 2 * e + 1]) - m) : 0.f;
-            const __half2 hp = __floats2half2_rn(p0, p1);
+            const __nv_bfloat162 hp = __floats2bfloat162_rn(p0, p1);
             // the sum uses the rounded values the MMA will see
-            const float2 hf = __half22float2(hp);
+            const float2 hf = __bfloat1622float2(hp);
             sum += hf.x + hf.y;
             o2[e] = hp;
           }
@@ -455,52 +478,8 @@ __global__ void __launch_bounds__(DENSE_THREADS, DenseCfg<SMALL>::MIN_BLOCKS)
     __half *arow = P.a + (r < n_valid ? (int64_t)P.perm[tok0 + r] * P.d_emb : 0);
     for (int h = 0; ok && h < n_op; ++h) {
       const int o_w = min(o_max, P.d_emb - h * o_max);
-      // this pass's V slices: bf16 -> fp16 in place, then hand them to the MMA
-      // warp. Warp sw owns ring slot sw (n_v <= 8) and converts every slice
-      // that lands there, in order, so the slices in the ring are converted
-      // side by side, each by one warp, instead of one after another by all
-      // eight (a chain of waits and proxy fences per slice); a warp never
-      // waits on a slot phase more than one ahead of the one it last saw.
-      const int v_vecs = V_ROWS * o_w / 8;
-      for (int gv = h * n_vc; gv < (h + 1) * n_vc; ++gv) {
-        const int i = gv % n_v;
-        if (i != sw) continue;
-        const uint32_t ph = (gv / n_v) & 1;
-        ok = __all_sync(0xffffffffu, mbar_wait(&b->vfull[i], ph, ab));
-        if (!ok) break;
-        uint4 *vb = reinterpret_cast<uint4 *>(vbuf + i * v_bytes);
-        // slice rows at or past d_t belong to the next token IDs: they are
-        // written as zeros, not converted, so that nothing in another ID's
-        // rows (an Inf, a NaN, a value past fp16's range) reaches this
-        // group's P V_t through a zero of P (static routing: a token's output
-        // depends on its own rows only)
-        const int live_rows = d - (gv % n_vc) * V_ROWS;  // >= 1
-        bool bad = false;
-        for (int e = lane; e < v_vecs; e += 32) {
-          // 16-byte vector e: 64-column block e / 128, row (e % 128) / 8 of it
-          const bool live = ((e & 127) >> 3) < live_rows;
-          uint4 w = vb[e];
-          const __nv_bfloat162 *in = reinterpret_cast<const __nv_bfloat162 *>(&w);
-          uint4 o = make_uint4(0u, 0u, 0u, 0u);
-          if (live) {
-            __half2 *out = reinterpret_cast<__half2 *>(&o);
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              const float2 f = __bfloat1622float2(in[k]);
-              bad |= fabsf(f.x) > 65504.f || fabsf(f.y) > 65504.f;
-              out[k] = __floats2half2_rn(f.x, f.y);
-            }
-          }
-          vb[e] = o;
-        }
-        if (bad) atomicOr(P.err, DEV_ERR_F16_RANGE);
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&b->vconv[i]);
-      }
-
       // epilogue: a = O / rowsum, fp16, to the token's original position
-      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&b->ofull, h & 1, ab));
+      ok = __all_sync(0xffffffffu, mbar_wait(&b->ofull, h & 1, ab));
       if (!ok) break;
       tc_fence_after();
       for (int c = half * 32; c < o_w; c += 64) {

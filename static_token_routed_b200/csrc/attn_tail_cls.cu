@@ -26,10 +26,15 @@
 // singletons) instead run one warp per item, eight items per CTA.
 #include <cuda_fp16.h>
 
+#include <algorithm>
+
 #include "l3_internal.cuh"
+#include "sm100.cuh"
 
 namespace l3 {
 namespace {
+
+using namespace sm100;
 
 constexpr int THREADS = 256;
 constexpr int MAX_DIN = 2048;
@@ -341,6 +346,267 @@ l3_status launch_class(const l3_plan_s *p, Params P, int64_t first, int64_t coun
   return L3_OK;
 }
 
+// ---------------------------------------------------------------------------
+// Short groups (d_t <= TAIL_SMALL_ROWS) of 2..8 tokens: the item's rows are
+// TMA-staged into shared memory once and reused by every token of the item.
+// A persistent CTA per SM; warp 0 issues, several items ahead, one 1-D bulk
+// copy per x row plus one for the item's K_t rows and one for its V_t rows
+// (both contiguous in the concatenated tables) into a ring of slots; warps
+// 1-4 and 5-8 are two groups that take alternate items: logits from shared
+// memory (warp per (token, row) pair, lanes across d_in), an exact softmax
+// per token, a = V_t^T p with threads across d_emb, stored at the tokens'
+// original positions. The slot size follows the largest d_t of the launch's
+// items (its first: the plan lists them largest first).
+// ---------------------------------------------------------------------------
+constexpr int STG_MAX_GROUPS = 4;  // compute groups of four warps
+constexpr int STG_THREADS = 32 + STG_MAX_GROUPS * 128;  // warp 0 copies, the rest compute
+constexpr int STG_MAX_SLOTS = 8;
+constexpr int STG_GROUP_THREADS = 128;
+
+struct StgHdr {
+  int nt, d;
+  int tok[TAIL_TOKENS];
+};
+struct StgShared {
+  uint64_t full[STG_MAX_SLOTS], empty[STG_MAX_SLOTS];
+  StgHdr hdr[STG_MAX_SLOTS];
+  float lg[STG_MAX_GROUPS][TAIL_TOKENS * TAIL_SMALL_ROWS];  // per group: logits, then p
+  int abort_flag;
+};
+
+__device__ __forceinline__ int stg_slot_bytes(int nt, int d, int d_in, int d_emb) {
+  return nt * d_in * 2 + (d > 1 ? d * d_in * 2 : 0) + d * d_emb * 2;
+}
+
+// barrier of one compute group (128 threads), ids 1..STG_MAX_GROUPS, ANDing a
+// flag across the group (every thread gets the AND)
+__device__ __forceinline__ bool group_sync_and(int g, bool ok) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 q, %1, 0;\n\t"
+      "bar.red.and.pred p, %2, %3, q;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(r)
+      : "r"((uint32_t)ok), "r"(1 + g), "n"(STG_GROUP_THREADS)
+      : "memory");
+  return r != 0;
+}
+__device__ __forceinline__ void group_sync(int g) {
+  asm volatile("bar.sync %0, %1;" ::"r"(1 + g), "n"(STG_GROUP_THREADS) : "memory");
+}
+
+template <int TBC>
+__global__ void __launch_bounds__(STG_THREADS, 1)
+    k_attn_tail_staged(Params P, int count, int ring_bytes, int *err) {
+  extern __shared__ __align__(128) uint8_t smem_stg[];
+  StgShared *S = reinterpret_cast<StgShared *>(smem_stg);
+  uint8_t *ring = smem_stg + ((sizeof(StgShared) + 127) & ~size_t(127));
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  // every thread sizes the ring the same way, from the largest d_t
+  const int dmax = P.items[0].d;
+  const int slot_bytes = (stg_slot_bytes(TBC, dmax, P.d_in, P.d_emb) + 127) & ~127;
+  const int raw_slots = min(STG_MAX_SLOTS, ring_bytes / slot_bytes);  // >= 2
+  // item q goes to group q % n_groups and slot q % n_slots; n_slots a multiple
+  // of n_groups, so a slot always serves the same group, which then never
+  // waits on a phase more than one ahead of the slot's
+  const int n_groups = raw_slots >= 4 ? 4 : 2;
+  const int n_slots = raw_slots / n_groups * n_groups;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < STG_MAX_SLOTS; ++i) {
+      mbar_init(&S->full[i], 1);
+      mbar_init(&S->empty[i], 1);
+    }
+    S->abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  const Abort ab{&S->abort_flag, err};
+  const int n_mine = count > (int)blockIdx.x ? (count - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+
+  if (warp == 0) {
+    // ------------------------------------------------ producer: bulk copies
+    bool ok = true;
+    bool armed[STG_MAX_SLOTS];
+    uint32_t armed_par[STG_MAX_SLOTS];
+    for (int i = 0; i < STG_MAX_SLOTS; ++i) armed[i] = false;
+    for (int q0 = 0; ok && q0 < n_mine; q0 += 32) {
+      // the next 32 items' records, one per lane, handed to lane 0 by shuffles
+      uint4 rec[3] = {};
+      if (q0 + lane < n_mine) {
+        const uint4 *src = reinterpret_cast<const uint4 *>(
+            P.items + blockIdx.x + (int64_t)(q0 + lane) * gridDim.x);
+        rec[0] = src[0];
+        rec[1] = src[1];
+        rec[2] = src[2];
+      }
+      const int n_here = min(32, n_mine - q0);
+      for (int u = 0; u < n_here; ++u) {
+        uint32_t w[12];
+#pragma unroll
+        for (int k = 0; k < 3; ++k) {
+          w[4 * k] = __shfl_sync(0xffffffffu, rec[k].x, u);
+          w[4 * k + 1] = __shfl_sync(0xffffffffu, rec[k].y, u);
+          w[4 * k + 2] = __shfl_sync(0xffffffffu, rec[k].z, u);
+          w[4 * k + 3] = __shfl_sync(0xffffffffu, rec[k].w, u);
+        }
+        const int q = q0 + u;
+        const int slot = q % n_slots;
+        const uint32_t par = (uint32_t)(q / n_slots) & 1;
+        if (lane == 0) {
+          // TailItem: r0, (d | nt << 16), tok[8], pad[2]
+          const int64_t r0 = (int32_t)w[0];
+          const int d = (int)(int16_t)(w[1] & 0xffff), nt = (int)(int16_t)(w[1] >> 16);
+          if (!mbar_wait(&S->empty[slot], par ^ 1, ab)) ok = false;
+          if (ok) {
+            StgHdr &h = S->hdr[slot];
+            h.nt = nt;
+            h.d = d;
+            for (int t = 0; t < TAIL_TOKENS; ++t) h.tok[t] = (int)w[2 + t];
+            uint8_t *xs = ring + slot * slot_bytes;
+            uint8_t *ks = xs + nt * P.d_in * 2;
+            uint8_t *vs = ks + (d > 1 ? d * P.d_in * 2 : 0);
+            mbar_arrive_expect_tx(&S->full[slot], (uint32_t)stg_slot_bytes(nt, d, P.d_in, P.d_emb));
+            armed[slot] = true;
+            armed_par[slot] = par;
+            for (int t = 0; t < nt; ++t)
+              bulk_load_1d(xs + t * P.d_in * 2, P.x + (int64_t)(int)w[2 + t] * P.d_in,
+                           (uint32_t)P.d_in * 2, &S->full[slot]);
+            if (d > 1)
+              bulk_load_1d(ks, P.W_K + r0 * P.d_in, (uint32_t)(d * P.d_in * 2), &S->full[slot]);
+            bulk_load_1d(vs, P.W_V + r0 * P.d_emb, (uint32_t)(d * P.d_emb * 2), &S->full[slot]);
+          }
+        }
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) break;
+      }
+    }
+    if (!ok && lane == 0) {
+      // after a give-up: wait (bounded) for the copies still landing
+      for (int i = 0; i < STG_MAX_SLOTS; ++i)
+        if (armed[i]) {
+          const uint32_t a = smem_u32(&S->full[i]);
+          const uint64_t t0 = globaltimer_ns();
+          while (!mbar_try_wait(a, armed_par[i]) && globaltimer_ns() - t0 < WAIT_LIMIT_NS) {
+          }
+        }
+    }
+  } else {
+    // ------------------------------------------------ compute groups
+    const int g = (warp - 1) / 4;
+    if (g >= n_groups) return;  // no barrier below involves this group
+    const int gt = threadIdx.x - 32 - g * STG_GROUP_THREADS;  // 0..127
+    const int gw = gt / 32;
+    float *lg = S->lg[g];
+    const int nvl = P.d_in / 256;  // 16-byte vectors per lane per row (d_in % 256 == 0)
+    const int nc = P.d_emb / 8;    // 16-byte vectors per V / a row
+    for (int q = g; q < n_mine; q += n_groups) {
+      const int slot = q % n_slots;
+      const uint32_t par = (uint32_t)(q / n_slots) & 1;
+      // the group leaves together (a thread that gave up alone would leave the
+      // others waiting at the group's barrier)
+      if (!group_sync_and(g, mbar_wait(&S->full[slot], par, ab))) break;
+      const StgHdr h = S->hdr[slot];
+      const int nt = h.nt, d = h.d;
+      const uint8_t *xs = ring + slot * slot_bytes;
+      const uint8_t *ks = xs + nt * P.d_in * 2;
+      const uint8_t *vs = ks + (d > 1 ? d * P.d_in * 2 : 0);
+      if (d > 1) {
+        // logits: warp gw takes tokens gw, gw + 4; one x vector against all
+        // d_t rows per step (d_t partial sums in registers), then one warp
+        // reduction per row
+        for (int t = gw; t < nt; t += 4) {
+          const uint4 *xr = reinterpret_cast<const uint4 *>(xs + t * P.d_in * 2);
+          float acc[TAIL_SMALL_ROWS];
+#pragma unroll
+          for (int j = 0; j < TAIL_SMALL_ROWS; ++j) acc[j] = 0.f;
+          for (int i = 0; i < nvl; ++i) {
+            float xf[8];
+            cvt8(xr[lane + 32 * i], xf);
+#pragma unroll
+            for (int j = 0; j < TAIL_SMALL_ROWS; ++j) {
+              if (j < d) {
+                float kf[8];
+                cvt8(reinterpret_cast<const uint4 *>(ks + j * P.d_in * 2)[lane + 32 * i], kf);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) acc[j] = fmaf(xf[e], kf[e], acc[j]);
+              }
+            }
+          }
+#pragma unroll
+          for (int j = 0; j < TAIL_SMALL_ROWS; ++j) {
+            if (j < d) {
+              float v = acc[j];
+#pragma unroll
+              for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+              if (lane == 0) lg[t * TAIL_SMALL_ROWS + j] = v;
+            }
+          }
+          __syncwarp();
+          // exact softmax of this token: lane j holds row j
+          const float s = lane < d ? lg[t * TAIL_SMALL_ROWS + lane] : -INFINITY;
+          float m = s;
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+          const float e = lane < d ? expf(s - m) : 0.f;
+          float sum = e;
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+          if (lane < d) lg[t * TAIL_SMALL_ROWS + lane] = e / sum;
+        }
+      } else if (gt < nt) {
+        lg[gt * TAIL_SMALL_ROWS] = 1.0f;  // one row: p = 1
+      }
+      group_sync(g);
+      // a = V_t^T p: thread per (token, 16-byte column vector)
+      const uint4 *vr = reinterpret_cast<const uint4 *>(vs);
+      for (int wi = gt; wi < nt * nc; wi += STG_GROUP_THREADS) {
+        const int t = wi / nc, c = wi - t * nc;
+        float acc[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+        for (int j = 0; j < d; ++j) {
+          const float pj = lg[t * TAIL_SMALL_ROWS + j];
+          float vf[8];
+          cvt8(vr[j * nc + c], vf);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) acc[e] = fmaf(pj, vf[e], acc[e]);
+        }
+        uint4 o;
+        __half2 *o2 = reinterpret_cast<__half2 *>(&o);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) o2[e] = __floats2half2_rn(acc[2 * e], acc[2 * e + 1]);
+        reinterpret_cast<uint4 *>(P.a + (int64_t)h.tok[t] * P.d_emb)[c] = o;
+      }
+      // every thread of the group is done with the slot and with lg
+      group_sync(g);
+      if (gt == 0) mbar_arrive(&S->empty[slot]);
+    }
+  }
+}
+
+template <int TBC>
+l3_status launch_staged(const l3_plan_s *p, Params P, int64_t first, int64_t count,
+                        cudaStream_t s) {
+  if (count <= 0) return L3_OK;
+  P.items = p->tail_items + first;
+  const size_t head = (sizeof(StgShared) + 127) & ~size_t(127);
+  const size_t smem = 227 * 1024;
+  static bool configured[64] = {};
+  if (!configured[p->device & 63]) {
+    L3_CUDA_TRY(cudaFuncSetAttribute(k_attn_tail_staged<TBC>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+    configured[p->device & 63] = true;
+  }
+  int n_sms = 148;
+  cudaDeviceGetAttribute(&n_sms, cudaDevAttrMultiProcessorCount, p->device);
+  const int grid = (int)std::min<int64_t>(count, n_sms);
+  k_attn_tail_staged<TBC><<<grid, STG_THREADS, smem, s>>>(P, (int)count, (int)(smem - head),
+                                                         p->dev_flags + 1);
+  L3_CUDA_TRY(cudaGetLastError());
+  return L3_OK;
+}
+
 }  // namespace
 
 bool tail_cls_supported(const l3_dims_t &d) {
@@ -378,9 +644,19 @@ l3_status launch_attn_tail_cls(const l3_plan_s *p, const void *x, const void *W_
           st = part == 0 ? launch_class<1>(p, P, first, last - first, s)
                          : launch_small<1>(p, P, first, last - first, s);
           break;
-        case 1: st = launch_class<2>(p, P, first, last - first, s); break;
-        case 2: st = launch_class<4>(p, P, first, last - first, s); break;
-        default: st = launch_class<8>(p, P, first, last - first, s); break;
+        // short groups of several tokens: rows staged in shared memory once
+        case 1:
+          st = part == 0 ? launch_class<2>(p, P, first, last - first, s)
+                         : launch_staged<2>(p, P, first, last - first, s);
+          break;
+        case 2:
+          st = part == 0 ? launch_class<4>(p, P, first, last - first, s)
+                         : launch_staged<4>(p, P, first, last - first, s);
+          break;
+        default:
+          st = part == 0 ? launch_class<8>(p, P, first, last - first, s)
+                         : launch_staged<8>(p, P, first, last - first, s);
+          break;
       }
     }
   }

@@ -226,3 +226,36 @@ def test_paper_shaped_every_token():
         assert within_bf16_bar(got, want, TOL["bf16"]), (err, rounding_floor(want))
     else:
         assert err <= TOL["bf16"], err
+
+
+@pytest.mark.parametrize("vocab,n,d_in,d_emb,dmax,seed", [
+    (500, 4000, 256, 64, 16, 1),     # 2-8 token items, d_t 1..16: the staged tail kernel
+    (300, 2500, 1024, 256, 4, 2),    # the uniform workload's shape of items
+    (200, 1700, 2048, 512, 16, 3),   # paper-shaped widths: largest staged slots
+    (64, 3000, 512, 128, 2, 4),      # d_t 1 and 2 only
+])
+def test_short_groups_all_tokens(vocab, n, d_in, d_emb, dmax, seed):
+    """Groups of 2-8 tokens with at most 16 rows, every token against the
+    oracle (the bf16 tail path that stages each item's rows in shared
+    memory), with ragged token counts per group."""
+    rng = np.random.default_rng(seed)
+    d = rng.integers(1, dmax + 1, size=vocab)
+    off = torch.from_numpy(np.concatenate([[0], np.cumsum(d)]).astype(np.int32))
+    v, d_up, d_out = int(off[-1]), 128, 64
+    g = torch.Generator().manual_seed(seed)
+    ids = torch.randint(0, vocab, (n,), generator=g, dtype=torch.int32)
+    mk = lambda *s: (torch.randn(*s, generator=g) / s[-1] ** 0.5).to(torch.bfloat16)  # noqa: E731
+    t = wl.Tables(off, mk(v, d_in) * 3, mk(v, d_emb), mk(d_up, d_emb),
+                  (1 + 0.1 * torch.randn(d_up, generator=g)).to(torch.bfloat16),
+                  (0.1 * torch.randn(d_up, generator=g)).to(torch.bfloat16), mk(d_out, d_up + d_in))
+    b = wl.Batch(ids, mk(n, d_in))
+    dims = l3.make_dims(vocab, v, int(d.max()), d_in, d_emb, d_up, d_out, torch.bfloat16, EPS)
+    dev = to_device(t, b)
+    plan = l3.l3_plan(dev["ids"], dev["offsets"], dims)
+    y = torch.empty(n, d_out, dtype=torch.bfloat16, device="cuda")
+    l3.l3_forward(dev["x"], plan, dev["W_K"], dev["W_V"], dev["W_up"], dev["ln_gamma"],
+                  dev["ln_beta"], dev["W_mix"], y)
+    l3.l3_forward_status(plan)
+    want = oracle_y(t, b)
+    err = rel_max_err(y.double().cpu().numpy(), want)
+    assert err <= TOL["bf16"], err
