@@ -585,6 +585,14 @@ __global__ void __launch_bounds__(STG_THREADS, 1)
   }
 }
 
+// the staged kernel keeps several items in flight per SM only when an item
+// of the class with TAIL_SMALL_ROWS rows takes at most a quarter of the ring;
+// with wider rows (d_in 2048) a CTA per item keeps more bytes in flight
+bool staged_pays(const Params &P, int tbc) {
+  const size_t slot = (size_t)tbc * P.d_in * 2 + (size_t)TAIL_SMALL_ROWS * (P.d_in + P.d_emb) * 2;
+  return slot * 4 <= 227 * 1024 - ((sizeof(StgShared) + 127) & ~size_t(127));
+}
+
 template <int TBC>
 l3_status launch_staged(const l3_plan_s *p, Params P, int64_t first, int64_t count,
                         cudaStream_t s) {
@@ -644,18 +652,20 @@ l3_status launch_attn_tail_cls(const l3_plan_s *p, const void *x, const void *W_
           st = part == 0 ? launch_class<1>(p, P, first, last - first, s)
                          : launch_small<1>(p, P, first, last - first, s);
           break;
-        // short groups of several tokens: rows staged in shared memory once
+        // short groups of several tokens: rows staged in shared memory once,
+        // where at least four items fit the staging ring at a time (narrow
+        // layers); otherwise a CTA per item
         case 1:
-          st = part == 0 ? launch_class<2>(p, P, first, last - first, s)
-                         : launch_staged<2>(p, P, first, last - first, s);
+          st = part == 0 || !staged_pays(P, 2) ? launch_class<2>(p, P, first, last - first, s)
+                                               : launch_staged<2>(p, P, first, last - first, s);
           break;
         case 2:
-          st = part == 0 ? launch_class<4>(p, P, first, last - first, s)
-                         : launch_staged<4>(p, P, first, last - first, s);
+          st = part == 0 || !staged_pays(P, 4) ? launch_class<4>(p, P, first, last - first, s)
+                                               : launch_staged<4>(p, P, first, last - first, s);
           break;
         default:
-          st = part == 0 ? launch_class<8>(p, P, first, last - first, s)
-                         : launch_staged<8>(p, P, first, last - first, s);
+          st = part == 0 || !staged_pays(P, 8) ? launch_class<8>(p, P, first, last - first, s)
+                                               : launch_staged<8>(p, P, first, last - first, s);
           break;
       }
     }

@@ -259,3 +259,40 @@ def test_short_groups_all_tokens(vocab, n, d_in, d_emb, dmax, seed):
     want = oracle_y(t, b)
     err = rel_max_err(y.double().cpu().numpy(), want)
     assert err <= TOL["bf16"], err
+
+
+@pytest.mark.parametrize("d_in,d_emb,rows,seed", [
+    (2048, 512, (17, 33, 512, 100, 255, 31, 257, 64, 480, 18), 5),   # paper widths
+    (1024, 256, (20, 512, 47, 129, 300, 16, 17, 250), 6),
+    (256, 64, (511, 23, 65, 200), 7),
+])
+def test_long_groups_few_tokens_all_tokens(d_in, d_emb, rows, seed):
+    """Groups of 1-4 tokens (under the dense threshold) with 17..512 rows: the
+    tail path that streams K_t / V_t through shared memory in 16-row chunks
+    with a softmax taken across the chunks (d_t = 17: a one-row last chunk;
+    d_t = 512: 32 chunks). Every token against the oracle."""
+    vocab = len(rows)
+    g = torch.Generator().manual_seed(seed)
+    off = torch.tensor([0] + list(rows), dtype=torch.int64).cumsum(0).to(torch.int32)
+    v, d_up, d_out = int(off[-1]), 128, 64
+    # 1-4 tokens per ID, shuffled
+    counts = [1 + (i * 7 + seed) % 4 for i in range(vocab)]
+    ids = torch.tensor([i for i, c in enumerate(counts) for _ in range(c)], dtype=torch.int32)
+    ids = ids[torch.randperm(len(ids), generator=g)].contiguous()
+    n = len(ids)
+    mk = lambda *s: (torch.randn(*s, generator=g) / s[-1] ** 0.5).to(torch.bfloat16)  # noqa: E731
+    t = wl.Tables(off, mk(v, d_in) * 3, mk(v, d_emb), mk(d_up, d_emb),
+                  (1 + 0.1 * torch.randn(d_up, generator=g)).to(torch.bfloat16),
+                  (0.1 * torch.randn(d_up, generator=g)).to(torch.bfloat16), mk(d_out, d_up + d_in))
+    b = wl.Batch(ids, mk(n, d_in))
+    dims = l3.make_dims(vocab, v, max(rows), d_in, d_emb, d_up, d_out, torch.bfloat16, EPS)
+    dev = to_device(t, b)
+    plan = l3.l3_plan(dev["ids"], dev["offsets"], dims)
+    assert plan.info().n_dense_tiles == 0
+    y = torch.empty(n, d_out, dtype=torch.bfloat16, device="cuda")
+    l3.l3_forward(dev["x"], plan, dev["W_K"], dev["W_V"], dev["W_up"], dev["ln_gamma"],
+                  dev["ln_beta"], dev["W_mix"], y)
+    l3.l3_forward_status(plan)
+    want = oracle_y(t, b)
+    err = rel_max_err(y.double().cpu().numpy(), want)
+    assert err <= TOL["bf16"], err
