@@ -116,3 +116,57 @@ def test_backward_on_its_own_stream_then_replan():
                         t.W_mix, EPS, dy)
     errs = {k: rel_max_err(got[k].double().cpu().numpy(), want[k]) for k in NAMES}
     assert all(e <= TOL["bf16"] for e in errs.values()), errs
+
+
+def test_backward_paper_shaped_full_batch_sampled_dy():
+    """The full paper-shaped batch (65,536 tokens: every dense tile, tail class
+    and launch the bench's backward runs), with dL/dy nonzero on 384 sampled
+    tokens only. The backward is linear in dL/dy and a token with zero dL/dy
+    contributes nothing, so every gradient equals the oracle's backward over
+    the sampled tokens alone: dx on those tokens (exactly zero elsewhere),
+    dW_K / dW_V on every row, dW_up, dgamma, dbeta and dW_mix in full."""
+    from l3_cases import host_workload, sample_tokens
+    w, t, b = host_workload("paper_shaped")
+    dev = to_device(t, b)
+    dims = l3.make_dims(w.vocab, w.v, w.k, w.d_in, w.d_emb, w.d_up, w.d_out, w.torch_dtype, EPS)
+    plan = l3.l3_plan(dev["ids"], dev["offsets"], dims)
+    y = torch.empty(w.n_tokens, w.d_out, dtype=w.torch_dtype, device="cuda")
+    l3.l3_forward(dev["x"], plan, dev["W_K"], dev["W_V"], dev["W_up"], dev["ln_gamma"],
+                  dev["ln_beta"], dev["W_mix"], y)
+    sel = sample_tokens(b.ids.numpy(), t.offsets.numpy(), 384, seed=3)
+    g = torch.Generator().manual_seed(4)
+    dy = torch.zeros(w.n_tokens, w.d_out, dtype=w.torch_dtype)
+    dy[torch.from_numpy(sel)] = torch.randn(len(sel), w.d_out, generator=g).to(w.torch_dtype)
+    got = l3.l3_backward(dev["x"], plan, dev["W_K"], dev["W_V"], dev["W_up"], dev["ln_gamma"],
+                         dev["ln_beta"], dev["W_mix"], dy.cuda())
+    l3.l3_forward_status(plan)
+    plan.destroy()
+    # the oracle on a compact table holding only the sampled tokens' IDs (the
+    # full tables in fp64 would take tens of GB of host memory)
+    ids_s = np.unique(b.ids.numpy()[sel])
+    off = t.offsets.numpy().astype(np.int64)
+    rows = np.concatenate([np.arange(off[i], off[i + 1]) for i in ids_s])
+    compact = {int(i): j for j, i in enumerate(ids_s)}
+    d_s = off[ids_s + 1] - off[ids_s]
+    off_c = torch.from_numpy(np.concatenate([[0], np.cumsum(d_s)]).astype(np.int32))
+    ids_c = torch.tensor([compact[int(i)] for i in b.ids.numpy()[sel]], dtype=torch.int32)
+    rows_h = torch.from_numpy(rows)
+    want = bwd.backward(ids_c, off_c, b.x[sel], t.W_K[rows_h], t.W_V[rows_h], t.W_up, t.ln_gamma,
+                        t.ln_beta, t.W_mix, EPS, dy[torch.from_numpy(sel)])
+    dx = got["x"]
+    mask = torch.ones(w.n_tokens, dtype=torch.bool)
+    mask[torch.from_numpy(sel)] = False
+    assert torch.count_nonzero(dx[mask.cuda()]) == 0
+    errs = {"x": rel_max_err(dx[torch.from_numpy(sel).cuda()].double().cpu().numpy(), want["x"])}
+    for k in ("W_up", "ln_gamma", "ln_beta", "W_mix"):
+        errs[k] = rel_max_err(got[k].double().cpu().numpy(), want[k])
+    # dW_K / dW_V: the rows of the sampled tokens' IDs carry the gradient; every
+    # other row must stay exactly zero
+    for k in ("W_K", "W_V"):
+        gk = got[k]
+        rows_t = torch.from_numpy(rows).cuda()
+        errs[k] = rel_max_err(gk[rows_t].double().cpu().numpy(), want[k])
+        other = torch.ones(gk.shape[0], dtype=torch.bool, device="cuda")
+        other[rows_t] = False
+        assert torch.count_nonzero(gk[other]) == 0, k
+    assert all(e <= TOL["bf16"] for e in errs.values()), errs
