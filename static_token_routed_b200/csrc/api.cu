@@ -42,28 +42,33 @@ cudaEvent_t take_event() {
 }
 
 
-// Per-device helper stream and events that let the two attention kernels
-// (CUDA-core tail, tensor-core dense) run side by side: they write disjoint
-// rows of a, and the tail's small CTAs fit next to a dense CTA on an SM.
+// Per-device helper streams and events that let the attention kernels run
+// side by side: the tensor-core dense kernel on the caller's stream, the
+// CUDA-core tail classes spread over the helper streams. They write disjoint
+// rows of a, and the tails' small CTAs fit next to a dense CTA on an SM.
+constexpr int N_AUX = 3;
 struct Aux {
   std::mutex mu;
-  cudaStream_t stream = nullptr;
-  cudaEvent_t fork = nullptr, join = nullptr;
+  cudaStream_t stream[N_AUX] = {};
+  cudaEvent_t fork = nullptr, join[N_AUX] = {};
 };
 Aux g_aux[64];
 
 l3_status aux_for(int device, Aux **out) {
   Aux &a = g_aux[device & 63];
-  if (!a.stream) {
+  std::lock_guard<std::mutex> lk(a.mu);
+  if (!a.stream[0]) {
     // highest priority: the block scheduler hands freed SM slots to the tail
     // attention's short CTAs before the next dense CTA, so the two overlap
     // instead of the tails waiting behind the dense launch (1.84 -> 1.69 ms per
     // paper_shaped batch)
     int lowest = 0, highest = 0;
     L3_CUDA_TRY(cudaDeviceGetStreamPriorityRange(&lowest, &highest));
-    L3_CUDA_TRY(cudaStreamCreateWithPriority(&a.stream, cudaStreamNonBlocking, highest));
+    for (int i = 0; i < N_AUX; ++i) {
+      L3_CUDA_TRY(cudaStreamCreateWithPriority(&a.stream[i], cudaStreamNonBlocking, highest));
+      L3_CUDA_TRY(cudaEventCreateWithFlags(&a.join[i], cudaEventDisableTiming));
+    }
     L3_CUDA_TRY(cudaEventCreateWithFlags(&a.fork, cudaEventDisableTiming));
-    L3_CUDA_TRY(cudaEventCreateWithFlags(&a.join, cudaEventDisableTiming));
   }
   *out = &a;
   return L3_OK;
@@ -436,28 +441,35 @@ l3_status l3_forward(const void *x, l3_plan_t p, const void *W_K, const void *W_
   const bool has_big = p->n_dense_tiles > p->n_dense_small;
   const bool has_small = p->n_dense_small > 0;
   const bool has_tail = p->n_tail_items > 0;
-  auto tail = [&](cudaStream_t q) {
-    return tail_cls_supported(p->dims) ? launch_attn_tail_cls(p, x, W_K, W_V, q)
-                                       : launch_attn_tail(p, x, W_K, W_V, q);
-  };
-  if ((has_big || has_small) && has_tail) {
+  if (has_tail && tail_cls_supported(p->dims)) {
     // fork: dense attention (both configurations, in turn) on the caller's
-    // stream; the tail attention, then the fp16 weight copies, on the
-    // high-priority helper stream, whose short CTAs fill the SM slots the long
-    // dense CTAs leave; join before W_up. The launches write disjoint rows of a.
+    // stream; the tail classes over the high-priority helper streams, whose
+    // short CTAs fill the SM slots the long dense CTAs leave, and the fp16
+    // weight copies after them; join before W_up. The launches write disjoint
+    // rows of a.
     Aux *aux = nullptr;
     if ((st = aux_for(p->device, &aux)) != L3_OK) return st;
     std::lock_guard<std::mutex> lk(aux->mu);
     L3_CUDA_TRY(cudaEventRecord(aux->fork, s));
-    L3_CUDA_TRY(cudaStreamWaitEvent(aux->stream, aux->fork, 0));
+    for (int i = 0; i < N_AUX; ++i) L3_CUDA_TRY(cudaStreamWaitEvent(aux->stream[i], aux->fork, 0));
     if (st == L3_OK) st = launch_attn_dense(p, x, W_K, W_V, false, s);
     if (st == L3_OK) st = launch_attn_dense(p, x, W_K, W_V, true, s);
-    if (st == L3_OK) st = tail(aux->stream);
-    if (st == L3_OK && p->tc_gemm) st = launch_weights_f16(p, W_up, W_mix, aux->stream);
-    L3_CUDA_TRY(cudaEventRecord(aux->join, aux->stream));
-    L3_CUDA_TRY(cudaStreamWaitEvent(s, aux->join, 0));
+    // next to the big dense configuration (one CTA per SM, streaming K_t)
+    // the tails stay on one helper stream: spread over three they take SMs
+    // and bandwidth from it (paper_shaped: 1.64 -> 1.72 ms per batch); with
+    // no such launch they spread over all three (small_bf16: 0.41 -> 0.34 ms)
+    if (st == L3_OK) st = launch_attn_tail_cls(p, x, W_K, W_V, aux->stream, has_big ? 1 : N_AUX);
+    if (st == L3_OK && p->tc_gemm) st = launch_weights_f16(p, W_up, W_mix, aux->stream[0]);
+    for (int i = 0; i < N_AUX; ++i) {
+      L3_CUDA_TRY(cudaEventRecord(aux->join[i], aux->stream[i]));
+      L3_CUDA_TRY(cudaStreamWaitEvent(s, aux->join[i], 0));
+    }
+  } else if (has_tail) {
+    st = launch_attn_tail(p, x, W_K, W_V, s);
+    if (st == L3_OK) st = launch_attn_dense(p, x, W_K, W_V, false, s);
+    if (st == L3_OK) st = launch_attn_dense(p, x, W_K, W_V, true, s);
+    if (st == L3_OK && p->tc_gemm) st = launch_weights_f16(p, W_up, W_mix, s);
   } else {
-    st = tail(s);
     if (st == L3_OK) st = launch_attn_dense(p, x, W_K, W_V, false, s);
     if (st == L3_OK) st = launch_attn_dense(p, x, W_K, W_V, true, s);
     if (st == L3_OK && p->tc_gemm) st = launch_weights_f16(p, W_up, W_mix, s);

@@ -625,7 +625,7 @@ bool tail_cls_supported(const l3_dims_t &d) {
 }
 
 l3_status launch_attn_tail_cls(const l3_plan_s *p, const void *x, const void *W_K,
-                               const void *W_V, cudaStream_t s) {
+                               const void *W_V, const cudaStream_t *streams, int n_streams) {
   if (p->n_tail_items == 0) return L3_OK;
   Params P;
   P.x = reinterpret_cast<const __nv_bfloat16 *>(x);
@@ -639,12 +639,31 @@ l3_status launch_attn_tail_cls(const l3_plan_s *p, const void *x, const void *W_
   static const char *names[8] = {"attn_tail_t1_big", "attn_tail_t1_small", "attn_tail_t2_big",
                                  "attn_tail_t2_small", "attn_tail_t4_big", "attn_tail_t4_small",
                                  "attn_tail_t8_big", "attn_tail_t8_small"};
+  // the eight (token class, d_t range) launches are independent: each goes to
+  // the stream with the least work so far (items, those with more than
+  // TAIL_SMALL_ROWS rows weighted 4x), largest launches first, so that one
+  // launch's last long items do not leave the SMs idle before the next
+  int order[8], n_l = 0;
+  int64_t weight[8];
+  for (int i = 0; i < 8; ++i) {
+    const int c = i / 2, part = i % 2;
+    const int64_t n = part == 0 ? spl[c] - off[c] : off[c + 1] - spl[c];
+    weight[i] = n * (part == 0 ? 4 : 1);
+    if (n > 0) order[n_l++] = i;
+  }
+  std::sort(order, order + n_l, [&](int a, int b) { return weight[a] > weight[b]; });
+  int64_t load[8] = {};
   l3_status st = L3_OK;
-  for (int c = 0; c < 4 && st == L3_OK; ++c) {
-    for (int part = 0; part < 2 && st == L3_OK; ++part) {
+  for (int li = 0; li < n_l && st == L3_OK; ++li) {
+    const int c = order[li] / 2, part = order[li] % 2;
+    int q = 0;
+    for (int j = 1; j < n_streams; ++j)
+      if (load[j] < load[q]) q = j;
+    load[q] += weight[order[li]];
+    const cudaStream_t s = streams[q];
+    {
       const int64_t first = part == 0 ? off[c] : spl[c];
       const int64_t last = part == 0 ? spl[c] : off[c + 1];
-      if (last <= first) continue;
       LaunchTimer t(names[2 * c + part], s);
       // single-token items with d_t <= TAIL_SMALL_ROWS run a warp per item
       switch (c) {

@@ -150,8 +150,10 @@ l3_status launch_attn_tail(const l3_plan_s *p, const void *x, const void *W_K, c
 
 // attention, CUDA-core path specialised by token count (attn_tail_cls.cu)
 bool tail_cls_supported(const l3_dims_t &d);
+// the class launches spread over n_streams streams (largest first, each to
+// the least loaded stream)
 l3_status launch_attn_tail_cls(const l3_plan_s *p, const void *x, const void *W_K,
-                               const void *W_V, cudaStream_t s);
+                               const void *W_V, const cudaStream_t *streams, int n_streams);
 
 // attention, tensor-core path (attn_dense.cu)
 bool dense_attention_supported(const l3_dims_t &d);
