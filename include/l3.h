@@ -218,9 +218,11 @@ l3_status l3_forward(const void *x, l3_plan_t plan, const void *W_K, const void 
  * on the tensor-core path) comes from the library's device block cache
  * (cudaMalloc on a miss) and goes back to it, ordered after the work on
  * `stream`. Enqueued on `stream`; does not synchronize. Errors: L3_ERR_INVALID_ARG (NULL pointer,
- * a staged plan, x / W_K / W_V / dx not 16-byte aligned when the plan has
- * dense tiles), L3_ERR_UNSUPPORTED (k > 1024, or d_in / d_emb / d_up too
- * wide for its shared-memory layout), L3_ERR_OOM, L3_ERR_CUDA.
+ * a staged plan, x / W_K / W_V / dx / dW_K / dW_V not 16-byte aligned, a
+ * different device than the plan's), L3_ERR_UNSUPPORTED (k > 1024, or d_in /
+ * d_emb / d_up too wide for its shared-memory layout), L3_ERR_OOM,
+ * L3_ERR_CUDA. The plan's last stream becomes `stream`: l3_plan_destroy and
+ * l3_forward_status order themselves after this call's work.
  */
 l3_status l3_backward(const void *x, l3_plan_t plan, const void *W_K, const void *W_V,
                       const void *W_up, const void *ln_gamma, const void *ln_beta,

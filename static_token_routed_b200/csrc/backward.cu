@@ -325,6 +325,18 @@ __device__ __forceinline__ float ldt(const void *p, int64_t i) {
   if (WT == T_F32) return reinterpret_cast<const float *>(p)[i];
   return __bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(p)[i]);
 }
+// four consecutive elements i .. i + 3 (i a multiple of 4) as fp32
+template <int WT>
+__device__ __forceinline__ float4 ldt4(const void *p, int64_t i) {
+  if (WT == T_F32) return reinterpret_cast<const float4 *>(p)[i / 4];
+  const uint2 u = reinterpret_cast<const uint2 *>(p)[i / 4];
+  const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.x));
+  const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.y));
+  return make_float4(a.x, a.y, b.x, b.y);
+}
+__device__ __forceinline__ float dot4(const float4 a, const float4 b, float acc) {
+  return fmaf(a.w, b.w, fmaf(a.z, b.z, fmaf(a.y, b.y, fmaf(a.x, b.x, acc))));
+}
 
 template <int NT, int WT>
 __global__ void __launch_bounds__(256)
@@ -355,23 +367,26 @@ __global__ void __launch_bounds__(256)
       gas[i] = t < nt ? g_a[(int64_t)tok[t] * d_emb + col] : 0.f;
     }
     __syncthreads();
-    // logits s = K_j . x_t and g_p = V_j . g_a_t, one warp per row
+    // logits s = K_j . x_t and g_p = V_j . g_a_t, one warp per row, four
+    // columns per lane per step
     for (int j = warp; j < d; j += 8) {
       float sv[NT], gv[NT];
 #pragma unroll
       for (int t = 0; t < NT; ++t) sv[t] = gv[t] = 0.f;
       if (d > 1)
-#pragma unroll 4
-        for (int col = lane; col < d_in; col += 32) {
-          const float kv = ldt<WT>(W_K, (r0 + j) * d_in + col);
+#pragma unroll 2
+        for (int c4 = lane * 4; c4 < d_in; c4 += 128) {
+          const float4 kv = ldt4<WT>(W_K, (r0 + j) * d_in + c4);
 #pragma unroll
-          for (int t = 0; t < NT; ++t) sv[t] = fmaf(kv, xs[t * d_in + col], sv[t]);
+          for (int t = 0; t < NT; ++t)
+            sv[t] = dot4(kv, *reinterpret_cast<const float4 *>(xs + t * d_in + c4), sv[t]);
         }
-#pragma unroll 4
-      for (int col = lane; col < d_emb; col += 32) {
-        const float vv = ldt<WT>(W_V, (r0 + j) * d_emb + col);
+#pragma unroll 2
+      for (int c4 = lane * 4; c4 < d_emb; c4 += 128) {
+        const float4 vv = ldt4<WT>(W_V, (r0 + j) * d_emb + c4);
 #pragma unroll
-        for (int t = 0; t < NT; ++t) gv[t] = fmaf(vv, gas[t * d_emb + col], gv[t]);
+        for (int t = 0; t < NT; ++t)
+          gv[t] = dot4(vv, *reinterpret_cast<const float4 *>(gas + t * d_emb + c4), gv[t]);
       }
 #pragma unroll
       for (int t = 0; t < NT; ++t) {
@@ -408,36 +423,59 @@ __global__ void __launch_bounds__(256)
       for (int j = lane; j < d; j += 32) gr[j] = pr[j] * (gr[j] - dot);
     }
     __syncthreads();
-    // dx_t += K_t^T g_s_t and dK_j (+)= sum_t g_s[t][j] x_t: thread per column
+    // dx_t += K_t^T g_s_t and dK_j (+)= sum_t g_s[t][j] x_t: thread per four
+    // columns, one vector atomic add per row
     if (d > 1) {
-      for (int col = threadIdx.x; col < d_in; col += blockDim.x) {
-        float acc[NT];
+      for (int c4 = threadIdx.x * 4; c4 < d_in; c4 += blockDim.x * 4) {
+        float4 acc[NT];
 #pragma unroll
-        for (int t = 0; t < NT; ++t) acc[t] = 0.f;
-#pragma unroll 4
+        for (int t = 0; t < NT; ++t) acc[t] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 2
         for (int j = 0; j < d; ++j) {
-          const int64_t kidx = (r0 + j) * d_in + col;
-          const float kv = ldt<WT>(W_K, kidx);
-          float gk = 0.f;
+          const int64_t kidx = (r0 + j) * d_in + c4;
+          const float4 kv = ldt4<WT>(W_K, kidx);
+          float4 gk = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
           for (int t = 0; t < NT; ++t) {
             const float gst = gs[t * A_MAX_K + j];
-            acc[t] = fmaf(gst, kv, acc[t]);
-            gk = fmaf(gst, xs[t * d_in + col], gk);
+            const float4 xv = *reinterpret_cast<const float4 *>(xs + t * d_in + c4);
+            acc[t].x = fmaf(gst, kv.x, acc[t].x);
+            acc[t].y = fmaf(gst, kv.y, acc[t].y);
+            acc[t].z = fmaf(gst, kv.z, acc[t].z);
+            acc[t].w = fmaf(gst, kv.w, acc[t].w);
+            gk.x = fmaf(gst, xv.x, gk.x);
+            gk.y = fmaf(gst, xv.y, gk.y);
+            gk.z = fmaf(gst, xv.z, gk.z);
+            gk.w = fmaf(gst, xv.w, gk.w);
           }
-          atomicAdd(dW_K + kidx, gk);
+          atomicAdd(reinterpret_cast<float4 *>(dW_K + kidx), gk);
         }
-        for (int t = 0; t < nt; ++t) dx[(int64_t)tok[t] * d_in + col] += acc[t];
+        for (int t = 0; t < nt; ++t) {
+          float4 *o = reinterpret_cast<float4 *>(dx + (int64_t)tok[t] * d_in + c4);
+          float4 v = *o;
+          v.x += acc[t].x;
+          v.y += acc[t].y;
+          v.z += acc[t].z;
+          v.w += acc[t].w;
+          *o = v;
+        }
       }
     }  // one row: p = 1, no gradient reaches K
     // dV_j (+)= sum_t p[t][j] g_a_t
-    for (int col = threadIdx.x; col < d_emb; col += blockDim.x) {
-#pragma unroll 4
+    for (int c4 = threadIdx.x * 4; c4 < d_emb; c4 += blockDim.x * 4) {
+#pragma unroll 2
       for (int j = 0; j < d; ++j) {
-        float gv = 0.f;
+        float4 gv = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-        for (int t = 0; t < NT; ++t) gv = fmaf(ps[t * A_MAX_K + j], gas[t * d_emb + col], gv);
-        atomicAdd(dW_V + (r0 + j) * d_emb + col, gv);
+        for (int t = 0; t < NT; ++t) {
+          const float pj = ps[t * A_MAX_K + j];
+          const float4 ga = *reinterpret_cast<const float4 *>(gas + t * d_emb + c4);
+          gv.x = fmaf(pj, ga.x, gv.x);
+          gv.y = fmaf(pj, ga.y, gv.y);
+          gv.z = fmaf(pj, ga.z, gv.z);
+          gv.w = fmaf(pj, ga.w, gv.w);
+        }
+        atomicAdd(reinterpret_cast<float4 *>(dW_V + (r0 + j) * d_emb + c4), gv);
       }
     }
     __syncthreads();
@@ -845,9 +883,8 @@ __device__ __forceinline__ void dense_dw(const __nv_bfloat16 *__restrict__ x,
       for (int h = 0; h < 2; ++h) {
         const int j = jb + mr + g + 8 * h;
         if (j >= d) continue;
-        float *o = out + (r0 + j) * width + col;
-        atomicAdd(o, acc[q][2 * h]);
-        atomicAdd(o + 1, acc[q][2 * h + 1]);
+        float *o = out + (r0 + j) * width + col;  // col is even: 8-byte aligned
+        atomicAdd(reinterpret_cast<float2 *>(o), make_float2(acc[q][2 * h], acc[q][2 * h + 1]));
       }
     }
   }
@@ -938,8 +975,8 @@ extern "C" l3_status l3_backward(const void *x, l3_plan_t p, const void *W_K, co
   auto a16 = [](const void *q) { return (reinterpret_cast<uintptr_t>(q) & 15u) == 0; };
   // checked before anything is enqueued: the tail kernels add into dW_K / dW_V,
   // so a rejection after them would leave a partial gradient behind
-  if (p->n_dense_tiles > 0 && !(a16(x) && a16(W_K) && a16(W_V) && a16(dx))) {
-    set_error("l3_backward: x, W_K, W_V and dx must be 16-byte aligned");
+  if (!(a16(x) && a16(W_K) && a16(W_V) && a16(dx) && a16(dW_K) && a16(dW_V))) {
+    set_error("l3_backward: x, W_K, W_V, dx, dW_K and dW_V must be 16-byte aligned");
     return L3_ERR_INVALID_ARG;
   }
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
