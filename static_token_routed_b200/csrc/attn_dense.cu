@@ -9,14 +9,15 @@
 // which is the layer's V_t^T softmax(K_t x) for every token of the group at
 // once (kimjy99 review, Method, eq. L³).
 //
-// One CTA takes one 128-token tile of one group:
+// The kernel is persistent: each CTA claims 128-token tiles of one group from a
+// counter until none are left, and for each tile
 //   - warps 2-3 gather the tile's x rows (through the sort permutation) into
-//     128-byte-swizzled shared memory with cp.async, 64 columns at a time and
-//     up to a ring's depth of slices ahead;
+//     128-byte-swizzled shared memory with cp.async, 64 columns at a time, in a
+//     ring of their own; each warp instruction copies whole 128-byte row
+//     segments of four rows;
 //   - warp 0 streams the matching 64-column slices of K_t with TMA (128 bytes
-//     of each row per request: half as many, twice as long DRAM reads as
-//     32-column slices, which streamed K_t markedly slower), as many slices in
-//     flight as the shared-memory ring holds for this d_t;
+//     of each row per request), one slice per half of S (at most 256 rows, one
+//     MMA's N), as many in flight as the rest of the shared memory holds;
 //   - warp 1 issues tcgen05.mma (M = 128 tokens, N = d_t up to 2 x 256) so that
 //     S accumulates in TMEM over d_in;
 //   - warps 4-11 (two per TMEM lane quarter, so two threads per token row,
@@ -28,6 +29,9 @@
 //     slice that lie past d_t;
 //   - warps 4-11 scale O by 1 / rowsum and store a[perm[i]] (fp16), i.e. already
 //     in the caller's token order.
+// The next tile's x and K_t slices start loading as soon as this tile's P V_t
+// MMAs are done, during its epilogue, and its S MMAs as soon as the epilogue
+// has read O out of TMEM.
 // K_t and V_t are read from HBM by the group's first tile; its other tiles run
 // at the same time and find them in L2.
 // Groups with d_t <= 256 run in a second launch with half the shared memory
@@ -37,6 +41,8 @@
 // exact, so P's rounding weighs only on the smaller weights.
 #include <cuda_fp16.h>
 #include <cudaTypedefs.h>
+
+#include <algorithm>
 
 #include "l3_internal.cuh"
 #include "sm100.cuh"
@@ -64,7 +70,8 @@ constexpr int MAX_STAGES = 8;
 // 256-column passes through the same TMEM columns.
 template <bool SMALL>
 struct DenseCfg {
-  static constexpr int REGION = SMALL ? 96 * 1024 : 192 * 1024;  // S ring, later P + V slices
+  static constexpr int REGION = SMALL ? 96 * 1024 : 192 * 1024;  // S-phase rings, later P + V slices
+  static constexpr int N_X = SMALL ? 2 : 4;  // x slices in flight (ring at the top of the region)
   static constexpr int TMEM_COLS = SMALL ? 256 : 512;
   static constexpr int MIN_BLOCKS = SMALL ? 2 : 1;
 };
@@ -75,13 +82,20 @@ constexpr int DENSE_THREADS = 384;  // 0 TMA, 1 MMA, 2-3 x gather, 4-11 softmax 
 constexpr int SOFTMAX_THREADS = 256;
 
 struct DenseBars {
-  uint64_t xfull[MAX_STAGES], kfull[MAX_STAGES], sempty[MAX_STAGES];
-  uint64_t sfull, pready, ofull;
+  uint64_t xfull[4], xempty[4];                // x slices (fixed depth N_X)
+  uint64_t kfull[MAX_STAGES], kempty[MAX_STAGES];  // K_t slices (depth from d_t)
   uint64_t vfull[MAX_STAGES], vempty[MAX_STAGES];
-  uint64_t odrained;  // the epilogue has read this O pass out of TMEM
+  uint64_t sfull;     // every S-phase MMA of the tile has completed
+  uint64_t pready;    // the softmax warps have written P
+  uint64_t ofull;     // an O pass has completed
+  uint64_t odrained;  // the epilogue has read an O pass that a later pass of the tile overwrites
+  uint64_t pvdone;    // every P V_t MMA of the tile has completed: P and the V slices are free
+  uint64_t tdrained;  // the epilogue has read the tile's last O pass: TMEM is free for the next S
+  uint64_t tfull[2], tempty[2];  // tile handoff from the TMA warp to the other warps
   uint64_t drain;
   uint32_t tmem_base;
   int abort_flag;
+  int tile_slot[2];
   float red_max[2][128];  // per row: max of each half of the columns
   float red_sum[2][128];
 };
@@ -94,6 +108,8 @@ struct DenseParams {
   const int32_t *group_row_start;
   const int32_t *group_rows;
   const DenseTile *tiles;
+  int n_tiles;
+  int *counter;    // [0] next tile to claim, [1] CTAs finished; the last CTA zeroes both
   int d_in, d_emb;
   int *err;
 };
@@ -148,6 +164,52 @@ __device__ __forceinline__ void spin_bounded(uint64_t *bar, uint32_t parity) {
   }
 }
 
+// Per-tile geometry, the same in every warp: the S ring and the P / V layout
+// follow from d_t.
+struct TileGeo {
+  int tok0, n_valid, r0, d, d16, d32, d64, n_vc, n_half, k_stage, n_k, p_bytes, n_v;
+  int h_rows0, h_rows1;  // K_t rows of each half of S (columns 0-255, 256-511)
+};
+
+template <int REGION, int N_X>
+__device__ __forceinline__ TileGeo tile_geo(const DenseParams &P, int ti, int v_bytes) {
+  TileGeo t;
+  const DenseTile tile = P.tiles[ti];
+  const int g = tile.group;
+  t.tok0 = tile.tok0;
+  t.n_valid = min(TM, P.group_tok_start[g + 1] - t.tok0);
+  t.r0 = P.group_row_start[g];
+  t.d = P.group_rows[g];
+  t.d16 = (t.d + 15) & ~15;  // N of the S product, K extent of the PV product
+  t.d32 = (t.d + 31) & ~31;  // softmax works in 32-column TMEM loads
+  t.d64 = (t.d + 63) & ~63;
+  t.n_vc = t.d16 / V_ROWS;
+  // A K_t slice is one 64-column slice of the rows of one half of S (at most
+  // 256 rows, one MMA's N), so the ring turns over in steps of at most 32 KB
+  t.n_half = t.d16 > 256 ? 2 : 1;
+  t.h_rows0 = min(t.d16, 256);
+  t.h_rows1 = t.d16 - 256;
+  // pipeline depth follows from d_t: below the x ring, the K_t ring holds as
+  // many slices as fit, and so do the V slices after P
+  t.k_stage = (t.n_half == 2 ? 256 : t.d64) * CK * 2;
+  t.n_k = min(MAX_STAGES, (REGION - N_X * X_BYTES) / t.k_stage);
+  t.p_bytes = (t.d64 / 64) * (TM * 128);
+  t.n_v = min(MAX_STAGES, (REGION - t.p_bytes) / v_bytes);
+  return t;
+}
+
+// The next tile index from the TMA warp (-1: none left). Every warp of a
+// consumer role calls this once per tile, in order.
+__device__ __forceinline__ int next_tile(DenseBars *b, int u, const Abort &ab, bool &ok,
+                                         int lane) {
+  const int j = u & 1;
+  ok = __all_sync(0xffffffffu, mbar_wait(&b->tfull[j], (u >> 1) & 1, ab));
+  const int ti = *reinterpret_cast<volatile int *>(&b->tile_slot[j]);
+  __syncwarp();
+  if (lane == 0) mbar_arrive(&b->tempty[j]);
+  return ok ? ti : -1;
+}
+
 template <bool SMALL>
 __global__ void __launch_bounds__(DENSE_THREADS, DenseCfg<SMALL>::MIN_BLOCKS)
     k_attn_dense(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUtensorMap mK16,
@@ -158,50 +220,34 @@ __global__ void __launch_bounds__(DENSE_THREADS, DenseCfg<SMALL>::MIN_BLOCKS)
   uint8_t *smem = align1024(smem_raw);
   DenseBars *b = reinterpret_cast<DenseBars *>(smem + REGION);
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-
-  const DenseTile tile = P.tiles[blockIdx.x];
-  const int g = tile.group;
-  const int tok0 = tile.tok0;
-  const int n_valid = min(TM, P.group_tok_start[g + 1] - tok0);
-  const int r0 = P.group_row_start[g];
-  const int d = P.group_rows[g];
-  const int d16 = (d + 15) & ~15;       // N of the S product, K extent of the PV product
-  const int d32 = (d + 31) & ~31;       // softmax works in 32-column TMEM loads
-  const int d64 = (d + 63) & ~63;
   const int n_kc = P.d_in / CK;
-  const int n_vc = d16 / V_ROWS;
-  // K_t rows per slice: whole 64-row TMA boxes, then 16-row boxes up to d16
-  // (the rows the MMA reads), so no slice fetches more than 15 rows past d_t
-  const int k_full = d16 / 64, k_rest = (d16 % 64) / 16;
-  const uint32_t k_slice_bytes = (uint32_t)(k_full * 64 + k_rest * 16) * CK * 2;
   // O = P V_t in passes of at most TMEM_COLS columns of d_emb
   const int o_max = min(P.d_emb, Cfg::TMEM_COLS);
   const int n_op = (P.d_emb + o_max - 1) / o_max;
-  const int n_vs = n_op * n_vc;         // V slices over all passes
-  // pipeline depth follows from d_t: the S ring holds as many slices as fit,
-  // and so do the V buffers after P
-  const int s_stage = X_BYTES + d64 * CK * 2;
-  const int n_s = min(MAX_STAGES, REGION / s_stage);
-  const int p_bytes = (d64 / 64) * (TM * 128);
   const int v_bytes = V_ROWS * o_max * 2;
-  const int n_v = min(MAX_STAGES, (REGION - p_bytes) / v_bytes);
-  uint8_t *pbuf = smem;                 // P slices (PV phase)
-  uint8_t *vbuf = smem + p_bytes;       // V slices (PV phase)
+  uint8_t *pbuf = smem;  // P slices (PV phase); V slices follow at p_bytes
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < MAX_STAGES; ++s) {
+    for (int s = 0; s < 4; ++s) {
       mbar_init(&b->xfull[s], 2);
+      mbar_init(&b->xempty[s], 1);
+    }
+    for (int s = 0; s < MAX_STAGES; ++s) {
       mbar_init(&b->kfull[s], 1);
-      mbar_init(&b->sempty[s], 1);
+      mbar_init(&b->kempty[s], 1);
+      mbar_init(&b->vfull[s], 1);
+      mbar_init(&b->vempty[s], 1);
     }
     mbar_init(&b->sfull, 1);
     mbar_init(&b->pready, 8);
     mbar_init(&b->ofull, 1);
-    for (int i = 0; i < MAX_STAGES; ++i) {
-      mbar_init(&b->vfull[i], 1);
-      mbar_init(&b->vempty[i], 1);
-    }
     mbar_init(&b->odrained, 8);
+    mbar_init(&b->pvdone, 1);
+    mbar_init(&b->tdrained, 8);
+    for (int j = 0; j < 2; ++j) {
+      mbar_init(&b->tfull[j], 1);
+      mbar_init(&b->tempty[j], 11);  // warps 1-11
+    }
     mbar_init(&b->drain, 1);
     b->abort_flag = 0;
     fence_mbar_init();
@@ -219,51 +265,79 @@ __global__ void __launch_bounds__(DENSE_THREADS, DenseCfg<SMALL>::MIN_BLOCKS)
   const uint32_t tmem = b->tmem_base;
   const Abort ab{&b->abort_flag, P.err};
 
+  // Persistent: each CTA claims tiles from a counter until none are left. A
+  // tile's S ring overlays the previous tile's P and V slices and its S the
+  // previous tile's O, so the TMA and gather warps start the next tile's
+  // slices as soon as the previous tile's P V_t MMAs are done (during its
+  // epilogue), and the MMA warp once the epilogue has read O. Every ring slot
+  // keeps a per-slot phase bit across tiles (the ring depth changes with d_t).
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (elect_one()) {
       bool ok = true;
-      bool armed[MAX_STAGES];
-      uint32_t armed_par[MAX_STAGES];
-      for (int i = 0; i < MAX_STAGES; ++i) armed[i] = false;
-      for (int kc = 0; kc < n_kc; ++kc) {
-        const int s = kc % n_s;
-        const uint32_t ph = (kc / n_s) & 1;
-        if (!mbar_wait(&b->sempty[s], ph ^ 1, ab)) {
+      uint32_t ku = 0, vu = 0;  // per slot: parity of its uses so far
+      bool armed[MAX_STAGES], varmed[MAX_STAGES];
+      uint32_t armed_par[MAX_STAGES], varmed_par[MAX_STAGES];
+      for (int i = 0; i < MAX_STAGES; ++i) armed[i] = varmed[i] = false;
+      for (int u = 0; ok; ++u) {
+        int ti = atomicAdd(P.counter, 1);
+        if (ti >= P.n_tiles) ti = -1;
+        const int j = u & 1;
+        if (!mbar_wait(&b->tempty[j], ((u >> 1) & 1) ^ 1, ab)) {
           ok = false;
           break;
         }
-        uint8_t *kdst = smem + s * s_stage + X_BYTES;
-        mbar_arrive_expect_tx(&b->kfull[s], k_slice_bytes);
-        armed[s] = true;
-        armed_par[s] = ph;
-        for (int bx = 0; bx < k_full; ++bx)
-          tma_load_2d(kdst + bx * 64 * CK * 2, &mK, &b->kfull[s], kc * CK, r0 + bx * 64);
-        for (int bx = 0; bx < k_rest; ++bx)
-          tma_load_2d(kdst + (k_full * 64 + bx * 16) * CK * 2, &mK16, &b->kfull[s], kc * CK,
-                      r0 + k_full * 64 + bx * 16);
-      }
-      // V slices go where the S ring was: wait until every S-phase MMA is done
-      if (ok) ok = mbar_wait(&b->sfull, 0, ab);
-      bool varmed[MAX_STAGES];
-      uint32_t varmed_par[MAX_STAGES];
-      for (int i = 0; i < MAX_STAGES; ++i) varmed[i] = false;
-      for (int gv = 0; ok && gv < n_vs; ++gv) {
-        const int h = gv / n_vc, vc = gv % n_vc;
-        const int v_boxes = min(o_max, P.d_emb - h * o_max) / 64;
-        const int i = gv % n_v;
-        const uint32_t ph = (gv / n_v) & 1;
-        if (!mbar_wait(&b->vempty[i], ph ^ 1, ab)) {
+        b->tile_slot[j] = ti;
+        mbar_arrive(&b->tfull[j]);
+        if (ti < 0) break;
+        const TileGeo t = tile_geo<REGION, Cfg::N_X>(P, ti, v_bytes);
+        if (u > 0 && !mbar_wait(&b->pvdone, (u - 1) & 1, ab)) {
           ok = false;
           break;
         }
-        uint8_t *vdst = vbuf + i * v_bytes;
-        mbar_arrive_expect_tx(&b->vfull[i], v_boxes * V_BLOCK);
-        varmed[i] = true;
-        varmed_par[i] = ph;
-        for (int bx = 0; bx < v_boxes; ++bx)
-          tma_load_2d(vdst + bx * V_BLOCK, &mV, &b->vfull[i], h * o_max + bx * 64,
-                      r0 + vc * V_ROWS);
+        for (int kh = 0; kh < n_kc * t.n_half; ++kh) {
+          const int kc = kh / t.n_half, hf = kh - kc * t.n_half;
+          const int s = kh % t.n_k;
+          const uint32_t ph = (ku >> s) & 1;
+          if (!mbar_wait(&b->kempty[s], ph ^ 1, ab)) {
+            ok = false;
+            break;
+          }
+          ku ^= 1u << s;
+          uint8_t *kdst = smem + s * t.k_stage;
+          // whole 64-row TMA boxes, then 16-row boxes up to d16 (the rows the
+          // MMA reads), so no slice fetches more than 15 rows past d_t
+          const int rows = hf ? t.h_rows1 : t.h_rows0, k_full = rows / 64, k_rest = (rows % 64) / 16;
+          const int row0 = t.r0 + hf * 256;
+          mbar_arrive_expect_tx(&b->kfull[s], (uint32_t)rows * CK * 2);
+          armed[s] = true;
+          armed_par[s] = ph;
+          for (int bx = 0; bx < k_full; ++bx)
+            tma_load_2d(kdst + bx * 64 * CK * 2, &mK, &b->kfull[s], kc * CK, row0 + bx * 64);
+          for (int bx = 0; bx < k_rest; ++bx)
+            tma_load_2d(kdst + (k_full * 64 + bx * 16) * CK * 2, &mK16, &b->kfull[s], kc * CK,
+                        row0 + k_full * 64 + bx * 16);
+        }
+        // V slices go where the S ring was: wait until every S-phase MMA is done
+        if (ok) ok = mbar_wait(&b->sfull, u & 1, ab);
+        for (int gv = 0; ok && gv < n_op * t.n_vc; ++gv) {
+          const int h = gv / t.n_vc, vc = gv % t.n_vc;
+          const int v_boxes = min(o_max, P.d_emb - h * o_max) / 64;
+          const int i = gv % t.n_v;
+          const uint32_t ph = (vu >> i) & 1;
+          if (!mbar_wait(&b->vempty[i], ph ^ 1, ab)) {
+            ok = false;
+            break;
+          }
+          vu ^= 1u << i;
+          uint8_t *vdst = smem + t.p_bytes + i * v_bytes;
+          mbar_arrive_expect_tx(&b->vfull[i], v_boxes * V_BLOCK);
+          varmed[i] = true;
+          varmed_par[i] = ph;
+          for (int bx = 0; bx < v_boxes; ++bx)
+            tma_load_2d(vdst + bx * V_BLOCK, &mV, &b->vfull[i], h * o_max + bx * 64,
+                        t.r0 + vc * V_ROWS);
+        }
       }
       if (!ok) {
         for (int s = 0; s < MAX_STAGES; ++s)
@@ -271,91 +345,117 @@ __global__ void __launch_bounds__(DENSE_THREADS, DenseCfg<SMALL>::MIN_BLOCKS)
         for (int i = 0; i < MAX_STAGES; ++i)
           if (varmed[i]) spin_bounded(&b->vfull[i], varmed_par[i]);
       }
+      // the last CTA to finish returns the counter to zero for the next launch
+      // (every CTA has made its last claim by then)
+      if (atomicAdd(P.counter + 1, 1) == (int)gridDim.x - 1) {
+        P.counter[0] = 0;
+        P.counter[1] = 0;
+      }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     // lane 0 issues; the whole warp waits for the V slices and zeroes the
     // padding rows of the last slice of each pass
     bool ok = true;
-    if (lane == 0) {
-      const int n_half = d16 > 256 ? 2 : 1;
-      const uint32_t id_s0 = idesc_f16(1, 0, TM, d16 > 256 ? 256 : d16);
-      const uint32_t id_s1 = idesc_f16(1, 0, TM, d16 > 256 ? d16 - 256 : 16);
-      for (int kc = 0; ok && kc < n_kc; ++kc) {
-        const int s = kc % n_s;
-        const uint32_t ph = (kc / n_s) & 1;
-        if (!mbar_wait(&b->xfull[s], ph, ab) || !mbar_wait(&b->kfull[s], ph, ab)) {
+    uint32_t mu = 0, mv = 0;  // per slot: parity of its uses so far (lane 0 / all lanes)
+    int gx = 0;               // x slices consumed so far (lane 0)
+    for (int u = 0; ok; ++u) {
+      const int ti = next_tile(b, u, ab, ok, lane);
+      if (!ok || ti < 0) break;
+      const TileGeo t = tile_geo<REGION, Cfg::N_X>(P, ti, v_bytes);
+      // S goes into the TMEM columns of the previous tile's O
+      ok = __all_sync(0xffffffffu, mbar_wait(&b->tdrained, (u & 1) ^ 1, ab));
+      if (!ok) break;
+      tc_fence_after();
+      if (lane == 0) {
+        const uint32_t id_s0 = idesc_f16(1, 0, TM, t.h_rows0);
+        const uint32_t id_s1 = idesc_f16(1, 0, TM, t.n_half == 2 ? t.h_rows1 : 16);
+        int kh = 0;
+        for (int kc = 0; ok && kc < n_kc; ++kc) {
+          const int xs = gx % Cfg::N_X;
+          if (!mbar_wait(&b->xfull[xs], (gx / Cfg::N_X) & 1, ab)) {
+            ok = false;
+            break;
+          }
+          ++gx;
+          const uint32_t xa = smem_u32(smem + REGION - (Cfg::N_X - xs) * X_BYTES);
+          for (int hf = 0; hf < t.n_half; ++hf, ++kh) {
+            const int s = kh % t.n_k;
+            if (!mbar_wait(&b->kfull[s], (mu >> s) & 1, ab)) {
+              ok = false;
+              break;
+            }
+            mu ^= 1u << s;
+            tc_fence_after();
+            const uint32_t ka = smem_u32(smem + s * t.k_stage);
+#pragma unroll
+            for (int k = 0; k < CK / 16; ++k)
+              umma_f16(tmem + hf * 256, sdesc_sw128(xa + k * 32, 16, 1024),
+                       sdesc_sw128(ka + k * 32, 16, 1024), hf ? id_s1 : id_s0, (kc | k) != 0);
+            umma_commit(&b->kempty[s]);
+          }
+          if (ok) umma_commit(&b->xempty[xs]);
+        }
+        if (ok) umma_commit(&b->sfull);
+      }
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      // P V_t into the TMEM columns S used, once the softmax warps have read S
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&b->pready, u & 1, ab));
+      const uint32_t pa = smem_u32(pbuf);
+      for (int h = 0; ok && h < n_op; ++h) {
+        // a later pass reuses the TMEM columns once the epilogue has read them
+        if (h > 0 &&
+            !__all_sync(0xffffffffu, mbar_wait(&b->odrained, (u * (n_op - 1) + h - 1) & 1, ab))) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint32_t xa = smem_u32(smem + s * s_stage);
-        const uint32_t ka = xa + X_BYTES;
-#pragma unroll
-        for (int k = 0; k < CK / 16; ++k) {
-          const uint64_t adesc = sdesc_sw128(xa + k * 32, 16, 1024);
-          umma_f16(tmem, adesc, sdesc_sw128(ka + k * 32, 16, 1024), id_s0, (kc | k) != 0);
-          if (n_half == 2)
-            umma_f16(tmem + 256, adesc, sdesc_sw128(ka + 256 * CK * 2 + k * 32, 16, 1024), id_s1,
-                     (kc | k) != 0);
-        }
-        umma_commit(&b->sempty[s]);
-      }
-      if (ok) umma_commit(&b->sfull);
-    }
-    ok = __shfl_sync(0xffffffffu, ok, 0);
-    // P V_t into the TMEM columns S used, once the softmax warps have read S
-    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&b->pready, 0, ab));
-    const uint32_t pa = smem_u32(pbuf);
-    for (int h = 0; ok && h < n_op; ++h) {
-      // a later pass reuses the TMEM columns once the epilogue has read them
-      if (h > 0 && !__all_sync(0xffffffffu, mbar_wait(&b->odrained, (h - 1) & 1, ab))) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      const int o_w = min(o_max, P.d_emb - h * o_max);
-      const int o_half = o_w > 256 ? 2 : 1;
-      const uint32_t id_o0 = idesc_f16(1, 1, TM, o_w > 256 ? 256 : o_w);
-      const uint32_t id_o1 = idesc_f16(1, 1, TM, o_w > 256 ? o_w - 256 : 16);
-      for (int vc = 0; vc < n_vc; ++vc) {
-        const int gv = h * n_vc + vc;
-        const int i = gv % n_v;
-        const uint32_t ph = (gv / n_v) & 1;
-        if (!__all_sync(0xffffffffu, mbar_wait(&b->vfull[i], ph, ab))) {
-          ok = false;
-          break;
-        }
-        const int live = d - vc * V_ROWS;  // rows of this slice that belong to the group
-        if (live < V_ROWS) {
-          // rows at or past d_t belong to the next token IDs: zero them, so that
-          // nothing in another ID's rows (an Inf, a NaN) reaches this group's
-          // P V_t through a zero of P (static routing: a token's output
-          // depends on its own rows only)
-          const int blocks = o_w / 64, per_block = (V_ROWS - live) * 8;
-          uint4 *vb = reinterpret_cast<uint4 *>(vbuf + i * v_bytes);
-          for (int e = lane; e < blocks * per_block; e += 32) {
-            const int bk = e / per_block, w = e - bk * per_block;
-            vb[bk * (V_BLOCK / 16) + live * 8 + w] = make_uint4(0u, 0u, 0u, 0u);
+        const int o_w = min(o_max, P.d_emb - h * o_max);
+        const int o_half = o_w > 256 ? 2 : 1;
+        const uint32_t id_o0 = idesc_f16(1, 1, TM, o_w > 256 ? 256 : o_w);
+        const uint32_t id_o1 = idesc_f16(1, 1, TM, o_w > 256 ? o_w - 256 : 16);
+        for (int vc = 0; vc < t.n_vc; ++vc) {
+          const int gv = h * t.n_vc + vc;
+          const int i = gv % t.n_v;
+          const uint32_t ph = (mv >> i) & 1;
+          if (!__all_sync(0xffffffffu, mbar_wait(&b->vfull[i], ph, ab))) {
+            ok = false;
+            break;
           }
-          fence_proxy_async_smem();
+          mv ^= 1u << i;
+          uint8_t *vslot = smem + t.p_bytes + i * v_bytes;
+          const int live = t.d - vc * V_ROWS;  // rows of this slice that belong to the group
+          if (live < V_ROWS) {
+            // rows at or past d_t belong to the next token IDs: zero them, so that
+            // nothing in another ID's rows (an Inf, a NaN) reaches this group's
+            // P V_t through a zero of P (static routing: a token's output
+            // depends on its own rows only)
+            const int blocks = o_w / 64, per_block = (V_ROWS - live) * 8;
+            uint4 *vb = reinterpret_cast<uint4 *>(vslot);
+            for (int e = lane; e < blocks * per_block; e += 32) {
+              const int bk = e / per_block, w = e - bk * per_block;
+              vb[bk * (V_BLOCK / 16) + live * 8 + w] = make_uint4(0u, 0u, 0u, 0u);
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+          }
+          tc_fence_after();
+          if (lane == 0) {
+            const uint32_t va = smem_u32(vslot);
+            const int kk = vc * V_ROWS;  // column of P / row of V_t
+            const uint64_t adesc =
+                sdesc_sw128(pa + (kk / 64) * (TM * 128) + (kk % 64) * 2, 16, 1024);
+            umma_f16(tmem, adesc, sdesc_sw128(va, V_BLOCK, 1024), id_o0, vc != 0);
+            if (o_half == 2)
+              umma_f16(tmem + 256, adesc, sdesc_sw128(va + 4 * V_BLOCK, V_BLOCK, 1024), id_o1,
+                       vc != 0);
+            umma_commit(&b->vempty[i]);
+          }
           __syncwarp();
         }
-        tc_fence_after();
-        if (lane == 0) {
-          const uint32_t va = smem_u32(vbuf + i * v_bytes);
-          const int kk = vc * V_ROWS;  // column of P / row of V_t
-          const uint64_t adesc =
-              sdesc_sw128(pa + (kk / 64) * (TM * 128) + (kk % 64) * 2, 16, 1024);
-          umma_f16(tmem, adesc, sdesc_sw128(va, V_BLOCK, 1024), id_o0, vc != 0);
-          if (o_half == 2)
-            umma_f16(tmem + 256, adesc, sdesc_sw128(va + 4 * V_BLOCK, V_BLOCK, 1024), id_o1,
-                     vc != 0);
-          umma_commit(&b->vempty[i]);
-        }
-        __syncwarp();
+        if (ok && lane == 0) umma_commit(&b->ofull);
       }
-      if (ok && lane == 0) umma_commit(&b->ofull);
+      if (ok && lane == 0) umma_commit(&b->pvdone);
     }
     if (!ok && lane == 0) {
       umma_commit(&b->drain);
@@ -363,147 +463,177 @@ __global__ void __launch_bounds__(DENSE_THREADS, DenseCfg<SMALL>::MIN_BLOCKS)
     }
   } else if (warp < 4) {
     // ------------------------------------------------------------ x-row gather
-    // cp.async copies (16 bytes each, zero-filled past the group's tokens),
-    // up to n_s - 1 slices ahead; a slice is handed to the MMA warp once this
-    // thread's copies for it have landed and been made visible to the async proxy.
-    const int t = (warp - 2) * 32 + lane;  // 0..63, rows t and t + 64
-    const __nv_bfloat16 *src_row[2];
-    uint32_t src_bytes[2];
-#pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      const int r = t + u * 64;
-      const bool valid = r < n_valid;
-      src_row[u] = P.x + (valid ? (int64_t)P.perm[tok0 + r] * P.d_in : 0);
-      src_bytes[u] = valid ? 16u : 0u;
-    }
-    const int lag = n_s - 1;
+    // cp.async copies (16 bytes each, zero-filled past the group's tokens)
+    // into a ring of N_X slices; a slice is handed to the MMA warp once this
+    // thread's copies for it have landed and been made visible to the async
+    // proxy, as soon as LAG later slices have been issued. With LAG = N_X - 2
+    // handing over slice n needs only slice n - 2 to have been consumed, so
+    // the handover does not wait for the MMAs of slice n - 1. Thread tw copies 16-byte chunk tw % 8 of rows tw / 8 + 8 i
+    // (i = 0..15), so every warp instruction reads four whole 128-byte row
+    // segments instead of one 16-byte piece of 32 rows.
+    const int tw = (warp - 2) * 32 + lane;  // 0..63
+    const int chunk = tw & 7, rb = tw >> 3;
     bool ok = true;
-    int issued = 0, done = 0;
-    for (int kc = 0; kc < n_kc; ++kc) {
-      const int s = kc % n_s;
-      const uint32_t ph = (kc / n_s) & 1;
-      ok = __all_sync(0xffffffffu, mbar_wait(&b->sempty[s], ph ^ 1, ab));
-      if (!ok) break;
-      uint8_t *xdst = smem + s * s_stage;
-      // 128-byte rows; the 128-byte swizzle XORs the 16-byte chunk index with
-      // bits 0-2 of the row
+    int gx = 0;  // x slices gathered so far
+    for (int u = 0; ok; ++u) {
+      const int ti = next_tile(b, u, ab, ok, lane);
+      if (!ok || ti < 0) break;
+      const TileGeo t = tile_geo<REGION, Cfg::N_X>(P, ti, v_bytes);
+      int src_row[16];  // original token of each of this thread's rows, -1 past the group
 #pragma unroll
-      for (int u = 0; u < 2; ++u) {
-        const int r = t + u * 64;
+      for (int i = 0; i < 16; ++i) {
+        const int r = rb + 8 * i;
+        src_row[i] = r < t.n_valid ? P.perm[t.tok0 + r] : -1;
+      }
+      if (u > 0 && !__all_sync(0xffffffffu, mbar_wait(&b->pvdone, (u - 1) & 1, ab))) {
+        ok = false;
+        break;
+      }
+      constexpr int lag = Cfg::N_X >= 3 ? Cfg::N_X - 2 : Cfg::N_X - 1;
+      int issued = 0, done = 0;
+      for (int kc = 0; kc < n_kc; ++kc) {
+        const int xs = (gx + kc) % Cfg::N_X;
+        ok = __all_sync(0xffffffffu,
+                        mbar_wait(&b->xempty[xs], (((gx + kc) / Cfg::N_X) & 1) ^ 1, ab));
+        if (!ok) break;
+        uint8_t *xdst = smem + REGION - (Cfg::N_X - xs) * X_BYTES;
+        const int col = kc * CK + chunk * 8;
+        // 128-byte rows; the 128-byte swizzle XORs the 16-byte chunk index with
+        // bits 0-2 of the row (here rb, since 8 i does not change them)
+        uint8_t *dcol = xdst + ((chunk ^ rb) << 4);
 #pragma unroll
-        for (int j = 0; j < 8; ++j)
-          cp_async16_zfill(xdst + r * 128 + ((j ^ (r & 7)) << 4), src_row[u] + kc * CK + j * 8,
-                           src_bytes[u]);
+        for (int i = 0; i < 16; ++i) {
+          const int r = rb + 8 * i;
+          const bool valid = src_row[i] >= 0;
+          cp_async16_zfill(dcol + r * 128,
+                           P.x + (valid ? (int64_t)src_row[i] * P.d_in + col : 0),
+                           valid ? 16u : 0u);
+        }
+        cp_async_commit();
+        ++issued;
+        if (issued - done > lag) {
+          cp_async_wait_group_lag(lag);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&b->xfull[(gx + done) % Cfg::N_X]);
+          ++done;
+        }
       }
-      cp_async_commit();
-      ++issued;
-      if (issued - done > lag) {
-        cp_async_wait_group_lag(lag);
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&b->xfull[done % n_s]);
-        ++done;
-      }
+      // the last slices, and on a give-up every copy still in flight
+      cp_async_wait_all();
+      fence_proxy_async_smem();
+      __syncwarp();
+      for (; ok && done < issued; ++done)
+        if (lane == 0) mbar_arrive(&b->xfull[(gx + done) % Cfg::N_X]);
+      gx += n_kc;
     }
-    // the last slices, and on a give-up every copy still in flight
-    cp_async_wait_all();
-    fence_proxy_async_smem();
-    __syncwarp();
-    for (; ok && done < issued; ++done)
-      if (lane == 0) mbar_arrive(&b->xfull[done % n_s]);
   } else {
-    // ------------------------------------------------------------ softmax, V convert, epilogue
+    // ------------------------------------------------------------ softmax, epilogue
     // warps 4-11: two warps per TMEM lane quarter, each taking every other
     // 32-column slice of the row; row max and row sum combine through shared
-    // memory at barriers of these 256 threads
+    // memory at barriers of these 256 threads, which all of them pass the same
+    // number of times
     const int sw = warp - 4;  // 0..7
     const int q = warp & 3;
     const int half = sw / 4;
     const int r = q * 32 + lane;
     const uint32_t trow = tmem + ((uint32_t)(q * 32) << 16);
-    float inv_sum = 0.f;
-    bool ok = __all_sync(0xffffffffu, mbar_wait(&b->sfull, 0, ab));
-    ok = softmax_sync_and(ok);
-    if (ok) {
-      tc_fence_after();
-      float m = -INFINITY;
-      for (int c = half * 32; c < d32; c += 64) {
-        uint32_t v[32];
-        tmem_ld32(trow + c, v);
-        tmem_wait_ld();
+    bool ok = true;
+    for (int u = 0; ok; ++u) {
+      const int ti = next_tile(b, u, ab, ok, lane);
+      ok = softmax_sync_and(ok);
+      if (!ok || ti < 0) break;
+      const TileGeo t = tile_geo<REGION, Cfg::N_X>(P, ti, v_bytes);
+      float inv_sum = 0.f;
+      ok = __all_sync(0xffffffffu, mbar_wait(&b->sfull, u & 1, ab));
+      ok = softmax_sync_and(ok);
+      if (ok) {
+        tc_fence_after();
+        float m = -INFINITY;
+        for (int c = half * 32; c < t.d32; c += 64) {
+          uint32_t v[32];
+          tmem_ld32(trow + c, v);
+          tmem_wait_ld();
 #pragma unroll
-        for (int j = 0; j < 32; ++j)
-          if (c + j < d) m = fmaxf(m, __uint_as_float(v[j]));
-      }
-      b->red_max[half][r] = m;
-    }
-    ok = softmax_sync_and(ok);
-    if (ok) {
-      const float m = fmaxf(b->red_max[0][r], b->red_max[1][r]);
-      float sum = 0.f;
-      for (int c = half * 32; c < d32; c += 64) {
-        uint32_t v[32];
-        tmem_ld32(trow + c, v);
-        tmem_wait_ld();
-        // 32 columns -> four 16-byte chunks of the 128-byte swizzled P row
-        uint8_t *prow = pbuf + (c / 64) * (TM * 128) + r * 128;
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          uint4 o;
-          __nv_bfloat162 *o2 = reinterpret_cast<__nv_bfloat162 *>(&o);
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int col = c + j * 8 + 2 * e;
-            const float p0 = col < d ? __expf(__uint_as_float(v[j * 8 + 2 * e]) - m) : 0.f;
-            const float p1 = col + 1 < d ? __expf(__uint_as_float(v[j * 8 + 2 * e + 1]) - m) : 0.f;
-            const __nv_bfloat162 hp = __floats2bfloat162_rn(p0, p1);
-            // the sum uses the rounded values the MMA will see
-            const float2 hf = __bfloat1622float2(hp);
-            sum += hf.x + hf.y;
-            o2[e] = hp;
-          }
-          const int chunk = ((c % 64) / 8) + j;  // 16-byte chunk index within the row
-          *reinterpret_cast<uint4 *>(prow + ((chunk ^ (r & 7)) << 4)) = o;
+          for (int j = 0; j < 32; ++j)
+            if (c + j < t.d) m = fmaxf(m, __uint_as_float(v[j]));
         }
+        b->red_max[half][r] = m;
       }
-      b->red_sum[half][r] = sum;
-    }
-    fence_proxy_async_smem();
-    tc_fence_before();
-    __syncwarp();
-    if (lane == 0 && ok) mbar_arrive(&b->pready);
-    ok = softmax_sync_and(ok);
-    if (ok) inv_sum = 1.0f / (b->red_sum[0][r] + b->red_sum[1][r]);
-
-    __half *arow = P.a + (r < n_valid ? (int64_t)P.perm[tok0 + r] * P.d_emb : 0);
-    for (int h = 0; ok && h < n_op; ++h) {
-      const int o_w = min(o_max, P.d_emb - h * o_max);
-      // epilogue: a = O / rowsum, fp16, to the token's original position
-      ok = __all_sync(0xffffffffu, mbar_wait(&b->ofull, h & 1, ab));
-      if (!ok) break;
-      tc_fence_after();
-      for (int c = half * 32; c < o_w; c += 64) {
-        uint32_t v[32];
-        tmem_ld32(trow + c, v);
-        tmem_wait_ld();
-        if (r < n_valid) {
+      ok = softmax_sync_and(ok);
+      if (ok) {
+        const float m = fmaxf(b->red_max[0][r], b->red_max[1][r]);
+        float sum = 0.f;
+        for (int c = half * 32; c < t.d32; c += 64) {
+          uint32_t v[32];
+          tmem_ld32(trow + c, v);
+          tmem_wait_ld();
+          // 32 columns -> four 16-byte chunks of the 128-byte swizzled P row
+          uint8_t *prow = pbuf + (c / 64) * (TM * 128) + r * 128;
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
             uint4 o;
-            __half2 *o2 = reinterpret_cast<__half2 *>(&o);
+            __nv_bfloat162 *o2 = reinterpret_cast<__nv_bfloat162 *>(&o);
 #pragma unroll
-            for (int e = 0; e < 4; ++e)
-              o2[e] = __floats2half2_rn(__uint_as_float(v[j * 8 + 2 * e]) * inv_sum,
-                                        __uint_as_float(v[j * 8 + 2 * e + 1]) * inv_sum);
-            *reinterpret_cast<uint4 *>(arow + h * o_max + c + j * 8) = o;
+            for (int e = 0; e < 4; ++e) {
+              const int col = c + j * 8 + 2 * e;
+              const float p0 = col < t.d ? __expf(__uint_as_float(v[j * 8 + 2 * e]) - m) : 0.f;
+              const float p1 =
+                  col + 1 < t.d ? __expf(__uint_as_float(v[j * 8 + 2 * e + 1]) - m) : 0.f;
+              const __nv_bfloat162 hp = __floats2bfloat162_rn(p0, p1);
+              // the sum uses the rounded values the MMA will see
+              const float2 hf = __bfloat1622float2(hp);
+              sum += hf.x + hf.y;
+              o2[e] = hp;
+            }
+            const int chunk = ((c % 64) / 8) + j;  // 16-byte chunk index within the row
+            *reinterpret_cast<uint4 *>(prow + ((chunk ^ (r & 7)) << 4)) = o;
           }
         }
+        b->red_sum[half][r] = sum;
       }
-      if (h + 1 < n_op) {
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&b->odrained);
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0 && ok) mbar_arrive(&b->pready);
+      ok = softmax_sync_and(ok);
+      if (ok) inv_sum = 1.0f / (b->red_sum[0][r] + b->red_sum[1][r]);
+
+      __half *arow = P.a + (r < t.n_valid ? (int64_t)P.perm[t.tok0 + r] * P.d_emb : 0);
+      for (int h = 0; ok && h < n_op; ++h) {
+        const int o_w = min(o_max, P.d_emb - h * o_max);
+        // epilogue: a = O / rowsum, fp16, to the token's original position
+        ok = __all_sync(0xffffffffu, mbar_wait(&b->ofull, (u * n_op + h) & 1, ab));
+        if (!ok) break;
+        tc_fence_after();
+        for (int c = half * 32; c < o_w; c += 64) {
+          uint32_t v[32];
+          tmem_ld32(trow + c, v);
+          tmem_wait_ld();
+          if (r < t.n_valid) {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              uint4 o;
+              __half2 *o2 = reinterpret_cast<__half2 *>(&o);
+#pragma unroll
+              for (int e = 0; e < 4; ++e)
+                o2[e] = __floats2half2_rn(__uint_as_float(v[j * 8 + 2 * e]) * inv_sum,
+                                          __uint_as_float(v[j * 8 + 2 * e + 1]) * inv_sum);
+              *reinterpret_cast<uint4 *>(arow + h * o_max + c + j * 8) = o;
+            }
+          }
+        }
+        if (h + 1 < n_op) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&b->odrained);
+        }
       }
+      // the tile's TMEM columns are free for the next tile's S
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0 && ok) mbar_arrive(&b->tdrained);
+      ok = softmax_sync_and(ok);
     }
   }
   __syncwarp();
@@ -520,10 +650,15 @@ constexpr size_t dense_smem() {
   return 1024 + DenseCfg<SMALL>::REGION + sizeof(DenseBars);
 }
 
+int sm_count(int device) {
+  static int n[64] = {};
+  if (n[device & 63] == 0) cudaDeviceGetAttribute(&n[device & 63], cudaDevAttrMultiProcessorCount, device);
+  return n[device & 63];
+}
+
 template <bool SMALL>
 l3_status launch_cfg(const CUtensorMap &mK, const CUtensorMap &mK16, const CUtensorMap &mV,
-                     const DenseParams &P,
-                     int64_t n_tiles, int device, const char *name, cudaStream_t s) {
+                     DenseParams P, int64_t n_tiles, int device, const char *name, cudaStream_t s) {
   if (n_tiles == 0) return L3_OK;
   static bool attr[64] = {};
   if (!attr[device & 63]) {
@@ -532,8 +667,11 @@ l3_status launch_cfg(const CUtensorMap &mK, const CUtensorMap &mK16, const CUten
                                      (int)dense_smem<SMALL>()));
     attr[device & 63] = true;
   }
+  // persistent: as many CTAs as fit at once, each claiming tiles until none are left
+  const int64_t grid = std::min<int64_t>(n_tiles, (int64_t)sm_count(device) * DenseCfg<SMALL>::MIN_BLOCKS);
+  P.n_tiles = (int)n_tiles;
   LaunchTimer t(name, s);
-  k_attn_dense<SMALL><<<(unsigned)n_tiles, DENSE_THREADS, dense_smem<SMALL>(), s>>>(mK, mK16, mV, P);
+  k_attn_dense<SMALL><<<(unsigned)grid, DENSE_THREADS, dense_smem<SMALL>(), s>>>(mK, mK16, mV, P);
   L3_CUDA_TRY(cudaGetLastError());
   return L3_OK;
 }
@@ -572,8 +710,10 @@ l3_status launch_attn_dense(const l3_plan_s *p, const void *x, const void *W_K, 
   P.d_in = (int)d.d_in;
   P.d_emb = (int)d.d_emb;
   P.err = p->dev_flags + 1;
+  P.counter = p->dev_flags + 4;
   if (!small) return launch_cfg<false>(mK, mK16, mV, P, n_big, p->device, "attn_dense", s);
   P.tiles = p->dense_tiles + n_big;
+  P.counter = p->dev_flags + 6;
   return launch_cfg<true>(mK, mK16, mV, P, p->n_dense_small, p->device, "attn_dense_small", s);
 }
 

@@ -107,7 +107,7 @@ struct l3_plan_s {
   int32_t *seg_rows = nullptr;         // [N+1]
   l3::DenseTile *dense_tiles = nullptr;
   l3::TailItem *tail_items = nullptr;
-  int32_t *dev_flags = nullptr;        // [0] plan errors, [1] forward errors, [2] work counter
+  int32_t *dev_flags = nullptr;        // [0] plan errors, [1] forward errors, [4..7] dense tile counters
   void *a_buf = nullptr;               // [N x d_emb] dtype, original token order
   void *h_buf = nullptr;               // [N x d_up] dtype
   float *z_buf = nullptr;              // [N x d_up] fp32 (CUDA-core GEMM path only)
