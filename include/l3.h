@@ -181,12 +181,17 @@ l3_status l3_plan_export(l3_plan_t plan, int32_t *perm, int32_t *inv_perm, int32
  *                                     output, columns d_up.. multiply x
  *   y         [N x d_out]             output, caller's token order
  * All in dims->dtype. Softmax has no 1/sqrt(d) scale (none appears in the
- * equation). The intermediates a = V_t^T p and h = LayerNorm(W_up a) are
- * stored once each, as fp16 for a bf16 layer (fp16's 10-bit mantissa keeps
- * the error that LayerNorm amplifies small) and as fp32 for an fp32 layer;
- * y is rounded once to dtype. The call only enqueues work on `stream` and never
- * synchronizes; a device-side wait that gives up is reported by
- * l3_forward_status. Errors: L3_ERR_INVALID_ARG, L3_ERR_CUDA.
+ * equation). For a bf16 layer the intermediates a = V_t^T p and z = W_up a
+ * are stored once each as fp16 (fp16's 10-bit mantissa keeps the error that
+ * LayerNorm amplifies small), and the LayerNorm is applied inside the W_mix
+ * product, W_mix[:, :d_up] LayerNorm(z) = r (W' z - mu W' 1) + W_mix[:, :d_up]
+ * beta with W' = W_mix[:, :d_up] diag(gamma) in fp16 and each row's mean mu
+ * and 1 / std r from z's fp32 values; for an fp32 layer a and h =
+ * LayerNorm(z) are stored as fp32. y is rounded once to dtype. The call only
+ * enqueues work on `stream` and never synchronizes; a device-side wait that
+ * gives up, and (bf16 layers) a W_up, W' or z value outside fp16's finite
+ * range, are reported by l3_forward_status. Errors: L3_ERR_INVALID_ARG,
+ * L3_ERR_CUDA.
  */
 l3_status l3_forward(const void *x, l3_plan_t plan, const void *W_K, const void *W_V,
                      const void *W_up, const void *ln_gamma, const void *ln_beta,
@@ -201,9 +206,11 @@ l3_status l3_forward(const void *x, l3_plan_t plan, const void *W_K, const void 
  * CUDA cores in fp32.
  *
  * Call after l3_forward on the same plan and the same inputs: it reuses the
- * a = V_t^T softmax(K_t x) and h = LayerNorm(W_up a) that forward stored
- * in the plan (and recomputes W_up a).
- *   x .. W_mix   as for l3_forward (dims->dtype); ln_beta is not read
+ * a = V_t^T softmax(K_t x) that forward stored in the plan, and h =
+ * LayerNorm(W_up a) as forward stored it (fp32 layers) or rebuilt from the z =
+ * W_up a and row statistics forward stored (bf16 layers); it also recomputes
+ * W_up a.
+ *   x .. W_mix   as for l3_forward (dims->dtype)
  *   dy           [N x d_out] dims->dtype, caller's token order
  *   dx           fp32 [N x d_in], out
  *   dW_K, dW_V   fp32 [v x d_in], [v x d_emb], in/out: the batch's
@@ -342,8 +349,9 @@ l3_status l3_check_bounded_wait(void *stream);
 
 /* Synchronizes the plan's last stream and returns L3_ERR_TIMEOUT if a
  * bounded wait inside an l3_forward kernel gave up since the plan was made
- * (the outputs of that call are then incomplete), L3_ERR_CUDA on a CUDA
- * error, L3_OK otherwise. */
+ * (the outputs of that call are then incomplete), L3_ERR_UNSUPPORTED if a bf16
+ * layer's fp16 operand (W_up, W_mix[:, :d_up] diag(ln_gamma), z = W_up a) fell
+ * outside fp16's finite range, L3_ERR_CUDA on a CUDA error, L3_OK otherwise. */
 l3_status l3_forward_status(l3_plan_t plan);
 
 /* Releases the plan. Its device memory returns to a small per-process cache

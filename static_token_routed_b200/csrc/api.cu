@@ -307,7 +307,9 @@ static l3_status plan_impl(const int32_t *token_ids, int64_t n_tokens, const int
       align256(p->tc_gemm ? 0 : n * dims->d_up * 4),              // z (CUDA-core GEMM path)
       align256(plan_scratch_bytes(n)),                            // plan-build scratch
       align256(p->tc_gemm ? dims->d_up * dims->d_emb * 2 : 0),    // fp16 W_up
-      align256(p->tc_gemm ? dims->d_out * dims->d_up * 2 : 0),    // fp16 W_mix[:, :d_up]
+      align256(p->tc_gemm ? dims->d_out * dims->d_up * 2 : 0),    // fp16 W_mix[:, :d_up] diag(gamma)
+      align256(p->tc_gemm ? n * ((dims->d_up + 255) / 256) * 8 : 0),  // (mean, M2) of z per 256 columns
+      align256(p->tc_gemm ? 2 * ((dims->d_out + 3) / 4 * 4) * 4 : 0),  // W' 1, W_mix[:, :d_up] beta
   };
   size_t total = 0;
   for (size_t b : sizes) total += b;
@@ -350,6 +352,8 @@ static l3_status plan_impl(const int32_t *token_ids, int64_t n_tokens, const int
   void *scratch = next(i++);
   p->w_up16 = next(i++);
   p->w_mixh16 = next(i++);
+  p->ln_stats = reinterpret_cast<float2 *>(next(i++));
+  p->mix_ccol = reinterpret_cast<float *>(next(i++));
 
   st = L3_OK;
   e = cudaMemsetAsync(p->dev_flags, 0, 64, s);
@@ -459,7 +463,8 @@ l3_status l3_forward(const void *x, l3_plan_t p, const void *W_K, const void *W_
     // and bandwidth from it (paper_shaped: 1.64 -> 1.72 ms per batch); with
     // no such launch they spread over all three (small_bf16: 0.41 -> 0.34 ms)
     if (st == L3_OK) st = launch_attn_tail_cls(p, x, W_K, W_V, aux->stream, has_big ? 1 : N_AUX);
-    if (st == L3_OK && p->tc_gemm) st = launch_weights_f16(p, W_up, W_mix, aux->stream[0]);
+    if (st == L3_OK && p->tc_gemm)
+      st = launch_weights_f16(p, W_up, W_mix, ln_gamma, ln_beta, aux->stream[0]);
     for (int i = 0; i < N_AUX; ++i) {
       L3_CUDA_TRY(cudaEventRecord(aux->join[i], aux->stream[i]));
       L3_CUDA_TRY(cudaStreamWaitEvent(s, aux->join[i], 0));
@@ -468,14 +473,14 @@ l3_status l3_forward(const void *x, l3_plan_t p, const void *W_K, const void *W_
     st = launch_attn_tail(p, x, W_K, W_V, s);
     if (st == L3_OK) st = launch_attn_dense(p, x, W_K, W_V, false, s);
     if (st == L3_OK) st = launch_attn_dense(p, x, W_K, W_V, true, s);
-    if (st == L3_OK && p->tc_gemm) st = launch_weights_f16(p, W_up, W_mix, s);
+    if (st == L3_OK && p->tc_gemm) st = launch_weights_f16(p, W_up, W_mix, ln_gamma, ln_beta, s);
   } else {
     if (st == L3_OK) st = launch_attn_dense(p, x, W_K, W_V, false, s);
     if (st == L3_OK) st = launch_attn_dense(p, x, W_K, W_V, true, s);
-    if (st == L3_OK && p->tc_gemm) st = launch_weights_f16(p, W_up, W_mix, s);
+    if (st == L3_OK && p->tc_gemm) st = launch_weights_f16(p, W_up, W_mix, ln_gamma, ln_beta, s);
   }
   if (p->tc_gemm) {
-    if (st == L3_OK) st = launch_up_ln_tc(p, ln_gamma, ln_beta, s);
+    if (st == L3_OK) st = launch_up_z_tc(p, s);
     if (st == L3_OK) st = launch_mix_tc(p, x, W_mix, y, s);
   } else {
     if (st == L3_OK) st = launch_up_ln_simt(p, W_up, ln_gamma, ln_beta, s);
@@ -498,8 +503,9 @@ l3_status l3_forward_status(l3_plan_t p) {
     return L3_ERR_TIMEOUT;
   }
   if (flags[1] & DEV_ERR_F16_RANGE) {
-    set_error("W_up or W_mix holds a value outside fp16's finite range (|w| > 65504), which "
-              "the bf16 layer's fp16 intermediate GEMMs cannot represent");
+    set_error("W_up, W_mix[:, :d_up] diag(ln_gamma) or z = W_up a holds a value outside "
+              "fp16's finite range (|v| > 65504), which the bf16 layer's fp16 intermediate "
+              "GEMMs cannot represent");
     return L3_ERR_UNSUPPORTED;
   }
   return L3_OK;

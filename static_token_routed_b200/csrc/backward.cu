@@ -118,15 +118,43 @@ l3_status gemm(Operand A, Operand B, int M, int N, int K, float *C, int64_t ldc,
 // last store of a row may run into out's padding up to ld_out).
 constexpr int TT = 64;
 
+// With `ln` set, each input row r is z of the tensor-core forward and is
+// normalised on the way, out[c][r] = gamma[c] (z[r][c] - mean_r) / std_r + beta[c],
+// from the forward's per-256-column (mean, M2) of each row.
+struct LnApply {
+  const float2 *stats;  // [R][n_chunks], nullptr: plain transpose
+  int n_chunks;
+  const void *gamma, *beta;
+  int wtype;  // weight type of gamma / beta
+  float eps;
+};
+
 template <typename Tin>
 __global__ void __launch_bounds__(256)
     k_transpose_bf16(const Tin *__restrict__ in, int64_t ld_in, int64_t R, int64_t C,
-                     __nv_bfloat16 *__restrict__ out, int64_t ld_out) {
+                     __nv_bfloat16 *__restrict__ out, int64_t ld_out, LnApply ln) {
   __shared__ float tile[TT][TT + 1];
+  __shared__ float row_mu[TT], row_rs[TT];
   const int64_t tiles_c = (C + TT - 1) / TT, n_tiles = tiles_c * ((R + TT - 1) / TT);
   const int tid = threadIdx.x;
   for (int64_t t = blockIdx.x; t < n_tiles; t += gridDim.x) {
     const int64_t r0 = (t / tiles_c) * TT, c0 = (t % tiles_c) * TT;
+    if (ln.stats) {
+      if (tid < TT && r0 + tid < R) {
+        float n = 0.f, mean = 0.f, m2 = 0.f;
+        for (int k = 0; k < ln.n_chunks; ++k) {
+          const float2 st = ln.stats[(r0 + tid) * ln.n_chunks + k];
+          const float nb = (float)min((int64_t)256, C - 256 * k);
+          const float nn = n + nb, dl = st.x - mean;
+          mean += dl * (nb / nn);
+          m2 += st.y + dl * dl * (n * nb / nn);
+          n = nn;
+        }
+        row_mu[tid] = mean;
+        row_rs[tid] = rsqrtf(m2 / n + ln.eps);
+      }
+      __syncthreads();
+    }
     // load: 8 threads per 64-element row, 32 rows per pass
     for (int rr = tid / 8; rr < TT; rr += 32) {
       const int cc = (tid % 8) * 8;
@@ -137,6 +165,11 @@ __global__ void __launch_bounds__(256)
         const Tin *e = reinterpret_cast<const Tin *>(&u);
 #pragma unroll
         for (int i = 0; i < 8; ++i) f[i] = static_cast<float>(e[i]);
+        if (ln.stats)
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            f[i] = ldx(ln.gamma, ln.wtype, c + i) * ((f[i] - row_mu[rr]) * row_rs[rr]) +
+                   ldx(ln.beta, ln.wtype, c + i);
       } else {
 #pragma unroll
         for (int i = 0; i < 8; ++i) f[i] = 0.f;
@@ -164,12 +197,12 @@ __global__ void __launch_bounds__(256)
 
 template <typename Tin>
 l3_status transpose_bf16(const void *in, int64_t ld_in, int64_t R, int64_t C, void *out,
-                         int64_t ld_out, int n_sms, cudaStream_t s) {
+                         int64_t ld_out, int n_sms, cudaStream_t s, LnApply ln = {}) {
   if (R == 0 || C == 0) return L3_OK;
   const int64_t n_tiles = ((R + TT - 1) / TT) * ((C + TT - 1) / TT);
   const unsigned grid = (unsigned)std::min<int64_t>(n_tiles, (int64_t)n_sms * 8);
   k_transpose_bf16<Tin><<<grid, 256, 0, s>>>(reinterpret_cast<const Tin *>(in), ld_in, R, C,
-                                             reinterpret_cast<__nv_bfloat16 *>(out), ld_out);
+                                             reinterpret_cast<__nv_bfloat16 *>(out), ld_out, ln);
   L3_CUDA_TRY(cudaGetLastError());
   return L3_OK;
 }
@@ -947,10 +980,9 @@ extern "C" l3_status l3_backward(const void *x, l3_plan_t p, const void *W_K, co
     set_error("plan is NULL");
     return L3_ERR_INVALID_ARG;
   }
-  (void)ln_beta;  // beta shifts h, which the forward stored; no step below reads it
   const l3_dims_t &d = p->dims;
   const int64_t N = p->n_tokens;
-  for (const void *q : {x, W_K, W_V, W_up, ln_gamma, W_mix, dy, (const void *)dx,
+  for (const void *q : {x, W_K, W_V, W_up, ln_gamma, ln_beta, W_mix, dy, (const void *)dx,
                         (const void *)dW_K, (const void *)dW_V, (const void *)dW_up,
                         (const void *)dgamma, (const void *)dbeta, (const void *)dW_mix})
     if (!q) {
@@ -1060,7 +1092,11 @@ extern "C" l3_status l3_backward(const void *x, l3_plan_t p, const void *W_K, co
     LaunchTimer t("bwd_transpose", s);
     if (st == L3_OK) st = transpose_bf16<BF>(W_mix, D, d.d_out, D, wmt, d.d_out, n_sms, s);
     if (st == L3_OK) st = transpose_bf16<BF>(dy, d.d_out, N, d.d_out, gyt, ldn, n_sms, s);
-    if (st == L3_OK) st = transpose_bf16<__half>(p->h_buf, d.d_up, N, d.d_up, hxt, ldn, n_sms, s);
+    // the tensor-core forward keeps z, not h: normalise it on the way (its
+    // per-256-column statistics are the forward's)
+    LnApply ln{p->ln_stats, (int)((d.d_up + 255) / 256), ln_gamma, ln_beta, wt, d.ln_eps};
+    if (st == L3_OK)
+      st = transpose_bf16<__half>(p->h_buf, d.d_up, N, d.d_up, hxt, ldn, n_sms, s, ln);
     if (st == L3_OK)
       st = transpose_bf16<BF>(x, d.d_in, N, d.d_in, hxt + d.d_up * ldn, ldn, n_sms, s);
     if (st == L3_OK) st = transpose_bf16<BF>(W_up, d.d_emb, d.d_up, d.d_emb, wut, d.d_up, n_sms, s);

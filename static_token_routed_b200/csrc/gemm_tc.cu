@@ -43,26 +43,22 @@ constexpr int BN = 256;  // output columns per tile (max N of one MMA)
 constexpr int A_BYTES = BM * BK * 2;
 constexpr int B_BYTES = BN * BK * 2;
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-constexpr int UP_STAGES = 2;  // two CTAs per SM: one drains its epilogue while the other computes
 constexpr int GEMM_THREADS = 192;  // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
 constexpr uint32_t IDESC_F16 = idesc_f16(0, 0, BM, BN);
 
 struct MixParams {
-  int M, N;        // tokens, d_out
-  int kb0, kb1;    // 64-wide k-blocks of the h range and of the x range
+  int M, N;        // rows (tokens), output columns
+  int kb0, kb1;    // 64-wide k-blocks of the first range (z, or A) and of the second (x, or A1)
   int n_tiles_n, n_tiles;
-  void *y;         // bf16 (the layer's y) or fp32 (the backward pass's GEMMs)
+  void *y;         // bf16 y (MODE_MIX_LN), fp32 C (MODE_F32) or fp16 z (MODE_UP_Z)
   int64_t ldy;
-  uint32_t idesc0, idesc1;  // instruction descriptors of the two ranges (fp32-output form)
-  int *err;
-};
-
-struct UpParams {
-  int M, N;        // tokens, d_up
-  int kb;          // k-blocks of d_emb
-  const __nv_bfloat16 *gamma, *beta;
+  uint32_t idesc0, idesc1;  // instruction descriptors of the two ranges (MODE_F32)
+  // MODE_UP_Z writes, MODE_MIX_LN reads: (mean, M2) of each row over each
+  // 256-column tile of z, [M][n_chunks]
+  float2 *stats;
+  int n_chunks;
+  const float *ccol, *dcol;  // MODE_MIX_LN: c = W' 1 and d = W_mix[:, :d_up] beta, [N] each
   float eps;
-  __half *h;
   int *err;
 };
 
@@ -164,21 +160,117 @@ __device__ __forceinline__ void umma_commit_pair(uint64_t *bar) {
       : "memory");
 }
 
-template <bool F32OUT>
+// (n_a, mean_a, M2_a) <- (n_a, mean_a, M2_a) (+) (n_b, mean_b, M2_b): Chan,
+// Golub and LeVeque's pairwise update of a mean and a sum of squared deviations
+__device__ __forceinline__ void chan_merge(float &n_a, float &mean_a, float &m2_a, float n_b,
+                                           float mean_b, float m2_b) {
+  const float n = n_a + n_b;
+  if (n_b == 0.f) return;
+  const float delta = mean_b - mean_a;
+  mean_a += delta * (n_b / n);
+  m2_a += m2_b + delta * delta * (n_a * n_b / n);
+  n_a = n;
+}
+
+// Kernel forms:
+//   MODE_F32:    C = A B^T (+ A1 B1^T), fp32 output (the backward pass's GEMMs)
+//   MODE_UP_Z:   z = a W_up^T, fp16 output through shared memory and TMA stores,
+//                plus each row's (mean, M2) over each 256-column tile of z
+//   MODE_MIX_LN: y = W_mix [LayerNorm(z) ; x] with the LayerNorm folded into the
+//                accumulator (see below)
+//
+// MODE_MIX_LN. With W' = W_mix[:, :d_up] diag(gamma), c = W' 1 and
+// d = W_mix[:, :d_up] beta, for a row with mean mu and 1 / std r,
+//     W_mix[:, :d_up] LayerNorm(z) = r (W' z - mu c) + d,
+// so the kernel accumulates W' z over the z range, the epilogue warps rewrite
+// that accumulator in TMEM as r (acc - mu c) + d, and the x range then
+// accumulates W_mix[:, d_up:] x on top. To keep the tensor cores busy while a
+// tile's accumulator is being rewritten, a pair runs its tiles two at a time:
+//     z(t) -> acc 0, z(t+1) -> acc 1, x(t) -> acc 0, x(t+1) -> acc 1
+// and the epilogue warps follow: rewrite t, rewrite t+1, store t, store t+1.
+enum : int { MODE_F32 = 0, MODE_UP_Z = 1, MODE_MIX_LN = 2 };
+
+template <int MODE>
+struct MixCfg {
+  static constexpr int STAGES = MODE == MODE_UP_Z ? 4 : MIX2_STAGES;
+  // MODE_UP_Z: 128 rows x 256 columns of fp16 z, four 64-column TMA boxes
+  static constexpr int STAGING = MODE == MODE_UP_Z ? (BN / 64) * BM * 128 : 0;
+};
+
+// The j-th (tile, range, accumulator) job of a pair that owns `k_tiles`
+// tiles; false past the last. Ranges: 0 = the first k-range (or both, when
+// the kernel does not split them), 1 = the second.
+template <int MODE>
+__device__ __forceinline__ bool mix_job(int j, int k_tiles, int &k, int &rng, int &acc) {
+  if (MODE != MODE_MIX_LN) {
+    if (j >= k_tiles) return false;
+    k = j;
+    rng = 0;
+    acc = j & 1;
+    return true;
+  }
+  const int n_full = k_tiles / 2;
+  if (j < 4 * n_full) {
+    const int w = j & 3;
+    k = 2 * (j >> 2) + (w & 1);
+    rng = w >> 1;
+    acc = w & 1;
+    return true;
+  }
+  const int j2 = j - 4 * n_full;
+  if ((k_tiles & 1) && j2 < 2) {
+    k = 2 * n_full;
+    rng = j2;
+    acc = 0;
+    return true;
+  }
+  return false;
+}
+
+// barriers of the four epilogue warps (128 threads): a plain one, and one
+// that ANDs a flag across them so that they leave their loop together
+__device__ __forceinline__ void epi_bar_sync() {
+  asm volatile("bar.sync 1, 128;" ::: "memory");
+}
+__device__ __forceinline__ bool epi4_sync_and(bool ok) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 q, %1, 0;\n\t"
+      "bar.red.and.pred p, 2, 128, q;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(r)
+      : "r"((uint32_t)ok)
+      : "memory");
+  return r != 0;
+}
+__device__ __forceinline__ void tma_store_2d_box(const CUtensorMap *map, const void *src, int x,
+                                                 int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(map),
+      "r"(smem_u32(src)), "r"(x), "r"(y)
+      : "memory");
+}
+
+template <int MODE>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
     k_mix_gemm_pair(const __grid_constant__ CUtensorMap mA0, const __grid_constant__ CUtensorMap mB0,
                     const __grid_constant__ CUtensorMap mA1, const __grid_constant__ CUtensorMap mB1,
-                    MixParams P) {
+                    const __grid_constant__ CUtensorMap mZ, MixParams P) {
+  using Cfg = MixCfg<MODE>;
+  constexpr int STAGES = Cfg::STAGES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = align1024(smem_raw);
   uint8_t *ring = smem;
-  Bars *b = reinterpret_cast<Bars *>(smem + MIX2_STAGES * STAGE2_BYTES);
+  uint8_t *staging = smem + STAGES * STAGE2_BYTES;  // MODE_UP_Z
+  Bars *b = reinterpret_cast<Bars *>(staging + Cfg::STAGING);
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const uint32_t rank = cluster_ctarank();  // 0 issues the MMAs
   const int pair_id = blockIdx.x / 2, n_pairs = gridDim.x / 2;
+  const int k_tiles = P.n_tiles > pair_id ? (P.n_tiles - pair_id + n_pairs - 1) / n_pairs : 0;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < MIX2_STAGES; ++s) {
+    for (int s = 0; s < STAGES; ++s) {
       mbar_init(&b->full[s], 2);   // used in CTA 0: one arrival per CTA, plus both CTAs' bytes
       mbar_init(&b->empty[s], 1);  // MMA completion, signalled in both CTAs
     }
@@ -207,20 +299,24 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   tc_fence_after();
   const uint32_t tmem = b->tmem_base;
   const Abort ab{&b->abort_flag, P.err};
-  const int n_kb = P.kb0 + P.kb1;
+  // k-blocks of a job's range
+  auto job_kb = [&](int rng) { return MODE == MODE_MIX_LN ? (rng ? P.kb1 : P.kb0) : P.kb0 + P.kb1; };
 
   if (warp == 0) {
     if (elect_one()) {
       int stage = 0;
       uint32_t phase = 0;
-      uint32_t armed_parity[MIX2_STAGES];
-      bool armed[MIX2_STAGES];
-      for (int s = 0; s < MIX2_STAGES; ++s) armed[s] = false;
+      uint32_t armed_parity[STAGES];
+      bool armed[STAGES];
+      for (int s = 0; s < STAGES; ++s) armed[s] = false;
       bool ok = true;
-      for (int tile = pair_id; ok && tile < P.n_tiles; tile += n_pairs) {
+      int k, rng, acc;
+      for (int j = 0; ok && mix_job<MODE>(j, k_tiles, k, rng, acc); ++j) {
+        const int tile = pair_id + k * n_pairs;
         const int m0 = (tile / P.n_tiles_n) * (2 * BM) + (int)rank * BM;
         const int n0 = (tile % P.n_tiles_n) * BN + (int)rank * B2_ROWS;
-        for (int kb = 0; kb < n_kb; ++kb) {
+        const int nkb = job_kb(rng);
+        for (int kb = 0; kb < nkb; ++kb) {
           if (!mbar_wait(&b->empty[stage], phase ^ 1, ab)) {
             ok = false;
             break;
@@ -230,14 +326,17 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           mbar_arrive_expect_tx_cluster(full0, STAGE2_BYTES);
           armed[stage] = true;
           armed_parity[stage] = phase;
-          if (kb < P.kb0) {
-            tma_load_2d_pair(sa, &mA0, full0, kb * BK, m0);
-            tma_load_2d_pair(sa + A_BYTES, &mB0, full0, kb * BK, n0);
+          // the first range: A0 / B0 (z / W', or A / B); the second: A1 / B1
+          const bool first = MODE == MODE_MIX_LN ? rng == 0 : kb < P.kb0;
+          const int kk = MODE == MODE_MIX_LN ? kb : (first ? kb : kb - P.kb0);
+          if (first) {
+            tma_load_2d_pair(sa, &mA0, full0, kk * BK, m0);
+            tma_load_2d_pair(sa + A_BYTES, &mB0, full0, kk * BK, n0);
           } else {
-            tma_load_2d_pair(sa, &mA1, full0, (kb - P.kb0) * BK, m0);
-            tma_load_2d_pair(sa + A_BYTES, &mB1, full0, (kb - P.kb0) * BK, n0);
+            tma_load_2d_pair(sa, &mA1, full0, kk * BK, m0);
+            tma_load_2d_pair(sa + A_BYTES, &mB1, full0, kk * BK, n0);
           }
-          if (++stage == MIX2_STAGES) {
+          if (++stage == STAGES) {
             stage = 0;
             phase ^= 1;
           }
@@ -245,23 +344,27 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       }
       // after a give-up CTA 0 waits for the phases it armed, which complete
       // only once both CTAs' copies have landed
-      if (!ok && rank == 0) drain_after_abort(b, MIX2_STAGES, armed_parity, armed, true, false, ab);
+      if (!ok && rank == 0) drain_after_abort(b, STAGES, armed_parity, armed, true, false, ab);
     }
   } else if (warp == 1) {
     if (rank == 0 && elect_one()) {
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
-      int it = 0;
-      for (int tile = pair_id; ok && tile < P.n_tiles; tile += n_pairs, ++it) {
-        const int acc = it & 1;
-        if (!mbar_wait(&b->tempty[acc], ((it >> 1) & 1) ^ 1, ab)) {
+      int n_acc[2] = {0, 0};  // jobs run so far on each accumulator
+      int k, rng, acc;
+      for (int j = 0; ok && mix_job<MODE>(j, k_tiles, k, rng, acc); ++j) {
+        const int na = acc ? n_acc[1] : n_acc[0];
+        if (acc) ++n_acc[1]; else ++n_acc[0];
+        // the epilogue has finished with this accumulator's previous job
+        if (!mbar_wait(&b->tempty[acc], (na & 1) ^ 1, ab)) {
           ok = false;
           break;
         }
         tc_fence_after();
         const uint32_t d = tmem + acc * BN;
-        for (int kb = 0; kb < n_kb; ++kb) {
+        const int nkb = job_kb(rng);
+        for (int kb = 0; kb < nkb; ++kb) {
           if (!mbar_wait(&b->full[stage], phase, ab)) {
             ok = false;
             break;
@@ -269,14 +372,18 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           tc_fence_after();
           const uint32_t sa = smem_u32(ring + stage * STAGE2_BYTES);
           const uint32_t sb = sa + A_BYTES;
-          const uint32_t idesc = F32OUT ? (kb < P.kb0 ? P.idesc0 : P.idesc1)
-                                        : (kb < P.kb0 ? IDESC2_F16 : IDESC2_BF16);
+          const bool first = MODE == MODE_MIX_LN ? rng == 0 : kb < P.kb0;
+          const uint32_t idesc = MODE == MODE_F32 ? (first ? P.idesc0 : P.idesc1)
+                                 : MODE == MODE_UP_Z ? IDESC2_F16
+                                                     : (first ? IDESC2_F16 : IDESC2_BF16);
+          // the x range adds onto the rewritten z-range accumulator
+          const bool fresh = MODE == MODE_MIX_LN ? rng == 0 && kb == 0 : kb == 0;
 #pragma unroll
-          for (int k = 0; k < BK / 16; ++k)
-            umma_f16_pair(d, sdesc_sw128(sa + k * 32, 16, 1024), sdesc_sw128(sb + k * 32, 16, 1024),
-                          idesc, (kb | k) != 0);
+          for (int kq = 0; kq < BK / 16; ++kq)
+            umma_f16_pair(d, sdesc_sw128(sa + kq * 32, 16, 1024),
+                          sdesc_sw128(sb + kq * 32, 16, 1024), idesc, !(fresh && kq == 0));
           umma_commit_pair(&b->empty[stage]);
-          if (++stage == MIX2_STAGES) {
+          if (++stage == STAGES) {
             stage = 0;
             phase ^= 1;
           }
@@ -293,46 +400,145 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     }
   } else {
     // epilogue: warp (2..5) % 4 selects the TMEM lane quarter it may read;
-    // each CTA drains its own 128 rows of the pair's tile
+    // each CTA handles its own 128 rows of the pair's tile
     const int q = warp & 3;
     const int r = q * 32 + lane;
     const uint32_t tempty0[2] = {map_shared_rank(&b->tempty[0], 0),
                                  map_shared_rank(&b->tempty[1], 0)};
-    int it = 0;
-    for (int tile = pair_id; tile < P.n_tiles; tile += n_pairs, ++it) {
-      const int acc = it & 1;
-      const bool got = __all_sync(0xffffffffu, mbar_wait(&b->tfull[acc], (it >> 1) & 1, ab));
+    int n_acc[2] = {0, 0};
+    int k, rng, acc;
+    bool stored = false;  // MODE_UP_Z: a TMA store may still be reading the staging buffer
+    for (int j = 0; mix_job<MODE>(j, k_tiles, k, rng, acc); ++j) {
+      const int na = acc ? n_acc[1] : n_acc[0];
+      if (acc) ++n_acc[1]; else ++n_acc[0];
+      bool got = __all_sync(0xffffffffu, mbar_wait(&b->tfull[acc], na & 1, ab));
+      // MODE_UP_Z's warps meet at named barriers below: they leave together
+      if (MODE == MODE_UP_Z) got = epi4_sync_and(got);
       if (!got) break;
       tc_fence_after();
+      const int tile = pair_id + k * n_pairs;
       const int m = (tile / P.n_tiles_n) * (2 * BM) + (int)rank * BM + r;
       const int n0 = (tile % P.n_tiles_n) * BN;
-      __nv_bfloat16 *yrow = reinterpret_cast<__nv_bfloat16 *>(P.y) + (int64_t)m * P.ldy + n0;
-      float *crow = reinterpret_cast<float *>(P.y) + (int64_t)m * P.ldy + n0;
-#pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
-        uint32_t v[32];
-        tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + acc * BN + c * 32, v);
-        tmem_wait_ld();
-        if (F32OUT) {
-          if (m < P.M) {
-#pragma unroll
-            for (int j = 0; j < 8; ++j)
-              if (n0 + c * 32 + j * 4 < P.N)
-                *reinterpret_cast<uint4 *>(crow + c * 32 + j * 4) =
-                    make_uint4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+      const uint32_t tacc = tmem + ((uint32_t)(q * 32) << 16) + acc * BN;
+      if (MODE == MODE_MIX_LN && rng == 0) {
+        // rewrite the z-range accumulator as r (acc - mu c) + d
+        float n_acc_f = 0.f, mean = 0.f, m2 = 0.f;
+        if (m < P.M)
+          for (int c = 0; c < P.n_chunks; ++c) {
+            const float2 st = P.stats[(int64_t)m * P.n_chunks + c];
+            chan_merge(n_acc_f, mean, m2, (float)min(BN, P.kb0 * BK - c * BN), st.x, st.y);
           }
-        } else if (m < P.M) {
+        const float rs = m < P.M ? rsqrtf(m2 / n_acc_f + P.eps) : 0.f;
+        const float mr = mean * rs;
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+          uint32_t v[32];
+          tmem_ld32(tacc + c * 32, v);
+          tmem_wait_ld();
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const int col = n0 + c * 32 + j * 8;
-            if (col < P.N) {
-              uint4 o;
-              __nv_bfloat162 *o2 = reinterpret_cast<__nv_bfloat162 *>(&o);
+          for (int e = 0; e < 32; e += 4) {
+            const int col = n0 + c * 32 + e;
+            const float4 cc = col < P.N ? __ldg(reinterpret_cast<const float4 *>(P.ccol + col))
+                                        : make_float4(0.f, 0.f, 0.f, 0.f);
+            const float4 dd = col < P.N ? __ldg(reinterpret_cast<const float4 *>(P.dcol + col))
+                                        : make_float4(0.f, 0.f, 0.f, 0.f);
+            v[e] = __float_as_uint(fmaf(__uint_as_float(v[e]), rs, fmaf(-mr, cc.x, dd.x)));
+            v[e + 1] = __float_as_uint(fmaf(__uint_as_float(v[e + 1]), rs, fmaf(-mr, cc.y, dd.y)));
+            v[e + 2] = __float_as_uint(fmaf(__uint_as_float(v[e + 2]), rs, fmaf(-mr, cc.z, dd.z)));
+            v[e + 3] = __float_as_uint(fmaf(__uint_as_float(v[e + 3]), rs, fmaf(-mr, cc.w, dd.w)));
+          }
+          tmem_st32(tacc + c * 32, v);
+        }
+        tmem_wait_st();
+      } else if (MODE == MODE_UP_Z) {
+        // z tile: per-row (mean, M2) in 32-column chunks merged in order, and
+        // the fp16 values into the staging boxes (128-byte swizzle)
+        if (stored) {
+          if (warp == 2 && lane == 0) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+          epi_bar_sync();
+        }
+        const int nv = min(BN, P.N - n0);
+        float n_acc_f = 0.f, mean = 0.f, m2 = 0.f;
+        bool range_ok = true;
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+          uint32_t v[32];
+          tmem_ld32(tacc + c * 32, v);
+          tmem_wait_ld();
+          const int cv = min(32, nv - c * 32);
+          if (cv > 0) {
+            float sum = 0.f;
 #pragma unroll
-              for (int e = 0; e < 4; ++e)
-                o2[e] = __floats2bfloat162_rn(__uint_as_float(v[j * 8 + 2 * e]),
-                                              __uint_as_float(v[j * 8 + 2 * e + 1]));
-              *reinterpret_cast<uint4 *>(yrow + c * 32 + j * 8) = o;
+            for (int e = 0; e < 32; ++e)
+              if (e < cv) sum += __uint_as_float(v[e]);
+            const float mc = sum / (float)cv;
+            float qc = 0.f;
+#pragma unroll
+            for (int e = 0; e < 32; ++e)
+              if (e < cv) {
+                const float dl = __uint_as_float(v[e]) - mc;
+                qc = fmaf(dl, dl, qc);
+              }
+            chan_merge(n_acc_f, mean, m2, (float)cv, mc, qc);
+          }
+          uint8_t *box = staging + (c / 2) * (BM * 128);
+#pragma unroll
+          for (int jj = 0; jj < 4; ++jj) {
+            uint4 o;
+            __half2 *o2 = reinterpret_cast<__half2 *>(&o);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float z0 = __uint_as_float(v[jj * 8 + 2 * e]);
+              const float z1 = __uint_as_float(v[jj * 8 + 2 * e + 1]);
+              range_ok &= fabsf(z0) <= 65504.f && fabsf(z1) <= 65504.f;
+              o2[e] = __floats2half2_rn(z0, z1);
+            }
+            const int chunk = (c % 2) * 4 + jj;  // 16-byte chunk within the box's 128-byte row
+            *reinterpret_cast<uint4 *>(box + r * 128 + ((chunk ^ (r & 7)) << 4)) = o;
+          }
+        }
+        if (m < P.M) {
+          P.stats[(int64_t)m * P.n_chunks + n0 / BN] = make_float2(mean, m2);
+          if (!range_ok) atomicOr(P.err, DEV_ERR_F16_RANGE);
+        }
+        fence_proxy_async_smem();
+        epi_bar_sync();
+        if (warp == 2 && lane == 0) {
+          const int mrow = (tile / P.n_tiles_n) * (2 * BM) + (int)rank * BM;
+          for (int bx = 0; bx * 64 < nv; ++bx)
+            tma_store_2d_box(&mZ, staging + bx * (BM * 128), n0 + bx * 64, mrow);
+          asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+        }
+        stored = true;
+      } else {
+        __nv_bfloat16 *yrow = reinterpret_cast<__nv_bfloat16 *>(P.y) + (int64_t)m * P.ldy + n0;
+        float *crow = reinterpret_cast<float *>(P.y) + (int64_t)m * P.ldy + n0;
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+          uint32_t v[32];
+          tmem_ld32(tacc + c * 32, v);
+          tmem_wait_ld();
+          if (MODE == MODE_F32) {
+            if (m < P.M) {
+#pragma unroll
+              for (int jj = 0; jj < 8; ++jj)
+                if (n0 + c * 32 + jj * 4 < P.N)
+                  *reinterpret_cast<uint4 *>(crow + c * 32 + jj * 4) =
+                      make_uint4(v[4 * jj], v[4 * jj + 1], v[4 * jj + 2], v[4 * jj + 3]);
+            }
+          } else if (m < P.M) {
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) {
+              const int col = n0 + c * 32 + jj * 8;
+              if (col < P.N) {
+                uint4 o;
+                __nv_bfloat162 *o2 = reinterpret_cast<__nv_bfloat162 *>(&o);
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                  o2[e] = __floats2bfloat162_rn(__uint_as_float(v[jj * 8 + 2 * e]),
+                                                __uint_as_float(v[jj * 8 + 2 * e + 1]));
+                *reinterpret_cast<uint4 *>(yrow + c * 32 + jj * 8) = o;
+              }
             }
           }
         }
@@ -341,6 +547,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(tempty0[acc]);
     }
+    if (MODE == MODE_UP_Z && stored && warp == 2 && lane == 0)
+      asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
   }
   __syncwarp();
   tc_fence_before();
@@ -350,282 +558,6 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(2 * BN)
                  : "memory");
-  }
-}
-
-// ---------------------------------------------------------------------------
-// h = LayerNorm(W_up a), one cluster of ceil(d_up / 256) CTAs per 128 tokens
-// ---------------------------------------------------------------------------
-constexpr int UP_THREADS = 320;  // warp 0 TMA, warp 1 MMA, warps 2-9 epilogue
-
-// barrier of the 256 epilogue threads of k_up_ln_gemm that ANDs a flag across them
-__device__ __forceinline__ bool epi_sync_and(bool ok) {
-  uint32_t r;
-  asm volatile(
-      "{\n\t.reg .pred p, q;\n\t"
-      "setp.ne.u32 q, %1, 0;\n\t"
-      "bar.red.and.pred p, 1, 256, q;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}\n"
-      : "=r"(r)
-      : "r"((uint32_t)ok)
-      : "memory");
-  return r != 0;
-}
-
-// (n_a, mean_a, M2_a) <- (n_a, mean_a, M2_a) (+) (n_b, mean_b, M2_b): Chan,
-// Golub and LeVeque's pairwise update of a mean and a sum of squared deviations
-__device__ __forceinline__ void chan_merge(float &n_a, float &mean_a, float &m2_a, float n_b,
-                                           float mean_b, float m2_b) {
-  const float n = n_a + n_b;
-  if (n_b == 0.f) return;
-  const float delta = mean_b - mean_a;
-  mean_a += delta * (n_b / n);
-  m2_a += m2_b + delta * delta * (n_a * n_b / n);
-  n_a = n;
-}
-
-__device__ __forceinline__ void st_shared_cluster_f32(uint32_t addr, float v) {
-  asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
-}
-__device__ __forceinline__ void cluster_arrive_relaxed() {
-  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void cluster_arrive_release() {
-  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void cluster_wait_acquire() {
-  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, const void *src, int x,
-                                             int y) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(map),
-      "r"(smem_u32(src)), "r"(x), "r"(y)
-      : "memory");
-}
-__device__ __forceinline__ void bulk_commit_and_wait_all() {
-  asm volatile("cp.async.bulk.commit_group;\n\tcp.async.bulk.wait_group 0;" ::: "memory");
-}
-
-__global__ void __launch_bounds__(UP_THREADS, 2)
-    k_up_ln_gemm(const __grid_constant__ CUtensorMap mA, const __grid_constant__ CUtensorMap mB,
-                 const __grid_constant__ CUtensorMap mH, UpParams P) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t *smem = align1024(smem_raw);
-  uint8_t *ring = smem;
-  Bars *b = reinterpret_cast<Bars *>(smem + UP_STAGES * STAGE_BYTES);
-  float *g_s = reinterpret_cast<float *>(b + 1);  // gamma of this CTA's 256 columns
-  float *b_s = g_s + BN;                          // beta
-  float(*red)[BM] = reinterpret_cast<float(*)[BM]>(b_s + BN);  // [4][BM]: mean, M2 of two halves
-  // [2][8][BM]: every slice's (mean, M2) per row, written by the cluster's CTAs
-  float(*st_all)[8][BM] = reinterpret_cast<float(*)[8][BM]>(red[4]);
-  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const uint32_t rank = cluster_ctarank();
-  const uint32_t n_ranks = gridDim.x;  // one cluster spans the grid's x dimension
-  const int m0 = blockIdx.y * BM;
-  const int n0 = (int)rank * BN;
-  const int n_valid = min(BN, P.N - n0);
-
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < UP_STAGES; ++s) {
-      mbar_init(&b->full[s], 1);
-      mbar_init(&b->empty[s], 1);
-    }
-    mbar_init(&b->tfull[0], 1);
-    mbar_init(&b->drain, 1);
-    b->abort_flag = 0;
-    fence_mbar_init();
-    prefetch_tensormap(&mA);
-    prefetch_tensormap(&mB);
-  }
-  if (warp == 1) {
-    tmem_alloc(&b->tmem_base, BN);
-    tmem_relinquish();
-  }
-  for (int i = threadIdx.x; i < BN; i += UP_THREADS) {
-    const bool v = n0 + i < P.N;
-    g_s[i] = v ? __bfloat162float(P.gamma[n0 + i]) : 0.f;
-    b_s[i] = v ? __bfloat162float(P.beta[n0 + i]) : 0.f;
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  // first phase of the cluster barrier: every CTA of the cluster has started
-  // before any writes into another's shared memory (waited on before that)
-  cluster_arrive_relaxed();
-  const uint32_t tmem = b->tmem_base;
-  const Abort ab{&b->abort_flag, P.err};
-
-  if (warp == 0) {
-    if (elect_one()) {
-      uint32_t armed_parity[UP_STAGES];
-      bool armed[UP_STAGES];
-      for (int s = 0; s < UP_STAGES; ++s) armed[s] = false;
-      int stage = 0;
-      uint32_t phase = 0;
-      bool ok = true;
-      for (int kb = 0; kb < P.kb; ++kb) {
-        if (!mbar_wait(&b->empty[stage], phase ^ 1, ab)) {
-          ok = false;
-          break;
-        }
-        uint8_t *sa = ring + stage * STAGE_BYTES;
-        mbar_arrive_expect_tx(&b->full[stage], STAGE_BYTES);
-        armed[stage] = true;
-        armed_parity[stage] = phase;
-        tma_load_2d(sa, &mA, &b->full[stage], kb * BK, m0);
-        tma_load_2d(sa + A_BYTES, &mB, &b->full[stage], kb * BK, n0);
-        if (++stage == UP_STAGES) {
-          stage = 0;
-          phase ^= 1;
-        }
-      }
-      if (!ok) drain_after_abort(b, UP_STAGES, armed_parity, armed, true, false, ab);
-    }
-  } else if (warp == 1) {
-    if (elect_one()) {
-      int stage = 0;
-      uint32_t phase = 0;
-      bool ok = true;
-      for (int kb = 0; kb < P.kb; ++kb) {
-        if (!mbar_wait(&b->full[stage], phase, ab)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const uint32_t sa = smem_u32(ring + stage * STAGE_BYTES);
-        const uint32_t sb = sa + A_BYTES;
-#pragma unroll
-        for (int k = 0; k < BK / 16; ++k)
-          umma_f16(tmem, sdesc_sw128(sa + k * 32, 16, 1024), sdesc_sw128(sb + k * 32, 16, 1024),
-                   IDESC_F16, (kb | k) != 0);
-        umma_commit(&b->empty[stage]);
-        if (++stage == UP_STAGES) {
-          stage = 0;
-          phase ^= 1;
-        }
-      }
-      if (ok) umma_commit(&b->tfull[0]);
-      else drain_after_abort(b, UP_STAGES, nullptr, nullptr, false, true, ab);
-    }
-  }
-
-  // epilogue part 1: per-row (mean, M2) of this CTA's slice in one pass over
-  // TMEM. Warps 2-9, two per TMEM lane quarter; each takes every other
-  // 32-column chunk, takes each chunk's exact mean and M2 in registers and
-  // merges chunks, then the two halves of a row merge through shared memory.
-  const bool epi = warp >= 2;
-  const int q = warp & 3;
-  const int half = (warp - 2) / 4;
-  const int r = q * 32 + lane;
-  const uint32_t trow = tmem + ((uint32_t)(q * 32) << 16);
-  bool have = false;
-  __syncwarp();
-  if (epi) {
-    have = __all_sync(0xffffffffu, mbar_wait(&b->tfull[0], 0, ab));
-    have = epi_sync_and(have);
-    tc_fence_after();
-    float n_acc = 0.f, mean_acc = 0.f, m2_acc = 0.f;
-    if (have) {
-#pragma unroll 1
-      for (int c = half; c < BN / 32; c += 2) {
-        const int nv = min(32, n_valid - c * 32);
-        if (nv <= 0) break;
-        uint32_t v[32];
-        tmem_ld32(trow + c * 32, v);
-        tmem_wait_ld();
-        float sum = 0.f;
-#pragma unroll
-        for (int j = 0; j < 32; ++j)
-          if (j < nv) sum += __uint_as_float(v[j]);
-        const float mc = sum / (float)nv;
-        float qc = 0.f;
-#pragma unroll
-        for (int j = 0; j < 32; ++j)
-          if (j < nv) {
-            const float dlt = __uint_as_float(v[j]) - mc;
-            qc = fmaf(dlt, dlt, qc);
-          }
-        chan_merge(n_acc, mean_acc, m2_acc, (float)nv, mc, qc);
-      }
-    }
-    red[2 * half][r] = mean_acc;
-    red[2 * half + 1][r] = m2_acc;
-    epi_sync_and(true);
-    if (half == 0) {
-      // this slice's statistics go to every CTA of the cluster (this one
-      // included); the other half's column count follows from n_valid
-      float n1 = 0.f;
-      for (int c = 1; c < BN / 32; c += 2) n1 += (float)max(0, min(32, n_valid - c * 32));
-      chan_merge(n_acc, mean_acc, m2_acc, n1, red[2][r], red[3][r]);
-      // wait for the start-up phase (every CTA of the cluster is running)
-      asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
-      for (uint32_t j = 0; j < n_ranks; ++j) {
-        st_shared_cluster_f32(map_shared_rank(&st_all[0][rank][r], j), mean_acc);
-        st_shared_cluster_f32(map_shared_rank(&st_all[1][rank][r], j), m2_acc);
-      }
-    } else {
-      asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
-    }
-  } else {
-    asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
-  }
-  __syncwarp();
-  // second phase: every CTA's statistics have landed in every CTA; nothing is
-  // read from or written to another CTA's shared memory after this
-  cluster_arrive_release();
-  cluster_wait_acquire();
-
-  if (epi) {
-    // merge the slices in rank order
-    float n_acc = 0.f, mean_acc = 0.f, m2_acc = 0.f;
-#pragma unroll 1
-    for (uint32_t j = 0; j < n_ranks; ++j)
-      chan_merge(n_acc, mean_acc, m2_acc, (float)min(BN, P.N - (int)j * BN), st_all[0][j][r],
-                 st_all[1][j][r]);
-    const float mu = mean_acc;
-    const float rstd = 1.0f / sqrtf(m2_acc / n_acc + P.eps);
-    // normalise into the (now idle) stage ring in the 128-byte-swizzled layout
-    // of 64-column TMA boxes, then one thread stores the boxes with TMA
-    if (have) {
-#pragma unroll 1
-      for (int c = half; c < BN / 32; c += 2) {
-        if (c * 32 >= n_valid) break;
-        uint32_t v[32];
-        tmem_ld32(trow + c * 32, v);
-        tmem_wait_ld();
-        uint8_t *box = ring + (c / 2) * (BM * 128);
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          uint4 o;
-          __half2 *o2 = reinterpret_cast<__half2 *>(&o);
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int k0 = c * 32 + j * 8 + 2 * e;
-            const float h0 = g_s[k0] * ((__uint_as_float(v[j * 8 + 2 * e]) - mu) * rstd) + b_s[k0];
-            const float h1 =
-                g_s[k0 + 1] * ((__uint_as_float(v[j * 8 + 2 * e + 1]) - mu) * rstd) + b_s[k0 + 1];
-            o2[e] = __floats2half2_rn(h0, h1);
-          }
-          const int chunk = (c % 2) * 4 + j;  // 16-byte chunk within the box's 128-byte row
-          *reinterpret_cast<uint4 *>(box + r * 128 + ((chunk ^ (r & 7)) << 4)) = o;
-        }
-      }
-    }
-    fence_proxy_async_smem();
-    have = epi_sync_and(have);
-    if (have && warp == 2 && lane == 0) {
-      for (int bx = 0; bx * 64 < n_valid; ++bx)
-        tma_store_2d(&mH, ring + bx * (BM * 128), n0 + bx * 64, m0);
-      bulk_commit_and_wait_all();
-    }
-  }
-  __syncwarp();
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 1) {
-    tc_fence_after();
-    tmem_dealloc(tmem, BN);
   }
 }
 
@@ -649,6 +581,52 @@ __global__ void k_to_f16(const __nv_bfloat16 *__restrict__ src, int64_t ld_src, 
       out[e] = __floats2half2_rn(f.x, f.y);
     }
     *reinterpret_cast<uint4 *>(dst + r * cols + c) = o;
+  }
+  if (bad) atomicOr(err, DEV_ERR_F16_RANGE);
+}
+
+// W' = W_mix[:, :d_up] diag(gamma) as fp16 (one warp per output row j), with
+// c[j] = sum_k W'[j][k] over the rounded values the MMAs see, and
+// d[j] = sum_k W_mix[j][k] beta[k]; flags products outside fp16's range
+__global__ void k_mix_ln_weights(const __nv_bfloat16 *__restrict__ W_mix, int64_t ld, int d_out,
+                                 int d_up, const __nv_bfloat16 *__restrict__ gamma,
+                                 const __nv_bfloat16 *__restrict__ beta, __half *__restrict__ w16,
+                                 float *__restrict__ ccol, float *__restrict__ dcol, int *err) {
+  const int lane = threadIdx.x % 32;
+  const int j = blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
+  if (j >= d_out) return;
+  float c = 0.f, dv = 0.f;
+  bool bad = false;
+  for (int k = lane * 8; k < d_up; k += 256) {
+    const uint4 w = *reinterpret_cast<const uint4 *>(W_mix + (int64_t)j * ld + k);
+    const uint4 g = *reinterpret_cast<const uint4 *>(gamma + k);
+    const uint4 bt = *reinterpret_cast<const uint4 *>(beta + k);
+    const __nv_bfloat162 *w2 = reinterpret_cast<const __nv_bfloat162 *>(&w);
+    const __nv_bfloat162 *g2 = reinterpret_cast<const __nv_bfloat162 *>(&g);
+    const __nv_bfloat162 *b2 = reinterpret_cast<const __nv_bfloat162 *>(&bt);
+    uint4 o;
+    __half2 *o2 = reinterpret_cast<__half2 *>(&o);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 wf = __bfloat1622float2(w2[e]), gf = __bfloat1622float2(g2[e]),
+                   bf = __bfloat1622float2(b2[e]);
+      const float p0 = wf.x * gf.x, p1 = wf.y * gf.y;
+      bad |= fabsf(p0) > 65504.f || fabsf(p1) > 65504.f;
+      o2[e] = __floats2half2_rn(p0, p1);
+      const float2 r = __half22float2(o2[e]);
+      c += r.x + r.y;
+      dv = fmaf(wf.x, bf.x, fmaf(wf.y, bf.y, dv));
+    }
+    *reinterpret_cast<uint4 *>(w16 + (int64_t)j * d_up + k) = o;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    c += __shfl_xor_sync(0xffffffffu, c, o);
+    dv += __shfl_xor_sync(0xffffffffu, dv, o);
+  }
+  if (lane == 0) {
+    ccol[j] = c;
+    dcol[j] = dv;
   }
   if (bad) atomicOr(err, DEV_ERR_F16_RANGE);
 }
@@ -706,11 +684,6 @@ int num_sms() {
   return g_num_sms[dev];
 }
 
-constexpr size_t MIX2_SMEM = 1024 + MIX2_STAGES * STAGE2_BYTES + sizeof(Bars);
-constexpr size_t UP_SMEM =
-    1024 + UP_STAGES * STAGE_BYTES + sizeof(Bars) + (2 * BN + 4 * BM + 2 * 8 * BM) * sizeof(float);
-static_assert(UP_STAGES * STAGE_BYTES >= (BN / 64) * BM * 128, "h staging fits the stage ring");
-
 }  // namespace
 
 l3_status make_map_2d16(CUtensorMap *m, const void *base, bool bf16, uint64_t rows, uint64_t cols,
@@ -739,7 +712,7 @@ bool tc_gemm_supported(const l3_dims_t &d) {
 }
 
 l3_status launch_weights_f16(const l3_plan_s *p, const void *W_up, const void *W_mix,
-                             cudaStream_t s) {
+                             const void *gamma, const void *beta, cudaStream_t s) {
   const l3_dims_t &d = p->dims;
   int *err = p->dev_flags + 1;
   {
@@ -747,60 +720,75 @@ l3_status launch_weights_f16(const l3_plan_s *p, const void *W_up, const void *W
     k_to_f16<<<num_sms() * 4, 256, 0, s>>>(reinterpret_cast<const __nv_bfloat16 *>(W_up), d.d_emb,
                                            d.d_up, d.d_emb, reinterpret_cast<__half *>(p->w_up16),
                                            err);
-    k_to_f16<<<num_sms() * 4, 256, 0, s>>>(reinterpret_cast<const __nv_bfloat16 *>(W_mix),
-                                           d.d_up + d.d_in, d.d_out, d.d_up,
-                                           reinterpret_cast<__half *>(p->w_mixh16), err);
+    k_mix_ln_weights<<<(unsigned)((d.d_out + 7) / 8), 256, 0, s>>>(
+        reinterpret_cast<const __nv_bfloat16 *>(W_mix), d.d_up + d.d_in, (int)d.d_out,
+        (int)d.d_up, reinterpret_cast<const __nv_bfloat16 *>(gamma),
+        reinterpret_cast<const __nv_bfloat16 *>(beta), reinterpret_cast<__half *>(p->w_mixh16),
+        p->mix_ccol, p->mix_ccol + (d.d_out + 3) / 4 * 4, err);
   }
   L3_CUDA_TRY(cudaGetLastError());
   return L3_OK;
 }
 
-l3_status launch_up_ln_tc(const l3_plan_s *p, const void *gamma, const void *beta,
-                          cudaStream_t s) {
-  const l3_dims_t &d = p->dims;
-  CUtensorMap mA, mB;
-  l3_status st;
-  if ((st = make_map(&mA, p->a_buf, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, p->n_tokens, d.d_emb, d.d_emb,
-                     BM)) != L3_OK)
-    return st;
-  if ((st = make_map(&mB, p->w_up16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, d.d_up, d.d_emb, d.d_emb,
-                     BN)) != L3_OK)
-    return st;
-  CUtensorMap mH;  // h is written with TMA from 64-column, 128-row boxes
-  if ((st = make_map(&mH, p->h_buf, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, p->n_tokens, d.d_up, d.d_up,
-                     BM)) != L3_OK)
-    return st;
-  UpParams P;
-  P.M = (int)p->n_tokens;
-  P.N = (int)d.d_up;
-  P.kb = (int)(d.d_emb / BK);
-  P.gamma = reinterpret_cast<const __nv_bfloat16 *>(gamma);
-  P.beta = reinterpret_cast<const __nv_bfloat16 *>(beta);
-  P.eps = d.ln_eps;
-  P.h = reinterpret_cast<__half *>(p->h_buf);
-  P.err = p->dev_flags + 1;
+template <int MODE>
+l3_status launch_pair(const CUtensorMap &mA0, const CUtensorMap &mB0, const CUtensorMap &mA1,
+                      const CUtensorMap &mB1, const CUtensorMap &mZ, const MixParams &P,
+                      int device, cudaStream_t s) {
+  constexpr size_t smem =
+      1024 + MixCfg<MODE>::STAGES * STAGE2_BYTES + MixCfg<MODE>::STAGING + sizeof(Bars);
   static bool attr[64] = {};
-  if (!attr[p->device & 63]) {
-    L3_CUDA_TRY(cudaFuncSetAttribute(k_up_ln_gemm, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     (int)UP_SMEM));
-    attr[p->device & 63] = true;
+  if (!attr[device & 63]) {
+    L3_CUDA_TRY(cudaFuncSetAttribute(k_mix_gemm_pair<MODE>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+    attr[device & 63] = true;
   }
-  const int cn = (int)((d.d_up + BN - 1) / BN);
+  // persistent: one CTA pair per two SMs, 256 x 256 tiles
+  const int pairs = std::min(P.n_tiles, num_sms() / 2);
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(cn, (unsigned)((p->n_tokens + BM - 1) / BM), 1);
-  cfg.blockDim = dim3(UP_THREADS, 1, 1);
-  cfg.dynamicSmemBytes = UP_SMEM;
+  cfg.gridDim = dim3(2 * pairs, 1, 1);
+  cfg.blockDim = dim3(GEMM_THREADS, 1, 1);
+  cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
   cudaLaunchAttribute at[1];
   at[0].id = cudaLaunchAttributeClusterDimension;
-  at[0].val.clusterDim.x = cn;
+  at[0].val.clusterDim.x = 2;
   at[0].val.clusterDim.y = 1;
   at[0].val.clusterDim.z = 1;
   cfg.attrs = at;
   cfg.numAttrs = 1;
-  LaunchTimer t("up_ln_gemm_tc", s);
-  L3_CUDA_TRY(cudaLaunchKernelEx(&cfg, k_up_ln_gemm, mA, mB, mH, P));
+  L3_CUDA_TRY(cudaLaunchKernelEx(&cfg, k_mix_gemm_pair<MODE>, mA0, mB0, mA1, mB1, mZ, P));
   return L3_OK;
+}
+
+l3_status launch_up_z_tc(const l3_plan_s *p, cudaStream_t s) {
+  const l3_dims_t &d = p->dims;
+  CUtensorMap mA, mB, mZ;
+  l3_status st;
+  const uint64_t M = p->n_tokens;
+  if ((st = make_map(&mA, p->a_buf, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, M, d.d_emb, d.d_emb, BM)) !=
+      L3_OK)
+    return st;
+  if ((st = make_map(&mB, p->w_up16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, d.d_up, d.d_emb, d.d_emb,
+                     B2_ROWS)) != L3_OK)
+    return st;
+  // z is stored with TMA from 64-column, 128-row boxes
+  if ((st = make_map(&mZ, p->h_buf, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, M, d.d_up, d.d_up, BM)) !=
+      L3_OK)
+    return st;
+  MixParams P = {};
+  P.M = (int)M;
+  P.N = (int)d.d_up;
+  P.kb0 = (int)(d.d_emb / BK);
+  P.kb1 = 0;
+  P.n_tiles_n = (int)((d.d_up + BN - 1) / BN);
+  P.n_tiles = (int)((M + 2 * BM - 1) / (2 * BM)) * P.n_tiles_n;
+  P.y = p->h_buf;
+  P.ldy = d.d_up;
+  P.stats = p->ln_stats;
+  P.n_chunks = P.n_tiles_n;
+  P.err = p->dev_flags + 1;
+  LaunchTimer t("up_z_gemm_tc", s);
+  return launch_pair<MODE_UP_Z>(mA, mB, mA, mB, mZ, P, p->device, s);
 }
 
 l3_status launch_mix_tc(const l3_plan_s *p, const void *x, const void *W_mix, void *y,
@@ -823,7 +811,7 @@ l3_status launch_mix_tc(const l3_plan_s *p, const void *x, const void *W_mix, vo
   if ((st = make_map(&mB1, wx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, d.d_out, d.d_in, d.d_up + d.d_in,
                      B2_ROWS)) != L3_OK)
     return st;
-  MixParams P;
+  MixParams P = {};
   P.M = (int)M;
   P.N = (int)d.d_out;
   P.kb0 = (int)(d.d_up / BK);
@@ -832,32 +820,14 @@ l3_status launch_mix_tc(const l3_plan_s *p, const void *x, const void *W_mix, vo
   P.n_tiles = (int)((M + 2 * BM - 1) / (2 * BM)) * P.n_tiles_n;
   P.y = y;
   P.ldy = d.d_out;
-  P.idesc0 = IDESC2_F16;
-  P.idesc1 = IDESC2_BF16;
+  P.stats = p->ln_stats;
+  P.n_chunks = (int)((d.d_up + BN - 1) / BN);
+  P.ccol = p->mix_ccol;
+  P.dcol = p->mix_ccol + (d.d_out + 3) / 4 * 4;
+  P.eps = d.ln_eps;
   P.err = p->dev_flags + 1;
-  static bool attr[64] = {};
-  if (!attr[p->device & 63]) {
-    L3_CUDA_TRY(cudaFuncSetAttribute(k_mix_gemm_pair<false>,
-                                     cudaFuncAttributeMaxDynamicSharedMemorySize, (int)MIX2_SMEM));
-    attr[p->device & 63] = true;
-  }
-  // persistent: one CTA pair per two SMs, 256 x 256 tiles
-  const int pairs = std::min(P.n_tiles, num_sms() / 2);
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(2 * pairs, 1, 1);
-  cfg.blockDim = dim3(GEMM_THREADS, 1, 1);
-  cfg.dynamicSmemBytes = MIX2_SMEM;
-  cfg.stream = s;
-  cudaLaunchAttribute at[1];
-  at[0].id = cudaLaunchAttributeClusterDimension;
-  at[0].val.clusterDim.x = 2;
-  at[0].val.clusterDim.y = 1;
-  at[0].val.clusterDim.z = 1;
-  cfg.attrs = at;
-  cfg.numAttrs = 1;
   LaunchTimer t("mix_gemm_tc", s);
-  L3_CUDA_TRY(cudaLaunchKernelEx(&cfg, k_mix_gemm_pair<false>, mA0, mB0, mA1, mB1, P));
-  return L3_OK;
+  return launch_pair<MODE_MIX_LN>(mA0, mB0, mA1, mB1, mA0, P, p->device, s);
 }
 
 l3_status launch_gemm_nt_tc(const void *A, const void *B, const void *A1, const void *B1, bool f16,
@@ -889,7 +859,7 @@ l3_status launch_gemm_nt_tc(const void *A, const void *B, const void *A1, const 
     mA1 = mA;  // never read (kb1 = 0)
     mB1 = mB;
   }
-  MixParams P;
+  MixParams P = {};
   P.M = (int)M;
   P.N = (int)N;
   P.kb0 = (int)((K + BK - 1) / BK);  // the K tail is zero-filled by TMA in both operands
@@ -900,27 +870,7 @@ l3_status launch_gemm_nt_tc(const void *A, const void *B, const void *A1, const 
   P.ldy = ldc;
   P.idesc0 = P.idesc1 = f16 ? IDESC2_F16 : IDESC2_BF16;
   P.err = err;
-  static bool attr[64] = {};
-  if (!attr[device & 63]) {
-    L3_CUDA_TRY(cudaFuncSetAttribute(k_mix_gemm_pair<true>,
-                                     cudaFuncAttributeMaxDynamicSharedMemorySize, (int)MIX2_SMEM));
-    attr[device & 63] = true;
-  }
-  const int pairs = std::min(P.n_tiles, num_sms() / 2);
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(2 * pairs, 1, 1);
-  cfg.blockDim = dim3(GEMM_THREADS, 1, 1);
-  cfg.dynamicSmemBytes = MIX2_SMEM;
-  cfg.stream = s;
-  cudaLaunchAttribute at[1];
-  at[0].id = cudaLaunchAttributeClusterDimension;
-  at[0].val.clusterDim.x = 2;
-  at[0].val.clusterDim.y = 1;
-  at[0].val.clusterDim.z = 1;
-  cfg.attrs = at;
-  cfg.numAttrs = 1;
-  L3_CUDA_TRY(cudaLaunchKernelEx(&cfg, k_mix_gemm_pair<true>, mA, mB, mA1, mB1, P));
-  return L3_OK;
+  return launch_pair<MODE_F32>(mA, mB, mA1, mB1, mA, P, device, s);
 }
 
 }  // namespace l3

@@ -29,7 +29,7 @@ enum : int32_t {
   DEV_ERR_TOKEN_RANGE = 1,
   DEV_ERR_BAD_OFFSETS = 2,
   DEV_ERR_TIMEOUT = 4,
-  DEV_ERR_F16_RANGE = 8,  // a bf16 weight outside fp16's finite range
+  DEV_ERR_F16_RANGE = 8,  // an fp16 operand (W_up, W', z) outside fp16's finite range
 };
 
 // ---------------------------------------------------------------------------
@@ -109,10 +109,14 @@ struct l3_plan_s {
   l3::TailItem *tail_items = nullptr;
   int32_t *dev_flags = nullptr;        // [0] plan errors, [1] forward errors, [4..7] dense tile counters
   void *a_buf = nullptr;               // [N x d_emb] dtype, original token order
-  void *h_buf = nullptr;               // [N x d_up] dtype
+  void *h_buf = nullptr;               // [N x d_up] h (CUDA-core path) or z = a W_up^T (fp16,
+                                       // tensor-core path: the LayerNorm is applied inside W_mix)
   float *z_buf = nullptr;              // [N x d_up] fp32 (CUDA-core GEMM path only)
   void *w_up16 = nullptr;              // [d_up x d_emb] fp16 copy of W_up (tensor-core path)
-  void *w_mixh16 = nullptr;            // [d_out x d_up] fp16 copy of W_mix[:, :d_up]
+  void *w_mixh16 = nullptr;            // [d_out x d_up] fp16 W_mix[:, :d_up] diag(gamma)
+  float2 *ln_stats = nullptr;          // [N x ceil(d_up / 256)] (mean, M2) of z per 256 columns
+  float *mix_ccol = nullptr;           // W' 1 [d_out], then W_mix[:, :d_up] beta at a 16-byte
+                                       // aligned offset
   bool tc_gemm = false;                // tensor-core GEMMs in use
 };
 
@@ -166,9 +170,8 @@ l3_status launch_attn_dense(const l3_plan_s *p, const void *x, const void *W_K, 
 // GEMMs + LayerNorm, tensor-core path (gemm_tc.cu)
 bool tc_gemm_supported(const l3_dims_t &d);
 l3_status launch_weights_f16(const l3_plan_s *p, const void *W_up, const void *W_mix,
-                             cudaStream_t s);
-l3_status launch_up_ln_tc(const l3_plan_s *p, const void *gamma, const void *beta,
-                          cudaStream_t s);
+                             const void *gamma, const void *beta, cudaStream_t s);
+l3_status launch_up_z_tc(const l3_plan_s *p, cudaStream_t s);
 l3_status launch_mix_tc(const l3_plan_s *p, const void *x, const void *W_mix, void *y,
                         cudaStream_t s);
 // C[M x N] (fp32, row stride ldc) = A[M x K] B[N x K]^T (+ A1 B1^T when A1

@@ -126,7 +126,7 @@ def test_tensor_core_kernels_run():
     run_forward(w, dev)
     kernels = l3.l3_profile_read()
     l3.l3_profile_enable(False)
-    assert "mix_gemm_tc" in kernels and "up_ln_gemm_tc" in kernels, kernels
+    assert "mix_gemm_tc" in kernels and "up_z_gemm_tc" in kernels, kernels
 
 
 @pytest.mark.parametrize("vocab,d_t,n,d_in,d_emb,d_up,d_out", [
