@@ -193,8 +193,13 @@ enum : int { MODE_F32 = 0, MODE_UP_Z = 1, MODE_MIX_LN = 2 };
 template <int MODE>
 struct MixCfg {
   static constexpr int STAGES = MODE == MODE_UP_Z ? 4 : MIX2_STAGES;
-  // MODE_UP_Z: 128 rows x 256 columns of fp16 z, four 64-column TMA boxes
-  static constexpr int STAGING = MODE == MODE_UP_Z ? (BN / 64) * BM * 128 : 0;
+  // MODE_UP_Z: 128 rows x 256 columns of fp16 z, four 64-column TMA boxes,
+  // then the two column halves' (count, mean, M2) of each row
+  static constexpr int STAGING = MODE == MODE_UP_Z ? (BN / 64) * BM * 128 + 2 * 3 * BM * 4 : 0;
+  // epilogue warps: two per TMEM lane quarter for MODE_UP_Z, whose epilogue
+  // has only 8 k-blocks of MMAs to hide behind; one per quarter otherwise
+  static constexpr int EPI_WARPS = MODE == MODE_UP_Z ? 8 : 4;
+  static constexpr int THREADS = 64 + 32 * EPI_WARPS;
 };
 
 // The j-th (tile, range, accumulator) job of a pair that owns `k_tiles`
@@ -227,20 +232,22 @@ __device__ __forceinline__ bool mix_job(int j, int k_tiles, int &k, int &rng, in
   return false;
 }
 
-// barriers of the four epilogue warps (128 threads): a plain one, and one
-// that ANDs a flag across them so that they leave their loop together
+// barriers of the epilogue warps (N threads): a plain one, and one that ANDs
+// a flag across them so that they leave their loop together
+template <int N>
 __device__ __forceinline__ void epi_bar_sync() {
-  asm volatile("bar.sync 1, 128;" ::: "memory");
+  asm volatile("bar.sync 1, %0;" ::"n"(N) : "memory");
 }
-__device__ __forceinline__ bool epi4_sync_and(bool ok) {
+template <int N>
+__device__ __forceinline__ bool epi_sync_and(bool ok) {
   uint32_t r;
   asm volatile(
       "{\n\t.reg .pred p, q;\n\t"
       "setp.ne.u32 q, %1, 0;\n\t"
-      "bar.red.and.pred p, 2, 128, q;\n\t"
+      "bar.red.and.pred p, 2, %2, q;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}\n"
       : "=r"(r)
-      : "r"((uint32_t)ok)
+      : "r"((uint32_t)ok), "n"(N)
       : "memory");
   return r != 0;
 }
@@ -253,12 +260,13 @@ __device__ __forceinline__ void tma_store_2d_box(const CUtensorMap *map, const v
 }
 
 template <int MODE>
-__global__ void __launch_bounds__(GEMM_THREADS, 1)
+__global__ void __launch_bounds__(MixCfg<MODE>::THREADS, 1)
     k_mix_gemm_pair(const __grid_constant__ CUtensorMap mA0, const __grid_constant__ CUtensorMap mB0,
                     const __grid_constant__ CUtensorMap mA1, const __grid_constant__ CUtensorMap mB1,
                     const __grid_constant__ CUtensorMap mZ, MixParams P) {
   using Cfg = MixCfg<MODE>;
   constexpr int STAGES = Cfg::STAGES;
+  constexpr int EPI_T = 32 * Cfg::EPI_WARPS;  // epilogue threads
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = align1024(smem_raw);
   uint8_t *ring = smem;
@@ -276,7 +284,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&b->tfull[a], 1);
-      mbar_init(&b->tempty[a], 8);  // used in CTA 0: four epilogue warps of each CTA
+      mbar_init(&b->tempty[a], 2 * Cfg::EPI_WARPS);  // used in CTA 0: every epilogue warp of both CTAs
     }
     mbar_init(&b->drain, 1);
     b->abort_flag = 0;
@@ -399,10 +407,12 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       }
     }
   } else {
-    // epilogue: warp (2..5) % 4 selects the TMEM lane quarter it may read;
-    // each CTA handles its own 128 rows of the pair's tile
+    // epilogue: warp % 4 selects the TMEM lane quarter it may read; each CTA
+    // handles its own 128 rows of the pair's tile; with eight warps, two per
+    // quarter, each takes every other 32-column chunk
     const int q = warp & 3;
     const int r = q * 32 + lane;
+    const int c_first = (warp - 2) / 4, c_step = Cfg::EPI_WARPS / 4;
     const uint32_t tempty0[2] = {map_shared_rank(&b->tempty[0], 0),
                                  map_shared_rank(&b->tempty[1], 0)};
     int n_acc[2] = {0, 0};
@@ -413,7 +423,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       if (acc) ++n_acc[1]; else ++n_acc[0];
       bool got = __all_sync(0xffffffffu, mbar_wait(&b->tfull[acc], na & 1, ab));
       // MODE_UP_Z's warps meet at named barriers below: they leave together
-      if (MODE == MODE_UP_Z) got = epi4_sync_and(got);
+      if (MODE == MODE_UP_Z) got = epi_sync_and<EPI_T>(got);
       if (!got) break;
       tc_fence_after();
       const int tile = pair_id + k * n_pairs;
@@ -455,13 +465,13 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         // the fp16 values into the staging boxes (128-byte swizzle)
         if (stored) {
           if (warp == 2 && lane == 0) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
-          epi_bar_sync();
+          epi_bar_sync<EPI_T>();
         }
         const int nv = min(BN, P.N - n0);
         float n_acc_f = 0.f, mean = 0.f, m2 = 0.f;
         bool range_ok = true;
 #pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
+        for (int c = c_first; c < BN / 32; c += c_step) {
           uint32_t v[32];
           tmem_ld32(tacc + c * 32, v);
           tmem_wait_ld();
@@ -497,12 +507,20 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             *reinterpret_cast<uint4 *>(box + r * 128 + ((chunk ^ (r & 7)) << 4)) = o;
           }
         }
-        if (m < P.M) {
-          P.stats[(int64_t)m * P.n_chunks + n0 / BN] = make_float2(mean, m2);
-          if (!range_ok) atomicOr(P.err, DEV_ERR_F16_RANGE);
+        if (!range_ok) atomicOr(P.err, DEV_ERR_F16_RANGE);
+        // the two column halves of a row (every other chunk each) merge in order
+        float *part = reinterpret_cast<float *>(staging + (BN / 64) * BM * 128);
+        if (c_first == 1) {
+          part[r] = n_acc_f;
+          part[BM + r] = mean;
+          part[2 * BM + r] = m2;
         }
         fence_proxy_async_smem();
-        epi_bar_sync();
+        epi_bar_sync<EPI_T>();
+        if (c_first == 0 && m < P.M) {
+          chan_merge(n_acc_f, mean, m2, part[r], part[BM + r], part[2 * BM + r]);
+          P.stats[(int64_t)m * P.n_chunks + n0 / BN] = make_float2(mean, m2);
+        }
         if (warp == 2 && lane == 0) {
           const int mrow = (tile / P.n_tiles_n) * (2 * BM) + (int)rank * BM;
           for (int bx = 0; bx * 64 < nv; ++bx)
@@ -746,7 +764,7 @@ l3_status launch_pair(const CUtensorMap &mA0, const CUtensorMap &mB0, const CUte
   const int pairs = std::min(P.n_tiles, num_sms() / 2);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * pairs, 1, 1);
-  cfg.blockDim = dim3(GEMM_THREADS, 1, 1);
+  cfg.blockDim = dim3(MixCfg<MODE>::THREADS, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
   cudaLaunchAttribute at[1];
