@@ -81,15 +81,18 @@ def attention_flops(ids: np.ndarray, offsets: np.ndarray, w: wl.Workload) -> int
 
 # DRAM bytes (read + write) per launch of a kernel, from one ncu capture of
 #   ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum,gpu__time_duration.sum
-#       --clock-control none -k regex:<kernel> -s 3 -c 1
-#       python bench.py --workload <w> --only --steps 1 --warmup 3 --no-e2e --cpu-seconds 0
+#       --clock-control none -k regex:k_mix_gemm_pair -s 6 -c 4
+#       python bench.py --workload <w> --only --steps 3 --warmup 3 --no-e2e --cpu-seconds 0
 # keyed by (kernel, workload, tokens), with the digest of the kernel's source
 # files at capture time: a figure is reported only while those sources are
 # unchanged (source_digest), else traffic is null
 TRAFFIC = {
-    ("mix_gemm_tc", "paper_shaped", 65536): {"bytes": 575813888 + 249530112,
+    ("mix_gemm_tc", "paper_shaped", 65536): {"bytes": 599436800 + 245141248,
                                              "sources": ("gemm_tc.cu", "sm100.cuh"),
-                                             "digest": "faed5e7597c03789", "captured": "2026-12"},
+                                             "digest": "a903dcb322c014cd", "captured": "2026-12"},
+    ("up_z_gemm_tc", "paper_shaped", 65536): {"bytes": 69584896 + 213250560,
+                                              "sources": ("gemm_tc.cu", "sm100.cuh"),
+                                              "digest": "a903dcb322c014cd", "captured": "2026-12"},
 }
 
 

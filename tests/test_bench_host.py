@@ -54,7 +54,7 @@ def test_traffic_only_for_unchanged_sources():
         assert bench.traffic_for("mix_gemm_tc", w)["traffic"] is None
         bench.TRAFFIC[key]["digest"] = bench.source_digest("gemm_tc.cu")
         assert bench.traffic_for("mix_gemm_tc", w)["traffic"] == 123
-        assert bench.traffic_for("up_z_gemm_tc", w)["traffic"] is None
+        assert bench.traffic_for("attn_tail_t1_big", w)["traffic"] is None
     finally:
         if saved is None:
             bench.TRAFFIC.pop(key, None)
