@@ -193,12 +193,13 @@ enum : int { MODE_F32 = 0, MODE_UP_Z = 1, MODE_MIX_LN = 2 };
 template <int MODE>
 struct MixCfg {
   static constexpr int STAGES = MODE == MODE_UP_Z ? 4 : MIX2_STAGES;
+  // epilogue warps: four per TMEM lane quarter for MODE_UP_Z, whose epilogue
+  // has only d_emb / 64 k-blocks of MMAs to hide behind; one per quarter otherwise
+  static constexpr int EPI_WARPS = MODE == MODE_UP_Z ? 16 : 4;
   // MODE_UP_Z: 128 rows x 256 columns of fp16 z, four 64-column TMA boxes,
-  // then the two column halves' (count, mean, M2) of each row
-  static constexpr int STAGING = MODE == MODE_UP_Z ? (BN / 64) * BM * 128 + 2 * 3 * BM * 4 : 0;
-  // epilogue warps: two per TMEM lane quarter for MODE_UP_Z, whose epilogue
-  // has only 8 k-blocks of MMAs to hide behind; one per quarter otherwise
-  static constexpr int EPI_WARPS = MODE == MODE_UP_Z ? 8 : 4;
+  // then the (count, mean, M2) of each row over the chunks of warps 2-3 of a quarter
+  static constexpr int STAGING =
+      MODE == MODE_UP_Z ? (BN / 64) * BM * 128 + (EPI_WARPS / 4 - 1) * 3 * BM * 4 : 0;
   static constexpr int THREADS = 64 + 32 * EPI_WARPS;
 };
 
@@ -408,8 +409,8 @@ __global__ void __launch_bounds__(MixCfg<MODE>::THREADS, 1)
     }
   } else {
     // epilogue: warp % 4 selects the TMEM lane quarter it may read; each CTA
-    // handles its own 128 rows of the pair's tile; with eight warps, two per
-    // quarter, each takes every other 32-column chunk
+    // handles its own 128 rows of the pair's tile; with several warps per
+    // quarter, warp j of a quarter takes 32-column chunks j, j + (warps per quarter), ...
     const int q = warp & 3;
     const int r = q * 32 + lane;
     const int c_first = (warp - 2) / 4, c_step = Cfg::EPI_WARPS / 4;
@@ -508,17 +509,22 @@ __global__ void __launch_bounds__(MixCfg<MODE>::THREADS, 1)
           }
         }
         if (!range_ok) atomicOr(P.err, DEV_ERR_F16_RANGE);
-        // the two column halves of a row (every other chunk each) merge in order
+        // the statistics of a row's chunk sets (one per warp of its quarter)
+        // merge in a fixed order
         float *part = reinterpret_cast<float *>(staging + (BN / 64) * BM * 128);
-        if (c_first == 1) {
-          part[r] = n_acc_f;
-          part[BM + r] = mean;
-          part[2 * BM + r] = m2;
+        if (c_first > 0) {
+          float *pp = part + (c_first - 1) * 3 * BM;
+          pp[r] = n_acc_f;
+          pp[BM + r] = mean;
+          pp[2 * BM + r] = m2;
         }
         fence_proxy_async_smem();
         epi_bar_sync<EPI_T>();
         if (c_first == 0 && m < P.M) {
-          chan_merge(n_acc_f, mean, m2, part[r], part[BM + r], part[2 * BM + r]);
+          for (int k = 0; k < c_step - 1; ++k) {
+            const float *pp = part + k * 3 * BM;
+            chan_merge(n_acc_f, mean, m2, pp[r], pp[BM + r], pp[2 * BM + r]);
+          }
           P.stats[(int64_t)m * P.n_chunks + n0 / BN] = make_float2(mean, m2);
         }
         if (warp == 2 && lane == 0) {
