@@ -507,7 +507,10 @@ def measure(w, args, dev, dist, world, rank, steps, warmup, with_e2e=True, with_
     plan0.destroy()
 
     # ---- timed region: K steps, plan + forward, device-timed ----
-    l3.l3_profile_enable(True)
+    # per-kernel CUDA events on the forward's launches (the plan's are not
+    # timed: their events cost host time in the loop and they are never the
+    # dominant kernel)
+    l3.l3_profile_enable(2)
     barrier()
     torch.cuda.synchronize(dev)
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)

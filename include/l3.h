@@ -364,11 +364,12 @@ const char *l3_last_error(void);
 
 /*
  * Per-kernel timing for profiling: while enabled, every kernel the library
- * launches is bracketed by CUDA events recorded on the stream it is launched
- * on. l3_profile_read synchronizes those streams and returns, per kernel
- * name, the number of launches and the summed device time since the last
- * l3_profile_enable(1). At most `max_entries` entries are written; the
- * return value is the number of distinct kernels (or -1 on error).
+ * launches (enable = 1), or every kernel but the plan's (enable = 2), is
+ * bracketed by CUDA events recorded on the stream it is launched on;
+ * enable = 0 turns timing off. l3_profile_read synchronizes those streams and
+ * returns, per kernel name, the number of launches and the summed device time
+ * since the last l3_profile_enable. At most `max_entries` entries are written;
+ * the return value is the number of distinct kernels (or -1 on error).
  */
 typedef struct {
   char name[48];

@@ -310,8 +310,9 @@ def l3_plan_destroy(plan: Plan):
     plan.destroy()
 
 
-def l3_profile_enable(enable: bool = True):
-    library().l3_profile_enable(1 if enable else 0)
+def l3_profile_enable(enable=True):
+    """True or 1: time every launch; 2: every launch but the plan's; False or 0: off."""
+    library().l3_profile_enable(int(enable) if not isinstance(enable, bool) else (1 if enable else 0))
 
 
 def l3_profile_read(max_entries: int = 64) -> dict:

@@ -5,6 +5,7 @@
 //   attention  a[n] = V_t^T softmax(K_t x_n)   (gather-attention kernels)
 //   up + LN    h = LayerNorm(W_up a)           (GEMM with LayerNorm epilogue)
 //   mix        y = W_mix[:, :d_up] h + W_mix[:, d_up:] x   (two accumulated K-ranges)
+#include <cstring>
 #include <mutex>
 #include <string>
 #include <unordered_map>
@@ -27,6 +28,7 @@ struct Record {
 };
 std::mutex g_prof_mu;
 bool g_prof_on = false;
+bool g_prof_plan = false;  // also time the plan's kernels
 std::vector<Record> g_records;
 std::vector<cudaEvent_t> g_free_events;
 
@@ -190,7 +192,7 @@ l3_status cuda_fail(cudaError_t e, const char *what) {
 
 LaunchTimer::LaunchTimer(const char *n, cudaStream_t s) : name(n), stream(s), slot(-1) {
   std::lock_guard<std::mutex> lk(g_prof_mu);
-  if (!g_prof_on) return;
+  if (!g_prof_on || (!g_prof_plan && std::strncmp(n, "plan", 4) == 0)) return;
   Record r{name, s, take_event(), take_event()};
   cudaEventRecord(r.start, s);
   slot = (int)g_records.size();
@@ -525,6 +527,7 @@ void l3_profile_enable(int enable) {
   }
   g_records.clear();
   g_prof_on = enable != 0;
+  g_prof_plan = enable == 1;
 }
 
 int l3_profile_read(l3_kernel_time_t *out, int max_entries) {
