@@ -80,11 +80,26 @@ __global__ void k_validate_offsets(const int32_t *__restrict__ offsets, int64_t 
 }
 
 // Digit histogram of one tile; counts land digit-major: hist[d * n_tiles + tile].
+// With vocab > 0 (the first pass) keys outside [0, vocab) are flagged, and
+// with `offsets` the CTAs also check the offsets array as k_validate_offsets
+// does (grid-stride), which saves that launch.
 __global__ void __launch_bounds__(SORT_THREADS)
     k_radix_hist(const int32_t *__restrict__ keys, int64_t n, int shift, int32_t *__restrict__ hist,
-                 int n_tiles, int64_t vocab, int32_t *info) {
+                 int n_tiles, int64_t vocab, int32_t *info, const int32_t *__restrict__ offsets,
+                 int64_t v, int64_t k_cap) {
   __shared__ int32_t cnt[RADIX];
   for (int i = threadIdx.x; i < RADIX; i += SORT_THREADS) cnt[i] = 0;
+  if (offsets) {
+    bool bad_off = false;
+    for (int64_t t = blockIdx.x * (int64_t)SORT_THREADS + threadIdx.x; t < vocab;
+         t += (int64_t)gridDim.x * SORT_THREADS) {
+      const int64_t d = (int64_t)offsets[t + 1] - offsets[t];
+      bad_off |= d < 1 || d > k_cap;
+      if (t == 0 && offsets[0] != 0) bad_off = true;
+      if (t == vocab - 1 && offsets[vocab] != v) bad_off = true;
+    }
+    if (bad_off) atomicOr(&info[INFO_ERR], DEV_ERR_BAD_OFFSETS);
+  }
   __syncthreads();
   int64_t base = (int64_t)blockIdx.x * SORT_TILE;
   bool bad = false;
@@ -104,15 +119,22 @@ __global__ void __launch_bounds__(SORT_THREADS)
 
 // Stable scatter of one tile. offs[d * n_tiles + tile] is the first output
 // position of digit d for this tile (exclusive scan of the histogram in
-// digit-major order). Each warp owns a contiguous span of the tile and walks
-// it in order, ranking equal digits with __match_any_sync, so the output keeps
-// input order among equal digits.
+// digit-major order), or, with `raw`, the histogram itself: the CTA then adds
+// up digit d's counts in the earlier tiles and in all tiles (few tiles:
+// FUSED_SCAN_TILES at most) and scans the digit totals itself, which saves a
+// scan launch per pass. Each warp owns a contiguous span of the tile and
+// walks it in order, ranking equal digits with __match_any_sync, so the output
+// keeps input order among equal digits.
+constexpr int FUSED_SCAN_TILES = 64;
+static_assert(RADIX == SORT_THREADS, "one thread per digit");
+
 __global__ void __launch_bounds__(SORT_THREADS)
     k_radix_scatter(const int32_t *__restrict__ keys_in, const int32_t *__restrict__ vals_in,
                     int32_t *__restrict__ keys_out, int32_t *__restrict__ vals_out, int64_t n,
-                    int shift, const int32_t *__restrict__ offs, int n_tiles) {
+                    int shift, const int32_t *__restrict__ offs, int n_tiles, int raw) {
   __shared__ int32_t whist[SORT_WARPS][RADIX];
   __shared__ int32_t dbase[RADIX];
+  __shared__ int32_t wtot[SORT_WARPS];
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   for (int i = threadIdx.x; i < SORT_WARPS * RADIX; i += SORT_THREADS) (&whist[0][0])[i] = 0;
   __syncthreads();
@@ -136,7 +158,8 @@ __global__ void __launch_bounds__(SORT_THREADS)
     __syncwarp();
   }
   __syncthreads();
-  for (int d = threadIdx.x; d < RADIX; d += SORT_THREADS) {
+  {
+    const int d = threadIdx.x;  // one digit per thread
     int32_t run = 0;
 #pragma unroll
     for (int w = 0; w < SORT_WARPS; ++w) {
@@ -144,7 +167,34 @@ __global__ void __launch_bounds__(SORT_THREADS)
       whist[w][d] = run;
       run += c;
     }
-    dbase[d] = offs[(int64_t)d * n_tiles + blockIdx.x];
+    if (!raw) {
+      dbase[d] = offs[(int64_t)d * n_tiles + blockIdx.x];
+    } else {
+      int32_t pre = 0, tot = 0;  // digit d in earlier tiles, in all tiles
+      const int32_t *row = offs + (int64_t)d * n_tiles;
+      for (int t0 = 0; t0 < n_tiles; t0 += 16) {
+        int32_t c[16];  // sixteen loads in flight
+#pragma unroll
+        for (int u = 0; u < 16; ++u) c[u] = t0 + u < n_tiles ? row[t0 + u] : 0;
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+          tot += c[u];
+          pre += t0 + u < (int)blockIdx.x ? c[u] : 0;
+        }
+      }
+      // exclusive scan of the digit totals across the CTA (digits in thread order)
+      int32_t incl = tot;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int32_t v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+      }
+      if (lane == 31) wtot[warp] = incl;
+      __syncthreads();
+      int32_t before = 0;
+      for (int w = 0; w < warp; ++w) before += wtot[w];
+      dbase[d] = before + incl - tot + pre;
+    }
   }
   __syncthreads();
 #pragma unroll
@@ -756,7 +806,8 @@ l3_status build_plan(l3_plan_s *p, const int32_t *ids, const int32_t *offsets, c
   }
 
   L3_CUDA_TRY(cudaMemsetAsync(info, 0, 64 * sizeof(int32_t), s));
-  {
+  if (n == 0) {
+    // (with tokens the first histogram pass checks the offsets)
     LaunchTimer t("plan_validate", s);
     k_validate_offsets<<<blocks_for(vocab, 256), 256, 0, s>>>(offsets, vocab, p->dims.v, p->dims.k,
                                                               info);
@@ -783,14 +834,16 @@ l3_status build_plan(l3_plan_s *p, const int32_t *ids, const int32_t *offsets, c
       int32_t *vout = vbuf[(pass + 1) % 2];
       {
         LaunchTimer t("plan_radix_hist", s);
-        k_radix_hist<<<(int)n_tiles, SORT_THREADS, 0, s>>>(kin, n, shift, hist, (int)n_tiles,
-                                                          pass == 0 ? vocab : 0, info);
+        k_radix_hist<<<(int)n_tiles, SORT_THREADS, 0, s>>>(
+            kin, n, shift, hist, (int)n_tiles, pass == 0 ? vocab : 0, info,
+            pass == 0 ? offsets : nullptr, p->dims.v, p->dims.k);
       }
-      scan_multi({{hist, hist, RADIX * n_tiles, nullptr}}, s);
+      const int raw = n_tiles <= FUSED_SCAN_TILES;
+      if (!raw) scan_multi({{hist, hist, RADIX * n_tiles, nullptr}}, s);
       {
         LaunchTimer t("plan_radix_scatter", s);
         k_radix_scatter<<<(int)n_tiles, SORT_THREADS, 0, s>>>(kin, vin, kout, vout, n, shift, hist,
-                                                             (int)n_tiles);
+                                                             (int)n_tiles, raw);
       }
       kin = kout;
       vin = vout;
@@ -920,12 +973,12 @@ l3_status radix_sort_pairs(const int32_t *keys_in, const int32_t *vals_in, int64
     const int shift = pass * RADIX_BITS;
     int32_t *kout = kbuf[(pass + 1) % 2], *vout = vbuf[(pass + 1) % 2];
     k_radix_hist<<<(int)n_tiles, SORT_THREADS, 0, s>>>(kin, n, shift, hist, (int)n_tiles, 0,
-                                                      nullptr);
+                                                      nullptr, nullptr, 0, 0);
     ScanJobs jobs{};
     jobs.job[0] = ScanJob{hist, hist, RADIX * n_tiles, nullptr};
     k_scan_multi<<<1, SCAN_THREADS, 0, s>>>(jobs);
     k_radix_scatter<<<(int)n_tiles, SORT_THREADS, 0, s>>>(kin, vin, kout, vout, n, shift, hist,
-                                                         (int)n_tiles);
+                                                         (int)n_tiles, 0);
     kin = kout;
     vin = vout;
   }
@@ -1061,14 +1114,14 @@ extern "C" l3_status l3_sort_tokens_noalloc(const int32_t *token_ids, int64_t n_
     int32_t *kout = kbuf[(pass + 1) % 2];
     int32_t *vout = vbuf[(pass + 1) % 2];
     k_radix_hist<<<(int)n_tiles, SORT_THREADS, 0, s>>>(kin, n, shift, hist, (int)n_tiles, 0,
-                                                      nullptr);
+                                                      nullptr, nullptr, 0, 0);
     {
       ScanJobs jobs{};
       jobs.job[0] = ScanJob{hist, hist, RADIX * n_tiles, nullptr};
       k_scan_multi<<<1, SCAN_THREADS, 0, s>>>(jobs);
     }
     k_radix_scatter<<<(int)n_tiles, SORT_THREADS, 0, s>>>(kin, vin, kout, vout, n, shift, hist,
-                                                         (int)n_tiles);
+                                                         (int)n_tiles, 0);
     kin = kout;
     vin = vout;
   }
