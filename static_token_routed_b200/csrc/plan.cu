@@ -131,7 +131,8 @@ static_assert(RADIX == SORT_THREADS, "one thread per digit");
 __global__ void __launch_bounds__(SORT_THREADS)
     k_radix_scatter(const int32_t *__restrict__ keys_in, const int32_t *__restrict__ vals_in,
                     int32_t *__restrict__ keys_out, int32_t *__restrict__ vals_out, int64_t n,
-                    int shift, const int32_t *__restrict__ offs, int n_tiles, int raw) {
+                    int shift, const int32_t *__restrict__ offs, int n_tiles, int raw,
+                    int32_t *__restrict__ inv_out) {
   __shared__ int32_t whist[SORT_WARPS][RADIX];
   __shared__ int32_t dbase[RADIX];
   __shared__ int32_t wtot[SORT_WARPS];
@@ -203,8 +204,10 @@ __global__ void __launch_bounds__(SORT_THREADS)
     if (i < n) {
       int d = digit[it];
       int32_t pos = dbase[d] + whist[warp][d] + rank[it];
+      const int32_t val = vals_in ? vals_in[i] : (int32_t)i;
       keys_out[pos] = key[it];
-      vals_out[pos] = vals_in ? vals_in[i] : (int32_t)i;
+      vals_out[pos] = val;
+      if (inv_out) inv_out[val] = pos;  // the last pass: the inverse permutation
     }
   }
 }
@@ -217,6 +220,7 @@ struct ScanJob {
   int32_t *out;
   int64_t n;
   int32_t *total;
+  const int32_t *n_dev;  // if set, only the first min(n, *n_dev) values are scanned
 };
 struct ScanJobs {
   ScanJob job[4];
@@ -231,6 +235,7 @@ __global__ void __launch_bounds__(SCAN_THREADS) k_scan_multi(ScanJobs jobs) {
   if (blockIdx.x == 2) J = jobs.job[2];
   if (blockIdx.x == 3) J = jobs.job[3];
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  if (J.n_dev) J.n = min(J.n, (int64_t)*J.n_dev);
   // Each warp owns a contiguous segment of SCAN_ITEMS * 32 values of the chunk
   // and walks it in rounds of 32 consecutive values (coalesced loads and
   // stores); a round's inclusive warp scan plus the carry of earlier rounds
@@ -296,32 +301,74 @@ l3_status scan_multi(std::initializer_list<ScanJob> js, cudaStream_t s) {
   return L3_OK;
 }
 
-// head[i] = 1 where a new ID starts in sorted order; inv_perm[perm[i]] = i.
-__global__ void k_group_heads(const int32_t *__restrict__ sorted, const int32_t *__restrict__ perm,
-                              int64_t n, int32_t *__restrict__ head, int32_t *__restrict__ inv_perm) {
-  int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
-  if (i >= n) return;
-  head[i] = (i == 0 || sorted[i] != sorted[i - 1]) ? 1 : 0;
-  inv_perm[perm[i]] = (int32_t)i;
-}
-
-__global__ void k_group_fill(const int32_t *__restrict__ sorted, const int32_t *__restrict__ head,
-                             const int32_t *__restrict__ gpos, int64_t n,
-                             const int32_t *__restrict__ offsets, int64_t vocab,
-                             int32_t *__restrict__ group_ids, int32_t *__restrict__ group_tok_start,
-                             int32_t *__restrict__ group_row_start, int32_t *__restrict__ group_rows,
-                             const int32_t *info) {
-  int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
-  if (i == 0) group_tok_start[info[INFO_G]] = (int32_t)n;
-  if (i >= n || !head[i]) return;
-  int32_t g = gpos[i];
-  int32_t id = sorted[i];
-  group_ids[g] = id;
-  group_tok_start[g] = (int32_t)i;
-  bool ok = id >= 0 && id < vocab;
-  int32_t r0 = ok ? offsets[id] : 0;
-  group_row_start[g] = r0;
-  group_rows[g] = ok ? offsets[id + 1] - r0 : 0;
+// The groups of a sorted batch in one CTA: head flags (a new ID starts at
+// sorted position i), their exclusive scan (the group of each head) and the
+// group arrays, in the coalesced warp-segment layout of k_scan_multi.
+__global__ void __launch_bounds__(SCAN_THREADS)
+    k_group_scan(const int32_t *__restrict__ sorted, int64_t n,
+                 const int32_t *__restrict__ offsets, int64_t vocab, int32_t *__restrict__ group_ids,
+                 int32_t *__restrict__ group_tok_start, int32_t *__restrict__ group_row_start,
+                 int32_t *__restrict__ group_rows, int32_t *info) {
+  __shared__ int32_t warp_sums[SCAN_THREADS / 32];
+  __shared__ int32_t chunk_total;
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  int32_t carry = 0;
+  for (int64_t base = 0; base < n; base += SCAN_CHUNK) {
+    const int64_t seg = base + (int64_t)warp * (SCAN_ITEMS * 32);
+    int32_t id[SCAN_ITEMS], v[SCAN_ITEMS], incl[SCAN_ITEMS];
+#pragma unroll
+    for (int r = 0; r < SCAN_ITEMS; ++r) {
+      const int64_t i = seg + r * 32 + lane;
+      id[r] = i < n ? sorted[i] : 0;
+      v[r] = i < n && (i == 0 || id[r] != sorted[i - 1]) ? 1 : 0;
+    }
+    int32_t run = 0;  // heads in earlier rounds of this warp's segment
+#pragma unroll
+    for (int r = 0; r < SCAN_ITEMS; ++r) {
+      int32_t x = v[r];
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int32_t t = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += t;
+      }
+      incl[r] = x + run;
+      run += __shfl_sync(0xffffffffu, x, 31);
+    }
+    if (lane == 0) warp_sums[warp] = run;
+    __syncthreads();
+    if (warp == 0) {
+      const int32_t w = warp_sums[lane];
+      int32_t wi = w;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int32_t t = __shfl_up_sync(0xffffffffu, wi, o);
+        if (lane >= o) wi += t;
+      }
+      warp_sums[lane] = wi - w;
+      if (lane == 31) chunk_total = wi;
+    }
+    __syncthreads();
+    const int32_t off = carry + warp_sums[warp];
+#pragma unroll
+    for (int r = 0; r < SCAN_ITEMS; ++r) {
+      if (v[r]) {
+        const int64_t i = seg + r * 32 + lane;
+        const int32_t g = off + incl[r] - 1;
+        group_ids[g] = id[r];
+        group_tok_start[g] = (int32_t)i;
+        const bool ok = id[r] >= 0 && id[r] < vocab;
+        const int32_t r0 = ok ? offsets[id[r]] : 0;
+        group_row_start[g] = r0;
+        group_rows[g] = ok ? offsets[id[r] + 1] - r0 : 0;
+      }
+    }
+    carry += chunk_total;
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    group_tok_start[carry] = (int32_t)n;
+    info[INFO_G] = carry;
+  }
 }
 
 __global__ void k_item_counts(const int32_t *__restrict__ group_tok_start,
@@ -690,7 +737,6 @@ size_t plan_scratch_bytes(int64_t n) {
   size_t ints = 0;
   ints += 2 * (size_t)n;                 // ping-pong keys / vals
   ints += (size_t)RADIX * tiles + 1;     // histogram / offsets
-  ints += 2 * ((size_t)n + 1);           // head flags, group positions
   ints += 2 * ((size_t)n + 1);           // dense tiles and tail items per group
   ints += 64;                            // info block
   ints += 2 * (N_CLASSES * MAX_DT_BUCKETS + 1);  // tail items per bucket, and their cursors
@@ -723,10 +769,6 @@ l3_status build_plan(l3_plan_s *p, const int32_t *ids, const int32_t *offsets, c
   int64_t n_tiles = std::max<int64_t>(1, (n + SORT_TILE - 1) / SORT_TILE);
   int32_t *hist = sp;
   sp += RADIX * n_tiles + 1;
-  int32_t *head = sp;
-  sp += cap;
-  int32_t *gpos = sp;
-  sp += cap;
   int32_t *tiles = sp;
   sp += cap;
   int32_t *tails = sp;
@@ -842,24 +884,18 @@ l3_status build_plan(l3_plan_s *p, const int32_t *ids, const int32_t *offsets, c
       if (!raw) scan_multi({{hist, hist, RADIX * n_tiles, nullptr}}, s);
       {
         LaunchTimer t("plan_radix_scatter", s);
-        k_radix_scatter<<<(int)n_tiles, SORT_THREADS, 0, s>>>(kin, vin, kout, vout, n, shift, hist,
-                                                             (int)n_tiles, raw);
+        k_radix_scatter<<<(int)n_tiles, SORT_THREADS, 0, s>>>(
+            kin, vin, kout, vout, n, shift, hist, (int)n_tiles, raw,
+            pass == passes - 1 ? p->inv_perm : nullptr);
       }
       kin = kout;
       vin = vout;
     }
     {
-      LaunchTimer t("plan_group_heads", s);
-      k_group_heads<<<blocks_for(n, 256), 256, 0, s>>>(p->sorted_ids, p->perm, n, head,
-                                                       p->inv_perm);
-    }
-    scan_multi({{head, gpos, n, &info[INFO_G]}}, s);
-    L3_CUDA_TRY(cudaMemsetAsync(p->group_rows, 0, cap * sizeof(int32_t), s));
-    {
-      LaunchTimer t("plan_group_fill", s);
-      k_group_fill<<<blocks_for(n, 256), 256, 0, s>>>(p->sorted_ids, head, gpos, n, offsets, vocab,
-                                                      p->group_ids, p->group_tok_start,
-                                                      p->group_row_start, p->group_rows, info);
+      LaunchTimer t("plan_group_scan", s);
+      k_group_scan<<<1, SCAN_THREADS, 0, s>>>(p->sorted_ids, n, offsets, vocab, p->group_ids,
+                                              p->group_tok_start, p->group_row_start,
+                                              p->group_rows, info);
     }
     const int n_buckets = N_CLASSES * (k_cap + 1);
     L3_CUDA_TRY(cudaMemsetAsync(dcount, 0, n_buckets * sizeof(int32_t), s));
@@ -873,7 +909,7 @@ l3_status build_plan(l3_plan_s *p, const int32_t *ids, const int32_t *offsets, c
     }
     // three independent scans in one launch: d_t over groups (segment row
     // offsets), dense tiles over d_t buckets, tail items over (class, d_t) buckets
-    scan_multi({{p->group_rows, p->seg_rows, n, &info[INFO_ROWS]},
+    scan_multi({{p->group_rows, p->seg_rows, n, &info[INFO_ROWS], &info[INFO_G]},
                 {tcount, tcursor, k_cap + 1, &info[INFO_TILES]},
                 {dcount, dcursor, n_buckets, &info[INFO_TAILS]}},
                s);
@@ -978,7 +1014,7 @@ l3_status radix_sort_pairs(const int32_t *keys_in, const int32_t *vals_in, int64
     jobs.job[0] = ScanJob{hist, hist, RADIX * n_tiles, nullptr};
     k_scan_multi<<<1, SCAN_THREADS, 0, s>>>(jobs);
     k_radix_scatter<<<(int)n_tiles, SORT_THREADS, 0, s>>>(kin, vin, kout, vout, n, shift, hist,
-                                                         (int)n_tiles, 0);
+                                                         (int)n_tiles, 0, nullptr);
     kin = kout;
     vin = vout;
   }
@@ -1121,7 +1157,7 @@ extern "C" l3_status l3_sort_tokens_noalloc(const int32_t *token_ids, int64_t n_
       k_scan_multi<<<1, SCAN_THREADS, 0, s>>>(jobs);
     }
     k_radix_scatter<<<(int)n_tiles, SORT_THREADS, 0, s>>>(kin, vin, kout, vout, n, shift, hist,
-                                                         (int)n_tiles, 0);
+                                                         (int)n_tiles, 0, nullptr);
     kin = kout;
     vin = vout;
   }
