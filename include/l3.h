@@ -261,7 +261,7 @@ l3_status l3_backward(const void *x, l3_plan_t plan, const void *W_K, const void
  * The four buffers must not overlap one another (an overlap is rejected with
  * L3_ERR_INVALID_ARG: the sort reads its input while other blocks write).
  *
- * Scratch: a file-scope device array of 557,312 bytes (2 x 65536 keys and
+ * Scratch: a file-scope device array of 590,080 bytes (2 x 65536 keys and
  * values plus the digit histogram) that every GPU which loads libl3.so holds
  * until the process exits. The first call on a device looks up the array's
  * device address (cudaGetSymbolAddress) with that device current; make that

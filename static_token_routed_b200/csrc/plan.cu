@@ -21,7 +21,7 @@
 namespace l3 {
 namespace {
 
-constexpr int RADIX_BITS = 8;
+constexpr int RADIX_BITS = 9;  // 18-bit IDs (vocab <= 262144) in two passes
 constexpr int RADIX = 1 << RADIX_BITS;
 constexpr int SORT_THREADS = 256;
 constexpr int SORT_WARPS = SORT_THREADS / 32;
@@ -126,7 +126,7 @@ __global__ void __launch_bounds__(SORT_THREADS)
 // walks it in order, ranking equal digits with __match_any_sync, so the output
 // keeps input order among equal digits.
 constexpr int FUSED_SCAN_TILES = 64;
-static_assert(RADIX == SORT_THREADS, "one thread per digit");
+static_assert(RADIX % SORT_THREADS == 0, "whole digits per thread");
 
 __global__ void __launch_bounds__(SORT_THREADS)
     k_radix_scatter(const int32_t *__restrict__ keys_in, const int32_t *__restrict__ vals_in,
@@ -160,31 +160,43 @@ __global__ void __launch_bounds__(SORT_THREADS)
   }
   __syncthreads();
   {
-    const int d = threadIdx.x;  // one digit per thread
-    int32_t run = 0;
+    // DPT consecutive digits per thread
+    constexpr int DPT = RADIX / SORT_THREADS;
+    int32_t pre[DPT], tot[DPT];
 #pragma unroll
-    for (int w = 0; w < SORT_WARPS; ++w) {
-      int32_t c = whist[w][d];
-      whist[w][d] = run;
-      run += c;
-    }
-    if (!raw) {
-      dbase[d] = offs[(int64_t)d * n_tiles + blockIdx.x];
-    } else {
-      int32_t pre = 0, tot = 0;  // digit d in earlier tiles, in all tiles
-      const int32_t *row = offs + (int64_t)d * n_tiles;
-      for (int t0 = 0; t0 < n_tiles; t0 += 16) {
-        int32_t c[16];  // sixteen loads in flight
+    for (int j = 0; j < DPT; ++j) {
+      const int d = threadIdx.x * DPT + j;
+      int32_t run = 0;
 #pragma unroll
-        for (int u = 0; u < 16; ++u) c[u] = t0 + u < n_tiles ? row[t0 + u] : 0;
+      for (int w = 0; w < SORT_WARPS; ++w) {
+        int32_t c = whist[w][d];
+        whist[w][d] = run;
+        run += c;
+      }
+      pre[j] = tot[j] = 0;
+      if (!raw) {
+        dbase[d] = offs[(int64_t)d * n_tiles + blockIdx.x];
+      } else {
+        // digit d in earlier tiles, in all tiles
+        const int32_t *row = offs + (int64_t)d * n_tiles;
+        for (int t0 = 0; t0 < n_tiles; t0 += 16) {
+          int32_t c[16];  // sixteen loads in flight
 #pragma unroll
-        for (int u = 0; u < 16; ++u) {
-          tot += c[u];
-          pre += t0 + u < (int)blockIdx.x ? c[u] : 0;
+          for (int u = 0; u < 16; ++u) c[u] = t0 + u < n_tiles ? row[t0 + u] : 0;
+#pragma unroll
+          for (int u = 0; u < 16; ++u) {
+            tot[j] += c[u];
+            pre[j] += t0 + u < (int)blockIdx.x ? c[u] : 0;
+          }
         }
       }
-      // exclusive scan of the digit totals across the CTA (digits in thread order)
-      int32_t incl = tot;
+    }
+    if (raw) {
+      // exclusive scan of the digit totals across the CTA (digits in order)
+      int32_t mine = 0;
+#pragma unroll
+      for (int j = 0; j < DPT; ++j) mine += tot[j];
+      int32_t incl = mine;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
         const int32_t v = __shfl_up_sync(0xffffffffu, incl, o);
@@ -192,9 +204,13 @@ __global__ void __launch_bounds__(SORT_THREADS)
       }
       if (lane == 31) wtot[warp] = incl;
       __syncthreads();
-      int32_t before = 0;
+      int32_t before = incl - mine;
       for (int w = 0; w < warp; ++w) before += wtot[w];
-      dbase[d] = before + incl - tot + pre;
+#pragma unroll
+      for (int j = 0; j < DPT; ++j) {
+        dbase[threadIdx.x * DPT + j] = before + pre[j];
+        before += tot[j];
+      }
     }
   }
   __syncthreads();
@@ -855,7 +871,7 @@ l3_status build_plan(l3_plan_s *p, const int32_t *ids, const int32_t *offsets, c
                                                               info);
   }
   if (n > 0) {
-    // number of 8-bit digits that cover IDs 0..vocab-1
+    // number of radix digits that cover IDs 0..vocab-1
     int bits = 1;
     while (bits < 31 && ((int64_t)1 << bits) < vocab) ++bits;
     int passes = (bits + RADIX_BITS - 1) / RADIX_BITS;

@@ -7,7 +7,7 @@ array inside libl3.so. Its outputs must equal, bit for bit (integer work),
 both the oracle's stable counting sort and what l3_plan produces for the
 same IDs, on two calls in a row, since the second call finds the first
 call's data in the shared array. The cases cover one, two and three radix
-passes (vocab <= 256, <= 65536, larger). This file is collected last so
+passes of 9-bit digits (vocab <= 512, <= 262144, larger). This file is collected last so
 that a failure here stops a `-x` run only after every other test has run.
 """
 import ctypes
@@ -47,7 +47,7 @@ def _noalloc_sort_via_c_abi(ids: torch.Tensor, vocab: int):
     return out
 
 
-@pytest.mark.parametrize("vocab,n", [(180000, 65536), (32000, 3000), (200, 5000)])
+@pytest.mark.parametrize("vocab,n", [(300000, 65536), (180000, 65536), (32000, 3000), (200, 5000)])
 def test_noalloc_sort_matches_plan_twice(vocab, n):
     for call, seed in enumerate((11, 12)):   # two calls in a row, different batches
         rng = np.random.default_rng(seed + vocab)
