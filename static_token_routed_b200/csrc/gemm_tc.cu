@@ -464,18 +464,27 @@ __global__ void __launch_bounds__(MixCfg<MODE>::THREADS, 1)
       } else if (MODE == MODE_UP_Z) {
         // z tile: per-row (mean, M2) in 32-column chunks merged in order, and
         // the fp16 values into the staging boxes (128-byte swizzle)
-        if (stored) {
-          if (warp == 2 && lane == 0) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
-          epi_bar_sync<EPI_T>();
-        }
         const int nv = min(BN, P.N - n0);
         float n_acc_f = 0.f, mean = 0.f, m2 = 0.f;
         bool range_ok = true;
+        bool staging_free = !stored;  // the same in every epilogue thread
 #pragma unroll 1
         for (int c = c_first; c < BN / 32; c += c_step) {
           uint32_t v[32];
           tmem_ld32(tacc + c * 32, v);
           tmem_wait_ld();
+          if (c + c_step >= BN / 32) {
+            // the tile's TMEM is read: the accumulator is free for the MMAs
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(tempty0[acc]);
+          }
+          if (!staging_free) {
+            // the previous tile's TMA store must have read the staging buffer
+            if (warp == 2 && lane == 0) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+            epi_bar_sync<EPI_T>();
+            staging_free = true;
+          }
           const int cv = min(32, nv - c * 32);
           if (cv > 0) {
             float sum = 0.f;
@@ -567,9 +576,11 @@ __global__ void __launch_bounds__(MixCfg<MODE>::THREADS, 1)
           }
         }
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(tempty0[acc]);
+      if (MODE != MODE_UP_Z) {  // MODE_UP_Z released the accumulator after its last TMEM read
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(tempty0[acc]);
+      }
     }
     if (MODE == MODE_UP_Z && stored && warp == 2 && lane == 0)
       asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
