@@ -122,7 +122,7 @@ constexpr int TT = 64;
 // normalised on the way, out[c][r] = gamma[c] (z[r][c] - mean_r) / std_r + beta[c],
 // from the forward's per-256-column (mean, M2) of each row.
 struct LnApply {
-  const float2 *stats;  // [R][n_chunks], nullptr: plain transpose
+  const float2 *stats;  // [n_chunks][R], nullptr: plain transpose
   int n_chunks;
   const void *gamma, *beta;
   int wtype;  // weight type of gamma / beta
@@ -143,7 +143,7 @@ __global__ void __launch_bounds__(256)
       if (tid < TT && r0 + tid < R) {
         float n = 0.f, mean = 0.f, m2 = 0.f;
         for (int k = 0; k < ln.n_chunks; ++k) {
-          const float2 st = ln.stats[(r0 + tid) * ln.n_chunks + k];
+          const float2 st = ln.stats[k * R + r0 + tid];
           const float nb = (float)min((int64_t)256, C - 256 * k);
           const float nn = n + nb, dl = st.x - mean;
           mean += dl * (nb / nn);

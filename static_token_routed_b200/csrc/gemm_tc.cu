@@ -54,7 +54,7 @@ struct MixParams {
   int64_t ldy;
   uint32_t idesc0, idesc1;  // instruction descriptors of the two ranges (MODE_F32)
   // MODE_UP_Z writes, MODE_MIX_LN reads: (mean, M2) of each row over each
-  // 256-column tile of z, [M][n_chunks]
+  // 256-column tile of z, [n_chunks][M] (a warp's 32 rows are adjacent)
   float2 *stats;
   int n_chunks;
   const float *ccol, *dcol;  // MODE_MIX_LN: c = W' 1 and d = W_mix[:, :d_up] beta, [N] each
@@ -172,6 +172,57 @@ __device__ __forceinline__ void chan_merge(float &n_a, float &mean_a, float &m2_
   n_a = n;
 }
 
+// Packed pairs of fp32 lanes (sm_100a `.f32x2` arithmetic): half the issue
+// slots of scalar adds and FMAs in the z epilogue's row statistics.
+__device__ __forceinline__ uint64_t f2_pack(uint32_t lo, uint32_t hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(lo), "r"(hi));
+  return r;
+}
+__device__ __forceinline__ float f2_hsum(uint64_t a) {
+  uint32_t lo, hi;
+  asm("mov.b64 {%0, %1}, %2;" : "=r"(lo), "=r"(hi) : "l"(a));
+  return __uint_as_float(lo) + __uint_as_float(hi);
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+
+// mean and sum of squared deviations of 32 fp32 values, in two passes (the
+// mean first, then the deviations from it), lanes paired, two partial sums
+// per pass
+__device__ __forceinline__ void stats32(const uint32_t (&v)[32], float &mean, float &m2) {
+  uint64_t s0 = f2_pack(v[0], v[1]), s1 = f2_pack(v[2], v[3]);
+#pragma unroll
+  for (int e = 4; e < 32; e += 4) {
+    s0 = f2_add(s0, f2_pack(v[e], v[e + 1]));
+    s1 = f2_add(s1, f2_pack(v[e + 2], v[e + 3]));
+  }
+  mean = f2_hsum(f2_add(s0, s1)) * (1.f / 32.f);
+  const uint64_t mm = f2_pack(__float_as_uint(mean), __float_as_uint(mean));
+  uint64_t q0 = 0, q1 = 0;  // (+0.f, +0.f)
+#pragma unroll
+  for (int e = 0; e < 32; e += 4) {
+    const uint64_t d0 = f2_sub(f2_pack(v[e], v[e + 1]), mm);
+    const uint64_t d1 = f2_sub(f2_pack(v[e + 2], v[e + 3]), mm);
+    q0 = f2_fma(d0, d0, q0);
+    q1 = f2_fma(d1, d1, q1);
+  }
+  m2 = f2_hsum(f2_add(q0, q1));
+}
+
 // Kernel forms:
 //   MODE_F32:    C = A B^T (+ A1 B1^T), fp32 output (the backward pass's GEMMs)
 //   MODE_UP_Z:   z = a W_up^T, fp16 output through shared memory and TMA stores,
@@ -266,6 +317,8 @@ __global__ void __launch_bounds__(MixCfg<MODE>::THREADS, 1)
                     const __grid_constant__ CUtensorMap mA1, const __grid_constant__ CUtensorMap mB1,
                     const __grid_constant__ CUtensorMap mZ, MixParams P) {
   using Cfg = MixCfg<MODE>;
+  // MODE_UP_Z's constant-weight statistics merge: two 32-column chunks per warp
+  static_assert(MODE != MODE_UP_Z || BN / 32 == 2 * (Cfg::EPI_WARPS / 4), "z epilogue chunk split");
   constexpr int STAGES = Cfg::STAGES;
   constexpr int EPI_T = 32 * Cfg::EPI_WARPS;  // epilogue threads
   extern __shared__ uint8_t smem_raw[];
@@ -436,7 +489,7 @@ __global__ void __launch_bounds__(MixCfg<MODE>::THREADS, 1)
         float n_acc_f = 0.f, mean = 0.f, m2 = 0.f;
         if (m < P.M)
           for (int c = 0; c < P.n_chunks; ++c) {
-            const float2 st = P.stats[(int64_t)m * P.n_chunks + c];
+            const float2 st = P.stats[(int64_t)c * P.M + m];
             chan_merge(n_acc_f, mean, m2, (float)min(BN, P.kb0 * BK - c * BN), st.x, st.y);
           }
         const float rs = m < P.M ? rsqrtf(m2 / n_acc_f + P.eps) : 0.f;
@@ -465,6 +518,9 @@ __global__ void __launch_bounds__(MixCfg<MODE>::THREADS, 1)
         // z tile: per-row (mean, M2) in 32-column chunks merged in order, and
         // the fp16 values into the staging boxes (128-byte swizzle)
         const int nv = min(BN, P.N - n0);
+        // every chunk of the tile holds 32 columns (d_up a multiple of 256
+        // or an inner tile): chunk sizes and merge weights are constants
+        const bool full = nv == BN;
         float n_acc_f = 0.f, mean = 0.f, m2 = 0.f;
         bool range_ok = true;
         bool staging_free = !stored;  // the same in every epilogue thread
@@ -486,7 +542,23 @@ __global__ void __launch_bounds__(MixCfg<MODE>::THREADS, 1)
             staging_free = true;
           }
           const int cv = min(32, nv - c * 32);
-          if (cv > 0) {
+          bool check = !full;  // test each value against fp16's range
+          if (full) {
+            float mc, qc;
+            stats32(v, mc, qc);
+            if (c == c_first) {
+              mean = mc;
+              m2 = qc;
+            } else {  // two 32-column chunk sets: weights 1/2 and 32 * 32 / 64
+              const float delta = mc - mean;
+              mean += delta * 0.5f;
+              m2 += qc + delta * delta * 16.f;
+            }
+            // every value lies within sqrt(qc) of mc; the margin below 65504
+            // covers the rounding of mc and qc, and NaN or Inf fail the test
+            const float lim = 65000.f - fabsf(mc);
+            check = !(lim > 0.f && qc <= lim * lim);
+          } else if (cv > 0) {
             float sum = 0.f;
 #pragma unroll
             for (int e = 0; e < 32; ++e)
@@ -501,18 +573,18 @@ __global__ void __launch_bounds__(MixCfg<MODE>::THREADS, 1)
               }
             chan_merge(n_acc_f, mean, m2, (float)cv, mc, qc);
           }
+          if (check)
+#pragma unroll
+            for (int e = 0; e < 32; ++e) range_ok &= fabsf(__uint_as_float(v[e])) <= 65504.f;
           uint8_t *box = staging + (c / 2) * (BM * 128);
 #pragma unroll
           for (int jj = 0; jj < 4; ++jj) {
             uint4 o;
             __half2 *o2 = reinterpret_cast<__half2 *>(&o);
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const float z0 = __uint_as_float(v[jj * 8 + 2 * e]);
-              const float z1 = __uint_as_float(v[jj * 8 + 2 * e + 1]);
-              range_ok &= fabsf(z0) <= 65504.f && fabsf(z1) <= 65504.f;
-              o2[e] = __floats2half2_rn(z0, z1);
-            }
+            for (int e = 0; e < 4; ++e)
+              o2[e] = __floats2half2_rn(__uint_as_float(v[jj * 8 + 2 * e]),
+                                        __uint_as_float(v[jj * 8 + 2 * e + 1]));
             const int chunk = (c % 2) * 4 + jj;  // 16-byte chunk within the box's 128-byte row
             *reinterpret_cast<uint4 *>(box + r * 128 + ((chunk ^ (r & 7)) << 4)) = o;
           }
@@ -530,11 +602,23 @@ __global__ void __launch_bounds__(MixCfg<MODE>::THREADS, 1)
         fence_proxy_async_smem();
         epi_bar_sync<EPI_T>();
         if (c_first == 0 && m < P.M) {
-          for (int k = 0; k < c_step - 1; ++k) {
-            const float *pp = part + k * 3 * BM;
-            chan_merge(n_acc_f, mean, m2, pp[r], pp[BM + r], pp[2 * BM + r]);
+          if (full) {
+            // equal 64-column sets: the k-th merge weighs 1 / (k + 2) and
+            // 64 (k + 1) / (k + 2)
+#pragma unroll
+            for (int k = 0; k < c_step - 1; ++k) {
+              const float *pp = part + k * 3 * BM;
+              const float delta = pp[BM + r] - mean;
+              mean += delta * (1.f / (float)(k + 2));
+              m2 += pp[2 * BM + r] + delta * delta * (64.f * (float)(k + 1) / (float)(k + 2));
+            }
+          } else {
+            for (int k = 0; k < c_step - 1; ++k) {
+              const float *pp = part + k * 3 * BM;
+              chan_merge(n_acc_f, mean, m2, pp[r], pp[BM + r], pp[2 * BM + r]);
+            }
           }
-          P.stats[(int64_t)m * P.n_chunks + n0 / BN] = make_float2(mean, m2);
+          P.stats[(int64_t)(n0 / BN) * P.M + m] = make_float2(mean, m2);
         }
         if (warp == 2 && lane == 0) {
           const int mrow = (tile / P.n_tiles_n) * (2 * BM) + (int)rank * BM;

@@ -114,7 +114,7 @@ struct l3_plan_s {
   float *z_buf = nullptr;              // [N x d_up] fp32 (CUDA-core GEMM path only)
   void *w_up16 = nullptr;              // [d_up x d_emb] fp16 copy of W_up (tensor-core path)
   void *w_mixh16 = nullptr;            // [d_out x d_up] fp16 W_mix[:, :d_up] diag(gamma)
-  float2 *ln_stats = nullptr;          // [N x ceil(d_up / 256)] (mean, M2) of z per 256 columns
+  float2 *ln_stats = nullptr;          // [ceil(d_up / 256) x N] (mean, M2) of z per 256 columns
   float *mix_ccol = nullptr;           // W' 1 [d_out], then W_mix[:, :d_up] beta at a 16-byte
                                        // aligned offset
   bool tc_gemm = false;                // tensor-core GEMMs in use
