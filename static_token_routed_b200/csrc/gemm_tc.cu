@@ -41,10 +41,6 @@ constexpr int BM = 128;  // tokens per tile (TMEM lanes)
 constexpr int BK = 64;   // 64 16-bit elements = one 128-byte swizzle row
 constexpr int BN = 256;  // output columns per tile (max N of one MMA)
 constexpr int A_BYTES = BM * BK * 2;
-constexpr int B_BYTES = BN * BK * 2;
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-constexpr int GEMM_THREADS = 192;  // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
-constexpr uint32_t IDESC_F16 = idesc_f16(0, 0, BM, BN);
 
 struct MixParams {
   int M, N;        // rows (tokens), output columns
@@ -471,7 +467,7 @@ __global__ void __launch_bounds__(MixCfg<MODE>::THREADS, 1)
                                  map_shared_rank(&b->tempty[1], 0)};
     int n_acc[2] = {0, 0};
     int k, rng, acc;
-    bool stored = false;  // MODE_UP_Z: a TMA store may still be reading the staging buffer
+    bool stored = false;  // MODE_UP_Z: TMA stores may still be reading the staging buffer
     for (int j = 0; mix_job<MODE>(j, k_tiles, k, rng, acc); ++j) {
       const int na = acc ? n_acc[1] : n_acc[0];
       if (acc) ++n_acc[1]; else ++n_acc[0];
@@ -523,30 +519,45 @@ __global__ void __launch_bounds__(MixCfg<MODE>::THREADS, 1)
         const bool full = nv == BN;
         float n_acc_f = 0.f, mean = 0.f, m2 = 0.f;
         bool range_ok = true;
-        bool staging_free = !stored;  // the same in every epilogue thread
+        const int mrow = (tile / P.n_tiles_n) * (2 * BM) + (int)rank * BM;
+        // The staging buffer's two halves (columns 0-127: every warp's first
+        // chunk; 128-255: its second) go out as separate TMA store groups, the
+        // first as soon as it is written, so each half has about half a tile's
+        // time to be read out before the next tile writes it again. Groups are
+        // committed in the order first(t-1), second(t-1), first(t), ...
 #pragma unroll 1
-        for (int c = c_first; c < BN / 32; c += c_step) {
+        for (int i = 0; i < 2; ++i) {
+          const int c = c_first + i * c_step;
           uint32_t v[32];
           tmem_ld32(tacc + c * 32, v);
           tmem_wait_ld();
-          if (c + c_step >= BN / 32) {
+          if (i == 1) {
             // the tile's TMEM is read: the accumulator is free for the MMAs
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(tempty0[acc]);
-          }
-          if (!staging_free) {
-            // the previous tile's TMA store must have read the staging buffer
+            // every warp has written the first half, and the previous tile's
+            // second half has been read out (the newest group): store the
+            // first half
             if (warp == 2 && lane == 0) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
             epi_bar_sync<EPI_T>();
-            staging_free = true;
+            if (warp == 2 && lane == 0) {
+              for (int bx = 0; bx < 2 && bx * 64 < nv; ++bx)
+                tma_store_2d_box(&mZ, staging + bx * (BM * 128), n0 + bx * 64, mrow);
+              asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+            }
+          } else if (stored) {
+            // the previous tile's first half has been read out (all groups
+            // but the newest)
+            if (warp == 2 && lane == 0) asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+            epi_bar_sync<EPI_T>();
           }
           const int cv = min(32, nv - c * 32);
           bool check = !full;  // test each value against fp16's range
           if (full) {
             float mc, qc;
             stats32(v, mc, qc);
-            if (c == c_first) {
+            if (i == 0) {
               mean = mc;
               m2 = qc;
             } else {  // two 32-column chunk sets: weights 1/2 and 32 * 32 / 64
@@ -588,6 +599,8 @@ __global__ void __launch_bounds__(MixCfg<MODE>::THREADS, 1)
             const int chunk = (c % 2) * 4 + jj;  // 16-byte chunk within the box's 128-byte row
             *reinterpret_cast<uint4 *>(box + r * 128 + ((chunk ^ (r & 7)) << 4)) = o;
           }
+          // this thread's staging writes, visible to the TMA store
+          fence_proxy_async_smem();
         }
         if (!range_ok) atomicOr(P.err, DEV_ERR_F16_RANGE);
         // the statistics of a row's chunk sets (one per warp of its quarter)
@@ -599,7 +612,6 @@ __global__ void __launch_bounds__(MixCfg<MODE>::THREADS, 1)
           pp[BM + r] = mean;
           pp[2 * BM + r] = m2;
         }
-        fence_proxy_async_smem();
         epi_bar_sync<EPI_T>();
         if (c_first == 0 && m < P.M) {
           if (full) {
@@ -620,9 +632,8 @@ __global__ void __launch_bounds__(MixCfg<MODE>::THREADS, 1)
           }
           P.stats[(int64_t)(n0 / BN) * P.M + m] = make_float2(mean, m2);
         }
-        if (warp == 2 && lane == 0) {
-          const int mrow = (tile / P.n_tiles_n) * (2 * BM) + (int)rank * BM;
-          for (int bx = 0; bx * 64 < nv; ++bx)
+        if (warp == 2 && lane == 0) {  // the second half
+          for (int bx = 2; bx * 64 < nv; ++bx)
             tma_store_2d_box(&mZ, staging + bx * (BM * 128), n0 + bx * 64, mrow);
           asm volatile("cp.async.bulk.commit_group;" ::: "memory");
         }
