@@ -415,6 +415,24 @@ l3_status l3_plan_export(l3_plan_t p, int32_t *perm, int32_t *inv_perm, int32_t 
   return L3_OK;
 }
 
+// Dense attention on the caller's stream: the d_t > 256 tiles of more than
+// SKINNY_TOKENS tokens (one CTA per SM, the longest), then every tile of at
+// most SKINNY_TOKENS tokens (transposed products, one CTA per SM beside the
+// tail kernels), then the other d_t <= 256 tiles. The skinny kernel takes its
+// tiles only where there are at least four per SM: with fewer, its launch
+// adds a ramp down of its own to the two others' (small_bf16, 271 such
+// tiles: 0.266 -> 0.278 ms per batch; dense_stress, 16: 0.837 -> 0.960 ms),
+// and the two configurations take all of their tiles.
+static l3_status launch_dense_all(const l3_plan_s *p, const void *x, const void *W_K,
+                                  const void *W_V, cudaStream_t s) {
+  const bool skinny = skinny_attention_supported(p->dims) &&
+                      p->n_skinny_big + p->n_skinny_small >= 4 * (int64_t)sm_count(p->device);
+  l3_status st = launch_attn_dense(p, x, W_K, W_V, false, skinny, s);
+  if (st == L3_OK && skinny) st = launch_attn_skinny(p, x, W_K, W_V, s);
+  if (st == L3_OK) st = launch_attn_dense(p, x, W_K, W_V, true, skinny, s);
+  return st;
+}
+
 l3_status l3_forward(const void *x, l3_plan_t p, const void *W_K, const void *W_V,
                      const void *W_up, const void *ln_gamma, const void *ln_beta,
                      const void *W_mix, void *y, void *stream) {
@@ -445,7 +463,6 @@ l3_status l3_forward(const void *x, l3_plan_t p, const void *W_K, const void *W_
   p->stream = s;
   l3_status st = L3_OK;
   const bool has_big = p->n_dense_tiles > p->n_dense_small;
-  const bool has_small = p->n_dense_small > 0;
   const bool has_tail = p->n_tail_items > 0;
   if (has_tail && tail_cls_supported(p->dims)) {
     // fork: dense attention (both configurations, in turn) on the caller's
@@ -458,8 +475,7 @@ l3_status l3_forward(const void *x, l3_plan_t p, const void *W_K, const void *W_
     std::lock_guard<std::mutex> lk(aux->mu);
     L3_CUDA_TRY(cudaEventRecord(aux->fork, s));
     for (int i = 0; i < N_AUX; ++i) L3_CUDA_TRY(cudaStreamWaitEvent(aux->stream[i], aux->fork, 0));
-    if (st == L3_OK) st = launch_attn_dense(p, x, W_K, W_V, false, s);
-    if (st == L3_OK) st = launch_attn_dense(p, x, W_K, W_V, true, s);
+    if (st == L3_OK) st = launch_dense_all(p, x, W_K, W_V, s);
     // next to the big dense configuration (one CTA per SM, streaming K_t)
     // the tails stay on one helper stream: spread over three they take SMs
     // and bandwidth from it (paper_shaped: 1.64 -> 1.72 ms per batch); with
@@ -475,12 +491,10 @@ l3_status l3_forward(const void *x, l3_plan_t p, const void *W_K, const void *W_
     }
   } else if (has_tail) {
     st = launch_attn_tail(p, x, W_K, W_V, s);
-    if (st == L3_OK) st = launch_attn_dense(p, x, W_K, W_V, false, s);
-    if (st == L3_OK) st = launch_attn_dense(p, x, W_K, W_V, true, s);
+    if (st == L3_OK) st = launch_dense_all(p, x, W_K, W_V, s);
     if (st == L3_OK && p->tc_gemm) st = launch_weights_f16(p, W_up, W_mix, ln_gamma, ln_beta, s);
   } else {
-    if (st == L3_OK) st = launch_attn_dense(p, x, W_K, W_V, false, s);
-    if (st == L3_OK) st = launch_attn_dense(p, x, W_K, W_V, true, s);
+    if (st == L3_OK) st = launch_dense_all(p, x, W_K, W_V, s);
     if (st == L3_OK && p->tc_gemm) st = launch_weights_f16(p, W_up, W_mix, ln_gamma, ln_beta, s);
   }
   if (p->tc_gemm) {

@@ -110,6 +110,7 @@ struct DenseParams {
   const DenseTile *tiles;
   int n_tiles;
   int *counter;    // [0] next tile to claim, [1] CTAs finished; the last CTA zeroes both
+  int skip_skinny;  // leave tiles of at most SKINNY_TOKENS tokens to attn_skinny.cu
   int d_in, d_emb;
   int *err;
 };
@@ -280,7 +281,11 @@ __global__ void __launch_bounds__(DENSE_THREADS, DenseCfg<SMALL>::MIN_BLOCKS)
       uint32_t armed_par[MAX_STAGES], varmed_par[MAX_STAGES];
       for (int i = 0; i < MAX_STAGES; ++i) armed[i] = varmed[i] = false;
       for (int u = 0; ok; ++u) {
-        int ti = atomicAdd(P.counter, 1);
+        int ti;
+        do {
+          ti = atomicAdd(P.counter, 1);
+        } while (P.skip_skinny && ti < P.n_tiles &&
+                 P.group_tok_start[P.tiles[ti].group + 1] - P.tiles[ti].tok0 <= SKINNY_TOKENS);
         if (ti >= P.n_tiles) ti = -1;
         const int j = u & 1;
         if (!mbar_wait(&b->tempty[j], ((u >> 1) & 1) ^ 1, ab)) {
@@ -650,15 +655,11 @@ constexpr size_t dense_smem() {
   return 1024 + DenseCfg<SMALL>::REGION + sizeof(DenseBars);
 }
 
-int sm_count(int device) {
-  static int n[64] = {};
-  if (n[device & 63] == 0) cudaDeviceGetAttribute(&n[device & 63], cudaDevAttrMultiProcessorCount, device);
-  return n[device & 63];
-}
 
 template <bool SMALL>
 l3_status launch_cfg(const CUtensorMap &mK, const CUtensorMap &mK16, const CUtensorMap &mV,
-                     DenseParams P, int64_t n_tiles, int device, const char *name, cudaStream_t s) {
+                     DenseParams P, int64_t n_tiles, int64_t n_own, int device, const char *name,
+                     cudaStream_t s) {
   if (n_tiles == 0) return L3_OK;
   static bool attr[64] = {};
   if (!attr[device & 63]) {
@@ -668,7 +669,8 @@ l3_status launch_cfg(const CUtensorMap &mK, const CUtensorMap &mK16, const CUten
     attr[device & 63] = true;
   }
   // persistent: as many CTAs as fit at once, each claiming tiles until none are left
-  const int64_t grid = std::min<int64_t>(n_tiles, (int64_t)sm_count(device) * DenseCfg<SMALL>::MIN_BLOCKS);
+  // (n_own of the n_tiles are this launch's: the others are skinny tiles)
+  const int64_t grid = std::min<int64_t>(n_own, (int64_t)sm_count(device) * DenseCfg<SMALL>::MIN_BLOCKS);
   P.n_tiles = (int)n_tiles;
   LaunchTimer t(name, s);
   k_attn_dense<SMALL><<<(unsigned)grid, DENSE_THREADS, dense_smem<SMALL>(), s>>>(mK, mK16, mV, P);
@@ -678,16 +680,24 @@ l3_status launch_cfg(const CUtensorMap &mK, const CUtensorMap &mK16, const CUten
 
 }  // namespace
 
+int sm_count(int device) {
+  static int n[64] = {};
+  if (n[device & 63] == 0) cudaDeviceGetAttribute(&n[device & 63], cudaDevAttrMultiProcessorCount, device);
+  return n[device & 63];
+}
+
 bool dense_attention_supported(const l3_dims_t &d) {
   return d.dtype == L3_BF16 && d.d_in % CK == 0 && d.d_emb % 64 == 0 && d.d_emb <= MAX_EMB;
 }
 int dense_attention_max_rows() { return MAX_D; }
 
 l3_status launch_attn_dense(const l3_plan_s *p, const void *x, const void *W_K, const void *W_V,
-                            bool small, cudaStream_t s) {
+                            bool small, bool skip_skinny, cudaStream_t s) {
   // the plan lists the tiles of groups with d_t > DENSE_SMALL_ROWS first
   const int64_t n_big = p->n_dense_tiles - p->n_dense_small;
-  if ((small ? p->n_dense_small : n_big) == 0) return L3_OK;
+  const int64_t n_own = small ? p->n_dense_small - (skip_skinny ? p->n_skinny_small : 0)
+                              : n_big - (skip_skinny ? p->n_skinny_big : 0);
+  if (n_own == 0) return L3_OK;
   const l3_dims_t &d = p->dims;
   CUtensorMap mK, mK16, mV;
   l3_status st;
@@ -711,10 +721,12 @@ l3_status launch_attn_dense(const l3_plan_s *p, const void *x, const void *W_K, 
   P.d_emb = (int)d.d_emb;
   P.err = p->dev_flags + 1;
   P.counter = p->dev_flags + 4;
-  if (!small) return launch_cfg<false>(mK, mK16, mV, P, n_big, p->device, "attn_dense", s);
+  P.skip_skinny = skip_skinny ? 1 : 0;
+  if (!small) return launch_cfg<false>(mK, mK16, mV, P, n_big, n_own, p->device, "attn_dense", s);
   P.tiles = p->dense_tiles + n_big;
   P.counter = p->dev_flags + 6;
-  return launch_cfg<true>(mK, mK16, mV, P, p->n_dense_small, p->device, "attn_dense_small", s);
+  return launch_cfg<true>(mK, mK16, mV, P, p->n_dense_small, n_own, p->device, "attn_dense_small",
+                          s);
 }
 
 }  // namespace l3

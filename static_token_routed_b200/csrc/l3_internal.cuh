@@ -70,6 +70,9 @@ constexpr int DENSE_MIN_ROWS = 32;
 // dense groups with at most this many rows run in a configuration that fits
 // two CTAs per SM (256 TMEM columns, O computed in 256-column passes)
 constexpr int DENSE_SMALL_ROWS = 256;
+// dense tiles with at most this many tokens (a group's last tile, or its only
+// one) run on the transposed-product kernel, tokens as the MMAs' N
+constexpr int SKINNY_TOKENS = 32;
 // tail items with at most this many rows are "small" (latency-bound)
 constexpr int TAIL_SMALL_ROWS = 16;
 
@@ -85,6 +88,9 @@ struct l3_plan_s {
   int64_t n_dense_groups = 0;
   int64_t n_dense_tiles = 0;
   int64_t n_dense_small = 0;  // the last n_dense_small tiles have d_t <= DENSE_SMALL_ROWS
+  // tiles of at most SKINNY_TOKENS tokens among the first n_dense_tiles -
+  // n_dense_small tiles and among the last n_dense_small
+  int64_t n_skinny_big = 0, n_skinny_small = 0;
   int64_t n_tail_items = 0;
   int64_t unique_rows = 0;
   int64_t unique_rows_multi = 0;
@@ -107,7 +113,7 @@ struct l3_plan_s {
   int32_t *seg_rows = nullptr;         // [N+1]
   l3::DenseTile *dense_tiles = nullptr;
   l3::TailItem *tail_items = nullptr;
-  int32_t *dev_flags = nullptr;        // [0] plan errors, [1] forward errors, [4..7] dense tile counters
+  int32_t *dev_flags = nullptr;        // [0] plan errors, [1] forward errors, [4..9] dense tile counters
   void *a_buf = nullptr;               // [N x d_emb] dtype, original token order
   void *h_buf = nullptr;               // [N x d_up] h (CUDA-core path) or z = a W_up^T (fp16,
                                        // tensor-core path: the LayerNorm is applied inside W_mix)
@@ -160,12 +166,18 @@ l3_status launch_attn_tail_cls(const l3_plan_s *p, const void *x, const void *W_
                                const void *W_V, const cudaStream_t *streams, int n_streams);
 
 // attention, tensor-core path (attn_dense.cu)
+int sm_count(int device);  // SMs of the device (cached per device)
 bool dense_attention_supported(const l3_dims_t &d);
 int dense_attention_max_rows();
 // one of the two launch configurations: tiles with d_t > DENSE_SMALL_ROWS
-// (small = false) or the others
+// (small = false) or the others; skip_skinny leaves the tiles of at most
+// SKINNY_TOKENS tokens to launch_attn_skinny
 l3_status launch_attn_dense(const l3_plan_s *p, const void *x, const void *W_K, const void *W_V,
-                            bool small, cudaStream_t s);
+                            bool small, bool skip_skinny, cudaStream_t s);
+// attention for dense tiles of at most SKINNY_TOKENS tokens (attn_skinny.cu)
+bool skinny_attention_supported(const l3_dims_t &d);
+l3_status launch_attn_skinny(const l3_plan_s *p, const void *x, const void *W_K, const void *W_V,
+                             cudaStream_t s);
 
 // GEMMs + LayerNorm, tensor-core path (gemm_tc.cu)
 bool tc_gemm_supported(const l3_dims_t &d);

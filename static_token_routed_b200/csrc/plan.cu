@@ -59,8 +59,11 @@ enum {
   INFO_CLS,              // 5 slots: first tail item of each token-count class, then the total
   INFO_SPLIT = INFO_CLS + 5,  // 4 slots: first item of each class with d_t <= TAIL_SMALL_ROWS
   INFO_DENSE_SMALL = INFO_SPLIT + 4,  // dense tiles of groups with d_t <= DENSE_SMALL_ROWS
+  INFO_SKINNY_BIG,    // dense tiles of at most SKINNY_TOKENS tokens, d_t > DENSE_SMALL_ROWS
+  INFO_SKINNY_SMALL,  // the same, d_t <= DENSE_SMALL_ROWS
   INFO_SLOTS
 };
+static_assert(INFO_SLOTS <= 64, "the plan zeroes 64 info words");
 
 __device__ __forceinline__ uint32_t lanemask_lt() {
   uint32_t m;
@@ -406,6 +409,9 @@ __global__ void k_item_counts(const int32_t *__restrict__ group_tok_start,
       nt = (c + DENSE_TILE_M - 1) / DENSE_TILE_M;
       atomicAdd(&info[INFO_DENSE_GROUPS], 1);
       if (rows <= DENSE_SMALL_ROWS) atomicAdd(&info[INFO_DENSE_SMALL], nt);
+      // the group's last tile holds c - (nt - 1) 128 tokens
+      if (c - (nt - 1) * DENSE_TILE_M <= SKINNY_TOKENS)
+        atomicAdd(&info[rows <= DENSE_SMALL_ROWS ? INFO_SKINNY_SMALL : INFO_SKINNY_BIG], 1);
       // dense tiles are listed largest d_t first (bucket k_cap - d_t): the
       // longest CTAs start first, and the d_t > DENSE_SMALL_ROWS tiles come
       // before the others
@@ -557,6 +563,7 @@ __global__ void __launch_bounds__(SMALL_THREADS, 1) k_plan_small(SmallPlanArgs A
   int32_t *tcount = dcount + (n_buckets + 1);                          // [k_cap + 2]
   int32_t *tmp = tcount + (k_cap + 2);                                 // [33]
   __shared__ int32_t s_err, s_rows_multi, s_max_tokens, s_dense_groups, s_dense_small;
+  __shared__ int32_t s_skinny[2];  // big, small
 
   if (tid == 0) {
     s_err = 0;
@@ -564,6 +571,7 @@ __global__ void __launch_bounds__(SMALL_THREADS, 1) k_plan_small(SmallPlanArgs A
     s_max_tokens = 0;
     s_dense_groups = 0;
     s_dense_small = 0;
+    s_skinny[0] = s_skinny[1] = 0;
   }
   for (int i = tid; i < n_buckets + 1; i += SMALL_THREADS) dcount[i] = 0;
   for (int i = tid; i < k_cap + 2; i += SMALL_THREADS) tcount[i] = 0;
@@ -641,6 +649,8 @@ __global__ void __launch_bounds__(SMALL_THREADS, 1) k_plan_small(SmallPlanArgs A
       const int nt = (c + DENSE_TILE_M - 1) / DENSE_TILE_M;
       atomicAdd(&s_dense_groups, 1);
       if (rows <= DENSE_SMALL_ROWS) atomicAdd(&s_dense_small, nt);
+      if (c - (nt - 1) * DENSE_TILE_M <= SKINNY_TOKENS)
+        atomicAdd(&s_skinny[rows <= DENSE_SMALL_ROWS ? 1 : 0], 1);
       atomicAdd(&tcount[db], nt);
     } else {
       const int full = c / TAIL_TOKENS, rest = c % TAIL_TOKENS;
@@ -670,6 +680,8 @@ __global__ void __launch_bounds__(SMALL_THREADS, 1) k_plan_small(SmallPlanArgs A
       info[INFO_CLS + c] = c < N_CLASSES ? dcount[c * (k_cap + 1)] : n_tails;
     for (int c = 0; c < N_CLASSES; ++c) info[INFO_SPLIT + c] = dcount[c * (k_cap + 1) + (k_cap - small)];
     info[INFO_DENSE_SMALL] = s_dense_small;
+    info[INFO_SKINNY_BIG] = s_skinny[0];
+    info[INFO_SKINNY_SMALL] = s_skinny[1];
   }
   __syncthreads();
 
@@ -970,6 +982,8 @@ l3_status finish_plan(l3_plan_s *p, const int32_t *info, int64_t n, cudaStream_t
   p->n_groups = host_info[INFO_G];
   p->n_dense_tiles = host_info[INFO_TILES];
   p->n_dense_small = host_info[INFO_DENSE_SMALL];
+  p->n_skinny_big = host_info[INFO_SKINNY_BIG];
+  p->n_skinny_small = host_info[INFO_SKINNY_SMALL];
   p->n_tail_items = host_info[INFO_TAILS];
   p->unique_rows = host_info[INFO_ROWS];
   p->unique_rows_multi = host_info[INFO_ROWS_MULTI];

@@ -129,6 +129,28 @@ def test_tensor_core_kernels_run():
     assert "mix_gemm_tc" in kernels and "up_z_gemm_tc" in kernels, kernels
 
 
+def want_dense_kernels(rows, ids, d_emb):
+    """The dense attention launches a batch needs: a group's whole 128-token
+    tiles, and its last tile when that holds more than 32 tokens, run on the
+    128-token kernel of its d_t range; a last tile of at most 32 tokens runs on
+    the transposed-product kernel when d_emb is a multiple of 128 and the batch
+    has at least four such tiles per SM (148 on a B200)."""
+    counts = torch.bincount(ids.long(), minlength=len(rows)).tolist()
+    n_skinny = sum(1 for r, c in zip(rows, counts)
+                   if c >= 5 and r >= 32 and c - 128 * ((c - 1) // 128) <= 32)
+    skinny_on = d_emb % 128 == 0 and n_skinny >= 4 * 148
+    want = set()
+    for r, c in zip(rows, counts):
+        if c < 5 or r < 32:   # a tail group
+            continue
+        full = "attn_dense" if r > 256 else "attn_dense_small"
+        last = c - 128 * ((c - 1) // 128)
+        if c > 128:
+            want.add(full)
+        want.add("attn_dense_skinny" if last <= 32 and skinny_on else full)
+    return want
+
+
 @pytest.mark.parametrize("vocab,d_t,n,d_in,d_emb,d_up,d_out", [
     (5, 37, 300, 128, 64, 64, 64),      # d_t not a multiple of 16, partial token tiles
     (3, 300, 400, 64, 192, 128, 48),    # two N halves for S, PV N = 192
@@ -164,10 +186,76 @@ def test_dense_attention_shapes(vocab, d_t, n, d_in, d_emb, d_up, d_out):
     l3.l3_forward_status(plan)
     kernels = l3.l3_profile_read()
     l3.l3_profile_enable(False)
-    want_cfg = {"attn_dense" if r > 256 else "attn_dense_small" for r in rows}
-    assert want_cfg <= set(kernels), kernels
+    assert want_dense_kernels(rows, ids, d_emb) <= set(kernels), kernels
     want = oracle_y(t, bt)
     err = rel_max_err(y.double().cpu().numpy(), want)
+    assert err <= TOL["bf16"], err
+
+
+def _grouped_layer(rows, counts, d_in, d_emb, d_up, d_out, seed):
+    """A layer whose ID i has rows[i] rows and appears counts[i] times in a
+    shuffled batch (inputs as in the shape test above)."""
+    g = torch.Generator().manual_seed(seed)
+    off = torch.tensor([0] + list(rows), dtype=torch.int64).cumsum(0).to(torch.int32)
+    v = int(off[-1])
+    mk = lambda *s: (torch.randn(*s, generator=g) / s[-1] ** 0.5).to(torch.bfloat16)  # noqa: E731
+    ids = torch.cat([torch.full((c,), i, dtype=torch.int32) for i, c in enumerate(counts)])
+    ids = ids[torch.randperm(len(ids), generator=g)].contiguous()
+    t = wl.Tables(off, mk(v, d_in) * 4, mk(v, d_emb), mk(d_up, d_emb),
+                  (1 + 0.1 * torch.randn(d_up, generator=g)).to(torch.bfloat16),
+                  (0.1 * torch.randn(d_up, generator=g)).to(torch.bfloat16), mk(d_out, d_up + d_in))
+    b = wl.Batch(ids, mk(len(ids), d_in) * 4)
+    dims = l3.make_dims(len(rows), v, max(rows), d_in, d_emb, d_up, d_out, torch.bfloat16, EPS)
+    return t, b, dims
+
+
+def _forward_kernels(t, b, dims):
+    dev = to_device(t, b)
+    plan = l3.l3_plan(dev["ids"], dev["offsets"], dims)
+    y = torch.empty(len(b.ids), dims.d_out, dtype=torch.bfloat16, device="cuda")
+    l3.l3_profile_enable(True)
+    l3.l3_forward(dev["x"], plan, dev["W_K"], dev["W_V"], dev["W_up"], dev["ln_gamma"],
+                  dev["ln_beta"], dev["W_mix"], y)
+    l3.l3_forward_status(plan)
+    kernels = l3.l3_profile_read()
+    l3.l3_profile_enable(False)
+    return y, plan, kernels
+
+
+# the transposed-product kernel takes a batch's tiles of at most 32 tokens when
+# there are at least four such tiles per SM (B200: 148 SMs)
+SKINNY_BATCH = 44
+
+
+@pytest.mark.parametrize("d_in,d_emb,seed", [(128, 512, 1), (64, 256, 2), (256, 128, 3)])
+def test_skinny_tiles_all_tokens(d_in, d_emb, seed):
+    """Dense groups of 5..32 tokens (every tile of at most 32 tokens) over
+    d_t from 32 to 512: the transposed-product kernel alone, in every M-block
+    count (d_t up to 128, 256, 384, 512), d_t on and off multiples of 16;
+    enough groups (660) for the forward to choose that kernel."""
+    base = (32, 33, 48, 100, 128, 129, 200, 256, 257, 300, 384, 385, 449, 511, 512)
+    rows = base * SKINNY_BATCH
+    counts = [5 + (3 * i + i // len(base)) % 28 for i in range(len(rows))]   # 5..32
+    counts[0], counts[-1] = 32, 5
+    t, b, dims = _grouped_layer(rows, counts, d_in, d_emb, 128, 64, seed)
+    y, plan, kernels = _forward_kernels(t, b, dims)
+    assert plan.info().n_dense_tiles == len(rows)
+    assert "attn_dense_skinny" in kernels, kernels
+    assert "attn_dense" not in kernels and "attn_dense_small" not in kernels, kernels
+    err = rel_max_err(y.double().cpu().numpy(), oracle_y(t, b))
+    assert err <= TOL["bf16"], err
+
+
+def test_skinny_and_full_tiles_together():
+    """Groups whose last tile has 32 tokens (skinny) or 33 (the 128-token
+    kernel) beside whole tiles, in both d_t configurations, among enough
+    short groups for the transposed-product kernel to run."""
+    rows = (300, 300, 300, 200, 200, 200, 512, 64) + (96, 260) * 330
+    counts = (160, 161, 128, 32, 33, 290, 37, 6) + (7, 19) * 330
+    t, b, dims = _grouped_layer(rows, counts, 128, 256, 64, 32, 7)
+    y, plan, kernels = _forward_kernels(t, b, dims)
+    assert {"attn_dense", "attn_dense_small", "attn_dense_skinny"} <= set(kernels), kernels
+    err = rel_max_err(y.double().cpu().numpy(), oracle_y(t, b))
     assert err <= TOL["bf16"], err
 
 
