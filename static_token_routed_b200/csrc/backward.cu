@@ -1200,18 +1200,23 @@ extern "C" l3_status l3_backward(const void *x, l3_plan_t p, const void *W_K, co
     if (e != cudaSuccess) st = cuda_fail(e, "attention backward (tail items)");
   }
   if (st == L3_OK && n_dt > 0) {
-    {
-      LaunchTimer t("bwd_dense_scores", s);
-      k_bwd_dense_scores<<<(unsigned)(n_dt * (slot_rows / DB_J)), 256, 0, s>>>(
-          x, W_K, W_V, wt, g_a, p->perm, p->group_tok_start, p->group_row_start, p->group_rows,
-          p->dense_tiles, slots, slot_rows, (int)d.d_in, (int)d.d_emb);
+    if (bwd_scores_tc_supported(d)) {
+      // S, G_p on tcgen05 with the tokens as N, softmax and g_s in the same kernel
+      st = launch_bwd_scores_tc(p, x, W_K, W_V, g_a, slots, slot_rows, s);
+    } else {
+      {
+        LaunchTimer t("bwd_dense_scores", s);
+        k_bwd_dense_scores<<<(unsigned)(n_dt * (slot_rows / DB_J)), 256, 0, s>>>(
+            x, W_K, W_V, wt, g_a, p->perm, p->group_tok_start, p->group_row_start, p->group_rows,
+            p->dense_tiles, slots, slot_rows, (int)d.d_in, (int)d.d_emb);
+      }
+      {
+        LaunchTimer t("bwd_dense_softmax", s);
+        k_bwd_dense_softmax<<<(unsigned)n_dt, DENSE_TILE_M, 0, s>>>(
+            p->group_tok_start, p->group_rows, p->dense_tiles, slots, slot_rows);
+      }
     }
-    {
-      LaunchTimer t("bwd_dense_softmax", s);
-      k_bwd_dense_softmax<<<(unsigned)n_dt, DENSE_TILE_M, 0, s>>>(
-          p->group_tok_start, p->group_rows, p->dense_tiles, slots, slot_rows);
-    }
-    {
+    if (st == L3_OK) {
       LaunchTimer t("bwd_dense_dx", s);
       k_bwd_dense_dx<<<(unsigned)(n_dt * (d.d_in / 64)), 256, 0, s>>>(
           W_K, wt, p->perm, p->group_tok_start, p->group_row_start, p->group_rows, p->dense_tiles,
@@ -1222,7 +1227,7 @@ extern "C" l3_status l3_backward(const void *x, l3_plan_t p, const void *W_K, co
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(k_attn_backward_dw, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                (int)dw_smem);
-    if (e == cudaSuccess) {
+    if (e == cudaSuccess && st == L3_OK) {
       LaunchTimer t("bwd_dense_dw", s);
       const int64_t n_cb = d.d_in / DW_C + d.d_emb / DW_C;
       k_attn_backward_dw<<<(unsigned)(n_dt * n_cb), 256, dw_smem, s>>>(

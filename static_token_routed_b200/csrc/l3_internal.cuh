@@ -174,6 +174,11 @@ int dense_attention_max_rows();
 // SKINNY_TOKENS tokens to launch_attn_skinny
 l3_status launch_attn_dense(const l3_plan_s *p, const void *x, const void *W_K, const void *W_V,
                             bool small, bool skip_skinny, cudaStream_t s);
+// backward of the dense tiles: p and g_s into the fp32 planes (bwd_scores_tc.cu)
+bool bwd_scores_tc_supported(const l3_dims_t &d);
+l3_status launch_bwd_scores_tc(const l3_plan_s *p, const void *x, const void *W_K,
+                               const void *W_V, const float *g_a, float *slots, int slot_rows,
+                               cudaStream_t s);
 // attention for dense tiles of at most SKINNY_TOKENS tokens (attn_skinny.cu)
 bool skinny_attention_supported(const l3_dims_t &d);
 l3_status launch_attn_skinny(const l3_plan_s *p, const void *x, const void *W_K, const void *W_V,
