@@ -1216,7 +1216,9 @@ extern "C" l3_status l3_backward(const void *x, l3_plan_t p, const void *W_K, co
             p->group_tok_start, p->group_rows, p->dense_tiles, slots, slot_rows);
       }
     }
-    if (st == L3_OK) {
+    if (st == L3_OK && bwd_dx_tc_supported(d)) {
+      st = launch_bwd_dx_tc(p, W_K, slots, slot_rows, dx, s);
+    } else if (st == L3_OK) {
       LaunchTimer t("bwd_dense_dx", s);
       k_bwd_dense_dx<<<(unsigned)(n_dt * (d.d_in / 64)), 256, 0, s>>>(
           W_K, wt, p->perm, p->group_tok_start, p->group_row_start, p->group_rows, p->dense_tiles,

@@ -50,6 +50,7 @@ constexpr int THREADS = 384;             // 0 TMA, 1 MMA, 2-3 B operands, 4-11 s
 constexpr int SM_THREADS = 256;
 constexpr int TMEM_COLS = 256;           // S^T at 0, G_p^T at 128
 constexpr int G_COL = 4 * TN;
+constexpr int V16_BOX() { return 16 * 128; }  // one 16-row, 64-column bf16 TMA box: 2 KB
 
 struct Bars {
   uint64_t bfull[N_B], bempty[N_B];
@@ -109,6 +110,12 @@ __device__ __forceinline__ void spin_bounded(uint64_t *bar, uint32_t parity) {
   const uint64_t t0 = globaltimer_ns();
   while (!mbar_try_wait(a, parity) && globaltimer_ns() - t0 < WAIT_LIMIT_NS) {
   }
+}
+
+// kind::f16 instruction descriptor with an MN-major A: the K-major form's bits
+// plus the A-major bit
+__host__ __device__ constexpr uint32_t idesc_f16_amn(uint32_t ab_format, uint32_t M, uint32_t N) {
+  return idesc_f16(ab_format, 0, M, N) | (1u << 15);
 }
 
 // Butterfly over the warp: v[t] is this lane's value for token t; the return
@@ -442,7 +449,274 @@ constexpr size_t scores_smem() {
 }
 static_assert(2 * (scores_smem() + 1024) <= 228 * 1024, "two CTAs per SM");
 
+// ---------------------------------------------------------------------------
+// dx_n += K_t^T g_s,n for the tokens of a dense tile, from the g_s plane the
+// kernel above wrote: per (tile, 32-token chunk, 256 columns of d_in)
+//     dx^T = K_t^T G_s     (M = 128 columns of d_in per block, N = 32, K = d_t)
+// with K_t in 16-row slices as an MN-major A operand (TMA, two 64-column boxes
+// per block) and G_s as a K-major B operand [token][row], bf16 hi + lo parts
+// converted from the fp32 plane. Each token's dx row belongs to one chunk, so
+// the epilogue adds into it without atomics: through a per-warp transpose,
+// 16-byte read-modify-writes of eight tokens' 128-byte row pieces.
+constexpr int DX_COLS = 256;                  // columns of d_in per CTA
+constexpr int DX_MB = DX_COLS / MB;           // 2 M blocks
+constexpr int DX_STAGE = V16_BOX() * (DX_COLS / 64);
+constexpr int DX_NS = 4;                      // K_t slices in flight
+constexpr int DX_THREADS = 192;               // 0 TMA, 1 MMA, 2-5 G_s conversion, then epilogue
+constexpr int DX_P_BLOCK = TN * 128;          // 64 rows of G_s^T for the 32 tokens: 4 KB
+constexpr int DX_WBUF = TN * TN * 4;          // fp32 32 x 32 transpose per epilogue warp
+
+struct DxBars {
+  uint64_t full[DX_NS], empty[DX_NS];
+  uint64_t bready;  // the epilogue warps have written G_s^T
+  uint64_t done;    // every MMA has completed
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+__global__ void __launch_bounds__(DX_THREADS, 2)
+    k_bwd_dx_tc(const __grid_constant__ CUtensorMap mK16, Params P, float *__restrict__ dx) {
+  constexpr int per_tile = DENSE_TILE_M / TN;
+  const int n_cg = P.d_in / DX_COLS;
+  const int ti = blockIdx.x / (per_tile * n_cg);
+  const int chunk = (blockIdx.x / n_cg) % per_tile, cg = blockIdx.x % n_cg;
+  const DenseTile tile = P.tiles[ti];
+  const int g = tile.group;
+  const int n_tile = min(DENSE_TILE_M, P.group_tok_start[g + 1] - tile.tok0);
+  const int tok0 = tile.tok0 + chunk * TN;
+  const int n_valid = min(TN, n_tile - chunk * TN);
+  if (n_valid <= 0) return;  // the whole CTA, before any barrier or TMEM
+  const int r0 = P.group_row_start[g], d = P.group_rows[g];
+  const int d16 = (d + 15) & ~15, d64 = (d + 63) & ~63, n_vc = d16 / 16;
+  const int col0 = cg * DX_COLS;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = align1024(smem_raw);
+  uint8_t *ring = smem;                                   // DX_NS slices of K_t
+  uint8_t *bhi = ring + DX_NS * DX_STAGE;                 // G_s^T hi, (d64 / 64) blocks of 4 KB
+  uint8_t *blo = bhi + (MAX_D / 64) * DX_P_BLOCK;         // G_s^T lo
+  // the epilogue's 4 transposes reuse G_s^T hi once every MMA has completed
+  uint8_t *wbufs = bhi;
+  static_assert(4 * DX_WBUF <= (MAX_D / 64) * DX_P_BLOCK, "transposes fit in G_s^T hi");
+  DxBars *b = reinterpret_cast<DxBars *>(blo + (MAX_D / 64) * DX_P_BLOCK);
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < DX_NS; ++s) {
+      mbar_init(&b->full[s], 1);
+      mbar_init(&b->empty[s], 1);
+    }
+    mbar_init(&b->bready, 4);
+    mbar_init(&b->done, 1);
+    mbar_init(&b->drain, 1);
+    b->abort_flag = 0;
+    fence_mbar_init();
+    prefetch_tensormap(&mK16);
+  }
+  if (warp == 1) {
+    tmem_alloc(&b->tmem_base, 64);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = b->tmem_base;
+  const Abort ab{&b->abort_flag, P.err};
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (elect_one()) {
+      bool ok = true;
+      bool armed[DX_NS];
+      uint32_t armed_par[DX_NS];
+      for (int i = 0; i < DX_NS; ++i) armed[i] = false;
+      for (int vc = 0; ok && vc < n_vc; ++vc) {
+        const int s = vc % DX_NS;
+        const uint32_t ph = (vc / DX_NS) & 1;
+        if (!mbar_wait(&b->empty[s], ph ^ 1, ab)) {
+          ok = false;
+          break;
+        }
+        mbar_arrive_expect_tx(&b->full[s], DX_STAGE);
+        armed[s] = true;
+        armed_par[s] = ph;
+        for (int bx = 0; bx < DX_COLS / 64; ++bx)
+          tma_load_2d(ring + s * DX_STAGE + bx * V16_BOX(), &mK16, &b->full[s], col0 + bx * 64,
+                      r0 + vc * 16);
+      }
+      if (!ok)
+        for (int s = 0; s < DX_NS; ++s)
+          if (armed[s]) spin_bounded(&b->full[s], armed_par[s]);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    // lane 0 issues; the whole warp waits and zeroes, in the last slice, the
+    // rows at or past d_t: they belong to the next IDs, and an Inf there
+    // would meet a zero of G_s
+    bool ok = __all_sync(0xffffffffu, mbar_wait(&b->bready, 0, ab));
+    tc_fence_after();
+    const uint32_t id = idesc_f16_amn(1, MB, TN);
+    const uint32_t ph = smem_u32(bhi), pl = smem_u32(blo);
+    for (int vc = 0; ok && vc < n_vc; ++vc) {
+      const int s = vc % DX_NS;
+      if (!__all_sync(0xffffffffu, mbar_wait(&b->full[s], (vc / DX_NS) & 1, ab))) {
+        ok = false;
+        break;
+      }
+      uint8_t *slice = ring + s * DX_STAGE;
+      const int live = d - vc * 16;
+      if (live < 16) {
+        const int per_box = (16 - live) * 8;  // 16-byte pieces past d_t in a box
+        uint4 *vb = reinterpret_cast<uint4 *>(slice);
+        for (int e = lane; e < (DX_COLS / 64) * per_box; e += 32) {
+          const int bx = e / per_box, w = e - bx * per_box;
+          vb[bx * (V16_BOX() / 16) + live * 8 + w] = make_uint4(0u, 0u, 0u, 0u);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+      }
+      tc_fence_after();
+      if (lane == 0) {
+        const uint32_t va = smem_u32(slice);
+        const int kk = vc * 16;  // row of K_t: the K index of both operands
+        const uint32_t boff = (kk / 64) * DX_P_BLOCK + (kk % 64) * 2;
+        for (int mb = 0; mb < DX_MB; ++mb) {
+          const uint64_t ad = sdesc_sw128(va + 2 * mb * V16_BOX(), V16_BOX(), 1024);
+          umma_f16(tmem + mb * TN, ad, sdesc_sw128(ph + boff, 16, 1024), id, vc != 0);
+          umma_f16(tmem + mb * TN, ad, sdesc_sw128(pl + boff, 16, 1024), id, 1);
+        }
+        umma_commit(&b->empty[s]);
+      }
+      __syncwarp();
+    }
+    if (lane == 0) {
+      if (ok) {
+        umma_commit(&b->done);
+      } else {
+        umma_commit(&b->drain);
+        spin_bounded(&b->drain, 0);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ G_s^T, then the epilogue
+    // warps 2-5: thread et takes rows et, et + 128, ... of the plane: its 32
+    // tokens' g_s, split into bf16 hi / lo, into [token][row] (128-byte
+    // swizzled 64-row blocks); rows from d up to d16 as zeros
+    const int et = threadIdx.x - 64;  // 0..127
+    const float *plane = P.slots + ((int64_t)ti * 2 + 1) * P.slot_rows * DENSE_TILE_M + chunk * TN;
+    for (int j = et; j < d16; j += 128) {
+      float f[TN];
+#pragma unroll
+      for (int e = 0; e < TN; e += 4) {
+        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (j < d) v = *reinterpret_cast<const float4 *>(plane + (int64_t)j * DENSE_TILE_M + e);
+        f[e] = v.x; f[e + 1] = v.y; f[e + 2] = v.z; f[e + 3] = v.w;
+      }
+      const int cj = (j % 64) / 8;
+      uint8_t *ch = bhi + (j / 64) * DX_P_BLOCK + (j % 8) * 2;
+      uint8_t *cl = blo + (j / 64) * DX_P_BLOCK + (j % 8) * 2;
+#pragma unroll
+      for (int t = 0; t < TN; ++t) {
+        // tokens past the chunk's count enter as zero
+        const float v = t < n_valid ? f[t] : 0.f;
+        const __nv_bfloat16 h = __float2bfloat16_rn(v);
+        const __nv_bfloat16 l = __float2bfloat16_rn(v - __bfloat162float(h));
+        const int off = t * 128 + ((cj ^ (t & 7)) << 4);
+        *reinterpret_cast<__nv_bfloat16 *>(ch + off) = h;
+        *reinterpret_cast<__nv_bfloat16 *>(cl + off) = l;
+      }
+    }
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&b->bready);
+    // epilogue: warp w reads TMEM lane quarter w % 4 of both blocks: column
+    // col0 + 128 mb + 32 q + lane of d_in for the 32 tokens
+    const int q = warp & 3;
+    uint8_t *wbuf = wbufs + (warp - 2) * DX_WBUF;
+    bool ok = __all_sync(0xffffffffu, mbar_wait(&b->done, 0, ab));
+    const int my_tok = lane < n_valid ? P.perm[tok0 + lane] : -1;
+    if (ok) {
+      tc_fence_after();
+      for (int mb = 0; mb < DX_MB; ++mb) {
+        uint32_t v[TN];
+        tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + mb * TN, v);
+        tmem_wait_ld();
+        // row t (token), column lane: 16-byte chunks XOR-swizzled by t & 7
+#pragma unroll
+        for (int t = 0; t < TN; ++t)
+          *reinterpret_cast<uint32_t *>(wbuf + t * 128 + ((((lane >> 2) ^ (t & 7))) << 4) +
+                                        (lane & 3) * 4) = v[t];
+        __syncwarp();
+        const int cb = col0 + mb * MB + q * 32;
+#pragma unroll
+        for (int k = 0; k < TN / 4; ++k) {
+          const int t = k * 4 + (lane >> 3), c8 = lane & 7;  // 4 tokens x 8 chunks
+          const float4 add =
+              *reinterpret_cast<const float4 *>(wbuf + t * 128 + ((c8 ^ (t & 7)) << 4));
+          const int tk = __shfl_sync(0xffffffffu, my_tok, t);
+          if (tk >= 0) {
+            float4 *o = reinterpret_cast<float4 *>(dx + (int64_t)tk * P.d_in + cb + c8 * 4);
+            float4 cur = *o;
+            cur.x += add.x; cur.y += add.y; cur.z += add.z; cur.w += add.w;
+            *o = cur;
+          }
+        }
+        __syncwarp();
+      }
+    }
+  }
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 64);
+  }
+}
+
+constexpr size_t dx_smem() {
+  return 1024 + DX_NS * DX_STAGE + 2 * (MAX_D / 64) * DX_P_BLOCK + sizeof(DxBars);
+}
+static_assert(2 * (dx_smem() + 1024) <= 228 * 1024, "two CTAs per SM");
+
 }  // namespace
+
+bool bwd_dx_tc_supported(const l3_dims_t &d) {
+  return d.dtype == L3_BF16 && d.d_in % DX_COLS == 0 && d.k <= MAX_D;
+}
+
+l3_status launch_bwd_dx_tc(const l3_plan_s *p, const void *W_K, const float *slots, int slot_rows,
+                           float *dx, cudaStream_t s) {
+  if (p->n_dense_tiles == 0) return L3_OK;
+  const l3_dims_t &d = p->dims;
+  CUtensorMap mK16;
+  l3_status st;
+  if ((st = make_map_2d16(&mK16, W_K, true, (uint64_t)d.v, d.d_in, d.d_in, CK, 16, 128)) != L3_OK)
+    return st;
+  Params P = {};
+  P.perm = p->perm;
+  P.group_tok_start = p->group_tok_start;
+  P.group_row_start = p->group_row_start;
+  P.group_rows = p->group_rows;
+  P.tiles = p->dense_tiles;
+  P.slots = const_cast<float *>(slots);
+  P.slot_rows = slot_rows;
+  P.d_in = (int)d.d_in;
+  P.d_emb = (int)d.d_emb;
+  P.err = p->dev_flags + 1;
+  static bool attr[64] = {};
+  if (!attr[p->device & 63]) {
+    L3_CUDA_TRY(cudaFuncSetAttribute(k_bwd_dx_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)dx_smem()));
+    attr[p->device & 63] = true;
+  }
+  const int64_t grid = p->n_dense_tiles * (DENSE_TILE_M / TN) * (d.d_in / DX_COLS);
+  LaunchTimer t("bwd_dense_dx_tc", s);
+  k_bwd_dx_tc<<<(unsigned)grid, DX_THREADS, dx_smem(), s>>>(mK16, P, dx);
+  L3_CUDA_TRY(cudaGetLastError());
+  return L3_OK;
+}
 
 bool bwd_scores_tc_supported(const l3_dims_t &d) {
   return d.dtype == L3_BF16 && d.d_in % CK == 0 && d.d_emb % CK == 0 && d.k <= MAX_D;

@@ -179,6 +179,10 @@ bool bwd_scores_tc_supported(const l3_dims_t &d);
 l3_status launch_bwd_scores_tc(const l3_plan_s *p, const void *x, const void *W_K,
                                const void *W_V, const float *g_a, float *slots, int slot_rows,
                                cudaStream_t s);
+// dx += K_t^T g_s of the dense tiles' tokens from the g_s plane (bwd_scores_tc.cu)
+bool bwd_dx_tc_supported(const l3_dims_t &d);
+l3_status launch_bwd_dx_tc(const l3_plan_s *p, const void *W_K, const float *slots, int slot_rows,
+                           float *dx, cudaStream_t s);
 // attention for dense tiles of at most SKINNY_TOKENS tokens (attn_skinny.cu)
 bool skinny_attention_supported(const l3_dims_t &d);
 l3_status launch_attn_skinny(const l3_plan_s *p, const void *x, const void *W_K, const void *W_V,

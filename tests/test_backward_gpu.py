@@ -16,7 +16,7 @@ pytestmark = pytest.mark.gpu
 NAMES = ("x", "W_K", "W_V", "W_up", "ln_gamma", "ln_beta", "W_mix")
 
 
-def check(w, t, b, dims, tol, seed=0):
+def check(w, t, b, dims, tol, seed=0, names=NAMES):
     dev = to_device(t, b)
     plan = l3.l3_plan(dev["ids"], dev["offsets"], dims)
     y = torch.empty(b.ids.numel(), w.d_out, dtype=w.torch_dtype, device="cuda")
@@ -29,13 +29,13 @@ def check(w, t, b, dims, tol, seed=0):
     l3.l3_forward_status(plan)
     want = bwd.backward(b.ids, t.offsets, b.x, t.W_K, t.W_V, t.W_up, t.ln_gamma, t.ln_beta,
                         t.W_mix, EPS, dy)
-    errs = {k: rel_max_err(got[k].double().cpu().numpy(), want[k]) for k in NAMES}
+    errs = {k: rel_max_err(got[k].double().cpu().numpy(), want[k]) for k in names}
     assert all(e <= tol for e in errs.values()), ", ".join(f"{k} {e:.3g}" for k, e in errs.items())
     # a second call gives the same bits, except dW_K / dW_V whose rows take
     # atomic adds from several units of a group
     again = l3.l3_backward(dev["x"], plan, dev["W_K"], dev["W_V"], dev["W_up"], dev["ln_gamma"],
                            dev["ln_beta"], dev["W_mix"], dy.cuda())
-    for k in NAMES:
+    for k in names:
         if k in ("W_K", "W_V"):
             assert rel_max_err(again[k].double().cpu().numpy(), want[k]) <= tol, k
         else:
@@ -86,7 +86,7 @@ def test_backward_neighbour_rows_never_reach_a_group():
     vocab = 5
     rows = (300, 5, 200, 7, 40)   # IDs 1 and 3 are never in the batch
     off = torch.tensor([0] + list(rows), dtype=torch.int64).cumsum(0).to(torch.int32)
-    v, d_in, d_emb, d_up, d_out = int(off[-1]), 128, 512, 64, 64
+    v, d_in, d_emb, d_up, d_out = int(off[-1]), 256, 512, 64, 64
     g = torch.Generator().manual_seed(12)
     mk = lambda *s: (torch.randn(*s, generator=g) / s[-1] ** 0.5).to(torch.bfloat16)  # noqa: E731
     W_K, W_V = mk(v, d_in), mk(v, d_emb)
@@ -107,6 +107,18 @@ def test_backward_neighbour_rows_never_reach_a_group():
     w = wl.Workload("case", vocab, v, max(rows), d_in, d_emb, d_up, d_out, n, "bf16", "zipf",
                     "zipf", 0, 0)
     check(w, t, b, dims, TOL["bf16"])
+
+
+def test_backward_dense_dx_on_tensor_cores():
+    """d_in a multiple of 256, so the dense tiles' dx = K_t^T g_s also runs on
+    the tensor cores (besides their scores): d_t on and off multiples of 16,
+    ragged 32-token chunks, a 512-row group. The attention gradients (x, W_K,
+    W_V) are this case's subject; the GEMM-side ones are covered above."""
+    vocab, rows, n, d_in, d_emb, d_up, d_out = 5, (512, 300, 257, 100, 37), 1100, 256, 256, 64, 32
+    t, b, dims = small_layer(vocab, rows, n, d_in, d_emb, d_up, d_out, torch.bfloat16, vocab)
+    w = wl.Workload("case", vocab, int(sum(rows)), max(rows), d_in, d_emb, d_up, d_out, n, "bf16",
+                    "zipf", "zipf", 0, 0)
+    check(w, t, b, dims, TOL["bf16"], names=("x", "W_K", "W_V"))
 
 
 def test_backward_on_its_own_stream_then_replan():
