@@ -451,17 +451,18 @@ static_assert(2 * (scores_smem() + 1024) <= 228 * 1024, "two CTAs per SM");
 
 // ---------------------------------------------------------------------------
 // dx_n += K_t^T g_s,n for the tokens of a dense tile, from the g_s plane the
-// kernel above wrote: per (tile, 32-token chunk, 256 columns of d_in)
+// kernel above wrote: per (tile, 32-token chunk, 512 columns of d_in)
 //     dx^T = K_t^T G_s     (M = 128 columns of d_in per block, N = 32, K = d_t)
 // with K_t in 16-row slices as an MN-major A operand (TMA, two 64-column boxes
 // per block) and G_s as a K-major B operand [token][row], bf16 hi + lo parts
 // converted from the fp32 plane. Each token's dx row belongs to one chunk, so
 // the epilogue adds into it without atomics: through a per-warp transpose,
 // 16-byte read-modify-writes of eight tokens' 128-byte row pieces.
-constexpr int DX_COLS = 256;                  // columns of d_in per CTA
-constexpr int DX_MB = DX_COLS / MB;           // 2 M blocks
+constexpr int DX_COLS = 512;                  // columns of d_in per CTA
+constexpr int DX_MB = DX_COLS / MB;           // 4 M blocks (fewer in a last, partial group)
+constexpr int DX_TMEM = DX_MB * TN;           // 128 TMEM columns
 constexpr int DX_STAGE = V16_BOX() * (DX_COLS / 64);
-constexpr int DX_NS = 4;                      // K_t slices in flight
+constexpr int DX_NS = 2;                      // K_t slices in flight
 constexpr int DX_THREADS = 192;               // 0 TMA, 1 MMA, 2-5 G_s conversion, then epilogue
 constexpr int DX_P_BLOCK = TN * 128;          // 64 rows of G_s^T for the 32 tokens: 4 KB
 constexpr int DX_WBUF = TN * TN * 4;          // fp32 32 x 32 transpose per epilogue warp
@@ -478,7 +479,7 @@ struct DxBars {
 __global__ void __launch_bounds__(DX_THREADS, 2)
     k_bwd_dx_tc(const __grid_constant__ CUtensorMap mK16, Params P, float *__restrict__ dx) {
   constexpr int per_tile = DENSE_TILE_M / TN;
-  const int n_cg = P.d_in / DX_COLS;
+  const int n_cg = (P.d_in + DX_COLS - 1) / DX_COLS;
   const int ti = blockIdx.x / (per_tile * n_cg);
   const int chunk = (blockIdx.x / n_cg) % per_tile, cg = blockIdx.x % n_cg;
   const DenseTile tile = P.tiles[ti];
@@ -490,6 +491,7 @@ __global__ void __launch_bounds__(DX_THREADS, 2)
   const int r0 = P.group_row_start[g], d = P.group_rows[g];
   const int d16 = (d + 15) & ~15, d64 = (d + 63) & ~63, n_vc = d16 / 16;
   const int col0 = cg * DX_COLS;
+  const int n_mb = min(DX_MB, (P.d_in - col0) / MB);  // d_in is a multiple of 128
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = align1024(smem_raw);
@@ -515,7 +517,7 @@ __global__ void __launch_bounds__(DX_THREADS, 2)
     prefetch_tensormap(&mK16);
   }
   if (warp == 1) {
-    tmem_alloc(&b->tmem_base, 64);
+    tmem_alloc(&b->tmem_base, DX_TMEM);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -538,10 +540,10 @@ __global__ void __launch_bounds__(DX_THREADS, 2)
           ok = false;
           break;
         }
-        mbar_arrive_expect_tx(&b->full[s], DX_STAGE);
+        mbar_arrive_expect_tx(&b->full[s], (uint32_t)(2 * n_mb * V16_BOX()));
         armed[s] = true;
         armed_par[s] = ph;
-        for (int bx = 0; bx < DX_COLS / 64; ++bx)
+        for (int bx = 0; bx < 2 * n_mb; ++bx)
           tma_load_2d(ring + s * DX_STAGE + bx * V16_BOX(), &mK16, &b->full[s], col0 + bx * 64,
                       r0 + vc * 16);
       }
@@ -569,7 +571,7 @@ __global__ void __launch_bounds__(DX_THREADS, 2)
       if (live < 16) {
         const int per_box = (16 - live) * 8;  // 16-byte pieces past d_t in a box
         uint4 *vb = reinterpret_cast<uint4 *>(slice);
-        for (int e = lane; e < (DX_COLS / 64) * per_box; e += 32) {
+        for (int e = lane; e < 2 * n_mb * per_box; e += 32) {
           const int bx = e / per_box, w = e - bx * per_box;
           vb[bx * (V16_BOX() / 16) + live * 8 + w] = make_uint4(0u, 0u, 0u, 0u);
         }
@@ -581,7 +583,7 @@ __global__ void __launch_bounds__(DX_THREADS, 2)
         const uint32_t va = smem_u32(slice);
         const int kk = vc * 16;  // row of K_t: the K index of both operands
         const uint32_t boff = (kk / 64) * DX_P_BLOCK + (kk % 64) * 2;
-        for (int mb = 0; mb < DX_MB; ++mb) {
+        for (int mb = 0; mb < n_mb; ++mb) {
           const uint64_t ad = sdesc_sw128(va + 2 * mb * V16_BOX(), V16_BOX(), 1024);
           umma_f16(tmem + mb * TN, ad, sdesc_sw128(ph + boff, 16, 1024), id, vc != 0);
           umma_f16(tmem + mb * TN, ad, sdesc_sw128(pl + boff, 16, 1024), id, 1);
@@ -638,7 +640,7 @@ __global__ void __launch_bounds__(DX_THREADS, 2)
     const int my_tok = lane < n_valid ? P.perm[tok0 + lane] : -1;
     if (ok) {
       tc_fence_after();
-      for (int mb = 0; mb < DX_MB; ++mb) {
+      for (int mb = 0; mb < n_mb; ++mb) {
         uint32_t v[TN];
         tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + mb * TN, v);
         tmem_wait_ld();
@@ -671,7 +673,7 @@ __global__ void __launch_bounds__(DX_THREADS, 2)
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, 64);
+    tmem_dealloc(tmem, DX_TMEM);
   }
 }
 
@@ -683,7 +685,7 @@ static_assert(2 * (dx_smem() + 1024) <= 228 * 1024, "two CTAs per SM");
 }  // namespace
 
 bool bwd_dx_tc_supported(const l3_dims_t &d) {
-  return d.dtype == L3_BF16 && d.d_in % DX_COLS == 0 && d.k <= MAX_D;
+  return d.dtype == L3_BF16 && d.d_in % MB == 0 && d.k <= MAX_D;
 }
 
 l3_status launch_bwd_dx_tc(const l3_plan_s *p, const void *W_K, const float *slots, int slot_rows,
@@ -711,7 +713,7 @@ l3_status launch_bwd_dx_tc(const l3_plan_s *p, const void *W_K, const float *slo
                                      (int)dx_smem()));
     attr[p->device & 63] = true;
   }
-  const int64_t grid = p->n_dense_tiles * (DENSE_TILE_M / TN) * (d.d_in / DX_COLS);
+  const int64_t grid = p->n_dense_tiles * (DENSE_TILE_M / TN) * ((d.d_in + DX_COLS - 1) / DX_COLS);
   LaunchTimer t("bwd_dense_dx_tc", s);
   k_bwd_dx_tc<<<(unsigned)grid, DX_THREADS, dx_smem(), s>>>(mK16, P, dx);
   L3_CUDA_TRY(cudaGetLastError());
