@@ -465,25 +465,26 @@ l3_status l3_forward(const void *x, l3_plan_t p, const void *W_K, const void *W_
   const bool has_big = p->n_dense_tiles > p->n_dense_small;
   const bool has_tail = p->n_tail_items > 0;
   if (has_tail && tail_cls_supported(p->dims)) {
-    // fork: dense attention (both configurations, in turn) on the caller's
-    // stream; the fp16 weight copies first on the last helper stream, then
-    // the tail classes over the high-priority helper streams, whose short
-    // CTAs fill the SM slots the long dense CTAs leave; join before W_up. The
-    // launches write disjoint rows of a.
+    // fork: dense attention (its launches in turn, see launch_dense_all) on
+    // the caller's stream; the fp16 weight copies first on the last helper
+    // stream, then the tail classes over the high-priority helper streams,
+    // whose short CTAs fill the SM slots the dense CTAs leave; join before
+    // W_up. The launches write disjoint rows of a.
     Aux *aux = nullptr;
     if ((st = aux_for(p->device, &aux)) != L3_OK) return st;
     std::lock_guard<std::mutex> lk(aux->mu);
     L3_CUDA_TRY(cudaEventRecord(aux->fork, s));
     for (int i = 0; i < N_AUX; ++i) L3_CUDA_TRY(cudaStreamWaitEvent(aux->stream[i], aux->fork, 0));
     if (st == L3_OK) st = launch_dense_all(p, x, W_K, W_V, s);
-    // next to the big dense configuration (one CTA per SM, streaming K_t)
-    // the tails stay on one helper stream: spread over three they take SMs
-    // and bandwidth from it (paper_shaped: 1.64 -> 1.72 ms per batch); with
-    // no such launch they spread over all three (small_bf16: 0.41 -> 0.34 ms)
     // the weight copies run beside the attention rather than after the tail
     // stream's last launch (paper_shaped: up_z started ~20 us later there)
     if (st == L3_OK && p->tc_gemm)
       st = launch_weights_f16(p, W_up, W_mix, ln_gamma, ln_beta, aux->stream[N_AUX - 1]);
+    // next to the big dense configuration (one CTA per SM, streaming K_t)
+    // the tails stay on one helper stream: spread over three they take SMs
+    // and bandwidth from it (paper_shaped: 1.64 -> 1.72 ms per batch, and
+    // 1.43 -> 1.49 beside the skinny kernel); with no such launch they spread
+    // over all three (small_bf16: 0.41 -> 0.34 ms)
     if (st == L3_OK) st = launch_attn_tail_cls(p, x, W_K, W_V, aux->stream, has_big ? 1 : N_AUX);
     for (int i = 0; i < N_AUX; ++i) {
       L3_CUDA_TRY(cudaEventRecord(aux->join[i], aux->stream[i]));
