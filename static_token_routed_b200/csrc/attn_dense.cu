@@ -45,6 +45,7 @@
 #include <algorithm>
 
 #include "l3_internal.cuh"
+#include "attn_common.cuh"
 #include "sm100.cuh"
 
 namespace l3 {
@@ -55,6 +56,7 @@ l3_status make_map_2d16(CUtensorMap *m, const void *base, bool bf16, uint64_t ro
 namespace {
 
 using namespace sm100;
+using namespace attn;
 
 constexpr int TM = 128;                 // tokens per tile
 constexpr int CK = 64;                  // d_in columns per S-phase slice (128-byte rows)
@@ -115,55 +117,12 @@ struct DenseParams {
   int *err;
 };
 
-__device__ __forceinline__ uint8_t *align1024(uint8_t *p) {
-  return reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
-}
-
-__device__ __forceinline__ void cp_async16_zfill(void *dst, const void *src, uint32_t src_bytes) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src),
-               "r"(src_bytes)
-               : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() {
-  asm volatile("cp.async.commit_group;" ::: "memory");
-}
-__device__ __forceinline__ void cp_async_wait_all() {
-  asm volatile("cp.async.wait_group 0;" ::: "memory");
-}
-// wait until at most `lag` committed groups of this thread are still in flight
-__device__ __forceinline__ void cp_async_wait_group_lag(int lag) {
-  switch (lag) {
-    case 0: asm volatile("cp.async.wait_group 0;" ::: "memory"); break;
-    case 1: asm volatile("cp.async.wait_group 1;" ::: "memory"); break;
-    case 2: asm volatile("cp.async.wait_group 2;" ::: "memory"); break;
-    case 3: asm volatile("cp.async.wait_group 3;" ::: "memory"); break;
-    case 4: asm volatile("cp.async.wait_group 4;" ::: "memory"); break;
-    case 5: asm volatile("cp.async.wait_group 5;" ::: "memory"); break;
-    case 6: asm volatile("cp.async.wait_group 6;" ::: "memory"); break;
-    default: asm volatile("cp.async.wait_group 7;" ::: "memory"); break;
-  }
-}
 
 // barrier of the 256 softmax / epilogue threads that ANDs a flag across them
 __device__ __forceinline__ bool softmax_sync_and(bool ok) {
-  uint32_t r;
-  asm volatile(
-      "{\n\t.reg .pred p, q;\n\t"
-      "setp.ne.u32 q, %1, 0;\n\t"
-      "bar.red.and.pred p, 1, %2, q;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}\n"
-      : "=r"(r)
-      : "r"((uint32_t)ok), "n"(SOFTMAX_THREADS)
-      : "memory");
-  return r != 0;
+  return sync_and<1, SOFTMAX_THREADS>(ok);
 }
 
-__device__ __forceinline__ void spin_bounded(uint64_t *bar, uint32_t parity) {
-  const uint32_t a = smem_u32(bar);
-  const uint64_t t0 = globaltimer_ns();
-  while (!mbar_try_wait(a, parity) && globaltimer_ns() - t0 < WAIT_LIMIT_NS) {
-  }
-}
 
 // Per-tile geometry, the same in every warp: the S ring and the P / V layout
 // follow from d_t.
@@ -517,7 +476,7 @@ __global__ void __launch_bounds__(DENSE_THREADS, DenseCfg<SMALL>::MIN_BLOCKS)
         cp_async_commit();
         ++issued;
         if (issued - done > lag) {
-          cp_async_wait_group_lag(lag);
+          cp_async_wait<lag>();
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) mbar_arrive(&b->xfull[(gx + done) % Cfg::N_X]);
@@ -525,7 +484,7 @@ __global__ void __launch_bounds__(DENSE_THREADS, DenseCfg<SMALL>::MIN_BLOCKS)
         }
       }
       // the last slices, and on a give-up every copy still in flight
-      cp_async_wait_all();
+      cp_async_wait<0>();
       fence_proxy_async_smem();
       __syncwarp();
       for (; ok && done < issued; ++done)

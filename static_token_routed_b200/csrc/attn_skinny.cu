@@ -40,6 +40,7 @@
 #include <algorithm>
 
 #include "l3_internal.cuh"
+#include "attn_common.cuh"
 #include "sm100.cuh"
 
 namespace l3 {
@@ -50,6 +51,7 @@ l3_status make_map_2d16(CUtensorMap *m, const void *base, bool bf16, uint64_t ro
 namespace {
 
 using namespace sm100;
+using namespace attn;
 
 constexpr int TN = SKINNY_TOKENS;          // token slots per tile: N of both products
 constexpr int MB = 128;                    // rows of an M block (one MMA's M)
@@ -106,70 +108,9 @@ struct SkParams {
   int *err;
 };
 
-__device__ __forceinline__ uint8_t *align1024(uint8_t *p) {
-  return reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
-}
-__device__ __forceinline__ void cp_async16_zfill(void *dst, const void *src, uint32_t src_bytes) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src),
-               "r"(src_bytes)
-               : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() {
-  asm volatile("cp.async.commit_group;" ::: "memory");
-}
-__device__ __forceinline__ void cp_async_wait_all() {
-  asm volatile("cp.async.wait_group 0;" ::: "memory");
-}
-__device__ __forceinline__ void cp_async_wait_lag() {
-  static_assert(X_LAG == 1, "the wait below holds X_LAG groups in flight");
-  asm volatile("cp.async.wait_group 1;" ::: "memory");
-}
-// barrier of the 256 softmax / epilogue threads ANDing a flag across them
-__device__ __forceinline__ bool sm_sync_and(bool ok) {
-  uint32_t r;
-  asm volatile(
-      "{\n\t.reg .pred p, q;\n\t"
-      "setp.ne.u32 q, %1, 0;\n\t"
-      "bar.red.and.pred p, 1, %2, q;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}\n"
-      : "=r"(r)
-      : "r"((uint32_t)ok), "n"(SM_THREADS)
-      : "memory");
-  return r != 0;
-}
-__device__ __forceinline__ void spin_bounded(uint64_t *bar, uint32_t parity) {
-  const uint32_t a = smem_u32(bar);
-  const uint64_t t0 = globaltimer_ns();
-  while (!mbar_try_wait(a, parity) && globaltimer_ns() - t0 < WAIT_LIMIT_NS) {
-  }
-}
-
-// kind::f16 instruction descriptor with an MN-major A (the V_t slices): the
-// K-major form's bits plus the A-major bit
-__host__ __device__ constexpr uint32_t idesc_f16_amn(uint32_t ab_format, uint32_t M, uint32_t N) {
-  return idesc_f16(ab_format, 0, M, N) | (1u << 15);
-}
-
-// Butterfly over the warp: v[t] holds this lane's value for token t; after
-// it the lane's return value is the max (SUM = false) or sum over all 32
-// lanes for token t = lane. Each step trades half of the values a lane still
-// holds with the partner lane and combines the other half.
-template <bool SUM>
-__device__ __forceinline__ float warp_transpose_reduce(float (&v)[TN], int lane) {
-#pragma unroll
-  for (int w = TN / 2; w >= 1; w >>= 1) {
-    const bool upper = (lane & w) != 0;
-#pragma unroll
-    for (int i = 0; i < w; ++i) {
-      // keep tokens i + (upper ? w : 0) of this block, send the others
-      const float keep = upper ? v[i + w] : v[i];
-      const float send = upper ? v[i] : v[i + w];
-      const float got = __shfl_xor_sync(0xffffffffu, send, w);
-      v[i] = SUM ? keep + got : fmaxf(keep, got);
-    }
-  }
-  return v[0];
-}
+// a slice is handed over once X_LAG later ones have been issued
+__device__ __forceinline__ void cp_async_wait_lag() { cp_async_wait<X_LAG>(); }
+__device__ __forceinline__ bool sm_sync_and(bool ok) { return sync_and<1, SM_THREADS>(ok); }
 
 struct SkGeo {
   int tok0, n_valid, r0, d, d16, d64, n_mb, n_vc, p_bytes, n_v;
@@ -476,7 +417,7 @@ __global__ void __launch_bounds__(THREADS, 2)
           ++done;
         }
       }
-      cp_async_wait_all();
+      cp_async_wait<0>();
       fence_proxy_async_smem();
       __syncwarp();
       for (; ok && done < issued; ++done)
