@@ -687,7 +687,7 @@ def measure(w, args, dev, dist, world, rank, steps, warmup, with_e2e=True, with_
                      "unique_rows": info.unique_rows}}
 
 
-# the BASELINE workloads besides the headline, each measured in the same run
+# the benchmark's other synthetic workloads besides the headline, each measured in the same run
 OTHER_WORKLOADS = ("tiny_fp32", "small_bf16", "decode", "dense_stress", "uniform")
 
 
@@ -750,7 +750,7 @@ def main():
                    with_e2e=not args.no_e2e, with_fwd_only=True, cpu_seconds=args.cpu_seconds)
     per_workload = None
     if world == 1 and not args.only and args.tokens == 0 and args.workload == "paper_shaped":
-        # the other BASELINE workloads at one GPU: shorter CPU samples, the
+        # the other synthetic workloads at one GPU: shorter CPU samples, the
         # same steps (each step is shorter than the headline's)
         torch.cuda.empty_cache()
         per_workload = {}
